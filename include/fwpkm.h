@@ -1,0 +1,186 @@
+/*
+ * fwpkm.h -- C ABI of the B200 (sm_100a) Fast-weight Product Key Memory step.
+ *
+ * The library implements the chunked read-then-write memory step of
+ * "Fast-weight Product Key Memory" (Zhao & Jones).  Citations name the page
+ * and section the operation comes from:
+ *   [GS-2]  gist.science "Fast-weight Product Key Memory", section 2
+ *           "Methodology" (Core Architecture; Key Technical Choices)
+ *   [AF]    agifrontier.github.io "Fast-weight Product Key Memory" tutorial
+ *           (memorisation update; product-key addressing; gating)
+ *   [PYPI]  pypi.org "fast-weight-product-key-memory" 0.2.2, Usage
+ *           (constructor arguments; chaining past/next memories)
+ *   [SS-TOC] sciencestack.ai "Fast-weight Product Key Memory", table of
+ *           contents (loss aggregation and gradient shaping; marginal
+ *           entropy loss)
+ *
+ * Conventions for every entry point:
+ *   - Tensor arguments are plain pointers to memory the CALLER owns.  Unless
+ *     stated otherwise they are DEVICE pointers (cudaMalloc / torch CUDA
+ *     tensors) on the current CUDA device, C-contiguous, 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously on it; nothing synchronises
+ *     unless stated.
+ *   - Every function returns FWPKM_OK (0) or a negative fwpkm_status; the
+ *     message of the last failure on the calling thread is available from
+ *     fwpkm_last_error().  Argument and shape checks run on the host BEFORE
+ *     anything is enqueued: a call that fails them launches nothing and
+ *     leaves the state unchanged.
+ *   - A state is not thread-safe; calls on one state must be serialised.
+ */
+#ifndef FWPKM_H_
+#define FWPKM_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct fwpkm_state fwpkm_state; /* opaque; owns the tables + scratch */
+
+typedef enum {
+  FWPKM_OK = 0,
+  FWPKM_EINVAL = -1,      /* bad pointer / enum / scalar argument            */
+  FWPKM_ESHAPE = -2,      /* sizes violate the constraints listed below      */
+  FWPKM_ENOMEM = -3,      /* device or host allocation failed                */
+  FWPKM_ECUDA = -4,       /* a CUDA call failed (message has the CUDA error)  */
+  FWPKM_EUNSUPPORTED = -5 /* valid request this build does not implement     */
+} fwpkm_status;
+
+/* Element types of Q and Vtarget. */
+enum { FWPKM_F32 = 0, FWPKM_BF16 = 1 };
+
+/* Upper bounds checked by fwpkm_state_init. */
+#define FWPKM_MAX_TOPK 32  /* top-k per head is held one slot per warp lane  */
+#define FWPKM_MAX_SUBKEYS 2048 /* n = sqrt(N): per-half scores live in registers */
+
+/*
+ * fwpkm_state_init -- create a memory of N = n*n slots.  [GS-2, PYPI]
+ *   N      number of value slots; must be a perfect square n*n, 4 <= n <= 2048.
+ *   dq     query width per head; a multiple of 16 (so dq/2, one half, is a
+ *          multiple of 8), dq/2 <= 1024.
+ *   dv     value width; a multiple of 4, <= 2048.
+ *   topk   slots read per head and token; 1 <= topk <= min(n, 32).
+ *   chunk  tokens per update chunk (>= 1); every chunk is read with the tables
+ *          left by the previous chunk, then written.  [GS-2 causality]
+ *   heads  query heads sharing the one value table (>= 1, <= 16); each head
+ *          has its own pair of sub-key tables.
+ * The tables start at ZERO; load them with fwpkm_state_set.  eps (the IDW
+ * constant) defaults to 1e-3.  On success *out receives the state; the state
+ * owns its device memory until fwpkm_state_free.
+ */
+fwpkm_status fwpkm_state_init(int64_t N, int dq, int dv, int topk, int chunk, int heads,
+                              fwpkm_state **out);
+
+/* Release the state and all memory it owns (NULL is a no-op).  Synchronises
+ * the device first so no enqueued work still uses the memory. */
+void fwpkm_state_free(fwpkm_state *s);
+
+/* IDW constant: score = -log(eps + ||q_half - K_row||^2).  [GS-2]  eps > 0. */
+fwpkm_status fwpkm_state_set_eps(fwpkm_state *s, float eps);
+
+/*
+ * fwpkm_step -- run the chunk loop over one call.  [GS-2, AF]
+ * For every chunk c = 0 .. ceil(T/chunk)-1 in order (the last may be
+ * shorter), over all B sequences at once (one shared memory):
+ *   read  : for each token t and head h, split q into halves q1 | q2, score
+ *           each half against its sub-key table with -log(eps + ||q - K||^2),
+ *           take the top-k of each half, merge the k*k Cartesian candidates
+ *           (score s1(i) + s2(j), slot i*n + j) to the top-k slots, weight
+ *           them by softmax, average the heads' weighted value rows into
+ *           yhat_t, and write out_t = gate_t * yhat_t;
+ *   write : with L = sum_t gate_t ||yhat_t - Vtarget_t||^2
+ *           + lambda_entropy * sum_i pbar_i log pbar_i   (pbar = the chunk's
+ *           marginal slot usage), update in place
+ *             V_i -= eta * (dL/dV_i) / C_i  (C_i = sum of w/heads on row i)
+ *             K   -= eta * dL/dK
+ *           on the touched value rows and sub-key rows only; no clipping.
+ * Arguments:
+ *   B, T      batch and tokens per sequence (>= 1).
+ *   Q         device [B][T][heads*dq], element type q_dtype.
+ *   Vtarget   device [B][T][dv], element type v_dtype (the caller aligns
+ *             targets with queries, e.g. the lookahead pairing q_t, v_{t+1}).
+ *   gate      device fp32 [B][T]; also the token weight of the MSE loss.
+ *   eta       learning rate (>= 0); 0 leaves the tables bit-unchanged.
+ *   lambda_entropy  weight of the marginal-entropy addressing term (>= 0).
+ *   out       device fp32 [B][T][dv], written for every token.
+ * Asynchronous on `stream`; kernel faults surface as FWPKM_ECUDA on a later
+ * call or at synchronisation.  Inputs must not alias `out` or the tables.
+ */
+fwpkm_status fwpkm_step(fwpkm_state *s, int B, int T, const void *Q, int q_dtype,
+                        const void *Vtarget, int v_dtype, const float *gate, float eta,
+                        float lambda_entropy, float *out, void *stream);
+
+/*
+ * fwpkm_step_host -- fwpkm_step over HOST buffers (same layouts).  Copies Q,
+ * Vtarget and gate to state-owned device staging buffers, runs the step, and
+ * copies `out` back; returns after the stream has finished.  Pinned host
+ * memory gives the fastest copies; pageable memory also works.
+ */
+fwpkm_status fwpkm_step_host(fwpkm_state *s, int B, int T, const void *Q_host, int q_dtype,
+                             const void *Vtarget_host, int v_dtype, const float *gate_host,
+                             float eta, float lambda_entropy, float *out_host, void *stream);
+
+/*
+ * fwpkm_state_get / fwpkm_state_set -- copy the fast weights out / in, for
+ * chaining memories across calls and for iterative re-reading.  [PYPI Usage]
+ *   subkeys  fp32 [heads][2][n][dq/2]   (half 0 scores the first dq/2 dims)
+ *   values   fp32 [N][dv]
+ * Either pointer may be NULL to skip that table.  Pointers may be device or
+ * host memory (stream-ordered copies).
+ */
+fwpkm_status fwpkm_state_get(const fwpkm_state *s, float *subkeys, float *values, void *stream);
+fwpkm_status fwpkm_state_set(fwpkm_state *s, const float *subkeys, const float *values,
+                             void *stream);
+
+/*
+ * fwpkm_record_selection -- arm a record of the slots and weights the NEXT
+ * fwpkm_step reads (device int32 / fp32, [B][T][heads][topk], best first),
+ * for inspection and parity checks.  Pass NULL, NULL to disarm.  The buffers
+ * must hold B*T*heads*topk entries of the next call's B and T.
+ */
+fwpkm_status fwpkm_record_selection(fwpkm_state *s, int32_t *slots, float *weights);
+
+/*
+ * fwpkm_force_selection -- for the NEXT fwpkm_step, make every token-head
+ * whose mask byte is non-zero read the given slots instead of its own top-k
+ * (their weights are still the softmax of the state's own scores of those
+ * slots).  slots: device int32 [B][T][heads][topk], values in [0, N) and
+ * distinct per token-head; mask: device uint8 [B][T][heads].  Used to replay
+ * a selection, e.g. an external decision at exact or near ties.  NULL, NULL
+ * disarms.  Out-of-range slots are clamped into [0, N).
+ */
+fwpkm_status fwpkm_force_selection(fwpkm_state *s, const int32_t *slots, const uint8_t *mask);
+
+/*
+ * Per-kernel timing.  With profiling on, fwpkm_step records a CUDA event pair
+ * around every kernel it enqueues; fwpkm_profile_read synchronises `stream`,
+ * adds up the elapsed times per kernel kind, and returns them:
+ *   names[i] (static strings), ms[i] (total milliseconds), launches[i],
+ *   for i < *count (<= max_kinds).  Reading resets the totals.
+ */
+fwpkm_status fwpkm_set_profiling(fwpkm_state *s, int enable);
+fwpkm_status fwpkm_profile_read(fwpkm_state *s, const char **names, double *ms,
+                                int64_t *launches, int max_kinds, int *count, void *stream);
+
+/*
+ * fwpkm_read_stats -- counters accumulated on the device since the last
+ * reset (synchronises `stream`): chunks processed, and the sums over those
+ * chunks of distinct value rows written and distinct sub-key rows written
+ * (the write traffic of the step is proportional to these).  device_errors
+ * receives the sticky device error bits (1 = a bounded wait in a kernel gave
+ * up); when any is set the call returns FWPKM_ECUDA.  reset != 0 zeroes the
+ * counters and the bits after reading.  Any output pointer may be NULL.
+ */
+fwpkm_status fwpkm_read_stats(fwpkm_state *s, int64_t *chunks, int64_t *value_rows,
+                              int64_t *key_rows, uint32_t *device_errors, int reset,
+                              void *stream);
+
+/* Message of the last failure on this thread ("" if none). */
+const char *fwpkm_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FWPKM_H_ */

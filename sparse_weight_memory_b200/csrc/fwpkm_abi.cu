@@ -1,0 +1,494 @@
+// fwpkm_abi.cu -- host side of the C ABI declared in include/fwpkm.h.
+//
+// The state owns the fast weights (sub-key tables and value table, fp32) and
+// one device scratch arena sized for the largest chunk seen.  fwpkm_step
+// validates everything on the host, then enqueues the per-chunk kernel
+// sequence on the caller's stream with no host synchronisation: chunk c+1's
+// kernels are ordered after chunk c's update by the stream itself
+// (gist.science section 2: updates are applied after a chunk; the next chunk
+// reads the updated weights).
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/fwpkm.h"
+#include "fwpkm_internal.cuh"
+
+using namespace fwpkm;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+fwpkm_status fail(fwpkm_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+fwpkm_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(FWPKM_ECUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+enum Kind { K_PREP, K_SCORE, K_TOPK, K_SCAN, K_READ, K_VAPPLY, K_PGRAD, K_KAPPLY, K_COUNT };
+const char *kKindNames[K_COUNT] = {"fwpkm_prep", "fwpkm_score",  "fwpkm_topk",  "fwpkm_scan",
+                                   "fwpkm_read", "fwpkm_vapply", "fwpkm_pgrad", "fwpkm_kapply"};
+
+struct Timing {
+  int kind;
+  cudaEvent_t a, b;
+};
+
+}  // namespace
+
+struct fwpkm_state {
+  int64_t N = 0;
+  int n = 0, dq = 0, dh = 0, dv = 0, k = 0, chunk = 0, H = 0;
+  int64_t G = 0;
+  float eps = 1e-3f;
+  int device = 0;
+  float *K = nullptr;  // [H][2][n][dh]
+  float *V = nullptr;  // [N][dv]
+  // scratch arena
+  void *arena = nullptr;
+  size_t arena_bytes = 0;
+  int64_t cap_rows = 0;
+  Scratch s{};
+  // optional per-step inputs / outputs, armed for the next step
+  Extras x{};
+  // host-buffer staging
+  void *stage = nullptr;
+  size_t stage_bytes = 0;
+  // profiling
+  bool profiling = false;
+  std::vector<Timing> timings;
+  std::vector<cudaEvent_t> event_pool;
+  double prof_ms[K_COUNT] = {};
+  int64_t prof_n[K_COUNT] = {};
+};
+
+namespace {
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Carve the scratch arena for `rows` token rows per chunk.
+fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
+  if (rows <= st->cap_rows) return FWPKM_OK;
+  const int64_t H = st->H, n = st->n, dh = st->dh, dv = st->dv, k = st->k;
+  const int64_t M = rows * H, P = M * k, G = st->G;
+  const int64_t tiles = (G + kScanTile - 1) / kScanTile;
+  struct Piece {
+    void **ptr;
+    size_t bytes;
+  };
+  Scratch s{};
+  std::vector<Piece> pieces = {
+      {(void **)&s.Qs, sizeof(float) * (size_t)(H * 2 * rows * dh)},
+      {(void **)&s.qn, sizeof(float) * (size_t)(H * 2 * rows)},
+      {(void **)&s.kn, sizeof(float) * (size_t)(H * 2 * n)},
+      {(void **)&s.D, sizeof(float) * (size_t)(H * 2 * rows * n)},
+      {(void **)&s.pslot, sizeof(int32_t) * (size_t)P},
+      {(void **)&s.pw, sizeof(float) * (size_t)P},
+      {(void **)&s.pclaim, sizeof(int32_t) * (size_t)P},
+      {(void **)&s.pa, sizeof(float) * (size_t)P},
+      {(void **)&s.pb, sizeof(float) * (size_t)P},
+      {(void **)&s.pdl, sizeof(float) * (size_t)P},
+      {(void **)&s.esub, sizeof(int32_t) * (size_t)(2 * P)},
+      {(void **)&s.emask, sizeof(uint32_t) * (size_t)(2 * P)},
+      {(void **)&s.einv, sizeof(float) * (size_t)(2 * P)},
+      {(void **)&s.eclaim, sizeof(int32_t) * (size_t)(2 * P)},
+      {(void **)&s.ecount, sizeof(int32_t) * (size_t)(2 * M)},
+      {(void **)&s.count, sizeof(int32_t) * (size_t)G},
+      {(void **)&s.goff, sizeof(int32_t) * (size_t)G},
+      {(void **)&s.uniq, sizeof(int32_t) * (size_t)(3 * P)},
+      {(void **)&s.useg_off, sizeof(int32_t) * (size_t)(3 * P)},
+      {(void **)&s.useg_len, sizeof(int32_t) * (size_t)(3 * P)},
+      {(void **)&s.sorted, sizeof(int32_t) * (size_t)(3 * P)},
+      {(void **)&s.E, sizeof(float) * (size_t)(rows * dv)},
+      {(void **)&s.tile_cnt, sizeof(int32_t) * (size_t)tiles},
+      {(void **)&s.tile_nz, sizeof(int32_t) * (size_t)tiles},
+      {(void **)&s.meta, sizeof(Meta)},
+  };
+  size_t total = 0;
+  for (auto &p : pieces) total = align_up(total, 256) + align_up(p.bytes, 256);
+  void *arena = nullptr;
+  cudaError_t e = cudaMalloc(&arena, total);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FWPKM_ENOMEM, "scratch allocation of %zu bytes failed: %s", total,
+                cudaGetErrorString(e));
+  }
+  size_t off = 0;
+  for (auto &p : pieces) {
+    off = align_up(off, 256);
+    *p.ptr = (char *)arena + off;
+    off += align_up(p.bytes, 256);
+  }
+  // Group counts start at zero; the meta block (stats) carries over.
+  e = cudaMemset(s.count, 0, sizeof(int32_t) * (size_t)G);
+  if (e == cudaSuccess) e = cudaMemset(s.meta, 0, sizeof(Meta));
+  if (e == cudaSuccess && st->s.meta)
+    e = cudaMemcpy(s.meta, st->s.meta, sizeof(Meta), cudaMemcpyDeviceToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(arena);
+    return cuda_fail(e, "scratch initialisation");
+  }
+  if (st->arena) {
+    cudaDeviceSynchronize();
+    cudaFree(st->arena);
+  }
+  st->arena = arena;
+  st->arena_bytes = total;
+  st->s = s;
+  st->cap_rows = rows;
+  return FWPKM_OK;
+}
+
+cudaEvent_t take_event(fwpkm_state *st) {
+  if (!st->event_pool.empty()) {
+    cudaEvent_t e = st->event_pool.back();
+    st->event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Launch wrapper: optional event pair around the kernel, error check after.
+template <typename F>
+fwpkm_status run(fwpkm_state *st, int kind, cudaStream_t stream, F &&launch) {
+  Timing t{kind, nullptr, nullptr};
+  if (st->profiling) {
+    t.a = take_event(st);
+    t.b = take_event(st);
+    cudaEventRecord(t.a, stream);
+  }
+  cudaError_t e = launch();
+  if (e != cudaSuccess) return cuda_fail(e, kKindNames[kind]);
+  if (st->profiling) {
+    cudaEventRecord(t.b, stream);
+    st->timings.push_back(t);
+  }
+  return FWPKM_OK;
+}
+
+bool is_dtype(int t) { return t == FWPKM_F32 || t == FWPKM_BF16; }
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char *fwpkm_last_error(void) { return g_last_error.c_str(); }
+
+fwpkm_status fwpkm_state_init(int64_t N, int dq, int dv, int topk, int chunk, int heads,
+                              fwpkm_state **out) {
+  if (!out) return fail(FWPKM_EINVAL, "state_init: out is NULL");
+  *out = nullptr;
+  int64_t n = (int64_t)std::llround(std::sqrt((double)N));
+  while (n * n > N) --n;
+  while ((n + 1) * (n + 1) <= N) ++n;
+  if (N < 16 || n * n != N || n > FWPKM_MAX_SUBKEYS)
+    return fail(FWPKM_ESHAPE, "state_init: N=%lld must be n*n with 4 <= n <= %d", (long long)N,
+                FWPKM_MAX_SUBKEYS);
+  if (dq < 16 || dq % 16 != 0 || dq / 2 > 1024)
+    return fail(FWPKM_ESHAPE, "state_init: dq=%d must be a multiple of 16 (dq/2 a multiple of 8), <= 2048", dq);
+  if (dv < 4 || dv % 4 != 0 || dv > 2048)
+    return fail(FWPKM_ESHAPE, "state_init: dv=%d must be a multiple of 4 in [4, 2048]", dv);
+  if (topk < 1 || topk > FWPKM_MAX_TOPK || topk > n)
+    return fail(FWPKM_ESHAPE, "state_init: topk=%d must be in [1, min(n=%lld, %d)]", topk,
+                (long long)n, FWPKM_MAX_TOPK);
+  if (chunk < 1 || chunk > (1 << 20))
+    return fail(FWPKM_ESHAPE, "state_init: chunk=%d must be in [1, 2^20]", chunk);
+  if (heads < 1 || heads > 16)
+    return fail(FWPKM_ESHAPE, "state_init: heads=%d must be in [1, 16]", heads);
+
+  fwpkm_state *st = new (std::nothrow) fwpkm_state();
+  if (!st) return fail(FWPKM_ENOMEM, "state_init: host allocation failed");
+  st->N = N;
+  st->n = (int)n;
+  st->dq = dq;
+  st->dh = dq / 2;
+  st->dv = dv;
+  st->k = topk;
+  st->chunk = chunk;
+  st->H = heads;
+  st->G = N + 2ll * heads * n;
+  cudaGetDevice(&st->device);
+  const size_t kbytes = sizeof(float) * (size_t)heads * 2 * n * st->dh;
+  const size_t vbytes = sizeof(float) * (size_t)N * dv;
+  cudaError_t e = cudaMalloc(&st->K, kbytes);
+  if (e == cudaSuccess) e = cudaMalloc(&st->V, vbytes);
+  if (e == cudaSuccess) e = cudaMemset(st->K, 0, kbytes);
+  if (e == cudaSuccess) e = cudaMemset(st->V, 0, vbytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(st->K);
+    cudaFree(st->V);
+    delete st;
+    return fail(e == cudaErrorMemoryAllocation ? FWPKM_ENOMEM : FWPKM_ECUDA,
+                "state_init: table allocation (%zu + %zu bytes): %s", kbytes, vbytes,
+                cudaGetErrorString(e));
+  }
+  fwpkm_status rc = ensure_scratch(st, chunk);
+  if (rc != FWPKM_OK) {
+    cudaFree(st->K);
+    cudaFree(st->V);
+    delete st;
+    return rc;
+  }
+  *out = st;
+  return FWPKM_OK;
+}
+
+void fwpkm_state_free(fwpkm_state *st) {
+  if (!st) return;
+  cudaDeviceSynchronize();
+  for (auto &t : st->timings) {
+    cudaEventDestroy(t.a);
+    cudaEventDestroy(t.b);
+  }
+  for (auto e : st->event_pool) cudaEventDestroy(e);
+  cudaFree(st->arena);
+  cudaFree(st->stage);
+  cudaFree(st->K);
+  cudaFree(st->V);
+  delete st;
+}
+
+fwpkm_status fwpkm_state_set_eps(fwpkm_state *st, float eps) {
+  if (!st) return fail(FWPKM_EINVAL, "set_eps: state is NULL");
+  if (!(eps > 0.f) || !std::isfinite(eps)) return fail(FWPKM_EINVAL, "set_eps: eps must be > 0");
+  st->eps = eps;
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtype,
+                        const void *Vtarget, int v_dtype, const float *gate, float eta,
+                        float lambda_entropy, float *out, void *stream_) {
+  if (!st) return fail(FWPKM_EINVAL, "step: state is NULL");
+  if (!Q || !Vtarget || !gate || !out) return fail(FWPKM_EINVAL, "step: NULL tensor pointer");
+  if (!is_dtype(q_dtype) || !is_dtype(v_dtype))
+    return fail(FWPKM_EINVAL, "step: dtype must be FWPKM_F32 or FWPKM_BF16");
+  if (B < 1 || T < 1) return fail(FWPKM_ESHAPE, "step: B=%d and T=%d must be >= 1", B, T);
+  if (!(eta >= 0.f) || !std::isfinite(eta))
+    return fail(FWPKM_EINVAL, "step: eta must be finite and >= 0");
+  if (!(lambda_entropy >= 0.f) || !std::isfinite(lambda_entropy))
+    return fail(FWPKM_EINVAL, "step: lambda_entropy must be finite and >= 0");
+  const int64_t rows_max = (int64_t)B * (T < st->chunk ? T : st->chunk);
+  if (rows_max * st->H * st->k * 3 >= (int64_t)1 << 31 || (int64_t)B * T * st->dv >= (int64_t)1 << 40)
+    return fail(FWPKM_ESHAPE, "step: B*chunk*heads*topk too large for 32-bit pair ids");
+  if ((((uintptr_t)Q) | ((uintptr_t)Vtarget) | ((uintptr_t)out)) & 15)
+    return fail(FWPKM_EINVAL, "step: Q, Vtarget and out must be 16-byte aligned");
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (dev != st->device)
+    return fail(FWPKM_EINVAL, "step: current device %d is not the state's device %d", dev,
+                st->device);
+  fwpkm_status rc = ensure_scratch(st, rows_max);
+  if (rc != FWPKM_OK) return rc;
+  cudaStream_t stream = (cudaStream_t)stream_;
+  Extras x = st->x;
+  st->x = Extras{};  // armed extras apply to this step only
+
+  const Scratch &s = st->s;
+  cudaError_t e = cudaMemsetAsync(s.count, 0, sizeof(int32_t) * (size_t)st->G, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "step: memset");
+  const int n_chunks = (T + st->chunk - 1) / st->chunk;
+  for (int c = 0; c < n_chunks; ++c) {
+    Dims d{};
+    d.n = st->n;
+    d.dq = st->dq;
+    d.dh = st->dh;
+    d.dv = st->dv;
+    d.k = st->k;
+    d.H = st->H;
+    d.N = st->N;
+    d.B = B;
+    d.T = T;
+    d.t0 = c * st->chunk;
+    d.Tc = (T - d.t0 < st->chunk) ? T - d.t0 : st->chunk;
+    d.rows = B * d.Tc;
+    d.M = d.rows * st->H;
+    d.G = (int)st->G;
+    d.eps = st->eps;
+    d.eta = eta;
+    d.lam = lambda_entropy;
+    if ((rc = run(st, K_PREP, stream, [&] { return launch_prep(d, Q, q_dtype, st->K, s, stream); })))
+      return rc;
+    if ((rc = run(st, K_SCORE, stream, [&] { return launch_score(d, st->K, s, stream); })))
+      return rc;
+    if ((rc = run(st, K_TOPK, stream, [&] { return launch_topk(d, s, x, stream); }))) return rc;
+    if ((rc = run(st, K_SCAN, stream, [&] { return launch_scan(d, s, stream, 0); }))) return rc;
+    if ((rc = run(st, K_SCAN, stream, [&] { return launch_scan(d, s, stream, 1); }))) return rc;
+    if ((rc = run(st, K_READ, stream, [&] {
+           return launch_read(d, st->V, Vtarget, v_dtype, gate, out, s, stream);
+         })))
+      return rc;
+    if ((rc = run(st, K_VAPPLY, stream, [&] { return launch_vapply(d, st->V, gate, s, stream); })))
+      return rc;
+    if ((rc = run(st, K_PGRAD, stream, [&] { return launch_pgrad(d, s, stream); }))) return rc;
+    if ((rc = run(st, K_KAPPLY, stream, [&] { return launch_kapply(d, st->K, s, stream); })))
+      return rc;
+  }
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_step_host(fwpkm_state *st, int B, int T, const void *Q_host, int q_dtype,
+                             const void *Vt_host, int v_dtype, const float *gate_host,
+                             float eta, float lambda_entropy, float *out_host, void *stream_) {
+  if (!st) return fail(FWPKM_EINVAL, "step_host: state is NULL");
+  if (!Q_host || !Vt_host || !gate_host || !out_host)
+    return fail(FWPKM_EINVAL, "step_host: NULL tensor pointer");
+  if (!is_dtype(q_dtype) || !is_dtype(v_dtype))
+    return fail(FWPKM_EINVAL, "step_host: dtype must be FWPKM_F32 or FWPKM_BF16");
+  if (B < 1 || T < 1) return fail(FWPKM_ESHAPE, "step_host: B=%d and T=%d must be >= 1", B, T);
+  const size_t tok = (size_t)B * T;
+  const size_t qb = tok * st->H * st->dq * (q_dtype == FWPKM_BF16 ? 2 : 4);
+  const size_t vb = tok * st->dv * (v_dtype == FWPKM_BF16 ? 2 : 4);
+  const size_t gb = tok * 4, ob = tok * st->dv * 4;
+  const size_t oq = 0, ov = align_up(qb, 256), og = ov + align_up(vb, 256),
+               oo = og + align_up(gb, 256), total = oo + align_up(ob, 256);
+  if (total > st->stage_bytes) {
+    cudaDeviceSynchronize();
+    cudaFree(st->stage);
+    st->stage = nullptr;
+    st->stage_bytes = 0;
+    cudaError_t e = cudaMalloc(&st->stage, total);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(FWPKM_ENOMEM, "step_host: staging allocation of %zu bytes failed", total);
+    }
+    st->stage_bytes = total;
+  }
+  cudaStream_t stream = (cudaStream_t)stream_;
+  char *base = (char *)st->stage;
+  cudaError_t e = cudaMemcpyAsync(base + oq, Q_host, qb, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(base + ov, Vt_host, vb, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(base + og, gate_host, gb, cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "step_host: host-to-device copy");
+  fwpkm_status rc = fwpkm_step(st, B, T, base + oq, q_dtype, base + ov, v_dtype,
+                               (const float *)(base + og), eta, lambda_entropy,
+                               (float *)(base + oo), stream_);
+  if (rc != FWPKM_OK) return rc;
+  e = cudaMemcpyAsync(out_host, base + oo, ob, cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "step_host: device-to-host copy");
+  e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "step_host: synchronise");
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_state_get(const fwpkm_state *st, float *subkeys, float *values, void *stream) {
+  if (!st) return fail(FWPKM_EINVAL, "state_get: state is NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (subkeys)
+    e = cudaMemcpyAsync(subkeys, st->K, sizeof(float) * (size_t)st->H * 2 * st->n * st->dh,
+                        cudaMemcpyDefault, s);
+  if (e == cudaSuccess && values)
+    e = cudaMemcpyAsync(values, st->V, sizeof(float) * (size_t)st->N * st->dv,
+                        cudaMemcpyDefault, s);
+  if (e != cudaSuccess) return cuda_fail(e, "state_get");
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_state_set(fwpkm_state *st, const float *subkeys, const float *values,
+                             void *stream) {
+  if (!st) return fail(FWPKM_EINVAL, "state_set: state is NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (subkeys)
+    e = cudaMemcpyAsync(st->K, subkeys, sizeof(float) * (size_t)st->H * 2 * st->n * st->dh,
+                        cudaMemcpyDefault, s);
+  if (e == cudaSuccess && values)
+    e = cudaMemcpyAsync(st->V, values, sizeof(float) * (size_t)st->N * st->dv,
+                        cudaMemcpyDefault, s);
+  if (e != cudaSuccess) return cuda_fail(e, "state_set");
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_record_selection(fwpkm_state *st, int32_t *slots, float *weights) {
+  if (!st) return fail(FWPKM_EINVAL, "record_selection: state is NULL");
+  if ((slots == nullptr) != (weights == nullptr))
+    return fail(FWPKM_EINVAL, "record_selection: give both buffers or neither");
+  st->x.rec_slots = slots;
+  st->x.rec_w = weights;
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_force_selection(fwpkm_state *st, const int32_t *slots, const uint8_t *mask) {
+  if (!st) return fail(FWPKM_EINVAL, "force_selection: state is NULL");
+  if ((slots == nullptr) != (mask == nullptr))
+    return fail(FWPKM_EINVAL, "force_selection: give both buffers or neither");
+  st->x.force_slots = slots;
+  st->x.force_mask = mask;
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_set_profiling(fwpkm_state *st, int enable) {
+  if (!st) return fail(FWPKM_EINVAL, "set_profiling: state is NULL");
+  st->profiling = enable != 0;
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_profile_read(fwpkm_state *st, const char **names, double *ms,
+                                int64_t *launches, int max_kinds, int *count, void *stream) {
+  if (!st) return fail(FWPKM_EINVAL, "profile_read: state is NULL");
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "profile_read: synchronise");
+  for (auto &t : st->timings) {
+    float dt = 0.f;
+    if (cudaEventElapsedTime(&dt, t.a, t.b) == cudaSuccess) {
+      st->prof_ms[t.kind] += dt;
+      st->prof_n[t.kind] += 1;
+    }
+    st->event_pool.push_back(t.a);
+    st->event_pool.push_back(t.b);
+  }
+  st->timings.clear();
+  int c = 0;
+  for (int i = 0; i < K_COUNT && c < max_kinds; ++i, ++c) {
+    if (names) names[c] = kKindNames[i];
+    if (ms) ms[c] = st->prof_ms[i];
+    if (launches) launches[c] = st->prof_n[i];
+    st->prof_ms[i] = 0.0;
+    st->prof_n[i] = 0;
+  }
+  if (count) *count = c;
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_read_stats(fwpkm_state *st, int64_t *chunks, int64_t *value_rows,
+                              int64_t *key_rows, uint32_t *device_errors, int reset,
+                              void *stream) {
+  if (!st) return fail(FWPKM_EINVAL, "read_stats: state is NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  Meta m{};
+  cudaError_t e = cudaMemcpyAsync(&m, st->s.meta, sizeof(Meta), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "read_stats");
+  if (chunks) *chunks = (int64_t)m.stat_chunks;
+  if (value_rows) *value_rows = (int64_t)m.stat_value_rows;
+  if (key_rows) *key_rows = (int64_t)(m.stat_total_rows - m.stat_value_rows);
+  if (device_errors) *device_errors = m.err;
+  if (reset) {
+    Meta z{};
+    e = cudaMemcpyAsync(st->s.meta, &z, sizeof(Meta), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "read_stats: reset");
+  }
+  if (m.err) return fail(FWPKM_ECUDA, "device error bits 0x%x (1 = bounded wait timed out)", m.err);
+  return FWPKM_OK;
+}
+
+}  // extern "C"

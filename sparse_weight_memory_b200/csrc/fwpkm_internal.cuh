@@ -1,0 +1,188 @@
+// fwpkm_internal.cuh -- shared declarations of the sm_100a FwPKM kernels.
+//
+// Per chunk the host enqueues, in order:
+//   prep    -> split the chunk's queries into halves (fp32), |q|^2, |K|^2
+//   score   -> D[h][half][row][i] = |q_half - K_h,half,i|^2 for every sub-key
+//   topk    -> per token-head: top-k per half, k*k merge, softmax; claims of
+//              the (slot) and (sub-key) groups the pair will write
+//   scan    -> group offsets / unique group list over slots and sub-keys
+//   read    -> gather the selected value rows, out = g * yhat, residual e,
+//              dL/dw per pair; scatter pair / entry ids into group order
+//   vapply  -> per touched value row: ordered segmented sum, V -= eta G / C,
+//              marginal p_bar -> entropy term per pair
+//   pgrad   -> per token-head: dL/ds through the softmax Jacobian
+//   kapply  -> per touched sub-key row: ordered sum, K -= eta dL/dK
+// No floating-point atomics anywhere: every sum runs in a fixed order
+// (pairs sorted by id inside each group), so two runs are bit-identical.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace fwpkm {
+
+constexpr unsigned FULL = 0xffffffffu;
+constexpr int kScanTile = 2048;      // group-count scan: elements per CTA
+constexpr int kWarpSortMax = 1024;   // largest group sorted in warp-private smem
+
+// Device-side error bits (meta->err).
+enum : unsigned {
+  ERR_MBAR_TIMEOUT = 1u,   // a bounded mbarrier wait gave up
+};
+
+// Written by the scan kernels, read by the apply kernels and the host.
+struct Meta {
+  int32_t U_v;            // distinct value rows touched in the chunk
+  int32_t U_total;        // distinct value rows + distinct sub-key rows
+  unsigned err;           // ERR_* bits, sticky until the host clears them
+  int32_t pad;
+  unsigned long long stat_chunks;      // chunks processed since reset
+  unsigned long long stat_value_rows;  // sum over chunks of U_v
+  unsigned long long stat_total_rows;  // sum over chunks of U_total
+};
+
+// Shapes of the chunk being processed.
+struct Dims {
+  int n, dq, dh, dv, k, H;
+  int64_t N;
+  int B, T, t0, Tc;   // batch, call length, first token of the chunk, its length
+  int rows;           // B * Tc
+  int M;              // rows * H token-heads
+  int G;              // N + 2*H*n groups (value rows, then sub-key rows)
+  float eps, eta, lam;
+};
+
+// Device scratch owned by the state (sized for the largest chunk seen).
+struct Scratch {
+  float *Qs;        // [H][2][rows][dh]   query halves of the chunk, fp32
+  float *qn;        // [H][2][rows]       |q_half|^2
+  float *kn;        // [H][2][n]          |K_row|^2
+  float *D;         // [H][2][rows][n]    squared distances
+  int32_t *pslot;   // [M*k] selected slot of pair p = m*k + r
+  float *pw;        // [M*k] softmax weight
+  int32_t *pclaim;  // [M*k] position inside the slot's group
+  float *pa;        // [M*k] dL_mse/dw
+  float *pb;        // [M*k] dL_addr/dw (lam > 0)
+  float *pdl;       // [M*k] dL/ds
+  int32_t *esub;    // [2*M*k] sub-key row of entry e = (m*2+half)*k + idx
+  uint32_t *emask;  // [2*M*k] pairs r of token-head m that use that row
+  float *einv;      // [2*M*k] 1 / (eps + d_half(row))
+  int32_t *eclaim;  // [2*M*k] position inside the sub-key row's group
+  int32_t *ecount;  // [M*2]   entries per (m, half)
+  int32_t *count;   // [G] members per group (zero between chunks)
+  int32_t *goff;    // [G] first position of the group in `sorted`
+  int32_t *uniq;    // [M*k*3] touched groups in group order
+  int32_t *useg_off;
+  int32_t *useg_len;
+  int32_t *sorted;  // [M*k*3] pair ids (value groups) then entry ids (sub-key groups)
+  float *E;         // [rows][dv] residual yhat - v
+  int32_t *tile_cnt;  // [ceil(G / kScanTile)]
+  int32_t *tile_nz;
+  Meta *meta;
+};
+
+// Optional per-step inputs/outputs.
+struct Extras {
+  const int32_t *force_slots;  // [B][T][H][k] or null
+  const uint8_t *force_mask;   // [B][T][H]
+  int32_t *rec_slots;          // [B][T][H][k] or null
+  float *rec_w;
+};
+
+// ------------------------------------------------------------------------
+// Device helpers
+// ------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, o));
+  return v;
+}
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+__device__ __forceinline__ float load_elem(const float *p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float load_elem(const __nv_bfloat16 *p, int64_t i) {
+  return __bfloat162float(p[i]);
+}
+// Four consecutive elements starting at a multiple of 4.
+__device__ __forceinline__ float4 load4(const float *p, int64_t i) {
+  return *reinterpret_cast<const float4 *>(p + i);
+}
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p, int64_t i) {
+  uint2 raw = *reinterpret_cast<const uint2 *>(p + i);
+  __nv_bfloat162 lo = *reinterpret_cast<__nv_bfloat162 *>(&raw.x);
+  __nv_bfloat162 hi = *reinterpret_cast<__nv_bfloat162 *>(&raw.y);
+  float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
+// --- mbarrier + bulk async copy (TMA, non-tensor form) -------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: gives up after `limit` polls (each try_wait may itself block
+// for a hardware-defined interval), records ERR_MBAR_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity, Meta *meta,
+                                                  long long limit = (1ll << 26)) {
+  for (long long it = 0; it < limit; ++it)
+    if (mbar_try_wait(bar, parity)) return true;
+  atomicOr(&meta->err, ERR_MBAR_TIMEOUT);
+  return false;
+}
+// 1-D bulk copy global -> shared, completion counted on `bar` (bytes % 16 == 0,
+// both addresses 16-byte aligned).
+__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, unsigned bytes,
+                                         uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst_smem)),
+      "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ------------------------------------------------------------------------
+// Host-side launchers (one per kernel file)
+// ------------------------------------------------------------------------
+cudaError_t launch_prep(const Dims &d, const void *Q, int q_dtype, const float *K,
+                        const Scratch &s, cudaStream_t st);
+cudaError_t launch_score(const Dims &d, const float *K, const Scratch &s, cudaStream_t st);
+cudaError_t launch_topk(const Dims &d, const Scratch &s, const Extras &x, cudaStream_t st);
+cudaError_t launch_scan(const Dims &d, const Scratch &s, cudaStream_t st, int part);
+cudaError_t launch_read(const Dims &d, const float *V, const void *Vt, int v_dtype,
+                        const float *gate, float *out, const Scratch &s, cudaStream_t st);
+cudaError_t launch_vapply(const Dims &d, float *V, const float *gate, const Scratch &s,
+                          cudaStream_t st);
+cudaError_t launch_pgrad(const Dims &d, const Scratch &s, cudaStream_t st);
+cudaError_t launch_kapply(const Dims &d, float *K, const Scratch &s, cudaStream_t st);
+
+}  // namespace fwpkm

@@ -1,0 +1,81 @@
+"""Host-only checks of the C ABI: the library loads without a GPU, exports
+every entry point include/fwpkm.h declares, and rejects bad arguments on the
+host with the documented status codes (before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_weight_memory_b200 import build as fwbuild
+from sparse_weight_memory_b200 import fwpkm
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fwpkm.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fwbuild.build()
+    return fwpkm.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fwpkm_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("fwpkm_state_init", "fwpkm_step", "fwpkm_state_get", "fwpkm_state_set",
+                     "fwpkm_state_free", "fwpkm_last_error"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in fwpkm.h but not exported"
+
+
+@pytest.mark.parametrize("N,dq,dv,topk,chunk,heads", [
+    (1000, 64, 64, 4, 32, 1),      # N not a perfect square
+    (9, 64, 64, 2, 32, 1),         # n = 3 < 4
+    (1024, 10, 64, 4, 32, 1),      # dq not a multiple of 16
+    (1024, 64, 6, 4, 32, 1),       # dv not a multiple of 4
+    (1024, 64, 64, 33, 32, 1),     # topk > 32
+    (16 * 16, 64, 64, 17, 32, 1),  # topk > n
+    (1024, 64, 64, 0, 32, 1),      # topk < 1
+    (1024, 64, 64, 4, 0, 1),       # chunk < 1
+    (1024, 64, 64, 4, 32, 0),      # heads < 1
+    (4096 * 4096, 64, 64, 4, 32, 1),  # n > 2048
+])
+def test_state_init_rejects_bad_shapes(lib, N, dq, dv, topk, chunk, heads):
+    h = ctypes.c_void_p()
+    rc = lib.fwpkm_state_init(N, dq, dv, topk, chunk, heads, ctypes.byref(h))
+    assert rc == fwpkm.FWPKM_ESHAPE
+    assert h.value is None
+    assert lib.fwpkm_last_error().decode()
+
+
+def test_null_arguments_are_rejected(lib):
+    assert lib.fwpkm_state_init(1024, 64, 64, 4, 32, 1, None) == fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_step(None, 1, 1, None, 0, None, 0, None, 1.0, 0.0, None, None) == \
+        fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_state_get(None, None, None, None) == fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_state_set(None, None, None, None) == fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_state_set_eps(None, 1e-3) == fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_record_selection(None, None, None) == fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_force_selection(None, None, None) == fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_read_stats(None, None, None, None, None, 0, None) == fwpkm.FWPKM_EINVAL
+    lib.fwpkm_state_free(None)  # no-op
+
+
+def test_product_path_has_no_oracle_or_fallback():
+    """The library package never imports the oracle (test infrastructure)."""
+    pkg = os.path.join(ROOT, "sparse_weight_memory_b200")
+    pat = re.compile(r"^\s*(from|import)\s+oracle\b|ctypes\.CDLL\(.*oracle", re.M)
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith(".py"):
+                assert not pat.search(open(os.path.join(dirpath, f)).read()), f
