@@ -1,0 +1,406 @@
+"""Benchmark of the FwPKM chunked read-then-write step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload library]
+                    [--impl reference]
+
+A step is one pass of the whole hot path over one batch of the workload: for
+the default `library` workload (B=2, T=4096, chunk 256, N=65,536 slots,
+dq=dv=512, topk 8) that is 3 chained calls = 48 chunks = 24,576 tokens,
+each chunk read and then written.  Inputs are resident in HBM when the timed
+region starts; between steps (untimed) the tables are reset to their initial
+values and L2 is flushed by writing a 256 MiB buffer.  Every step is timed
+with CUDA events on the launching stream.
+
+Multi-GPU: the step does not shard (chunks are sequential and all token-heads
+of a chunk write one shared table), so `--gpus N` runs N independent
+replicas, one per GPU, with no collective on the data path (weak scaling);
+torch.distributed only provides the barrier and the max-over-ranks time.
+
+`--impl reference` times the fp64 CPU oracle (the only reference this method
+has) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_weight_memory_b200.workloads import BF16, WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "FwPKM tokens/sec (read+write per chunk), 1xB200; % of HBM/tensor roofline"
+UNIT = "tokens/s"
+
+
+def describe(wl) -> str:
+    s = (f"{wl.name}: B={wl.B} T={wl.T} chunk={wl.chunk} heads={wl.heads} dq={wl.dq} "
+         f"n={wl.n} (N={wl.N}) dv={wl.dv} topk={wl.topk} eta={wl.eta} "
+         f"lambda={wl.lam} gate={wl.gate} inputs={'bf16' if wl.in_dtype == BF16 else 'f32'}")
+    if wl.calls > 1:
+        s += f" x{wl.calls} chained calls"
+    if wl.passes > 1:
+        s += f" x{wl.passes} passes"
+    return s
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except FileNotFoundError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# oracle (CPU) arm
+# ---------------------------------------------------------------------------
+def oracle_sample(wl, inp, budget_s: float = 20.0):
+    """Time the fp64 oracle on the first calls of one workload step (all chunks
+    of each call it starts), stopping once `budget_s` of CPU time is spent."""
+    from oracle import oracle as orc
+    st = orc.State(inp.subkeys, inp.values, topk=wl.topk, chunk=wl.chunk, eps=wl.eps)
+    tokens, elapsed, calls = 0, 0.0, 0
+    n_chunks = wl.n_chunks()
+    per_call_chunks = n_chunks
+    seq = []
+    for c in range(wl.calls):
+        sl = slice(c * wl.T, (c + 1) * wl.T)
+        for _ in range(wl.passes):
+            seq.append(sl)
+    for sl in seq:
+        Q = inp.q_f32()[:, sl].astype(np.float64)
+        Vt = inp.vt_f32()[:, sl].astype(np.float64)
+        g = inp.gate[:, sl]
+        # a bounded number of chunks per call when one call alone is too long
+        t0 = time.perf_counter()
+        st.step(Q, Vt, g, wl.eta, wl.lam, max_chunks=per_call_chunks)
+        dt = time.perf_counter() - t0
+        elapsed += dt
+        tokens += wl.B * min(wl.T, per_call_chunks * wl.chunk)
+        calls += 1
+        if elapsed >= budget_s:
+            break
+        if calls == 1 and dt > budget_s / 2 and per_call_chunks > 1:
+            per_call_chunks = max(1, int(per_call_chunks * (budget_s / 2) / dt))
+    sample = (f"{calls} call(s) of the workload step, {tokens} tokens "
+              f"({'all' if per_call_chunks == n_chunks else per_call_chunks} of {n_chunks} "
+              f"chunks per call), fp64 oracle")
+    return tokens / elapsed, elapsed, sample, orc.num_threads()
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = make_inputs(wl)
+    vals = []
+    info = None
+    for i in range(args.warmup + args.steps):
+        v, el, sample, cores = oracle_sample(wl, inp, budget_s=args.ref_budget)
+        if i >= args.warmup:
+            vals.append((v, el))
+        info = (sample, cores)
+    tok_s = statistics.median([v for v, _ in vals])
+    ms = statistics.median([el for _, el in vals]) * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": tok_s, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(wl)},
+            "cpu_baseline": {"value": tok_s, "unit": UNIT, "cores": info[1], "kind": "oracle",
+                             "sample": info[0]},
+            "e2e": {"value": tok_s, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def algorithmic_work(wl, tokens, value_rows, key_rows):
+    """Algorithmic bytes (HBM-bound kernels) or flops (score) over `tokens`
+    tokens whose chunks wrote `value_rows` / `key_rows` distinct rows."""
+    in_b = 2 if wl.in_dtype == BF16 else 4
+    gather = tokens * wl.heads * wl.topk * wl.dv * 4
+    return {
+        # gathered value rows + Vtarget read + out written
+        "fwpkm_read": ("hbm", gather + tokens * wl.dv * in_b + tokens * wl.dv * 4),
+        # read-modify-write of every touched value row and sub-key row
+        "fwpkm_apply": ("hbm", 2 * value_rows * wl.dv * 4 + 2 * key_rows * (wl.dq // 2) * 4),
+        # q_half . K_row for every sub-key of both halves
+        "fwpkm_score": ("alu", 2.0 * tokens * wl.heads * wl.n * wl.dq),
+    }
+
+
+# fp32 FMA peak of the SIMT pipes: 148 SMs x 128 lanes x 2 flops x 1.965 GHz
+SIMT_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_gpu(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    from sparse_weight_memory_b200 import FwPKMState, load_library
+    from sparse_weight_memory_b200 import build as fwbuild
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    if rank == 0:
+        fwbuild.build()
+    if world > 1:
+        dist.barrier()
+    load_library()
+
+    dev = torch.device("cuda", local)
+    inp = make_inputs(wl, seed=wl.seed + rank)  # independent replica per rank
+
+    def to_dev(a):
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    K0, V0 = to_dev(inp.subkeys), to_dev(inp.values)
+    segs = []
+    for c in range(wl.calls):
+        sl = slice(c * wl.T, (c + 1) * wl.T)
+        dq_, dv_, dg_ = to_dev(inp.Q[:, sl]), to_dev(inp.Vt[:, sl]), to_dev(inp.gate[:, sl])
+        for _ in range(wl.passes):
+            segs.append((dq_, dv_, dg_))
+    outs = [torch.empty((wl.B, wl.T, wl.dv), dtype=torch.float32, device=dev) for _ in segs]
+    st = FwPKMState(wl.N, wl.dq, wl.dv, wl.topk, wl.chunk, wl.heads, eps=wl.eps)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def reset():
+        st.set_tables(K0, V0)
+        flush.zero_()
+
+    def one_step():
+        for (q, v, g), o in zip(segs, outs):
+            st.step(q, v, g, wl.eta, wl.lam, out=o)
+
+    for _ in range(args.warmup):
+        reset()
+        one_step()
+    torch.cuda.synchronize()
+    st.read_stats(reset=True)
+
+    times = []
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for _ in range(args.steps):
+            reset()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            one_step()
+            b.record(stream)
+            times.append((a, b))
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in times]
+    total_ms = sum(step_ms)
+    stats = st.read_stats(reset=True)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms_max = float(t.item())
+    tokens_per_step = wl.tokens_per_step
+    value = tokens_per_step * args.steps * world / (total_ms_max / 1e3)
+
+    # per-kernel event timing (separate, instrumented steps)
+    st.set_profiling(True)
+    prof_steps = max(1, min(args.steps, 3))
+    for _ in range(prof_steps):
+        reset()
+        one_step()
+    torch.cuda.synchronize()
+    prof = st.profile_read()
+    st.set_profiling(False)
+    pstats = st.read_stats(reset=True)
+
+    # end to end through the C ABI with pinned host buffers
+    hsegs = []
+    for c in range(wl.calls):
+        sl = slice(c * wl.T, (c + 1) * wl.T)
+        hq = torch.from_numpy(np.ascontiguousarray(inp.Q[:, sl])).pin_memory().numpy()
+        hv = torch.from_numpy(np.ascontiguousarray(inp.Vt[:, sl])).pin_memory().numpy()
+        hg = torch.from_numpy(np.ascontiguousarray(inp.gate[:, sl])).pin_memory().numpy()
+        for _ in range(wl.passes):
+            hsegs.append((hq, hv, hg))
+    hout = torch.empty((wl.B, wl.T, wl.dv), dtype=torch.float32).pin_memory().numpy()
+    h2d = sum(q.nbytes + v.nbytes + g.nbytes for q, v, g in hsegs)
+    d2h = hout.nbytes * len(hsegs)
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        reset()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for q, v, g in hsegs:
+            st.step_host(q, v, g, wl.eta, wl.lam, out=hout)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    te = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = tokens_per_step * args.steps * world / (float(te.item()) / 1e3)
+
+    if rank == 0:
+        hbm_gbs, bf16_tf, peak_kind = peaks()
+        rows_sum = wl.B * wl.T * wl.calls * wl.passes * prof_steps
+        work = algorithmic_work(wl, rows_sum, pstats["value_rows"], pstats["key_rows"])
+        dominant = max(prof.items(), key=lambda kv: kv[1][0])[0]
+        dom_ms, dom_n = prof[dominant]
+        roofline = None
+        if dominant in work and dom_n > 0:
+            bound, amount = work[dominant]
+            per_launch = amount / dom_n
+            sec = dom_ms / dom_n / 1e3
+            if bound == "hbm":
+                achieved, peak, unit = per_launch / sec / 1e9, hbm_gbs, "GB/s"
+            else:
+                achieved, peak, unit = per_launch / sec / 1e12, SIMT_FP32_TFLOPS, "TFLOP/s"
+            roofline = {"kernel": dominant, "bound": bound, "achieved": achieved,
+                        "peak": peak, "unit": unit, "frac": achieved / peak,
+                        "traffic": None,
+                        "peak_kind": peak_kind if bound == "hbm" else "derived: SM count x clock"}
+        kernels = {k: {"ms_per_step": v[0] / prof_steps, "launches_per_step": v[1] / prof_steps}
+                   for k, v in prof.items()}
+        # whole-step roofline: gathered + scattered + streamed bytes at HBM peak
+        vrows = stats["value_rows"] / args.steps
+        in_b = 2 if wl.in_dtype == BF16 else 4
+        tok = wl.tokens_per_step
+        step_bytes = (tok * wl.heads * wl.topk * wl.dv * 4 + 2 * vrows * wl.dv * 4 +
+                      tok * (wl.heads * wl.dq * in_b + wl.dv * in_b + 4 + wl.dv * 4))
+        step_flops = 2.0 * tok * wl.heads * wl.n * wl.dq
+        t_roof = max(step_bytes / (hbm_gbs * 1e9), step_flops / (bf16_tf / 2 * 1e12))
+        clocks = clk.summary()
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            v, el, sample, cores = oracle_sample(wl, inp, budget_s=args.ref_budget)
+            cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        launches = sum(int(round(x["launches_per_step"])) for x in kernels.values()) * args.steps
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": describe(wl), "parallelism": f"replicas{world}",
+                       "l2": "flushed between steps (256 MiB write), tables reset untimed",
+                       "tokens_per_step": tokens_per_step},
+            "roofline": roofline,
+            "step_roofline": {"bytes_per_step": step_bytes, "flops_per_step": step_flops,
+                              "t_roof_ms": t_roof * 1e3,
+                              "frac": t_roof * 1e3 / (total_ms_max / args.steps),
+                              "value_rows_per_step": vrows},
+            "kernels": kernels,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    st.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="library", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--ref-budget", type=float, default=8.0,
+                    help="seconds of oracle time per reference sample (one step, or "
+                         "a prefix of it when one step takes longer)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_gpu(args, wl)
+
+
+if __name__ == "__main__":
+    main()

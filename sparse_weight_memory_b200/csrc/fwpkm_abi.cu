@@ -37,9 +37,9 @@ fwpkm_status cuda_fail(cudaError_t e, const char *what) {
   return fail(FWPKM_ECUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-enum Kind { K_PREP, K_SCORE, K_TOPK, K_SCAN, K_READ, K_VAPPLY, K_PGRAD, K_KAPPLY, K_COUNT };
-const char *kKindNames[K_COUNT] = {"fwpkm_prep", "fwpkm_score",  "fwpkm_topk",  "fwpkm_scan",
-                                   "fwpkm_read", "fwpkm_vapply", "fwpkm_pgrad", "fwpkm_kapply"};
+enum Kind { K_PREP, K_SCORE, K_TOPK, K_SCAN, K_READ, K_BSORT, K_APPLY, K_PGRAD, K_COUNT };
+const char *kKindNames[K_COUNT] = {"fwpkm_prep", "fwpkm_score", "fwpkm_topk",  "fwpkm_scan",
+                                   "fwpkm_read", "fwpkm_bsort", "fwpkm_apply", "fwpkm_pgrad"};
 
 struct Timing {
   int kind;
@@ -51,9 +51,9 @@ struct Timing {
 struct fwpkm_state {
   int64_t N = 0;
   int n = 0, dq = 0, dh = 0, dv = 0, k = 0, chunk = 0, H = 0;
-  int64_t G = 0;
   float eps = 1e-3f;
   int device = 0;
+  int sm_count = 148;
   float *K = nullptr;  // [H][2][n][dh]
   float *V = nullptr;  // [N][dv]
   // scratch arena
@@ -78,12 +78,25 @@ namespace {
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Value rows are bucketed by slot >> vshift, at most 8192 buckets.
+int value_shift(int64_t N) {
+  int sh = 0;
+  while (((N + (1ll << sh) - 1) >> sh) > 8192) ++sh;
+  return sh;
+}
+int64_t value_buckets(int64_t N) {
+  const int sh = value_shift(N);
+  return (N + (1ll << sh) - 1) >> sh;
+}
+
 // Carve the scratch arena for `rows` token rows per chunk.
 fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
   if (rows <= st->cap_rows) return FWPKM_OK;
   const int64_t H = st->H, n = st->n, dh = st->dh, dv = st->dv, k = st->k;
-  const int64_t M = rows * H, P = M * k, G = st->G;
-  const int64_t tiles = (G + kScanTile - 1) / kScanTile;
+  const int64_t M = rows * H, P = M * k, NB = value_buckets(st->N) + 2 * H * n;
+  const int64_t Lcap = 3 * P;  // pairs + at most 2 entries per pair
+  const int64_t pool_cap = 2 * Lcap / 32 + 2;  // long-group blocks of 32 members
+  const int pwidth = 4 + (int)(dv > dh ? dv : dh);
   struct Piece {
     void **ptr;
     size_t bytes;
@@ -99,23 +112,27 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
       {(void **)&s.pclaim, sizeof(int32_t) * (size_t)P},
       {(void **)&s.pa, sizeof(float) * (size_t)P},
       {(void **)&s.pb, sizeof(float) * (size_t)P},
-      {(void **)&s.pdl, sizeof(float) * (size_t)P},
       {(void **)&s.esub, sizeof(int32_t) * (size_t)(2 * P)},
       {(void **)&s.emask, sizeof(uint32_t) * (size_t)(2 * P)},
       {(void **)&s.einv, sizeof(float) * (size_t)(2 * P)},
       {(void **)&s.eclaim, sizeof(int32_t) * (size_t)(2 * P)},
+      {(void **)&s.ealpha, sizeof(float) * (size_t)(2 * P)},
       {(void **)&s.ecount, sizeof(int32_t) * (size_t)(2 * M)},
-      {(void **)&s.count, sizeof(int32_t) * (size_t)G},
-      {(void **)&s.goff, sizeof(int32_t) * (size_t)G},
-      {(void **)&s.uniq, sizeof(int32_t) * (size_t)(3 * P)},
-      {(void **)&s.useg_off, sizeof(int32_t) * (size_t)(3 * P)},
-      {(void **)&s.useg_len, sizeof(int32_t) * (size_t)(3 * P)},
-      {(void **)&s.sorted, sizeof(int32_t) * (size_t)(3 * P)},
+      {(void **)&s.bcnt, sizeof(int32_t) * (size_t)NB},
+      {(void **)&s.boff, sizeof(int32_t) * (size_t)(NB + 1)},
+      {(void **)&s.rec_in, sizeof(Member) * (size_t)Lcap},
+      {(void **)&s.rec, sizeof(Member) * (size_t)Lcap},
+      {(void **)&s.posmap, sizeof(int32_t) * (size_t)Lcap},
+      {(void **)&s.slotmap, sizeof(int32_t) * (size_t)Lcap},
+      {(void **)&s.sort_tmp, sizeof(uint64_t) * (size_t)(2 * Lcap)},
+      {(void **)&s.partial, sizeof(float) * (size_t)pool_cap * pwidth},
+      {(void **)&s.segcnt, sizeof(int32_t) * (size_t)Lcap},
       {(void **)&s.E, sizeof(float) * (size_t)(rows * dv)},
-      {(void **)&s.tile_cnt, sizeof(int32_t) * (size_t)tiles},
-      {(void **)&s.tile_nz, sizeof(int32_t) * (size_t)tiles},
       {(void **)&s.meta, sizeof(Meta)},
   };
+  s.Lcap = Lcap;
+  s.pwidth = pwidth;
+  s.pool_cap = (int)pool_cap;
   size_t total = 0;
   for (auto &p : pieces) total = align_up(total, 256) + align_up(p.bytes, 256);
   void *arena = nullptr;
@@ -131,8 +148,10 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
     *p.ptr = (char *)arena + off;
     off += align_up(p.bytes, 256);
   }
-  // Group counts start at zero; the meta block (stats) carries over.
-  e = cudaMemset(s.count, 0, sizeof(int32_t) * (size_t)G);
+  // Bucket counts and crossing-group counters start at zero (the kernels
+  // leave them at zero); the meta block (stats) carries over.
+  e = cudaMemset(s.bcnt, 0, sizeof(int32_t) * (size_t)NB);
+  if (e == cudaSuccess) e = cudaMemset(s.segcnt, 0, sizeof(int32_t) * (size_t)Lcap);
   if (e == cudaSuccess) e = cudaMemset(s.meta, 0, sizeof(Meta));
   if (e == cudaSuccess && st->s.meta)
     e = cudaMemcpy(s.meta, st->s.meta, sizeof(Meta), cudaMemcpyDeviceToDevice);
@@ -223,8 +242,9 @@ fwpkm_status fwpkm_state_init(int64_t N, int dq, int dv, int topk, int chunk, in
   st->k = topk;
   st->chunk = chunk;
   st->H = heads;
-  st->G = N + 2ll * heads * n;
   cudaGetDevice(&st->device);
+  cudaDeviceGetAttribute(&st->sm_count, cudaDevAttrMultiProcessorCount, st->device);
+  if (st->sm_count < 1) st->sm_count = 1;
   const size_t kbytes = sizeof(float) * (size_t)heads * 2 * n * st->dh;
   const size_t vbytes = sizeof(float) * (size_t)N * dv;
   cudaError_t e = cudaMalloc(&st->K, kbytes);
@@ -302,8 +322,6 @@ fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtyp
   st->x = Extras{};  // armed extras apply to this step only
 
   const Scratch &s = st->s;
-  cudaError_t e = cudaMemsetAsync(s.count, 0, sizeof(int32_t) * (size_t)st->G, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "step: memset");
   const int n_chunks = (T + st->chunk - 1) / st->chunk;
   for (int c = 0; c < n_chunks; ++c) {
     Dims d{};
@@ -320,26 +338,34 @@ fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtyp
     d.Tc = (T - d.t0 < st->chunk) ? T - d.t0 : st->chunk;
     d.rows = B * d.Tc;
     d.M = d.rows * st->H;
-    d.G = (int)st->G;
+    d.vshift = value_shift(st->N);
+    d.NBv = (int)value_buckets(st->N);
+    d.NB = d.NBv + 2 * st->H * st->n;
+    d.sm_count = st->sm_count;
     d.eps = st->eps;
     d.eta = eta;
     d.lam = lambda_entropy;
-    if ((rc = run(st, K_PREP, stream, [&] { return launch_prep(d, Q, q_dtype, st->K, s, stream); })))
+    float *V = st->V, *K = st->K;
+    if ((rc = run(st, K_PREP, stream, [&] { return launch_prep(d, Q, q_dtype, K, s, stream); })))
       return rc;
-    if ((rc = run(st, K_SCORE, stream, [&] { return launch_score(d, st->K, s, stream); })))
-      return rc;
+    if ((rc = run(st, K_SCORE, stream, [&] { return launch_score(d, K, s, stream); }))) return rc;
     if ((rc = run(st, K_TOPK, stream, [&] { return launch_topk(d, s, x, stream); }))) return rc;
-    if ((rc = run(st, K_SCAN, stream, [&] { return launch_scan(d, s, stream, 0); }))) return rc;
-    if ((rc = run(st, K_SCAN, stream, [&] { return launch_scan(d, s, stream, 1); }))) return rc;
+    if ((rc = run(st, K_SCAN, stream, [&] { return launch_scan(d, s, stream); }))) return rc;
     if ((rc = run(st, K_READ, stream, [&] {
-           return launch_read(d, st->V, Vtarget, v_dtype, gate, out, s, stream);
+           return launch_read(d, V, Vtarget, v_dtype, gate, out, s, stream);
          })))
       return rc;
-    if ((rc = run(st, K_VAPPLY, stream, [&] { return launch_vapply(d, st->V, gate, s, stream); })))
-      return rc;
-    if ((rc = run(st, K_PGRAD, stream, [&] { return launch_pgrad(d, s, stream); }))) return rc;
-    if ((rc = run(st, K_KAPPLY, stream, [&] { return launch_kapply(d, st->K, s, stream); })))
-      return rc;
+    if ((rc = run(st, K_BSORT, stream, [&] { return launch_bsort(d, s, stream); }))) return rc;
+    if (lambda_entropy == 0.f) {
+      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, s, stream, 0); })))
+        return rc;
+    } else {
+      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, s, stream, 1); })))
+        return rc;
+      if ((rc = run(st, K_PGRAD, stream, [&] { return launch_pgrad(d, s, stream); }))) return rc;
+      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, s, stream, 2); })))
+        return rc;
+    }
   }
   return FWPKM_OK;
 }
@@ -479,7 +505,7 @@ fwpkm_status fwpkm_read_stats(fwpkm_state *st, int64_t *chunks, int64_t *value_r
   if (e != cudaSuccess) return cuda_fail(e, "read_stats");
   if (chunks) *chunks = (int64_t)m.stat_chunks;
   if (value_rows) *value_rows = (int64_t)m.stat_value_rows;
-  if (key_rows) *key_rows = (int64_t)(m.stat_total_rows - m.stat_value_rows);
+  if (key_rows) *key_rows = (int64_t)m.stat_key_rows;
   if (device_errors) *device_errors = m.err;
   if (reset) {
     Meta z{};

@@ -3,17 +3,19 @@
 // Per chunk the host enqueues, in order:
 //   prep    -> split the chunk's queries into halves (fp32), |q|^2, |K|^2
 //   score   -> D[h][half][row][i] = |q_half - K_h,half,i|^2 for every sub-key
-//   topk    -> per token-head: top-k per half, k*k merge, softmax; claims of
-//              the (slot) and (sub-key) groups the pair will write
-//   scan    -> group offsets / unique group list over slots and sub-keys
+//   topk    -> per token-head: top-k per half, k*k merge, softmax; each pair
+//              (value row) and each distinct sub-key row it uses (an "entry")
+//              counts itself into a bucket and claims a position there
+//   scan    -> bucket offsets
 //   read    -> gather the selected value rows, out = g * yhat, residual e,
-//              dL/dw per pair; scatter pair / entry ids into group order
-//   vapply  -> per touched value row: ordered segmented sum, V -= eta G / C,
-//              marginal p_bar -> entropy term per pair
-//   pgrad   -> per token-head: dL/ds through the softmax Jacobian
-//   kapply  -> per touched sub-key row: ordered sum, K -= eta dL/dK
-// No floating-point atomics anywhere: every sum runs in a fixed order
-// (pairs sorted by id inside each group), so two runs are bit-identical.
+//              dL/dw per pair; scatter member ids into their buckets
+//   bsort   -> sort every bucket by (group, member id)
+//   apply   -> fixed 32-member tiles of the sorted array: ordered per-group
+//              sums, V -= eta G / C and K -= eta dL/dK on touched rows
+//   (lam > 0: apply(values) -> pgrad (softmax Jacobian) -> apply(sub-keys))
+// No floating-point atomics anywhere: every sum runs in a fixed order (members
+// sorted by id inside each group, tiles combined in tile order), so two runs
+// are bit-identical, whatever the skew of slot usage.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -23,23 +25,21 @@
 namespace fwpkm {
 
 constexpr unsigned FULL = 0xffffffffu;
-constexpr int kScanTile = 2048;      // group-count scan: elements per CTA
-constexpr int kWarpSortMax = 1024;   // largest group sorted in warp-private smem
-
 // Device-side error bits (meta->err).
 enum : unsigned {
   ERR_MBAR_TIMEOUT = 1u,   // a bounded mbarrier wait gave up
+  ERR_POOL_OVERFLOW = 2u,  // more long-group blocks than the partial pool holds
 };
 
-// Written by the scan kernels, read by the apply kernels and the host.
+// Written by the kernels, read by later kernels and by the host.
 struct Meta {
-  int32_t U_v;            // distinct value rows touched in the chunk
-  int32_t U_total;        // distinct value rows + distinct sub-key rows
+  int32_t L;              // members of the chunk (pairs + sub-key entries)
+  int32_t Lv;             // pairs (value-row members come first)
   unsigned err;           // ERR_* bits, sticky until the host clears them
-  int32_t pad;
+  int32_t pool_next;      // next free partial slot (reset per chunk)
   unsigned long long stat_chunks;      // chunks processed since reset
-  unsigned long long stat_value_rows;  // sum over chunks of U_v
-  unsigned long long stat_total_rows;  // sum over chunks of U_total
+  unsigned long long stat_value_rows;  // sum over chunks of distinct value rows written
+  unsigned long long stat_key_rows;    // sum over chunks of distinct sub-key rows written
 };
 
 // Shapes of the chunk being processed.
@@ -49,7 +49,10 @@ struct Dims {
   int B, T, t0, Tc;   // batch, call length, first token of the chunk, its length
   int rows;           // B * Tc
   int M;              // rows * H token-heads
-  int G;              // N + 2*H*n groups (value rows, then sub-key rows)
+  int NBv;            // value buckets: slot >> vshift
+  int vshift;
+  int NB;             // NBv value buckets + 2*H*n sub-key rows
+  int sm_count;       // multiprocessors of the device (grid sizing)
   float eps, eta, lam;
 };
 
@@ -61,25 +64,44 @@ struct Scratch {
   float *D;         // [H][2][rows][n]    squared distances
   int32_t *pslot;   // [M*k] selected slot of pair p = m*k + r
   float *pw;        // [M*k] softmax weight
-  int32_t *pclaim;  // [M*k] position inside the slot's group
+  int32_t *pclaim;  // [M*k] position inside the pair's bucket
   float *pa;        // [M*k] dL_mse/dw
   float *pb;        // [M*k] dL_addr/dw (lam > 0)
-  float *pdl;       // [M*k] dL/ds
   int32_t *esub;    // [2*M*k] sub-key row of entry e = (m*2+half)*k + idx
   uint32_t *emask;  // [2*M*k] pairs r of token-head m that use that row
   float *einv;      // [2*M*k] 1 / (eps + d_half(row))
-  int32_t *eclaim;  // [2*M*k] position inside the sub-key row's group
+  int32_t *eclaim;  // [2*M*k] position inside the entry's bucket
+  float *ealpha;    // [2*M*k] sum of dL/ds over the entry's pairs / (eps + d)
   int32_t *ecount;  // [M*2]   entries per (m, half)
-  int32_t *count;   // [G] members per group (zero between chunks)
-  int32_t *goff;    // [G] first position of the group in `sorted`
-  int32_t *uniq;    // [M*k*3] touched groups in group order
-  int32_t *useg_off;
-  int32_t *useg_len;
-  int32_t *sorted;  // [M*k*3] pair ids (value groups) then entry ids (sub-key groups)
+  int32_t *bcnt;    // [NB]    members per bucket (zero between chunks)
+  int32_t *boff;    // [NB+1]  bucket offsets into rec_in / rec
+  struct Member *rec_in;  // [Lcap] member records in bucket (claim) order
+  struct Member *rec;     // [Lcap] the same records sorted by (group, id)
+  uint64_t *sort_tmp;  // [2*Lcap] merge buffers for oversized buckets
+  int32_t *posmap;  // [Lcap]  position inside its bucket, by member id (oversized buckets)
+  int32_t *slotmap; // [Lcap]  partial-pool slot of the block starting here
+  float *partial;   // [pool_cap][pwidth] block partial sums of long groups
+  int32_t *segcnt;  // [Lcap] arrived blocks per long group, at its first position
+                    // (zero between chunks)
   float *E;         // [rows][dv] residual yhat - v
-  int32_t *tile_cnt;  // [ceil(G / kScanTile)]
-  int32_t *tile_nz;
   Meta *meta;
+  int64_t Lcap;     // member capacity (3 * M*k)
+  int pwidth;       // 4 + max(dv, dh) floats
+  int pool_cap;     // partial slots: 2 * Lcap / 32
+};
+
+// One member of a group (32 bytes).  Value rows: a pair p; sub-key rows: an
+// entry e.  Written by the read kernel into the member's bucket, sorted by
+// (g, id) and completed (gstart, glen) by the bucket sort.
+struct __align__(16) Member {
+  uint32_t g;      // group: slot (< N) or N + (h*2+half)*n + row
+  uint32_t id;     // pair id p = m*k + r, or entry id e = (m*2+half)*k + idx
+  int32_t srow;    // source row: E row (value rows) or Qs row (sub-key rows)
+  int32_t gstart;  // position of the group's first member
+  float coef;      // value rows: 2 g_t w / H; sub-key rows: alpha (lam == 0)
+  float c0;        // value rows: w / H;       sub-key rows: alpha
+  float c1;        // value rows: w
+  int32_t glen;    // members in the group
 };
 
 // Optional per-step inputs/outputs.
@@ -177,12 +199,13 @@ cudaError_t launch_prep(const Dims &d, const void *Q, int q_dtype, const float *
                         const Scratch &s, cudaStream_t st);
 cudaError_t launch_score(const Dims &d, const float *K, const Scratch &s, cudaStream_t st);
 cudaError_t launch_topk(const Dims &d, const Scratch &s, const Extras &x, cudaStream_t st);
-cudaError_t launch_scan(const Dims &d, const Scratch &s, cudaStream_t st, int part);
+cudaError_t launch_scan(const Dims &d, const Scratch &s, cudaStream_t st);
 cudaError_t launch_read(const Dims &d, const float *V, const void *Vt, int v_dtype,
                         const float *gate, float *out, const Scratch &s, cudaStream_t st);
-cudaError_t launch_vapply(const Dims &d, float *V, const float *gate, const Scratch &s,
-                          cudaStream_t st);
+cudaError_t launch_bsort(const Dims &d, const Scratch &s, cudaStream_t st);
+// part 0: all groups; 1: value rows only; 2: sub-key rows only
+cudaError_t launch_apply(const Dims &d, float *V, float *K, const Scratch &s, cudaStream_t st,
+                         int part);
 cudaError_t launch_pgrad(const Dims &d, const Scratch &s, cudaStream_t st);
-cudaError_t launch_kapply(const Dims &d, float *K, const Scratch &s, cudaStream_t st);
 
 }  // namespace fwpkm

@@ -8,304 +8,619 @@
 //   value row i : V_i -= eta * G_i / C_i,
 //                 G_i = sum over its pairs of (2 g_t / H) w e_t,
 //                 C_i = sum over its pairs of w / H
-//   sub-key row : K -= eta * sum over its pairs of dL/ds * 2 (q - K)/(eps + d)
+//   sub-key row : K -= eta * 2 * (sum_e alpha_e q_e - (sum_e alpha_e) K)
+//                 alpha_e = (1/(eps + d)) * sum of dL/ds over the entry's pairs
 //   marginal    : pbar_i = (1/M) sum over its pairs of w;
 //                 dL_addr/dw = (lam/M) (log pbar_i + 1)
 //
-// Groups are value rows [0, N) and sub-key rows N + (h*2+half)*n + i.  The
-// selection kernel counted members per group and claimed a position; the scan
-// below turns counts into offsets and a list of touched groups; the read
-// kernel scatters member ids to offset + claim.  Claim order depends on atomic
-// timing, so every group sorts its member ids before summing: the sums run in
-// id order and the result is independent of scheduling.
+// Members: pairs p = m*k + r (value rows) and entries e = (m*2+half)*k + idx
+// (sub-key rows), each carried by a 32-byte Member record.  Buckets: value
+// bucket slot >> vshift (a range of at most 2^vshift consecutive slots, <= 8192
+// buckets), then one bucket per sub-key row, NBv + (h*2+half)*n + row.  The
+// selection kernel counted members per bucket and claimed a position; `scan`
+// turns counts into bucket offsets; the read kernel writes each record at
+// offset + claim (rec_in); `bsort` sorts every bucket by (group, id) into rec,
+// so the records are globally ordered by group and, inside a group, by id;
+// `apply` sums every group's members in that order and writes the row.  No
+// floating-point atomics: the result does not depend on scheduling, whatever
+// the skew of slot usage.
 #include <math_constants.h>
 
 #include "fwpkm_internal.cuh"
 
 namespace fwpkm {
 
-// ---------------------------------------------------------------------------
-// Scan over the group counts.
-// ---------------------------------------------------------------------------
-constexpr int kScanThreads = 256;
-constexpr int kScanPer = kScanTile / kScanThreads;  // 8 consecutive groups per thread
-
-__device__ __forceinline__ int block_sum_int(int v, int *red) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-  __syncthreads();
-  if (lane == 0) red[w] = v;
-  __syncthreads();
-  int t = 0;
-  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
-  return t;
+__device__ __forceinline__ Member load_member(const Member *p) {
+  const int4 a = *reinterpret_cast<const int4 *>(p);
+  const int4 b = *(reinterpret_cast<const int4 *>(p) + 1);
+  Member m;
+  m.g = (uint32_t)a.x;
+  m.id = (uint32_t)a.y;
+  m.srow = a.z;
+  m.gstart = a.w;
+  m.coef = __int_as_float(b.x);
+  m.c0 = __int_as_float(b.y);
+  m.c1 = __int_as_float(b.z);
+  m.glen = b.w;
+  return m;
+}
+__device__ __forceinline__ void store_member(Member *p, const Member &m) {
+  *reinterpret_cast<int4 *>(p) = make_int4((int)m.g, (int)m.id, m.srow, m.gstart);
+  *(reinterpret_cast<int4 *>(p) + 1) =
+      make_int4(__float_as_int(m.coef), __float_as_int(m.c0), __float_as_int(m.c1), m.glen);
 }
 
-// Exclusive prefix over the block (thread order); returns the block total.
-__device__ __forceinline__ int block_excl_scan(int v, int *red, int &total) {
+// ---------------------------------------------------------------------------
+// scan: bucket offsets (single CTA).  Each thread owns a contiguous run of
+// buckets; its counts are loaded before the block-wide scan.
+// ---------------------------------------------------------------------------
+constexpr int kScanThreads = 1024;
+constexpr int kScanRun = 16;  // counts held in registers per thread and pass
+
+__global__ void __launch_bounds__(kScanThreads) k_bucket_scan(Dims d, Scratch s) {
+  __shared__ int red[32];
+  const int NB = d.NB;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int incl = v;
+  const int per = (NB + kScanThreads - 1) / kScanThreads;  // buckets per thread
+  const int b0 = min(threadIdx.x * per, NB), b1 = min(b0 + per, NB);
+  int total = 0;
+  for (int b = b0; b < b1; b += kScanRun) {
+    int v[kScanRun];
+#pragma unroll
+    for (int i = 0; i < kScanRun; ++i) v[i] = b + i < b1 ? s.bcnt[b + i] : 0;
+#pragma unroll
+    for (int i = 0; i < kScanRun; ++i) total += v[i];
+  }
+  // exclusive scan of the per-thread totals
+  int incl = total;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    int t = __shfl_up_sync(FULL, incl, o);
+    const int t = __shfl_up_sync(FULL, incl, o);
     if (lane >= o) incl += t;
   }
-  __syncthreads();
   if (lane == 31) red[w] = incl;
   __syncthreads();
-  int before = 0, tot = 0;
-  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
-    if (i < w) before += red[i];
-    tot += red[i];
-  }
-  total = tot;
-  return before + incl - v;
-}
-
-__global__ void __launch_bounds__(kScanThreads) k_scan_tiles(Dims d, Scratch s) {
-  __shared__ int red[kScanThreads / 32];
-  const int64_t g0 = (int64_t)blockIdx.x * kScanTile + (int64_t)threadIdx.x * kScanPer;
-  int c = 0, nz = 0;
+  if (w == 0) {
+    int x = red[lane];
 #pragma unroll
-  for (int i = 0; i < kScanPer; ++i) {
-    const int64_t g = g0 + i;
-    const int v = g < d.G ? s.count[g] : 0;
-    c += v;
-    nz += v > 0;
-  }
-  c = block_sum_int(c, red);
-  nz = block_sum_int(nz, red);
-  if (threadIdx.x == 0) {
-    s.tile_cnt[blockIdx.x] = c;
-    s.tile_nz[blockIdx.x] = nz;
-  }
-}
-
-__global__ void __launch_bounds__(kScanThreads) k_scan_write(Dims d, Scratch s) {
-  __shared__ int red[kScanThreads / 32];
-  const int tile = blockIdx.x;
-  // Offsets of this tile: sums over the previous tiles.
-  int bc = 0, bn = 0;
-  for (int t = threadIdx.x; t < tile; t += blockDim.x) {
-    bc += s.tile_cnt[t];
-    bn += s.tile_nz[t];
-  }
-  bc = block_sum_int(bc, red);
-  bn = block_sum_int(bn, red);
-  const int64_t g0 = (int64_t)tile * kScanTile + (int64_t)threadIdx.x * kScanPer;
-  int cv[kScanPer];
-  int c = 0, nz = 0;
-#pragma unroll
-  for (int i = 0; i < kScanPer; ++i) {
-    const int64_t g = g0 + i;
-    cv[i] = g < d.G ? s.count[g] : 0;
-    c += cv[i];
-    nz += cv[i] > 0;
-  }
-  int tot_c, tot_nz;
-  int ec = block_excl_scan(c, red, tot_c);
-  int en = block_excl_scan(nz, red, tot_nz);
-#pragma unroll
-  for (int i = 0; i < kScanPer; ++i) {
-    const int64_t g = g0 + i;
-    if (g >= d.G) break;
-    if (g == d.N) {  // first sub-key group: everything before it is a value row
-      s.meta->U_v = bn + en;
-      atomicAdd(&s.meta->stat_value_rows, (unsigned long long)(bn + en));
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(FULL, x, o);
+      if (lane >= o) x += t;
     }
-    if (cv[i] > 0) {
-      const int off = bc + ec;
-      const int u = bn + en;
-      s.goff[g] = off;
-      s.uniq[u] = (int)g;
-      s.useg_off[u] = off;
-      s.useg_len[u] = cv[i];
-      s.count[g] = 0;  // ready for the next chunk
-      ec += cv[i];
-      en += 1;
+    red[lane] = x;
+  }
+  __syncthreads();
+  int run = (w > 0 ? red[w - 1] : 0) + incl - total;
+  for (int b = b0; b < b1; b += kScanRun) {
+    int v[kScanRun];
+#pragma unroll
+    for (int i = 0; i < kScanRun; ++i) v[i] = b + i < b1 ? s.bcnt[b + i] : 0;
+#pragma unroll
+    for (int i = 0; i < kScanRun; ++i) {
+      if (b + i < b1) {
+        s.boff[b + i] = run;
+        if (b + i == d.NBv) s.meta->Lv = run;  // value buckets come first
+        s.bcnt[b + i] = 0;                       // ready for the next chunk
+        run += v[i];
+      }
     }
   }
-  if (tile == (int)gridDim.x - 1 && threadIdx.x == 0) {
-    s.meta->U_total = bn + tot_nz;
-    atomicAdd(&s.meta->stat_total_rows, (unsigned long long)(bn + tot_nz));
-    atomicAdd(&s.meta->stat_chunks, 1ull);
+  if (threadIdx.x == kScanThreads - 1) {
+    const int L = red[31];
+    s.boff[NB] = L;
+    s.meta->L = L;
+    if (d.NBv == NB) s.meta->Lv = L;
+    s.meta->stat_chunks += 1ull;
+    s.meta->pool_next = 0;
   }
 }
 
-cudaError_t launch_scan(const Dims &d, const Scratch &s, cudaStream_t st, int part) {
-  const int tiles = (int)((d.G + kScanTile - 1) / kScanTile);
-  if (part == 0)
-    k_scan_tiles<<<tiles, kScanThreads, 0, st>>>(d, s);
-  else
-    k_scan_write<<<tiles, kScanThreads, 0, st>>>(d, s);
+cudaError_t launch_scan(const Dims &d, const Scratch &s, cudaStream_t st) {
+  k_bucket_scan<<<1, kScanThreads, 0, st>>>(d, s);
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// Ordered member iteration of one group (warp-cooperative).
-//   len <= 32            : ids sorted across the lanes (bitonic)
-//   len <= kWarpSortMax  : ids sorted in warp-private shared memory
-//   otherwise            : `scan(id)` enumerates every candidate id in order
-// `body(id)` is called by the whole warp, in increasing id order.
+// bsort: sort each bucket's records (rec_in, claim order) by (group, id) into
+// rec, and stamp every record with its group's first position and length.
+// Buckets are dealt round-robin to warps.  A bucket of <= 32 members is sorted
+// by its warp in registers; larger ones afterwards by the whole CTA in shared
+// memory (bitonic over packed keys that carry the record's local index), or,
+// beyond kSortCap members, in runs merged through global memory.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ int lane_sort32(int v) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      const int o = __shfl_xor_sync(FULL, v, stride);
-      const bool up = (lane & size) == 0 || size == 32;
-      const bool lower = (lane & stride) == 0;
-      const bool keep = (lower == up) ? (v <= o) : (v >= o);
-      if (!keep) v = o;
-    }
-  }
-  return v;
+constexpr int kSortThreads = 512;
+constexpr int kSortWarps = kSortThreads / 32;
+constexpr int kSortCap = 4096;  // largest bucket sorted in shared memory (12-bit index)
+
+__device__ __forceinline__ uint64_t shfl_xor64(uint64_t v, int o) {
+  const uint32_t lo = __shfl_xor_sync(FULL, (uint32_t)v, o);
+  const uint32_t hi = __shfl_xor_sync(FULL, (uint32_t)(v >> 32), o);
+  return ((uint64_t)hi << 32) | lo;
 }
 
-// Sort buf[0..len) ascending in place (warp-private smem, len <= kWarpSortMax).
-__device__ void warp_smem_sort(int *buf, int len) {
-  const int lane = threadIdx.x & 31;
-  int n2 = 64;
-  while (n2 < len) n2 <<= 1;
-  for (int i = len + lane; i < n2; i += 32) buf[i] = 0x7fffffff;
-  __syncwarp();
+// In-place ascending bitonic sort of buf[0..n2), n2 a power of two, CTA-wide.
+__device__ void block_bitonic(uint64_t *buf, int n2) {
   for (int size = 2; size <= n2; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = lane; i < n2; i += 32) {
-        const int l = i ^ stride;
-        if (l > i) {
-          const int a = buf[i], b = buf[l];
-          const bool up = (i & size) == 0;
-          if ((a > b) == up) {
-            buf[i] = b;
-            buf[l] = a;
+      for (int i = threadIdx.x; i < (n2 >> 1); i += blockDim.x) {
+        const int lo = 2 * i - (i & (stride - 1));  // index with the stride bit clear
+        const int hi = lo + stride;
+        const uint64_t a = buf[lo], b = buf[hi];
+        const bool up = (lo & size) == 0;
+        if ((a > b) == up) {
+          buf[lo] = b;
+          buf[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Count of elements < key in the sorted run [r, r+len).
+__device__ __forceinline__ int lower_rank(const uint64_t *r, int len, uint64_t key) {
+  int lo = 0, hi = len;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (r[mid] < key) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// CTA-wide sort of one bucket with more than 32 members.
+__device__ void sort_big_bucket(const Scratch &s, int off, int len, bool value, uint32_t gbase,
+                                uint64_t *buf, int *nseg) {
+  int my_seg = 0;
+  if (len <= kSortCap) {
+    // key = (g - gbase) << 43 | id << 12 | local index   (g - gbase < 2^21, id < 2^31)
+    int n2 = 64;
+    while (n2 < len) n2 <<= 1;
+    for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+      if (i < len) {
+        const int4 a = *reinterpret_cast<const int4 *>(s.rec_in + off + i);
+        buf[i] = ((uint64_t)((uint32_t)a.x - gbase) << 43) | ((uint64_t)(uint32_t)a.y << 12) |
+                 (uint64_t)i;
+      } else {
+        buf[i] = ~0ull;
+      }
+    }
+    __syncthreads();
+    block_bitonic(buf, n2);
+    for (int i = threadIdx.x; i < len; i += blockDim.x) {
+      const uint64_t kv = buf[i];
+      const uint64_t grp = kv >> 43;
+      const int first = lower_rank(buf, len, grp << 43);
+      const int end = (grp + 1) >= (1ull << 21) ? len : lower_rank(buf, len, (grp + 1) << 43);
+      Member m = load_member(s.rec_in + off + (int)(kv & 4095u));
+      m.gstart = off + first;
+      m.glen = end - first;
+      store_member(s.rec + off + i, m);
+      my_seg += first == i ? 1 : 0;
+    }
+  } else {
+    // Oversized bucket: keys (g << 32 | id) sorted in runs of kSortCap in
+    // shared memory, runs merged pairwise through global memory; each record
+    // found again through its position, stored by id in posmap.
+    const int pbase = value ? 0 : (int)(s.Lcap / 3);  // pair ids and entry ids apart
+    uint64_t *A = s.sort_tmp + off;
+    uint64_t *Bb = s.sort_tmp + (size_t)s.Lcap + off;
+    for (int i = threadIdx.x; i < len; i += blockDim.x)
+      s.posmap[pbase + (int)s.rec_in[off + i].id] = i;
+    for (int r0 = 0; r0 < len; r0 += kSortCap) {
+      const int rl = min(kSortCap, len - r0);
+      int n2 = 64;
+      while (n2 < rl) n2 <<= 1;
+      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+        if (i < rl) {
+          const int4 a = *reinterpret_cast<const int4 *>(s.rec_in + off + r0 + i);
+          buf[i] = ((uint64_t)(uint32_t)a.x << 32) | (uint32_t)a.y;
+        } else {
+          buf[i] = ~0ull;
+        }
+      }
+      __syncthreads();
+      block_bitonic(buf, n2);
+      for (int i = threadIdx.x; i < rl; i += blockDim.x) A[r0 + i] = buf[i];
+      __syncthreads();
+    }
+    uint64_t *src = A, *dst = Bb;
+    for (int width = kSortCap; width < len; width <<= 1) {
+      for (int i = threadIdx.x; i < len; i += blockDim.x) {
+        const int a0 = (i / (2 * width)) * 2 * width;
+        const int alen = min(width, len - a0);
+        const int b0 = a0 + alen;
+        const int blen = max(0, min(width, len - b0));
+        const uint64_t key = src[i];
+        const int pos = i < b0 ? (i - a0) + lower_rank(src + b0, blen, key)
+                               : (i - b0) + lower_rank(src + a0, alen, key);
+        dst[a0 + pos] = key;
+      }
+      __syncthreads();
+      uint64_t *t = src;
+      src = dst;
+      dst = t;
+    }
+    for (int i = threadIdx.x; i < len; i += blockDim.x) {
+      const uint64_t kv = src[i];
+      const uint64_t grp = kv >> 32;
+      const int first = lower_rank(src, len, grp << 32);
+      const int end = lower_rank(src, len, (grp + 1) << 32);
+      Member m = load_member(s.rec_in + off + s.posmap[pbase + (int)(uint32_t)kv]);
+      m.gstart = off + first;
+      m.glen = end - first;
+      store_member(s.rec + off + i, m);
+      my_seg += first == i ? 1 : 0;
+    }
+  }
+  if (my_seg) atomicAdd(nseg, my_seg);
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s) {
+  __shared__ uint64_t buf[kSortCap];
+  __shared__ int nseg[2];  // distinct value rows / sub-key rows seen by this CTA
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  if (threadIdx.x < 2) nseg[threadIdx.x] = 0;
+  __syncthreads();
+  const int stride = gridDim.x * kSortWarps;
+  // phase 1: small buckets, one warp each
+  for (int b = blockIdx.x * kSortWarps + wib; b < d.NB; b += stride) {
+    const int off = s.boff[b], len = s.boff[b + 1] - off;
+    if (len == 0 || len > 32) continue;
+    Member m{};
+    uint64_t key = ~0ull;
+    if (lane < len) {
+      m = load_member(s.rec_in + off + lane);
+      key = ((uint64_t)m.g << 32) | m.id;
+    }
+    // bitonic sort of (key, source lane) across the warp
+    int src = lane;
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+      for (int st = size >> 1; st > 0; st >>= 1) {
+        const uint64_t ok = shfl_xor64(key, st);
+        const int os = __shfl_xor_sync(FULL, src, st);
+        const bool up = (lane & size) == 0 || size == 32;
+        const bool lower = (lane & st) == 0;
+        const bool keep = (lower == up) ? (key <= ok) : (key >= ok);
+        if (!keep) {
+          key = ok;
+          src = os;
+        }
+      }
+    }
+    // the record of rank `lane` comes from lane `src`
+    Member r;
+    r.g = __shfl_sync(FULL, m.g, src);
+    r.id = __shfl_sync(FULL, m.id, src);
+    r.srow = __shfl_sync(FULL, m.srow, src);
+    r.coef = __shfl_sync(FULL, m.coef, src);
+    r.c0 = __shfl_sync(FULL, m.c0, src);
+    r.c1 = __shfl_sync(FULL, m.c1, src);
+    const uint32_t prev_g = __shfl_up_sync(FULL, r.g, 1);
+    const bool head = lane < len && (lane == 0 || prev_g != r.g);
+    const unsigned heads = __ballot_sync(FULL, head);
+    if (lane < len) {
+      const unsigned upto = heads & ((2u << lane) - 1u);  // heads at or below this lane
+      const int h0 = 31 - __clz(upto);
+      const unsigned after = heads & ~((2u << h0) - 1u);  // heads after the group's first
+      r.gstart = off + h0;
+      r.glen = (after ? __ffs(after) - 1 : len) - h0;
+      store_member(s.rec + off + lane, r);
+    }
+    if (lane == 0) atomicAdd(&nseg[b < d.NBv ? 0 : 1], __popc(heads));
+  }
+  __syncthreads();
+  // phase 2: large buckets of this CTA's warps, by the whole CTA
+  for (int base = blockIdx.x * kSortWarps; base < d.NB; base += stride) {
+    for (int w = 0; w < kSortWarps && base + w < d.NB; ++w) {
+      const int b = base + w;
+      const int off = s.boff[b], len = s.boff[b + 1] - off;
+      if (len <= 32) continue;
+      const bool value = b < d.NBv;
+      const uint32_t gbase =
+          value ? ((uint32_t)b << d.vshift) : (uint32_t)d.N + (uint32_t)(b - d.NBv);
+      sort_big_bucket(s, off, len, value, gbase, buf, &nseg[value ? 0 : 1]);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (nseg[0]) atomicAdd(&s.meta->stat_value_rows, (unsigned long long)nseg[0]);
+    if (nseg[1]) atomicAdd(&s.meta->stat_key_rows, (unsigned long long)nseg[1]);
+  }
+}
+
+cudaError_t launch_bsort(const Dims &d, const Scratch &s, cudaStream_t st) {
+  static int per_sm = 0;
+  if (!per_sm) {
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_bucket_sort, kSortThreads, 0);
+    if (per_sm < 1) per_sm = 1;
+  }
+  int blocks = (d.NB + kSortWarps - 1) / kSortWarps;
+  if (blocks > d.sm_count * per_sm) blocks = d.sm_count * per_sm;
+  k_bucket_sort<<<blocks, kSortThreads, 0, st>>>(d, s);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// apply: every group is cut into blocks of kBlock members counted from the
+// group's first member; the warp that meets a block's first position sums the
+// block in order, loading a few source rows at a time (E rows for value rows,
+// query halves for sub-key rows) together with the target row.  A group of
+// one block is written at once.  A longer group publishes one partial per
+// block in a pool; the last block to arrive adds the partials in block order
+// and writes the row.  Work per warp is bounded by kBlock members whatever the
+// skew, and no sum depends on scheduling.
+// ---------------------------------------------------------------------------
+constexpr int kApplyWarps = 8;
+constexpr int kBlock = 32;
+
+// Columns are processed in blocks of 32 * Q4 float4 (<= 512 floats), so the
+// registers a warp holds stay bounded for any row width.
+template <int Q4>
+__device__ __forceinline__ void load_row(const float *src, int cb, int n4, float4 (&r)[Q4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int q = 0; q < Q4; ++q) {
+    const int c4 = cb + lane + 32 * q;
+    r[q] = c4 < n4 ? *reinterpret_cast<const float4 *>(src + 4 * c4)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+template <int Q4>
+__device__ __forceinline__ void fma_row(float4 (&acc)[Q4], float c, const float4 (&r)[Q4]) {
+#pragma unroll
+  for (int q = 0; q < Q4; ++q) {
+    acc[q].x = fmaf(c, r[q].x, acc[q].x);
+    acc[q].y = fmaf(c, r[q].y, acc[q].y);
+    acc[q].z = fmaf(c, r[q].z, acc[q].z);
+    acc[q].w = fmaf(c, r[q].w, acc[q].w);
+  }
+}
+
+// Row update (column block at cb) from a group's complete sum.
+template <int Q4>
+__device__ __forceinline__ void update_row(const Dims &d, bool value, float *dst, int cb,
+                                           int n4, const float4 (&row)[Q4],
+                                           const float4 (&acc)[Q4], float c0) {
+  const int lane = threadIdx.x & 31;
+  if (value) {
+    if (!(c0 > 0.f)) return;
+    const float scale = d.eta / c0;
+#pragma unroll
+    for (int q = 0; q < Q4; ++q) {
+      const int c4 = cb + lane + 32 * q;
+      if (c4 < n4) {
+        float4 v = row[q];
+        v.x -= scale * acc[q].x;
+        v.y -= scale * acc[q].y;
+        v.z -= scale * acc[q].z;
+        v.w -= scale * acc[q].w;
+        *reinterpret_cast<float4 *>(dst + 4 * c4) = v;
+      }
+    }
+  } else {
+    const float two_eta = 2.f * d.eta;
+#pragma unroll
+    for (int q = 0; q < Q4; ++q) {
+      const int c4 = cb + lane + 32 * q;
+      if (c4 < n4) {
+        float4 kv = row[q];
+        kv.x -= two_eta * (acc[q].x - c0 * kv.x);
+        kv.y -= two_eta * (acc[q].y - c0 * kv.y);
+        kv.z -= two_eta * (acc[q].z - c0 * kv.z);
+        kv.w -= two_eta * (acc[q].w - c0 * kv.w);
+        *reinterpret_cast<float4 *>(dst + 4 * c4) = kv;
+      }
+    }
+  }
+}
+
+// Entropy term of a value row: dL_addr/dw = (lam/M)(log pbar + 1) for every
+// pair of the group, pbar = (sum of the group's weights) / M.
+__device__ __forceinline__ void write_entropy_term(const Dims &d, const Scratch &s, float wsum,
+                                                   int g0, int len) {
+  const float pbar = wsum / (float)d.M;
+  const float bterm = (d.lam / (float)d.M) * (logf(pbar) + 1.f);
+  for (int x = g0 + (threadIdx.x & 31); x < g0 + len; x += 32) s.pb[s.rec[x].id] = bterm;
+}
+
+// Ordered sum over the block's members (member j's metadata in lane j),
+// column block cb, a few source rows in flight at a time.
+template <int Q4>
+__device__ __forceinline__ void sum_block(const Dims &d, const Scratch &s, bool value, int cnt,
+                                          int srow_l, float coef_l, int cb, int n4,
+                                          float4 (&acc)[Q4]) {
+  constexpr int kBatch = Q4 >= 4 ? 2 : 4;
+  const float *base = value ? s.E : s.Qs;
+  const int width = value ? d.dv : d.dh;
+#pragma unroll
+  for (int q = 0; q < Q4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < cnt; j += kBatch) {
+    float4 r[kBatch][Q4];
+    float cf[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int sr = __shfl_sync(FULL, srow_l, (j + u) & 31);
+      cf[u] = __shfl_sync(FULL, coef_l, (j + u) & 31);
+      if (j + u < cnt) load_row<Q4>(base + (int64_t)sr * width, cb, n4, r[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+      if (j + u < cnt) fma_row<Q4>(acc, cf[u], r[u]);
+  }
+}
+
+// Last block of a long group: add the block partials in block order and
+// write the row (kept out of line so the common path keeps its registers).
+template <int Q4>
+__device__ __noinline__ void combine_partials(const Dims &d, const Scratch &s, bool value,
+                                              float *dst, int n4, int g0, int len,
+                                              int nblocks) {
+  constexpr int CB = 32 * Q4;
+  const int lane = threadIdx.x & 31;
+  float4 acc[Q4], row[Q4];
+  float C = 0.f, W = 0.f;
+  for (int b = 0; b < nblocks; ++b) {
+    const float *pp = s.partial + (size_t)__ldcg(&s.slotmap[g0 + b * kBlock]) * s.pwidth;
+    C += __ldcg(pp);
+    W += __ldcg(pp + 1);
+  }
+  for (int cb = 0; cb < n4; cb += CB) {
+    load_row<Q4>(dst, cb, n4, row);
+#pragma unroll
+    for (int q = 0; q < Q4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int b = 0; b < nblocks; b += 2) {
+      float4 pv[2][Q4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (b + u < nblocks) {
+          const float *pp =
+              s.partial + (size_t)__ldcg(&s.slotmap[g0 + (b + u) * kBlock]) * s.pwidth;
+#pragma unroll
+          for (int q = 0; q < Q4; ++q) {
+            const int c4 = cb + lane + 32 * q;
+            pv[u][q] = c4 < n4 ? __ldcg(reinterpret_cast<const float4 *>(pp + 4 + 4 * c4))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
           }
         }
       }
-      __syncwarp();
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (b + u < nblocks) {
+#pragma unroll
+          for (int q = 0; q < Q4; ++q) {
+            acc[q].x += pv[u][q].x;
+            acc[q].y += pv[u][q].y;
+            acc[q].z += pv[u][q].z;
+            acc[q].w += pv[u][q].w;
+          }
+        }
+      }
     }
+    update_row<Q4>(d, value, dst, cb, n4, row, acc, C);
   }
+  if (value && d.lam != 0.f) write_entropy_term(d, s, W, g0, len);
 }
 
-template <typename Body, typename Match>
-__device__ __forceinline__ void for_members_ordered(const int *ids, int len, int *wbuf,
-                                                    int64_t scan_n, Match match, Body body) {
+template <int Q4>
+__global__ void __launch_bounds__(kApplyWarps * 32) k_apply(Dims d, float *__restrict__ V,
+                                                            float *__restrict__ K, Scratch s,
+                                                            int part) {
+  constexpr int CB = 32 * Q4;  // float4 columns per block
   const int lane = threadIdx.x & 31;
-  if (len <= 32) {
-    int v = lane < len ? ids[lane] : 0x7fffffff;
-    v = lane_sort32(v);
-    for (int r = 0; r < len; ++r) body(__shfl_sync(FULL, v, r));
-  } else if (len <= kWarpSortMax) {
-    for (int i = lane; i < len; i += 32) wbuf[i] = ids[i];
-    __syncwarp();
-    warp_smem_sort(wbuf, len);
-    for (int r = 0; r < len; ++r) body(wbuf[r]);
-    __syncwarp();
-  } else {
-    for (int64_t base = 0; base < scan_n; base += 32) {
-      const int64_t id = base + lane;
-      unsigned hit = __ballot_sync(FULL, id < scan_n && match((int)id));
-      while (hit) {
-        const int l = __ffs(hit) - 1;
-        hit &= hit - 1;
-        body((int)(base + l));
+  const int L = s.meta->L, Lv = s.meta->Lv;
+  const int lo = part == 2 ? Lv : 0;  // part 0: all, 1: value rows, 2: sub-key rows
+  const int hi = part == 1 ? Lv : L;
+  const bool alpha_later = d.lam != 0.f;  // sub-key alphas come from pgrad
+  for (int x = lo + blockIdx.x * kApplyWarps + (threadIdx.x >> 5); x < hi;
+       x += gridDim.x * kApplyWarps) {
+    const int4 head = *reinterpret_cast<const int4 *>(s.rec + x);  // g, id, srow, gstart
+    const int g0 = head.w;
+    if ((x - g0) % kBlock != 0) continue;  // not the first member of a block
+    const int len = s.rec[x].glen;
+    const int cnt = min(kBlock, g0 + len - x);
+    const uint32_t g = (uint32_t)head.x;
+    const bool value = g < (uint32_t)d.N;
+    const int n4 = (value ? d.dv : d.dh) >> 2;
+    float *dst = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.N) * d.dh;
+    // lane j: metadata of member x + j
+    int srow_l = 0;
+    float coef_l = 0.f, c0_l = 0.f, c1_l = 0.f;
+    if (lane < cnt) {
+      const Member m = load_member(s.rec + x + lane);
+      srow_l = m.srow;
+      coef_l = m.coef;
+      c0_l = m.c0;
+      c1_l = m.c1;
+      if (!value && alpha_later) {
+        coef_l = s.ealpha[m.id];
+        c0_l = coef_l;
       }
     }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// vapply: per touched value row.
-// ---------------------------------------------------------------------------
-constexpr int kApplyWarps = 8;
-
-template <int Q4>  // float4 columns per lane: dv <= 128 * Q4
-__global__ void __launch_bounds__(kApplyWarps * 32) k_vapply(Dims d, float *__restrict__ V,
-                                                             const float *__restrict__ gate,
-                                                             Scratch s) {
-  __shared__ int wbuf_all[kApplyWarps][kWarpSortMax];
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  int *wbuf = wbuf_all[wib];
-  const int U_v = s.meta->U_v;
-  const int HK = d.H * d.k;
-  const int dv4 = d.dv >> 2;
-  const float invH = 1.f / (float)d.H;
-  const int64_t P = (int64_t)d.M * d.k;
-  for (int u = blockIdx.x * kApplyWarps + wib; u < U_v; u += gridDim.x * kApplyWarps) {
-    const int slot = s.uniq[u];
-    const int off = s.useg_off[u], len = s.useg_len[u];
-    float4 G[Q4];
-#pragma unroll
-    for (int q = 0; q < Q4; ++q) G[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    float C = 0.f, wsum = 0.f;
-    auto body = [&](int p) {
-      const int row = p / HK;
-      const int b = row / d.Tc, tl = row % d.Tc;
-      const float g = gate[(int64_t)b * d.T + d.t0 + tl];
-      const float w = s.pw[p];
-      const float coef = 2.f * g * invH * w;
-      const float *e = s.E + (int64_t)row * d.dv;
-#pragma unroll
-      for (int q = 0; q < Q4; ++q) {
-        const int c4 = lane + 32 * q;
-        if (c4 < dv4) {
-          const float4 ev = *reinterpret_cast<const float4 *>(e + 4 * c4);
-          G[q].x = fmaf(coef, ev.x, G[q].x);
-          G[q].y = fmaf(coef, ev.y, G[q].y);
-          G[q].z = fmaf(coef, ev.z, G[q].z);
-          G[q].w = fmaf(coef, ev.w, G[q].w);
-        }
+    // ordered scalar sums over the block
+    float c0 = 0.f, c1 = 0.f;
+    for (int j = 0; j < cnt; ++j) {
+      c0 += __shfl_sync(FULL, c0_l, j);
+      c1 += __shfl_sync(FULL, c1_l, j);
+    }
+    const bool whole = len <= kBlock;  // the whole group is in this block
+    float *p = nullptr;
+    if (!whole) {  // long group: this block's partial goes to a pool slot
+      int slot = 0;
+      if (lane == 0) slot = atomicAdd(&s.meta->pool_next, 1);
+      slot = __shfl_sync(FULL, slot, 0);
+      if (slot >= s.pool_cap) {  // cannot happen: the pool holds 2*Lcap/kBlock blocks
+        if (lane == 0) atomicOr(&s.meta->err, ERR_POOL_OVERFLOW);
+        continue;
       }
-      C += w * invH;
-      wsum += w;
-    };
-    auto match = [&](int p) { return s.pslot[p] == slot; };
-    for_members_ordered(s.sorted + off, len, wbuf, P, match, body);
-    if (C > 0.f) {
-      const float scale = d.eta / C;
-      float *vr = V + (int64_t)slot * d.dv;
+      p = s.partial + (size_t)slot * s.pwidth;
+      if (lane == 0) s.slotmap[x] = slot;
+    }
+    float4 acc[Q4], row[Q4];
+    for (int cb = 0; cb < n4; cb += CB) {
+      if (whole) load_row<Q4>(dst, cb, n4, row);  // in flight with the first sources
+      sum_block<Q4>(d, s, value, cnt, srow_l, coef_l, cb, n4, acc);
+      if (whole) {
+        update_row<Q4>(d, value, dst, cb, n4, row, acc, c0);
+      } else {
 #pragma unroll
-      for (int q = 0; q < Q4; ++q) {
-        const int c4 = lane + 32 * q;
-        if (c4 < dv4) {
-          float4 v = *reinterpret_cast<float4 *>(vr + 4 * c4);
-          v.x -= scale * G[q].x;
-          v.y -= scale * G[q].y;
-          v.z -= scale * G[q].z;
-          v.w -= scale * G[q].w;
-          *reinterpret_cast<float4 *>(vr + 4 * c4) = v;
+        for (int q = 0; q < Q4; ++q) {
+          const int c4 = cb + lane + 32 * q;
+          if (c4 < n4) *reinterpret_cast<float4 *>(p + 4 + 4 * c4) = acc[q];
         }
       }
     }
-    if (d.lam != 0.f) {
-      const float pbar = wsum / (float)d.M;
-      const float bterm = (d.lam / (float)d.M) * (logf(pbar) + 1.f);
-      for (int i = lane; i < len; i += 32) s.pb[s.sorted[off + i]] = bterm;
+    if (whole) {
+      if (value && d.lam != 0.f) write_entropy_term(d, s, c1, g0, len);
+      continue;
     }
+    if (lane == 0) {
+      p[0] = c0;
+      p[1] = c1;
+    }
+    __threadfence();
+    __syncwarp();
+    const int nblocks = (len + kBlock - 1) / kBlock;
+    int old = 0;
+    if (lane == 0) old = atomicAdd(&s.segcnt[g0], 1);
+    old = __shfl_sync(FULL, old, 0);
+    if (old != nblocks - 1) continue;
+    // last block in: add the partials in block order
+    __threadfence();
+    combine_partials<Q4>(d, s, value, dst, n4, g0, len, nblocks);
+    if (lane == 0) s.segcnt[g0] = 0;  // ready for the next chunk
   }
 }
 
-cudaError_t launch_vapply(const Dims &d, float *V, const float *gate, const Scratch &s,
-                          cudaStream_t st) {
-  const int64_t maxU = (int64_t)d.M * d.k;
-  int blocks = (int)((maxU + kApplyWarps - 1) / kApplyWarps);
-  if (blocks > 148 * 8) blocks = 148 * 8;
-  if (blocks < 1) blocks = 1;
-  const int q4 = (d.dv / 4 + 31) / 32;
-  if (q4 <= 1) k_vapply<1><<<blocks, kApplyWarps * 32, 0, st>>>(d, V, gate, s);
-  else if (q4 <= 2) k_vapply<2><<<blocks, kApplyWarps * 32, 0, st>>>(d, V, gate, s);
-  else if (q4 <= 4) k_vapply<4><<<blocks, kApplyWarps * 32, 0, st>>>(d, V, gate, s);
-  else if (q4 <= 8) k_vapply<8><<<blocks, kApplyWarps * 32, 0, st>>>(d, V, gate, s);
-  else if (q4 <= 16) k_vapply<16><<<blocks, kApplyWarps * 32, 0, st>>>(d, V, gate, s);
-  else return cudaErrorInvalidValue;
+template <int Q4>
+static cudaError_t launch_apply_t(const Dims &d, float *V, float *K, const Scratch &s,
+                                  cudaStream_t st, int part) {
+  static int per_sm = 0;
+  if (!per_sm) {
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_apply<Q4>, kApplyWarps * 32, 0);
+    if (per_sm < 1) per_sm = 1;
+  }
+  int64_t blocks = (s.Lcap + kApplyWarps - 1) / kApplyWarps;
+  if (blocks > (int64_t)d.sm_count * per_sm) blocks = (int64_t)d.sm_count * per_sm;
+  k_apply<Q4><<<(int)blocks, kApplyWarps * 32, 0, st>>>(d, V, K, s, part);
   return cudaGetLastError();
 }
 
+cudaError_t launch_apply(const Dims &d, float *V, float *K, const Scratch &s, cudaStream_t st,
+                         int part) {
+  const int w4 = ((d.dv > d.dh ? d.dv : d.dh) / 4 + 31) / 32;
+  if (w4 <= 1) return launch_apply_t<1>(d, V, K, s, st, part);
+  if (w4 <= 2) return launch_apply_t<2>(d, V, K, s, st, part);
+  return launch_apply_t<4>(d, V, K, s, st, part);
+}
+
 // ---------------------------------------------------------------------------
-// pgrad: dL/ds_r = w_r (gamma_r - sum_r' w_r' gamma_r'), gamma = dL/dw.
+// pgrad (lam > 0 only): dL/ds_r = w_r (gamma_r - sum_r' w_r' gamma_r'),
+// gamma = dL_mse/dw + dL_addr/dw, then alpha of the token-head's entries.
 // Warp per token-head, lane r.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_pgrad(Dims d, Scratch s) {
@@ -316,93 +631,25 @@ __global__ void __launch_bounds__(256) k_pgrad(Dims d, Scratch s) {
   float w = 0.f, gam = 0.f;
   if (lane < d.k) {
     w = s.pw[p];
-    gam = s.pa[p] + (d.lam != 0.f ? s.pb[p] : 0.f);
+    gam = s.pa[p] + s.pb[p];
   }
   const float S = warp_sum(w * gam);
-  if (lane < d.k) s.pdl[p] = w * (gam - S);
-}
-
-cudaError_t launch_pgrad(const Dims &d, const Scratch &s, cudaStream_t st) {
-  k_pgrad<<<(d.M + 7) / 8, 256, 0, st>>>(d, s);
-  return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------------------
-// kapply: per touched sub-key row (h, half, i):
-//   alpha_e = (1/(eps + d)) * sum over the entry's pairs of dL/ds
-//   K_i -= eta * 2 * (sum_e alpha_e q_e - (sum_e alpha_e) K_i)
-// ---------------------------------------------------------------------------
-template <int Q4>  // float4 columns per lane: dh <= 128 * Q4
-__global__ void __launch_bounds__(kApplyWarps * 32) k_kapply(Dims d, float *__restrict__ K,
-                                                             Scratch s) {
-  __shared__ int wbuf_all[kApplyWarps][kWarpSortMax];
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  int *wbuf = wbuf_all[wib];
-  const int U_v = s.meta->U_v, U_total = s.meta->U_total;
-  const int dh4 = d.dh >> 2;
-  const int k = d.k, n = d.n;
-  const int64_t E = (int64_t)d.M * 2 * k;
-  for (int u = U_v + blockIdx.x * kApplyWarps + wib; u < U_total;
-       u += gridDim.x * kApplyWarps) {
-    const int bucket = (int)(s.uniq[u] - d.N);  // (h*2+half)*n + sub
-    const int hh = bucket / n, sub = bucket % n;
-    const int off = s.useg_off[u], len = s.useg_len[u];
-    float4 G[Q4];
+  const float dl = lane < d.k ? w * (gam - S) : 0.f;
 #pragma unroll
-    for (int q = 0; q < Q4; ++q) G[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    float A = 0.f;
-    auto body = [&](int e) {
-      const int m = e / (2 * k);
-      const int row = m / d.H;
+  for (int half = 0; half < 2; ++half) {
+    const int mh = m * 2 + half;
+    const int ne = s.ecount[mh];
+    for (int idx = 0; idx < ne; ++idx) {
+      const int64_t e = (int64_t)mh * d.k + idx;
       const unsigned mask = s.emask[e];
-      const float v = (lane < k && ((mask >> lane) & 1u)) ? s.pdl[(int64_t)m * k + lane] : 0.f;
-      const float alpha = s.einv[e] * warp_sum(v);
-      const float *q = s.Qs + ((int64_t)hh * d.rows + row) * d.dh;
-#pragma unroll
-      for (int qq = 0; qq < Q4; ++qq) {
-        const int c4 = lane + 32 * qq;
-        if (c4 < dh4) {
-          const float4 qv = *reinterpret_cast<const float4 *>(q + 4 * c4);
-          G[qq].x = fmaf(alpha, qv.x, G[qq].x);
-          G[qq].y = fmaf(alpha, qv.y, G[qq].y);
-          G[qq].z = fmaf(alpha, qv.z, G[qq].z);
-          G[qq].w = fmaf(alpha, qv.w, G[qq].w);
-        }
-      }
-      A += alpha;
-    };
-    auto match = [&](int e) {
-      const int mh = e / k, idx = e % k;  // mh = m*2 + half
-      const int m = mh >> 1, half = mh & 1;
-      return (m % d.H) * 2 + half == hh && idx < s.ecount[mh] && s.esub[e] == sub;
-    };
-    for_members_ordered(s.sorted + off, len, wbuf, E, match, body);
-    float *kr = K + ((int64_t)hh * n + sub) * d.dh;
-    const float two_eta = 2.f * d.eta;
-#pragma unroll
-    for (int qq = 0; qq < Q4; ++qq) {
-      const int c4 = lane + 32 * qq;
-      if (c4 < dh4) {
-        float4 kv = *reinterpret_cast<float4 *>(kr + 4 * c4);
-        kv.x -= two_eta * (G[qq].x - A * kv.x);
-        kv.y -= two_eta * (G[qq].y - A * kv.y);
-        kv.z -= two_eta * (G[qq].z - A * kv.z);
-        kv.w -= two_eta * (G[qq].w - A * kv.w);
-        *reinterpret_cast<float4 *>(kr + 4 * c4) = kv;
-      }
+      const float sum = warp_sum((mask >> lane) & 1u ? dl : 0.f);
+      if (lane == 0) s.ealpha[e] = s.einv[e] * sum;
     }
   }
 }
 
-cudaError_t launch_kapply(const Dims &d, float *K, const Scratch &s, cudaStream_t st) {
-  int blocks = (2 * d.H * d.n + kApplyWarps - 1) / kApplyWarps;
-  if (blocks > 148 * 8) blocks = 148 * 8;
-  const int q4 = (d.dh / 4 + 31) / 32;
-  if (q4 <= 1) k_kapply<1><<<blocks, kApplyWarps * 32, 0, st>>>(d, K, s);
-  else if (q4 <= 2) k_kapply<2><<<blocks, kApplyWarps * 32, 0, st>>>(d, K, s);
-  else if (q4 <= 4) k_kapply<4><<<blocks, kApplyWarps * 32, 0, st>>>(d, K, s);
-  else if (q4 <= 8) k_kapply<8><<<blocks, kApplyWarps * 32, 0, st>>>(d, K, s);
-  else return cudaErrorInvalidValue;
+cudaError_t launch_pgrad(const Dims &d, const Scratch &s, cudaStream_t st) {
+  k_pgrad<<<(d.M + 7) / 8, 256, 0, st>>>(d, s);
   return cudaGetLastError();
 }
 

@@ -8,6 +8,9 @@
 // token's gate, sciencestack table of contents sections 8-12):
 //   e_t          = yhat_t - v_t
 //   dL/dw_{t,h,r} = (2 g_t / H) e_t . V[slot_{t,h,r}]   (pre-update rows)
+// and, when the entropy term is off (so dL/dw is complete here), the softmax
+// Jacobian dL/ds_r = w_r (dL/dw_r - sum_r' w_r' dL/dw_r') and, per sub-key
+// entry, alpha = (sum of dL/ds over its pairs) / (eps + d).
 // One CTA per token row.  The H*k value rows are fetched by 1-D bulk async
 // copies (TMA) straight into shared memory, completing on one mbarrier, so
 // the whole gather of a token is in flight at once; both passes (weighted
@@ -23,10 +26,10 @@ constexpr size_t kReadSmemBudget = 200 * 1024;
 // Dynamic shared memory layout (bytes):
 //   [0, 16)            mbarrier
 //   [128, 128+R)       staged rows, R = H*k*dv*4 (staged variant only)
-//   then               e (dv floats), w (H*k floats), slot (H*k ints)
+//   then               e (dv floats), w (H*k floats), slot (H*k ints), a (H*k floats)
 static size_t read_smem_bytes(const Dims &d, bool staged) {
   const size_t HK = (size_t)d.H * d.k;
-  return 128 + (staged ? HK * d.dv * 4 : 0) + (size_t)d.dv * 4 + HK * 8;
+  return 128 + (staged ? HK * d.dv * 4 : 0) + (size_t)d.dv * 4 + HK * 12;
 }
 
 template <typename TV, bool kStaged>
@@ -41,6 +44,7 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   float *e_s = rows_s + (kStaged ? (size_t)HK * dv : 0);
   float *w_s = e_s + dv;
   int *slot_s = reinterpret_cast<int *>(w_s + HK);
+  float *a_s = reinterpret_cast<float *>(slot_s + HK);
 
   const int row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -106,14 +110,50 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
       acc = fmaf(e.w, v.w, acc);
     }
     acc = warp_sum(acc);
-    if (lane == 0) s.pa[p0 + j] = coef * acc;
+    if (lane == 0) {
+      s.pa[p0 + j] = coef * acc;
+      a_s[j] = coef * acc;
+    }
   }
 
-  // Scatter member ids into group order: pairs -> value-row groups,
-  // entries -> sub-key-row groups.
+  // dL/ds and alpha per entry when the entropy term is off (dL/dw complete)
+  __syncthreads();
+  const bool alpha_now = d.lam == 0.f;
+  if (alpha_now) {
+    for (int h = wid; h < d.H; h += kReadThreads / 32) {
+      const int j = h * d.k + lane;
+      const float w = lane < d.k ? w_s[j] : 0.f;
+      const float a = lane < d.k ? a_s[j] : 0.f;
+      const float S = warp_sum(w * a);
+      const float dl = w * (a - S);
+      for (int half = 0; half < 2; ++half) {
+        const int64_t mh = ((int64_t)row * d.H + h) * 2 + half;
+        const int ecnt = s.ecount[mh];
+        for (int idx = 0; idx < ecnt; ++idx) {
+          const int64_t e = mh * d.k + idx;
+          const unsigned mask = s.emask[e];
+          const float sum = warp_sum(((mask >> lane) & 1u) ? dl : 0.f);
+          if (lane == 0) s.ealpha[e] = s.einv[e] * sum;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  // Member records into their buckets: pairs -> value bucket slot >> vshift,
+  // entries -> sub-key row bucket NBv + (h*2+half)*n + row.
   for (int j = tid; j < HK; j += blockDim.x) {
     const int64_t p = p0 + j;
-    s.sorted[s.goff[slot_s[j]] + s.pclaim[p]] = (int)p;
+    const float w = w_s[j];
+    Member m;
+    m.g = (uint32_t)slot_s[j];
+    m.id = (uint32_t)p;
+    m.srow = row;
+    m.gstart = 0;
+    m.coef = 2.f * g * w * invH;
+    m.c0 = w * invH;
+    m.c1 = w;
+    m.glen = 0;
+    s.rec_in[s.boff[slot_s[j] >> d.vshift] + s.pclaim[p]] = m;
   }
   const int ne = 2 * HK;  // entries of this row: (h*2 + half)*k + idx
   for (int x = tid; x < ne; x += blockDim.x) {
@@ -121,8 +161,18 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
     const int64_t mhg = (int64_t)row * 2 * d.H + mh;
     if (idx < s.ecount[mhg]) {
       const int64_t e = mhg * d.k + idx;
-      const int64_t grp = d.N + (int64_t)mh * d.n + s.esub[e];
-      s.sorted[s.goff[grp] + s.eclaim[e]] = (int)e;
+      const int sub = s.esub[e];
+      const float alpha = alpha_now ? s.ealpha[e] : 0.f;
+      Member m;
+      m.g = (uint32_t)d.N + (uint32_t)(mh * d.n + sub);
+      m.id = (uint32_t)e;
+      m.srow = mh * d.rows + row;
+      m.gstart = 0;
+      m.coef = alpha;
+      m.c0 = alpha;
+      m.c1 = 0.f;
+      m.glen = 0;
+      s.rec_in[s.boff[d.NBv + mh * d.n + sub] + s.eclaim[e]] = m;
     }
   }
 }

@@ -70,68 +70,82 @@ cudaError_t launch_prep(const Dims &d, const void *Q, int q_dtype, const float *
 }
 
 // ---------------------------------------------------------------------------
-// score: per (h, half) a [rows x dh] . [dh x n] product, 64x64 tiles,
-// 256 threads with 4x4 outputs each, k-steps of 8 (dh % 8 == 0).
+// score: per (h, half) a [rows x dh] . [dh x n] product.  32x64 tiles, 128
+// threads with 4x4 outputs each, k-slices of 8 (dh % 8 == 0); the next slice
+// is fetched into registers while the current one is multiplied.
 // ---------------------------------------------------------------------------
-constexpr int ST_M = 64, ST_N = 64, ST_K = 8;
+constexpr int ST_M = 32, ST_N = 64, ST_K = 8;
 
-__global__ void __launch_bounds__(256) k_score_simt(Dims d, const float *__restrict__ K,
+__global__ void __launch_bounds__(128) k_score_simt(Dims d, const float *__restrict__ K,
                                                     Scratch s) {
-  __shared__ float As[ST_K][ST_M + 4];
-  __shared__ float Bs[ST_K][ST_N + 4];
+  __shared__ float As[2][ST_K][ST_M + 4];
+  __shared__ float Bs[2][ST_K][ST_N + 4];
   const int hh = blockIdx.z;
   const int m0 = blockIdx.y * ST_M, n0 = blockIdx.x * ST_N;
   const int rows = d.rows, n = d.n, dh = d.dh;
   const float *A = s.Qs + (int64_t)hh * rows * dh;
   const float *Bm = K + (int64_t)hh * n * dh;
   const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;  // 16 x 16 threads, 4x4 outputs each
+  const int tx = tid & 15, ty = tid >> 4;  // 16 x 8 threads, 4x4 outputs each
   float acc[4][4] = {};
-  // loader: 128 threads for A (64 rows x 2 float4), 128 for B
-  const int lrow = (tid & 127) >> 1, lq = tid & 1;
-  for (int k0 = 0; k0 < dh; k0 += ST_K) {
-    if (tid < 128) {
-      int r = m0 + lrow;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < rows) v = *reinterpret_cast<const float4 *>(A + (int64_t)r * dh + k0 + lq * 4);
-      As[lq * 4 + 0][lrow] = v.x;
-      As[lq * 4 + 1][lrow] = v.y;
-      As[lq * 4 + 2][lrow] = v.z;
-      As[lq * 4 + 3][lrow] = v.w;
-    } else {
-      int r = n0 + lrow;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < n) v = *reinterpret_cast<const float4 *>(Bm + (int64_t)r * dh + k0 + lq * 4);
-      Bs[lq * 4 + 0][lrow] = v.x;
-      Bs[lq * 4 + 1][lrow] = v.y;
-      Bs[lq * 4 + 2][lrow] = v.z;
-      Bs[lq * 4 + 3][lrow] = v.w;
+  // loaders: A slice = 32 rows x 2 float4 (threads 0..63), B slice = 64 rows x
+  // 2 float4 (all 128 threads)
+  const int arow = tid >> 1, aq = tid & 1;
+  const int brow = tid >> 1, bq = tid & 1;
+  auto fetch = [&](int k0, float4 &va, float4 &vb) {
+    va = make_float4(0.f, 0.f, 0.f, 0.f);
+    vb = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tid < 64 && m0 + arow < rows)
+      va = *reinterpret_cast<const float4 *>(A + (int64_t)(m0 + arow) * dh + k0 + aq * 4);
+    if (n0 + brow < n)
+      vb = *reinterpret_cast<const float4 *>(Bm + (int64_t)(n0 + brow) * dh + k0 + bq * 4);
+  };
+  auto stash = [&](int buf, const float4 &va, const float4 &vb) {
+    if (tid < 64) {
+      As[buf][aq * 4 + 0][arow] = va.x;
+      As[buf][aq * 4 + 1][arow] = va.y;
+      As[buf][aq * 4 + 2][arow] = va.z;
+      As[buf][aq * 4 + 3][arow] = va.w;
     }
-    __syncthreads();
+    Bs[buf][bq * 4 + 0][brow] = vb.x;
+    Bs[buf][bq * 4 + 1][brow] = vb.y;
+    Bs[buf][bq * 4 + 2][brow] = vb.z;
+    Bs[buf][bq * 4 + 3][brow] = vb.w;
+  };
+  float4 va, vb;
+  fetch(0, va, vb);
+  stash(0, va, vb);
+  __syncthreads();
+  int buf = 0;
+  for (int k0 = 0; k0 < dh; k0 += ST_K) {
+    const bool more = k0 + ST_K < dh;
+    if (more) fetch(k0 + ST_K, va, vb);  // in flight during the multiply below
 #pragma unroll
     for (int kk = 0; kk < ST_K; ++kk) {
-      float4 a = *reinterpret_cast<const float4 *>(&As[kk][ty * 4]);
-      float4 b = *reinterpret_cast<const float4 *>(&Bs[kk][tx * 4]);
-      float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+      const float4 a = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
+    if (more) stash(buf ^ 1, va, vb);
     __syncthreads();
+    buf ^= 1;
   }
   const float *qn = s.qn + (int64_t)hh * rows;
   const float *kn = s.kn + (int64_t)hh * n;
   float *D = s.D + (int64_t)hh * rows * n;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    int r = m0 + ty * 4 + i;
+    const int r = m0 + ty * 4 + i;
     if (r >= rows) continue;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      int c = n0 + tx * 4 + j;
+      const int c = n0 + tx * 4 + j;
       if (c >= n) continue;
-      float v = qn[r] + kn[c] - 2.f * acc[i][j];
+      const float v = qn[r] + kn[c] - 2.f * acc[i][j];
       D[(int64_t)r * n + c] = v > 0.f ? v : 0.f;
     }
   }
@@ -139,7 +153,7 @@ __global__ void __launch_bounds__(256) k_score_simt(Dims d, const float *__restr
 
 cudaError_t launch_score(const Dims &d, const float *K, const Scratch &s, cudaStream_t st) {
   dim3 grid((d.n + ST_N - 1) / ST_N, (d.rows + ST_M - 1) / ST_M, 2 * d.H);
-  k_score_simt<<<grid, 256, 0, st>>>(d, K, s);
+  k_score_simt<<<grid, 128, 0, st>>>(d, K, s);
   return cudaGetLastError();
 }
 

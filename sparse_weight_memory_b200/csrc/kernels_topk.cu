@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(128) k_topk(Dims d, Scratch s, Extras x) {
   if (lane < k) {
     s.pslot[p] = slot_r;
     s.pw[p] = w;
-    s.pclaim[p] = atomicAdd(&s.count[slot_r], 1);
+    s.pclaim[p] = atomicAdd(&s.bcnt[slot_r >> d.vshift], 1);  // value bucket
     if (x.rec_slots) {
       x.rec_slots[th * k + lane] = slot_r;
       x.rec_w[th * k + lane] = w;
@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(128) k_topk(Dims d, Scratch s, Extras x) {
       s.esub[e] = sub;
       s.emask[e] = peers;
       s.einv[e] = 1.f / (eps + dist);
-      s.eclaim[e] = atomicAdd(&s.count[d.N + (int64_t)(h * 2 + half) * n + sub], 1);
+      s.eclaim[e] = atomicAdd(&s.bcnt[d.NBv + (h * 2 + half) * n + sub], 1);
     }
     if (lane == 0) s.ecount[(int64_t)m * 2 + half] = __popc(lb);
   }

@@ -175,10 +175,12 @@ def test_edge_shapes(oracle, name):
     compare_runs(wl, inp, g, o, name)
 
 
-@pytest.mark.parametrize("T,chunk", [(96, 96), (1100, 1100)])
+@pytest.mark.parametrize("T,chunk", [(96, 96), (1100, 1100), (5000, 5000)])
 def test_degenerate_identical_queries(oracle, T, chunk):
-    """Every token reads the same slots: one group per slot with T*H members,
-    exercising the shared-memory sort (> 32) and the ordered-scan path (> 1024)."""
+    """Every token reads the same slots: one group per slot with T members.
+    Covers groups split into blocks with partials (> 32 members), buckets
+    sorted by the whole CTA (> 32) and buckets merged through global memory
+    (> 4096)."""
     wl = Workload("deg", B=1, T=T, chunk=chunk, heads=1, dq=32, n=8, dv=16, topk=4, eta=0.5,
                   lam=0.3, gate="uniform")
     inp = make_inputs(wl)
