@@ -177,6 +177,35 @@ fwpkm_status fwpkm_read_stats(fwpkm_state *s, int64_t *chunks, int64_t *value_ro
                               int64_t *key_rows, uint32_t *device_errors, int reset,
                               void *stream);
 
+/*
+ * fwpkm_select_noalloc -- the product-key selection of the read, for callers
+ * that cannot allocate device memory when they call (a serving process that
+ * plans every device byte ahead and runs with a fixed budget, or a plugin
+ * whose host framework owns the device allocator; cudaMalloc may also
+ * synchronise the device).  The paper has no counterpart of this entry point;
+ * it is a deployment variant of the selection done inside fwpkm_step.
+ *   For every token t of the B sequences and every head h, scores both query
+ *   halves against the state's current sub-key tables, takes the product-key
+ *   top-k and writes the slots and their softmax weights -- the same values
+ *   fwpkm_step reads for that token with the same tables.  No readout and no
+ *   update: the tables are not modified.
+ *   Q        device [B][T][heads*dq], element type q_dtype (FWPKM_F32/BF16).
+ *   slots    device int32 [B][T][heads][topk] (output, best first).
+ *   weights  device fp32  [B][T][heads][topk] (output).
+ * Allocates nothing: all scratch is one 16 MiB array in the library's device
+ * image (resident on every GPU that loads the library until exit), used in
+ * passes of as many time steps as fit.  A call whose single time step needs
+ * more than 16 MiB (B x (2*heads*(dq/2 + n + 1)) x 4 bytes plus the sub-key
+ * norms) is rejected with FWPKM_ESHAPE before anything is enqueued.  The
+ * first call on a device looks the array's address up (cudaGetSymbolAddress,
+ * once per device, with that device current); make that first call before any
+ * stream capture.  All calls share the array: calls that overlap on the GPU
+ * (other streams or threads) race and must be ordered by the caller.
+ * Asynchronous on `stream`.
+ */
+fwpkm_status fwpkm_select_noalloc(fwpkm_state *s, int B, int T, const void *Q, int q_dtype,
+                                  int32_t *slots, float *weights, void *stream);
+
 /* Message of the last failure on this thread ("" if none). */
 const char *fwpkm_last_error(void);
 

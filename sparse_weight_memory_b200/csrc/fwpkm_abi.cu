@@ -203,6 +203,26 @@ bool is_dtype(int t) { return t == FWPKM_F32 || t == FWPKM_BF16; }
 
 }  // namespace
 
+namespace fwpkm {
+bool state_view(const fwpkm_state *st, StateView *v) {
+  if (!st || !v) return false;
+  v->N = st->N;
+  v->n = st->n;
+  v->dq = st->dq;
+  v->dh = st->dh;
+  v->dv = st->dv;
+  v->k = st->k;
+  v->chunk = st->chunk;
+  v->H = st->H;
+  v->device = st->device;
+  v->sm_count = st->sm_count;
+  v->eps = st->eps;
+  v->K = st->K;
+  return true;
+}
+void set_last_error(const char *msg) { g_last_error = msg; }
+}  // namespace fwpkm
+
 // ===========================================================================
 // C ABI
 // ===========================================================================

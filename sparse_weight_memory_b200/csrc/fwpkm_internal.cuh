@@ -22,6 +22,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+struct fwpkm_state;
+
 namespace fwpkm {
 
 constexpr unsigned FULL = 0xffffffffu;
@@ -199,6 +201,9 @@ cudaError_t launch_prep(const Dims &d, const void *Q, int q_dtype, const float *
                         const Scratch &s, cudaStream_t st);
 cudaError_t launch_score(const Dims &d, const float *K, const Scratch &s, cudaStream_t st);
 cudaError_t launch_topk(const Dims &d, const Scratch &s, const Extras &x, cudaStream_t st);
+// Selection only: fills x.rec_slots / x.rec_w from the distances in s.D.
+cudaError_t launch_topk_select(const Dims &d, const Scratch &s, const Extras &x,
+                               cudaStream_t st);
 cudaError_t launch_scan(const Dims &d, const Scratch &s, cudaStream_t st);
 cudaError_t launch_read(const Dims &d, const float *V, const void *Vt, int v_dtype,
                         const float *gate, float *out, const Scratch &s, cudaStream_t st);
@@ -207,5 +212,16 @@ cudaError_t launch_bsort(const Dims &d, const Scratch &s, cudaStream_t st);
 cudaError_t launch_apply(const Dims &d, float *V, float *K, const Scratch &s, cudaStream_t st,
                          int part);
 cudaError_t launch_pgrad(const Dims &d, const Scratch &s, cudaStream_t st);
+
+// Read-only view of a state's shape and sub-key tables (fwpkm_abi.cu).
+struct StateView {
+  int64_t N;
+  int n, dq, dh, dv, k, chunk, H, device, sm_count;
+  float eps;
+  const float *K;
+};
+bool state_view(const struct ::fwpkm_state *st, StateView *v);
+// Records `msg` as the calling thread's last error (fwpkm_last_error).
+void set_last_error(const char *msg);
 
 }  // namespace fwpkm

@@ -1,0 +1,141 @@
+// fwpkm_noalloc.cu -- product-key selection that allocates no device memory.
+//
+// fwpkm_select_noalloc runs the selection half of the read (query halves ->
+// sub-key distances -> top-k per half -> k*k merge -> softmax) against a
+// state's current sub-key tables and writes the chosen slots and weights.  It
+// never calls cudaMalloc or cudaFree: its scratch (query halves, norms and the
+// distance matrix) lives in one file-scope device array, g_noalloc_scratch,
+// that is part of the library image.  That serves callers that cannot
+// allocate at call time: a serving process that plans every device byte up
+// front and runs with a fixed budget, or a plugin inside a host framework
+// whose allocator owns the device; cudaMalloc can also synchronise the whole
+// device, which a latency-bound caller cannot afford.
+//
+// The array is shared by every call in the process: concurrent calls that
+// overlap on the GPU (different streams or threads) race on it, so callers
+// must order them.  Nothing in it needs to start at zero: each call writes
+// every scratch element it later reads.  The array stays resident on every
+// GPU that loads the library until the process exits.
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/fwpkm.h"
+#include "fwpkm_internal.cuh"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 16u << 20;  // 16 MiB per device
+
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// The array's device address, looked up once per device with that device
+// current (host code cannot use the symbol itself as a device pointer).
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void *g_scratch_ptr[kMaxDevices] = {};
+
+cudaError_t scratch_on(int dev, void **out) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!g_scratch_ptr[dev]) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+fwpkm_status fail(fwpkm_status st, const char *msg) {
+  fwpkm::set_last_error(msg);
+  return st;
+}
+
+}  // namespace
+
+extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, const void *Q,
+                                             int q_dtype, int32_t *slots, float *weights,
+                                             void *stream_) {
+  using namespace fwpkm;
+  StateView v;
+  if (!state_view(state, &v)) return fail(FWPKM_EINVAL, "select_noalloc: state is NULL");
+  if (!Q || !slots || !weights) return fail(FWPKM_EINVAL, "select_noalloc: NULL pointer");
+  if (q_dtype != FWPKM_F32 && q_dtype != FWPKM_BF16)
+    return fail(FWPKM_EINVAL, "select_noalloc: q_dtype must be FWPKM_F32 or FWPKM_BF16");
+  if (B < 1 || T < 1) return fail(FWPKM_ESHAPE, "select_noalloc: B and T must be >= 1");
+  if (((uintptr_t)Q) & 15) return fail(FWPKM_EINVAL, "select_noalloc: Q must be 16-byte aligned");
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (dev != v.device)
+    return fail(FWPKM_EINVAL, "select_noalloc: current device is not the state's device");
+
+  // Scratch of one pass of `rows` token rows: Qs [2H][rows][dh], qn [2H][rows],
+  // kn [2H][n], D [2H][rows][n] (fp32), each piece 256-byte aligned.
+  const size_t H2 = 2 * (size_t)v.H;
+  const size_t fixed = up256(H2 * v.n * 4) + 3 * 256;
+  const size_t per_row = (H2 * v.dh + H2 + H2 * v.n) * 4;
+  if (fixed + per_row * (size_t)B > kNoAllocScratchBytes) {
+    char msg[256];
+    snprintf(msg, sizeof msg,
+             "select_noalloc: one time step of B=%d sequences needs %zu bytes of scratch, "
+             "more than the %zu-byte static scratch; call it with a smaller B",
+             B, fixed + per_row * (size_t)B, kNoAllocScratchBytes);
+    return fail(FWPKM_ESHAPE, msg);
+  }
+  const int steps_per_pass = (int)((kNoAllocScratchBytes - fixed) / (per_row * (size_t)B));
+  const int Tc = steps_per_pass < T ? steps_per_pass : T;
+  const int rows_max = B * Tc;
+
+  void *base = nullptr;
+  const cudaError_t e = scratch_on(dev, &base);
+  if (e != cudaSuccess) {
+    char msg[256];
+    snprintf(msg, sizeof msg, "select_noalloc: cudaGetSymbolAddress failed: %s",
+             cudaGetErrorString(e));
+    return fail(FWPKM_ECUDA, msg);
+  }
+  char *p = static_cast<char *>(base);
+  Scratch s{};
+  s.Qs = reinterpret_cast<float *>(p);
+  p += up256(H2 * rows_max * v.dh * 4);
+  s.qn = reinterpret_cast<float *>(p);
+  p += up256(H2 * rows_max * 4);
+  s.kn = reinterpret_cast<float *>(p);
+  p += up256(H2 * v.n * 4);
+  s.D = reinterpret_cast<float *>(p);
+
+  Extras x{};
+  x.rec_slots = slots;
+  x.rec_w = weights;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  for (int t0 = 0; t0 < T; t0 += Tc) {
+    Dims d{};
+    d.n = v.n;
+    d.dq = v.dq;
+    d.dh = v.dh;
+    d.dv = v.dv;
+    d.k = v.k;
+    d.H = v.H;
+    d.N = v.N;
+    d.B = B;
+    d.T = T;
+    d.t0 = t0;
+    d.Tc = T - t0 < Tc ? T - t0 : Tc;
+    d.rows = B * d.Tc;
+    d.M = d.rows * v.H;
+    d.sm_count = v.sm_count;
+    d.eps = v.eps;
+    cudaError_t ke = launch_prep(d, Q, q_dtype, v.K, s, stream);
+    if (ke == cudaSuccess) ke = launch_score(d, v.K, s, stream);
+    if (ke == cudaSuccess) ke = launch_topk_select(d, s, x, stream);
+    if (ke != cudaSuccess) {
+      char msg[256];
+      snprintf(msg, sizeof msg, "select_noalloc: launch failed: %s", cudaGetErrorString(ke));
+      return fail(FWPKM_ECUDA, msg);
+    }
+  }
+  return FWPKM_OK;
+}

@@ -121,7 +121,9 @@ __device__ void half_topk(const float *__restrict__ drow, int n, int k, float &d
   i_out = (int)ki;
 }
 
-template <int NV>
+// kSelectOnly: write only the selection record (x.rec_slots / x.rec_w); no
+// pair, entry or bucket outputs.
+template <int NV, bool kSelectOnly>
 __global__ void __launch_bounds__(128) k_topk(Dims d, Scratch s, Extras x) {
   __shared__ uint2 wbuf_all[4][32];
   const int lane = threadIdx.x & 31;
@@ -203,6 +205,13 @@ __global__ void __launch_bounds__(128) k_topk(Dims d, Scratch s, Extras x) {
   const float z = warp_sum(ex);
   const float w = ex / z;
 
+  if (kSelectOnly) {
+    if (lane < k) {
+      x.rec_slots[th * k + lane] = slot_r;
+      x.rec_w[th * k + lane] = w;
+    }
+    return;
+  }
   const int64_t p = (int64_t)m * k + lane;
   if (lane < k) {
     s.pslot[p] = slot_r;
@@ -235,18 +244,29 @@ __global__ void __launch_bounds__(128) k_topk(Dims d, Scratch s, Extras x) {
   }
 }
 
-cudaError_t launch_topk(const Dims &d, const Scratch &s, const Extras &x, cudaStream_t st) {
+template <bool kSelectOnly>
+static cudaError_t launch_topk_t(const Dims &d, const Scratch &s, const Extras &x,
+                                 cudaStream_t st) {
   const int blocks = (d.M + 3) / 4;
   const int nv = (d.n + 31) / 32;
-  if (nv <= 1) k_topk<1><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 2) k_topk<2><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 4) k_topk<4><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 8) k_topk<8><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 16) k_topk<16><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 32) k_topk<32><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 64) k_topk<64><<<blocks, 128, 0, st>>>(d, s, x);
+  if (nv <= 1) k_topk<1, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
+  else if (nv <= 2) k_topk<2, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
+  else if (nv <= 4) k_topk<4, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
+  else if (nv <= 8) k_topk<8, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
+  else if (nv <= 16) k_topk<16, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
+  else if (nv <= 32) k_topk<32, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
+  else if (nv <= 64) k_topk<64, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const Dims &d, const Scratch &s, const Extras &x, cudaStream_t st) {
+  return launch_topk_t<false>(d, s, x, st);
+}
+
+cudaError_t launch_topk_select(const Dims &d, const Scratch &s, const Extras &x,
+                               cudaStream_t st) {
+  return launch_topk_t<true>(d, s, x, st);
 }
 
 }  // namespace fwpkm

@@ -59,10 +59,11 @@ def load_library():
                                      ctypes.POINTER(ctypes.c_double), i64p, i32,
                                      ctypes.POINTER(i32), _vp]
     L.fwpkm_read_stats.argtypes = [_vp, i64p, i64p, i64p, u32p, i32, _vp]
+    L.fwpkm_select_noalloc.argtypes = [_vp, i32, i32, _vp, i32, _vp, _vp, _vp]
     for name in ("fwpkm_state_init", "fwpkm_state_set_eps", "fwpkm_step", "fwpkm_step_host",
                  "fwpkm_state_get", "fwpkm_state_set", "fwpkm_record_selection",
                  "fwpkm_force_selection", "fwpkm_set_profiling", "fwpkm_profile_read",
-                 "fwpkm_read_stats"):
+                 "fwpkm_read_stats", "fwpkm_select_noalloc"):
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -181,6 +182,14 @@ class FwPKMState:
 
     def force_selection(self, slots=None, mask=None):
         _check(load_library().fwpkm_force_selection(self._h, _ptr(slots), _ptr(mask)))
+
+    def select_noalloc(self, Q, slots, weights, stream=None):
+        """Selection only (slots, weights) into caller buffers; allocates nothing."""
+        B, T = Q.shape[0], Q.shape[1]
+        _check(load_library().fwpkm_select_noalloc(self._h, B, T, _ptr(Q), _dtype_code(Q),
+                                                   _ptr(slots), _ptr(weights),
+                                                   _stream(stream)))
+        return slots, weights
 
     # -- measurement -------------------------------------------------------
     def set_profiling(self, enable: bool):
