@@ -61,6 +61,7 @@ struct fwpkm_state {
   size_t arena_bytes = 0;
   int64_t cap_rows = 0;
   Scratch s{};
+  TcMaps maps{};  // TMA descriptors of the score operands in the arena
   // optional per-step inputs / outputs, armed for the next step
   Extras x{};
   // host-buffer staging
@@ -92,6 +93,7 @@ int64_t value_buckets(int64_t N) {
 // Carve the scratch arena for `rows` token rows per chunk.
 fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
   if (rows <= st->cap_rows) return FWPKM_OK;
+  rows = (rows + 127) / 128 * 128;  // query-half stride: whole 128-row score tiles
   const int64_t H = st->H, n = st->n, dh = st->dh, dv = st->dv, k = st->k;
   const int64_t M = rows * H, P = M * k, NB = value_buckets(st->N) + 2 * H * n;
   const int64_t Lcap = 3 * P;  // pairs + at most 2 entries per pair
@@ -104,7 +106,11 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
   Scratch s{};
   std::vector<Piece> pieces = {
       {(void **)&s.Qs, sizeof(float) * (size_t)(H * 2 * rows * dh)},
+      {(void **)&s.Qs_hi, sizeof(float) * (size_t)(H * 2 * rows * dh)},
+      {(void **)&s.Qs_lo, sizeof(float) * (size_t)(H * 2 * rows * dh)},
       {(void **)&s.qn, sizeof(float) * (size_t)(H * 2 * rows)},
+      {(void **)&s.K_hi, sizeof(float) * (size_t)((H * 2 * n + 128) * dh)},
+      {(void **)&s.K_lo, sizeof(float) * (size_t)((H * 2 * n + 128) * dh)},
       {(void **)&s.kn, sizeof(float) * (size_t)(H * 2 * n)},
       {(void **)&s.D, sizeof(float) * (size_t)(H * 2 * rows * n)},
       {(void **)&s.pslot, sizeof(int32_t) * (size_t)P},
@@ -159,10 +165,17 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
     cudaFree(arena);
     return cuda_fail(e, "scratch initialisation");
   }
+  TcMaps maps;
+  e = encode_score_maps(&maps, s, (int)H, (int)rows, (int)n, (int)dh);
+  if (e != cudaSuccess) {
+    cudaFree(arena);
+    return cuda_fail(e, "scratch initialisation: tensor maps");
+  }
   if (st->arena) {
     cudaDeviceSynchronize();
     cudaFree(st->arena);
   }
+  st->maps = maps;
   st->arena = arena;
   st->arena_bytes = total;
   st->s = s;
@@ -357,6 +370,7 @@ fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtyp
     d.t0 = c * st->chunk;
     d.Tc = (T - d.t0 < st->chunk) ? T - d.t0 : st->chunk;
     d.rows = B * d.Tc;
+    d.qstride = (int)st->cap_rows;
     d.M = d.rows * st->H;
     d.vshift = value_shift(st->N);
     d.NBv = (int)value_buckets(st->N);
@@ -368,7 +382,8 @@ fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtyp
     float *V = st->V, *K = st->K;
     if ((rc = run(st, K_PREP, stream, [&] { return launch_prep(d, Q, q_dtype, K, s, stream); })))
       return rc;
-    if ((rc = run(st, K_SCORE, stream, [&] { return launch_score(d, K, s, stream); }))) return rc;
+    if ((rc = run(st, K_SCORE, stream, [&] { return launch_score(d, s, st->maps, stream); })))
+      return rc;
     if ((rc = run(st, K_TOPK, stream, [&] { return launch_topk(d, s, x, stream); }))) return rc;
     if ((rc = run(st, K_SCAN, stream, [&] { return launch_scan(d, s, stream); }))) return rc;
     if ((rc = run(st, K_READ, stream, [&] {

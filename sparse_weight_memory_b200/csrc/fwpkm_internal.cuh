@@ -50,6 +50,7 @@ struct Dims {
   int64_t N;
   int B, T, t0, Tc;   // batch, call length, first token of the chunk, its length
   int rows;           // B * Tc
+  int qstride;        // row stride of the query-half arrays (capacity rows)
   int M;              // rows * H token-heads
   int NBv;            // value buckets: slot >> vshift
   int vshift;
@@ -60,9 +61,13 @@ struct Dims {
 
 // Device scratch owned by the state (sized for the largest chunk seen).
 struct Scratch {
-  float *Qs;        // [H][2][rows][dh]   query halves of the chunk, fp32
-  float *qn;        // [H][2][rows]       |q_half|^2
-  float *kn;        // [H][2][n]          |K_row|^2
+  float *Qs;        // [H][2][qstride][dh] query halves of the chunk, fp32 (may be null)
+  float *Qs_hi;     // [H][2][qstride][dh] TF32-rounded query halves
+  float *Qs_lo;     // [H][2][qstride][dh] query halves minus their TF32 part
+  float *qn;        // [H][2][qstride]     |q_half|^2
+  float *K_hi;      // [H][2][n][dh] + 128 padding rows: TF32-rounded sub-keys
+  float *K_lo;      // same shape: sub-keys minus their TF32 part
+  float *kn;        // [H][2][n]           |K_row|^2
   float *D;         // [H][2][rows][n]    squared distances
   int32_t *pslot;   // [M*k] selected slot of pair p = m*k + r
   float *pw;        // [M*k] softmax weight
@@ -199,7 +204,19 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
 // ------------------------------------------------------------------------
 cudaError_t launch_prep(const Dims &d, const void *Q, int q_dtype, const float *K,
                         const Scratch &s, cudaStream_t st);
-cudaError_t launch_score(const Dims &d, const float *K, const Scratch &s, cudaStream_t st);
+// TMA descriptors (CUtensorMap, 128 bytes each) of the score operands.
+struct TcMaps {
+  alignas(64) unsigned char a_hi[128];
+  alignas(64) unsigned char a_lo[128];
+  alignas(64) unsigned char b_hi[4][128];  // column tiles of 16, 32, 64, 128
+  alignas(64) unsigned char b_lo[4][128];
+};
+// Encodes the four maps over Qs_hi / Qs_lo ([2H*qstride][dh], qstride a
+// multiple of 128) and K_hi / K_lo ([2H*n + 128][dh]).  Host only; returns a
+// CUDA error code.
+cudaError_t encode_score_maps(TcMaps *maps, const Scratch &s, int H, int qstride, int n,
+                              int dh);
+cudaError_t launch_score(const Dims &d, const Scratch &s, const TcMaps &maps, cudaStream_t st);
 cudaError_t launch_topk(const Dims &d, const Scratch &s, const Extras &x, cudaStream_t st);
 // Selection only: fills x.rec_slots / x.rec_w from the distances in s.D.
 cudaError_t launch_topk_select(const Dims &d, const Scratch &s, const Extras &x,

@@ -1,7 +1,8 @@
 // fwpkm_noalloc.cu -- product-key selection that allocates no device memory.
 //
 // fwpkm_select_noalloc runs the selection half of the read (query halves ->
-// sub-key distances -> top-k per half -> k*k merge -> softmax) against a
+// sub-key distances on the tensor cores -> top-k per half -> k*k merge ->
+// softmax) against a
 // state's current sub-key tables and writes the chosen slots and weights.  It
 // never calls cudaMalloc or cudaFree: its scratch (query halves, norms and the
 // distance matrix) lives in one file-scope device array, g_noalloc_scratch,
@@ -72,22 +73,25 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
   if (dev != v.device)
     return fail(FWPKM_EINVAL, "select_noalloc: current device is not the state's device");
 
-  // Scratch of one pass of `rows` token rows: Qs [2H][rows][dh], qn [2H][rows],
-  // kn [2H][n], D [2H][rows][n] (fp32), each piece 256-byte aligned.
+  // Scratch of one pass of `rows` token rows (fp32, each piece 256-byte
+  // aligned; rows rounded up to 128): Qs_hi, Qs_lo [2H][rows][dh], qn
+  // [2H][rows], D [2H][rows][n]; fixed: K_hi, K_lo [2H*n + 128][dh], kn [2H][n].
   const size_t H2 = 2 * (size_t)v.H;
-  const size_t fixed = up256(H2 * v.n * 4) + 3 * 256;
-  const size_t per_row = (H2 * v.dh + H2 + H2 * v.n) * 4;
+  const size_t fixed = 2 * up256((H2 * v.n + 128) * v.dh * 4) + up256(H2 * v.n * 4) +
+                       4 * 256 + 128 * (2 * H2 * v.dh + H2 + H2 * v.n) * 4;
+  const size_t per_row = (2 * H2 * v.dh + H2 + H2 * v.n) * 4;
   if (fixed + per_row * (size_t)B > kNoAllocScratchBytes) {
     char msg[256];
     snprintf(msg, sizeof msg,
              "select_noalloc: one time step of B=%d sequences needs %zu bytes of scratch, "
-             "more than the %zu-byte static scratch; call it with a smaller B",
+             "more than the %zu-byte static scratch; call it with a smaller B (or a "
+             "smaller memory)",
              B, fixed + per_row * (size_t)B, kNoAllocScratchBytes);
     return fail(FWPKM_ESHAPE, msg);
   }
   const int steps_per_pass = (int)((kNoAllocScratchBytes - fixed) / (per_row * (size_t)B));
   const int Tc = steps_per_pass < T ? steps_per_pass : T;
-  const int rows_max = B * Tc;
+  const int rows_max = (B * Tc + 127) / 128 * 128;  // whole 128-row score tiles
 
   void *base = nullptr;
   const cudaError_t e = scratch_on(dev, &base);
@@ -99,13 +103,23 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
   }
   char *p = static_cast<char *>(base);
   Scratch s{};
-  s.Qs = reinterpret_cast<float *>(p);
+  s.Qs = nullptr;  // the plain halves are only needed by the update
+  s.Qs_hi = reinterpret_cast<float *>(p);
+  p += up256(H2 * rows_max * v.dh * 4);
+  s.Qs_lo = reinterpret_cast<float *>(p);
   p += up256(H2 * rows_max * v.dh * 4);
   s.qn = reinterpret_cast<float *>(p);
   p += up256(H2 * rows_max * 4);
+  s.K_hi = reinterpret_cast<float *>(p);
+  p += up256((H2 * v.n + 128) * v.dh * 4);
+  s.K_lo = reinterpret_cast<float *>(p);
+  p += up256((H2 * v.n + 128) * v.dh * 4);
   s.kn = reinterpret_cast<float *>(p);
   p += up256(H2 * v.n * 4);
   s.D = reinterpret_cast<float *>(p);
+  TcMaps maps;  // host-side descriptors of the operands above (no allocation)
+  const cudaError_t me = encode_score_maps(&maps, s, v.H, rows_max, v.n, v.dh);
+  if (me != cudaSuccess) return fail(FWPKM_ECUDA, "select_noalloc: tensor map encoding failed");
 
   Extras x{};
   x.rec_slots = slots;
@@ -125,11 +139,12 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
     d.t0 = t0;
     d.Tc = T - t0 < Tc ? T - t0 : Tc;
     d.rows = B * d.Tc;
+    d.qstride = rows_max;
     d.M = d.rows * v.H;
     d.sm_count = v.sm_count;
     d.eps = v.eps;
     cudaError_t ke = launch_prep(d, Q, q_dtype, v.K, s, stream);
-    if (ke == cudaSuccess) ke = launch_score(d, v.K, s, stream);
+    if (ke == cudaSuccess) ke = launch_score(d, s, maps, stream);
     if (ke == cudaSuccess) ke = launch_topk_select(d, s, x, stream);
     if (ke != cudaSuccess) {
       char msg[256];

@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
       Member m;
       m.g = (uint32_t)d.N + (uint32_t)(mh * d.n + sub);
       m.id = (uint32_t)e;
-      m.srow = mh * d.rows + row;
+      m.srow = mh * d.qstride + row;
       m.gstart = 0;
       m.coef = alpha;
       m.c0 = alpha;

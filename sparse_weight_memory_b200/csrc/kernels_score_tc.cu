@@ -1,0 +1,312 @@
+// kernels_score_tc.cu -- sub-key distances on the 5th-generation tensor cores.
+//
+// IDW scoring (gist.science "Fast-weight Product Key Memory", section 2, Key
+// Technical Choices) needs ||q_half - K_i||^2 for every sub-key of both halves:
+// the step's only dense contraction, q_half . K_i.  Per (head, half) it is a
+// [rows x dh] . [dh x n] product; this kernel computes it with tcgen05.mma
+// (kind::tf32, fp32 accumulate in tensor memory) on operand tiles brought in
+// by TMA, and writes
+//     D[h][half][row][i] = |q|^2 + |K_i|^2 - 2 q.K_i      (clamped at 0)
+//
+// Precision: three TF32 products, hi*hi + hi*lo + lo*hi, where x = hi + lo and
+// hi is x rounded to TF32 (the prep kernel writes both parts).  The dropped
+// lo*lo term and the truncation of lo are ~2^-21 relative, so the distances
+// match an fp32 evaluation to a few ulps and the selection is decided at
+// fp32 accuracy.
+//
+// CTA = one 128-row x BN-column output tile of one (head, half); 4 warps.
+//   warp 0, one lane: TMA producer over k-blocks of 32 elements (128 bytes,
+//                     128-byte swizzle), kStages-deep ring;
+//   warp 1:           allocates the accumulator columns in tensor memory;
+//                     one lane issues the MMAs and commits each stage back;
+//   warps 0-3:        epilogue, one accumulator lane (= output row) per thread.
+// Every mbarrier wait is bounded; a wait that gives up sets an error bit,
+// the kernel still releases its tensor memory and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "fwpkm_internal.cuh"
+
+namespace fwpkm {
+
+constexpr int kTcRows = 128;      // M of every MMA (cta_group::1)
+constexpr int kTcKBlock = 32;     // fp32 elements per 128-byte swizzle row
+constexpr int kTcStages = 3;
+
+// --- tcgen05 helpers (inline PTX, sm_100a) --------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t *slot_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(slot_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::tf32.
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` once every MMA issued so far by this thread has completed.
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+// 32 consecutive fp32 columns of this thread's accumulator lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 2-D tiled TMA load (no multicast) of box {32 elements, rows} at {x, y}.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), leading offset field 1, descriptor version 1.
+__device__ __forceinline__ uint64_t kmajor_sw128_desc(const void *smem_tile) {
+  const uint64_t start = (uint64_t)(smem_u32(smem_tile) >> 4) & 0x3fffull;
+  return start | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor: D f32, A and B tf32, both K-major, M = 128, N = BN.
+template <int BN>
+__device__ __forceinline__ uint32_t idesc_tf32() {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(BN >> 3) << 17) |
+         ((uint32_t)(kTcRows >> 4) << 24);
+}
+
+template <int BN>
+struct TcSmem {
+
+  static constexpr int kA = kTcRows * kTcKBlock * 4;  // 16 KiB per operand part
+  static constexpr int kB = BN * kTcKBlock * 4;
+  static constexpr int kStage = 2 * kA + 2 * kB;      // hi and lo of A and B
+  static constexpr int kBytes = kTcStages * kStage + 1024 /* align */ + 256 /* barriers */;
+  static_assert(kStage >= 4 * 32 * 33 * 4, "epilogue tile fits in stage 0");
+};
+
+template <int BN>
+__global__ void __launch_bounds__(128, 1)
+    k_score_tc(const __grid_constant__ CUtensorMap mapAhi, const __grid_constant__ CUtensorMap mapAlo,
+               const __grid_constant__ CUtensorMap mapBhi, const __grid_constant__ CUtensorMap mapBlo,
+               Dims d, Scratch s) {
+  extern __shared__ unsigned char smem_raw[];
+  using L = TcSmem<BN>;
+  constexpr uint32_t kCols = BN < 32 ? 32 : BN;  // tensor-memory columns (power of 2)
+  unsigned char *smem =
+      reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kTcStages * L::kStage);
+  uint64_t *empty = full + kTcStages;
+  uint64_t *done = empty + kTcStages;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hh = blockIdx.z;
+  const int m0 = blockIdx.y * kTcRows, n0 = blockIdx.x * BN;
+  const int nkb = (d.dh + kTcKBlock - 1) / kTcKBlock;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kTcStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(done, 1);
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mapAhi)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mapBhi)) : "memory");
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer ----------------
+    const int ya = hh * d.qstride + m0;  // row of the query-half tensor
+    const int yb = hh * d.n + n0;        // row of the sub-key tensor
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int st = kb % kTcStages, round = kb / kTcStages;
+      if (!mbar_wait_bounded(&empty[st], (round & 1) ^ 1, s.meta)) break;
+      unsigned char *stage = smem + st * L::kStage;
+      mbar_arrive_expect_tx(&full[st], L::kStage);
+      const int x = kb * kTcKBlock;
+      tma_load_2d(stage, &mapAhi, x, ya, &full[st]);
+      tma_load_2d(stage + L::kA, &mapAlo, x, ya, &full[st]);
+      tma_load_2d(stage + 2 * L::kA, &mapBhi, x, yb, &full[st]);
+      tma_load_2d(stage + 2 * L::kA + L::kB, &mapBlo, x, yb, &full[st]);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer ----------------
+    const uint32_t idesc = idesc_tf32<BN>();
+    bool ok = true;
+    for (int kb = 0; kb < nkb && ok; ++kb) {
+      const int st = kb % kTcStages, round = kb / kTcStages;
+      ok = mbar_wait_bounded(&full[st], round & 1, s.meta);
+      if (!ok) break;
+      tc_fence_after();
+      const unsigned char *stage = smem + st * L::kStage;
+      const unsigned char *ahi = stage, *alo = stage + L::kA;
+      const unsigned char *bhi = stage + 2 * L::kA, *blo = stage + 2 * L::kA + L::kB;
+#pragma unroll
+      for (int k8 = 0; k8 < kTcKBlock / 8; ++k8) {  // 8 tf32 = 32 bytes per MMA
+        const int off = k8 * 32;
+        const uint32_t acc = (kb > 0 || k8 > 0) ? 1u : 0u;
+        mma_tf32(tmem, kmajor_sw128_desc(ahi + off), kmajor_sw128_desc(bhi + off), idesc, acc);
+        mma_tf32(tmem, kmajor_sw128_desc(ahi + off), kmajor_sw128_desc(blo + off), idesc, 1u);
+        mma_tf32(tmem, kmajor_sw128_desc(alo + off), kmajor_sw128_desc(bhi + off), idesc, 1u);
+      }
+      mma_commit(&empty[st]);  // stage free once these MMAs have read it
+    }
+    mma_commit(done);  // accumulator complete (or abandoned after an error)
+  }
+  __syncwarp();
+
+  // ---------------- epilogue: TMEM -> distances ----------------
+  // Each warp owns 32 accumulator lanes (rows).  Per block of 32 columns the
+  // values go through a padded shared-memory tile (the stage buffers are free
+  // now) so that every store writes 32 consecutive columns of one row.
+  // warp-uniform: tcgen05.ld below is a warp-collective instruction
+  const bool ready = __all_sync(FULL, mbar_wait_bounded(done, 0, s.meta));
+  tc_fence_after();
+  if (ready) {
+    float *tile = reinterpret_cast<float *>(smem) + warp * 32 * 33;
+    const int row0 = m0 + warp * 32;
+    const int my_row = row0 + lane;
+    const float my_qn = my_row < d.rows ? s.qn[(int64_t)hh * d.qstride + my_row] : 0.f;
+    const float *kn = s.kn + (int64_t)hh * d.n;
+    float *Dh = s.D + (int64_t)hh * d.rows * d.n;
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+      float v[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) tile[lane * 33 + j] = v[j];
+      __syncwarp();
+      const int col = n0 + c0 + lane;
+      const bool col_ok = col < d.n && c0 + lane < BN;
+      const float kn_l = col_ok ? kn[col] : 0.f;
+#pragma unroll 4
+      for (int r = 0; r < 32; ++r) {
+        const float qn_r = __shfl_sync(FULL, my_qn, r);
+        const float dist = qn_r + kn_l - 2.f * tile[r * 33 + lane];
+        if (col_ok && row0 + r < d.rows)
+          Dh[(int64_t)(row0 + r) * d.n + col] = dist > 0.f ? dist : 0.f;
+      }
+      __syncwarp();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCols);
+  }
+}
+
+// --- host side -------------------------------------------------------------
+template <int BN>
+static cudaError_t launch_tc(const Dims &d, const Scratch &s, const TcMaps &maps, int v,
+                             cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_score_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         TcSmem<BN>::kBytes);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid((d.n + BN - 1) / BN, (d.rows + kTcRows - 1) / kTcRows, 2 * d.H);
+  k_score_tc<BN><<<grid, 128, TcSmem<BN>::kBytes, st>>>(
+      *reinterpret_cast<const CUtensorMap *>(maps.a_hi), *reinterpret_cast<const CUtensorMap *>(maps.a_lo),
+      *reinterpret_cast<const CUtensorMap *>(maps.b_hi[v]),
+      *reinterpret_cast<const CUtensorMap *>(maps.b_lo[v]), d, s);
+  return cudaGetLastError();
+}
+
+// Column-tile width: the widest of 128 / 64 / 32 / 16 that still gives at
+// least one CTA per multiprocessor (narrower tiles when the chunk is small).
+cudaError_t launch_score(const Dims &d, const Scratch &s, const TcMaps &maps, cudaStream_t st) {
+  const int64_t base = (int64_t)((d.rows + kTcRows - 1) / kTcRows) * 2 * d.H;
+  int bn = 128;
+  while (bn > 16 && (bn >= 2 * d.n || base * ((d.n + bn - 1) / bn) < d.sm_count)) bn >>= 1;
+  if (bn == 16) return launch_tc<16>(d, s, maps, 0, st);
+  if (bn == 32) return launch_tc<32>(d, s, maps, 1, st);
+  if (bn == 64) return launch_tc<64>(d, s, maps, 2, st);
+  return launch_tc<128>(d, s, maps, 3, st);
+}
+
+// fp32 [rows][inner] tensor, box {32 elements, box_rows}, 128-byte swizzle,
+// out-of-range elements read as zero.
+static cudaError_t encode_2d(void *out, const float *base, uint64_t inner, uint64_t rows,
+                             uint32_t box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return e;
+    if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * sizeof(float)};
+  const cuuint32_t box[2] = {(cuuint32_t)kTcKBlock, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(reinterpret_cast<CUtensorMap *>(out), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                            const_cast<float *>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// qstride must be a multiple of 128 and K_hi / K_lo must hold 128 rows past
+// the 2*H*n sub-key rows, so that every box lies inside its tensor.
+cudaError_t encode_score_maps(TcMaps *maps, const Scratch &s, int H, int qstride, int n,
+                              int dh) {
+  if (qstride % kTcRows) return cudaErrorInvalidValue;
+  const uint64_t qrows = 2ull * H * qstride, krows = 2ull * H * n + kTcRows;
+  cudaError_t e = encode_2d(maps->a_hi, s.Qs_hi, dh, qrows, kTcRows);
+  if (e == cudaSuccess) e = encode_2d(maps->a_lo, s.Qs_lo, dh, qrows, kTcRows);
+  for (int v = 0; v < 4 && e == cudaSuccess; ++v) {  // column tiles of 16, 32, 64, 128
+    e = encode_2d(maps->b_hi[v], s.K_hi, dh, krows, 16u << v);
+    if (e == cudaSuccess) e = encode_2d(maps->b_lo[v], s.K_lo, dh, krows, 16u << v);
+  }
+  return e;
+}
+
+}  // namespace fwpkm
