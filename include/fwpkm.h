@@ -136,7 +136,8 @@ fwpkm_status fwpkm_state_set(fwpkm_state *s, const float *subkeys, const float *
 
 /*
  * fwpkm_record_selection -- arm a record of the slots and weights the NEXT
- * fwpkm_step reads (device int32 / fp32, [B][T][heads][topk], best first),
+ * fwpkm_step reads (device int32 / fp32, [B][T][heads][topk]; the k slots of
+ * a token-head in no particular order),
  * for inspection and parity checks.  Pass NULL, NULL to disarm.  The buffers
  * must hold B*T*heads*topk entries of the next call's B and T.
  */
@@ -190,7 +191,8 @@ fwpkm_status fwpkm_read_stats(fwpkm_state *s, int64_t *chunks, int64_t *value_ro
  *   fwpkm_step reads for that token with the same tables.  No readout and no
  *   update: the tables are not modified.
  *   Q        device [B][T][heads*dq], element type q_dtype (FWPKM_F32/BF16).
- *   slots    device int32 [B][T][heads][topk] (output, best first).
+ *   slots    device int32 [B][T][heads][topk] (output; the k slots of a
+ *            token-head in no particular order, the same order fwpkm_step reads).
  *   weights  device fp32  [B][T][heads][topk] (output).
  * Allocates nothing: all scratch is one 16 MiB array in the library's device
  * image (resident on every GPU that loads the library until exit), used in

@@ -130,6 +130,8 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
       {(void **)&s.rec, sizeof(Member) * (size_t)Lcap},
       {(void **)&s.posmap, sizeof(int32_t) * (size_t)Lcap},
       {(void **)&s.slotmap, sizeof(int32_t) * (size_t)Lcap},
+      {(void **)&s.shortlist, sizeof(int32_t) * (size_t)Lcap},
+      {(void **)&s.longlist, sizeof(int32_t) * (size_t)Lcap},
       {(void **)&s.sort_tmp, sizeof(uint64_t) * (size_t)(2 * Lcap)},
       {(void **)&s.partial, sizeof(float) * (size_t)pool_cap * pwidth},
       {(void **)&s.segcnt, sizeof(int32_t) * (size_t)Lcap},

@@ -39,6 +39,9 @@ struct Meta {
   int32_t Lv;             // pairs (value-row members come first)
   unsigned err;           // ERR_* bits, sticky until the host clears them
   int32_t pool_next;      // next free partial slot (reset per chunk)
+  int32_t nshort;         // groups of <= 2 members listed in shortlist (reset per chunk)
+  int32_t nlong;          // 32-member blocks of longer groups in longlist (reset per chunk)
+  int32_t pad2;
   unsigned long long stat_chunks;      // chunks processed since reset
   unsigned long long stat_value_rows;  // sum over chunks of distinct value rows written
   unsigned long long stat_key_rows;    // sum over chunks of distinct sub-key rows written
@@ -87,6 +90,8 @@ struct Scratch {
   uint64_t *sort_tmp;  // [2*Lcap] merge buffers for oversized buckets
   int32_t *posmap;  // [Lcap]  position inside its bucket, by member id (oversized buckets)
   int32_t *slotmap; // [Lcap]  partial-pool slot of the block starting here
+  int32_t *shortlist;  // [Lcap] first position of every group of <= 2 members
+  int32_t *longlist;   // [Lcap] first position of every 32-member block of longer groups
   float *partial;   // [pool_cap][pwidth] block partial sums of long groups
   int32_t *segcnt;  // [Lcap] arrived blocks per long group, at its first position
                     // (zero between chunks)

@@ -51,67 +51,85 @@ __device__ __forceinline__ void store_member(Member *p, const Member &m) {
 }
 
 // ---------------------------------------------------------------------------
-// scan: bucket offsets (single CTA).  Each thread owns a contiguous run of
-// buckets; its counts are loaded before the block-wide scan.
+// scan: bucket offsets (single CTA).  The counts are staged in shared memory
+// with coalesced 16-byte loads, each thread scans a contiguous run there, and
+// the offsets go back with coalesced stores; pieces of kScanPiece buckets.
 // ---------------------------------------------------------------------------
 constexpr int kScanThreads = 1024;
-constexpr int kScanRun = 16;  // counts held in registers per thread and pass
+constexpr int kScanPiece = 8192;
 
 __global__ void __launch_bounds__(kScanThreads) k_bucket_scan(Dims d, Scratch s) {
+  __shared__ __align__(16) int cnt[kScanPiece];
   __shared__ int red[32];
+  __shared__ int carry_s;
   const int NB = d.NB;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int per = (NB + kScanThreads - 1) / kScanThreads;  // buckets per thread
-  const int b0 = min(threadIdx.x * per, NB), b1 = min(b0 + per, NB);
-  int total = 0;
-  for (int b = b0; b < b1; b += kScanRun) {
-    int v[kScanRun];
-#pragma unroll
-    for (int i = 0; i < kScanRun; ++i) v[i] = b + i < b1 ? s.bcnt[b + i] : 0;
-#pragma unroll
-    for (int i = 0; i < kScanRun; ++i) total += v[i];
-  }
-  // exclusive scan of the per-thread totals
-  int incl = total;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int t = __shfl_up_sync(FULL, incl, o);
-    if (lane >= o) incl += t;
-  }
-  if (lane == 31) red[w] = incl;
-  __syncthreads();
-  if (w == 0) {
-    int x = red[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(FULL, x, o);
-      if (lane >= o) x += t;
-    }
-    red[lane] = x;
-  }
-  __syncthreads();
-  int run = (w > 0 ? red[w - 1] : 0) + incl - total;
-  for (int b = b0; b < b1; b += kScanRun) {
-    int v[kScanRun];
-#pragma unroll
-    for (int i = 0; i < kScanRun; ++i) v[i] = b + i < b1 ? s.bcnt[b + i] : 0;
-#pragma unroll
-    for (int i = 0; i < kScanRun; ++i) {
-      if (b + i < b1) {
-        s.boff[b + i] = run;
-        if (b + i == d.NBv) s.meta->Lv = run;  // value buckets come first
-        s.bcnt[b + i] = 0;                       // ready for the next chunk
-        run += v[i];
+  constexpr int per = kScanPiece / kScanThreads;  // 8 buckets per thread and piece
+  int carry = 0;
+  for (int p0 = 0; p0 < NB; p0 += kScanPiece) {
+    const int np = min(kScanPiece, NB - p0);
+    // bcnt and boff are 256-byte aligned; p0 is a multiple of 8192
+    for (int i = threadIdx.x * 4; i < np; i += kScanThreads * 4) {
+      if (i + 4 <= np) {
+        *reinterpret_cast<int4 *>(cnt + i) = *reinterpret_cast<const int4 *>(s.bcnt + p0 + i);
+        *reinterpret_cast<int4 *>(s.bcnt + p0 + i) = make_int4(0, 0, 0, 0);  // next chunk
+      } else {
+        for (int j = i; j < np; ++j) {
+          cnt[j] = s.bcnt[p0 + j];
+          s.bcnt[p0 + j] = 0;
+        }
       }
     }
+    __syncthreads();
+    const int b0 = threadIdx.x * per;
+    int v[per];
+    int total = 0;
+#pragma unroll
+    for (int i = 0; i < per; ++i) {
+      v[i] = b0 + i < np ? cnt[b0 + i] : 0;
+      total += v[i];
+    }
+    int incl = total;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(FULL, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane == 31) red[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+      int x = red[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(FULL, x, o);
+        if (lane >= o) x += t;
+      }
+      red[lane] = x;
+    }
+    __syncthreads();
+    int run = carry + (w > 0 ? red[w - 1] : 0) + incl - total;
+#pragma unroll
+    for (int i = 0; i < per; ++i) {
+      cnt[b0 + i] = run;  // exclusive offsets, in place
+      run += v[i];
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < np; i += kScanThreads) s.boff[p0 + i] = cnt[i];
+    if (threadIdx.x == 0) {
+      if (d.NBv >= p0 && d.NBv < p0 + np) s.meta->Lv = cnt[d.NBv - p0];
+      carry_s = carry + red[31];
+    }
+    __syncthreads();
+    carry = carry_s;
   }
-  if (threadIdx.x == kScanThreads - 1) {
-    const int L = red[31];
-    s.boff[NB] = L;
-    s.meta->L = L;
-    if (d.NBv == NB) s.meta->Lv = L;
+  if (threadIdx.x == 0) {
+    s.boff[NB] = carry;
+    s.meta->L = carry;
+    if (d.NBv >= NB) s.meta->Lv = carry;
     s.meta->stat_chunks += 1ull;
     s.meta->pool_next = 0;
+    s.meta->nshort = 0;
+    s.meta->nlong = 0;
   }
 }
 
@@ -168,6 +186,22 @@ __device__ __forceinline__ int lower_rank(const uint64_t *r, int len, uint64_t k
   return lo;
 }
 
+constexpr int kShortMax = 2;  // groups up to this size are applied by one warp
+constexpr int kBlock = 32;    // longer groups are applied in blocks of this many members
+
+// Work lists of the apply kernel for a group that starts at position x0:
+// a short group goes to shortlist, a longer one to longlist, one entry per
+// block of kBlock members.  Thread-level (one call per group head).
+__device__ __forceinline__ void list_group(const Scratch &s, int x0, int len) {
+  if (len <= kShortMax) {
+    s.shortlist[atomicAdd(&s.meta->nshort, 1)] = x0;
+  } else {
+    const int nb = (len + kBlock - 1) / kBlock;
+    const int base = atomicAdd(&s.meta->nlong, nb);
+    for (int b = 0; b < nb; ++b) s.longlist[base + b] = x0 + b * kBlock;
+  }
+}
+
 // CTA-wide sort of one bucket with more than 32 members.
 __device__ void sort_big_bucket(const Scratch &s, int off, int len, bool value, uint32_t gbase,
                                 uint64_t *buf, int *nseg) {
@@ -191,12 +225,15 @@ __device__ void sort_big_bucket(const Scratch &s, int off, int len, bool value, 
       const uint64_t kv = buf[i];
       const uint64_t grp = kv >> 43;
       const int first = lower_rank(buf, len, grp << 43);
-      const int end = (grp + 1) >= (1ull << 21) ? len : lower_rank(buf, len, (grp + 1) << 43);
+      const int end = lower_rank(buf, len, (grp + 1) << 43);
       Member m = load_member(s.rec_in + off + (int)(kv & 4095u));
       m.gstart = off + first;
       m.glen = end - first;
       store_member(s.rec + off + i, m);
-      my_seg += first == i ? 1 : 0;
+      if (first == i) {
+        my_seg += 1;
+        list_group(s, off + i, end - first);
+      }
     }
   } else {
     // Oversized bucket: keys (g << 32 | id) sorted in runs of kSortCap in
@@ -250,7 +287,10 @@ __device__ void sort_big_bucket(const Scratch &s, int off, int len, bool value, 
       m.gstart = off + first;
       m.glen = end - first;
       store_member(s.rec + off + i, m);
-      my_seg += first == i ? 1 : 0;
+      if (first == i) {
+        my_seg += 1;
+        list_group(s, off + i, end - first);
+      }
     }
   }
   if (my_seg) atomicAdd(nseg, my_seg);
@@ -260,14 +300,27 @@ __device__ void sort_big_bucket(const Scratch &s, int off, int len, bool value, 
 __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s) {
   __shared__ uint64_t buf[kSortCap];
   __shared__ int nseg[2];  // distinct value rows / sub-key rows seen by this CTA
+  __shared__ int big_n;
+  __shared__ int big_b[kSortWarps * 8];  // large buckets met in phase 1
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   if (threadIdx.x < 2) nseg[threadIdx.x] = 0;
+  if (threadIdx.x == 0) big_n = 0;
   __syncthreads();
   const int stride = gridDim.x * kSortWarps;
-  // phase 1: small buckets, one warp each
-  for (int b = blockIdx.x * kSortWarps + wib; b < d.NB; b += stride) {
+  // phase 1: small buckets, one warp each; large ones are listed.  Bucket b
+  // goes to CTA b % gridDim.x: neighbouring buckets (slots of one popular
+  // sub-key row) land in different CTAs.
+  for (int b = blockIdx.x + gridDim.x * wib; b < d.NB; b += stride) {
     const int off = s.boff[b], len = s.boff[b + 1] - off;
-    if (len == 0 || len > 32) continue;
+    if (len == 0) continue;
+    if (len > 32) {
+      if (lane == 0) {
+        const int slot = atomicAdd(&big_n, 1);
+        if (slot < kSortWarps * 8) big_b[slot] = b;
+        else atomicOr(&s.meta->err, ERR_POOL_OVERFLOW);  // cannot happen: see launch_bsort
+      }
+      continue;
+    }
     Member m{};
     uint64_t key = ~0ull;
     if (lane < len) {
@@ -302,28 +355,39 @@ __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s)
     const uint32_t prev_g = __shfl_up_sync(FULL, r.g, 1);
     const bool head = lane < len && (lane == 0 || prev_g != r.g);
     const unsigned heads = __ballot_sync(FULL, head);
+    int glen = 0;
     if (lane < len) {
       const unsigned upto = heads & ((2u << lane) - 1u);  // heads at or below this lane
       const int h0 = 31 - __clz(upto);
       const unsigned after = heads & ~((2u << h0) - 1u);  // heads after the group's first
       r.gstart = off + h0;
-      r.glen = (after ? __ffs(after) - 1 : len) - h0;
+      r.glen = glen = (after ? __ffs(after) - 1 : len) - h0;
       store_member(s.rec + off + lane, r);
     }
+    // work lists: short groups, and the blocks of longer ones
+    const bool sh = head && glen <= kShortMax;
+    const unsigned sb = __ballot_sync(FULL, sh);
+    int sbase = 0;
+    if (lane == 0 && sb) sbase = atomicAdd(&s.meta->nshort, __popc(sb));
+    sbase = __shfl_sync(FULL, sbase, 0);
+    if (sh) s.shortlist[sbase + __popc(sb & lanemask_lt())] = off + lane;
+    const unsigned lb = __ballot_sync(FULL, head && glen > kShortMax);  // <= 32 members: 1 block
+    int lbase = 0;
+    if (lane == 0 && lb) lbase = atomicAdd(&s.meta->nlong, __popc(lb));
+    lbase = __shfl_sync(FULL, lbase, 0);
+    if (head && glen > kShortMax) s.longlist[lbase + __popc(lb & lanemask_lt())] = off + lane;
     if (lane == 0) atomicAdd(&nseg[b < d.NBv ? 0 : 1], __popc(heads));
   }
   __syncthreads();
-  // phase 2: large buckets of this CTA's warps, by the whole CTA
-  for (int base = blockIdx.x * kSortWarps; base < d.NB; base += stride) {
-    for (int w = 0; w < kSortWarps && base + w < d.NB; ++w) {
-      const int b = base + w;
-      const int off = s.boff[b], len = s.boff[b + 1] - off;
-      if (len <= 32) continue;
-      const bool value = b < d.NBv;
-      const uint32_t gbase =
-          value ? ((uint32_t)b << d.vshift) : (uint32_t)d.N + (uint32_t)(b - d.NBv);
-      sort_big_bucket(s, off, len, value, gbase, buf, &nseg[value ? 0 : 1]);
-    }
+  // phase 2: the large buckets, each by the whole CTA
+  const int nbig = min(big_n, kSortWarps * 8);
+  for (int i = 0; i < nbig; ++i) {
+    const int b = big_b[i];
+    const int off = s.boff[b], len = s.boff[b + 1] - off;
+    const bool value = b < d.NBv;
+    const uint32_t gbase =
+        value ? ((uint32_t)b << d.vshift) : (uint32_t)d.N + (uint32_t)(b - d.NBv);
+    sort_big_bucket(s, off, len, value, gbase, buf, &nseg[value ? 0 : 1]);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -332,6 +396,8 @@ __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s)
   }
 }
 
+// Every CTA meets at most 8 buckets per warp (so big_b cannot overflow):
+// the grid holds at least NB / (8 * kSortWarps) CTAs.
 cudaError_t launch_bsort(const Dims &d, const Scratch &s, cudaStream_t st) {
   static int per_sm = 0;
   if (!per_sm) {
@@ -339,26 +405,30 @@ cudaError_t launch_bsort(const Dims &d, const Scratch &s, cudaStream_t st) {
     if (per_sm < 1) per_sm = 1;
   }
   int blocks = (d.NB + kSortWarps - 1) / kSortWarps;
-  if (blocks > d.sm_count * per_sm) blocks = d.sm_count * per_sm;
+  const int min_blocks = (d.NB + 8 * kSortWarps - 1) / (8 * kSortWarps);
+  int cap = d.sm_count * per_sm;
+  if (cap < min_blocks) cap = min_blocks;
+  if (blocks > cap) blocks = cap;
   k_bucket_sort<<<blocks, kSortThreads, 0, st>>>(d, s);
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// apply: every group is cut into blocks of kBlock members counted from the
-// group's first member; the warp that meets a block's first position sums the
-// block in order, loading a few source rows at a time (E rows for value rows,
-// query halves for sub-key rows) together with the target row.  A group of
-// one block is written at once.  A longer group publishes one partial per
-// block in a pool; the last block to arrive adds the partials in block order
-// and writes the row.  Work per warp is bounded by kBlock members whatever the
-// skew, and no sum depends on scheduling.
+// apply: the row updates, from the two work lists bsort wrote.
+//   phase A, one CTA per block of up to kBlock members of a longer group: the
+//     8 warps each take members m = w, w+8, w+16, w+24 and have all their
+//     source rows in flight at once (E rows for value rows, query halves for
+//     sub-key rows); the warps' sums are added in warp order.  A one-block
+//     group is written at once; otherwise the block publishes a partial and
+//     the last block of the group adds the partials in block order.
+//   phase B, one warp per group of <= kShortMax members: both source rows and
+//     the target row are loaded together, then the row is written.
+// Column blocks of 32 * Q4 float4 bound the registers for any row width.
+// Every sum runs in an order fixed by the data, whatever the scheduling.
 // ---------------------------------------------------------------------------
-constexpr int kApplyWarps = 8;
-constexpr int kBlock = 32;
+constexpr int kApplyThreads = 256;
+constexpr int kApplyWarps = kApplyThreads / 32;
 
-// Columns are processed in blocks of 32 * Q4 float4 (<= 512 floats), so the
-// registers a warp holds stay bounded for any row width.
 template <int Q4>
 __device__ __forceinline__ void load_row(const float *src, int cb, int n4, float4 (&r)[Q4]) {
   const int lane = threadIdx.x & 31;
@@ -370,229 +440,225 @@ __device__ __forceinline__ void load_row(const float *src, int cb, int n4, float
   }
 }
 
-template <int Q4>
-__device__ __forceinline__ void fma_row(float4 (&acc)[Q4], float c, const float4 (&r)[Q4]) {
-#pragma unroll
-  for (int q = 0; q < Q4; ++q) {
-    acc[q].x = fmaf(c, r[q].x, acc[q].x);
-    acc[q].y = fmaf(c, r[q].y, acc[q].y);
-    acc[q].z = fmaf(c, r[q].z, acc[q].z);
-    acc[q].w = fmaf(c, r[q].w, acc[q].w);
-  }
+__device__ __forceinline__ void fma4(float4 &a, float c, const float4 &x) {
+  a.x = fmaf(c, x.x, a.x);
+  a.y = fmaf(c, x.y, a.y);
+  a.z = fmaf(c, x.z, a.z);
+  a.w = fmaf(c, x.w, a.w);
+}
+__device__ __forceinline__ void add4(float4 &a, const float4 &x) {
+  a.x += x.x;
+  a.y += x.y;
+  a.z += x.z;
+  a.w += x.w;
 }
 
-// Row update (column block at cb) from a group's complete sum.
-template <int Q4>
-__device__ __forceinline__ void update_row(const Dims &d, bool value, float *dst, int cb,
-                                           int n4, const float4 (&row)[Q4],
-                                           const float4 (&acc)[Q4], float c0) {
-  const int lane = threadIdx.x & 31;
+// New value of one float4 of a target row from the group's complete sums.
+//   value row : v - (eta / C) * G          (C = sum of w/H)
+//   sub-key   : k - 2 eta (G - A k)        (A = sum of alpha)
+__device__ __forceinline__ float4 updated(const Dims &d, bool value, const float4 &t,
+                                          const float4 &g, float c0) {
   if (value) {
-    if (!(c0 > 0.f)) return;
-    const float scale = d.eta / c0;
-#pragma unroll
-    for (int q = 0; q < Q4; ++q) {
-      const int c4 = cb + lane + 32 * q;
-      if (c4 < n4) {
-        float4 v = row[q];
-        v.x -= scale * acc[q].x;
-        v.y -= scale * acc[q].y;
-        v.z -= scale * acc[q].z;
-        v.w -= scale * acc[q].w;
-        *reinterpret_cast<float4 *>(dst + 4 * c4) = v;
-      }
-    }
-  } else {
-    const float two_eta = 2.f * d.eta;
-#pragma unroll
-    for (int q = 0; q < Q4; ++q) {
-      const int c4 = cb + lane + 32 * q;
-      if (c4 < n4) {
-        float4 kv = row[q];
-        kv.x -= two_eta * (acc[q].x - c0 * kv.x);
-        kv.y -= two_eta * (acc[q].y - c0 * kv.y);
-        kv.z -= two_eta * (acc[q].z - c0 * kv.z);
-        kv.w -= two_eta * (acc[q].w - c0 * kv.w);
-        *reinterpret_cast<float4 *>(dst + 4 * c4) = kv;
-      }
-    }
+    const float sc = d.eta / c0;
+    return make_float4(t.x - sc * g.x, t.y - sc * g.y, t.z - sc * g.z, t.w - sc * g.w);
   }
+  const float te = 2.f * d.eta;
+  return make_float4(t.x - te * (g.x - c0 * t.x), t.y - te * (g.y - c0 * t.y),
+                     t.z - te * (g.z - c0 * t.z), t.w - te * (g.w - c0 * t.w));
 }
 
 // Entropy term of a value row: dL_addr/dw = (lam/M)(log pbar + 1) for every
 // pair of the group, pbar = (sum of the group's weights) / M.
-__device__ __forceinline__ void write_entropy_term(const Dims &d, const Scratch &s, float wsum,
-                                                   int g0, int len) {
-  const float pbar = wsum / (float)d.M;
-  const float bterm = (d.lam / (float)d.M) * (logf(pbar) + 1.f);
-  for (int x = g0 + (threadIdx.x & 31); x < g0 + len; x += 32) s.pb[s.rec[x].id] = bterm;
+__device__ __forceinline__ float entropy_term(const Dims &d, float wsum) {
+  return (d.lam / (float)d.M) * (logf(wsum / (float)d.M) + 1.f);
 }
 
-// Ordered sum over the block's members (member j's metadata in lane j),
-// column block cb, a few source rows in flight at a time.
-template <int Q4>
-__device__ __forceinline__ void sum_block(const Dims &d, const Scratch &s, bool value, int cnt,
-                                          int srow_l, float coef_l, int cb, int n4,
-                                          float4 (&acc)[Q4]) {
-  constexpr int kBatch = Q4 >= 4 ? 2 : 4;
-  const float *base = value ? s.E : s.Qs;
-  const int width = value ? d.dv : d.dh;
-#pragma unroll
-  for (int q = 0; q < Q4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j = 0; j < cnt; j += kBatch) {
-    float4 r[kBatch][Q4];
-    float cf[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int sr = __shfl_sync(FULL, srow_l, (j + u) & 31);
-      cf[u] = __shfl_sync(FULL, coef_l, (j + u) & 31);
-      if (j + u < cnt) load_row<Q4>(base + (int64_t)sr * width, cb, n4, r[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u)
-      if (j + u < cnt) fma_row<Q4>(acc, cf[u], r[u]);
-  }
-}
-
-// Last block of a long group: add the block partials in block order and
-// write the row (kept out of line so the common path keeps its registers).
-template <int Q4>
-__device__ __noinline__ void combine_partials(const Dims &d, const Scratch &s, bool value,
-                                              float *dst, int n4, int g0, int len,
-                                              int nblocks) {
-  constexpr int CB = 32 * Q4;
-  const int lane = threadIdx.x & 31;
-  float4 acc[Q4], row[Q4];
-  float C = 0.f, W = 0.f;
-  for (int b = 0; b < nblocks; ++b) {
-    const float *pp = s.partial + (size_t)__ldcg(&s.slotmap[g0 + b * kBlock]) * s.pwidth;
-    C += __ldcg(pp);
-    W += __ldcg(pp + 1);
-  }
-  for (int cb = 0; cb < n4; cb += CB) {
-    load_row<Q4>(dst, cb, n4, row);
-#pragma unroll
-    for (int q = 0; q < Q4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int b = 0; b < nblocks; b += 2) {
-      float4 pv[2][Q4];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        if (b + u < nblocks) {
-          const float *pp =
-              s.partial + (size_t)__ldcg(&s.slotmap[g0 + (b + u) * kBlock]) * s.pwidth;
-#pragma unroll
-          for (int q = 0; q < Q4; ++q) {
-            const int c4 = cb + lane + 32 * q;
-            pv[u][q] = c4 < n4 ? __ldcg(reinterpret_cast<const float4 *>(pp + 4 + 4 * c4))
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        if (b + u < nblocks) {
-#pragma unroll
-          for (int q = 0; q < Q4; ++q) {
-            acc[q].x += pv[u][q].x;
-            acc[q].y += pv[u][q].y;
-            acc[q].z += pv[u][q].z;
-            acc[q].w += pv[u][q].w;
-          }
-        }
-      }
-    }
-    update_row<Q4>(d, value, dst, cb, n4, row, acc, C);
-  }
-  if (value && d.lam != 0.f) write_entropy_term(d, s, W, g0, len);
+__device__ __forceinline__ const float *source_row(const Dims &d, const Scratch &s, bool value,
+                                                   int srow) {
+  return value ? s.E + (int64_t)srow * d.dv : s.Qs + (int64_t)srow * d.dh;
 }
 
 template <int Q4>
-__global__ void __launch_bounds__(kApplyWarps * 32) k_apply(Dims d, float *__restrict__ V,
-                                                            float *__restrict__ K, Scratch s,
-                                                            int part) {
-  constexpr int CB = 32 * Q4;  // float4 columns per block
-  const int lane = threadIdx.x & 31;
-  const int L = s.meta->L, Lv = s.meta->Lv;
-  const int lo = part == 2 ? Lv : 0;  // part 0: all, 1: value rows, 2: sub-key rows
-  const int hi = part == 1 ? Lv : L;
+__global__ void __launch_bounds__(kApplyThreads) k_apply(Dims d, float *__restrict__ V,
+                                                         float *__restrict__ K, Scratch s,
+                                                         int part) {
+  constexpr int CB = 32 * Q4;  // float4 columns per column block
+  __shared__ float4 red[kApplyWarps][CB];
+  __shared__ int m_srow[kBlock];
+  __shared__ float m_coef[kBlock], m_c0[kBlock], m_c1[kBlock];
+  __shared__ int m_id[kBlock];
+  __shared__ int s_slot, s_last;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool alpha_later = d.lam != 0.f;  // sub-key alphas come from pgrad
-  for (int x = lo + blockIdx.x * kApplyWarps + (threadIdx.x >> 5); x < hi;
-       x += gridDim.x * kApplyWarps) {
+  auto wanted = [&](uint32_t g) {         // part 0: all, 1: value rows, 2: sub-key rows
+    const bool value = g < (uint32_t)d.N;
+    return part == 0 || (part == 1) == value;
+  };
+
+  // ---------------- phase A: blocks of longer groups ----------------
+  const int nlong = s.meta->nlong;
+  for (int it = blockIdx.x; it < nlong; it += gridDim.x) {
+    const int x = s.longlist[it];
     const int4 head = *reinterpret_cast<const int4 *>(s.rec + x);  // g, id, srow, gstart
-    const int g0 = head.w;
-    if ((x - g0) % kBlock != 0) continue;  // not the first member of a block
-    const int len = s.rec[x].glen;
-    const int cnt = min(kBlock, g0 + len - x);
     const uint32_t g = (uint32_t)head.x;
+    if (!wanted(g)) continue;
+    const int g0 = head.w, len = s.rec[x].glen;
+    const int cnt = min(kBlock, g0 + len - x);
+    const int nblocks = (len + kBlock - 1) / kBlock;
     const bool value = g < (uint32_t)d.N;
     const int n4 = (value ? d.dv : d.dh) >> 2;
     float *dst = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.N) * d.dh;
-    // lane j: metadata of member x + j
-    int srow_l = 0;
-    float coef_l = 0.f, c0_l = 0.f, c1_l = 0.f;
-    if (lane < cnt) {
-      const Member m = load_member(s.rec + x + lane);
-      srow_l = m.srow;
-      coef_l = m.coef;
-      c0_l = m.c0;
-      c1_l = m.c1;
-      if (!value && alpha_later) {
-        coef_l = s.ealpha[m.id];
-        c0_l = coef_l;
-      }
+    if (tid < cnt) {
+      const Member m = load_member(s.rec + x + tid);
+      m_srow[tid] = m.srow;
+      m_id[tid] = (int)m.id;
+      float coef = m.coef, c0 = m.c0;
+      if (!value && alpha_later) coef = c0 = s.ealpha[m.id];
+      m_coef[tid] = coef;
+      m_c0[tid] = c0;
+      m_c1[tid] = m.c1;
     }
-    // ordered scalar sums over the block
-    float c0 = 0.f, c1 = 0.f;
+    if (tid == 0 && nblocks > 1) {
+      s_slot = atomicAdd(&s.meta->pool_next, 1);
+      if (s_slot >= s.pool_cap) atomicOr(&s.meta->err, ERR_POOL_OVERFLOW);
+    }
+    __syncthreads();
+    float C = 0.f, W = 0.f;  // ordered scalar sums of the block (same in every thread)
     for (int j = 0; j < cnt; ++j) {
-      c0 += __shfl_sync(FULL, c0_l, j);
-      c1 += __shfl_sync(FULL, c1_l, j);
+      C += m_c0[j];
+      W += m_c1[j];
     }
-    const bool whole = len <= kBlock;  // the whole group is in this block
-    float *p = nullptr;
-    if (!whole) {  // long group: this block's partial goes to a pool slot
-      int slot = 0;
-      if (lane == 0) slot = atomicAdd(&s.meta->pool_next, 1);
-      slot = __shfl_sync(FULL, slot, 0);
-      if (slot >= s.pool_cap) {  // cannot happen: the pool holds 2*Lcap/kBlock blocks
-        if (lane == 0) atomicOr(&s.meta->err, ERR_POOL_OVERFLOW);
-        continue;
-      }
-      p = s.partial + (size_t)slot * s.pwidth;
-      if (lane == 0) s.slotmap[x] = slot;
-    }
-    float4 acc[Q4], row[Q4];
+    const int slot = nblocks > 1 ? s_slot : 0;
+    const bool slot_ok = nblocks == 1 || slot < s.pool_cap;
+    float *part_out = s.partial + (size_t)slot * s.pwidth;
     for (int cb = 0; cb < n4; cb += CB) {
-      if (whole) load_row<Q4>(dst, cb, n4, row);  // in flight with the first sources
-      sum_block<Q4>(d, s, value, cnt, srow_l, coef_l, cb, n4, acc);
-      if (whole) {
-        update_row<Q4>(d, value, dst, cb, n4, row, acc, c0);
-      } else {
+      float4 r[4][Q4];
 #pragma unroll
-        for (int q = 0; q < Q4; ++q) {
-          const int c4 = cb + lane + 32 * q;
-          if (c4 < n4) *reinterpret_cast<float4 *>(p + 4 + 4 * c4) = acc[q];
+      for (int u = 0; u < 4; ++u) {
+        const int j = warp + kApplyWarps * u;
+        if (j < cnt) load_row<Q4>(source_row(d, s, value, m_srow[j]), cb, n4, r[u]);
+      }
+      float4 acc[Q4];
+#pragma unroll
+      for (int q = 0; q < Q4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = warp + kApplyWarps * u;
+        if (j < cnt) {
+#pragma unroll
+          for (int q = 0; q < Q4; ++q) fma4(acc[q], m_coef[j], r[u][q]);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < Q4; ++q) red[warp][lane + 32 * q] = acc[q];
+      __syncthreads();
+      if (tid < CB && cb + tid < n4) {
+        const int c4 = cb + tid;
+        float4 tot = red[0][tid];
+#pragma unroll
+        for (int w = 1; w < kApplyWarps; ++w) add4(tot, red[w][tid]);
+        if (nblocks == 1) {
+          if (!value || C > 0.f) {
+            const float4 t = *reinterpret_cast<const float4 *>(dst + 4 * c4);
+            *reinterpret_cast<float4 *>(dst + 4 * c4) = updated(d, value, t, tot, C);
+          }
+        } else if (slot_ok) {
+          *reinterpret_cast<float4 *>(part_out + 4 + 4 * c4) = tot;
+          __threadfence();  // visible before the group's arrival count moves
+        }
+      }
+      __syncthreads();
+    }
+    if (nblocks == 1) {
+      if (value && d.lam != 0.f && tid < cnt) s.pb[m_id[tid]] = entropy_term(d, W);
+      __syncthreads();
+      continue;
+    }
+    // longer group: publish the partial; the group's last block combines
+    if (tid == 0) {
+      if (slot_ok) {
+        part_out[0] = C;
+        part_out[1] = W;
+      }
+      s.slotmap[x] = slot_ok ? slot : -1;
+      __threadfence();
+      s_last = atomicAdd(&s.segcnt[g0], 1) == nblocks - 1;
+    }
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      float Ct = 0.f, Wt = 0.f;
+      bool all_ok = true;
+      for (int b = 0; b < nblocks; ++b) {
+        const int sl = __ldcg(&s.slotmap[g0 + b * kBlock]);
+        if (sl < 0) {
+          all_ok = false;
+          continue;
+        }
+        const float *pp = s.partial + (size_t)sl * s.pwidth;
+        Ct += __ldcg(pp);
+        Wt += __ldcg(pp + 1);
+      }
+      for (int c4 = tid; c4 < n4 && all_ok; c4 += blockDim.x) {
+        float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int b = 0; b < nblocks; ++b) {
+          const float *pp =
+              s.partial + (size_t)__ldcg(&s.slotmap[g0 + b * kBlock]) * s.pwidth;
+          add4(tot, __ldcg(reinterpret_cast<const float4 *>(pp + 4 + 4 * c4)));
+        }
+        if (!value || Ct > 0.f) {
+          const float4 t = *reinterpret_cast<const float4 *>(dst + 4 * c4);
+          *reinterpret_cast<float4 *>(dst + 4 * c4) = updated(d, value, t, tot, Ct);
+        }
+      }
+      if (value && d.lam != 0.f && all_ok) {
+        const float bt = entropy_term(d, Wt);
+        for (int j = tid; j < len; j += blockDim.x) s.pb[s.rec[g0 + j].id] = bt;
+      }
+      if (tid == 0) s.segcnt[g0] = 0;  // ready for the next chunk
+    }
+    __syncthreads();
+  }
+
+  // ---------------- phase B: groups of <= kShortMax members ----------------
+  const int nshort = s.meta->nshort;
+  for (int it = blockIdx.x * kApplyWarps + warp; it < nshort; it += gridDim.x * kApplyWarps) {
+    const int x = s.shortlist[it];
+    const Member m0 = load_member(s.rec + x);
+    if (!wanted(m0.g)) continue;
+    const bool value = m0.g < (uint32_t)d.N;
+    const int len = m0.glen;
+    Member m1 = m0;
+    if (len > 1) m1 = load_member(s.rec + x + 1);
+    float coef0 = m0.coef, coef1 = m1.coef, c00 = m0.c0, c01 = m1.c0;
+    if (!value && alpha_later) {
+      coef0 = c00 = s.ealpha[m0.id];
+      if (len > 1) coef1 = c01 = s.ealpha[m1.id];
+    }
+    const float C = len > 1 ? c00 + c01 : c00;
+    const float W = len > 1 ? m0.c1 + m1.c1 : m0.c1;
+    const int n4 = (value ? d.dv : d.dh) >> 2;
+    float *dst = value ? V + (int64_t)m0.g * d.dv : K + (int64_t)(m0.g - (uint32_t)d.N) * d.dh;
+    const float *s0 = source_row(d, s, value, m0.srow);
+    const float *s1 = source_row(d, s, value, m1.srow);
+    for (int cb = 0; cb < n4; cb += CB) {
+      float4 t[Q4], a[Q4], b[Q4];
+      load_row<Q4>(dst, cb, n4, t);
+      load_row<Q4>(s0, cb, n4, a);
+      if (len > 1) load_row<Q4>(s1, cb, n4, b);
+      if (value && !(C > 0.f)) continue;
+#pragma unroll
+      for (int q = 0; q < Q4; ++q) {
+        const int c4 = cb + lane + 32 * q;
+        if (c4 < n4) {
+          float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
+          fma4(g, coef0, a[q]);
+          if (len > 1) fma4(g, coef1, b[q]);
+          *reinterpret_cast<float4 *>(dst + 4 * c4) = updated(d, value, t[q], g, C);
         }
       }
     }
-    if (whole) {
-      if (value && d.lam != 0.f) write_entropy_term(d, s, c1, g0, len);
-      continue;
-    }
-    if (lane == 0) {
-      p[0] = c0;
-      p[1] = c1;
-    }
-    __threadfence();
-    __syncwarp();
-    const int nblocks = (len + kBlock - 1) / kBlock;
-    int old = 0;
-    if (lane == 0) old = atomicAdd(&s.segcnt[g0], 1);
-    old = __shfl_sync(FULL, old, 0);
-    if (old != nblocks - 1) continue;
-    // last block in: add the partials in block order
-    __threadfence();
-    combine_partials<Q4>(d, s, value, dst, n4, g0, len, nblocks);
-    if (lane == 0) s.segcnt[g0] = 0;  // ready for the next chunk
+    if (value && d.lam != 0.f && lane < len) s.pb[lane == 0 ? m0.id : m1.id] = entropy_term(d, W);
   }
 }
 
@@ -601,12 +667,10 @@ static cudaError_t launch_apply_t(const Dims &d, float *V, float *K, const Scrat
                                   cudaStream_t st, int part) {
   static int per_sm = 0;
   if (!per_sm) {
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_apply<Q4>, kApplyWarps * 32, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_apply<Q4>, kApplyThreads, 0);
     if (per_sm < 1) per_sm = 1;
   }
-  int64_t blocks = (s.Lcap + kApplyWarps - 1) / kApplyWarps;
-  if (blocks > (int64_t)d.sm_count * per_sm) blocks = (int64_t)d.sm_count * per_sm;
-  k_apply<Q4><<<(int)blocks, kApplyWarps * 32, 0, st>>>(d, V, K, s, part);
+  k_apply<Q4><<<d.sm_count * per_sm, kApplyThreads, 0, st>>>(d, V, K, s, part);
   return cudaGetLastError();
 }
 

@@ -26,10 +26,10 @@ constexpr size_t kReadSmemBudget = 200 * 1024;
 // Dynamic shared memory layout (bytes):
 //   [0, 16)            mbarrier
 //   [128, 128+R)       staged rows, R = H*k*dv*4 (staged variant only)
-//   then               e (dv floats), w (H*k floats), slot (H*k ints), a (H*k floats)
+//   then               e (dv floats), w, slot, a, dL/ds (H*k each)
 static size_t read_smem_bytes(const Dims &d, bool staged) {
   const size_t HK = (size_t)d.H * d.k;
-  return 128 + (staged ? HK * d.dv * 4 : 0) + (size_t)d.dv * 4 + HK * 12;
+  return 128 + (staged ? HK * d.dv * 4 : 0) + (size_t)d.dv * 4 + HK * 16;
 }
 
 template <typename TV, bool kStaged>
@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   float *w_s = e_s + dv;
   int *slot_s = reinterpret_cast<int *>(w_s + HK);
   float *a_s = reinterpret_cast<float *>(slot_s + HK);
+  float *dl_s = a_s + HK;
 
   const int row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -125,16 +126,23 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
       const float w = lane < d.k ? w_s[j] : 0.f;
       const float a = lane < d.k ? a_s[j] : 0.f;
       const float S = warp_sum(w * a);
-      const float dl = w * (a - S);
-      for (int half = 0; half < 2; ++half) {
-        const int64_t mh = ((int64_t)row * d.H + h) * 2 + half;
-        const int ecnt = s.ecount[mh];
-        for (int idx = 0; idx < ecnt; ++idx) {
-          const int64_t e = mh * d.k + idx;
-          const unsigned mask = s.emask[e];
-          const float sum = warp_sum(((mask >> lane) & 1u) ? dl : 0.f);
-          if (lane == 0) s.ealpha[e] = s.einv[e] * sum;
+      if (lane < d.k) dl_s[j] = w * (a - S);
+    }
+    __syncthreads();
+    // alpha of every entry of this row, one thread each
+    for (int x = tid; x < 2 * HK; x += blockDim.x) {
+      const int mh = x / d.k, idx = x % d.k;  // mh = h*2 + half
+      const int64_t mhg = (int64_t)row * 2 * d.H + mh;
+      if (idx < s.ecount[mhg]) {
+        const int64_t e = mhg * d.k + idx;
+        unsigned mask = s.emask[e];
+        const float *dl = dl_s + (mh >> 1) * d.k;
+        float sum = 0.f;
+        while (mask) {
+          sum += dl[__ffs(mask) - 1];
+          mask &= mask - 1;
         }
+        s.ealpha[e] = s.einv[e] * sum;
       }
     }
     __syncthreads();

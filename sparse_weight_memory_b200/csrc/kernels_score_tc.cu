@@ -16,7 +16,7 @@
 //
 // CTA = one 128-row x BN-column output tile of one (head, half); 4 warps.
 //   warp 0, one lane: TMA producer over k-blocks of 32 elements (128 bytes,
-//                     128-byte swizzle), kStages-deep ring;
+//                     128-byte swizzle), 3- to 5-deep ring;
 //   warp 1:           allocates the accumulator columns in tensor memory;
 //                     one lane issues the MMAs and commits each stage back;
 //   warps 0-3:        epilogue, one accumulator lane (= output row) per thread.
@@ -31,7 +31,11 @@ namespace fwpkm {
 
 constexpr int kTcRows = 128;      // M of every MMA (cta_group::1)
 constexpr int kTcKBlock = 32;     // fp32 elements per 128-byte swizzle row
-constexpr int kTcStages = 3;
+// Ring depth: as many 32-element k-blocks in flight as fit in ~200 KB.
+template <int BN>
+constexpr int tc_stages() {
+  return BN <= 32 ? 5 : (BN <= 64 ? 4 : 3);
+}
 
 // --- tcgen05 helpers (inline PTX, sm_100a) --------------------------------
 __device__ __forceinline__ void tmem_alloc(uint32_t *slot_smem, uint32_t ncols) {
@@ -117,7 +121,8 @@ struct TcSmem {
   static constexpr int kA = kTcRows * kTcKBlock * 4;  // 16 KiB per operand part
   static constexpr int kB = BN * kTcKBlock * 4;
   static constexpr int kStage = 2 * kA + 2 * kB;      // hi and lo of A and B
-  static constexpr int kBytes = kTcStages * kStage + 1024 /* align */ + 256 /* barriers */;
+  static constexpr int kStages = tc_stages<BN>();
+  static constexpr int kBytes = kStages * kStage + 1024 /* align */ + 256 /* barriers */;
   static_assert(kStage >= 4 * 32 * 33 * 4, "epilogue tile fits in stage 0");
 };
 
@@ -131,6 +136,7 @@ __global__ void __launch_bounds__(128, 1)
   constexpr uint32_t kCols = BN < 32 ? 32 : BN;  // tensor-memory columns (power of 2)
   unsigned char *smem =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  constexpr int kTcStages = L::kStages;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kTcStages * L::kStage);
   uint64_t *empty = full + kTcStages;
   uint64_t *done = empty + kTcStages;

@@ -10,17 +10,17 @@
 //
 // One warp per token-head.  Each lane holds n/32 squared distances of a half
 // in registers; an MSB-first bisection over the fp32 bit patterns (distances
-// are >= 0, so the bit order is the value order) finds the k-th smallest
-// distance; the k winners are sorted in registers (bitonic across lanes), and
-// a frontier merge (one pointer per half-1 rank) extracts the top-k of the
-// k*k grid in k rounds of a warp arg-max.
+// are >= 0, so the bit order is the value order) finds the k smallest, which
+// are compacted one per lane.  For the merge each lane holds one row of the
+// k*k candidate grid and the same bisection, over order-preserving keys of
+// the negated scores, picks the k best.
 #include <math_constants.h>
 
 #include "fwpkm_internal.cuh"
 
 namespace fwpkm {
 
-// Number of keys (distances) strictly below t across the warp.
+// Number of keys strictly below t across the warp.
 template <int NV>
 __device__ __forceinline__ int count_lt(const uint32_t (&key)[NV], uint32_t t) {
   int c = 0;
@@ -29,101 +29,131 @@ __device__ __forceinline__ int count_lt(const uint32_t (&key)[NV], uint32_t t) {
   return __reduce_add_sync(FULL, c);
 }
 
-// Top-k smallest of the row `drow[0..n)` (n <= 32*NV) under (distance asc,
-// index asc).  Lane r < k returns the r-th best (distance, index).
+// Marks the k smallest keys held across the warp (NV per lane; an unused
+// entry holds 0xffffffff and there are at least k used ones).  Equal keys at
+// the boundary are taken in increasing `tie` order (tie values are unique).
+// Returns this lane's selection as a bit mask over v.
+//
+// MSB-first bisection over the key bits: t grows one bit at a time while
+// fewer than k keys lie below it; it stops early once exactly k do.
 template <int NV>
-__device__ void half_topk(const float *__restrict__ drow, int n, int k, float &d_out,
-                          int &i_out, uint2 *wbuf) {
-  const int lane = threadIdx.x & 31;
-  uint32_t key[NV];
-#pragma unroll
-  for (int v = 0; v < NV; ++v) {
-    int idx = lane + 32 * v;
-    key[v] = idx < n ? __float_as_uint(drow[idx]) : 0xffffffffu;
-  }
-  // Range of the real keys (padding lanes hold the largest key and never win).
+__device__ uint32_t warp_select_smallest(const uint32_t (&key)[NV], const uint32_t (&tie)[NV],
+                                         int k) {
   uint32_t kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
   for (int v = 0; v < NV; ++v) {
-    if (lane + 32 * v < n) {
+    if (key[v] != 0xffffffffu) {
       kmin = min(kmin, key[v]);
       kmax = max(kmax, key[v]);
     }
   }
   kmin = __reduce_min_sync(FULL, kmin);
   kmax = __reduce_max_sync(FULL, kmax);
-
-  // kstar: the k-th smallest key, or `thr` with exactly k keys below it.
-  uint32_t kstar = kmin;
-  bool exact = false;
-  uint32_t thr = 0;
+  uint32_t kstar = kmin;  // the k-th smallest key unless `exact`
   if (kmin != kmax) {
     const int hb = 31 - __clz(kmin ^ kmax);
     kstar = kmin & ~((2u << hb) - 1u);  // common prefix; every key >= kstar
     for (int bit = hb; bit >= 0; --bit) {
       const uint32_t t = kstar | (1u << bit);
       const int c = count_lt<NV>(key, t);
-      if (c == k) {
-        exact = true;
-        thr = t;
-        break;
+      if (c == k) {  // exactly k keys below t: done, no tie to break
+        uint32_t sel = 0;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) sel |= (key[v] < t ? 1u : 0u) << v;
+        return sel;
       }
       if (c < k) kstar = t;
     }
   }
-  // Compact the winners into wbuf (warp-private) in index order.
-  int need_ties = 0;
-  if (!exact) need_ties = k - count_lt<NV>(key, kstar);
-  int base = 0, ties_seen = 0;
-  const unsigned lt = lanemask_lt();
+  uint32_t sel = 0, tied = 0;
 #pragma unroll
   for (int v = 0; v < NV; ++v) {
-    bool sel;
-    if (exact) {
-      sel = key[v] < thr;
-    } else {
-      const bool tie = key[v] == kstar;
-      const unsigned tb = __ballot_sync(FULL, tie);
-      const int rank = ties_seen + __popc(tb & lt);
-      ties_seen += __popc(tb);
-      sel = key[v] < kstar || (tie && rank < need_ties);
-    }
-    const unsigned sb = __ballot_sync(FULL, sel);
-    if (sel) wbuf[base + __popc(sb & lt)] = make_uint2(key[v], (uint32_t)(lane + 32 * v));
+    sel |= (key[v] < kstar ? 1u : 0u) << v;
+    tied |= (key[v] == kstar ? 1u : 0u) << v;
+  }
+  // the remaining places go to the tied keys with the smallest tie values
+  for (int need = k - __reduce_add_sync(FULL, __popc(sel)); need > 0; --need) {
+    uint32_t best = 0xffffffffu;
+#pragma unroll
+    for (int v = 0; v < NV; ++v)
+      if ((tied >> v) & 1u) best = min(best, tie[v]);
+    const uint32_t win = __reduce_min_sync(FULL, best);
+#pragma unroll
+    for (int v = 0; v < NV; ++v)
+      if (((tied >> v) & 1u) && tie[v] == win) {
+        sel |= 1u << v;
+        tied &= ~(1u << v);
+      }
+  }
+  return sel;
+}
+
+// Lane r < (number selected) receives the r-th selected entry, in (v, lane)
+// order: its value a[v], b[v] and its v.
+template <int NV>
+__device__ __forceinline__ void compact_selected(uint32_t sel, const uint32_t (&a)[NV],
+                                                 const uint32_t (&b)[NV], uint2 *wbuf,
+                                                 uint32_t &a_out, uint32_t &b_out,
+                                                 int &v_out, int &src_lane) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = lanemask_lt();
+  int base = 0;
+#pragma unroll
+  for (int v = 0; v < NV; ++v) {
+    const bool on = (sel >> v) & 1u;
+    const unsigned sb = __ballot_sync(FULL, on);
+    if (on) wbuf[base + __popc(sb & lt)] = make_uint2((uint32_t)(v << 5 | lane), 0u);
     base += __popc(sb);
   }
   __syncwarp();
-  uint32_t kk = 0xffffffffu, ki = 0xffffffffu;
-  if (lane < k) {
-    uint2 e = wbuf[lane];
-    kk = e.x;
-    ki = e.y;
-  }
+  const uint32_t where = lane < base ? wbuf[lane].x : 0u;
   __syncwarp();
-  // Bitonic sort of the 32 lanes by (key asc, index asc).
+  v_out = (int)(where >> 5);
+  src_lane = (int)(where & 31u);
+  // fetch the values from the lane that holds them (all lanes take part)
+  a_out = 0;
+  b_out = 0;
 #pragma unroll
-  for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      const uint32_t ok = __shfl_xor_sync(FULL, kk, stride);
-      const uint32_t oi = __shfl_xor_sync(FULL, ki, stride);
-      const bool up = (lane & size) == 0 || size == 32;
-      const bool lower = (lane & stride) == 0;
-      const bool mine_less = kk < ok || (kk == ok && ki < oi);
-      const bool keep = (lower == up) ? mine_less : !mine_less;
-      if (!keep) {
-        kk = ok;
-        ki = oi;
-      }
+  for (int v = 0; v < NV; ++v) {
+    const uint32_t av = __shfl_sync(FULL, a[v], src_lane);
+    const uint32_t bv = __shfl_sync(FULL, b[v], src_lane);
+    if (v == v_out) {
+      a_out = av;
+      b_out = bv;
     }
   }
+}
+
+// Order-preserving map of a float to an unsigned key (larger float, larger key).
+__device__ __forceinline__ uint32_t float_order(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Top-k smallest distances of one half row drow[0..n) (n <= 32*NV), ties by
+// index.  Lane r < k returns one winner (distance, index); order unspecified.
+template <int NV>
+__device__ __forceinline__ void half_topk(const float *__restrict__ drow, int n, int k,
+                                          float &d_out, int &i_out, uint2 *wbuf) {
+  const int lane = threadIdx.x & 31;
+  uint32_t key[NV], idx[NV];
+#pragma unroll
+  for (int v = 0; v < NV; ++v) {
+    const int i = lane + 32 * v;
+    key[v] = i < n ? __float_as_uint(drow[i]) : 0xffffffffu;  // d >= 0: bits order = value order
+    idx[v] = (uint32_t)i;
+  }
+  const uint32_t sel = warp_select_smallest<NV>(key, idx, k);
+  uint32_t kk, ii;
+  int v_out, src;
+  compact_selected<NV>(sel, key, idx, wbuf, kk, ii, v_out, src);
   d_out = __uint_as_float(kk);
-  i_out = (int)ki;
+  i_out = (int)ii;
 }
 
 // kSelectOnly: write only the selection record (x.rec_slots / x.rec_w); no
 // pair, entry or bucket outputs.
-template <int NV, bool kSelectOnly>
+template <int NV, int KV, bool kSelectOnly>
 __global__ void __launch_bounds__(128) k_topk(Dims d, Scratch s, Extras x) {
   __shared__ uint2 wbuf_all[4][32];
   const int lane = threadIdx.x & 31;
@@ -160,42 +190,38 @@ __global__ void __launch_bounds__(128) k_topk(Dims d, Scratch s, Extras x) {
     int ia, jb;
     half_topk<NV>(D1, n, k, da, ia, wbuf);
     half_topk<NV>(D2, n, k, db, jb, wbuf);
-    const float sa = -logf(eps + da);  // lane a: a-th best of half 1
-    const float sb = -logf(eps + db);  // lane b: b-th best of half 2
-    // Frontier merge: lane a (< k) walks its row (a, 0), (a, 1), ...
-    int ptr = 0;
-    for (int r = 0; r < k; ++r) {
-      const int src = ptr < 32 ? ptr : 31;
-      const float s2p = __shfl_sync(FULL, sb, src);
-      const int j2p = __shfl_sync(FULL, jb, src);
-      float cs = (lane < k && ptr < k) ? sa + s2p : -CUDART_INF_F;
-      int cslot = (lane < k && ptr < k) ? ia * n + j2p : 0x7fffffff;
-      int clane = lane;
+    const float sa = -logf(eps + da);  // lane a < k: one winner of half 1
+    const float sb = -logf(eps + db);  // lane b < k: one winner of half 2
+    // Lane a holds row a of the k x k candidate grid: s = sa + sb[b], slot =
+    // ia * n + jb[b]; the k best candidates (score desc, slot asc) are the
+    // k smallest keys of the negated scores, ties by slot.
+    uint32_t key[KV], slot[KV];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float os = __shfl_xor_sync(FULL, cs, o);
-        const int oslot = __shfl_xor_sync(FULL, cslot, o);
-        const int olane = __shfl_xor_sync(FULL, clane, o);
-        if (os > cs || (os == cs && oslot < cslot)) {
-          cs = os;
-          cslot = oslot;
-          clane = olane;
-        }
-      }
-      const int wptr = __shfl_sync(FULL, ptr, clane);
-      const float wd1 = __shfl_sync(FULL, da, clane);
-      const int wi = __shfl_sync(FULL, ia, clane);
-      const float wd2 = __shfl_sync(FULL, db, wptr);
-      const int wj = __shfl_sync(FULL, jb, wptr);
-      if (lane == r) {
-        s_r = cs;
-        slot_r = cslot;
-        i_r = wi;
-        j_r = wj;
-        d1_r = wd1;
-        d2_r = wd2;
-      }
-      if (lane == clane) ++ptr;
+    for (int b = 0; b < KV; ++b) {
+      const float s2 = __shfl_sync(FULL, sb, b);
+      const int j2 = __shfl_sync(FULL, jb, b);
+      const bool ok = lane < k && b < k;
+      key[b] = ok ? float_order(-(sa + s2)) : 0xffffffffu;
+      slot[b] = ok ? (uint32_t)(ia * n + j2) : 0xffffffffu;
+    }
+    const uint32_t sel = warp_select_smallest<KV>(key, slot, k);
+    uint32_t wkey, wslot;
+    int b_out, a_out;
+    compact_selected<KV>(sel, key, slot, wbuf, wkey, wslot, b_out, a_out);
+    // winner r (lane r): row a_out of half 1, column b_out of half 2
+    const float w_sa = __shfl_sync(FULL, sa, a_out);
+    const float w_sb = __shfl_sync(FULL, sb, b_out);
+    const float w_d1 = __shfl_sync(FULL, da, a_out);
+    const float w_d2 = __shfl_sync(FULL, db, b_out);
+    const int w_i = __shfl_sync(FULL, ia, a_out);
+    const int w_j = __shfl_sync(FULL, jb, b_out);
+    if (lane < k) {
+      s_r = w_sa + w_sb;
+      slot_r = (int)wslot;
+      i_r = w_i;
+      j_r = w_j;
+      d1_r = w_d1;
+      d2_r = w_d2;
     }
   }
 
@@ -244,20 +270,28 @@ __global__ void __launch_bounds__(128) k_topk(Dims d, Scratch s, Extras x) {
   }
 }
 
+template <int KV, bool kSelectOnly>
+static cudaError_t launch_topk_kv(const Dims &d, const Scratch &s, const Extras &x,
+                                  cudaStream_t st) {
+  const int blocks = (d.M + 3) / 4;
+  const int nv = (d.n + 31) / 32;
+  if (nv <= 1) k_topk<1, KV, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
+  else if (nv <= 2) k_topk<2, KV, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
+  else if (nv <= 4) k_topk<4, KV, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
+  else if (nv <= 8) k_topk<8, KV, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
+  else if (nv <= 16) k_topk<16, KV, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
+  else if (nv <= 32) k_topk<32, KV, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
+  else if (nv <= 64) k_topk<64, KV, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
 template <bool kSelectOnly>
 static cudaError_t launch_topk_t(const Dims &d, const Scratch &s, const Extras &x,
                                  cudaStream_t st) {
-  const int blocks = (d.M + 3) / 4;
-  const int nv = (d.n + 31) / 32;
-  if (nv <= 1) k_topk<1, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 2) k_topk<2, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 4) k_topk<4, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 8) k_topk<8, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 16) k_topk<16, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 32) k_topk<32, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 64) k_topk<64, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
-  else return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  if (d.k <= 8) return launch_topk_kv<8, kSelectOnly>(d, s, x, st);
+  if (d.k <= 16) return launch_topk_kv<16, kSelectOnly>(d, s, x, st);
+  return launch_topk_kv<32, kSelectOnly>(d, s, x, st);
 }
 
 cudaError_t launch_topk(const Dims &d, const Scratch &s, const Extras &x, cudaStream_t st) {
