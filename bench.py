@@ -25,7 +25,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -51,6 +50,31 @@ def describe(wl) -> str:
     return s
 
 
+def config_for(wl, world: int) -> dict:
+    """The `config` object both arms print for a workload."""
+    return {"workload": describe(wl), "parallelism": f"replicas{world}",
+            "l2": "flushed between steps (256 MiB write), tables reset untimed",
+            "tokens_per_step": wl.tokens_per_step}
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank number over the process group (identity when there
+    is no group).  Every rank must call it at the same point."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_step_per_rank: float, steps: int, world: int,
+                   total_ms_max: float) -> float:
+    """Units all ranks processed / the slowest rank's time (weak scaling)."""
+    return units_per_step_per_rank * steps * world / (total_ms_max / 1e3)
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -64,53 +88,71 @@ def peaks():
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Polls the GPU's SM clock and clock-event reasons through NVML (read
+    only) every few milliseconds while the timed region runs."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
+    # NVML clock-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown"}
+
+    def __init__(self, torch_device_index: int, period_s: float = 0.002):
+        self.dev = torch_device_index
+        self.period = period_s
+        self.samples = []
+        self.mx = None
+        self._stop = None
+        self._thread = None
+        self.error = None
+
+    def _handle(self, nv):
+        import torch
+        try:
+            p = torch.cuda.get_device_properties(self.dev)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.dev)
+
+    def _run(self, nv, h):
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((sm, bits))
+            except Exception as e:  # keep the timed region going
+                self.error = repr(e)
+                return
+            self._stop.wait(self.period)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except FileNotFoundError:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        except Exception as e:
+            self.error = repr(e)
+            return self
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._run, args=(nv, h), daemon=True)
+        self._thread.start()
         return self
 
     def __exit__(self, *a):
-        self.lines = []
-        if self.proc is not None:
-            time.sleep(0.25)
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
 
     def summary(self) -> dict:
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in getattr(self, "lines", []):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for name, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [x for x, _ in self.samples]
+        reasons = sorted({name for _, bits in self.samples
+                          for bit, name in self.REASONS.items() if bits & bit})
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.mx,
+               "reasons": reasons, "samples": len(sm), "source": "nvml"}
+        if self.error:
+            out["error"] = self.error
+        return out
 
 
 # ---------------------------------------------------------------------------
@@ -168,7 +210,7 @@ def run_reference(args, wl):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": describe(wl)},
+            "config": config_for(wl, args.gpus),
             "cpu_baseline": {"value": tok_s, "unit": UNIT, "cores": info[1], "kind": "oracle",
                              "sample": info[0]},
             "e2e": {"value": tok_s, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -189,13 +231,44 @@ def algorithmic_work(wl, tokens, value_rows, key_rows):
         "fwpkm_read": ("hbm", gather + tokens * wl.dv * in_b + tokens * wl.dv * 4),
         # read-modify-write of every touched value row and sub-key row
         "fwpkm_apply": ("hbm", 2 * value_rows * wl.dv * 4 + 2 * key_rows * (wl.dq // 2) * 4),
-        # q_half . K_row for every sub-key of both halves
-        "fwpkm_score": ("alu", 2.0 * tokens * wl.heads * wl.n * wl.dq),
+        # q_half . K_row for every sub-key of both halves (fp32 products)
+        "fwpkm_score": ("tensor", 2.0 * tokens * wl.heads * wl.n * wl.dq),
+        # distance matrix read once, slots + weights written
+        "fwpkm_topk": ("hbm", tokens * wl.heads * (2 * wl.n * 4 + wl.topk * 8)),
+        # queries read once, split into hi/lo halves + norms written
+        "fwpkm_prep": ("hbm", tokens * wl.heads * wl.dq * (in_b + 8) + tokens * wl.heads * 8),
     }
 
 
-# fp32 FMA peak of the SIMT pipes: 148 SMs x 128 lanes x 2 flops x 1.965 GHz
-SIMT_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
+# kernels as last captured with ncu on the library workload, keyed by kernel;
+# the capture and its command are summarised in profiles/.  None = no capture
+# of the current kernel.
+NCU_TRAFFIC = {"library": {}}
+
+
+def tensor_peak_tf32(bf16_tf):
+    """Dense tf32 tensor peak: the measured bf16 figure x the nominal ratio
+    1.1 / 2.25 PFLOP/s.  The score kernel issues three tf32 products per fp32
+    product (hi*hi + hi*lo + lo*hi), so its fp32-equivalent ceiling is a third
+    of this."""
+    return bf16_tf * 1.1 / 2.25
+
+
+def kernel_roofline(name, work, ms, launches, hbm_gbs, bf16_tf, peak_kind, traffic):
+    bound, amount = work
+    per_launch = amount / launches
+    sec = ms / launches / 1e3
+    if bound == "hbm":
+        achieved, peak, unit = per_launch / sec / 1e9, hbm_gbs, "GB/s"
+        note = f"{peak_kind} copy bandwidth"
+    else:
+        achieved, peak, unit = per_launch / sec / 1e12, tensor_peak_tf32(bf16_tf), "TFLOP/s"
+        note = (f"{peak_kind} bf16 x 1.1/2.25 (tf32); achieved counts fp32 products once, "
+                f"the 3xTF32 split issues 3 tf32 products each, so frac <= 1/3")
+    return {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": traffic,
+            "algorithmic_per_launch": per_launch, "us_per_launch": sec * 1e6, "peak_kind": note}
 
 
 def run_gpu(args, wl):
@@ -273,12 +346,9 @@ def run_gpu(args, wl):
     step_ms = [a.elapsed_time(b) for a, b in times]
     total_ms = sum(step_ms)
     stats = st.read_stats(reset=True)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms_max = float(t.item())
+    total_ms_max = max_over_ranks(total_ms, dev)
     tokens_per_step = wl.tokens_per_step
-    value = tokens_per_step * args.steps * world / (total_ms_max / 1e3)
+    value = whole_job_rate(tokens_per_step, args.steps, world, total_ms_max)
 
     # per-kernel event timing (separate, instrumented steps)
     st.set_profiling(True)
@@ -316,31 +386,25 @@ def run_gpu(args, wl):
         torch.cuda.synchronize()
         if i >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
-    te = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = tokens_per_step * args.steps * world / (float(te.item()) / 1e3)
+    e2e_value = whole_job_rate(tokens_per_step, args.steps, world,
+                               max_over_ranks(sum(e2e_ms), dev))
 
     if rank == 0:
         hbm_gbs, bf16_tf, peak_kind = peaks()
         rows_sum = wl.B * wl.T * wl.calls * wl.passes * prof_steps
         work = algorithmic_work(wl, rows_sum, pstats["value_rows"], pstats["key_rows"])
+        traffic = NCU_TRAFFIC.get(wl.name, {})
+        fracs = {k: kernel_roofline(k, work[k], ms, n, hbm_gbs, bf16_tf, peak_kind,
+                                    traffic.get(k))
+                 for k, (ms, n) in prof.items() if k in work and n > 0}
         dominant = max(prof.items(), key=lambda kv: kv[1][0])[0]
-        dom_ms, dom_n = prof[dominant]
-        roofline = None
-        if dominant in work and dom_n > 0:
-            bound, amount = work[dominant]
-            per_launch = amount / dom_n
-            sec = dom_ms / dom_n / 1e3
-            if bound == "hbm":
-                achieved, peak, unit = per_launch / sec / 1e9, hbm_gbs, "GB/s"
-            else:
-                achieved, peak, unit = per_launch / sec / 1e12, SIMT_FP32_TFLOPS, "TFLOP/s"
-            roofline = {"kernel": dominant, "bound": bound, "achieved": achieved,
-                        "peak": peak, "unit": unit, "frac": achieved / peak,
-                        "traffic": None,
-                        "peak_kind": peak_kind if bound == "hbm" else "derived: SM count x clock"}
-        kernels = {k: {"ms_per_step": v[0] / prof_steps, "launches_per_step": v[1] / prof_steps}
+        roofline = fracs.get(dominant)
+        if roofline is None:  # the longest kernel has no algorithmic-work model
+            roofline = {"kernel": dominant, "bound": None, "achieved": None, "peak": None,
+                        "unit": None, "frac": None, "traffic": None}
+        kernels = {k: {"ms_per_step": v[0] / prof_steps, "launches_per_step": v[1] / prof_steps,
+                       "share": v[0] / sum(x[0] for x in prof.values()),
+                       "frac": fracs[k]["frac"] if k in fracs else None}
                    for k, v in prof.items()}
         # whole-step roofline: gathered + scattered + streamed bytes at HBM peak
         vrows = stats["value_rows"] / args.steps
@@ -349,7 +413,8 @@ def run_gpu(args, wl):
         step_bytes = (tok * wl.heads * wl.topk * wl.dv * 4 + 2 * vrows * wl.dv * 4 +
                       tok * (wl.heads * wl.dq * in_b + wl.dv * in_b + 4 + wl.dv * 4))
         step_flops = 2.0 * tok * wl.heads * wl.n * wl.dq
-        t_roof = max(step_bytes / (hbm_gbs * 1e9), step_flops / (bf16_tf / 2 * 1e12))
+        t_roof = max(step_bytes / (hbm_gbs * 1e9),
+                     step_flops / (tensor_peak_tf32(bf16_tf) / 3 * 1e12))
         clocks = clk.summary()
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -361,9 +426,7 @@ def run_gpu(args, wl):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": describe(wl), "parallelism": f"replicas{world}",
-                       "l2": "flushed between steps (256 MiB write), tables reset untimed",
-                       "tokens_per_step": tokens_per_step},
+            "config": config_for(wl, world),
             "roofline": roofline,
             "step_roofline": {"bytes_per_step": step_bytes, "flops_per_step": step_flops,
                               "t_roof_ms": t_roof * 1e3,

@@ -378,6 +378,7 @@ fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtyp
     d.NBv = (int)value_buckets(st->N);
     d.NB = d.NBv + 2 * st->H * st->n;
     d.sm_count = st->sm_count;
+    d.pdl = st->profiling ? 0 : 1;  // per-kernel events need plain stream order
     d.eps = st->eps;
     d.eta = eta;
     d.lam = lambda_entropy;

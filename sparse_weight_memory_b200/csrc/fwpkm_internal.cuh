@@ -59,6 +59,7 @@ struct Dims {
   int vshift;
   int NB;             // NBv value buckets + 2*H*n sub-key rows
   int sm_count;       // multiprocessors of the device (grid sizing)
+  int pdl;            // launch with programmatic dependent launch (see launch_k)
   float eps, eta, lam;
 };
 
@@ -202,6 +203,35 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
           "r"(smem_u32(dst_smem)),
       "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Programmatic dependent launch.  A kernel started by launch_k with d.pdl set
+// may become resident while its predecessor on the stream is still running;
+// griddep_wait() blocks until that predecessor has completed and its writes
+// are visible, so every kernel calls it before its first global-memory access
+// (and griddep_launch() right after, letting its own successor get scheduled
+// early).  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t st, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 // ------------------------------------------------------------------------

@@ -142,6 +142,7 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
     d.qstride = rows_max;
     d.M = d.rows * v.H;
     d.sm_count = v.sm_count;
+    d.pdl = 1;
     d.eps = v.eps;
     cudaError_t ke = launch_prep(d, Q, q_dtype, v.K, s, stream);
     if (ke == cudaSuccess) ke = launch_score(d, s, maps, stream);

@@ -59,6 +59,8 @@ constexpr int kScanThreads = 1024;
 constexpr int kScanPiece = 8192;
 
 __global__ void __launch_bounds__(kScanThreads) k_bucket_scan(Dims d, Scratch s) {
+  griddep_wait();
+  griddep_launch();
   __shared__ __align__(16) int cnt[kScanPiece];
   __shared__ int red[32];
   __shared__ int carry_s;
@@ -134,8 +136,7 @@ __global__ void __launch_bounds__(kScanThreads) k_bucket_scan(Dims d, Scratch s)
 }
 
 cudaError_t launch_scan(const Dims &d, const Scratch &s, cudaStream_t st) {
-  k_bucket_scan<<<1, kScanThreads, 0, st>>>(d, s);
-  return cudaGetLastError();
+  return launch_k(d.pdl, k_bucket_scan, 1, kScanThreads, 0, st, d, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -302,6 +303,8 @@ __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s)
   __shared__ int nseg[2];  // distinct value rows / sub-key rows seen by this CTA
   __shared__ int big_n;
   __shared__ int big_b[kSortWarps * 8];  // large buckets met in phase 1
+  griddep_wait();
+  griddep_launch();
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   if (threadIdx.x < 2) nseg[threadIdx.x] = 0;
   if (threadIdx.x == 0) big_n = 0;
@@ -409,8 +412,7 @@ cudaError_t launch_bsort(const Dims &d, const Scratch &s, cudaStream_t st) {
   int cap = d.sm_count * per_sm;
   if (cap < min_blocks) cap = min_blocks;
   if (blocks > cap) blocks = cap;
-  k_bucket_sort<<<blocks, kSortThreads, 0, st>>>(d, s);
-  return cudaGetLastError();
+  return launch_k(d.pdl, k_bucket_sort, blocks, kSortThreads, 0, st, d, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -488,6 +490,8 @@ __global__ void __launch_bounds__(kApplyThreads) k_apply(Dims d, float *__restri
   __shared__ float m_coef[kBlock], m_c0[kBlock], m_c1[kBlock];
   __shared__ int m_id[kBlock];
   __shared__ int s_slot, s_last;
+  griddep_wait();
+  griddep_launch();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool alpha_later = d.lam != 0.f;  // sub-key alphas come from pgrad
   auto wanted = [&](uint32_t g) {         // part 0: all, 1: value rows, 2: sub-key rows
@@ -670,8 +674,8 @@ static cudaError_t launch_apply_t(const Dims &d, float *V, float *K, const Scrat
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_apply<Q4>, kApplyThreads, 0);
     if (per_sm < 1) per_sm = 1;
   }
-  k_apply<Q4><<<d.sm_count * per_sm, kApplyThreads, 0, st>>>(d, V, K, s, part);
-  return cudaGetLastError();
+  return launch_k(d.pdl, k_apply<Q4>, d.sm_count * per_sm, kApplyThreads, 0, st, d, V, K, s,
+                  part);
 }
 
 cudaError_t launch_apply(const Dims &d, float *V, float *K, const Scratch &s, cudaStream_t st,
@@ -688,6 +692,8 @@ cudaError_t launch_apply(const Dims &d, float *V, float *K, const Scratch &s, cu
 // Warp per token-head, lane r.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_pgrad(Dims d, Scratch s) {
+  griddep_wait();
+  griddep_launch();
   const int lane = threadIdx.x & 31;
   const int m = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (m >= d.M) return;
@@ -713,8 +719,7 @@ __global__ void __launch_bounds__(256) k_pgrad(Dims d, Scratch s) {
 }
 
 cudaError_t launch_pgrad(const Dims &d, const Scratch &s, cudaStream_t st) {
-  k_pgrad<<<(d.M + 7) / 8, 256, 0, st>>>(d, s);
-  return cudaGetLastError();
+  return launch_k(d.pdl, k_pgrad, (d.M + 7) / 8, 256, 0, st, d, s);
 }
 
 }  // namespace fwpkm

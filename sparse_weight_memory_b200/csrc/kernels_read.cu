@@ -37,6 +37,8 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
                                                        const TV *__restrict__ Vt,
                                                        const float *__restrict__ gate,
                                                        float *__restrict__ out, Scratch s) {
+  griddep_wait();
+  griddep_launch();
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
   const int HK = d.H * d.k, dv = d.dv, dv4 = dv >> 2;
@@ -193,13 +195,14 @@ static cudaError_t launch_read_t(const Dims &d, const float *V, const TV *Vt, co
   if (staged) {
     cudaFuncSetAttribute(k_read<TV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
-    k_read<TV, true><<<d.rows, kReadThreads, smem, st>>>(d, V, Vt, gate, out, s);
+    return launch_k(d.pdl, k_read<TV, true>, d.rows, kReadThreads, smem, st, d, V, Vt, gate,
+                    out, s);
   } else {
     cudaFuncSetAttribute(k_read<TV, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
-    k_read<TV, false><<<d.rows, kReadThreads, smem, st>>>(d, V, Vt, gate, out, s);
+    return launch_k(d.pdl, k_read<TV, false>, d.rows, kReadThreads, smem, st, d, V, Vt, gate,
+                    out, s);
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_read(const Dims &d, const float *V, const void *Vt, int v_dtype,

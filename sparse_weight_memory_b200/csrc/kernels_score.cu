@@ -32,6 +32,8 @@ __device__ __forceinline__ void split_store(float *hi, float *lo, int c, const f
 template <typename TQ>
 __global__ void __launch_bounds__(256) k_prep(Dims d, const TQ *__restrict__ Q,
                                               const float *__restrict__ K, Scratch s) {
+  griddep_wait();
+  griddep_launch();
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nq = (int64_t)2 * d.H * d.rows;
@@ -79,10 +81,9 @@ cudaError_t launch_prep(const Dims &d, const void *Q, int q_dtype, const float *
   const int64_t warps = (int64_t)2 * d.H * d.rows + (int64_t)2 * d.H * d.n;
   const int blocks = (int)((warps + 7) / 8);
   if (q_dtype == 1)
-    k_prep<__nv_bfloat16><<<blocks, 256, 0, st>>>(d, (const __nv_bfloat16 *)Q, K, s);
-  else
-    k_prep<float><<<blocks, 256, 0, st>>>(d, (const float *)Q, K, s);
-  return cudaGetLastError();
+    return launch_k(d.pdl, k_prep<__nv_bfloat16>, blocks, 256, 0, st, d,
+                    (const __nv_bfloat16 *)Q, K, s);
+  return launch_k(d.pdl, k_prep<float>, blocks, 256, 0, st, d, (const float *)Q, K, s);
 }
 
 }  // namespace fwpkm

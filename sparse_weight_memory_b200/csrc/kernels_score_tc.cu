@@ -161,6 +161,8 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();
+  griddep_launch();
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer ----------------
@@ -257,11 +259,11 @@ static cudaError_t launch_tc(const Dims &d, const Scratch &s, const TcMaps &maps
     attr = true;
   }
   dim3 grid((d.n + BN - 1) / BN, (d.rows + kTcRows - 1) / kTcRows, 2 * d.H);
-  k_score_tc<BN><<<grid, 128, TcSmem<BN>::kBytes, st>>>(
-      *reinterpret_cast<const CUtensorMap *>(maps.a_hi), *reinterpret_cast<const CUtensorMap *>(maps.a_lo),
-      *reinterpret_cast<const CUtensorMap *>(maps.b_hi[v]),
-      *reinterpret_cast<const CUtensorMap *>(maps.b_lo[v]), d, s);
-  return cudaGetLastError();
+  return launch_k(d.pdl, k_score_tc<BN>, grid, 128, TcSmem<BN>::kBytes, st,
+                  *reinterpret_cast<const CUtensorMap *>(maps.a_hi),
+                  *reinterpret_cast<const CUtensorMap *>(maps.a_lo),
+                  *reinterpret_cast<const CUtensorMap *>(maps.b_hi[v]),
+                  *reinterpret_cast<const CUtensorMap *>(maps.b_lo[v]), d, s);
 }
 
 // Column-tile width: the widest of 128 / 64 / 32 / 16 that still gives at

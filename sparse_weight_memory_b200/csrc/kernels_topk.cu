@@ -159,6 +159,8 @@ __global__ void __launch_bounds__(128) k_topk(Dims d, Scratch s, Extras x) {
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
   const int m = blockIdx.x * 4 + wib;  // token-head m = row*H + h
+  griddep_wait();
+  griddep_launch();
   if (m >= d.M) return;
   const int row = m / d.H, h = m % d.H;
   const int k = d.k, n = d.n;
@@ -275,15 +277,14 @@ static cudaError_t launch_topk_kv(const Dims &d, const Scratch &s, const Extras 
                                   cudaStream_t st) {
   const int blocks = (d.M + 3) / 4;
   const int nv = (d.n + 31) / 32;
-  if (nv <= 1) k_topk<1, KV, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 2) k_topk<2, KV, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 4) k_topk<4, KV, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 8) k_topk<8, KV, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 16) k_topk<16, KV, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 32) k_topk<32, KV, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
-  else if (nv <= 64) k_topk<64, KV, kSelectOnly><<<blocks, 128, 0, st>>>(d, s, x);
-  else return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  if (nv <= 1) return launch_k(d.pdl, k_topk<1, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
+  if (nv <= 2) return launch_k(d.pdl, k_topk<2, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
+  if (nv <= 4) return launch_k(d.pdl, k_topk<4, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
+  if (nv <= 8) return launch_k(d.pdl, k_topk<8, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
+  if (nv <= 16) return launch_k(d.pdl, k_topk<16, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
+  if (nv <= 32) return launch_k(d.pdl, k_topk<32, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
+  if (nv <= 64) return launch_k(d.pdl, k_topk<64, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
+  return cudaErrorInvalidValue;
 }
 
 template <bool kSelectOnly>

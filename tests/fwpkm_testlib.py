@@ -63,8 +63,11 @@ class RunResult:
     touched: Optional[int] = None
 
 
-def oracle_run(wl: Workload, inp: Inputs, oracle, max_chunks: int = 0) -> RunResult:
-    st = oracle.State(inp.subkeys, inp.values, topk=wl.topk, chunk=wl.chunk, eps=wl.eps)
+def oracle_run(wl: Workload, inp: Inputs, oracle, max_chunks: int = 0,
+               state=None) -> RunResult:
+    """Oracle over the workload's calls; continues `state` in place if given."""
+    st = state if state is not None else oracle.State(inp.subkeys, inp.values, topk=wl.topk,
+                                                      chunk=wl.chunk, eps=wl.eps)
     outs, sels, ws, gaps, touched = [], [], [], [], 0
     for Q, Vt, g in schedule(wl, inp):
         r = st.step(widen(Q), widen(Vt), g, wl.eta, wl.lam, want_sel=True, want_gap=True,
@@ -74,7 +77,8 @@ def oracle_run(wl: Workload, inp: Inputs, oracle, max_chunks: int = 0) -> RunRes
         ws.append(r["sel_w"])
         gaps.append(r["gap"])
         touched += int(r["touched"].sum())
-    return RunResult(outs, sels, ws, gaps, st.K, st.V, touched)
+    K, V = (st.K.copy(), st.V.copy()) if state is not None else (st.K, st.V)
+    return RunResult(outs, sels, ws, gaps, K, V, touched)
 
 
 def gpu_run(wl: Workload, inp: Inputs, ref: Optional[RunResult] = None, force: bool = True,
