@@ -457,8 +457,13 @@ def main():
                     help="seconds of oracle time per reference sample (one step, or "
                          "a prefix of it when one step takes longer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="tokens per sequence and call (default: the workload's T); a "
+                         "shorter run of the same shape, for profiler captures")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
+    if args.tokens:
+        wl = wl.replace(T=args.tokens)
     if args.impl == "reference":
         run_reference(args, wl)
     else:

@@ -79,14 +79,20 @@ namespace {
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Value rows are bucketed by slot >> vshift, at most 8192 buckets.
-int value_shift(int64_t N) {
+// Value rows are bucketed by slot >> vshift.  The bucket count follows the
+// chunk's pair capacity P: at least 8192 buckets (a few slots each, so rows
+// that many pairs share rarely meet in one bucket), more for large chunks
+// (about four pairs per bucket without skew), at most 65536 and never more
+// than N.  A bucket is then usually small enough for one warp to sort.
+int value_shift(int64_t N, int64_t P) {
+  int64_t target = 8192;
+  while (target < P / 4 && target < 65536) target <<= 1;
   int sh = 0;
-  while (((N + (1ll << sh) - 1) >> sh) > 8192) ++sh;
+  while (sh < 40 && ((N + (1ll << sh) - 1) >> sh) > target) ++sh;
   return sh;
 }
-int64_t value_buckets(int64_t N) {
-  const int sh = value_shift(N);
+int64_t value_buckets(int64_t N, int64_t P) {
+  const int sh = value_shift(N, P);
   return (N + (1ll << sh) - 1) >> sh;
 }
 
@@ -95,7 +101,7 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
   if (rows <= st->cap_rows) return FWPKM_OK;
   rows = (rows + 127) / 128 * 128;  // query-half stride: whole 128-row score tiles
   const int64_t H = st->H, n = st->n, dh = st->dh, dv = st->dv, k = st->k;
-  const int64_t M = rows * H, P = M * k, NB = value_buckets(st->N) + 2 * H * n;
+  const int64_t M = rows * H, P = M * k, NB = value_buckets(st->N, P) + 2 * H * n;
   const int64_t Lcap = 3 * P;  // pairs + at most 2 entries per pair
   const int64_t pool_cap = 2 * Lcap / 32 + 2;  // long-group blocks of 32 members
   const int pwidth = 4 + (int)(dv > dh ? dv : dh);
@@ -374,8 +380,9 @@ fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtyp
     d.rows = B * d.Tc;
     d.qstride = (int)st->cap_rows;
     d.M = d.rows * st->H;
-    d.vshift = value_shift(st->N);
-    d.NBv = (int)value_buckets(st->N);
+    const int64_t cap_pairs = st->cap_rows * st->H * st->k;  // bcnt was sized for this
+    d.vshift = value_shift(st->N, cap_pairs);
+    d.NBv = (int)value_buckets(st->N, cap_pairs);
     d.NB = d.NBv + 2 * st->H * st->n;
     d.sm_count = st->sm_count;
     d.pdl = st->profiling ? 0 : 1;  // per-kernel events need plain stream order

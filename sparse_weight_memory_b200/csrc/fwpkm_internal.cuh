@@ -91,7 +91,7 @@ struct Scratch {
   uint64_t *sort_tmp;  // [2*Lcap] merge buffers for oversized buckets
   int32_t *posmap;  // [Lcap]  position inside its bucket, by member id (oversized buckets)
   int32_t *slotmap; // [Lcap]  partial-pool slot of the block starting here
-  int32_t *shortlist;  // [Lcap] first position of every group of <= 2 members
+  int32_t *shortlist;  // [Lcap] first position of every group of <= 32 members
   int32_t *longlist;   // [Lcap] first position of every 32-member block of longer groups
   float *partial;   // [pool_cap][pwidth] block partial sums of long groups
   int32_t *segcnt;  // [Lcap] arrived blocks per long group, at its first position
@@ -218,20 +218,39 @@ __device__ __forceinline__ void griddep_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Launch with optional programmatic dependent launch and a thread-block
+// cluster of `cluster` CTAs along x (1 = no cluster).
 template <typename... KArgs, typename... Args>
-cudaError_t launch_k(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                     cudaStream_t st, Args &&...args) {
+cudaError_t launch_kc(bool pdl, int cluster, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                      size_t smem, cudaStream_t st, Args &&...args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  unsigned na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (cluster > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = (unsigned)cluster;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t st, Args &&...args) {
+  return launch_kc(pdl, 1, kernel, grid, block, smem, st, static_cast<Args &&>(args)...);
 }
 
 // ------------------------------------------------------------------------

@@ -187,7 +187,17 @@ __device__ __forceinline__ int lower_rank(const uint64_t *r, int len, uint64_t k
   return lo;
 }
 
-constexpr int kShortMax = 2;  // groups up to this size are applied by one warp
+// A record on its way from rec_in to rec.  When the entropy term is off the
+// read kernel has already computed every entry's alpha (ealpha): it becomes
+// the sub-key record's coefficient here.  With the term on, alpha is known
+// only after pgrad and the apply reads it itself.
+__device__ __forceinline__ Member fetch_member(const Dims &d, const Scratch &s, const Member *p) {
+  Member m = load_member(p);
+  if (d.lam == 0.f && m.g >= (uint32_t)d.N) m.coef = m.c0 = s.ealpha[m.id];
+  return m;
+}
+
+constexpr int kShortMax = 32;  // groups up to this size are applied by one warp
 constexpr int kBlock = 32;    // longer groups are applied in blocks of this many members
 
 // Work lists of the apply kernel for a group that starts at position x0:
@@ -204,8 +214,8 @@ __device__ __forceinline__ void list_group(const Scratch &s, int x0, int len) {
 }
 
 // CTA-wide sort of one bucket with more than 32 members.
-__device__ void sort_big_bucket(const Scratch &s, int off, int len, bool value, uint32_t gbase,
-                                uint64_t *buf, int *nseg) {
+__device__ void sort_big_bucket(const Dims &d, const Scratch &s, int off, int len, bool value,
+                                uint32_t gbase, uint64_t *buf, int *nseg) {
   int my_seg = 0;
   if (len <= kSortCap) {
     // key = (g - gbase) << 43 | id << 12 | local index   (g - gbase < 2^21, id < 2^31)
@@ -227,7 +237,7 @@ __device__ void sort_big_bucket(const Scratch &s, int off, int len, bool value, 
       const uint64_t grp = kv >> 43;
       const int first = lower_rank(buf, len, grp << 43);
       const int end = lower_rank(buf, len, (grp + 1) << 43);
-      Member m = load_member(s.rec_in + off + (int)(kv & 4095u));
+      Member m = fetch_member(d, s, s.rec_in + off + (int)(kv & 4095u));
       m.gstart = off + first;
       m.glen = end - first;
       store_member(s.rec + off + i, m);
@@ -284,7 +294,7 @@ __device__ void sort_big_bucket(const Scratch &s, int off, int len, bool value, 
       const uint64_t grp = kv >> 32;
       const int first = lower_rank(src, len, grp << 32);
       const int end = lower_rank(src, len, (grp + 1) << 32);
-      Member m = load_member(s.rec_in + off + s.posmap[pbase + (int)(uint32_t)kv]);
+      Member m = fetch_member(d, s, s.rec_in + off + s.posmap[pbase + (int)(uint32_t)kv]);
       m.gstart = off + first;
       m.glen = end - first;
       store_member(s.rec + off + i, m);
@@ -327,7 +337,7 @@ __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s)
     Member m{};
     uint64_t key = ~0ull;
     if (lane < len) {
-      m = load_member(s.rec_in + off + lane);
+      m = fetch_member(d, s, s.rec_in + off + lane);
       key = ((uint64_t)m.g << 32) | m.id;
     }
     // bitonic sort of (key, source lane) across the warp
@@ -390,7 +400,7 @@ __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s)
     const bool value = b < d.NBv;
     const uint32_t gbase =
         value ? ((uint32_t)b << d.vshift) : (uint32_t)d.N + (uint32_t)(b - d.NBv);
-    sort_big_bucket(s, off, len, value, gbase, buf, &nseg[value ? 0 : 1]);
+    sort_big_bucket(d, s, off, len, value, gbase, buf, &nseg[value ? 0 : 1]);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -423,8 +433,9 @@ cudaError_t launch_bsort(const Dims &d, const Scratch &s, cudaStream_t st) {
 //     sub-key rows); the warps' sums are added in warp order.  A one-block
 //     group is written at once; otherwise the block publishes a partial and
 //     the last block of the group adds the partials in block order.
-//   phase B, one warp per group of <= kShortMax members: both source rows and
-//     the target row are loaded together, then the row is written.
+//   phase B, one warp per group of <= kShortMax members: the lanes hold the
+//     records, the members' source rows are summed in member order with a
+//     few rows in flight, then the row is written.
 // Column blocks of 32 * Q4 float4 bound the registers for any row width.
 // Every sum runs in an order fixed by the data, whatever the scheduling.
 // ---------------------------------------------------------------------------
@@ -481,7 +492,7 @@ __device__ __forceinline__ const float *source_row(const Dims &d, const Scratch 
 }
 
 template <int Q4>
-__global__ void __launch_bounds__(kApplyThreads) k_apply(Dims d, float *__restrict__ V,
+__global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__restrict__ V,
                                                          float *__restrict__ K, Scratch s,
                                                          int part) {
   constexpr int CB = 32 * Q4;  // float4 columns per column block
@@ -624,45 +635,64 @@ __global__ void __launch_bounds__(kApplyThreads) k_apply(Dims d, float *__restri
     __syncthreads();
   }
 
-  // ---------------- phase B: groups of <= kShortMax members ----------------
+  // ---------------- phase B: groups of <= kShortMax members, a warp each ----------------
+  // Lane j holds member j's record; the members' rows are summed in member
+  // order, kU rows in flight, for every column block of the target row.
+  constexpr int kU = 4;
   const int nshort = s.meta->nshort;
   for (int it = blockIdx.x * kApplyWarps + warp; it < nshort; it += gridDim.x * kApplyWarps) {
     const int x = s.shortlist[it];
-    const Member m0 = load_member(s.rec + x);
-    if (!wanted(m0.g)) continue;
-    const bool value = m0.g < (uint32_t)d.N;
-    const int len = m0.glen;
-    Member m1 = m0;
-    if (len > 1) m1 = load_member(s.rec + x + 1);
-    float coef0 = m0.coef, coef1 = m1.coef, c00 = m0.c0, c01 = m1.c0;
-    if (!value && alpha_later) {
-      coef0 = c00 = s.ealpha[m0.id];
-      if (len > 1) coef1 = c01 = s.ealpha[m1.id];
+    Member mj{};
+    if ((int64_t)x + lane < s.Lcap) mj = load_member(s.rec + x + lane);  // past the group: unused
+    const uint32_t g = __shfl_sync(FULL, mj.g, 0);
+    const int len = __shfl_sync(FULL, mj.glen, 0);
+    if (!wanted(g)) continue;
+    const bool value = g < (uint32_t)d.N;
+    float coef = 0.f, c0 = 0.f, c1 = 0.f;
+    if (lane < len) {
+      coef = mj.coef;
+      c0 = mj.c0;
+      c1 = mj.c1;
+      if (!value && alpha_later) coef = c0 = s.ealpha[mj.id];
     }
-    const float C = len > 1 ? c00 + c01 : c00;
-    const float W = len > 1 ? m0.c1 + m1.c1 : m0.c1;
+    // butterfly sums: every lane ends with the same value, in a fixed order
+    float C = c0, W = c1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      C += __shfl_xor_sync(FULL, C, o);
+      W += __shfl_xor_sync(FULL, W, o);
+    }
     const int n4 = (value ? d.dv : d.dh) >> 2;
-    float *dst = value ? V + (int64_t)m0.g * d.dv : K + (int64_t)(m0.g - (uint32_t)d.N) * d.dh;
-    const float *s0 = source_row(d, s, value, m0.srow);
-    const float *s1 = source_row(d, s, value, m1.srow);
-    for (int cb = 0; cb < n4; cb += CB) {
-      float4 t[Q4], a[Q4], b[Q4];
+    float *dst = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.N) * d.dh;
+    const bool write = !value || C > 0.f;
+    for (int cb = 0; cb < n4 && write; cb += CB) {
+      float4 t[Q4], acc[Q4];
       load_row<Q4>(dst, cb, n4, t);
-      load_row<Q4>(s0, cb, n4, a);
-      if (len > 1) load_row<Q4>(s1, cb, n4, b);
-      if (value && !(C > 0.f)) continue;
+#pragma unroll
+      for (int q = 0; q < Q4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j0 = 0; j0 < len; j0 += kU) {
+        float4 r[kU][Q4];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int sr = __shfl_sync(FULL, mj.srow, (j0 + u) & 31);
+          if (j0 + u < len) load_row<Q4>(source_row(d, s, value, sr), cb, n4, r[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const float cj = __shfl_sync(FULL, coef, (j0 + u) & 31);
+          if (j0 + u < len) {
+#pragma unroll
+            for (int q = 0; q < Q4; ++q) fma4(acc[q], cj, r[u][q]);
+          }
+        }
+      }
 #pragma unroll
       for (int q = 0; q < Q4; ++q) {
         const int c4 = cb + lane + 32 * q;
-        if (c4 < n4) {
-          float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
-          fma4(g, coef0, a[q]);
-          if (len > 1) fma4(g, coef1, b[q]);
-          *reinterpret_cast<float4 *>(dst + 4 * c4) = updated(d, value, t[q], g, C);
-        }
+        if (c4 < n4) *reinterpret_cast<float4 *>(dst + 4 * c4) = updated(d, value, t[q], acc[q], C);
       }
     }
-    if (value && d.lam != 0.f && lane < len) s.pb[lane == 0 ? m0.id : m1.id] = entropy_term(d, W);
+    if (value && d.lam != 0.f && lane < len) s.pb[mj.id] = entropy_term(d, W);
   }
 }
 
@@ -680,10 +710,11 @@ static cudaError_t launch_apply_t(const Dims &d, float *V, float *K, const Scrat
 
 cudaError_t launch_apply(const Dims &d, float *V, float *K, const Scratch &s, cudaStream_t st,
                          int part) {
+  // rows up to 128 floats in one column block; wider rows in blocks of 256
+  // (2 float4 per lane keeps kU source rows in flight without spilling)
   const int w4 = ((d.dv > d.dh ? d.dv : d.dh) / 4 + 31) / 32;
   if (w4 <= 1) return launch_apply_t<1>(d, V, K, s, st, part);
-  if (w4 <= 2) return launch_apply_t<2>(d, V, K, s, st, part);
-  return launch_apply_t<4>(d, V, K, s, st, part);
+  return launch_apply_t<2>(d, V, K, s, st, part);
 }
 
 // ---------------------------------------------------------------------------

@@ -11,45 +11,114 @@
 // and, when the entropy term is off (so dL/dw is complete here), the softmax
 // Jacobian dL/ds_r = w_r (dL/dw_r - sum_r' w_r' dL/dw_r') and, per sub-key
 // entry, alpha = (sum of dL/ds over its pairs) / (eps + d).
-// One CTA per token row.  The H*k value rows are fetched by 1-D bulk async
-// copies (TMA) straight into shared memory, completing on one mbarrier, so
-// the whole gather of a token is in flight at once; both passes (weighted
-// sum, then the dot products with e_t) read the staged rows.  Rows that do
-// not fit in shared memory are read from global memory in both passes.
+//
+// One thread-block cluster of G CTAs per token row.  The token's H*k value
+// rows are split into G consecutive ranges; each CTA fetches its range by
+// 1-D bulk async copies (TMA) straight into its shared memory, completing on
+// one mbarrier, and writes its share of the token's member records while the
+// rows land.  Each CTA then forms the partial weighted sum of its rows; the
+// cluster exchanges the partials through distributed shared memory and every
+// CTA adds them in rank order (the same yhat everywhere), so each can take
+// the dot products of its own rows with e_t.  G grows with the token's gather
+// (about 32 KB of rows per CTA) so that several tokens are in flight per
+// multiprocessor whatever H*k*dv is.  Rows that do not fit in shared memory
+// are read from global memory in both passes.
 #include "fwpkm_internal.cuh"
 
 namespace fwpkm {
 
 constexpr int kReadThreads = 128;
 constexpr size_t kReadSmemBudget = 200 * 1024;
+constexpr size_t kReadCtaRows = 32 * 1024;  // staged bytes per CTA the cluster size aims at
+constexpr int kReadMaxCluster = 8;          // portable cluster size
+
+struct ReadPlan {
+  int G;        // CTAs per token (cluster size, a power of two <= 8)
+  int per;      // pairs per CTA, ceil(H*k / G)
+  bool staged;  // rows staged in shared memory
+  size_t smem;  // dynamic shared memory per CTA
+};
 
 // Dynamic shared memory layout (bytes):
-//   [0, 16)            mbarrier
-//   [128, 128+R)       staged rows, R = H*k*dv*4 (staged variant only)
-//   then               e (dv floats), w, slot, a, dL/ds (H*k each)
-static size_t read_smem_bytes(const Dims &d, bool staged) {
+//   [0, 16)               mbarrier
+//   [128, 128 + R)        staged rows of this CTA, R = per*dv*4 (staged only)
+//   then ypart, e         dv floats each (ypart is read by the whole cluster)
+//   then w, slot, a, dl   H*k each (a is read by the whole cluster)
+static size_t read_smem_bytes(const Dims &d, int per, bool staged) {
   const size_t HK = (size_t)d.H * d.k;
-  return 128 + (staged ? HK * d.dv * 4 : 0) + (size_t)d.dv * 4 + HK * 16;
+  return 128 + (staged ? (size_t)per * d.dv * 4 : 0) + 2 * (size_t)d.dv * 4 + HK * 16;
+}
+
+static ReadPlan read_plan(const Dims &d) {
+  const int HK = d.H * d.k;
+  const size_t row_bytes = (size_t)d.dv * 4;
+  ReadPlan p;
+  p.G = 1;
+  while (p.G < kReadMaxCluster && p.G < HK &&
+         (size_t)((HK + p.G - 1) / p.G) * row_bytes > kReadCtaRows)
+    p.G <<= 1;
+  p.per = (HK + p.G - 1) / p.G;
+  p.staged = read_smem_bytes(d, p.per, true) <= kReadSmemBudget;
+  p.smem = read_smem_bytes(d, p.per, p.staged);
+  return p;
+}
+
+// --- cluster helpers -------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// All threads of every CTA of the cluster; orders shared-memory writes before
+// the barrier with the other CTAs' reads after it.
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::
+          : "memory");
+}
+// Address of `p` (this CTA's shared memory) in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_smem(const void *p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ float4 ld_peer4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ float ld_peer(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 template <typename TV, bool kStaged>
 __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__restrict__ V,
                                                        const TV *__restrict__ Vt,
                                                        const float *__restrict__ gate,
-                                                       float *__restrict__ out, Scratch s) {
+                                                       float *__restrict__ out, Scratch s, int G,
+                                                       int per) {
   griddep_wait();
   griddep_launch();
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
   const int HK = d.H * d.k, dv = d.dv, dv4 = dv >> 2;
   float *rows_s = reinterpret_cast<float *>(smem + 128);
-  float *e_s = rows_s + (kStaged ? (size_t)HK * dv : 0);
+  float *ypart = rows_s + (kStaged ? (size_t)per * dv : 0);
+  float *e_s = ypart + dv;
   float *w_s = e_s + dv;
   int *slot_s = reinterpret_cast<int *>(w_s + HK);
   float *a_s = reinterpret_cast<float *>(slot_s + HK);
   float *dl_s = a_s + HK;
 
-  const int row = blockIdx.x;
+  const int rank = G > 1 ? (int)cluster_rank() : 0;
+  const int row = blockIdx.x / G;
+  const int j0 = min(HK, rank * per), j1 = min(HK, j0 + per);  // this CTA's pairs
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int b = row / d.Tc, tl = row % d.Tc;
   const int64_t tok = (int64_t)b * d.T + d.t0 + tl;
@@ -59,50 +128,105 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
     w_s[j] = s.pw[p0 + j];
     slot_s[j] = s.pslot[p0 + j];
   }
-  if (kStaged) {
-    if (tid == 0) mbar_init(bar, 1);
-    __syncthreads();
-    if (tid == 0) {
-      const unsigned row_bytes = (unsigned)dv * 4u;
-      mbar_arrive_expect_tx(bar, row_bytes * (unsigned)HK);
-      for (int j = 0; j < HK; ++j)
-        bulk_g2s(rows_s + (size_t)j * dv, V + (int64_t)slot_s[j] * dv, row_bytes, bar);
-    }
-    if (!mbar_wait_bounded(bar, 0, s.meta)) {
-      mbar_wait_bounded(bar, 0, s.meta);  // let copies in flight land before exit
-      return;
-    }
-  } else {
-    __syncthreads();
+  if (kStaged && tid == 0) mbar_init(bar, 1);
+  __syncthreads();
+  const unsigned row_bytes = (unsigned)dv * 4u;
+  if (kStaged && wid == 0 && j1 > j0) {
+    if (lane == 0) mbar_arrive_expect_tx(bar, row_bytes * (unsigned)(j1 - j0));
+    __syncwarp();
+    for (int j = j0 + lane; j < j1; j += 32)
+      bulk_g2s(rows_s + (size_t)(j - j0) * dv, V + (int64_t)slot_s[j] * dv, row_bytes, bar);
   }
-
   const float g = gate[tok];
   const float invH = 1.f / (float)d.H;
+
+  // Member records go to their buckets while the gather is in flight (none
+  // of their fields depends on the rows): this CTA's pairs -> value bucket
+  // slot >> vshift; entries x = rank (mod G) -> sub-key row bucket
+  // NBv + (h*2+half)*n + row.  An entry's alpha is filled in later from
+  // ealpha (by the sort, or by the apply when the entropy term is on).
+  for (int j = j0 + tid; j < j1; j += blockDim.x) {
+    const int64_t p = p0 + j;
+    const float w = w_s[j];
+    Member m;
+    m.g = (uint32_t)slot_s[j];
+    m.id = (uint32_t)p;
+    m.srow = row;
+    m.gstart = 0;
+    m.coef = 2.f * g * w * invH;
+    m.c0 = w * invH;
+    m.c1 = w;
+    m.glen = 0;
+    s.rec_in[s.boff[slot_s[j] >> d.vshift] + s.pclaim[p]] = m;
+  }
+  for (int x = rank + G * tid; x < 2 * HK; x += G * blockDim.x) {
+    const int mh = x / d.k, idx = x % d.k;  // entry (h*2 + half)*k + idx of this row
+    const int64_t mhg = (int64_t)row * 2 * d.H + mh;
+    if (idx < s.ecount[mhg]) {
+      const int64_t e = mhg * d.k + idx;
+      const int sub = s.esub[e];
+      Member m;
+      m.g = (uint32_t)d.N + (uint32_t)(mh * d.n + sub);
+      m.id = (uint32_t)e;
+      m.srow = mh * d.qstride + row;
+      m.gstart = 0;
+      m.coef = 0.f;
+      m.c0 = 0.f;
+      m.c1 = 0.f;
+      m.glen = 0;
+      s.rec_in[s.boff[d.NBv + mh * d.n + sub] + s.eclaim[e]] = m;
+    }
+  }
+  // On a timeout the error bit is set and the CTA still takes every cluster
+  // barrier (its results are then meaningless, and the host reports it).
+  if (kStaged && j1 > j0 && !mbar_wait_bounded(bar, 0, s.meta))
+    mbar_wait_bounded(bar, 0, s.meta);  // let copies in flight land
+
+  // pass 1: partial weighted sum of this CTA's rows
   for (int c4 = tid; c4 < dv4; c4 += blockDim.x) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < HK; ++j) {
+    for (int j = j0; j < j1; ++j) {
       const float w = w_s[j];
-      const float4 v = kStaged ? *reinterpret_cast<const float4 *>(rows_s + (size_t)j * dv + 4 * c4)
-                               : *reinterpret_cast<const float4 *>(V + (int64_t)slot_s[j] * dv + 4 * c4);
+      const float4 v =
+          kStaged ? *reinterpret_cast<const float4 *>(rows_s + (size_t)(j - j0) * dv + 4 * c4)
+                  : *reinterpret_cast<const float4 *>(V + (int64_t)slot_s[j] * dv + 4 * c4);
       acc.x = fmaf(w, v.x, acc.x);
       acc.y = fmaf(w, v.y, acc.y);
       acc.z = fmaf(w, v.z, acc.z);
       acc.w = fmaf(w, v.w, acc.w);
     }
-    const float4 y = make_float4(acc.x * invH, acc.y * invH, acc.z * invH, acc.w * invH);
-    *reinterpret_cast<float4 *>(out + tok * dv + 4 * c4) =
-        make_float4(g * y.x, g * y.y, g * y.z, g * y.w);
+    *reinterpret_cast<float4 *>(ypart + 4 * c4) = acc;
+  }
+  if (G > 1) cluster_barrier();
+  else __syncthreads();
+
+  // yhat = (partials added in rank order) / H, identical in every CTA
+  for (int c4 = tid; c4 < dv4; c4 += blockDim.x) {
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = 0; r < G; ++r) {
+      const float4 v = G > 1 ? ld_peer4(peer_smem(ypart + 4 * c4, (uint32_t)r))
+                             : *reinterpret_cast<const float4 *>(ypart + 4 * c4);
+      y.x += v.x;
+      y.y += v.y;
+      y.z += v.z;
+      y.w += v.w;
+    }
+    y = make_float4(y.x * invH, y.y * invH, y.z * invH, y.w * invH);
     const float4 t = load4(Vt, tok * dv + 4 * c4);
     const float4 e = make_float4(y.x - t.x, y.y - t.y, y.z - t.z, y.w - t.w);
-    *reinterpret_cast<float4 *>(s.E + (int64_t)row * dv + 4 * c4) = e;
+    if (rank == 0) {
+      *reinterpret_cast<float4 *>(out + tok * dv + 4 * c4) =
+          make_float4(g * y.x, g * y.y, g * y.z, g * y.w);
+      *reinterpret_cast<float4 *>(s.E + (int64_t)row * dv + 4 * c4) = e;
+    }
     *reinterpret_cast<float4 *>(e_s + 4 * c4) = e;
   }
   __syncthreads();
 
-  // dL/dw per pair: warp `wid` takes pairs j = wid, wid + 4, ...
+  // dL/dw of this CTA's pairs: warp `wid` takes pairs j0 + wid, j0 + wid + 4, ...
   const float coef = 2.f * g * invH;
-  for (int j = wid; j < HK; j += kReadThreads / 32) {
-    const float *vr = kStaged ? rows_s + (size_t)j * dv : V + (int64_t)slot_s[j] * dv;
+  for (int j = j0 + wid; j < j1; j += kReadThreads / 32) {
+    const float *vr = kStaged ? rows_s + (size_t)(j - j0) * dv : V + (int64_t)slot_s[j] * dv;
     float acc = 0.f;
     for (int c4 = lane; c4 < dv4; c4 += 32) {
       const float4 v = *reinterpret_cast<const float4 *>(vr + 4 * c4);
@@ -118,21 +242,25 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
       a_s[j] = coef * acc;
     }
   }
+  // every CTA is done reading the partials, and the a values are published
+  if (G > 1) cluster_barrier();
+  else __syncthreads();
 
   // dL/ds and alpha per entry when the entropy term is off (dL/dw complete)
-  __syncthreads();
-  const bool alpha_now = d.lam == 0.f;
-  if (alpha_now) {
+  if (d.lam == 0.f) {
     for (int h = wid; h < d.H; h += kReadThreads / 32) {
       const int j = h * d.k + lane;
-      const float w = lane < d.k ? w_s[j] : 0.f;
-      const float a = lane < d.k ? a_s[j] : 0.f;
+      float w = 0.f, a = 0.f;
+      if (lane < d.k) {
+        w = w_s[j];
+        a = G > 1 ? ld_peer(peer_smem(a_s + j, (uint32_t)(j / per))) : a_s[j];
+      }
       const float S = warp_sum(w * a);
       if (lane < d.k) dl_s[j] = w * (a - S);
     }
     __syncthreads();
-    // alpha of every entry of this row, one thread each
-    for (int x = tid; x < 2 * HK; x += blockDim.x) {
+    // alpha of the entries x = rank (mod G) of this row, one thread each
+    for (int x = rank + G * tid; x < 2 * HK; x += G * blockDim.x) {
       const int mh = x / d.k, idx = x % d.k;  // mh = h*2 + half
       const int64_t mhg = (int64_t)row * 2 * d.H + mh;
       if (idx < s.ecount[mhg]) {
@@ -147,62 +275,21 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
         s.ealpha[e] = s.einv[e] * sum;
       }
     }
-    __syncthreads();
-  }
-  // Member records into their buckets: pairs -> value bucket slot >> vshift,
-  // entries -> sub-key row bucket NBv + (h*2+half)*n + row.
-  for (int j = tid; j < HK; j += blockDim.x) {
-    const int64_t p = p0 + j;
-    const float w = w_s[j];
-    Member m;
-    m.g = (uint32_t)slot_s[j];
-    m.id = (uint32_t)p;
-    m.srow = row;
-    m.gstart = 0;
-    m.coef = 2.f * g * w * invH;
-    m.c0 = w * invH;
-    m.c1 = w;
-    m.glen = 0;
-    s.rec_in[s.boff[slot_s[j] >> d.vshift] + s.pclaim[p]] = m;
-  }
-  const int ne = 2 * HK;  // entries of this row: (h*2 + half)*k + idx
-  for (int x = tid; x < ne; x += blockDim.x) {
-    const int mh = x / d.k, idx = x % d.k;  // mh = h*2 + half
-    const int64_t mhg = (int64_t)row * 2 * d.H + mh;
-    if (idx < s.ecount[mhg]) {
-      const int64_t e = mhg * d.k + idx;
-      const int sub = s.esub[e];
-      const float alpha = alpha_now ? s.ealpha[e] : 0.f;
-      Member m;
-      m.g = (uint32_t)d.N + (uint32_t)(mh * d.n + sub);
-      m.id = (uint32_t)e;
-      m.srow = mh * d.qstride + row;
-      m.gstart = 0;
-      m.coef = alpha;
-      m.c0 = alpha;
-      m.c1 = 0.f;
-      m.glen = 0;
-      s.rec_in[s.boff[d.NBv + mh * d.n + sub] + s.eclaim[e]] = m;
-    }
+    // no CTA leaves while another may still read its a values
+    if (G > 1) cluster_barrier();
   }
 }
 
 template <typename TV>
 static cudaError_t launch_read_t(const Dims &d, const float *V, const TV *Vt, const float *gate,
                                  float *out, const Scratch &s, cudaStream_t st) {
-  const bool staged = read_smem_bytes(d, true) <= kReadSmemBudget;
-  const size_t smem = read_smem_bytes(d, staged);
-  if (staged) {
-    cudaFuncSetAttribute(k_read<TV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    return launch_k(d.pdl, k_read<TV, true>, d.rows, kReadThreads, smem, st, d, V, Vt, gate,
-                    out, s);
-  } else {
-    cudaFuncSetAttribute(k_read<TV, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    return launch_k(d.pdl, k_read<TV, false>, d.rows, kReadThreads, smem, st, d, V, Vt, gate,
-                    out, s);
-  }
+  const ReadPlan p = read_plan(d);
+  auto kernel = p.staged ? k_read<TV, true> : k_read<TV, false>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+  if (e != cudaSuccess) return e;
+  return launch_kc(d.pdl, p.G, kernel, d.rows * p.G, kReadThreads, p.smem, st, d, V, Vt, gate,
+                   out, s, p.G, p.per);
 }
 
 cudaError_t launch_read(const Dims &d, const float *V, const void *Vt, int v_dtype,
