@@ -156,10 +156,13 @@ fwpkm_status fwpkm_force_selection(fwpkm_state *s, const int32_t *slots, const u
 
 /*
  * Per-kernel timing.  With profiling on, fwpkm_step records a CUDA event pair
- * around every kernel it enqueues; fwpkm_profile_read synchronises `stream`,
- * adds up the elapsed times per kernel kind, and returns them:
- *   names[i] (static strings), ms[i] (total milliseconds), launches[i],
- *   for i < *count (<= max_kinds).  Reading resets the totals.
+ * around every step of the chunk it enqueues (one kernel, or two for
+ * fwpkm_apply: the member pass and the combine of longer groups) and launches
+ * without programmatic dependent launch; fwpkm_profile_read synchronises
+ * `stream`, adds up the elapsed times per kind, and returns them:
+ *   names[i] (static strings), ms[i] (total milliseconds), launches[i]
+ *   (kernels launched), for i < *count (<= max_kinds).  Reading resets the
+ *   totals.
  */
 fwpkm_status fwpkm_set_profiling(fwpkm_state *s, int enable);
 fwpkm_status fwpkm_profile_read(fwpkm_state *s, const char **names, double *ms,

@@ -40,6 +40,9 @@ fwpkm_status cuda_fail(cudaError_t e, const char *what) {
 enum Kind { K_PREP, K_SCORE, K_TOPK, K_SCAN, K_READ, K_BSORT, K_APPLY, K_PGRAD, K_COUNT };
 const char *kKindNames[K_COUNT] = {"fwpkm_prep", "fwpkm_score", "fwpkm_topk",  "fwpkm_scan",
                                    "fwpkm_read", "fwpkm_bsort", "fwpkm_apply", "fwpkm_pgrad"};
+// Kernels one call of a kind enqueues (the apply is a member pass plus the
+// combine of longer groups).
+const int kKernelsPerCall[K_COUNT] = {1, 1, 1, 1, 1, 1, 2, 1};
 
 struct Timing {
   int kind;
@@ -103,7 +106,9 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
   const int64_t H = st->H, n = st->n, dh = st->dh, dv = st->dv, k = st->k;
   const int64_t M = rows * H, P = M * k, NB = value_buckets(st->N, P) + 2 * H * n;
   const int64_t Lcap = 3 * P;  // pairs + at most 2 entries per pair
-  const int64_t pool_cap = 2 * Lcap / 32 + 2;  // long-group blocks of 32 members
+  // Blocks of groups of more than 4 members, 32 members a block: at most
+  // L/32 + L/5 of them, under L/4.
+  const int64_t pool_cap = Lcap / 4 + 2;
   const int pwidth = 4 + (int)(dv > dh ? dv : dh);
   struct Piece {
     void **ptr;
@@ -135,12 +140,14 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
       {(void **)&s.rec_in, sizeof(Member) * (size_t)Lcap},
       {(void **)&s.rec, sizeof(Member) * (size_t)Lcap},
       {(void **)&s.posmap, sizeof(int32_t) * (size_t)Lcap},
-      {(void **)&s.slotmap, sizeof(int32_t) * (size_t)Lcap},
-      {(void **)&s.shortlist, sizeof(int32_t) * (size_t)Lcap},
-      {(void **)&s.longlist, sizeof(int32_t) * (size_t)Lcap},
+      {(void **)&s.shortlist[0], sizeof(int32_t) * (size_t)Lcap},
+      {(void **)&s.shortlist[1], sizeof(int32_t) * (size_t)Lcap},
+      {(void **)&s.longlist[0], sizeof(int32_t) * (size_t)Lcap},
+      {(void **)&s.longlist[1], sizeof(int32_t) * (size_t)Lcap},
+      {(void **)&s.glist[0], sizeof(int32_t) * (size_t)Lcap},
+      {(void **)&s.glist[1], sizeof(int32_t) * (size_t)Lcap},
       {(void **)&s.sort_tmp, sizeof(uint64_t) * (size_t)(2 * Lcap)},
       {(void **)&s.partial, sizeof(float) * (size_t)pool_cap * pwidth},
-      {(void **)&s.segcnt, sizeof(int32_t) * (size_t)Lcap},
       {(void **)&s.E, sizeof(float) * (size_t)(rows * dv)},
       {(void **)&s.meta, sizeof(Meta)},
   };
@@ -162,10 +169,9 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
     *p.ptr = (char *)arena + off;
     off += align_up(p.bytes, 256);
   }
-  // Bucket counts and crossing-group counters start at zero (the kernels
-  // leave them at zero); the meta block (stats) carries over.
+  // Bucket counts start at zero (the kernels leave them at zero); the meta
+  // block (stats) carries over.
   e = cudaMemset(s.bcnt, 0, sizeof(int32_t) * (size_t)NB);
-  if (e == cudaSuccess) e = cudaMemset(s.segcnt, 0, sizeof(int32_t) * (size_t)Lcap);
   if (e == cudaSuccess) e = cudaMemset(s.meta, 0, sizeof(Meta));
   if (e == cudaSuccess && st->s.meta)
     e = cudaMemcpy(s.meta, st->s.meta, sizeof(Meta), cudaMemcpyDeviceToDevice);
@@ -521,7 +527,7 @@ fwpkm_status fwpkm_profile_read(fwpkm_state *st, const char **names, double *ms,
     float dt = 0.f;
     if (cudaEventElapsedTime(&dt, t.a, t.b) == cudaSuccess) {
       st->prof_ms[t.kind] += dt;
-      st->prof_n[t.kind] += 1;
+      st->prof_n[t.kind] += kKernelsPerCall[t.kind];
     }
     st->event_pool.push_back(t.a);
     st->event_pool.push_back(t.b);

@@ -38,9 +38,11 @@ struct Meta {
   int32_t L;              // members of the chunk (pairs + sub-key entries)
   int32_t Lv;             // pairs (value-row members come first)
   unsigned err;           // ERR_* bits, sticky until the host clears them
-  int32_t pool_next;      // next free partial slot (reset per chunk)
-  int32_t nshort;         // groups of <= 2 members listed in shortlist (reset per chunk)
-  int32_t nlong;          // 32-member blocks of longer groups in longlist (reset per chunk)
+  // Work lists of the chunk, per kind (0: value rows, 1: sub-key rows),
+  // reset per chunk by the scan:
+  int32_t nshort[2];      // groups of <= 4 members in shortlist[kind]
+  int32_t nlong[2];       // 32-member blocks of longer groups in longlist[kind]
+  int32_t ngroup[2];      // longer groups in glist[kind]
   int32_t pad2;
   unsigned long long stat_chunks;      // chunks processed since reset
   unsigned long long stat_value_rows;  // sum over chunks of distinct value rows written
@@ -90,17 +92,18 @@ struct Scratch {
   struct Member *rec;     // [Lcap] the same records sorted by (group, id)
   uint64_t *sort_tmp;  // [2*Lcap] merge buffers for oversized buckets
   int32_t *posmap;  // [Lcap]  position inside its bucket, by member id (oversized buckets)
-  int32_t *slotmap; // [Lcap]  partial-pool slot of the block starting here
-  int32_t *shortlist;  // [Lcap] first position of every group of <= 32 members
-  int32_t *longlist;   // [Lcap] first position of every 32-member block of longer groups
-  float *partial;   // [pool_cap][pwidth] block partial sums of long groups
-  int32_t *segcnt;  // [Lcap] arrived blocks per long group, at its first position
+  int32_t *shortlist[2];  // [Lcap] per kind: first position of every group of <= 4 members
+  int32_t *longlist[2];   // [Lcap] per kind: first position of every 32-member block of a
+                          //        longer group (a group's blocks are consecutive)
+  int32_t *glist[2];      // [Lcap] per kind: index in longlist of every longer group's first block
+  float *partial;   // [pool_cap][pwidth] block partial sums: value blocks at their longlist
+                    // index, sub-key blocks after all value blocks
                     // (zero between chunks)
   float *E;         // [rows][dv] residual yhat - v
   Meta *meta;
   int64_t Lcap;     // member capacity (3 * M*k)
   int pwidth;       // 4 + max(dv, dh) floats
-  int pool_cap;     // partial slots: 2 * Lcap / 32
+  int pool_cap;     // partial slots: Lcap / 4 + 2
 };
 
 // One member of a group (32 bytes).  Value rows: a pair p; sub-key rows: an

@@ -129,9 +129,12 @@ __global__ void __launch_bounds__(kScanThreads) k_bucket_scan(Dims d, Scratch s)
     s.meta->L = carry;
     if (d.NBv >= NB) s.meta->Lv = carry;
     s.meta->stat_chunks += 1ull;
-    s.meta->pool_next = 0;
-    s.meta->nshort = 0;
-    s.meta->nlong = 0;
+#pragma unroll
+    for (int kind = 0; kind < 2; ++kind) {
+      s.meta->nshort[kind] = 0;
+      s.meta->nlong[kind] = 0;
+      s.meta->ngroup[kind] = 0;
+    }
   }
 }
 
@@ -197,25 +200,128 @@ __device__ __forceinline__ Member fetch_member(const Dims &d, const Scratch &s, 
   return m;
 }
 
-constexpr int kShortMax = 32;  // groups up to this size are applied by one warp
+constexpr int kShortMax = 4;  // groups up to this size are applied by one warp, whole rows
 constexpr int kBlock = 32;    // longer groups are applied in blocks of this many members
 
-// Work lists of the apply kernel for a group that starts at position x0:
-// a short group goes to shortlist, a longer one to longlist, one entry per
-// block of kBlock members.  Thread-level (one call per group head).
-__device__ __forceinline__ void list_group(const Scratch &s, int x0, int len) {
+// Work lists of the apply kernels for a group of kind `kind` (0: value row,
+// 1: sub-key row) that starts at position x0: a short group goes to
+// shortlist, a longer one to longlist, one entry per block of kBlock members
+// (consecutive entries), plus its first block's index to glist.  Thread-level
+// (one call per group head).
+__device__ __forceinline__ void list_group(const Scratch &s, int kind, int x0, int len) {
   if (len <= kShortMax) {
-    s.shortlist[atomicAdd(&s.meta->nshort, 1)] = x0;
+    s.shortlist[kind][atomicAdd(&s.meta->nshort[kind], 1)] = x0;
   } else {
     const int nb = (len + kBlock - 1) / kBlock;
-    const int base = atomicAdd(&s.meta->nlong, nb);
-    for (int b = 0; b < nb; ++b) s.longlist[base + b] = x0 + b * kBlock;
+    const int base = atomicAdd(&s.meta->nlong[kind], nb);
+    for (int b = 0; b < nb; ++b) s.longlist[kind][base + b] = x0 + b * kBlock;
+    s.glist[kind][atomicAdd(&s.meta->ngroup[kind], 1)] = base;
   }
+}
+
+// Rank sort of one bucket with more than 32 members.  Inside a group, every
+// member comes from a different token-head m (a token-head's k slots are
+// distinct, and its sub-key entries are de-duplicated per row), and member
+// ids grow with m (pair p = m*k + r, entry e = (m*2 + half)*k + idx).  So the
+// (group, id) order is the (group, m) order, and a member's rank is found
+// without sorting: one bitmap of token-heads per group of the bucket, an
+// exclusive prefix of the words' popcounts (flat over groups, then words)
+// gives every group's start and every member's place.  A few barriers instead
+// of a bitonic network's dozens.  Returns false, having written nothing,
+// when the bitmaps do not fit or a group repeats a token-head (forced
+// selections with duplicate slots); the caller then sorts.
+constexpr int kRankWords = kSortCap;  // bitmap words (the prefix takes as many)
+constexpr int kRankGroups = 256;      // groups per bucket (slots per value bucket)
+
+struct RankSmem {
+  uint32_t *bits;  // [kRankWords]
+  uint32_t *pre;   // [kRankWords]
+  int *gcnt;       // [kRankGroups]
+  int *red;        // [32]
+  int *flag;
+};
+
+__device__ bool rank_big_bucket(const Dims &d, const Scratch &s, int off, int len, bool value,
+                                uint32_t gbase, const RankSmem &r, int *nseg) {
+  const int G = value ? (1 << d.vshift) : 1;
+  const int Mw = (d.M + 31) >> 5;
+  const int W = G * Mw;
+  if (G > kRankGroups || W > kRankWords) return false;  // the same in every thread
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t kdiv = value ? (uint32_t)d.k : 2u * (uint32_t)d.k;  // id -> token-head
+  for (int i = tid; i < W; i += blockDim.x) r.bits[i] = 0u;
+  for (int i = tid; i < G; i += blockDim.x) r.gcnt[i] = 0;
+  if (tid == 0) *r.flag = 0;
+  __syncthreads();
+  for (int i = tid; i < len; i += blockDim.x) {
+    const int2 gi = *reinterpret_cast<const int2 *>(s.rec_in + off + i);  // g, id
+    const int lg = value ? (int)((uint32_t)gi.x - gbase) : 0;
+    const uint32_t m = (uint32_t)gi.y / kdiv;
+    const uint32_t bit = 1u << (m & 31u);
+    if (atomicOr(&r.bits[lg * Mw + (int)(m >> 5)], bit) & bit) *r.flag = 1;
+    atomicAdd(&r.gcnt[lg], 1);
+  }
+  __syncthreads();
+  if (*r.flag) return false;
+  // exclusive prefix of the popcounts, kRankWords / kSortThreads words per thread
+  constexpr int per = kRankWords / kSortThreads;
+  const int w0 = tid * per;
+  int v[per], tot = 0;
+#pragma unroll
+  for (int q = 0; q < per; ++q) {
+    v[q] = w0 + q < W ? __popc(r.bits[w0 + q]) : 0;
+    tot += v[q];
+  }
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(FULL, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) r.red[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int x = lane < kSortWarps ? r.red[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(FULL, x, o);
+      if (lane >= o) x += t;
+    }
+    r.red[lane] = x;
+  }
+  __syncthreads();
+  int run = (warp > 0 ? r.red[warp - 1] : 0) + incl - tot;
+#pragma unroll
+  for (int q = 0; q < per; ++q) {
+    if (w0 + q < W) r.pre[w0 + q] = run;
+    run += v[q];
+  }
+  __syncthreads();
+  int my_seg = 0;
+  for (int i = tid; i < len; i += blockDim.x) {
+    Member mr = fetch_member(d, s, s.rec_in + off + i);
+    const int lg = value ? (int)(mr.g - gbase) : 0;
+    const uint32_t m = mr.id / kdiv;
+    const int wi = lg * Mw + (int)(m >> 5);
+    const int pos = (int)r.pre[wi] + __popc(r.bits[wi] & ((1u << (m & 31u)) - 1u));
+    const int first = (int)r.pre[lg * Mw];
+    mr.gstart = off + first;
+    mr.glen = r.gcnt[lg];
+    store_member(s.rec + off + pos, mr);
+    if (pos == first) {
+      my_seg += 1;
+      list_group(s, value ? 0 : 1, off + pos, mr.glen);
+    }
+  }
+  if (my_seg) atomicAdd(nseg, my_seg);
+  __syncthreads();
+  return true;
 }
 
 // CTA-wide sort of one bucket with more than 32 members.
 __device__ void sort_big_bucket(const Dims &d, const Scratch &s, int off, int len, bool value,
-                                uint32_t gbase, uint64_t *buf, int *nseg) {
+                                uint32_t gbase, uint64_t *buf, const RankSmem &rs, int *nseg) {
+  if (rank_big_bucket(d, s, off, len, value, gbase, rs, nseg)) return;
   int my_seg = 0;
   if (len <= kSortCap) {
     // key = (g - gbase) << 43 | id << 12 | local index   (g - gbase < 2^21, id < 2^31)
@@ -243,7 +349,7 @@ __device__ void sort_big_bucket(const Dims &d, const Scratch &s, int off, int le
       store_member(s.rec + off + i, m);
       if (first == i) {
         my_seg += 1;
-        list_group(s, off + i, end - first);
+        list_group(s, value ? 0 : 1, off + i, end - first);
       }
     }
   } else {
@@ -300,7 +406,7 @@ __device__ void sort_big_bucket(const Dims &d, const Scratch &s, int off, int le
       store_member(s.rec + off + i, m);
       if (first == i) {
         my_seg += 1;
-        list_group(s, off + i, end - first);
+        list_group(s, value ? 0 : 1, off + i, end - first);
       }
     }
   }
@@ -313,6 +419,7 @@ __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s)
   __shared__ int nseg[2];  // distinct value rows / sub-key rows seen by this CTA
   __shared__ int big_n;
   __shared__ int big_b[kSortWarps * 8];  // large buckets met in phase 1
+  __shared__ int rank_gcnt[kRankGroups], rank_red[32], rank_flag;
   griddep_wait();
   griddep_launch();
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
@@ -377,18 +484,27 @@ __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s)
       r.glen = glen = (after ? __ffs(after) - 1 : len) - h0;
       store_member(s.rec + off + lane, r);
     }
-    // work lists: short groups, and the blocks of longer ones
-    const bool sh = head && glen <= kShortMax;
-    const unsigned sb = __ballot_sync(FULL, sh);
-    int sbase = 0;
-    if (lane == 0 && sb) sbase = atomicAdd(&s.meta->nshort, __popc(sb));
+    // work lists: short groups; longer ones (one block each, <= 32 members)
+    const int kind = b < d.NBv ? 0 : 1;
+    const bool sh = head && glen <= kShortMax, lg = head && glen > kShortMax;
+    const unsigned sb = __ballot_sync(FULL, sh), lb = __ballot_sync(FULL, lg);
+    int sbase = 0, lbase = 0, gbase = 0;
+    if (lane == 0) {
+      if (sb) sbase = atomicAdd(&s.meta->nshort[kind], __popc(sb));
+      if (lb) {
+        lbase = atomicAdd(&s.meta->nlong[kind], __popc(lb));
+        gbase = atomicAdd(&s.meta->ngroup[kind], __popc(lb));
+      }
+    }
     sbase = __shfl_sync(FULL, sbase, 0);
-    if (sh) s.shortlist[sbase + __popc(sb & lanemask_lt())] = off + lane;
-    const unsigned lb = __ballot_sync(FULL, head && glen > kShortMax);  // <= 32 members: 1 block
-    int lbase = 0;
-    if (lane == 0 && lb) lbase = atomicAdd(&s.meta->nlong, __popc(lb));
     lbase = __shfl_sync(FULL, lbase, 0);
-    if (head && glen > kShortMax) s.longlist[lbase + __popc(lb & lanemask_lt())] = off + lane;
+    gbase = __shfl_sync(FULL, gbase, 0);
+    if (sh) s.shortlist[kind][sbase + __popc(sb & lanemask_lt())] = off + lane;
+    if (lg) {
+      const int li = lbase + __popc(lb & lanemask_lt());
+      s.longlist[kind][li] = off + lane;
+      s.glist[kind][gbase + __popc(lb & lanemask_lt())] = li;
+    }
     if (lane == 0) atomicAdd(&nseg[b < d.NBv ? 0 : 1], __popc(heads));
   }
   __syncthreads();
@@ -400,7 +516,9 @@ __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s)
     const bool value = b < d.NBv;
     const uint32_t gbase =
         value ? ((uint32_t)b << d.vshift) : (uint32_t)d.N + (uint32_t)(b - d.NBv);
-    sort_big_bucket(d, s, off, len, value, gbase, buf, &nseg[value ? 0 : 1]);
+    const RankSmem rs{reinterpret_cast<uint32_t *>(buf), reinterpret_cast<uint32_t *>(buf) + kRankWords,
+                      rank_gcnt, rank_red, &rank_flag};
+    sort_big_bucket(d, s, off, len, value, gbase, buf, rs, &nseg[value ? 0 : 1]);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -426,31 +544,29 @@ cudaError_t launch_bsort(const Dims &d, const Scratch &s, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------------------
-// apply: the row updates, from the two work lists bsort wrote.
-//   phase A, one CTA per block of up to kBlock members of a longer group: the
-//     8 warps each take members m = w, w+8, w+16, w+24 and have all their
-//     source rows in flight at once (E rows for value rows, query halves for
-//     sub-key rows); the warps' sums are added in warp order.  A one-block
-//     group is written at once; otherwise the block publishes a partial and
-//     the last block of the group adds the partials in block order.
-//   phase B, one warp per group of <= kShortMax members: the lanes hold the
-//     records, the members' source rows are summed in member order with a
-//     few rows in flight, then the row is written.
-// Column blocks of 32 * Q4 float4 bound the registers for any row width.
-// Every sum runs in an order fixed by the data, whatever the scheduling.
+// apply: the row updates, from the work lists bsort wrote, in two kernels.
+// The unit of work for longer groups is (block, column chunk of 128 floats),
+// one warp each, a float4 per lane: many short dependence chains rather than
+// a few long ones, whatever the skew.
+//   k_apply: a group of <= kShortMax members is summed and its whole row
+//     written at once (two chunks at a time); a column chunk of a block of
+//     kBlock members of a longer group is summed into the partial-pool slot
+//     of the block's work-list entry.  Lane j holds member
+//     j's record; the members' source rows (E rows for value rows, query
+//     halves for sub-key rows) are summed in member order, kU rows in flight.
+//   k_combine: for each (longer group, column chunk), adds the blocks'
+//     partials in block order and writes the row chunk.
+// Every sum runs in an order fixed by the data, whatever the scheduling, and
+// nothing is atomic but the work-list counters of the sort.
 // ---------------------------------------------------------------------------
 constexpr int kApplyThreads = 256;
 constexpr int kApplyWarps = kApplyThreads / 32;
+constexpr int kChunk4 = 32;  // float4 per column chunk (one per lane)
+constexpr int kU = 8;        // source rows in flight per warp
 
-template <int Q4>
-__device__ __forceinline__ void load_row(const float *src, int cb, int n4, float4 (&r)[Q4]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int q = 0; q < Q4; ++q) {
-    const int c4 = cb + lane + 32 * q;
-    r[q] = c4 < n4 ? *reinterpret_cast<const float4 *>(src + 4 * c4)
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+__device__ __forceinline__ float4 load_chunk(const float *row, int c4, int n4) {
+  return c4 < n4 ? *reinterpret_cast<const float4 *>(row + 4 * c4)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 __device__ __forceinline__ void fma4(float4 &a, float c, const float4 &x) {
@@ -491,165 +607,86 @@ __device__ __forceinline__ const float *source_row(const Dims &d, const Scratch 
   return value ? s.E + (int64_t)srow * d.dv : s.Qs + (int64_t)srow * d.dh;
 }
 
-template <int Q4>
+// Sum of a warp's members (lane j < cnt holds member j's srow and coef) over
+// the float4 columns cb + lane + 32*q, q < Q, member order, KU rows in flight.
+template <int Q, int KU>
+__device__ __forceinline__ void sum_members(const Dims &d, const Scratch &s, bool value, int cnt,
+                                            int srow, float coef, int cb, int n4,
+                                            float4 (&acc)[Q]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int q = 0; q < Q; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j0 = 0; j0 < cnt; j0 += KU) {
+    float4 r[KU][Q];
+#pragma unroll
+    for (int u = 0; u < KU; ++u) {
+      const int sr = __shfl_sync(FULL, srow, (j0 + u) & 31);
+      const float *src = source_row(d, s, value, sr);
+#pragma unroll
+      for (int q = 0; q < Q; ++q)
+        r[u][q] = j0 + u < cnt ? load_chunk(src, cb + lane + 32 * q, n4)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < KU; ++u) {
+      const float cj = __shfl_sync(FULL, coef, (j0 + u) & 31);
+      if (j0 + u < cnt) {
+#pragma unroll
+        for (int q = 0; q < Q; ++q) fma4(acc[q], cj, r[u][q]);
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__restrict__ V,
-                                                         float *__restrict__ K, Scratch s,
-                                                         int part) {
-  constexpr int CB = 32 * Q4;  // float4 columns per column block
-  __shared__ float4 red[kApplyWarps][CB];
-  __shared__ int m_srow[kBlock];
-  __shared__ float m_coef[kBlock], m_c0[kBlock], m_c1[kBlock];
-  __shared__ int m_id[kBlock];
-  __shared__ int s_slot, s_last;
+                                                            float *__restrict__ K, Scratch s,
+                                                            int part) {
   griddep_wait();
   griddep_launch();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * kApplyWarps + (threadIdx.x >> 5);
+  const int nw = gridDim.x * kApplyWarps;
   const bool alpha_later = d.lam != 0.f;  // sub-key alphas come from pgrad
-  auto wanted = [&](uint32_t g) {         // part 0: all, 1: value rows, 2: sub-key rows
-    const bool value = g < (uint32_t)d.N;
-    return part == 0 || (part == 1) == value;
-  };
-
-  // ---------------- phase A: blocks of longer groups ----------------
-  const int nlong = s.meta->nlong;
-  for (int it = blockIdx.x; it < nlong; it += gridDim.x) {
-    const int x = s.longlist[it];
-    const int4 head = *reinterpret_cast<const int4 *>(s.rec + x);  // g, id, srow, gstart
-    const uint32_t g = (uint32_t)head.x;
-    if (!wanted(g)) continue;
-    const int g0 = head.w, len = s.rec[x].glen;
-    const int cnt = min(kBlock, g0 + len - x);
-    const int nblocks = (len + kBlock - 1) / kBlock;
-    const bool value = g < (uint32_t)d.N;
-    const int n4 = (value ? d.dv : d.dh) >> 2;
-    float *dst = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.N) * d.dh;
-    if (tid < cnt) {
-      const Member m = load_member(s.rec + x + tid);
-      m_srow[tid] = m.srow;
-      m_id[tid] = (int)m.id;
-      float coef = m.coef, c0 = m.c0;
-      if (!value && alpha_later) coef = c0 = s.ealpha[m.id];
-      m_coef[tid] = coef;
-      m_c0[tid] = c0;
-      m_c1[tid] = m.c1;
+  const int cv = (d.dv / 4 + kChunk4 - 1) / kChunk4, ck = (d.dh / 4 + kChunk4 - 1) / kChunk4;
+  // Work items, longer groups' blocks first: value blocks and sub-key blocks
+  // (one item per column chunk), then value groups and sub-key groups (one
+  // item per group, whole rows), each present when `part` takes its kind
+  // (0: both, 1: value rows, 2: sub-key rows).
+  const int nlv = part != 2 ? s.meta->nlong[0] * cv : 0;
+  const int nlk = part != 1 ? s.meta->nlong[1] * ck : 0;
+  const int nsv = part != 2 ? s.meta->nshort[0] : 0;
+  const int nsk = part != 1 ? s.meta->nshort[1] : 0;
+  const int kslot0 = s.meta->nlong[0];  // sub-key partial slots follow the value blocks
+  const int total = nlv + nlk + nsv + nsk;
+  for (int it = gw; it < total; it += nw) {
+    int i = it, kind = 0;
+    bool block = true;
+    if (i < nlv) {
+    } else if ((i -= nlv) < nlk) {
+      kind = 1;
+    } else if ((i -= nlk) < nsv) {
+      block = false;
+    } else {
+      i -= nsv;
+      kind = 1;
+      block = false;
     }
-    if (tid == 0 && nblocks > 1) {
-      s_slot = atomicAdd(&s.meta->pool_next, 1);
-      if (s_slot >= s.pool_cap) atomicOr(&s.meta->err, ERR_POOL_OVERFLOW);
+    const bool value = kind == 0;
+    int chunk = 0;
+    if (block) {
+      const int nch = value ? cv : ck;
+      chunk = i % nch;
+      i /= nch;
     }
-    __syncthreads();
-    float C = 0.f, W = 0.f;  // ordered scalar sums of the block (same in every thread)
-    for (int j = 0; j < cnt; ++j) {
-      C += m_c0[j];
-      W += m_c1[j];
-    }
-    const int slot = nblocks > 1 ? s_slot : 0;
-    const bool slot_ok = nblocks == 1 || slot < s.pool_cap;
-    float *part_out = s.partial + (size_t)slot * s.pwidth;
-    for (int cb = 0; cb < n4; cb += CB) {
-      float4 r[4][Q4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = warp + kApplyWarps * u;
-        if (j < cnt) load_row<Q4>(source_row(d, s, value, m_srow[j]), cb, n4, r[u]);
-      }
-      float4 acc[Q4];
-#pragma unroll
-      for (int q = 0; q < Q4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = warp + kApplyWarps * u;
-        if (j < cnt) {
-#pragma unroll
-          for (int q = 0; q < Q4; ++q) fma4(acc[q], m_coef[j], r[u][q]);
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < Q4; ++q) red[warp][lane + 32 * q] = acc[q];
-      __syncthreads();
-      if (tid < CB && cb + tid < n4) {
-        const int c4 = cb + tid;
-        float4 tot = red[0][tid];
-#pragma unroll
-        for (int w = 1; w < kApplyWarps; ++w) add4(tot, red[w][tid]);
-        if (nblocks == 1) {
-          if (!value || C > 0.f) {
-            const float4 t = *reinterpret_cast<const float4 *>(dst + 4 * c4);
-            *reinterpret_cast<float4 *>(dst + 4 * c4) = updated(d, value, t, tot, C);
-          }
-        } else if (slot_ok) {
-          *reinterpret_cast<float4 *>(part_out + 4 + 4 * c4) = tot;
-          __threadfence();  // visible before the group's arrival count moves
-        }
-      }
-      __syncthreads();
-    }
-    if (nblocks == 1) {
-      if (value && d.lam != 0.f && tid < cnt) s.pb[m_id[tid]] = entropy_term(d, W);
-      __syncthreads();
-      continue;
-    }
-    // longer group: publish the partial; the group's last block combines
-    if (tid == 0) {
-      if (slot_ok) {
-        part_out[0] = C;
-        part_out[1] = W;
-      }
-      s.slotmap[x] = slot_ok ? slot : -1;
-      __threadfence();
-      s_last = atomicAdd(&s.segcnt[g0], 1) == nblocks - 1;
-    }
-    __syncthreads();
-    if (s_last) {
-      __threadfence();
-      float Ct = 0.f, Wt = 0.f;
-      bool all_ok = true;
-      for (int b = 0; b < nblocks; ++b) {
-        const int sl = __ldcg(&s.slotmap[g0 + b * kBlock]);
-        if (sl < 0) {
-          all_ok = false;
-          continue;
-        }
-        const float *pp = s.partial + (size_t)sl * s.pwidth;
-        Ct += __ldcg(pp);
-        Wt += __ldcg(pp + 1);
-      }
-      for (int c4 = tid; c4 < n4 && all_ok; c4 += blockDim.x) {
-        float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int b = 0; b < nblocks; ++b) {
-          const float *pp =
-              s.partial + (size_t)__ldcg(&s.slotmap[g0 + b * kBlock]) * s.pwidth;
-          add4(tot, __ldcg(reinterpret_cast<const float4 *>(pp + 4 + 4 * c4)));
-        }
-        if (!value || Ct > 0.f) {
-          const float4 t = *reinterpret_cast<const float4 *>(dst + 4 * c4);
-          *reinterpret_cast<float4 *>(dst + 4 * c4) = updated(d, value, t, tot, Ct);
-        }
-      }
-      if (value && d.lam != 0.f && all_ok) {
-        const float bt = entropy_term(d, Wt);
-        for (int j = tid; j < len; j += blockDim.x) s.pb[s.rec[g0 + j].id] = bt;
-      }
-      if (tid == 0) s.segcnt[g0] = 0;  // ready for the next chunk
-    }
-    __syncthreads();
-  }
-
-  // ---------------- phase B: groups of <= kShortMax members, a warp each ----------------
-  // Lane j holds member j's record; the members' rows are summed in member
-  // order, kU rows in flight, for every column block of the target row.
-  constexpr int kU = 4;
-  const int nshort = s.meta->nshort;
-  for (int it = blockIdx.x * kApplyWarps + warp; it < nshort; it += gridDim.x * kApplyWarps) {
-    const int x = s.shortlist[it];
+    const int x = block ? s.longlist[kind][i] : s.shortlist[kind][i];
     Member mj{};
-    if ((int64_t)x + lane < s.Lcap) mj = load_member(s.rec + x + lane);  // past the group: unused
+    if ((int64_t)x + lane < s.Lcap) mj = load_member(s.rec + x + lane);  // past the item: unused
     const uint32_t g = __shfl_sync(FULL, mj.g, 0);
+    const int g0 = __shfl_sync(FULL, mj.gstart, 0);
     const int len = __shfl_sync(FULL, mj.glen, 0);
-    if (!wanted(g)) continue;
-    const bool value = g < (uint32_t)d.N;
+    const int cnt = block ? min(kBlock, g0 + len - x) : len;
     float coef = 0.f, c0 = 0.f, c1 = 0.f;
-    if (lane < len) {
+    if (lane < cnt) {
       coef = mj.coef;
       c0 = mj.c0;
       c1 = mj.c1;
@@ -663,58 +700,112 @@ __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__res
       W += __shfl_xor_sync(FULL, W, o);
     }
     const int n4 = (value ? d.dv : d.dh) >> 2;
-    float *dst = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.N) * d.dh;
-    const bool write = !value || C > 0.f;
-    for (int cb = 0; cb < n4 && write; cb += CB) {
-      float4 t[Q4], acc[Q4];
-      load_row<Q4>(dst, cb, n4, t);
-#pragma unroll
-      for (int q = 0; q < Q4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int j0 = 0; j0 < len; j0 += kU) {
-        float4 r[kU][Q4];
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int sr = __shfl_sync(FULL, mj.srow, (j0 + u) & 31);
-          if (j0 + u < len) load_row<Q4>(source_row(d, s, value, sr), cb, n4, r[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const float cj = __shfl_sync(FULL, coef, (j0 + u) & 31);
-          if (j0 + u < len) {
-#pragma unroll
-            for (int q = 0; q < Q4; ++q) fma4(acc[q], cj, r[u][q]);
-          }
-        }
+    if (block) {
+      // one column chunk of a longer group's block, into its partial slot
+      const int slot = (value ? 0 : kslot0) + i;
+      if (slot >= s.pool_cap) {  // cannot happen: the pool holds Lcap / 4 + 2 blocks
+        if (lane == 0) atomicOr(&s.meta->err, ERR_POOL_OVERFLOW);
+        continue;
       }
-#pragma unroll
-      for (int q = 0; q < Q4; ++q) {
-        const int c4 = cb + lane + 32 * q;
-        if (c4 < n4) *reinterpret_cast<float4 *>(dst + 4 * c4) = updated(d, value, t[q], acc[q], C);
+      float *dst = s.partial + (size_t)slot * s.pwidth;
+      if (chunk == 0 && lane == 0) {
+        dst[0] = C;
+        dst[1] = W;
+      }
+      float4 acc[1];
+      const int cb = chunk * kChunk4;
+      sum_members<1, kU>(d, s, value, cnt, mj.srow, coef, cb, n4, acc);
+      if (cb + lane < n4) *reinterpret_cast<float4 *>(dst + 4 + 4 * (cb + lane)) = acc[0];
+      continue;
+    }
+    // a short group: the whole row, two column chunks at a time
+    float *dst = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.N) * d.dh;
+    if (!value || C > 0.f) {
+      for (int cb = 0; cb < n4; cb += 2 * kChunk4) {
+        const float4 t0 = load_chunk(dst, cb + lane, n4);
+        const float4 t1 = load_chunk(dst, cb + lane + 32, n4);
+        float4 acc[2];
+        sum_members<2, 2>(d, s, value, cnt, mj.srow, coef, cb, n4, acc);
+        if (cb + lane < n4)
+          *reinterpret_cast<float4 *>(dst + 4 * (cb + lane)) = updated(d, value, t0, acc[0], C);
+        if (cb + lane + 32 < n4)
+          *reinterpret_cast<float4 *>(dst + 4 * (cb + lane + 32)) =
+              updated(d, value, t1, acc[1], C);
       }
     }
     if (value && d.lam != 0.f && lane < len) s.pb[mj.id] = entropy_term(d, W);
   }
 }
 
-template <int Q4>
-static cudaError_t launch_apply_t(const Dims &d, float *V, float *K, const Scratch &s,
-                                  cudaStream_t st, int part) {
-  static int per_sm = 0;
-  if (!per_sm) {
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_apply<Q4>, kApplyThreads, 0);
-    if (per_sm < 1) per_sm = 1;
+__global__ void __launch_bounds__(kApplyThreads) k_combine(Dims d, float *__restrict__ V,
+                                                           float *__restrict__ K, Scratch s,
+                                                           int part) {
+  griddep_wait();
+  griddep_launch();
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * kApplyWarps + (threadIdx.x >> 5);
+  const int nw = gridDim.x * kApplyWarps;
+  const int cv = (d.dv / 4 + kChunk4 - 1) / kChunk4, ck = (d.dh / 4 + kChunk4 - 1) / kChunk4;
+  const int ngv = part != 2 ? s.meta->ngroup[0] * cv : 0;
+  const int ngk = part != 1 ? s.meta->ngroup[1] * ck : 0;
+  const int kslot0 = s.meta->nlong[0];
+  for (int it = gw; it < ngv + ngk; it += nw) {
+    const bool value = it < ngv;
+    const int kind = value ? 0 : 1;
+    const int nch = value ? cv : ck;
+    const int j = value ? it : it - ngv;
+    const int chunk = j % nch;
+    const int base = s.glist[kind][j / nch];
+    const int x = s.longlist[kind][base];  // the group's first member
+    const Member m0 = load_member(s.rec + x);
+    const int len = m0.glen, nb = (len + kBlock - 1) / kBlock;
+    const int slot0 = (value ? 0 : kslot0) + base;
+    if (slot0 + nb > s.pool_cap) continue;  // flagged by k_apply
+    const float *pp = s.partial + (size_t)slot0 * s.pwidth;
+    float C = 0.f, W = 0.f;  // block order
+    for (int b = 0; b < nb; ++b) {
+      C += pp[(size_t)b * s.pwidth];
+      W += pp[(size_t)b * s.pwidth + 1];
+    }
+    const int n4 = (value ? d.dv : d.dh) >> 2;
+    const int c4 = chunk * kChunk4 + lane;
+    float *dst = value ? V + (int64_t)m0.g * d.dv : K + (int64_t)(m0.g - (uint32_t)d.N) * d.dh;
+    if (!value || C > 0.f) {
+      const float4 t = load_chunk(dst, c4, n4);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int b0 = 0; b0 < nb; b0 += kU) {
+        float4 r[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+          r[u] = b0 + u < nb ? load_chunk(pp + (size_t)(b0 + u) * s.pwidth + 4, c4, n4)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+          if (b0 + u < nb) add4(acc, r[u]);
+      }
+      if (c4 < n4) *reinterpret_cast<float4 *>(dst + 4 * c4) = updated(d, value, t, acc, C);
+    }
+    if (chunk == 0 && value && d.lam != 0.f) {
+      const float bt = entropy_term(d, W);
+      for (int q = lane; q < len; q += 32) s.pb[s.rec[x + q].id] = bt;
+    }
   }
-  return launch_k(d.pdl, k_apply<Q4>, d.sm_count * per_sm, kApplyThreads, 0, st, d, V, K, s,
-                  part);
 }
 
 cudaError_t launch_apply(const Dims &d, float *V, float *K, const Scratch &s, cudaStream_t st,
                          int part) {
-  // rows up to 128 floats in one column block; wider rows in blocks of 256
-  // (2 float4 per lane keeps kU source rows in flight without spilling)
-  const int w4 = ((d.dv > d.dh ? d.dv : d.dh) / 4 + 31) / 32;
-  if (w4 <= 1) return launch_apply_t<1>(d, V, K, s, st, part);
-  return launch_apply_t<2>(d, V, K, s, st, part);
+  static int per_sm = 0, per_sm_c = 0;
+  if (!per_sm) {
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_apply, kApplyThreads, 0);
+    if (per_sm < 1) per_sm = 1;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_c, k_combine, kApplyThreads, 0);
+    if (per_sm_c < 1) per_sm_c = 1;
+  }
+  cudaError_t e =
+      launch_k(d.pdl, k_apply, d.sm_count * per_sm, kApplyThreads, 0, st, d, V, K, s, part);
+  if (e != cudaSuccess) return e;
+  return launch_k(d.pdl, k_combine, d.sm_count * per_sm_c, kApplyThreads, 0, st, d, V, K, s,
+                  part);
 }
 
 // ---------------------------------------------------------------------------
