@@ -80,7 +80,7 @@ struct Scratch {
   int32_t *pclaim;  // [M*k] position inside the pair's bucket
   float *pa;        // [M*k] dL_mse/dw
   float *pb;        // [M*k] dL_addr/dw (lam > 0)
-  int32_t *esub;    // [2*M*k] sub-key row of entry e = (m*2+half)*k + idx
+  int32_t *esub;    // [2*M*k] sub-key row of entry e = (m*2+half)*k + idx; -1 past ecount
   uint32_t *emask;  // [2*M*k] pairs r of token-head m that use that row
   float *einv;      // [2*M*k] 1 / (eps + d_half(row))
   int32_t *eclaim;  // [2*M*k] position inside the entry's bucket

@@ -40,13 +40,15 @@ struct ReadPlan {
 };
 
 // Dynamic shared memory layout (bytes):
-//   [0, 16)               mbarrier
-//   [128, 128 + R)        staged rows of this CTA, R = per*dv*4 (staged only)
-//   then ypart, e         dv floats each (ypart is read by the whole cluster)
-//   then w, slot, a, dl   H*k each (a is read by the whole cluster)
+//   [0, 16)                      mbarrier
+//   [128, 128 + R)               staged rows of this CTA, R = per*dv*4 (staged only)
+//   then ypart, e                dv floats each (ypart is read by the whole cluster)
+//   then w, slot, a, dl, claim   H*k each (a is read by the whole cluster)
+//   then esub, eclaim, emask, einv   2*H*k each (this CTA's entries only)
 static size_t read_smem_bytes(const Dims &d, int per, bool staged) {
   const size_t HK = (size_t)d.H * d.k;
-  return 128 + (staged ? (size_t)per * d.dv * 4 : 0) + 2 * (size_t)d.dv * 4 + HK * 16;
+  return 128 + (staged ? (size_t)per * d.dv * 4 : 0) + 2 * (size_t)d.dv * 4 + HK * 20 +
+         2 * HK * 16;
 }
 
 static ReadPlan read_plan(const Dims &d) {
@@ -115,6 +117,11 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   int *slot_s = reinterpret_cast<int *>(w_s + HK);
   float *a_s = reinterpret_cast<float *>(slot_s + HK);
   float *dl_s = a_s + HK;
+  int *claim_s = reinterpret_cast<int *>(dl_s + HK);
+  int *esub_s = claim_s + HK;
+  int *eclaim_s = esub_s + 2 * HK;
+  unsigned *emask_s = reinterpret_cast<unsigned *>(eclaim_s + 2 * HK);
+  float *einv_s = reinterpret_cast<float *>(emask_s + 2 * HK);
 
   const int rank = G > 1 ? (int)cluster_rank() : 0;
   const int row = blockIdx.x / G;
@@ -124,9 +131,20 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   const int64_t tok = (int64_t)b * d.T + d.t0 + tl;
   const int64_t p0 = (int64_t)row * HK;
 
+  // Everything that does not depend on the rows is loaded at once: the
+  // token's pairs, this CTA's entries (x = rank mod G), the gate and the
+  // target row.
   for (int j = tid; j < HK; j += blockDim.x) {
     w_s[j] = s.pw[p0 + j];
     slot_s[j] = s.pslot[p0 + j];
+    claim_s[j] = s.pclaim[p0 + j];
+  }
+  const int64_t e0 = (int64_t)row * 2 * HK;  // entries of this row: e0 + (h*2 + half)*k + idx
+  for (int x = rank + G * tid; x < 2 * HK; x += G * blockDim.x) {
+    esub_s[x] = s.esub[e0 + x];
+    eclaim_s[x] = s.eclaim[e0 + x];
+    emask_s[x] = s.emask[e0 + x];
+    einv_s[x] = s.einv[e0 + x];
   }
   if (kStaged && tid == 0) mbar_init(bar, 1);
   __syncthreads();
@@ -139,6 +157,14 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   }
   const float g = gate[tok];
   const float invH = 1.f / (float)d.H;
+  // the token's target row, loaded now so that it is here when e is formed
+  constexpr int kVt = 4;  // float4 per thread held (dv <= 4 * 4 * kReadThreads)
+  float4 vt[kVt];
+#pragma unroll
+  for (int q = 0; q < kVt; ++q) {
+    const int c4 = tid + q * kReadThreads;
+    vt[q] = c4 < dv4 ? load4(Vt, tok * dv + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 
   // Member records go to their buckets while the gather is in flight (none
   // of their fields depends on the rows): this CTA's pairs -> value bucket
@@ -157,14 +183,13 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
     m.c0 = w * invH;
     m.c1 = w;
     m.glen = 0;
-    s.rec_in[s.boff[slot_s[j] >> d.vshift] + s.pclaim[p]] = m;
+    s.rec_in[s.boff[slot_s[j] >> d.vshift] + claim_s[j]] = m;
   }
   for (int x = rank + G * tid; x < 2 * HK; x += G * blockDim.x) {
-    const int mh = x / d.k, idx = x % d.k;  // entry (h*2 + half)*k + idx of this row
-    const int64_t mhg = (int64_t)row * 2 * d.H + mh;
-    if (idx < s.ecount[mhg]) {
-      const int64_t e = mhg * d.k + idx;
-      const int sub = s.esub[e];
+    const int mh = x / d.k;  // entry (h*2 + half)*k + idx of this row
+    const int sub = esub_s[x];
+    if (sub >= 0) {
+      const int64_t e = e0 + x;
       Member m;
       m.g = (uint32_t)d.N + (uint32_t)(mh * d.n + sub);
       m.id = (uint32_t)e;
@@ -174,7 +199,7 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
       m.c0 = 0.f;
       m.c1 = 0.f;
       m.glen = 0;
-      s.rec_in[s.boff[d.NBv + mh * d.n + sub] + s.eclaim[e]] = m;
+      s.rec_in[s.boff[d.NBv + mh * d.n + sub] + eclaim_s[x]] = m;
     }
   }
   // On a timeout the error bit is set and the CTA still takes every cluster
@@ -201,7 +226,10 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   else __syncthreads();
 
   // yhat = (partials added in rank order) / H, identical in every CTA
-  for (int c4 = tid; c4 < dv4; c4 += blockDim.x) {
+#pragma unroll
+  for (int q = 0; q < kVt; ++q) {
+    const int c4 = tid + q * kReadThreads;
+    if (c4 >= dv4) break;
     float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int r = 0; r < G; ++r) {
       const float4 v = G > 1 ? ld_peer4(peer_smem(ypart + 4 * c4, (uint32_t)r))
@@ -212,7 +240,7 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
       y.w += v.w;
     }
     y = make_float4(y.x * invH, y.y * invH, y.z * invH, y.w * invH);
-    const float4 t = load4(Vt, tok * dv + 4 * c4);
+    const float4 t = vt[q];
     const float4 e = make_float4(y.x - t.x, y.y - t.y, y.z - t.z, y.w - t.w);
     if (rank == 0) {
       *reinterpret_cast<float4 *>(out + tok * dv + 4 * c4) =
@@ -261,18 +289,15 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
     __syncthreads();
     // alpha of the entries x = rank (mod G) of this row, one thread each
     for (int x = rank + G * tid; x < 2 * HK; x += G * blockDim.x) {
-      const int mh = x / d.k, idx = x % d.k;  // mh = h*2 + half
-      const int64_t mhg = (int64_t)row * 2 * d.H + mh;
-      if (idx < s.ecount[mhg]) {
-        const int64_t e = mhg * d.k + idx;
-        unsigned mask = s.emask[e];
-        const float *dl = dl_s + (mh >> 1) * d.k;
+      if (esub_s[x] >= 0) {
+        unsigned mask = emask_s[x];
+        const float *dl = dl_s + (x / d.k >> 1) * d.k;  // head h = (h*2 + half) >> 1
         float sum = 0.f;
         while (mask) {
           sum += dl[__ffs(mask) - 1];
           mask &= mask - 1;
         }
-        s.ealpha[e] = s.einv[e] * sum;
+        s.ealpha[e0 + x] = einv_s[x] * sum;
       }
     }
     // no CTA leaves while another may still read its a values

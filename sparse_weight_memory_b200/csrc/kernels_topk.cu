@@ -268,6 +268,8 @@ __global__ void __launch_bounds__(128) k_topk(Dims d, Scratch s, Extras x) {
       s.einv[e] = 1.f / (eps + dist);
       s.eclaim[e] = atomicAdd(&s.bcnt[d.NBv + (h * 2 + half) * n + sub], 1);
     }
+    // unused entry slots of this half are marked -1
+    if (lane >= __popc(lb) && lane < k) s.esub[((int64_t)m * 2 + half) * k + lane] = -1;
     if (lane == 0) s.ecount[(int64_t)m * 2 + half] = __popc(lb);
   }
 }
