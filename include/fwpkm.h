@@ -155,6 +155,18 @@ fwpkm_status fwpkm_record_selection(fwpkm_state *s, int32_t *slots, float *weigh
 fwpkm_status fwpkm_force_selection(fwpkm_state *s, const int32_t *slots, const uint8_t *mask);
 
 /*
+ * fwpkm_set_graphs -- enable (default) or disable the replay of repeated calls
+ * as CUDA graphs.  When enabled, a fwpkm_step whose arguments (B, T, tensor
+ * pointers, dtypes, eta, lambda, the armed force/record buffers) repeat those
+ * of an earlier call -- the usual case of a training or serving loop over
+ * fixed buffers -- is captured the second time it is seen and replayed as one
+ * graph launch afterwards (at most 8 graphs per state, least recently used
+ * dropped).  The results are identical either way.  Graphs are dropped when
+ * the scratch grows or eps changes, and never used while profiling is on.
+ */
+fwpkm_status fwpkm_set_graphs(fwpkm_state *s, int enable);
+
+/*
  * Per-kernel timing.  With profiling on, fwpkm_step records a CUDA event pair
  * around every step of the chunk it enqueues (one kernel, or two for
  * fwpkm_apply: the member pass and the combine of longer groups) and launches

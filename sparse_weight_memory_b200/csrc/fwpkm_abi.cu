@@ -51,6 +51,31 @@ struct Timing {
 
 }  // namespace
 
+// Everything a call's enqueued work depends on besides the state's own
+// buffers: a call with the same key enqueues exactly the same kernels with
+// the same parameters, so it can replay a captured graph.
+struct StepKey {
+  int B, T, q_dtype, v_dtype;
+  const void *Q, *Vt;
+  const float *gate;
+  float *out;
+  float eta, lam;
+  Extras x;
+  bool operator==(const StepKey &o) const {
+    return B == o.B && T == o.T && q_dtype == o.q_dtype && v_dtype == o.v_dtype && Q == o.Q &&
+           Vt == o.Vt && gate == o.gate && out == o.out && eta == o.eta && lam == o.lam &&
+           x.force_slots == o.x.force_slots && x.force_mask == o.x.force_mask &&
+           x.rec_slots == o.x.rec_slots && x.rec_w == o.x.rec_w;
+  }
+};
+struct StepGraph {
+  StepKey key;
+  cudaGraphExec_t exec;
+  uint64_t last_use;
+};
+constexpr size_t kGraphCache = 8;
+constexpr size_t kGraphSeen = 16;
+
 struct fwpkm_state {
   int64_t N = 0;
   int n = 0, dq = 0, dh = 0, dv = 0, k = 0, chunk = 0, H = 0;
@@ -76,6 +101,12 @@ struct fwpkm_state {
   std::vector<cudaEvent_t> event_pool;
   double prof_ms[K_COUNT] = {};
   int64_t prof_n[K_COUNT] = {};
+  // replay of repeated calls as CUDA graphs
+  bool graphs = true;
+  cudaStream_t capture_stream = nullptr;
+  std::vector<StepGraph> graph_cache;   // at most kGraphCache, least recently used first out
+  std::vector<StepKey> graph_seen;      // keys met once, most recent last
+  uint64_t graph_tick = 0;
 };
 
 namespace {
@@ -98,6 +129,8 @@ int64_t value_buckets(int64_t N, int64_t P) {
   const int sh = value_shift(N, P);
   return (N + (1ll << sh) - 1) >> sh;
 }
+
+void clear_graphs(fwpkm_state *st);
 
 // Carve the scratch arena for `rows` token rows per chunk.
 fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
@@ -189,6 +222,7 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
     cudaDeviceSynchronize();
     cudaFree(st->arena);
   }
+  clear_graphs(st);  // captured graphs hold the old arena's addresses
   st->maps = maps;
   st->arena = arena;
   st->arena_bytes = total;
@@ -227,6 +261,102 @@ fwpkm_status run(fwpkm_state *st, int kind, cudaStream_t stream, F &&launch) {
 }
 
 bool is_dtype(int t) { return t == FWPKM_F32 || t == FWPKM_BF16; }
+
+// The chunk loop of one call: every kernel of every chunk, in order, on
+// `stream`.  No host synchronisation.
+fwpkm_status enqueue_chunks(fwpkm_state *st, int B, int T, const void *Q, int q_dtype,
+                            const void *Vtarget, int v_dtype, const float *gate, float eta,
+                            float lambda_entropy, float *out, const Extras &x,
+                            cudaStream_t stream) {
+  fwpkm_status rc = FWPKM_OK;
+
+  const Scratch &s = st->s;
+  const int n_chunks = (T + st->chunk - 1) / st->chunk;
+  for (int c = 0; c < n_chunks; ++c) {
+    Dims d{};
+    d.n = st->n;
+    d.dq = st->dq;
+    d.dh = st->dh;
+    d.dv = st->dv;
+    d.k = st->k;
+    d.H = st->H;
+    d.N = st->N;
+    d.B = B;
+    d.T = T;
+    d.t0 = c * st->chunk;
+    d.Tc = (T - d.t0 < st->chunk) ? T - d.t0 : st->chunk;
+    d.rows = B * d.Tc;
+    d.qstride = (int)st->cap_rows;
+    d.M = d.rows * st->H;
+    const int64_t cap_pairs = st->cap_rows * st->H * st->k;  // bcnt was sized for this
+    d.vshift = value_shift(st->N, cap_pairs);
+    d.NBv = (int)value_buckets(st->N, cap_pairs);
+    d.NB = d.NBv + 2 * st->H * st->n;
+    d.sm_count = st->sm_count;
+    d.pdl = st->profiling ? 0 : 1;  // per-kernel events need plain stream order
+    d.eps = st->eps;
+    d.eta = eta;
+    d.lam = lambda_entropy;
+    float *V = st->V, *K = st->K;
+    if ((rc = run(st, K_PREP, stream, [&] { return launch_prep(d, Q, q_dtype, K, s, stream); })))
+      return rc;
+    if ((rc = run(st, K_SCORE, stream, [&] { return launch_score(d, s, st->maps, stream); })))
+      return rc;
+    if ((rc = run(st, K_TOPK, stream, [&] { return launch_topk(d, s, x, stream); }))) return rc;
+    if ((rc = run(st, K_SCAN, stream, [&] { return launch_scan(d, s, stream); }))) return rc;
+    if ((rc = run(st, K_READ, stream, [&] {
+           return launch_read(d, V, Vtarget, v_dtype, gate, out, s, stream);
+         })))
+      return rc;
+    if ((rc = run(st, K_BSORT, stream, [&] { return launch_bsort(d, s, stream); }))) return rc;
+    if (lambda_entropy == 0.f) {
+      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, s, stream, 0); })))
+        return rc;
+    } else {
+      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, s, stream, 1); })))
+        return rc;
+      if ((rc = run(st, K_PGRAD, stream, [&] { return launch_pgrad(d, s, stream); }))) return rc;
+      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, s, stream, 2); })))
+        return rc;
+    }
+  }
+  return FWPKM_OK;
+}
+
+// Captures the chunk loop of `key` into an executable graph on the state's
+// own stream (the caller's stream may be the legacy default stream, which
+// cannot be captured).  Returns null when capture or instantiation fails.
+cudaGraphExec_t capture_chunks(fwpkm_state *st, const StepKey &key) {
+  if (!st->capture_stream &&
+      cudaStreamCreateWithFlags(&st->capture_stream, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaGetLastError();
+    st->capture_stream = nullptr;
+    return nullptr;
+  }
+  if (cudaStreamBeginCapture(st->capture_stream, cudaStreamCaptureModeRelaxed) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  const fwpkm_status rc =
+      enqueue_chunks(st, key.B, key.T, key.Q, key.q_dtype, key.Vt, key.v_dtype, key.gate, key.eta,
+                     key.lam, key.out, key.x, st->capture_stream);
+  cudaGraph_t graph = nullptr;
+  const cudaError_t e = cudaStreamEndCapture(st->capture_stream, &graph);
+  cudaGraphExec_t exec = nullptr;
+  if (rc == FWPKM_OK && e == cudaSuccess && graph &&
+      cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess)
+    exec = nullptr;
+  if (graph) cudaGraphDestroy(graph);
+  cudaGetLastError();  // a failed capture leaves nothing sticky behind
+  return exec;
+}
+
+void clear_graphs(fwpkm_state *st) {
+  for (auto &g : st->graph_cache) cudaGraphExecDestroy(g.exec);
+  st->graph_cache.clear();
+  st->graph_seen.clear();
+}
+
 
 }  // namespace
 
@@ -326,6 +456,8 @@ void fwpkm_state_free(fwpkm_state *st) {
     cudaEventDestroy(t.b);
   }
   for (auto e : st->event_pool) cudaEventDestroy(e);
+  clear_graphs(st);
+  if (st->capture_stream) cudaStreamDestroy(st->capture_stream);
   cudaFree(st->arena);
   cudaFree(st->stage);
   cudaFree(st->K);
@@ -337,6 +469,14 @@ fwpkm_status fwpkm_state_set_eps(fwpkm_state *st, float eps) {
   if (!st) return fail(FWPKM_EINVAL, "set_eps: state is NULL");
   if (!(eps > 0.f) || !std::isfinite(eps)) return fail(FWPKM_EINVAL, "set_eps: eps must be > 0");
   st->eps = eps;
+  clear_graphs(st);  // eps is a kernel parameter of the captured launches
+  return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_set_graphs(fwpkm_state *st, int enable) {
+  if (!st) return fail(FWPKM_EINVAL, "set_graphs: state is NULL");
+  st->graphs = enable != 0;
+  if (!st->graphs) clear_graphs(st);
   return FWPKM_OK;
 }
 
@@ -365,60 +505,50 @@ fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtyp
   fwpkm_status rc = ensure_scratch(st, rows_max);
   if (rc != FWPKM_OK) return rc;
   cudaStream_t stream = (cudaStream_t)stream_;
-  Extras x = st->x;
+  const Extras x = st->x;
   st->x = Extras{};  // armed extras apply to this step only
-
-  const Scratch &s = st->s;
-  const int n_chunks = (T + st->chunk - 1) / st->chunk;
-  for (int c = 0; c < n_chunks; ++c) {
-    Dims d{};
-    d.n = st->n;
-    d.dq = st->dq;
-    d.dh = st->dh;
-    d.dv = st->dv;
-    d.k = st->k;
-    d.H = st->H;
-    d.N = st->N;
-    d.B = B;
-    d.T = T;
-    d.t0 = c * st->chunk;
-    d.Tc = (T - d.t0 < st->chunk) ? T - d.t0 : st->chunk;
-    d.rows = B * d.Tc;
-    d.qstride = (int)st->cap_rows;
-    d.M = d.rows * st->H;
-    const int64_t cap_pairs = st->cap_rows * st->H * st->k;  // bcnt was sized for this
-    d.vshift = value_shift(st->N, cap_pairs);
-    d.NBv = (int)value_buckets(st->N, cap_pairs);
-    d.NB = d.NBv + 2 * st->H * st->n;
-    d.sm_count = st->sm_count;
-    d.pdl = st->profiling ? 0 : 1;  // per-kernel events need plain stream order
-    d.eps = st->eps;
-    d.eta = eta;
-    d.lam = lambda_entropy;
-    float *V = st->V, *K = st->K;
-    if ((rc = run(st, K_PREP, stream, [&] { return launch_prep(d, Q, q_dtype, K, s, stream); })))
-      return rc;
-    if ((rc = run(st, K_SCORE, stream, [&] { return launch_score(d, s, st->maps, stream); })))
-      return rc;
-    if ((rc = run(st, K_TOPK, stream, [&] { return launch_topk(d, s, x, stream); }))) return rc;
-    if ((rc = run(st, K_SCAN, stream, [&] { return launch_scan(d, s, stream); }))) return rc;
-    if ((rc = run(st, K_READ, stream, [&] {
-           return launch_read(d, V, Vtarget, v_dtype, gate, out, s, stream);
-         })))
-      return rc;
-    if ((rc = run(st, K_BSORT, stream, [&] { return launch_bsort(d, s, stream); }))) return rc;
-    if (lambda_entropy == 0.f) {
-      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, s, stream, 0); })))
-        return rc;
-    } else {
-      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, s, stream, 1); })))
-        return rc;
-      if ((rc = run(st, K_PGRAD, stream, [&] { return launch_pgrad(d, s, stream); }))) return rc;
-      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, s, stream, 2); })))
-        return rc;
+  if (!st->graphs || st->profiling)
+    return enqueue_chunks(st, B, T, Q, q_dtype, Vtarget, v_dtype, gate, eta, lambda_entropy, out,
+                          x, stream);
+  // A call that repeats an earlier call's arguments replays a CUDA graph of
+  // its whole chunk sequence (captured the second time the arguments are
+  // seen); anything else is launched kernel by kernel.
+  const StepKey key{B, T, q_dtype, v_dtype, Q, Vtarget, gate, out, eta, lambda_entropy, x};
+  for (auto &g : st->graph_cache) {
+    if (g.key == key) {
+      g.last_use = ++st->graph_tick;
+      const cudaError_t e = cudaGraphLaunch(g.exec, stream);
+      return e == cudaSuccess ? FWPKM_OK : cuda_fail(e, "step: graph launch");
     }
   }
-  return FWPKM_OK;
+  bool seen = false;
+  for (size_t i = 0; i < st->graph_seen.size(); ++i) {
+    if (st->graph_seen[i] == key) {
+      seen = true;
+      st->graph_seen.erase(st->graph_seen.begin() + (long)i);
+      break;
+    }
+  }
+  if (!seen) {
+    if (st->graph_seen.size() >= kGraphSeen) st->graph_seen.erase(st->graph_seen.begin());
+    st->graph_seen.push_back(key);
+    return enqueue_chunks(st, B, T, Q, q_dtype, Vtarget, v_dtype, gate, eta, lambda_entropy, out,
+                          x, stream);
+  }
+  cudaGraphExec_t exec = capture_chunks(st, key);
+  if (!exec)  // not capturable here: launch directly (reports any real error)
+    return enqueue_chunks(st, B, T, Q, q_dtype, Vtarget, v_dtype, gate, eta, lambda_entropy, out,
+                          x, stream);
+  if (st->graph_cache.size() >= kGraphCache) {
+    size_t lru = 0;
+    for (size_t i = 1; i < st->graph_cache.size(); ++i)
+      if (st->graph_cache[i].last_use < st->graph_cache[lru].last_use) lru = i;
+    cudaGraphExecDestroy(st->graph_cache[lru].exec);
+    st->graph_cache.erase(st->graph_cache.begin() + (long)lru);
+  }
+  st->graph_cache.push_back(StepGraph{key, exec, ++st->graph_tick});
+  const cudaError_t e = cudaGraphLaunch(exec, stream);
+  return e == cudaSuccess ? FWPKM_OK : cuda_fail(e, "step: graph launch");
 }
 
 fwpkm_status fwpkm_step_host(fwpkm_state *st, int B, int T, const void *Q_host, int q_dtype,

@@ -55,6 +55,7 @@ def load_library():
     L.fwpkm_record_selection.argtypes = [_vp, _vp, _vp]
     L.fwpkm_force_selection.argtypes = [_vp, _vp, _vp]
     L.fwpkm_set_profiling.argtypes = [_vp, i32]
+    L.fwpkm_set_graphs.argtypes = [_vp, i32]
     L.fwpkm_profile_read.argtypes = [_vp, ctypes.POINTER(ctypes.c_char_p),
                                      ctypes.POINTER(ctypes.c_double), i64p, i32,
                                      ctypes.POINTER(i32), _vp]
@@ -63,7 +64,7 @@ def load_library():
     for name in ("fwpkm_state_init", "fwpkm_state_set_eps", "fwpkm_step", "fwpkm_step_host",
                  "fwpkm_state_get", "fwpkm_state_set", "fwpkm_record_selection",
                  "fwpkm_force_selection", "fwpkm_set_profiling", "fwpkm_profile_read",
-                 "fwpkm_read_stats", "fwpkm_select_noalloc"):
+                 "fwpkm_read_stats", "fwpkm_select_noalloc", "fwpkm_set_graphs"):
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -190,6 +191,10 @@ class FwPKMState:
                                                    _ptr(slots), _ptr(weights),
                                                    _stream(stream)))
         return slots, weights
+
+    def set_graphs(self, enable: bool):
+        """Replay repeated calls as CUDA graphs (default on)."""
+        _check(load_library().fwpkm_set_graphs(self._h, int(bool(enable))))
 
     # -- measurement -------------------------------------------------------
     def set_profiling(self, enable: bool):
