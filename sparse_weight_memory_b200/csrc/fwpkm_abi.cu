@@ -177,8 +177,8 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
       {(void **)&s.shortlist[1], sizeof(int32_t) * (size_t)Lcap},
       {(void **)&s.longlist[0], sizeof(int32_t) * (size_t)Lcap},
       {(void **)&s.longlist[1], sizeof(int32_t) * (size_t)Lcap},
-      {(void **)&s.glist[0], sizeof(int32_t) * (size_t)Lcap},
-      {(void **)&s.glist[1], sizeof(int32_t) * (size_t)Lcap},
+      {(void **)&s.glist[0], sizeof(int4) * (size_t)Lcap},
+      {(void **)&s.glist[1], sizeof(int4) * (size_t)Lcap},
       {(void **)&s.sort_tmp, sizeof(uint64_t) * (size_t)(2 * Lcap)},
       {(void **)&s.partial, sizeof(float) * (size_t)pool_cap * pwidth},
       {(void **)&s.E, sizeof(float) * (size_t)(rows * dv)},

@@ -95,7 +95,8 @@ struct Scratch {
   int32_t *shortlist[2];  // [Lcap] per kind: first position of every group of <= 4 members
   int32_t *longlist[2];   // [Lcap] per kind: first position of every 32-member block of a
                           //        longer group (a group's blocks are consecutive)
-  int32_t *glist[2];      // [Lcap] per kind: index in longlist of every longer group's first block
+  int4 *glist[2];         // [Lcap] per kind, one per longer group: {index in longlist of its
+                          //        first block, first position, row g, member count}
   float *partial;   // [pool_cap][pwidth] block partial sums: value blocks at their longlist
                     // index, sub-key blocks after all value blocks
                     // (zero between chunks)

@@ -204,18 +204,19 @@ constexpr int kShortMax = 4;  // groups up to this size are applied by one warp,
 constexpr int kBlock = 32;    // longer groups are applied in blocks of this many members
 
 // Work lists of the apply kernels for a group of kind `kind` (0: value row,
-// 1: sub-key row) that starts at position x0: a short group goes to
+// 1: sub-key row) of row g that starts at position x0: a short group goes to
 // shortlist, a longer one to longlist, one entry per block of kBlock members
-// (consecutive entries), plus its first block's index to glist.  Thread-level
-// (one call per group head).
-__device__ __forceinline__ void list_group(const Scratch &s, int kind, int x0, int len) {
+// (consecutive entries), plus {first block's index, x0, g, len} to glist.
+// Thread-level (one call per group head).
+__device__ __forceinline__ void list_group(const Scratch &s, int kind, int x0, int len,
+                                           uint32_t g) {
   if (len <= kShortMax) {
     s.shortlist[kind][atomicAdd(&s.meta->nshort[kind], 1)] = x0;
   } else {
     const int nb = (len + kBlock - 1) / kBlock;
     const int base = atomicAdd(&s.meta->nlong[kind], nb);
     for (int b = 0; b < nb; ++b) s.longlist[kind][base + b] = x0 + b * kBlock;
-    s.glist[kind][atomicAdd(&s.meta->ngroup[kind], 1)] = base;
+    s.glist[kind][atomicAdd(&s.meta->ngroup[kind], 1)] = make_int4(base, x0, (int)g, len);
   }
 }
 
@@ -310,7 +311,7 @@ __device__ bool rank_big_bucket(const Dims &d, const Scratch &s, int off, int le
     store_member(s.rec + off + pos, mr);
     if (pos == first) {
       my_seg += 1;
-      list_group(s, value ? 0 : 1, off + pos, mr.glen);
+      list_group(s, value ? 0 : 1, off + pos, mr.glen, mr.g);
     }
   }
   if (my_seg) atomicAdd(nseg, my_seg);
@@ -349,7 +350,7 @@ __device__ void sort_big_bucket(const Dims &d, const Scratch &s, int off, int le
       store_member(s.rec + off + i, m);
       if (first == i) {
         my_seg += 1;
-        list_group(s, value ? 0 : 1, off + i, end - first);
+        list_group(s, value ? 0 : 1, off + i, end - first, m.g);
       }
     }
   } else {
@@ -406,7 +407,7 @@ __device__ void sort_big_bucket(const Dims &d, const Scratch &s, int off, int le
       store_member(s.rec + off + i, m);
       if (first == i) {
         my_seg += 1;
-        list_group(s, value ? 0 : 1, off + i, end - first);
+        list_group(s, value ? 0 : 1, off + i, end - first, m.g);
       }
     }
   }
@@ -503,7 +504,7 @@ __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s)
     if (lg) {
       const int li = lbase + __popc(lb & lanemask_lt());
       s.longlist[kind][li] = off + lane;
-      s.glist[kind][gbase + __popc(lb & lanemask_lt())] = li;
+      s.glist[kind][gbase + __popc(lb & lanemask_lt())] = make_int4(li, off + lane, (int)r.g, glen);
     }
     if (lane == 0) atomicAdd(&nseg[b < d.NBv ? 0 : 1], __popc(heads));
   }
@@ -755,21 +756,29 @@ __global__ void __launch_bounds__(kApplyThreads) k_combine(Dims d, float *__rest
     const int nch = value ? cv : ck;
     const int j = value ? it : it - ngv;
     const int chunk = j % nch;
-    const int base = s.glist[kind][j / nch];
-    const int x = s.longlist[kind][base];  // the group's first member
-    const Member m0 = load_member(s.rec + x);
-    const int len = m0.glen, nb = (len + kBlock - 1) / kBlock;
+    const int4 grp = s.glist[kind][j / nch];  // first block, first position, row, count
+    const int base = grp.x, x = grp.y, len = grp.w, nb = (len + kBlock - 1) / kBlock;
+    const uint32_t g = (uint32_t)grp.z;
     const int slot0 = (value ? 0 : kslot0) + base;
     if (slot0 + nb > s.pool_cap) continue;  // flagged by k_apply
     const float *pp = s.partial + (size_t)slot0 * s.pwidth;
     float C = 0.f, W = 0.f;  // block order
-    for (int b = 0; b < nb; ++b) {
-      C += pp[(size_t)b * s.pwidth];
-      W += pp[(size_t)b * s.pwidth + 1];
+    for (int b0 = 0; b0 < nb; b0 += 4) {
+      float2 cw[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        cw[u] = b0 + u < nb ? *reinterpret_cast<const float2 *>(pp + (size_t)(b0 + u) * s.pwidth)
+                            : make_float2(0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (b0 + u < nb) {
+          C += cw[u].x;
+          W += cw[u].y;
+        }
     }
     const int n4 = (value ? d.dv : d.dh) >> 2;
     const int c4 = chunk * kChunk4 + lane;
-    float *dst = value ? V + (int64_t)m0.g * d.dv : K + (int64_t)(m0.g - (uint32_t)d.N) * d.dh;
+    float *dst = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.N) * d.dh;
     if (!value || C > 0.f) {
       const float4 t = load_chunk(dst, c4, n4);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
