@@ -221,9 +221,10 @@ def run_reference(args, wl):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
-def algorithmic_work(wl, tokens, value_rows, key_rows):
+def algorithmic_work(wl, tokens, value_rows, key_rows, records):
     """Algorithmic bytes (HBM-bound kernels) or flops (score) over `tokens`
-    tokens whose chunks wrote `value_rows` / `key_rows` distinct rows."""
+    tokens whose chunks wrote `value_rows` / `key_rows` distinct rows and
+    grouped `records` member records."""
     in_b = 2 if wl.in_dtype == BF16 else 4
     gather = tokens * wl.heads * wl.topk * wl.dv * 4
     return {
@@ -233,6 +234,8 @@ def algorithmic_work(wl, tokens, value_rows, key_rows):
         "fwpkm_apply": ("hbm", 2 * value_rows * wl.dv * 4 + 2 * key_rows * (wl.dq // 2) * 4),
         # q_half . K_row for every sub-key of both halves (fp32 products)
         "fwpkm_score": ("tensor", 2.0 * tokens * wl.heads * wl.n * wl.dq),
+        # member records read in claim order and written grouped (32 bytes each)
+        "fwpkm_bsort": ("hbm", 2 * 32 * records),
         # distance matrix read once, slots + weights written
         "fwpkm_topk": ("hbm", tokens * wl.heads * (2 * wl.n * 4 + wl.topk * 8)),
         # queries read once, split into hi/lo halves + norms written
@@ -392,7 +395,8 @@ def run_gpu(args, wl):
     if rank == 0:
         hbm_gbs, bf16_tf, peak_kind = peaks()
         rows_sum = wl.B * wl.T * wl.calls * wl.passes * prof_steps
-        work = algorithmic_work(wl, rows_sum, pstats["value_rows"], pstats["key_rows"])
+        work = algorithmic_work(wl, rows_sum, pstats["value_rows"], pstats["key_rows"],
+                                pstats["records"])
         traffic = NCU_TRAFFIC.get(wl.name, {})
         fracs = {k: kernel_roofline(k, work[k], ms, n, hbm_gbs, bf16_tf, peak_kind,
                                     traffic.get(k))

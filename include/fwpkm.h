@@ -183,15 +183,18 @@ fwpkm_status fwpkm_profile_read(fwpkm_state *s, const char **names, double *ms,
 /*
  * fwpkm_read_stats -- counters accumulated on the device since the last
  * reset (synchronises `stream`): chunks processed, and the sums over those
- * chunks of distinct value rows written and distinct sub-key rows written
- * (the write traffic of the step is proportional to these).  device_errors
- * receives the sticky device error bits (1 = a bounded wait in a kernel gave
- * up); when any is set the call returns FWPKM_ECUDA.  reset != 0 zeroes the
- * counters and the bits after reading.  Any output pointer may be NULL.
+ * chunks of distinct value rows written, distinct sub-key rows written and
+ * member records grouped (pairs plus sub-key entries; the write traffic of
+ * the step is proportional to these).  device_errors receives the sticky
+ * device error bits (1 = a bounded wait on a bulk copy gave up, 2 = the
+ * partial pool overflowed, 4 = a bucket-scan CTA gave up waiting for an
+ * earlier one); when any is set the call returns FWPKM_ECUDA.  reset != 0
+ * zeroes the counters and the bits after reading.  Any output pointer may be
+ * NULL.
  */
 fwpkm_status fwpkm_read_stats(fwpkm_state *s, int64_t *chunks, int64_t *value_rows,
-                              int64_t *key_rows, uint32_t *device_errors, int reset,
-                              void *stream);
+                              int64_t *key_rows, int64_t *records, uint32_t *device_errors,
+                              int reset, void *stream);
 
 /*
  * fwpkm_select_noalloc -- the product-key selection of the read, for callers

@@ -181,6 +181,7 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
       {(void **)&s.glist[1], sizeof(int4) * (size_t)Lcap},
       {(void **)&s.sort_tmp, sizeof(uint64_t) * (size_t)(2 * Lcap)},
       {(void **)&s.partial, sizeof(float) * (size_t)pool_cap * pwidth},
+      {(void **)&s.scan_sync, sizeof(unsigned long long) * (size_t)(1 + kScanMaxCtas)},
       {(void **)&s.E, sizeof(float) * (size_t)(rows * dv)},
       {(void **)&s.meta, sizeof(Meta)},
   };
@@ -205,6 +206,8 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
   // Bucket counts start at zero (the kernels leave them at zero); the meta
   // block (stats) carries over.
   e = cudaMemset(s.bcnt, 0, sizeof(int32_t) * (size_t)NB);
+  if (e == cudaSuccess)
+    e = cudaMemset(s.scan_sync, 0, sizeof(unsigned long long) * (size_t)(1 + kScanMaxCtas));
   if (e == cudaSuccess) e = cudaMemset(s.meta, 0, sizeof(Meta));
   if (e == cudaSuccess && st->s.meta)
     e = cudaMemcpy(s.meta, st->s.meta, sizeof(Meta), cudaMemcpyDeviceToDevice);
@@ -676,8 +679,8 @@ fwpkm_status fwpkm_profile_read(fwpkm_state *st, const char **names, double *ms,
 }
 
 fwpkm_status fwpkm_read_stats(fwpkm_state *st, int64_t *chunks, int64_t *value_rows,
-                              int64_t *key_rows, uint32_t *device_errors, int reset,
-                              void *stream) {
+                              int64_t *key_rows, int64_t *records, uint32_t *device_errors,
+                              int reset, void *stream) {
   if (!st) return fail(FWPKM_EINVAL, "read_stats: state is NULL");
   cudaStream_t s = (cudaStream_t)stream;
   Meta m{};
@@ -687,6 +690,7 @@ fwpkm_status fwpkm_read_stats(fwpkm_state *st, int64_t *chunks, int64_t *value_r
   if (chunks) *chunks = (int64_t)m.stat_chunks;
   if (value_rows) *value_rows = (int64_t)m.stat_value_rows;
   if (key_rows) *key_rows = (int64_t)m.stat_key_rows;
+  if (records) *records = (int64_t)m.stat_records;
   if (device_errors) *device_errors = m.err;
   if (reset) {
     Meta z{};
@@ -694,7 +698,11 @@ fwpkm_status fwpkm_read_stats(fwpkm_state *st, int64_t *chunks, int64_t *value_r
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "read_stats: reset");
   }
-  if (m.err) return fail(FWPKM_ECUDA, "device error bits 0x%x (1 = bounded wait timed out)", m.err);
+  if (m.err)
+    return fail(FWPKM_ECUDA,
+                "device error bits 0x%x (1 = bulk-copy wait timed out, 2 = partial pool "
+                "overflow, 4 = bucket-scan wait timed out)",
+                m.err);
   return FWPKM_OK;
 }
 

@@ -31,22 +31,25 @@ constexpr unsigned FULL = 0xffffffffu;
 enum : unsigned {
   ERR_MBAR_TIMEOUT = 1u,   // a bounded mbarrier wait gave up
   ERR_POOL_OVERFLOW = 2u,  // more long-group blocks than the partial pool holds
+  ERR_SCAN_TIMEOUT = 4u,   // a scan CTA gave up waiting for an earlier CTA's total
 };
 
 // Written by the kernels, read by later kernels and by the host.
 struct Meta {
   int32_t L;              // members of the chunk (pairs + sub-key entries)
-  int32_t Lv;             // pairs (value-row members come first)
+  int32_t pad1;
   unsigned err;           // ERR_* bits, sticky until the host clears them
   // Work lists of the chunk, per kind (0: value rows, 1: sub-key rows),
   // reset per chunk by the scan:
   int32_t nshort[2];      // groups of <= 4 members in shortlist[kind]
-  int32_t nlong[2];       // 32-member blocks of longer groups in longlist[kind]
-  int32_t ngroup[2];      // longer groups in glist[kind]
   int32_t pad2;
+  // longer groups: (groups in glist[kind] << 32) | (32-member blocks in
+  // longlist[kind]), advanced by one atomic per emitter
+  unsigned long long nlong[2];
   unsigned long long stat_chunks;      // chunks processed since reset
   unsigned long long stat_value_rows;  // sum over chunks of distinct value rows written
   unsigned long long stat_key_rows;    // sum over chunks of distinct sub-key rows written
+  unsigned long long stat_records;     // sum over chunks of member records (pairs + entries)
 };
 
 // Shapes of the chunk being processed.
@@ -66,6 +69,8 @@ struct Dims {
 };
 
 // Device scratch owned by the state (sized for the largest chunk seen).
+constexpr int kScanMaxCtas = 8;  // bucket-scan CTAs: 8 x 16384 buckets
+
 struct Scratch {
   float *Qs;        // [H][2][qstride][dh] query halves of the chunk, fp32 (may be null)
   float *Qs_hi;     // [H][2][qstride][dh] TF32-rounded query halves
@@ -97,6 +102,10 @@ struct Scratch {
                           //        longer group (a group's blocks are consecutive)
   int4 *glist[2];         // [Lcap] per kind, one per longer group: {index in longlist of its
                           //        first block, first position, row g, member count}
+  // Cross-CTA state of the bucket scan, never reset by the host: [0] the
+  // chunk epoch (advanced by the selection), [1 + c] CTA c's total tagged
+  // with the epoch it belongs to.
+  unsigned long long *scan_sync;  // [1 + kScanMaxCtas]
   float *partial;   // [pool_cap][pwidth] block partial sums: value blocks at their longlist
                     // index, sub-key blocks after all value blocks
                     // (zero between chunks)

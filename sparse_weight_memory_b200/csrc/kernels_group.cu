@@ -51,95 +51,140 @@ __device__ __forceinline__ void store_member(Member *p, const Member &m) {
 }
 
 // ---------------------------------------------------------------------------
-// scan: bucket offsets (single CTA).  The counts are staged in shared memory
-// with coalesced 16-byte loads, each thread scans a contiguous run there, and
-// the offsets go back with coalesced stores; pieces of kScanPiece buckets.
+// scan: bucket offsets, one pass over up to kScanMaxCtas CTAs.  Each CTA
+// holds kScanTile counts in registers (16-byte loads), scans them, publishes
+// its total tagged with the chunk's epoch, and adds the totals of the CTAs
+// before it (all CTAs of the grid are resident together: at most 8).  The
+// waits for those totals are bounded; a timeout sets ERR_SCAN_TIMEOUT.
+// Counts are zeroed for the next chunk; CTA 0 resets the work-list counters.
 // ---------------------------------------------------------------------------
 constexpr int kScanThreads = 1024;
-constexpr int kScanPiece = 8192;
+constexpr int kScanPer = 16;                        // counts per thread
+constexpr int kScanTile = kScanThreads * kScanPer;  // counts per CTA
+constexpr long long kScanSpinLimit = 1ll << 24;
+
+__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
 
 __global__ void __launch_bounds__(kScanThreads) k_bucket_scan(Dims d, Scratch s) {
   griddep_wait();
   griddep_launch();
-  __shared__ __align__(16) int cnt[kScanPiece];
   __shared__ int red[32];
-  __shared__ int carry_s;
-  const int NB = d.NB;
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  constexpr int per = kScanPiece / kScanThreads;  // 8 buckets per thread and piece
-  int carry = 0;
-  for (int p0 = 0; p0 < NB; p0 += kScanPiece) {
-    const int np = min(kScanPiece, NB - p0);
-    // bcnt and boff are 256-byte aligned; p0 is a multiple of 8192
-    for (int i = threadIdx.x * 4; i < np; i += kScanThreads * 4) {
-      if (i + 4 <= np) {
-        *reinterpret_cast<int4 *>(cnt + i) = *reinterpret_cast<const int4 *>(s.bcnt + p0 + i);
-        *reinterpret_cast<int4 *>(s.bcnt + p0 + i) = make_int4(0, 0, 0, 0);  // next chunk
-      } else {
-        for (int j = i; j < np; ++j) {
-          cnt[j] = s.bcnt[p0 + j];
-          s.bcnt[p0 + j] = 0;
-        }
-      }
-    }
-    __syncthreads();
-    const int b0 = threadIdx.x * per;
-    int v[per];
-    int total = 0;
+  __shared__ int prefix_s;
+  const int NB = d.NB, c = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const unsigned long long epoch = s.scan_sync[0];  // advanced by this chunk's selection
+  const int b0 = c * kScanTile + tid * kScanPer;
+  int v[kScanPer];
+  if (b0 + kScanPer <= NB) {  // bcnt is 256-byte aligned and b0 a multiple of 16
 #pragma unroll
-    for (int i = 0; i < per; ++i) {
-      v[i] = b0 + i < np ? cnt[b0 + i] : 0;
-      total += v[i];
+    for (int q = 0; q < kScanPer / 4; ++q) {
+      const int4 x = *reinterpret_cast<const int4 *>(s.bcnt + b0 + 4 * q);
+      v[4 * q] = x.x;
+      v[4 * q + 1] = x.y;
+      v[4 * q + 2] = x.z;
+      v[4 * q + 3] = x.w;
+      *reinterpret_cast<int4 *>(s.bcnt + b0 + 4 * q) = make_int4(0, 0, 0, 0);  // next chunk
     }
-    int incl = total;
+  } else {
+#pragma unroll
+    for (int i = 0; i < kScanPer; ++i) {
+      v[i] = b0 + i < NB ? s.bcnt[b0 + i] : 0;
+      if (b0 + i < NB) s.bcnt[b0 + i] = 0;
+    }
+  }
+  int total = 0;
+#pragma unroll
+  for (int i = 0; i < kScanPer; ++i) total += v[i];
+  int incl = total;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(FULL, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) red[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int x = red[lane];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(FULL, incl, o);
-      if (lane >= o) incl += t;
+      const int t = __shfl_up_sync(FULL, x, o);
+      if (lane >= o) x += t;
     }
-    if (lane == 31) red[w] = incl;
-    __syncthreads();
-    if (w == 0) {
-      int x = red[lane];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(FULL, x, o);
-        if (lane >= o) x += t;
+    red[lane] = x;
+  }
+  __syncthreads();
+  const int cta_total = red[31];
+  if (tid == 0 && gridDim.x > 1)
+    st_release_u64(&s.scan_sync[1 + c], (epoch << 32) | (unsigned)cta_total);
+  if (w == 0) {
+    int pre = 0;
+    if (lane < c) {
+      bool ok = false;
+      unsigned long long a = 0;
+      for (long long it = 0; it < kScanSpinLimit; ++it) {
+        a = ld_acquire_u64(&s.scan_sync[1 + lane]);
+        if ((a >> 32) == (epoch & 0xffffffffull)) {
+          ok = true;
+          break;
+        }
       }
-      red[lane] = x;
+      if (!ok) atomicOr(&s.meta->err, ERR_SCAN_TIMEOUT);
+      pre = ok ? (int)(unsigned)a : 0;
     }
-    __syncthreads();
-    int run = carry + (w > 0 ? red[w - 1] : 0) + incl - total;
 #pragma unroll
-    for (int i = 0; i < per; ++i) {
-      cnt[b0 + i] = run;  // exclusive offsets, in place
+    for (int o = 16; o > 0; o >>= 1) pre += __shfl_xor_sync(FULL, pre, o);
+    if (lane == 0) prefix_s = pre;
+  }
+  __syncthreads();
+  int run = prefix_s + (w > 0 ? red[w - 1] : 0) + incl - total;
+  if (b0 + kScanPer <= NB) {
+#pragma unroll
+    for (int q = 0; q < kScanPer / 4; ++q) {
+      int4 o;
+      o.x = run;
+      run += v[4 * q];
+      o.y = run;
+      run += v[4 * q + 1];
+      o.z = run;
+      run += v[4 * q + 2];
+      o.w = run;
+      run += v[4 * q + 3];
+      *reinterpret_cast<int4 *>(s.boff + b0 + 4 * q) = o;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kScanPer; ++i) {
+      if (b0 + i < NB) s.boff[b0 + i] = run;
       run += v[i];
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < np; i += kScanThreads) s.boff[p0 + i] = cnt[i];
-    if (threadIdx.x == 0) {
-      if (d.NBv >= p0 && d.NBv < p0 + np) s.meta->Lv = cnt[d.NBv - p0];
-      carry_s = carry + red[31];
-    }
-    __syncthreads();
-    carry = carry_s;
   }
-  if (threadIdx.x == 0) {
-    s.boff[NB] = carry;
-    s.meta->L = carry;
-    if (d.NBv >= NB) s.meta->Lv = carry;
+  if (tid == 0 && c == gridDim.x - 1) {
+    const int L = prefix_s + cta_total;
+    s.boff[NB] = L;
+    s.meta->L = L;
+    s.meta->stat_records += (unsigned long long)L;
+  }
+  if (tid == 0 && c == 0) {
     s.meta->stat_chunks += 1ull;
 #pragma unroll
     for (int kind = 0; kind < 2; ++kind) {
       s.meta->nshort[kind] = 0;
-      s.meta->nlong[kind] = 0;
-      s.meta->ngroup[kind] = 0;
+      s.meta->nlong[kind] = 0ull;
     }
   }
 }
 
 cudaError_t launch_scan(const Dims &d, const Scratch &s, cudaStream_t st) {
-  return launch_k(d.pdl, k_bucket_scan, 1, kScanThreads, 0, st, d, s);
+  const int ctas = (d.NB + kScanTile - 1) / kScanTile;
+  if (ctas > kScanMaxCtas) return cudaErrorInvalidValue;
+  return launch_k(d.pdl, k_bucket_scan, ctas, kScanThreads, 0, st, d, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -214,9 +259,10 @@ __device__ __forceinline__ void list_group(const Scratch &s, int kind, int x0, i
     s.shortlist[kind][atomicAdd(&s.meta->nshort[kind], 1)] = x0;
   } else {
     const int nb = (len + kBlock - 1) / kBlock;
-    const int base = atomicAdd(&s.meta->nlong[kind], nb);
+    const unsigned long long at = atomicAdd(&s.meta->nlong[kind], (1ull << 32) | (unsigned)nb);
+    const int base = (int)(unsigned)at;
     for (int b = 0; b < nb; ++b) s.longlist[kind][base + b] = x0 + b * kBlock;
-    s.glist[kind][atomicAdd(&s.meta->ngroup[kind], 1)] = make_int4(base, x0, (int)g, len);
+    s.glist[kind][(int)(at >> 32)] = make_int4(base, x0, (int)g, len);
   }
 }
 
@@ -431,8 +477,16 @@ __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s)
   // phase 1: small buckets, one warp each; large ones are listed.  Bucket b
   // goes to CTA b % gridDim.x: neighbouring buckets (slots of one popular
   // sub-key row) land in different CTAs.
-  for (int b = blockIdx.x + gridDim.x * wib; b < d.NB; b += stride) {
-    const int off = s.boff[b], len = s.boff[b + 1] - off;
+  // The offsets of a warp's next 32 buckets are loaded together, one per lane.
+  int nxt_off = 0, nxt_end = 0;
+  for (int b = blockIdx.x + gridDim.x * wib, i = 0; b < d.NB; b += stride, ++i) {
+    if ((i & 31) == 0) {
+      const int bl = b + lane * stride;
+      nxt_off = bl < d.NB ? s.boff[bl] : 0;
+      nxt_end = bl < d.NB ? s.boff[bl + 1] : 0;
+    }
+    const int off = __shfl_sync(FULL, nxt_off, i & 31);
+    const int len = __shfl_sync(FULL, nxt_end, i & 31) - off;
     if (len == 0) continue;
     if (len > 32) {
       if (lane == 0) {
@@ -493,8 +547,10 @@ __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s)
     if (lane == 0) {
       if (sb) sbase = atomicAdd(&s.meta->nshort[kind], __popc(sb));
       if (lb) {
-        lbase = atomicAdd(&s.meta->nlong[kind], __popc(lb));
-        gbase = atomicAdd(&s.meta->ngroup[kind], __popc(lb));
+        const unsigned long long at =
+            atomicAdd(&s.meta->nlong[kind], ((unsigned long long)__popc(lb) << 32) | __popc(lb));
+        lbase = (int)(unsigned)at;
+        gbase = (int)(at >> 32);
       }
     }
     sbase = __shfl_sync(FULL, sbase, 0);
@@ -653,11 +709,11 @@ __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__res
   // (one item per column chunk), then value groups and sub-key groups (one
   // item per group, whole rows), each present when `part` takes its kind
   // (0: both, 1: value rows, 2: sub-key rows).
-  const int nlv = part != 2 ? s.meta->nlong[0] * cv : 0;
-  const int nlk = part != 1 ? s.meta->nlong[1] * ck : 0;
+  const int nlv = part != 2 ? (int)(unsigned)s.meta->nlong[0] * cv : 0;
+  const int nlk = part != 1 ? (int)(unsigned)s.meta->nlong[1] * ck : 0;
   const int nsv = part != 2 ? s.meta->nshort[0] : 0;
   const int nsk = part != 1 ? s.meta->nshort[1] : 0;
-  const int kslot0 = s.meta->nlong[0];  // sub-key partial slots follow the value blocks
+  const int kslot0 = (int)(unsigned)s.meta->nlong[0];  // sub-key partial slots follow the value blocks
   const int total = nlv + nlk + nsv + nsk;
   for (int it = gw; it < total; it += nw) {
     int i = it, kind = 0;
@@ -747,9 +803,9 @@ __global__ void __launch_bounds__(kApplyThreads) k_combine(Dims d, float *__rest
   const int gw = blockIdx.x * kApplyWarps + (threadIdx.x >> 5);
   const int nw = gridDim.x * kApplyWarps;
   const int cv = (d.dv / 4 + kChunk4 - 1) / kChunk4, ck = (d.dh / 4 + kChunk4 - 1) / kChunk4;
-  const int ngv = part != 2 ? s.meta->ngroup[0] * cv : 0;
-  const int ngk = part != 1 ? s.meta->ngroup[1] * ck : 0;
-  const int kslot0 = s.meta->nlong[0];
+  const int ngv = part != 2 ? (int)(s.meta->nlong[0] >> 32) * cv : 0;
+  const int ngk = part != 1 ? (int)(s.meta->nlong[1] >> 32) * ck : 0;
+  const int kslot0 = (int)(unsigned)s.meta->nlong[0];
   for (int it = gw; it < ngv + ngk; it += nw) {
     const bool value = it < ngv;
     const int kind = value ? 0 : 1;

@@ -72,11 +72,22 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   return r;
 }
 // All threads of every CTA of the cluster; orders shared-memory writes before
-// the barrier with the other CTAs' reads after it.
+// the barrier with the other CTAs' reads after it.  The release waits for
+// every earlier write of the CTA, global stores included, so the kernel keeps
+// its global stores after the last such barrier.
 __device__ __forceinline__ void cluster_barrier() {
   asm volatile(
       "barrier.cluster.arrive.release.aligned;\n\t"
       "barrier.cluster.wait.acquire.aligned;" ::
+          : "memory");
+}
+// The same meeting point without ordering: only keeps every CTA's shared
+// memory alive until the others are done reading it (their loads have been
+// consumed before they arrive).
+__device__ __forceinline__ void cluster_barrier_relaxed() {
+  asm volatile(
+      "barrier.cluster.arrive.relaxed.aligned;\n\t"
+      "barrier.cluster.wait.aligned;" ::
           : "memory");
 }
 // Address of `p` (this CTA's shared memory) in CTA `rank` of the cluster.
@@ -225,29 +236,27 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   if (G > 1) cluster_barrier();
   else __syncthreads();
 
-  // yhat = (partials added in rank order) / H, identical in every CTA
+  // yhat = (partials added in rank order) / H, identical in every CTA; kept
+  // in registers (y, e) until the global stores at the end
+  float4 y[kVt], e[kVt];
 #pragma unroll
   for (int q = 0; q < kVt; ++q) {
     const int c4 = tid + q * kReadThreads;
-    if (c4 >= dv4) break;
-    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+    y[q] = e[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (c4 >= dv4) continue;
+    float4 yy = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int r = 0; r < G; ++r) {
       const float4 v = G > 1 ? ld_peer4(peer_smem(ypart + 4 * c4, (uint32_t)r))
                              : *reinterpret_cast<const float4 *>(ypart + 4 * c4);
-      y.x += v.x;
-      y.y += v.y;
-      y.z += v.z;
-      y.w += v.w;
+      yy.x += v.x;
+      yy.y += v.y;
+      yy.z += v.z;
+      yy.w += v.w;
     }
-    y = make_float4(y.x * invH, y.y * invH, y.z * invH, y.w * invH);
+    y[q] = make_float4(yy.x * invH, yy.y * invH, yy.z * invH, yy.w * invH);
     const float4 t = vt[q];
-    const float4 e = make_float4(y.x - t.x, y.y - t.y, y.z - t.z, y.w - t.w);
-    if (rank == 0) {
-      *reinterpret_cast<float4 *>(out + tok * dv + 4 * c4) =
-          make_float4(g * y.x, g * y.y, g * y.z, g * y.w);
-      *reinterpret_cast<float4 *>(s.E + (int64_t)row * dv + 4 * c4) = e;
-    }
-    *reinterpret_cast<float4 *>(e_s + 4 * c4) = e;
+    e[q] = make_float4(y[q].x - t.x, y[q].y - t.y, y[q].z - t.z, y[q].w - t.w);
+    *reinterpret_cast<float4 *>(e_s + 4 * c4) = e[q];
   }
   __syncthreads();
 
@@ -265,14 +274,27 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
       acc = fmaf(e.w, v.w, acc);
     }
     acc = warp_sum(acc);
-    if (lane == 0) {
-      s.pa[p0 + j] = coef * acc;
-      a_s[j] = coef * acc;
+    if (lane == 0) a_s[j] = coef * acc;
+  }
+  // Every CTA is done reading the partials; with the entropy term off the
+  // a values are published to the cluster for the alphas.
+  if (G > 1) {
+    if (d.lam == 0.f) cluster_barrier();
+    else cluster_barrier_relaxed();
+  }
+  __syncthreads();  // this CTA's a values, for its own stores below
+  // global stores: out and the residual (rank 0), dL/dw of this CTA's pairs
+  if (rank == 0) {
+#pragma unroll
+    for (int q = 0; q < kVt; ++q) {
+      const int c4 = tid + q * kReadThreads;
+      if (c4 >= dv4) continue;
+      *reinterpret_cast<float4 *>(out + tok * dv + 4 * c4) =
+          make_float4(g * y[q].x, g * y[q].y, g * y[q].z, g * y[q].w);
+      *reinterpret_cast<float4 *>(s.E + (int64_t)row * dv + 4 * c4) = e[q];
     }
   }
-  // every CTA is done reading the partials, and the a values are published
-  if (G > 1) cluster_barrier();
-  else __syncthreads();
+  for (int j = j0 + tid; j < j1; j += blockDim.x) s.pa[p0 + j] = a_s[j];
 
   // dL/ds and alpha per entry when the entropy term is off (dL/dw complete)
   if (d.lam == 0.f) {
@@ -301,7 +323,7 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
       }
     }
     // no CTA leaves while another may still read its a values
-    if (G > 1) cluster_barrier();
+    if (G > 1) cluster_barrier_relaxed();
   }
 }
 

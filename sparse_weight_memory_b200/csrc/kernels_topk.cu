@@ -161,6 +161,8 @@ __global__ void __launch_bounds__(128) k_topk(Dims d, Scratch s, Extras x) {
   const int m = blockIdx.x * 4 + wib;  // token-head m = row*H + h
   griddep_wait();
   griddep_launch();
+  // a new chunk epoch for the bucket scan that follows (the step, not the selection-only call)
+  if (!kSelectOnly && blockIdx.x == 0 && threadIdx.x == 0) s.scan_sync[0] += 1ull;
   if (m >= d.M) return;
   const int row = m / d.H, h = m % d.H;
   const int k = d.k, n = d.n;

@@ -59,7 +59,7 @@ def load_library():
     L.fwpkm_profile_read.argtypes = [_vp, ctypes.POINTER(ctypes.c_char_p),
                                      ctypes.POINTER(ctypes.c_double), i64p, i32,
                                      ctypes.POINTER(i32), _vp]
-    L.fwpkm_read_stats.argtypes = [_vp, i64p, i64p, i64p, u32p, i32, _vp]
+    L.fwpkm_read_stats.argtypes = [_vp, i64p, i64p, i64p, i64p, u32p, i32, _vp]
     L.fwpkm_select_noalloc.argtypes = [_vp, i32, i32, _vp, i32, _vp, _vp, _vp]
     for name in ("fwpkm_state_init", "fwpkm_state_set_eps", "fwpkm_step", "fwpkm_step_host",
                  "fwpkm_state_get", "fwpkm_state_set", "fwpkm_record_selection",
@@ -210,10 +210,10 @@ class FwPKMState:
         return {names[i].decode(): (ms[i], n[i]) for i in range(cnt.value)}
 
     def read_stats(self, reset: bool = False, stream=None) -> dict:
-        c, v, k = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        c, v, k, r = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
         err = ctypes.c_uint32()
         _check(load_library().fwpkm_read_stats(self._h, ctypes.byref(c), ctypes.byref(v),
-                                               ctypes.byref(k), ctypes.byref(err), int(reset),
-                                               _stream(stream)))
-        return {"chunks": c.value, "value_rows": v.value, "key_rows": k.value,
+                                               ctypes.byref(k), ctypes.byref(r), ctypes.byref(err),
+                                               int(reset), _stream(stream)))
+        return {"chunks": c.value, "value_rows": v.value, "key_rows": k.value, "records": r.value,
                 "device_errors": err.value}

@@ -67,7 +67,7 @@ def test_null_arguments_are_rejected(lib):
     assert lib.fwpkm_state_set_eps(None, 1e-3) == fwpkm.FWPKM_EINVAL
     assert lib.fwpkm_record_selection(None, None, None) == fwpkm.FWPKM_EINVAL
     assert lib.fwpkm_force_selection(None, None, None) == fwpkm.FWPKM_EINVAL
-    assert lib.fwpkm_read_stats(None, None, None, None, None, 0, None) == fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_read_stats(None, None, None, None, None, None, 0, None) == fwpkm.FWPKM_EINVAL
     lib.fwpkm_state_free(None)  # no-op
 
 
