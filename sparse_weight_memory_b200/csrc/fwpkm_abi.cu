@@ -40,9 +40,8 @@ fwpkm_status cuda_fail(cudaError_t e, const char *what) {
 enum Kind { K_PREP, K_SCORE, K_TOPK, K_SCAN, K_READ, K_BSORT, K_APPLY, K_PGRAD, K_COUNT };
 const char *kKindNames[K_COUNT] = {"fwpkm_prep", "fwpkm_score", "fwpkm_topk",  "fwpkm_scan",
                                    "fwpkm_read", "fwpkm_bsort", "fwpkm_apply", "fwpkm_pgrad"};
-// Kernels one call of a kind enqueues (the apply is a member pass plus the
-// combine of longer groups).
-const int kKernelsPerCall[K_COUNT] = {1, 1, 1, 1, 1, 1, 2, 1};
+// Kernels one call of a kind enqueues.
+const int kKernelsPerCall[K_COUNT] = {1, 1, 1, 1, 1, 1, 1, 1};
 
 struct Timing {
   int kind;
@@ -142,7 +141,7 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
   // Blocks of groups of more than 4 members, 32 members a block: at most
   // L/32 + L/5 of them, under L/4.
   const int64_t pool_cap = Lcap / 4 + 2;
-  const int pwidth = 4 + (int)(dv > dh ? dv : dh);
+  const int pwidth = kPartHead + (int)(dv > dh ? dv : dh);
   struct Piece {
     void **ptr;
     size_t bytes;
@@ -177,8 +176,7 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
       {(void **)&s.shortlist[1], sizeof(int32_t) * (size_t)Lcap},
       {(void **)&s.longlist[0], sizeof(int32_t) * (size_t)Lcap},
       {(void **)&s.longlist[1], sizeof(int32_t) * (size_t)Lcap},
-      {(void **)&s.glist[0], sizeof(int4) * (size_t)Lcap},
-      {(void **)&s.glist[1], sizeof(int4) * (size_t)Lcap},
+      {(void **)&s.arrive, sizeof(int32_t) * (size_t)pool_cap * kMaxChunks},
       {(void **)&s.sort_tmp, sizeof(uint64_t) * (size_t)(2 * Lcap)},
       {(void **)&s.partial, sizeof(float) * (size_t)pool_cap * pwidth},
       {(void **)&s.scan_sync, sizeof(unsigned long long) * (size_t)(1 + kScanMaxCtas)},
@@ -206,6 +204,7 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
   // Bucket counts start at zero (the kernels leave them at zero); the meta
   // block (stats) carries over.
   e = cudaMemset(s.bcnt, 0, sizeof(int32_t) * (size_t)NB);
+  if (e == cudaSuccess) e = cudaMemset(s.arrive, 0, sizeof(int32_t) * (size_t)pool_cap * kMaxChunks);
   if (e == cudaSuccess)
     e = cudaMemset(s.scan_sync, 0, sizeof(unsigned long long) * (size_t)(1 + kScanMaxCtas));
   if (e == cudaSuccess) e = cudaMemset(s.meta, 0, sizeof(Meta));

@@ -42,10 +42,8 @@ struct Meta {
   // Work lists of the chunk, per kind (0: value rows, 1: sub-key rows),
   // reset per chunk by the scan:
   int32_t nshort[2];      // groups of <= 4 members in shortlist[kind]
-  int32_t pad2;
-  // longer groups: (groups in glist[kind] << 32) | (32-member blocks in
-  // longlist[kind]), advanced by one atomic per emitter
-  unsigned long long nlong[2];
+  int32_t nlong[2];       // 32-member blocks of longer groups in longlist[kind]
+  int32_t pad2[2];
   unsigned long long stat_chunks;      // chunks processed since reset
   unsigned long long stat_value_rows;  // sum over chunks of distinct value rows written
   unsigned long long stat_key_rows;    // sum over chunks of distinct sub-key rows written
@@ -70,6 +68,8 @@ struct Dims {
 
 // Device scratch owned by the state (sized for the largest chunk seen).
 constexpr int kScanMaxCtas = 8;  // bucket-scan CTAs: 8 x 16384 buckets
+constexpr int kMaxChunks = 16;   // 128-float column chunks of the widest row (2048 floats)
+constexpr int kPartHead = 2 * kMaxChunks;  // partial slot header: (C, W) per column chunk
 
 struct Scratch {
   float *Qs;        // [H][2][qstride][dh] query halves of the chunk, fp32 (may be null)
@@ -100,19 +100,20 @@ struct Scratch {
   int32_t *shortlist[2];  // [Lcap] per kind: first position of every group of <= 4 members
   int32_t *longlist[2];   // [Lcap] per kind: first position of every 32-member block of a
                           //        longer group (a group's blocks are consecutive)
-  int4 *glist[2];         // [Lcap] per kind, one per longer group: {index in longlist of its
-                          //        first block, first position, row g, member count}
+  int32_t *arrive;        // [pool_cap][kMaxChunks] blocks of a longer group done with a
+                          //        column chunk, at the group's first block (reset to 0)
   // Cross-CTA state of the bucket scan, never reset by the host: [0] the
   // chunk epoch (advanced by the selection), [1 + c] CTA c's total tagged
   // with the epoch it belongs to.
   unsigned long long *scan_sync;  // [1 + kScanMaxCtas]
   float *partial;   // [pool_cap][pwidth] block partial sums: value blocks at their longlist
-                    // index, sub-key blocks after all value blocks
+                    // index, sub-key blocks after all value blocks; a header of
+                    // kPartHead floats (the block's scalar sums per column chunk), then the row
                     // (zero between chunks)
   float *E;         // [rows][dv] residual yhat - v
   Meta *meta;
   int64_t Lcap;     // member capacity (3 * M*k)
-  int pwidth;       // 4 + max(dv, dh) floats
+  int pwidth;       // kPartHead + max(dv, dh) floats
   int pool_cap;     // partial slots: Lcap / 4 + 2
 };
 

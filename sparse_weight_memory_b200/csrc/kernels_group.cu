@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(kScanThreads) k_bucket_scan(Dims d, Scratch s)
 #pragma unroll
     for (int kind = 0; kind < 2; ++kind) {
       s.meta->nshort[kind] = 0;
-      s.meta->nlong[kind] = 0ull;
+      s.meta->nlong[kind] = 0;
     }
   }
 }
@@ -248,21 +248,17 @@ __device__ __forceinline__ Member fetch_member(const Dims &d, const Scratch &s, 
 constexpr int kShortMax = 4;  // groups up to this size are applied by one warp, whole rows
 constexpr int kBlock = 32;    // longer groups are applied in blocks of this many members
 
-// Work lists of the apply kernels for a group of kind `kind` (0: value row,
-// 1: sub-key row) of row g that starts at position x0: a short group goes to
+// Work lists of the apply kernel for a group of kind `kind` (0: value row,
+// 1: sub-key row) that starts at position x0: a short group goes to
 // shortlist, a longer one to longlist, one entry per block of kBlock members
-// (consecutive entries), plus {first block's index, x0, g, len} to glist.
-// Thread-level (one call per group head).
-__device__ __forceinline__ void list_group(const Scratch &s, int kind, int x0, int len,
-                                           uint32_t g) {
+// (consecutive entries).  Thread-level (one call per group head).
+__device__ __forceinline__ void list_group(const Scratch &s, int kind, int x0, int len) {
   if (len <= kShortMax) {
     s.shortlist[kind][atomicAdd(&s.meta->nshort[kind], 1)] = x0;
   } else {
     const int nb = (len + kBlock - 1) / kBlock;
-    const unsigned long long at = atomicAdd(&s.meta->nlong[kind], (1ull << 32) | (unsigned)nb);
-    const int base = (int)(unsigned)at;
+    const int base = atomicAdd(&s.meta->nlong[kind], nb);
     for (int b = 0; b < nb; ++b) s.longlist[kind][base + b] = x0 + b * kBlock;
-    s.glist[kind][(int)(at >> 32)] = make_int4(base, x0, (int)g, len);
   }
 }
 
@@ -357,7 +353,7 @@ __device__ bool rank_big_bucket(const Dims &d, const Scratch &s, int off, int le
     store_member(s.rec + off + pos, mr);
     if (pos == first) {
       my_seg += 1;
-      list_group(s, value ? 0 : 1, off + pos, mr.glen, mr.g);
+      list_group(s, value ? 0 : 1, off + pos, mr.glen);
     }
   }
   if (my_seg) atomicAdd(nseg, my_seg);
@@ -396,7 +392,7 @@ __device__ void sort_big_bucket(const Dims &d, const Scratch &s, int off, int le
       store_member(s.rec + off + i, m);
       if (first == i) {
         my_seg += 1;
-        list_group(s, value ? 0 : 1, off + i, end - first, m.g);
+        list_group(s, value ? 0 : 1, off + i, end - first);
       }
     }
   } else {
@@ -453,7 +449,7 @@ __device__ void sort_big_bucket(const Dims &d, const Scratch &s, int off, int le
       store_member(s.rec + off + i, m);
       if (first == i) {
         my_seg += 1;
-        list_group(s, value ? 0 : 1, off + i, end - first, m.g);
+        list_group(s, value ? 0 : 1, off + i, end - first);
       }
     }
   }
@@ -543,25 +539,15 @@ __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s)
     const int kind = b < d.NBv ? 0 : 1;
     const bool sh = head && glen <= kShortMax, lg = head && glen > kShortMax;
     const unsigned sb = __ballot_sync(FULL, sh), lb = __ballot_sync(FULL, lg);
-    int sbase = 0, lbase = 0, gbase = 0;
+    int sbase = 0, lbase = 0;
     if (lane == 0) {
       if (sb) sbase = atomicAdd(&s.meta->nshort[kind], __popc(sb));
-      if (lb) {
-        const unsigned long long at =
-            atomicAdd(&s.meta->nlong[kind], ((unsigned long long)__popc(lb) << 32) | __popc(lb));
-        lbase = (int)(unsigned)at;
-        gbase = (int)(at >> 32);
-      }
+      if (lb) lbase = atomicAdd(&s.meta->nlong[kind], __popc(lb));
     }
     sbase = __shfl_sync(FULL, sbase, 0);
     lbase = __shfl_sync(FULL, lbase, 0);
-    gbase = __shfl_sync(FULL, gbase, 0);
     if (sh) s.shortlist[kind][sbase + __popc(sb & lanemask_lt())] = off + lane;
-    if (lg) {
-      const int li = lbase + __popc(lb & lanemask_lt());
-      s.longlist[kind][li] = off + lane;
-      s.glist[kind][gbase + __popc(lb & lanemask_lt())] = make_int4(li, off + lane, (int)r.g, glen);
-    }
+    if (lg) s.longlist[kind][lbase + __popc(lb & lanemask_lt())] = off + lane;
     if (lane == 0) atomicAdd(&nseg[b < d.NBv ? 0 : 1], __popc(heads));
   }
   __syncthreads();
@@ -601,20 +587,21 @@ cudaError_t launch_bsort(const Dims &d, const Scratch &s, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------------------
-// apply: the row updates, from the work lists bsort wrote, in two kernels.
-// The unit of work for longer groups is (block, column chunk of 128 floats),
-// one warp each, a float4 per lane: many short dependence chains rather than
-// a few long ones, whatever the skew.
-//   k_apply: a group of <= kShortMax members is summed and its whole row
-//     written at once (two chunks at a time); a column chunk of a block of
-//     kBlock members of a longer group is summed into the partial-pool slot
-//     of the block's work-list entry.  Lane j holds member
-//     j's record; the members' source rows (E rows for value rows, query
-//     halves for sub-key rows) are summed in member order, kU rows in flight.
-//   k_combine: for each (longer group, column chunk), adds the blocks'
+// apply: the row updates, from the work lists bsort wrote.  One warp per
+// work item:
+//   - a group of <= kShortMax members: its members are summed over whole rows
+//     (two column chunks at a time) and the row is written at once;
+//   - a column chunk (128 floats, a float4 per lane) of a block of kBlock
+//     members of a longer group: summed into the partial-pool slot of the
+//     block's work-list entry, with the block's scalar sums in the slot's
+//     header.  The last of a group's blocks to finish a chunk (an integer
+//     arrival counter per group and chunk, after a fence) adds the blocks'
 //     partials in block order and writes the row chunk.
-// Every sum runs in an order fixed by the data, whatever the scheduling, and
-// nothing is atomic but the work-list counters of the sort.
+// Lane j holds member j's record; the members' source rows (E rows for value
+// rows, query halves for sub-key rows) are summed in member order, kU rows in
+// flight.  Many short dependence chains rather than a few long ones, whatever
+// the skew.  Every sum runs in an order fixed by the data, whatever the
+// scheduling; nothing is atomic but integer counters.
 // ---------------------------------------------------------------------------
 constexpr int kApplyThreads = 256;
 constexpr int kApplyWarps = kApplyThreads / 32;
@@ -709,11 +696,11 @@ __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__res
   // (one item per column chunk), then value groups and sub-key groups (one
   // item per group, whole rows), each present when `part` takes its kind
   // (0: both, 1: value rows, 2: sub-key rows).
-  const int nlv = part != 2 ? (int)(unsigned)s.meta->nlong[0] * cv : 0;
-  const int nlk = part != 1 ? (int)(unsigned)s.meta->nlong[1] * ck : 0;
+  const int nlv = part != 2 ? s.meta->nlong[0] * cv : 0;
+  const int nlk = part != 1 ? s.meta->nlong[1] * ck : 0;
   const int nsv = part != 2 ? s.meta->nshort[0] : 0;
   const int nsk = part != 1 ? s.meta->nshort[1] : 0;
-  const int kslot0 = (int)(unsigned)s.meta->nlong[0];  // sub-key partial slots follow the value blocks
+  const int kslot0 = s.meta->nlong[0];  // sub-key partial slots follow the value blocks
   const int total = nlv + nlk + nsv + nsk;
   for (int it = gw; it < total; it += nw) {
     int i = it, kind = 0;
@@ -765,14 +752,60 @@ __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__res
         continue;
       }
       float *dst = s.partial + (size_t)slot * s.pwidth;
-      if (chunk == 0 && lane == 0) {
-        dst[0] = C;
-        dst[1] = W;
+      if (lane == 0) {
+        dst[2 * chunk] = C;
+        dst[2 * chunk + 1] = W;
       }
       float4 acc[1];
       const int cb = chunk * kChunk4;
       sum_members<1, kU>(d, s, value, cnt, mj.srow, coef, cb, n4, acc);
-      if (cb + lane < n4) *reinterpret_cast<float4 *>(dst + 4 + 4 * (cb + lane)) = acc[0];
+      if (cb + lane < n4)
+        *reinterpret_cast<float4 *>(dst + kPartHead + 4 * (cb + lane)) = acc[0];
+      // The last of the group's blocks to finish this chunk adds the blocks'
+      // partials in block order and writes the row chunk.
+      const int nb = (len + kBlock - 1) / kBlock;
+      const int slot0 = slot - (x - g0) / kBlock;  // the group's first block
+      __threadfence();
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) {
+        int *cnt_at = s.arrive + (size_t)slot0 * kMaxChunks + chunk;
+        last = atomicAdd(cnt_at, 1) == nb - 1;
+        if (last) *cnt_at = 0;  // ready for the next chunk
+      }
+      if (!__shfl_sync(FULL, last, 0)) continue;
+      __threadfence();
+      const float *pp = s.partial + (size_t)slot0 * s.pwidth;
+      float Ct = 0.f, Wt = 0.f;  // block order
+      for (int b = 0; b < nb; ++b) {
+        const float2 cw = __ldcg(reinterpret_cast<const float2 *>(pp + (size_t)b * s.pwidth +
+                                                                  2 * chunk));
+        Ct += cw.x;
+        Wt += cw.y;
+      }
+      float *row = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.N) * d.dh;
+      if (!value || Ct > 0.f) {
+        const int c4 = cb + lane;
+        const float4 t = load_chunk(row, c4, n4);
+        float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int b0 = 0; b0 < nb; b0 += kU) {
+          float4 r[kU];
+#pragma unroll
+          for (int u = 0; u < kU; ++u)
+            r[u] = b0 + u < nb && c4 < n4
+                       ? __ldcg(reinterpret_cast<const float4 *>(
+                             pp + (size_t)(b0 + u) * s.pwidth + kPartHead + 4 * c4))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int u = 0; u < kU; ++u)
+            if (b0 + u < nb) add4(tot, r[u]);
+        }
+        if (c4 < n4) *reinterpret_cast<float4 *>(row + 4 * c4) = updated(d, value, t, tot, Ct);
+      }
+      if (chunk == 0 && value && d.lam != 0.f) {
+        const float bt = entropy_term(d, Wt);
+        for (int q = lane; q < len; q += 32) s.pb[s.rec[g0 + q].id] = bt;
+      }
       continue;
     }
     // a short group: the whole row, two column chunks at a time
@@ -794,83 +827,14 @@ __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__res
   }
 }
 
-__global__ void __launch_bounds__(kApplyThreads) k_combine(Dims d, float *__restrict__ V,
-                                                           float *__restrict__ K, Scratch s,
-                                                           int part) {
-  griddep_wait();
-  griddep_launch();
-  const int lane = threadIdx.x & 31;
-  const int gw = blockIdx.x * kApplyWarps + (threadIdx.x >> 5);
-  const int nw = gridDim.x * kApplyWarps;
-  const int cv = (d.dv / 4 + kChunk4 - 1) / kChunk4, ck = (d.dh / 4 + kChunk4 - 1) / kChunk4;
-  const int ngv = part != 2 ? (int)(s.meta->nlong[0] >> 32) * cv : 0;
-  const int ngk = part != 1 ? (int)(s.meta->nlong[1] >> 32) * ck : 0;
-  const int kslot0 = (int)(unsigned)s.meta->nlong[0];
-  for (int it = gw; it < ngv + ngk; it += nw) {
-    const bool value = it < ngv;
-    const int kind = value ? 0 : 1;
-    const int nch = value ? cv : ck;
-    const int j = value ? it : it - ngv;
-    const int chunk = j % nch;
-    const int4 grp = s.glist[kind][j / nch];  // first block, first position, row, count
-    const int base = grp.x, x = grp.y, len = grp.w, nb = (len + kBlock - 1) / kBlock;
-    const uint32_t g = (uint32_t)grp.z;
-    const int slot0 = (value ? 0 : kslot0) + base;
-    if (slot0 + nb > s.pool_cap) continue;  // flagged by k_apply
-    const float *pp = s.partial + (size_t)slot0 * s.pwidth;
-    float C = 0.f, W = 0.f;  // block order
-    for (int b0 = 0; b0 < nb; b0 += 4) {
-      float2 cw[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        cw[u] = b0 + u < nb ? *reinterpret_cast<const float2 *>(pp + (size_t)(b0 + u) * s.pwidth)
-                            : make_float2(0.f, 0.f);
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (b0 + u < nb) {
-          C += cw[u].x;
-          W += cw[u].y;
-        }
-    }
-    const int n4 = (value ? d.dv : d.dh) >> 2;
-    const int c4 = chunk * kChunk4 + lane;
-    float *dst = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.N) * d.dh;
-    if (!value || C > 0.f) {
-      const float4 t = load_chunk(dst, c4, n4);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int b0 = 0; b0 < nb; b0 += kU) {
-        float4 r[kU];
-#pragma unroll
-        for (int u = 0; u < kU; ++u)
-          r[u] = b0 + u < nb ? load_chunk(pp + (size_t)(b0 + u) * s.pwidth + 4, c4, n4)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int u = 0; u < kU; ++u)
-          if (b0 + u < nb) add4(acc, r[u]);
-      }
-      if (c4 < n4) *reinterpret_cast<float4 *>(dst + 4 * c4) = updated(d, value, t, acc, C);
-    }
-    if (chunk == 0 && value && d.lam != 0.f) {
-      const float bt = entropy_term(d, W);
-      for (int q = lane; q < len; q += 32) s.pb[s.rec[x + q].id] = bt;
-    }
-  }
-}
-
 cudaError_t launch_apply(const Dims &d, float *V, float *K, const Scratch &s, cudaStream_t st,
                          int part) {
-  static int per_sm = 0, per_sm_c = 0;
+  static int per_sm = 0;
   if (!per_sm) {
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_apply, kApplyThreads, 0);
     if (per_sm < 1) per_sm = 1;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_c, k_combine, kApplyThreads, 0);
-    if (per_sm_c < 1) per_sm_c = 1;
   }
-  cudaError_t e =
-      launch_k(d.pdl, k_apply, d.sm_count * per_sm, kApplyThreads, 0, st, d, V, K, s, part);
-  if (e != cudaSuccess) return e;
-  return launch_k(d.pdl, k_combine, d.sm_count * per_sm_c, kApplyThreads, 0, st, d, V, K, s,
-                  part);
+  return launch_k(d.pdl, k_apply, d.sm_count * per_sm, kApplyThreads, 0, st, d, V, K, s, part);
 }
 
 // ---------------------------------------------------------------------------
