@@ -91,7 +91,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-// 2-D tiled TMA load (no multicast) of box {32 elements, rows} at {x, y}.
+// 2-D tiled TMA load, into this CTA's shared memory only, of box {32 elements, rows} at {x, y}.
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
                                             uint64_t *bar) {
   asm volatile(
