@@ -243,11 +243,17 @@ def algorithmic_work(wl, tokens, value_rows, key_rows, records):
     }
 
 
-# Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
-# kernels as last captured with ncu on the library workload, keyed by kernel;
-# the capture and its command are summarised in profiles/.  None = no capture
-# of the current kernel.
-NCU_TRAFFIC = {"library": {}}
+# Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, bytes)
+# of the kernels as last captured with ncu (cold caches), keyed by workload and
+# kernel; the captures and their commands are summarised in profiles/.
+# Missing = no capture of the current kernel.
+NCU_TRAFFIC = {
+    # library: captures of commit d6e5ae0 (fwpkm_score: b492536, kernel unchanged since)
+    "library": {"fwpkm_apply": 10.42e6, "fwpkm_bsort": 0.369e6, "fwpkm_topk": 1.134e6,
+                "fwpkm_score": 3.17e6},
+    # long-context shape, chunk 28 of a 32-chunk call (commit d6e5ae0)
+    "longctx": {"fwpkm_read": 12.95e6, "fwpkm_apply": 16.29e6},
+}
 
 
 def tensor_peak_tf32(bf16_tf):
@@ -269,9 +275,12 @@ def kernel_roofline(name, work, ms, launches, hbm_gbs, bf16_tf, peak_kind, traff
         achieved, peak, unit = per_launch / sec / 1e12, tensor_peak_tf32(bf16_tf), "TFLOP/s"
         note = (f"{peak_kind} bf16 x 1.1/2.25 (tf32); achieved counts fp32 products once, "
                 f"the 3xTF32 split issues 3 tf32 products each, so frac <= 1/3")
-    return {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-            "frac": achieved / peak, "traffic": traffic,
-            "algorithmic_per_launch": per_launch, "us_per_launch": sec * 1e6, "peak_kind": note}
+    out = {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+           "frac": achieved / peak, "traffic": traffic,
+           "algorithmic_per_launch": per_launch, "us_per_launch": sec * 1e6, "peak_kind": note}
+    if bound == "hbm":
+        out["frac_vs_nominal_8000"] = achieved / 8000.0  # HBM3e nominal, GB/s
+    return out
 
 
 def run_gpu(args, wl):
@@ -347,6 +356,26 @@ def run_gpu(args, wl):
     if world > 1:
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in times]
+    recall = None
+    if len(inp.plants):
+        # Planted recalls (a position repeating an earlier (q, v) pair): the
+        # squared error of the readout there against the planted target, next
+        # to the same at all other positions, from the last timed step.
+        pos = torch.from_numpy(inp.plants[:, 0]).to(dev)
+        err = []
+        for c in range(wl.calls):
+            o = outs[c * wl.passes + wl.passes - 1]
+            lo, hi = c * wl.T, (c + 1) * wl.T
+            sel = pos[(pos >= lo) & (pos < hi)] - lo
+            vt = torch.from_numpy(np.ascontiguousarray(inp.vt_f32()[:, lo:hi])).to(dev)
+            se = ((o - vt) ** 2).mean(dim=-1)  # [B, T]
+            mask = torch.zeros(wl.T, dtype=torch.bool, device=dev)
+            mask[sel] = True
+            err.append((se[:, mask].sum().item(), int(mask.sum().item()) * wl.B,
+                        se[:, ~mask].sum().item(), int((~mask).sum().item()) * wl.B))
+        recall = {"planted_mse": sum(e[0] for e in err) / max(1, sum(e[1] for e in err)),
+                  "other_mse": sum(e[2] for e in err) / max(1, sum(e[3] for e in err)),
+                  "planted_positions": int(sum(e[1] for e in err))}
     total_ms = sum(step_ms)
     stats = st.read_stats(reset=True)
     total_ms_max = max_over_ranks(total_ms, dev)
@@ -428,7 +457,9 @@ def run_gpu(args, wl):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
+            "ms_per_step": total_ms_max / args.steps,
+            "step_ms": {"median": statistics.median(step_ms), "best": min(step_ms)},
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": config_for(wl, world),
             "roofline": roofline,
@@ -441,6 +472,7 @@ def run_gpu(args, wl):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
+            "recall": recall,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
