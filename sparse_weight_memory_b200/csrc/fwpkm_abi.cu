@@ -100,6 +100,8 @@ struct fwpkm_state {
   std::vector<cudaEvent_t> event_pool;
   double prof_ms[K_COUNT] = {};
   int64_t prof_n[K_COUNT] = {};
+  // the TF32 split and chunk norms of the sub-key rows in the arena are out of date
+  bool subkey_split_stale = true;
   // replay of repeated calls as CUDA graphs
   bool graphs = true;
   cudaStream_t capture_stream = nullptr;
@@ -148,13 +150,12 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
   };
   Scratch s{};
   std::vector<Piece> pieces = {
-      {(void **)&s.Qs, sizeof(float) * (size_t)(H * 2 * rows * dh)},
       {(void **)&s.Qs_hi, sizeof(float) * (size_t)(H * 2 * rows * dh)},
       {(void **)&s.Qs_lo, sizeof(float) * (size_t)(H * 2 * rows * dh)},
       {(void **)&s.qn, sizeof(float) * (size_t)(H * 2 * rows)},
       {(void **)&s.K_hi, sizeof(float) * (size_t)((H * 2 * n + 128) * dh)},
       {(void **)&s.K_lo, sizeof(float) * (size_t)((H * 2 * n + 128) * dh)},
-      {(void **)&s.kn, sizeof(float) * (size_t)(H * 2 * n)},
+      {(void **)&s.kn, sizeof(float) * (size_t)(H * 2 * n * kKnChunks)},
       {(void **)&s.D, sizeof(float) * (size_t)(H * 2 * rows * n)},
       {(void **)&s.pslot, sizeof(int32_t) * (size_t)P},
       {(void **)&s.pw, sizeof(float) * (size_t)P},
@@ -230,6 +231,7 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
   st->arena_bytes = total;
   st->s = s;
   st->cap_rows = rows;
+  st->subkey_split_stale = true;  // the new arena holds no sub-key split yet
   return FWPKM_OK;
 }
 
@@ -264,6 +266,43 @@ fwpkm_status run(fwpkm_state *st, int kind, cudaStream_t stream, F &&launch) {
 
 bool is_dtype(int t) { return t == FWPKM_F32 || t == FWPKM_BF16; }
 
+// Shapes of chunk c of a call (B sequences of T tokens).
+Dims chunk_dims(const fwpkm_state *st, int B, int T, int c, float eta, float lambda_entropy) {
+  Dims d{};
+  d.n = st->n;
+  d.dq = st->dq;
+  d.dh = st->dh;
+  d.dv = st->dv;
+  d.k = st->k;
+  d.H = st->H;
+  d.N = st->N;
+  d.B = B;
+  d.T = T;
+  d.t0 = c * st->chunk;
+  d.Tc = (T - d.t0 < st->chunk) ? T - d.t0 : st->chunk;
+  d.rows = B * d.Tc;
+  d.qstride = (int)st->cap_rows;
+  d.M = d.rows * st->H;
+  const int64_t cap_pairs = st->cap_rows * st->H * st->k;  // bcnt was sized for this
+  d.vshift = value_shift(st->N, cap_pairs);
+  d.NBv = (int)value_buckets(st->N, cap_pairs);
+  d.NB = d.NBv + 2 * st->H * st->n;
+  d.sm_count = st->sm_count;
+  d.pdl = st->profiling ? 0 : 1;  // per-kernel events need plain stream order
+  d.eps = st->eps;
+  d.eta = eta;
+  d.lam = lambda_entropy;
+  return d;
+}
+
+// The TF32 split and chunk norms of every sub-key row (new tables or a new
+// scratch arena); afterwards the update keeps those of the rows it writes.
+fwpkm_status split_all_subkeys(fwpkm_state *st, cudaStream_t stream) {
+  Dims d = chunk_dims(st, 1, 1, 0, 0.f, 0.f);
+  d.pdl = 0;
+  return run(st, K_PREP, stream, [&] { return launch_prep_k(d, st->K, st->s, stream); });
+}
+
 // The chunk loop of one call: every kernel of every chunk, in order, on
 // `stream`.  No host synchronisation.
 fwpkm_status enqueue_chunks(fwpkm_state *st, int B, int T, const void *Q, int q_dtype,
@@ -275,32 +314,14 @@ fwpkm_status enqueue_chunks(fwpkm_state *st, int B, int T, const void *Q, int q_
   const Scratch &s = st->s;
   const int n_chunks = (T + st->chunk - 1) / st->chunk;
   for (int c = 0; c < n_chunks; ++c) {
-    Dims d{};
-    d.n = st->n;
-    d.dq = st->dq;
-    d.dh = st->dh;
-    d.dv = st->dv;
-    d.k = st->k;
-    d.H = st->H;
-    d.N = st->N;
-    d.B = B;
-    d.T = T;
-    d.t0 = c * st->chunk;
-    d.Tc = (T - d.t0 < st->chunk) ? T - d.t0 : st->chunk;
-    d.rows = B * d.Tc;
-    d.qstride = (int)st->cap_rows;
-    d.M = d.rows * st->H;
-    const int64_t cap_pairs = st->cap_rows * st->H * st->k;  // bcnt was sized for this
-    d.vshift = value_shift(st->N, cap_pairs);
-    d.NBv = (int)value_buckets(st->N, cap_pairs);
-    d.NB = d.NBv + 2 * st->H * st->n;
-    d.sm_count = st->sm_count;
-    d.pdl = st->profiling ? 0 : 1;  // per-kernel events need plain stream order
-    d.eps = st->eps;
-    d.eta = eta;
-    d.lam = lambda_entropy;
+    const Dims d = chunk_dims(st, B, T, c, eta, lambda_entropy);
+    // the next chunk of this call, whose query halves the sort prepares
+    Dims dn{};
+    if (c + 1 < n_chunks) dn = chunk_dims(st, B, T, c + 1, eta, lambda_entropy);
     float *V = st->V, *K = st->K;
-    if ((rc = run(st, K_PREP, stream, [&] { return launch_prep(d, Q, q_dtype, K, s, stream); })))
+    // the first chunk's query halves; later chunks' come with the previous sort
+    if (c == 0 &&
+        (rc = run(st, K_PREP, stream, [&] { return launch_prep_q(d, Q, q_dtype, s, stream); })))
       return rc;
     if ((rc = run(st, K_SCORE, stream, [&] { return launch_score(d, s, st->maps, stream); })))
       return rc;
@@ -310,15 +331,17 @@ fwpkm_status enqueue_chunks(fwpkm_state *st, int B, int T, const void *Q, int q_
            return launch_read(d, V, Vtarget, v_dtype, gate, out, s, stream);
          })))
       return rc;
-    if ((rc = run(st, K_BSORT, stream, [&] { return launch_bsort(d, s, stream); }))) return rc;
+    if ((rc = run(st, K_BSORT, stream,
+                  [&] { return launch_bsort(d, s, dn, Q, q_dtype, stream); })))
+      return rc;
     if (lambda_entropy == 0.f) {
-      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, s, stream, 0); })))
+      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, Q, q_dtype, s, stream, 0); })))
         return rc;
     } else {
-      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, s, stream, 1); })))
+      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, Q, q_dtype, s, stream, 1); })))
         return rc;
       if ((rc = run(st, K_PGRAD, stream, [&] { return launch_pgrad(d, s, stream); }))) return rc;
-      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, s, stream, 2); })))
+      if ((rc = run(st, K_APPLY, stream, [&] { return launch_apply(d, V, K, Q, q_dtype, s, stream, 2); })))
         return rc;
     }
   }
@@ -507,6 +530,10 @@ fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtyp
   fwpkm_status rc = ensure_scratch(st, rows_max);
   if (rc != FWPKM_OK) return rc;
   cudaStream_t stream = (cudaStream_t)stream_;
+  if (st->subkey_split_stale) {  // never inside a captured graph: a new arena drops them
+    if ((rc = split_all_subkeys(st, stream))) return rc;
+    st->subkey_split_stale = false;
+  }
   const Extras x = st->x;
   st->x = Extras{};  // armed extras apply to this step only
   if (!st->graphs || st->profiling)
@@ -623,6 +650,11 @@ fwpkm_status fwpkm_state_set(fwpkm_state *st, const float *subkeys, const float 
     e = cudaMemcpyAsync(st->V, values, sizeof(float) * (size_t)st->N * st->dv,
                         cudaMemcpyDefault, s);
   if (e != cudaSuccess) return cuda_fail(e, "state_set");
+  if (subkeys && st->arena) {  // new sub-keys: their split, stream-ordered after the copy
+    const fwpkm_status rc = split_all_subkeys(st, s);
+    if (rc != FWPKM_OK) return rc;
+    st->subkey_split_stale = false;
+  }
   return FWPKM_OK;
 }
 

@@ -68,17 +68,18 @@ struct Dims {
 
 // Device scratch owned by the state (sized for the largest chunk seen).
 constexpr int kScanMaxCtas = 8;  // bucket-scan CTAs: 8 x 16384 buckets
+constexpr int kKnChunks = 8;     // 128-float chunks of a sub-key row (dq/2 <= 1024)
 constexpr int kMaxChunks = 16;   // 128-float column chunks of the widest row (2048 floats)
 constexpr int kPartHead = 2 * kMaxChunks;  // partial slot header: (C, W) per column chunk
 
 struct Scratch {
-  float *Qs;        // [H][2][qstride][dh] query halves of the chunk, fp32 (may be null)
   float *Qs_hi;     // [H][2][qstride][dh] TF32-rounded query halves
   float *Qs_lo;     // [H][2][qstride][dh] query halves minus their TF32 part
   float *qn;        // [H][2][qstride]     |q_half|^2
   float *K_hi;      // [H][2][n][dh] + 128 padding rows: TF32-rounded sub-keys
   float *K_lo;      // same shape: sub-keys minus their TF32 part
-  float *kn;        // [H][2][n]           |K_row|^2
+  float *kn;        // [H][2][n][kKnChunks] |K_row|^2 of each 128-float chunk of the row
+                    // (chunk_sqnorm); the row's norm is their sum in chunk order
   float *D;         // [H][2][rows][n]    squared distances
   int32_t *pslot;   // [M*k] selected slot of pair p = m*k + r
   float *pw;        // [M*k] softmax weight
@@ -123,7 +124,8 @@ struct Scratch {
 struct __align__(16) Member {
   uint32_t g;      // group: slot (< N) or N + (h*2+half)*n + row
   uint32_t id;     // pair id p = m*k + r, or entry id e = (m*2+half)*k + idx
-  int32_t srow;    // source row: E row (value rows) or Qs row (sub-key rows)
+  int32_t srow;    // source row: E row (value rows); for sub-key rows the query half
+                   // tok*2H + h*2 + half of the caller's Q (element offset srow * dq/2)
   int32_t gstart;  // position of the group's first member
   float coef;      // value rows: 2 g_t w / H; sub-key rows: alpha (lam == 0)
   float c0;        // value rows: w / H;       sub-key rows: alpha
@@ -175,6 +177,28 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16 *p, int64_t i) {
 }
 
 // --- mbarrier + bulk async copy (TMA, non-tensor form) -------------------
+// TF32 part of x (round to nearest); x - tf32_part(x) is the remainder.
+__device__ __forceinline__ float tf32_part(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+__device__ __forceinline__ void split_store(float *hi, float *lo, int c, const float4 &v) {
+  const float4 h = make_float4(tf32_part(v.x), tf32_part(v.y), tf32_part(v.z), tf32_part(v.w));
+  *reinterpret_cast<float4 *>(hi + c) = h;
+  *reinterpret_cast<float4 *>(lo + c) = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+}
+// Squared norm of a 128-float chunk held as one float4 per lane (lane l:
+// floats 4l .. 4l+3; lanes past the row's end hold zeros), summed in a fixed
+// order; every lane gets the same value.  The prep and the update both use
+// it, so a sub-key row's norm does not depend on which of them wrote it.
+__device__ __forceinline__ float chunk_sqnorm(const float4 &v) {
+  float a = fmaf(v.w, v.w, fmaf(v.z, v.z, fmaf(v.y, v.y, v.x * v.x)));
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+  return a;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -208,6 +232,35 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity
   atomicOr(&meta->err, ERR_MBAR_TIMEOUT);
   return false;
 }
+// One query half (warp w = (h*2 + half)*rows + row of chunk d) into its TF32
+// split and squared norm: Qs_hi / Qs_lo [h][half][row][:], qn (rows at
+// stride qstride).  Warp-level; used by the prep and by the bucket sort's
+// extra CTAs (the next chunk's halves).
+template <typename TQ>
+__device__ __forceinline__ void prep_query_half(const Dims &d, const TQ *__restrict__ Q,
+                                                const Scratch &s, int64_t w) {
+  const int lane = threadIdx.x & 31;
+  const int dh = d.dh;
+  const int hh = (int)(w / d.rows);  // h*2 + half
+  const int row = (int)(w % d.rows);
+  const int h = hh >> 1, half = hh & 1;
+  const int b = row / d.Tc, tl = row % d.Tc;
+  const int64_t src = ((int64_t)b * d.T + d.t0 + tl) * ((int64_t)d.H * d.dq) +
+                      (int64_t)h * d.dq + (int64_t)half * dh;
+  const int64_t o = ((int64_t)hh * d.qstride + row) * dh;
+  float acc = 0.f;
+  for (int c = lane * 4; c < dh; c += 128) {
+    const float4 v = load4(Q, src + c);
+    split_store(s.Qs_hi + o, s.Qs_lo + o, c, v);
+    acc = fmaf(v.x, v.x, acc);
+    acc = fmaf(v.y, v.y, acc);
+    acc = fmaf(v.z, v.z, acc);
+    acc = fmaf(v.w, v.w, acc);
+  }
+  acc = warp_sum(acc);
+  if (lane == 0) s.qn[(int64_t)hh * d.qstride + row] = acc;
+}
+
 // 1-D bulk copy global -> shared, completion counted on `bar` (bytes % 16 == 0,
 // both addresses 16-byte aligned).
 __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, unsigned bytes,
@@ -270,8 +323,14 @@ cudaError_t launch_k(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, 
 // ------------------------------------------------------------------------
 // Host-side launchers (one per kernel file)
 // ------------------------------------------------------------------------
+// Query halves and sub-key rows of one chunk (the selection-only entry point).
 cudaError_t launch_prep(const Dims &d, const void *Q, int q_dtype, const float *K,
                         const Scratch &s, cudaStream_t st);
+// Query halves of one chunk only (the sub-key split is kept by the update).
+cudaError_t launch_prep_q(const Dims &d, const void *Q, int q_dtype, const Scratch &s,
+                          cudaStream_t st);
+// Sub-key rows only (after the tables are set or the scratch is new).
+cudaError_t launch_prep_k(const Dims &d, const float *K, const Scratch &s, cudaStream_t st);
 // TMA descriptors (CUtensorMap, 128 bytes each) of the score operands.
 struct TcMaps {
   alignas(64) unsigned char a_hi[128];
@@ -292,10 +351,15 @@ cudaError_t launch_topk_select(const Dims &d, const Scratch &s, const Extras &x,
 cudaError_t launch_scan(const Dims &d, const Scratch &s, cudaStream_t st);
 cudaError_t launch_read(const Dims &d, const float *V, const void *Vt, int v_dtype,
                         const float *gate, float *out, const Scratch &s, cudaStream_t st);
-cudaError_t launch_bsort(const Dims &d, const Scratch &s, cudaStream_t st);
-// part 0: all groups; 1: value rows only; 2: sub-key rows only
-cudaError_t launch_apply(const Dims &d, float *V, float *K, const Scratch &s, cudaStream_t st,
-                         int part);
+// The bucket sort; with dn.rows > 0 extra CTAs also prepare the query halves
+// of the next chunk dn (nothing reads this chunk's halves after the score).
+cudaError_t launch_bsort(const Dims &d, const Scratch &s, const Dims &dn, const void *Q,
+                         int q_dtype, cudaStream_t st);
+// part 0: all groups; 1: value rows only; 2: sub-key rows only.  Sub-key
+// sources are the caller's query halves Q (q_dtype); updated sub-key rows get
+// their TF32 split and chunk norms rewritten.
+cudaError_t launch_apply(const Dims &d, float *V, float *K, const void *Q, int q_dtype,
+                         const Scratch &s, cudaStream_t st, int part);
 cudaError_t launch_pgrad(const Dims &d, const Scratch &s, cudaStream_t st);
 
 // Read-only view of a state's shape and sub-key tables (fwpkm_abi.cu).

@@ -75,9 +75,10 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
 
   // Scratch of one pass of `rows` token rows (fp32, each piece 256-byte
   // aligned; rows rounded up to 128): Qs_hi, Qs_lo [2H][rows][dh], qn
-  // [2H][rows], D [2H][rows][n]; fixed: K_hi, K_lo [2H*n + 128][dh], kn [2H][n].
+  // [2H][rows], D [2H][rows][n]; fixed: K_hi, K_lo [2H*n + 128][dh], kn
+  // [2H][n][kKnChunks].
   const size_t H2 = 2 * (size_t)v.H;
-  const size_t fixed = 2 * up256((H2 * v.n + 128) * v.dh * 4) + up256(H2 * v.n * 4) +
+  const size_t fixed = 2 * up256((H2 * v.n + 128) * v.dh * 4) + up256(H2 * v.n * kKnChunks * 4) +
                        4 * 256 + 128 * (2 * H2 * v.dh + H2 + H2 * v.n) * 4;
   const size_t per_row = (2 * H2 * v.dh + H2 + H2 * v.n) * 4;
   if (fixed + per_row * (size_t)B > kNoAllocScratchBytes) {
@@ -103,7 +104,6 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
   }
   char *p = static_cast<char *>(base);
   Scratch s{};
-  s.Qs = nullptr;  // the plain halves are only needed by the update
   s.Qs_hi = reinterpret_cast<float *>(p);
   p += up256(H2 * rows_max * v.dh * 4);
   s.Qs_lo = reinterpret_cast<float *>(p);
@@ -115,7 +115,7 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
   s.K_lo = reinterpret_cast<float *>(p);
   p += up256((H2 * v.n + 128) * v.dh * 4);
   s.kn = reinterpret_cast<float *>(p);
-  p += up256(H2 * v.n * 4);
+  p += up256(H2 * v.n * kKnChunks * 4);
   s.D = reinterpret_cast<float *>(p);
   TcMaps maps;  // host-side descriptors of the operands above (no allocation)
   const cudaError_t me = encode_score_maps(&maps, s, v.H, rows_max, v.n, v.dh);

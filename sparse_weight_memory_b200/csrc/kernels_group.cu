@@ -457,7 +457,9 @@ __device__ void sort_big_bucket(const Dims &d, const Scratch &s, int off, int le
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s) {
+template <typename TQ>
+__global__ void __launch_bounds__(kSortThreads)
+    k_bucket_sort(Dims d, Scratch s, Dims dn, const TQ *__restrict__ Q, int sort_blocks) {
   __shared__ uint64_t buf[kSortCap];
   __shared__ int nseg[2];  // distinct value rows / sub-key rows seen by this CTA
   __shared__ int big_n;
@@ -466,16 +468,23 @@ __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s)
   griddep_wait();
   griddep_launch();
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  if ((int)blockIdx.x >= sort_blocks) {
+    // Extra CTAs: the next chunk's query halves, one warp each (this chunk's
+    // halves are not read after its score).
+    const int64_t w = (int64_t)(blockIdx.x - sort_blocks) * kSortWarps + wib;
+    if (w < (int64_t)2 * dn.H * dn.rows) prep_query_half(dn, Q, s, w);
+    return;
+  }
   if (threadIdx.x < 2) nseg[threadIdx.x] = 0;
   if (threadIdx.x == 0) big_n = 0;
   __syncthreads();
-  const int stride = gridDim.x * kSortWarps;
+  const int stride = sort_blocks * kSortWarps;
   // phase 1: small buckets, one warp each; large ones are listed.  Bucket b
-  // goes to CTA b % gridDim.x: neighbouring buckets (slots of one popular
+  // goes to CTA b % sort_blocks: neighbouring buckets (slots of one popular
   // sub-key row) land in different CTAs.
   // The offsets of a warp's next 32 buckets are loaded together, one per lane.
   int nxt_off = 0, nxt_end = 0;
-  for (int b = blockIdx.x + gridDim.x * wib, i = 0; b < d.NB; b += stride, ++i) {
+  for (int b = blockIdx.x + sort_blocks * wib, i = 0; b < d.NB; b += stride, ++i) {
     if ((i & 31) == 0) {
       const int bl = b + lane * stride;
       nxt_off = bl < d.NB ? s.boff[bl] : 0;
@@ -571,11 +580,14 @@ __global__ void __launch_bounds__(kSortThreads) k_bucket_sort(Dims d, Scratch s)
 }
 
 // Every CTA meets at most 8 buckets per warp (so big_b cannot overflow):
-// the grid holds at least NB / (8 * kSortWarps) CTAs.
-cudaError_t launch_bsort(const Dims &d, const Scratch &s, cudaStream_t st) {
+// the sorting grid holds at least NB / (8 * kSortWarps) CTAs.  The extra
+// CTAs after it prepare the next chunk's query halves (dn.rows > 0).
+template <typename TQ>
+static cudaError_t launch_bsort_t(const Dims &d, const Scratch &s, const Dims &dn, const TQ *Q,
+                                  cudaStream_t st) {
   static int per_sm = 0;
   if (!per_sm) {
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_bucket_sort, kSortThreads, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_bucket_sort<TQ>, kSortThreads, 0);
     if (per_sm < 1) per_sm = 1;
   }
   int blocks = (d.NB + kSortWarps - 1) / kSortWarps;
@@ -583,7 +595,16 @@ cudaError_t launch_bsort(const Dims &d, const Scratch &s, cudaStream_t st) {
   int cap = d.sm_count * per_sm;
   if (cap < min_blocks) cap = min_blocks;
   if (blocks > cap) blocks = cap;
-  return launch_k(d.pdl, k_bucket_sort, blocks, kSortThreads, 0, st, d, s);
+  const int64_t qwarps = dn.rows > 0 ? (int64_t)2 * dn.H * dn.rows : 0;
+  const int extra = (int)((qwarps + kSortWarps - 1) / kSortWarps);
+  return launch_k(d.pdl, k_bucket_sort<TQ>, blocks + extra, kSortThreads, 0, st, d, s, dn, Q,
+                  blocks);
+}
+
+cudaError_t launch_bsort(const Dims &d, const Scratch &s, const Dims &dn, const void *Q,
+                         int q_dtype, cudaStream_t st) {
+  if (q_dtype == 1) return launch_bsort_t(d, s, dn, (const __nv_bfloat16 *)Q, st);
+  return launch_bsort_t(d, s, dn, (const float *)Q, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -611,6 +632,9 @@ constexpr int kU = 8;        // source rows in flight per warp
 __device__ __forceinline__ float4 load_chunk(const float *row, int c4, int n4) {
   return c4 < n4 ? *reinterpret_cast<const float4 *>(row + 4 * c4)
                  : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+__device__ __forceinline__ float4 load_chunk(const __nv_bfloat16 *row, int c4, int n4) {
+  return c4 < n4 ? load4(row, 4 * (int64_t)c4) : make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 __device__ __forceinline__ void fma4(float4 &a, float c, const float4 &x) {
@@ -646,17 +670,13 @@ __device__ __forceinline__ float entropy_term(const Dims &d, float wsum) {
   return (d.lam / (float)d.M) * (logf(wsum / (float)d.M) + 1.f);
 }
 
-__device__ __forceinline__ const float *source_row(const Dims &d, const Scratch &s, bool value,
-                                                   int srow) {
-  return value ? s.E + (int64_t)srow * d.dv : s.Qs + (int64_t)srow * d.dh;
-}
-
 // Sum of a warp's members (lane j < cnt holds member j's srow and coef) over
-// the float4 columns cb + lane + 32*q, q < Q, member order, KU rows in flight.
-template <int Q, int KU>
-__device__ __forceinline__ void sum_members(const Dims &d, const Scratch &s, bool value, int cnt,
-                                            int srow, float coef, int cb, int n4,
-                                            float4 (&acc)[Q]) {
+// the float4 columns cb + lane + 32*q, q < Q, member order, KU rows in flight;
+// member j's source row is base + srow_j * stride (E rows for value rows, the
+// caller's query halves for sub-key rows).
+template <int Q, int KU, typename TS>
+__device__ __forceinline__ void sum_members(const TS *base, int64_t stride, int cnt, int srow,
+                                            float coef, int cb, int n4, float4 (&acc)[Q]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int q = 0; q < Q; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -665,7 +685,7 @@ __device__ __forceinline__ void sum_members(const Dims &d, const Scratch &s, boo
 #pragma unroll
     for (int u = 0; u < KU; ++u) {
       const int sr = __shfl_sync(FULL, srow, (j0 + u) & 31);
-      const float *src = source_row(d, s, value, sr);
+      const TS *src = base + (int64_t)sr * stride;
 #pragma unroll
       for (int q = 0; q < Q; ++q)
         r[u][q] = j0 + u < cnt ? load_chunk(src, cb + lane + 32 * q, n4)
@@ -682,8 +702,19 @@ __device__ __forceinline__ void sum_members(const Dims &d, const Scratch &s, boo
   }
 }
 
+// A rewritten sub-key row chunk (one float4 per lane, zeros past the row)
+// also gets its TF32 split and its chunk norm, exactly as the prep makes them.
+__device__ __forceinline__ void resplit_key_chunk(const Dims &d, const Scratch &s, int64_t r,
+                                                  int ch, int c4, int n4, const float4 &v) {
+  if (c4 < n4) split_store(s.K_hi + r * d.dh, s.K_lo + r * d.dh, 4 * c4, v);
+  const float sq = chunk_sqnorm(c4 < n4 ? v : make_float4(0.f, 0.f, 0.f, 0.f));
+  if ((threadIdx.x & 31) == 0) s.kn[r * kKnChunks + ch] = sq;
+}
+
+template <typename TQ>
 __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__restrict__ V,
-                                                            float *__restrict__ K, Scratch s,
+                                                            float *__restrict__ K,
+                                                            const TQ *__restrict__ Qin, Scratch s,
                                                             int part) {
   griddep_wait();
   griddep_launch();
@@ -758,7 +789,8 @@ __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__res
       }
       float4 acc[1];
       const int cb = chunk * kChunk4;
-      sum_members<1, kU>(d, s, value, cnt, mj.srow, coef, cb, n4, acc);
+      if (value) sum_members<1, kU>(s.E, d.dv, cnt, mj.srow, coef, cb, n4, acc);
+      else sum_members<1, kU>(Qin, d.dh, cnt, mj.srow, coef, cb, n4, acc);
       if (cb + lane < n4)
         *reinterpret_cast<float4 *>(dst + kPartHead + 4 * (cb + lane)) = acc[0];
       // The last of the group's blocks to finish this chunk adds the blocks'
@@ -800,7 +832,9 @@ __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__res
           for (int u = 0; u < kU; ++u)
             if (b0 + u < nb) add4(tot, r[u]);
         }
-        if (c4 < n4) *reinterpret_cast<float4 *>(row + 4 * c4) = updated(d, value, t, tot, Ct);
+        const float4 nv = updated(d, value, t, tot, Ct);
+        if (c4 < n4) *reinterpret_cast<float4 *>(row + 4 * c4) = nv;
+        if (!value) resplit_key_chunk(d, s, (int64_t)(g - (uint32_t)d.N), chunk, c4, n4, nv);
       }
       if (chunk == 0 && value && d.lam != 0.f) {
         const float bt = entropy_term(d, Wt);
@@ -815,26 +849,39 @@ __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__res
         const float4 t0 = load_chunk(dst, cb + lane, n4);
         const float4 t1 = load_chunk(dst, cb + lane + 32, n4);
         float4 acc[2];
-        sum_members<2, 2>(d, s, value, cnt, mj.srow, coef, cb, n4, acc);
-        if (cb + lane < n4)
-          *reinterpret_cast<float4 *>(dst + 4 * (cb + lane)) = updated(d, value, t0, acc[0], C);
-        if (cb + lane + 32 < n4)
-          *reinterpret_cast<float4 *>(dst + 4 * (cb + lane + 32)) =
-              updated(d, value, t1, acc[1], C);
+        if (value) sum_members<2, 2>(s.E, d.dv, cnt, mj.srow, coef, cb, n4, acc);
+        else sum_members<2, 2>(Qin, d.dh, cnt, mj.srow, coef, cb, n4, acc);
+        const float4 nv0 = updated(d, value, t0, acc[0], C);
+        const float4 nv1 = updated(d, value, t1, acc[1], C);
+        if (cb + lane < n4) *reinterpret_cast<float4 *>(dst + 4 * (cb + lane)) = nv0;
+        if (cb + lane + 32 < n4) *reinterpret_cast<float4 *>(dst + 4 * (cb + lane + 32)) = nv1;
+        if (!value) {
+          const int64_t r = (int64_t)(g - (uint32_t)d.N);
+          resplit_key_chunk(d, s, r, cb / kChunk4, cb + lane, n4, nv0);
+          if (cb + kChunk4 < n4) resplit_key_chunk(d, s, r, cb / kChunk4 + 1, cb + lane + 32, n4, nv1);
+        }
       }
     }
     if (value && d.lam != 0.f && lane < len) s.pb[mj.id] = entropy_term(d, W);
   }
 }
 
-cudaError_t launch_apply(const Dims &d, float *V, float *K, const Scratch &s, cudaStream_t st,
-                         int part) {
+template <typename TQ>
+static cudaError_t launch_apply_t(const Dims &d, float *V, float *K, const TQ *Q,
+                                  const Scratch &s, cudaStream_t st, int part) {
   static int per_sm = 0;
   if (!per_sm) {
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_apply, kApplyThreads, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_apply<TQ>, kApplyThreads, 0);
     if (per_sm < 1) per_sm = 1;
   }
-  return launch_k(d.pdl, k_apply, d.sm_count * per_sm, kApplyThreads, 0, st, d, V, K, s, part);
+  return launch_k(d.pdl, k_apply<TQ>, d.sm_count * per_sm, kApplyThreads, 0, st, d, V, K, Q, s,
+                  part);
+}
+
+cudaError_t launch_apply(const Dims &d, float *V, float *K, const void *Q, int q_dtype,
+                         const Scratch &s, cudaStream_t st, int part) {
+  if (q_dtype == 1) return launch_apply_t(d, V, K, (const __nv_bfloat16 *)Q, s, st, part);
+  return launch_apply_t(d, V, K, (const float *)Q, s, st, part);
 }
 
 // ---------------------------------------------------------------------------

@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
       Member m;
       m.g = (uint32_t)d.N + (uint32_t)(mh * d.n + sub);
       m.id = (uint32_t)e;
-      m.srow = mh * d.qstride + row;
+      m.srow = (int)(tok * 2 * d.H + mh);  // this query half in the caller's Q
       m.gstart = 0;
       m.coef = 0.f;
       m.c0 = 0.f;

@@ -9,7 +9,8 @@
 //     D[h][half][row][i] = |q|^2 + |K_i|^2 - 2 q.K_i      (clamped at 0)
 //
 // Precision: three TF32 products, hi*hi + hi*lo + lo*hi, where x = hi + lo and
-// hi is x rounded to TF32 (the prep kernel writes both parts).  The dropped
+// hi is x rounded to TF32 (the prep writes both parts, and the update rewrites
+// them for the sub-key rows it changes).  The dropped
 // lo*lo term and the truncation of lo are ~2^-21 relative, so the distances
 // match an fp32 evaluation to a few ulps and the selection is decided at
 // fp32 accuracy.
@@ -217,7 +218,8 @@ __global__ void __launch_bounds__(128, 1)
     const int row0 = m0 + warp * 32;
     const int my_row = row0 + lane;
     const float my_qn = my_row < d.rows ? s.qn[(int64_t)hh * d.qstride + my_row] : 0.f;
-    const float *kn = s.kn + (int64_t)hh * d.n;
+    const float *kn = s.kn + (int64_t)hh * d.n * kKnChunks;
+    const int nkc = (d.dh / 4 + 31) / 32;  // 128-float chunks of a sub-key row
     float *Dh = s.D + (int64_t)hh * d.rows * d.n;
 #pragma unroll 1
     for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -228,7 +230,9 @@ __global__ void __launch_bounds__(128, 1)
       __syncwarp();
       const int col = n0 + c0 + lane;
       const bool col_ok = col < d.n && c0 + lane < BN;
-      const float kn_l = col_ok ? kn[col] : 0.f;
+      float kn_l = 0.f;  // |K_col|^2: the chunk norms in chunk order
+      if (col_ok)
+        for (int ch = 0; ch < nkc; ++ch) kn_l += kn[(int64_t)col * kKnChunks + ch];
 #pragma unroll 4
       for (int r = 0; r < 32; ++r) {
         const float qn_r = __shfl_sync(FULL, my_qn, r);
