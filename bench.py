@@ -248,11 +248,8 @@ def algorithmic_work(wl, tokens, value_rows, key_rows, records):
 # kernel; the captures and their commands are summarised in profiles/.
 # Missing = no capture of the current kernel.
 NCU_TRAFFIC = {
-    # library: captures of commit d6e5ae0 (fwpkm_score: b492536, kernel unchanged since)
-    "library": {"fwpkm_apply": 10.42e6, "fwpkm_bsort": 0.369e6, "fwpkm_topk": 1.134e6,
-                "fwpkm_score": 3.17e6},
-    # long-context shape, chunk 28 of a 32-chunk call (commit d6e5ae0)
-    "longctx": {"fwpkm_read": 12.95e6, "fwpkm_apply": 16.29e6},
+    # library: captures of commit 1b28857 (fwpkm_topk: d6e5ae0, kernel unchanged since)
+    "library": {"fwpkm_apply": 10.44e6, "fwpkm_bsort": 1.425e6, "fwpkm_topk": 1.134e6},
 }
 
 
