@@ -115,8 +115,13 @@ fwpkm_status fwpkm_step(fwpkm_state *s, int B, int T, const void *Q, int q_dtype
 /*
  * fwpkm_step_host -- fwpkm_step over HOST buffers (same layouts).  Copies Q,
  * Vtarget and gate to state-owned device staging buffers, runs the step, and
- * copies `out` back; returns after the stream has finished.  Pinned host
- * memory gives the fastest copies; pageable memory also works.
+ * copies `out` back, chunk by chunk: a chunk's input rows go in on one copy
+ * stream of the state and its output rows come back on another while later
+ * chunks compute on `stream`, so the copies overlap the step.  Work already
+ * enqueued on `stream` comes first; the call returns once everything it
+ * enqueued has finished.  Pinned host memory gives the fastest copies (and
+ * the overlap); pageable memory also works.  Calls are not replayed as
+ * graphs.
  */
 fwpkm_status fwpkm_step_host(fwpkm_state *s, int B, int T, const void *Q_host, int q_dtype,
                              const void *Vtarget_host, int v_dtype, const float *gate_host,

@@ -11,6 +11,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <functional>
 #include <string>
 #include <vector>
 
@@ -102,6 +103,8 @@ struct fwpkm_state {
   int64_t prof_n[K_COUNT] = {};
   // the TF32 split and chunk norms of the sub-key rows in the arena are out of date
   bool subkey_split_stale = true;
+  // host-buffer calls: copy streams (inputs in, outputs out)
+  cudaStream_t h2d_stream = nullptr, d2h_stream = nullptr;
   // replay of repeated calls as CUDA graphs
   bool graphs = true;
   cudaStream_t capture_stream = nullptr;
@@ -303,13 +306,39 @@ fwpkm_status split_all_subkeys(fwpkm_state *st, cudaStream_t stream) {
   return run(st, K_PREP, stream, [&] { return launch_prep_k(d, st->K, st->s, stream); });
 }
 
+// Scratch for chunks of `rows_max` rows, and the sub-key split if it is out
+// of date (never inside a captured graph: a new arena drops them).
+fwpkm_status prepare_step(fwpkm_state *st, int64_t rows_max, cudaStream_t stream) {
+  fwpkm_status rc = ensure_scratch(st, rows_max);
+  if (rc != FWPKM_OK) return rc;
+  if (st->subkey_split_stale) {
+    if ((rc = split_all_subkeys(st, stream))) return rc;
+    st->subkey_split_stale = false;
+  }
+  return FWPKM_OK;
+}
+
+// Points of the chunk loop where a host-buffer call synchronises its copies:
+// need_inputs(c) before the first kernel that reads chunk c's inputs (the
+// first chunk's prep, else the previous chunk's sort, which prepares chunk
+// c's query halves), read_done(c) once chunk c's outputs are written.
+struct ChunkHooks {
+  std::function<cudaError_t(int)> need_inputs;
+  std::function<cudaError_t(int)> read_done;
+};
+
 // The chunk loop of one call: every kernel of every chunk, in order, on
 // `stream`.  No host synchronisation.
 fwpkm_status enqueue_chunks(fwpkm_state *st, int B, int T, const void *Q, int q_dtype,
                             const void *Vtarget, int v_dtype, const float *gate, float eta,
                             float lambda_entropy, float *out, const Extras &x,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, const ChunkHooks *hooks = nullptr) {
   fwpkm_status rc = FWPKM_OK;
+  auto hook = [&](const std::function<cudaError_t(int)> &f, int c) -> fwpkm_status {
+    if (!hooks || !f) return FWPKM_OK;
+    const cudaError_t e = f(c);
+    return e == cudaSuccess ? FWPKM_OK : cuda_fail(e, "step_host: copy pipeline");
+  };
 
   const Scratch &s = st->s;
   const int n_chunks = (T + st->chunk - 1) / st->chunk;
@@ -320,6 +349,7 @@ fwpkm_status enqueue_chunks(fwpkm_state *st, int B, int T, const void *Q, int q_
     if (c + 1 < n_chunks) dn = chunk_dims(st, B, T, c + 1, eta, lambda_entropy);
     float *V = st->V, *K = st->K;
     // the first chunk's query halves; later chunks' come with the previous sort
+    if (c == 0 && (rc = hook(hooks ? hooks->need_inputs : nullptr, 0))) return rc;
     if (c == 0 &&
         (rc = run(st, K_PREP, stream, [&] { return launch_prep_q(d, Q, q_dtype, s, stream); })))
       return rc;
@@ -331,6 +361,8 @@ fwpkm_status enqueue_chunks(fwpkm_state *st, int B, int T, const void *Q, int q_
            return launch_read(d, V, Vtarget, v_dtype, gate, out, s, stream);
          })))
       return rc;
+    if ((rc = hook(hooks ? hooks->read_done : nullptr, c))) return rc;
+    if (dn.rows > 0 && (rc = hook(hooks ? hooks->need_inputs : nullptr, c + 1))) return rc;
     if ((rc = run(st, K_BSORT, stream,
                   [&] { return launch_bsort(d, s, dn, Q, q_dtype, stream); })))
       return rc;
@@ -483,6 +515,8 @@ void fwpkm_state_free(fwpkm_state *st) {
   for (auto e : st->event_pool) cudaEventDestroy(e);
   clear_graphs(st);
   if (st->capture_stream) cudaStreamDestroy(st->capture_stream);
+  if (st->h2d_stream) cudaStreamDestroy(st->h2d_stream);
+  if (st->d2h_stream) cudaStreamDestroy(st->d2h_stream);
   cudaFree(st->arena);
   cudaFree(st->stage);
   cudaFree(st->K);
@@ -527,13 +561,9 @@ fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtyp
   if (dev != st->device)
     return fail(FWPKM_EINVAL, "step: current device %d is not the state's device %d", dev,
                 st->device);
-  fwpkm_status rc = ensure_scratch(st, rows_max);
-  if (rc != FWPKM_OK) return rc;
   cudaStream_t stream = (cudaStream_t)stream_;
-  if (st->subkey_split_stale) {  // never inside a captured graph: a new arena drops them
-    if ((rc = split_all_subkeys(st, stream))) return rc;
-    st->subkey_split_stale = false;
-  }
+  fwpkm_status rc = prepare_step(st, rows_max, stream);
+  if (rc != FWPKM_OK) return rc;
   const Extras x = st->x;
   st->x = Extras{};  // armed extras apply to this step only
   if (!st->graphs || st->profiling)
@@ -589,12 +619,25 @@ fwpkm_status fwpkm_step_host(fwpkm_state *st, int B, int T, const void *Q_host, 
   if (!is_dtype(q_dtype) || !is_dtype(v_dtype))
     return fail(FWPKM_EINVAL, "step_host: dtype must be FWPKM_F32 or FWPKM_BF16");
   if (B < 1 || T < 1) return fail(FWPKM_ESHAPE, "step_host: B=%d and T=%d must be >= 1", B, T);
+  if (!(eta >= 0.f) || !std::isfinite(eta))
+    return fail(FWPKM_EINVAL, "step_host: eta must be finite and >= 0");
+  if (!(lambda_entropy >= 0.f) || !std::isfinite(lambda_entropy))
+    return fail(FWPKM_EINVAL, "step_host: lambda_entropy must be finite and >= 0");
+  const int64_t rows_max = (int64_t)B * (T < st->chunk ? T : st->chunk);
+  if (rows_max * st->H * st->k * 3 >= (int64_t)1 << 31 || (int64_t)B * T * st->dv >= (int64_t)1 << 40)
+    return fail(FWPKM_ESHAPE, "step_host: B*chunk*heads*topk too large for 32-bit pair ids");
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (dev != st->device)
+    return fail(FWPKM_EINVAL, "step_host: current device %d is not the state's device %d", dev,
+                st->device);
+  // per-token row bytes of each tensor; the staging copy has the caller's layout
+  const size_t qrow = (size_t)st->H * st->dq * (q_dtype == FWPKM_BF16 ? 2 : 4);
+  const size_t vrow = (size_t)st->dv * (v_dtype == FWPKM_BF16 ? 2 : 4);
+  const size_t grow = 4, orow = (size_t)st->dv * 4;
   const size_t tok = (size_t)B * T;
-  const size_t qb = tok * st->H * st->dq * (q_dtype == FWPKM_BF16 ? 2 : 4);
-  const size_t vb = tok * st->dv * (v_dtype == FWPKM_BF16 ? 2 : 4);
-  const size_t gb = tok * 4, ob = tok * st->dv * 4;
-  const size_t oq = 0, ov = align_up(qb, 256), og = ov + align_up(vb, 256),
-               oo = og + align_up(gb, 256), total = oo + align_up(ob, 256);
+  const size_t oq = 0, ov = align_up(tok * qrow, 256), og = ov + align_up(tok * vrow, 256),
+               oo = og + align_up(tok * grow, 256), total = oo + align_up(tok * orow, 256);
   if (total > st->stage_bytes) {
     cudaDeviceSynchronize();
     cudaFree(st->stage);
@@ -607,20 +650,79 @@ fwpkm_status fwpkm_step_host(fwpkm_state *st, int B, int T, const void *Q_host, 
     }
     st->stage_bytes = total;
   }
+  for (cudaStream_t *cs : {&st->h2d_stream, &st->d2h_stream}) {
+    if (!*cs && cudaStreamCreateWithFlags(cs, cudaStreamNonBlocking) != cudaSuccess) {
+      cudaGetLastError();
+      *cs = nullptr;
+      return fail(FWPKM_ECUDA, "step_host: copy stream creation failed");
+    }
+  }
   cudaStream_t stream = (cudaStream_t)stream_;
-  char *base = (char *)st->stage;
-  cudaError_t e = cudaMemcpyAsync(base + oq, Q_host, qb, cudaMemcpyHostToDevice, stream);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(base + ov, Vt_host, vb, cudaMemcpyHostToDevice, stream);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(base + og, gate_host, gb, cudaMemcpyHostToDevice, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "step_host: host-to-device copy");
-  fwpkm_status rc = fwpkm_step(st, B, T, base + oq, q_dtype, base + ov, v_dtype,
-                               (const float *)(base + og), eta, lambda_entropy,
-                               (float *)(base + oo), stream_);
+  fwpkm_status rc = prepare_step(st, rows_max, stream);
   if (rc != FWPKM_OK) return rc;
-  e = cudaMemcpyAsync(out_host, base + oo, ob, cudaMemcpyDeviceToHost, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "step_host: device-to-host copy");
-  e = cudaStreamSynchronize(stream);
-  if (e != cudaSuccess) return cuda_fail(e, "step_host: synchronise");
+
+  // Copies pipelined with the chunk loop: chunk c's input rows (strided over
+  // the B sequences) go in on one copy stream, its output rows come back on
+  // the other as soon as its read has run; the compute stream waits for a
+  // chunk's inputs only before the first kernel that reads them.
+  char *base = (char *)st->stage;
+  const int n_chunks = (T + st->chunk - 1) / st->chunk;
+  std::vector<cudaEvent_t> in_ev(n_chunks), out_ev(n_chunks);
+  for (auto &e : in_ev) e = take_event(st);
+  for (auto &e : out_ev) e = take_event(st);
+  cudaEvent_t start = take_event(st);
+  cudaError_t e = cudaEventRecord(start, stream);  // after earlier work on the caller's stream
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st->h2d_stream, start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st->d2h_stream, start, 0);
+  auto rows_of = [&](int c, int64_t *t0, int64_t *tc) {
+    *t0 = (int64_t)c * st->chunk;
+    *tc = T - *t0 < st->chunk ? T - *t0 : st->chunk;
+  };
+  for (int c = 0; c < n_chunks && e == cudaSuccess; ++c) {
+    int64_t t0, tc;
+    rows_of(c, &t0, &tc);
+    e = cudaMemcpy2DAsync(base + oq + t0 * qrow, T * qrow, (const char *)Q_host + t0 * qrow,
+                          T * qrow, tc * qrow, B, cudaMemcpyHostToDevice, st->h2d_stream);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(base + ov + t0 * vrow, T * vrow, (const char *)Vt_host + t0 * vrow,
+                            T * vrow, tc * vrow, B, cudaMemcpyHostToDevice, st->h2d_stream);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(base + og + t0 * grow, T * grow, (const char *)gate_host + t0 * grow,
+                            T * grow, tc * grow, B, cudaMemcpyHostToDevice, st->h2d_stream);
+    if (e == cudaSuccess) e = cudaEventRecord(in_ev[c], st->h2d_stream);
+  }
+  if (e != cudaSuccess) rc = cuda_fail(e, "step_host: host-to-device copy");
+  if (rc == FWPKM_OK) {
+    const Extras x = st->x;
+    st->x = Extras{};  // armed extras apply to this step only
+    ChunkHooks hooks;
+    hooks.need_inputs = [&](int c) { return cudaStreamWaitEvent(stream, in_ev[c], 0); };
+    hooks.read_done = [&](int c) {
+      int64_t t0, tc;
+      rows_of(c, &t0, &tc);
+      cudaError_t r = cudaEventRecord(out_ev[c], stream);
+      if (r == cudaSuccess) r = cudaStreamWaitEvent(st->d2h_stream, out_ev[c], 0);
+      if (r == cudaSuccess)
+        r = cudaMemcpy2DAsync((char *)out_host + t0 * orow, T * orow, base + oo + t0 * orow,
+                              T * orow, tc * orow, B, cudaMemcpyDeviceToHost, st->d2h_stream);
+      return r;
+    };
+    rc = enqueue_chunks(st, B, T, base + oq, q_dtype, base + ov, v_dtype,
+                        (const float *)(base + og), eta, lambda_entropy, (float *)(base + oo), x,
+                        stream, &hooks);
+  }
+  // everything this call enqueued is done before it returns (and before its
+  // events go back to the pool)
+  const cudaError_t s1 = cudaStreamSynchronize(st->d2h_stream);
+  const cudaError_t s2 = cudaStreamSynchronize(stream);
+  const cudaError_t s3 = cudaStreamSynchronize(st->h2d_stream);
+  for (auto ev : in_ev) st->event_pool.push_back(ev);
+  for (auto ev : out_ev) st->event_pool.push_back(ev);
+  st->event_pool.push_back(start);
+  if (rc != FWPKM_OK) return rc;
+  if (s1 != cudaSuccess || s2 != cudaSuccess || s3 != cudaSuccess)
+    return cuda_fail(s1 != cudaSuccess ? s1 : (s2 != cudaSuccess ? s2 : s3),
+                     "step_host: synchronise");
   return FWPKM_OK;
 }
 

@@ -159,11 +159,19 @@ def test_second_pass_equals_step_from_pass1_state():
     assert np.array_equal(two.V, again.V) and np.array_equal(two.K, again.K)
 
 
-def test_host_buffer_step_equals_device_step():
+@pytest.mark.parametrize("case", ["library", "multihead", "ragged"])
+def test_host_buffer_step_equals_device_step(case):
+    """Host buffers (copied in and out chunk by chunk, overlapping the step)
+    give the device call's results bit for bit: several sequences, bf16
+    inputs, a ragged last chunk."""
     import torch
 
     from sparse_weight_memory_b200 import FwPKMState
-    wl = REDUCED["library"].replace(calls=1)
+    if case == "ragged":
+        base = REDUCED["library"]
+        wl = base.replace(calls=1, B=3, T=3 * base.chunk + 7)
+    else:
+        wl = REDUCED[case].replace(calls=1, passes=1)
     inp = make_inputs(wl)
     res = []
     for host in (False, True):
