@@ -97,8 +97,12 @@ fwpkm_status fwpkm_state_set_eps(fwpkm_state *s, float eps);
  *             K   -= eta * dL/dK
  *           on the touched value rows and sub-key rows only; no clipping.
  * Arguments:
- *   B, T      batch and tokens per sequence (>= 1).
- *   Q         device [B][T][heads*dq], element type q_dtype.
+ *   B, T      batch and tokens per sequence (>= 1); FWPKM_ESHAPE when
+ *             B*T*2*heads >= 2^31 or B*chunk*heads*topk*3 >= 2^31 (32-bit
+ *             indices of query halves and pairs).
+ *   Q         device [B][T][heads*dq], element type q_dtype; read by the
+ *             selection and, for the sub-key gradients, by the update, so it
+ *             must stay unchanged until the step has run.
  *   Vtarget   device [B][T][dv], element type v_dtype (the caller aligns
  *             targets with queries, e.g. the lookahead pairing q_t, v_{t+1}).
  *   gate      device fp32 [B][T]; also the token weight of the MSE loss.

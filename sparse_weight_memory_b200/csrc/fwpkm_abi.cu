@@ -554,6 +554,8 @@ fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtyp
   const int64_t rows_max = (int64_t)B * (T < st->chunk ? T : st->chunk);
   if (rows_max * st->H * st->k * 3 >= (int64_t)1 << 31 || (int64_t)B * T * st->dv >= (int64_t)1 << 40)
     return fail(FWPKM_ESHAPE, "step: B*chunk*heads*topk too large for 32-bit pair ids");
+  if ((int64_t)B * T * 2 * st->H >= (int64_t)1 << 31)
+    return fail(FWPKM_ESHAPE, "step: B*T*heads too large for 32-bit query-half indices");
   if ((((uintptr_t)Q) | ((uintptr_t)Vtarget) | ((uintptr_t)out)) & 15)
     return fail(FWPKM_EINVAL, "step: Q, Vtarget and out must be 16-byte aligned");
   int dev = -1;
@@ -626,6 +628,8 @@ fwpkm_status fwpkm_step_host(fwpkm_state *st, int B, int T, const void *Q_host, 
   const int64_t rows_max = (int64_t)B * (T < st->chunk ? T : st->chunk);
   if (rows_max * st->H * st->k * 3 >= (int64_t)1 << 31 || (int64_t)B * T * st->dv >= (int64_t)1 << 40)
     return fail(FWPKM_ESHAPE, "step_host: B*chunk*heads*topk too large for 32-bit pair ids");
+  if ((int64_t)B * T * 2 * st->H >= (int64_t)1 << 31)
+    return fail(FWPKM_ESHAPE, "step_host: B*T*heads too large for 32-bit query-half indices");
   int dev = -1;
   cudaGetDevice(&dev);
   if (dev != st->device)
