@@ -255,13 +255,10 @@ __global__ void __launch_bounds__(128, 1)
 template <int BN>
 static cudaError_t launch_tc(const Dims &d, const Scratch &s, const TcMaps &maps, int v,
                              cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_score_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         TcSmem<BN>::kBytes);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  // set on every launch: the attribute belongs to the current device's context
+  cudaError_t e = cudaFuncSetAttribute(k_score_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       TcSmem<BN>::kBytes);
+  if (e != cudaSuccess) return e;
   dim3 grid((d.n + BN - 1) / BN, (d.rows + kTcRows - 1) / kTcRows, 2 * d.H);
   return launch_k(d.pdl, k_score_tc<BN>, grid, 128, TcSmem<BN>::kBytes, st,
                   *reinterpret_cast<const CUtensorMap *>(maps.a_hi),
