@@ -2,7 +2,9 @@
 
 Each mutant is a copy of ``oracle/fwpkm_oracle.c`` with one plausible mistake
 planted (a flipped sign, a dropped factor, a swapped index ...), compiled on
-the CPU.  The pin suite is run against it in a child process and must fail.
+the CPU.  The pin suite is run against it in a child process and must fail;
+so must the hand-worked examples of ``tests/golden/`` on their own, except
+where a mutant's mistake cannot show in them (listed in GOLDEN_BLIND).
 """
 import os
 import subprocess
@@ -37,6 +39,17 @@ MUTANTS = {
 }
 
 
+# The hand-worked examples have one head, so head averaging cannot show there.
+GOLDEN_BLIND = {"heads_summed_not_averaged"}
+
+
+def _fails(test_file, env) -> tuple:
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q",
+                        os.path.join(ROOT, "tests", test_file)],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return r.returncode != 0, r.stdout[-2000:]
+
+
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_mutant_is_caught(name, tmp_path):
     before, after = MUTANTS[name]
@@ -48,7 +61,8 @@ def test_mutant_is_caught(name, tmp_path):
     subprocess.check_call(["gcc", "-O2", "-fopenmp", "-std=c11", "-shared", "-fPIC", "-o",
                            str(so), str(mut_c), "-lm"])
     env = dict(os.environ, FWPKM_ORACLE_LIB=str(so), OMP_NUM_THREADS="2")
-    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
+    failed, out = _fails("test_oracle_pins.py", env)
+    assert failed, f"mutant {name} survived the pins:\n{out}"
+    if name not in GOLDEN_BLIND:
+        failed, out = _fails("test_golden.py", env)
+        assert failed, f"mutant {name} survived the hand-worked examples:\n{out}"
