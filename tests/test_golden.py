@@ -17,9 +17,12 @@ from golden_lib import arr, frac, load_hand_step, log_sum
 RTOL = 1e-12
 
 
-@pytest.fixture(scope="module")
-def hs():
-    return load_hand_step()
+FIXTURES = ["hand_step_three_tokens.yaml", "hand_step_two_heads.yaml"]
+
+
+@pytest.fixture(scope="module", params=FIXTURES)
+def hs(request):
+    return load_hand_step(request.param)
 
 
 def _state(hs):

@@ -3,8 +3,7 @@
 Each mutant is a copy of ``oracle/fwpkm_oracle.c`` with one plausible mistake
 planted (a flipped sign, a dropped factor, a swapped index ...), compiled on
 the CPU.  The pin suite is run against it in a child process and must fail;
-so must the hand-worked examples of ``tests/golden/`` on their own, except
-where a mutant's mistake cannot show in them (listed in GOLDEN_BLIND).
+so must the hand-worked examples of ``tests/golden/`` on their own.
 """
 import os
 import subprocess
@@ -39,10 +38,6 @@ MUTANTS = {
 }
 
 
-# The hand-worked examples have one head, so head averaging cannot show there.
-GOLDEN_BLIND = {"heads_summed_not_averaged"}
-
-
 def _fails(test_file, env) -> tuple:
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q",
                         os.path.join(ROOT, "tests", test_file)],
@@ -63,6 +58,5 @@ def test_mutant_is_caught(name, tmp_path):
     env = dict(os.environ, FWPKM_ORACLE_LIB=str(so), OMP_NUM_THREADS="2")
     failed, out = _fails("test_oracle_pins.py", env)
     assert failed, f"mutant {name} survived the pins:\n{out}"
-    if name not in GOLDEN_BLIND:
-        failed, out = _fails("test_golden.py", env)
-        assert failed, f"mutant {name} survived the hand-worked examples:\n{out}"
+    failed, out = _fails("test_golden.py", env)
+    assert failed, f"mutant {name} survived the hand-worked examples:\n{out}"
