@@ -223,9 +223,12 @@ fwpkm_status fwpkm_read_stats(fwpkm_state *s, int64_t *chunks, int64_t *value_ro
  *   weights  device fp32  [B][T][heads][topk] (output).
  * Allocates nothing: all scratch is one 16 MiB array in the library's device
  * image (resident on every GPU that loads the library until exit), used in
- * passes of as many time steps as fit.  A call whose single time step needs
- * more than 16 MiB (B x (2*heads*(dq/2 + n + 1)) x 4 bytes plus the sub-key
- * norms) is rejected with FWPKM_ESHAPE before anything is enqueued.  The
+ * passes of as many time steps as fit.  A time step of B sequences takes
+ * B x 2*heads*(dq + n + 1) x 4 bytes (both TF32 parts of each query half,
+ * its norm, its n distances); on top comes a fixed part: the hi/lo split of
+ * the sub-key tables, their norms, and rounding to whole 128-row score tiles.
+ * A call whose single time step does not fit in 16 MiB is rejected with
+ * FWPKM_ESHAPE before anything is enqueued.  The
  * first call on a device looks the array's address up (cudaGetSymbolAddress,
  * once per device, with that device current); make that first call before any
  * stream capture.  All calls share the array: calls that overlap on the GPU

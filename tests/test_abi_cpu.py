@@ -68,7 +68,25 @@ def test_null_arguments_are_rejected(lib):
     assert lib.fwpkm_record_selection(None, None, None) == fwpkm.FWPKM_EINVAL
     assert lib.fwpkm_force_selection(None, None, None) == fwpkm.FWPKM_EINVAL
     assert lib.fwpkm_read_stats(None, None, None, None, None, None, 0, None) == fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_step_host(None, 1, 1, None, 0, None, 0, None, 1.0, 0.0, None, None) == \
+        fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_set_graphs(None, 1) == fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_set_profiling(None, 1) == fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_profile_read(None, None, None, None, 0, None, None) == fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_select_noalloc(None, 1, 1, None, 0, None, None, None) == \
+        fwpkm.FWPKM_EINVAL
     lib.fwpkm_state_free(None)  # no-op
+
+
+def test_every_entry_point_rejects_a_null_state(lib):
+    """Each fwpkm_* call that takes a state is covered by the NULL checks above."""
+    src = open(os.path.join(ROOT, "tests", "test_abi_cpu.py")).read()
+    body = src[src.index("def test_null_arguments_are_rejected"):
+               src.index("def test_every_entry_point_rejects_a_null_state")]
+    for name in declared_functions():
+        if name in ("fwpkm_last_error",):
+            continue
+        assert f"lib.{name}(" in body, f"{name} has no NULL-argument check"
 
 
 def test_product_path_has_no_oracle_or_fallback():
