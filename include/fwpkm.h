@@ -195,9 +195,11 @@ fwpkm_status fwpkm_profile_read(fwpkm_state *s, const char **names, double *ms,
  * chunks of distinct value rows written, distinct sub-key rows written and
  * member records grouped (pairs plus sub-key entries; the write traffic of
  * the step is proportional to these).  device_errors receives the sticky
- * device error bits (1 = a bounded wait on a bulk copy gave up, 2 = the
- * partial pool overflowed, 4 = a bucket-scan CTA gave up waiting for an
- * earlier one); when any is set the call returns FWPKM_ECUDA.  reset != 0
+ * device error bits (1 = a bounded mbarrier wait -- the score's TMA ring or
+ * the read's bulk copies -- gave up, 2 = a capacity the launch sizing rules
+ * out was exceeded and the excess work skipped, 4 = a bucket-scan CTA gave
+ * up waiting for an earlier one); when any is set the call returns
+ * FWPKM_ECUDA.  reset != 0
  * zeroes the counters and the bits after reading.  Any output pointer may be
  * NULL.
  */
