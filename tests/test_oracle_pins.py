@@ -300,6 +300,23 @@ def test_chaining_equals_one_long_call(oracle):
     assert np.array_equal(one.K, ch.K) and np.array_equal(one.V, ch.V)
 
 
+def test_second_pass_equals_a_fresh_state_from_the_first(oracle):
+    """Iterative reading: pass 2 over the same sequence equals a step started
+    from a new state holding pass 1's tables (the tables are the whole state)."""
+    rng = np.random.default_rng(18)
+    K, V, Q, Vt, g = tiny_case(rng, B=2, T=12, H=2, dq=8, n=6, dv=4, k=3)
+    a = make_state(oracle, K, V, 3, 4)
+    a.step(Q, Vt, g, 0.5, 0.2)
+    b = make_state(oracle, a.K, a.V, 3, 4)
+    r2 = a.step(Q, Vt, g, 0.5, 0.2)
+    rb = b.step(Q, Vt, g, 0.5, 0.2)
+    assert np.array_equal(r2["out"], rb["out"])
+    assert np.array_equal(a.K, b.K) and np.array_equal(a.V, b.V)
+    # and the second pass reads differently from the first
+    r1 = make_state(oracle, K, V, 3, 4).step(Q, Vt, g, 0.5, 0.2)
+    assert not np.array_equal(r1["out"], r2["out"])
+
+
 def test_ragged_last_chunk(oracle):
     """T = 10 with chunk 4: chunks of 4, 4, 2; the split is the same as three calls."""
     rng = np.random.default_rng(16)
