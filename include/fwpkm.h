@@ -177,9 +177,9 @@ fwpkm_status fwpkm_set_graphs(fwpkm_state *s, int enable);
 
 /*
  * Per-kernel timing.  With profiling on, fwpkm_step records a CUDA event pair
- * around every step of the chunk it enqueues (one kernel, or two for
- * fwpkm_apply: the member pass and the combine of longer groups) and launches
- * without programmatic dependent launch; fwpkm_profile_read synchronises
+ * around every kernel of the chunk it enqueues and launches without
+ * programmatic dependent launch or graphs, so the per-kernel times add up to
+ * more than an unprofiled step takes; fwpkm_profile_read synchronises
  * `stream`, adds up the elapsed times per kind, and returns them:
  *   names[i] (static strings), ms[i] (total milliseconds), launches[i]
  *   (kernels launched), for i < *count (<= max_kinds).  Reading resets the
