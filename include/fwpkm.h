@@ -62,7 +62,7 @@ enum { FWPKM_F32 = 0, FWPKM_BF16 = 1 };
  *          multiple of 8), dq/2 <= 1024.
  *   dv     value width; a multiple of 4, <= 2048.
  *   topk   slots read per head and token; 1 <= topk <= min(n, 32).
- *   chunk  tokens per update chunk (>= 1); every chunk is read with the tables
+ *   chunk  tokens per update chunk, 1 <= chunk <= 2^20; every chunk is read with the tables
  *          left by the previous chunk, then written.  [GS-2 causality]
  *   heads  query heads sharing the one value table (>= 1, <= 16); each head
  *          has its own pair of sub-key tables.

@@ -49,6 +49,10 @@ def test_every_declared_symbol_is_exported(lib):
     (1024, 64, 64, 4, 0, 1),       # chunk < 1
     (1024, 64, 64, 4, 32, 0),      # heads < 1
     (4096 * 4096, 64, 64, 4, 32, 1),  # n > 2048
+    (1024, 2064, 64, 4, 32, 1),    # dq/2 > 1024
+    (1024, 64, 2052, 4, 32, 1),    # dv > 2048
+    (1024, 64, 64, 4, (1 << 20) + 1, 1),  # chunk > 2^20
+    (1024, 64, 64, 4, 32, 17),     # heads > 16
 ])
 def test_state_init_rejects_bad_shapes(lib, N, dq, dv, topk, chunk, heads):
     h = ctypes.c_void_p()
