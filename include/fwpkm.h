@@ -53,11 +53,13 @@ enum { FWPKM_F32 = 0, FWPKM_BF16 = 1 };
 
 /* Upper bounds checked by fwpkm_state_init. */
 #define FWPKM_MAX_TOPK 32  /* top-k per head is held one slot per warp lane  */
-#define FWPKM_MAX_SUBKEYS 2048 /* n = sqrt(N): per-half scores live in registers */
+#define FWPKM_MAX_SUBKEYS 1024 /* n = sqrt(N): a half's n scores live in registers, n/32 per
+                                 * lane, selected through one 32-bit mask per lane */
 
 /*
  * fwpkm_state_init -- create a memory of N = n*n slots.  [GS-2, PYPI]
- *   N      number of value slots; must be a perfect square n*n, 4 <= n <= 2048.
+ *   N      number of value slots; must be a perfect square n*n, 4 <= n <= 1024
+ *          (N <= 1,048,576).
  *   dq     query width per head; a multiple of 16 (so dq/2, one half, is a
  *          multiple of 8), dq/2 <= 1024.
  *   dv     value width; a multiple of 4, <= 2048.

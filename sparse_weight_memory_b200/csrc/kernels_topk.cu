@@ -32,13 +32,14 @@ __device__ __forceinline__ int count_lt(const uint32_t (&key)[NV], uint32_t t) {
 // Marks the k smallest keys held across the warp (NV per lane; an unused
 // entry holds 0xffffffff and there are at least k used ones).  Equal keys at
 // the boundary are taken in increasing `tie` order (tie values are unique).
-// Returns this lane's selection as a bit mask over v.
+// Returns this lane's selection as a bit mask over v (so NV <= 32: n <= 1024).
 //
 // MSB-first bisection over the key bits: t grows one bit at a time while
 // fewer than k keys lie below it; it stops early once exactly k do.
 template <int NV>
 __device__ uint32_t warp_select_smallest(const uint32_t (&key)[NV], const uint32_t (&tie)[NV],
                                          int k) {
+  static_assert(NV <= 32, "the selection is one bit per register entry of a 32-bit mask");
   uint32_t kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
   for (int v = 0; v < NV; ++v) {
@@ -287,8 +288,7 @@ static cudaError_t launch_topk_kv(const Dims &d, const Scratch &s, const Extras 
   if (nv <= 8) return launch_k(d.pdl, k_topk<8, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
   if (nv <= 16) return launch_k(d.pdl, k_topk<16, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
   if (nv <= 32) return launch_k(d.pdl, k_topk<32, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
-  if (nv <= 64) return launch_k(d.pdl, k_topk<64, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
-  return cudaErrorInvalidValue;
+  return cudaErrorInvalidValue;  // n > 1024: rejected when the state is made
 }
 
 template <bool kSelectOnly>

@@ -48,7 +48,8 @@ def test_every_declared_symbol_is_exported(lib):
     (1024, 64, 64, 0, 32, 1),      # topk < 1
     (1024, 64, 64, 4, 0, 1),       # chunk < 1
     (1024, 64, 64, 4, 32, 0),      # heads < 1
-    (4096 * 4096, 64, 64, 4, 32, 1),  # n > 2048
+    (4096 * 4096, 64, 64, 4, 32, 1),  # n > 1024
+    (1025 * 1025, 64, 64, 4, 32, 1),  # n > 1024 (the selection masks hold 32 entries per lane)
     (1024, 2064, 64, 4, 32, 1),    # dq/2 > 1024
     (1024, 64, 2052, 4, 32, 1),    # dv > 2048
     (1024, 64, 64, 4, (1 << 20) + 1, 1),  # chunk > 2^20
