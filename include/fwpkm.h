@@ -101,7 +101,8 @@ fwpkm_status fwpkm_state_set_eps(fwpkm_state *s, float eps);
  * Arguments:
  *   B, T      batch and tokens per sequence (>= 1); FWPKM_ESHAPE when
  *             B*T*2*heads >= 2^31 or B*chunk*heads*topk*3 >= 2^31 (32-bit
- *             indices of query halves and pairs).
+ *             indices of query halves and pairs), or when a chunk's B*chunk
+ *             rows exceed 65535 tiles of 128 rows (the score grid).
  *   Q         device [B][T][heads*dq], element type q_dtype; read by the
  *             selection and, for the sub-key gradients, by the update, so it
  *             must stay unchanged until the step has run.

@@ -556,6 +556,9 @@ fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtyp
     return fail(FWPKM_ESHAPE, "step: B*chunk*heads*topk too large for 32-bit pair ids");
   if ((int64_t)B * T * 2 * st->H >= (int64_t)1 << 31)
     return fail(FWPKM_ESHAPE, "step: B*T*heads too large for 32-bit query-half indices");
+  if ((rows_max + 127) / 128 > 65535)  // row tiles of the score grid (grid y)
+    return fail(FWPKM_ESHAPE, "step: B*chunk = %lld rows exceeds 65535 tiles of 128 rows",
+                (long long)rows_max);
   if ((((uintptr_t)Q) | ((uintptr_t)Vtarget) | ((uintptr_t)out)) & 15)
     return fail(FWPKM_EINVAL, "step: Q, Vtarget and out must be 16-byte aligned");
   int dev = -1;
@@ -630,6 +633,9 @@ fwpkm_status fwpkm_step_host(fwpkm_state *st, int B, int T, const void *Q_host, 
     return fail(FWPKM_ESHAPE, "step_host: B*chunk*heads*topk too large for 32-bit pair ids");
   if ((int64_t)B * T * 2 * st->H >= (int64_t)1 << 31)
     return fail(FWPKM_ESHAPE, "step_host: B*T*heads too large for 32-bit query-half indices");
+  if ((rows_max + 127) / 128 > 65535)  // row tiles of the score grid (grid y)
+    return fail(FWPKM_ESHAPE, "step_host: B*chunk = %lld rows exceeds 65535 tiles of 128 rows",
+                (long long)rows_max);
   int dev = -1;
   cudaGetDevice(&dev);
   if (dev != st->device)
