@@ -192,8 +192,15 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
   s.pool_cap = (int)pool_cap;
   size_t total = 0;
   for (auto &p : pieces) total = align_up(total, 256) + align_up(p.bytes, 256);
+  cudaError_t e = cudaSuccess;
+  if (st->arena) {
+    // Work still in flight may use the old arena and update the stats block
+    // that is carried over below.
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "scratch growth: synchronise");
+  }
   void *arena = nullptr;
-  cudaError_t e = cudaMalloc(&arena, total);
+  e = cudaMalloc(&arena, total);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return fail(FWPKM_ENOMEM, "scratch allocation of %zu bytes failed: %s", total,
@@ -214,6 +221,10 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
   if (e == cudaSuccess) e = cudaMemset(s.meta, 0, sizeof(Meta));
   if (e == cudaSuccess && st->s.meta)
     e = cudaMemcpy(s.meta, st->s.meta, sizeof(Meta), cudaMemcpyDeviceToDevice);
+  // The initialisation ran on the legacy default stream, which a caller's
+  // non-blocking stream does not wait for: finish it before any kernel can
+  // touch the arena.
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     cudaFree(arena);
     return cuda_fail(e, "scratch initialisation");
@@ -224,10 +235,7 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
     cudaFree(arena);
     return cuda_fail(e, "scratch initialisation: tensor maps");
   }
-  if (st->arena) {
-    cudaDeviceSynchronize();
-    cudaFree(st->arena);
-  }
+  if (st->arena) cudaFree(st->arena);  // drained above
   clear_graphs(st);  // captured graphs hold the old arena's addresses
   st->maps = maps;
   st->arena = arena;
@@ -494,6 +502,9 @@ fwpkm_status fwpkm_state_init(int64_t N, int dq, int dv, int topk, int chunk, in
                 "state_init: table allocation (%zu + %zu bytes): %s", kbytes, vbytes,
                 cudaGetErrorString(e));
   }
+  // ensure_scratch ends with a device synchronisation, so the zeroed tables
+  // are in place before a caller's stream (non-blocking ones included) copies
+  // into them.
   fwpkm_status rc = ensure_scratch(st, chunk);
   if (rc != FWPKM_OK) {
     cudaFree(st->K);
