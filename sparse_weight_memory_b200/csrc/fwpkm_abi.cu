@@ -854,8 +854,8 @@ fwpkm_status fwpkm_read_stats(fwpkm_state *st, int64_t *chunks, int64_t *value_r
   }
   if (m.err)
     return fail(FWPKM_ECUDA,
-                "device error bits 0x%x (1 = bulk-copy wait timed out, 2 = partial pool "
-                "overflow, 4 = bucket-scan wait timed out)",
+                "device error bits 0x%x (1 = an mbarrier wait timed out, 2 = a capacity "
+                "was exceeded and work skipped, 4 = a bucket-scan wait timed out)",
                 m.err);
   return FWPKM_OK;
 }
