@@ -27,6 +27,9 @@
  *     anything is enqueued: a call that fails them launches nothing and
  *     leaves the state unchanged.
  *   - A state is not thread-safe; calls on one state must be serialised.
+ *     Their device work shares the state's scratch, so calls on one state
+ *     that use different streams must also be ordered on the device by the
+ *     caller (for example with an event); calls on one stream already are.
  */
 #ifndef FWPKM_H_
 #define FWPKM_H_
