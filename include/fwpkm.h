@@ -48,7 +48,7 @@ typedef enum {
   FWPKM_ESHAPE = -2,      /* sizes violate the constraints listed below      */
   FWPKM_ENOMEM = -3,      /* device or host allocation failed                */
   FWPKM_ECUDA = -4,       /* a CUDA call failed (message has the CUDA error)  */
-  FWPKM_EUNSUPPORTED = -5 /* valid request this build does not implement     */
+  FWPKM_EUNSUPPORTED = -5 /* valid request the library does not implement    */
 } fwpkm_status;
 
 /* Element types of Q and Vtarget. */
