@@ -32,7 +32,10 @@
  *   - slot score s(i,j) = s1(i) + s2(j), slot = i*n + j;
  *   - ties ordered by (score desc, index asc);
  *   - weights = plain softmax over the k selected slot scores;
- *   - L_MSE = sum_t w_t ||yhat_t - v_t||^2 with token weight w_t = g_t;
+ *   - L_MSE = sum_t w_t ||yhat_t - v_t||^2 with token weight w_t = g_t
+ *     unless a separate per-token weight omega is given (the lookahead
+ *     pairing q_t -> v_{t+1} gives the last token of a call weight 0: it has
+ *     no target there);
  *   - multi-head: one sub-key pair per head, one shared value table, head
  *     readouts averaged;
  *   - one memory shared by all B sequences; M = B*Tc*H token-heads per chunk;
@@ -212,6 +215,7 @@ static const double *row_of(const double *base, int T, int b, int t, int width) 
 /* chunk's gradient step.  Tokens t0 .. t0+Tc-1 of every sequence b.         */
 /*                                                                          */
 /* Token-head m = (b*Tc + tl)*H + h; pair p = m*k + r.                       */
+/* omega [B][T] (optional): the MSE weight of each token; NULL = the gate.   */
 /*                                                                          */
 /* Optional outputs (NULL to skip):                                          */
 /*   out      [B][T][dv]   g_t * yhat_t for the chunk's tokens               */
@@ -225,7 +229,8 @@ static const double *row_of(const double *base, int T, int b, int t, int width) 
 /*   n_touched scalar      number of distinct value rows written              */
 /* ------------------------------------------------------------------------ */
 static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t0, int Tc,
-                     const double *Q, const double *Vt, const double *gate, double eta,
+                     const double *Q, const double *Vt, const double *gate,
+                     const double *omega, double eta,
                      double lam, int apply, double *out, int64_t *sel_slot, double *sel_w,
                      double *gap, double *dLdV, double *dLdK, double *pbar_out,
                      double *loss, int64_t *n_touched, int64_t *rowmap) {
@@ -341,7 +346,7 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
   for (int64_t m = 0; m < M; ++m) {
     int64_t bt = m / H;
     int b = (int)(bt / Tc), tl = (int)(bt % Tc);
-    double g = row_of(gate, T, b, t0 + tl, 1)[0];
+    double om = row_of(omega ? omega : gate, T, b, t0 + tl, 1)[0]; /* token weight */
     const double *ev = e + bt * dv;
     for (int r = 0; r < k; ++r) {
       int64_t s_ = slot[m * k + r];
@@ -351,7 +356,7 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
       }
       int64_t u = rowmap[s_];
       double wr = w[m * k + r];
-      for (int c = 0; c < dv; ++c) GV[u * dv + c] += (2.0 * g / H) * wr * ev[c];
+      for (int c = 0; c < dv; ++c) GV[u * dv + c] += (2.0 * om / H) * wr * ev[c];
       Csum[u] += wr / H;
       psum[u] += wr;
     }
@@ -360,7 +365,7 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
   for (int64_t u = 0; u < U; ++u) psum[u] /= (double)M;
 
   /* 4. Gradient of L w.r.t. the selected slot scores, then the sub-keys.    */
-  /*    dL/dw_r = (2 g/H) e.V[slot_r] + (lam/M)(log p_bar[slot_r] + 1)        */
+  /*    dL/dw_r = (2 w_t/H) e.V[slot_r] + (lam/M)(log p_bar[slot_r] + 1)      */
   /*    dL/ds_r = w_r (gamma_r - sum_r' w_r' gamma_r')  (softmax Jacobian)    */
   /*    ds/dK_h,i = 2 (q_h - K_h,i) / (eps + d_h(i))   (IDW score)            */
   {
@@ -373,7 +378,7 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
       int h = (int)(m % H);
       int64_t bt = m / H;
       int b = (int)(bt / Tc), tl = (int)(bt % Tc);
-      double g = row_of(gate, T, b, t0 + tl, 1)[0];
+      double om = row_of(omega ? omega : gate, T, b, t0 + tl, 1)[0]; /* token weight */
       const double *ev = e + bt * dv;
       const double *q = row_of(Q, T, b, t0 + tl, H * dq) + (int64_t)h * dq;
       double wg = 0.0;
@@ -381,7 +386,7 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
         const double *vr = V + slot[m * k + r] * dv;
         double dot = 0.0;
         for (int c = 0; c < dv; ++c) dot += ev[c] * vr[c];
-        gam[r] = (2.0 * g / H) * dot;
+        gam[r] = (2.0 * om / H) * dot;
         if (lam != 0.0) gam[r] += (lam / (double)M) * (log(psum[rowmap[slot[m * k + r]]]) + 1.0);
         wg += w[m * k + r] * gam[r];
       }
@@ -416,11 +421,11 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
     double L = 0.0;
     for (int b = 0; b < B; ++b)
       for (int tl = 0; tl < Tc; ++tl) {
-        double g = row_of(gate, T, b, t0 + tl, 1)[0];
+        double om = row_of(omega ? omega : gate, T, b, t0 + tl, 1)[0]; /* token weight */
         const double *ev = e + ((int64_t)b * Tc + tl) * dv;
         double sq = 0.0;
         for (int c = 0; c < dv; ++c) sq += ev[c] * ev[c];
-        L += g * sq;
+        L += om * sq;
       }
     double negH = 0.0;
     for (int64_t u = 0; u < U; ++u)
@@ -456,10 +461,12 @@ done:
  * tables left by the previous chunk [GS-2 causality].  The last chunk may be
  * shorter.  K [H][2][n][dq/2] and V [N][dv] are updated in place; they are the
  * memory carried to the next call.  touched [n_chunks] (optional) receives the
- * number of distinct value rows written per chunk. */
+ * number of distinct value rows written per chunk.  omega [B][T] (optional)
+ * is the MSE weight of each token; NULL = the gate. */
 int orc_step(int64_t N, int n, int dq, int dv, int topk, int chunk, int heads, double eps,
              double *K, double *V, int B, int T, const double *Q, const double *Vt,
-             const double *gate, double eta, double lam, double *out, int64_t *sel_slot,
+             const double *gate, const double *omega, double eta, double lam, double *out,
+             int64_t *sel_slot,
              double *sel_w, double *gap, int64_t *touched, int max_chunks) {
   int rc = check_dims(N, n, dq, dv, topk, chunk, heads);
   if (rc) return rc;
@@ -474,8 +481,8 @@ int orc_step(int64_t N, int n, int dq, int dv, int topk, int chunk, int heads, d
     int t0 = c * chunk;
     int Tc = (T - t0 < chunk) ? T - t0 : chunk;
     int64_t U = 0;
-    rc = orc_chunk(&dm, K, V, B, T, t0, Tc, Q, Vt, gate, eta, lam, 1, out, sel_slot, sel_w,
-                   gap, NULL, NULL, NULL, NULL, &U, rowmap);
+    rc = orc_chunk(&dm, K, V, B, T, t0, Tc, Q, Vt, gate, omega, eta, lam, 1, out, sel_slot,
+                   sel_w, gap, NULL, NULL, NULL, NULL, &U, rowmap);
     if (touched) touched[c] = U;
   }
   free(rowmap);
@@ -486,17 +493,17 @@ int orc_step(int64_t N, int n, int dq, int dv, int topk, int chunk, int heads, d
  * loss and p_bar for finite-difference and invariant checks. */
 int orc_chunk_grads(int64_t N, int n, int dq, int dv, int topk, int chunk, int heads,
                     double eps, const double *K, const double *V, int B, int T, int t0,
-                    int Tc, const double *Q, const double *Vt, const double *gate, double lam,
-                    double *dLdV, double *dLdK, double *pbar, double *loss,
-                    int64_t *sel_slot, double *sel_w) {
+                    int Tc, const double *Q, const double *Vt, const double *gate,
+                    const double *omega, double lam, double *dLdV, double *dLdK, double *pbar,
+                    double *loss, int64_t *sel_slot, double *sel_w) {
   int rc = check_dims(N, n, dq, dv, topk, chunk, heads);
   if (rc) return rc;
   dims_t dm = {N, n, dq, dq / 2, dv, topk, chunk, heads, eps};
   int64_t *rowmap = (int64_t *)malloc(sizeof(int64_t) * (size_t)N);
   if (!rowmap) return -3;
   for (int64_t i = 0; i < N; ++i) rowmap[i] = -1;
-  rc = orc_chunk(&dm, (double *)K, (double *)V, B, T, t0, Tc, Q, Vt, gate, 0.0, lam, 0, NULL,
-                 sel_slot, sel_w, NULL, dLdV, dLdK, pbar, loss, NULL, rowmap);
+  rc = orc_chunk(&dm, (double *)K, (double *)V, B, T, t0, Tc, Q, Vt, gate, omega, 0.0, lam, 0,
+                 NULL, sel_slot, sel_w, NULL, dLdV, dLdK, pbar, loss, NULL, rowmap);
   free(rowmap);
   return rc;
 }
@@ -505,12 +512,13 @@ int orc_chunk_grads(int64_t N, int n, int dq, int dv, int topk, int chunk, int h
  * slots [B][Tc][H][k] (as returned by orc_chunk_grads for the same chunk):
  *   s_r = -log(eps + ||q1 - K1[i_r]||^2) - log(eps + ||q2 - K2[j_r]||^2)
  *   w   = softmax(s);  yhat_t = (1/H) sum_h sum_r w_r V[slot_r]
- *   L   = sum_t g_t ||yhat_t - v_t||^2 + lam * sum_i p_bar_i log p_bar_i
+ *   L   = sum_t w_t ||yhat_t - v_t||^2 + lam * sum_i p_bar_i log p_bar_i
+ *         (w_t = omega_t if omega is given, else the gate g_t)
  * Used only for finite differences of the analytic gradients. */
 double orc_chunk_loss(int64_t N, int n, int dq, int dv, int topk, int heads, double eps,
                       const double *K, const double *V, int B, int T, int t0, int Tc,
-                      const double *Q, const double *Vt, const double *gate, double lam,
-                      const int64_t *slots) {
+                      const double *Q, const double *Vt, const double *gate,
+                      const double *omega, double lam, const int64_t *slots) {
   const int dh = dq / 2, k = topk, H = heads;
   const int64_t M = (int64_t)B * Tc * H;
   double *pb = (double *)calloc((size_t)N, sizeof(double));
@@ -541,14 +549,14 @@ double orc_chunk_loss(int64_t N, int n, int dq, int dv, int topk, int heads, dou
           pb[sl[r]] += w[r] / (double)M;
         }
       }
-      double g = row_of(gate, T, b, t0 + tl, 1)[0];
+      double wt = row_of(omega ? omega : gate, T, b, t0 + tl, 1)[0];
       const double *vt = row_of(Vt, T, b, t0 + tl, dv);
       double sq = 0.0;
       for (int c = 0; c < dv; ++c) {
         double ec = y[c] / H - vt[c];
         sq += ec * ec;
       }
-      L += g * sq;
+      L += wt * sq;
     }
   double negH = 0.0;
   for (int64_t i = 0; i < N; ++i)

@@ -50,12 +50,12 @@ def lib():
         L.orc_brute_select.argtypes = [_dp, _dp, i32, i32, _ip, _dp]
         L.orc_softmax.argtypes = [_dp, i32, _dp]
         L.orc_step.argtypes = [i64, i32, i32, i32, i32, i32, i32, f64, _dp, _dp, i32, i32,
-                               _dp, _dp, _dp, f64, f64, _dp, _ip, _dp, _dp, _ip, i32]
+                               _dp, _dp, _dp, _dp, f64, f64, _dp, _ip, _dp, _dp, _ip, i32]
         L.orc_chunk_grads.argtypes = [i64, i32, i32, i32, i32, i32, i32, f64, _dp, _dp, i32,
-                                      i32, i32, i32, _dp, _dp, _dp, f64, _dp, _dp, _dp, _dp,
-                                      _ip, _dp]
+                                      i32, i32, i32, _dp, _dp, _dp, _dp, f64, _dp, _dp, _dp,
+                                      _dp, _ip, _dp]
         L.orc_chunk_loss.argtypes = [i64, i32, i32, i32, i32, i32, f64, _dp, _dp, i32, i32,
-                                     i32, i32, _dp, _dp, _dp, f64, _ip]
+                                     i32, i32, _dp, _dp, _dp, _dp, f64, _ip]
         L.orc_chunk_loss.restype = f64
         _lib = L
     return _lib
@@ -130,6 +130,19 @@ def softmax(s):
     return w
 
 
+def lookahead_targets(Vt, weight):
+    """Targets and token weights of the lookahead pairing q_t -> v_{t+1}
+    (gist.science section 2, lookahead targets): token t < T-1 takes the
+    next token's target; the last token of the call has none, so its weight
+    is 0 (it is still read)."""
+    Vt, weight = _f64(Vt), _f64(weight)
+    shifted = Vt.copy()
+    shifted[:, :-1] = Vt[:, 1:]
+    w = weight.copy()
+    w[:, -1] = 0.0
+    return shifted, w
+
+
 # --------------------------------------------------------------------------
 # Memory state and the step
 # --------------------------------------------------------------------------
@@ -156,15 +169,22 @@ class State:
         return (self.N, self.n, self.dq, self.dv, self.topk, self.chunk, self.H, self.eps)
 
     def step(self, Q, Vt, gate, eta: float, lam: float, *, want_sel: bool = False,
-             want_gap: bool = False, max_chunks: int = 0) -> dict:
+             want_gap: bool = False, max_chunks: int = 0, omega=None,
+             lookahead: bool = False) -> dict:
         """Run the chunk loop over one call; updates the state in place.
 
         Q [B][T][H*dq], Vt [B][T][dv], gate [B][T] (any float dtype; widened).
         ``max_chunks`` > 0 stops after that many chunks (outputs of later
-        tokens stay zero).
+        tokens stay zero).  ``omega`` [B][T]: the MSE weight of each token
+        (default: the gate).  ``lookahead``: query q_t is written towards
+        target v_{t+1} (gist.science section 2, lookahead targets); the last
+        token of the call has no target and gets weight 0.
         """
         Q, Vt, gate = _f64(Q), _f64(Vt), _f64(gate)
         B, T = gate.shape
+        omega = None if omega is None else _f64(omega).copy()
+        if lookahead:
+            Vt, omega = lookahead_targets(Vt, gate if omega is None else omega)
         assert Q.shape == (B, T, self.H * self.dq) and Vt.shape == (B, T, self.dv)
         out = np.zeros((B, T, self.dv))
         k, H = self.topk, self.H
@@ -174,14 +194,15 @@ class State:
         n_chunks = -(-T // self.chunk)
         touched = np.zeros(n_chunks, np.int64)
         rc = lib().orc_step(*self._dims(), _p(self.K), _p(self.V), B, T, _p(Q), _p(Vt),
-                            _p(gate), eta, lam, _p(out), _p(sel), _p(selw), _p(gap),
-                            _p(touched), max_chunks)
+                            _p(gate), _p(omega), eta, lam, _p(out), _p(sel), _p(selw),
+                            _p(gap), _p(touched), max_chunks)
         _check(rc, "step")
         return {"out": out, "sel_slot": sel, "sel_w": selw, "gap": gap, "touched": touched}
 
-    def chunk_grads(self, Q, Vt, gate, lam: float, t0: int, Tc: int) -> dict:
+    def chunk_grads(self, Q, Vt, gate, lam: float, t0: int, Tc: int, omega=None) -> dict:
         """Raw gradients of one chunk without updating (dense; tiny shapes)."""
         Q, Vt, gate = _f64(Q), _f64(Vt), _f64(gate)
+        omega = None if omega is None else _f64(omega)
         B, T = gate.shape
         dLdV = np.zeros((self.N, self.dv))
         dLdK = np.zeros_like(self.K)
@@ -193,7 +214,7 @@ class State:
         sel_full = np.full((B, T, self.H, self.topk), -1, np.int64)
         selw_full = np.zeros((B, T, self.H, self.topk))
         rc = lib().orc_chunk_grads(*self._dims(), _p(self.K), _p(self.V), B, T, t0, Tc,
-                                   _p(Q), _p(Vt), _p(gate), lam, _p(dLdV), _p(dLdK),
+                                   _p(Q), _p(Vt), _p(gate), _p(omega), lam, _p(dLdV), _p(dLdK),
                                    _p(pbar), _p(loss), _p(sel_full), _p(selw_full))
         _check(rc, "chunk_grads")
         sel[:] = sel_full[:, t0:t0 + Tc]
@@ -201,11 +222,14 @@ class State:
         return {"dLdV": dLdV, "dLdK": dLdK, "pbar": pbar, "loss": float(loss[0]),
                 "sel_slot": sel, "sel_w": selw}
 
-    def chunk_loss(self, Q, Vt, gate, lam: float, t0: int, Tc: int, slots) -> float:
+    def chunk_loss(self, Q, Vt, gate, lam: float, t0: int, Tc: int, slots,
+                   omega=None) -> float:
         """Loss of one chunk for a frozen selection ``slots`` [B][Tc][H][k]."""
         Q, Vt, gate = _f64(Q), _f64(Vt), _f64(gate)
+        omega = None if omega is None else _f64(omega)
         B, T = gate.shape
         slots = np.ascontiguousarray(slots, dtype=np.int64)
         return float(lib().orc_chunk_loss(self.N, self.n, self.dq, self.dv, self.topk, self.H,
                                           self.eps, _p(self.K), _p(self.V), B, T, t0, Tc,
-                                          _p(Q), _p(Vt), _p(gate), lam, _p(slots)))
+                                          _p(Q), _p(Vt), _p(gate), _p(omega), lam,
+                                          _p(slots)))

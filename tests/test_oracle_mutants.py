@@ -22,7 +22,7 @@ MUTANTS = {
     "heads_summed_not_averaged": ("for (int c = 0; c < dv; ++c) y[c] /= H;", ""),
     "no_row_contribution_average": ("vr[c] -= eta * GV[u * dv + c] / Csum[u];",
                                     "vr[c] -= eta * GV[u * dv + c];"),
-    "gate_not_weighting_mse": ("GV[u * dv + c] += (2.0 * g / H) * wr * ev[c];",
+    "gate_not_weighting_mse": ("GV[u * dv + c] += (2.0 * om / H) * wr * ev[c];",
                                "GV[u * dv + c] += (2.0 / H) * wr * ev[c];"),
     "softmax_not_normalised": ("for (int r = 0; r < k; ++r) w[r] /= z;", ""),
     "slot_index_transposed": ("cand[a * k + b].idx = top1[a] * (int64_t)n + top2[b];",
@@ -33,7 +33,8 @@ MUTANTS = {
     "marginal_not_normalised": ("for (int64_t u = 0; u < U; ++u) psum[u] /= (double)M;",
                                 "for (int64_t u = 0; u < U; ++u) psum[u] /= (double)(M + 1);"),
     "distance_of_wrong_half_index": ("d1[m * k + r] = dd1[a_[r]];", "d1[m * k + r] = dd1[b_[r]];"),
-    "mse_grad_factor_two_dropped": ("gam[r] = (2.0 * g / H) * dot;", "gam[r] = (1.0 * g / H) * dot;"),
+    "mse_grad_factor_two_dropped": ("gam[r] = (2.0 * om / H) * dot;",
+                                    "gam[r] = (1.0 * om / H) * dot;"),
     "keys_not_updated": ("if (ktouched[row])", "if (0)"),
 }
 
