@@ -12,7 +12,7 @@ import pytest
 
 from oracle import oracle
 
-from golden_lib import arr, frac, load_hand_step, log_sum
+from golden_lib import arr, frac, load_hand_step, log_sum, row_key
 
 RTOL = 1e-12
 
@@ -73,3 +73,30 @@ def test_hand_step_entropy_term(hs):
     st.step(hs.Q, hs.Vt, hs.gate, hs.eta, lam)
     np.testing.assert_allclose(st.V, hs.values_after(), rtol=RTOL, atol=0)
     np.testing.assert_allclose(st.K, hs.subkeys_after(lam), rtol=1e-10, atol=1e-15)
+
+
+def test_hand_step_lookahead(hs):
+    """The same step with the lookahead pairing q_t -> v_{t+1}: the reads are
+    unchanged, the writes follow the hand-worked values."""
+    la = hs.raw.get("lookahead")
+    if la is None:
+        pytest.skip("this example has no lookahead part")
+    st = _state(hs)
+    res = st.step(hs.Q, hs.Vt, hs.gate, hs.eta, 0.0, want_sel=True, lookahead=True)
+    np.testing.assert_allclose(res["out"], arr(hs.expected["out"]), rtol=RTOL)
+    V = hs.V.copy()
+    for r, row in la["values_after"].items():
+        V[int(r)] = arr(row)
+    np.testing.assert_allclose(st.V, V, rtol=RTOL, atol=0)
+    K = hs.K.copy()
+    for key, row in la["subkeys_after"].items():
+        K[row_key(key)] = arr(row)
+    np.testing.assert_allclose(st.K, K, rtol=RTOL, atol=1e-15)
+    # the raw gradient and the loss, through the targets and weights the pairing gives
+    Vt, om = oracle.lookahead_targets(hs.Vt, hs.gate)
+    gr = _state(hs).chunk_grads(hs.Q, Vt, hs.gate, 0.0, 0, hs.chunk, omega=om)
+    assert gr["loss"] == pytest.approx(sum(frac(x) for x in la["loss"]), rel=RTOL)
+    dK = np.zeros_like(hs.K)
+    for key, row in la["dLdK"].items():
+        dK[row_key(key)] = arr(row)
+    np.testing.assert_allclose(gr["dLdK"], dK, rtol=RTOL, atol=1e-15)
