@@ -1,15 +1,16 @@
 """Benchmark of the FwPKM chunked read-then-write step on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload library]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload longctx]
                     [--impl reference]
 
 A step is one pass of the whole hot path over one batch of the workload: for
-the default `library` workload (B=2, T=4096, chunk 256, N=65,536 slots,
-dq=dv=512, topk 8) that is 3 chained calls = 48 chunks = 24,576 tokens,
-each chunk read and then written.  Inputs are resident in HBM when the timed
-region starts; between steps (untimed) the tables are reset to their initial
-values and L2 is flushed by writing a 256 MiB buffer.  Every step is timed
-with CUDA events on the launching stream.
+the default `longctx` workload (B=1, T=131,072, chunk 1024, N=1,048,576 slots
+(a 2 GiB value table), dq=dv=512, topk 32, 1% planted recalls) that is one
+call of 128 chunks = 131,072 tokens, each chunk read and then written.
+Inputs are resident in HBM when the timed region starts; between steps
+(untimed) the tables are reset to their initial values and L2 is flushed by
+writing a 256 MiB buffer.  Every step is timed with CUDA events on the
+launching stream.
 
 Multi-GPU: the step does not shard (chunks are sequential and all token-heads
 of a chunk write one shared table), so `--gpus N` runs N independent
@@ -33,7 +34,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from sparse_weight_memory_b200.workloads import BF16, WORKLOADS, make_inputs  # noqa: E402
+from sparse_weight_memory_b200.workloads import (BF16, WORKLOADS, bf16_bits_to_f32,  # noqa: E402
+                                                make_inputs)
 
 METRIC = "FwPKM tokens/sec (read+write per chunk), 1xB200; % of HBM/tensor roofline"
 UNIT = "tokens/s"
@@ -158,38 +160,55 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # oracle (CPU) arm
 # ---------------------------------------------------------------------------
-def oracle_sample(wl, inp, budget_s: float = 20.0):
-    """Time the fp64 oracle on the first calls of one workload step (all chunks
-    of each call it starts), stopping once `budget_s` of CPU time is spent."""
-    from oracle import oracle as orc
-    st = orc.State(inp.subkeys, inp.values, topk=wl.topk, chunk=wl.chunk, eps=wl.eps)
-    tokens, elapsed, calls = 0, 0.0, 0
-    n_chunks = wl.n_chunks()
-    per_call_chunks = n_chunks
-    seq = []
-    for c in range(wl.calls):
-        sl = slice(c * wl.T, (c + 1) * wl.T)
-        for _ in range(wl.passes):
-            seq.append(sl)
-    for sl in seq:
-        Q = inp.q_f32()[:, sl].astype(np.float64)
-        Vt = inp.vt_f32()[:, sl].astype(np.float64)
-        g = inp.gate[:, sl]
-        # a bounded number of chunks per call when one call alone is too long
-        t0 = time.perf_counter()
-        st.step(Q, Vt, g, wl.eta, wl.lam, max_chunks=per_call_chunks)
-        dt = time.perf_counter() - t0
-        elapsed += dt
-        tokens += wl.B * min(wl.T, per_call_chunks * wl.chunk)
-        calls += 1
-        if elapsed >= budget_s:
-            break
-        if calls == 1 and dt > budget_s / 2 and per_call_chunks > 1:
-            per_call_chunks = max(1, int(per_call_chunks * (budget_s / 2) / dt))
-    sample = (f"{calls} call(s) of the workload step, {tokens} tokens "
-              f"({'all' if per_call_chunks == n_chunks else per_call_chunks} of {n_chunks} "
-              f"chunks per call), fp64 oracle")
-    return tokens / elapsed, elapsed, sample, orc.num_threads()
+def widen_inputs(a) -> np.ndarray:
+    """fp32, or bf16 bit patterns, widened exactly to fp64."""
+    if a.dtype == np.uint16:
+        return bf16_bits_to_f32(a).astype(np.float64)
+    return a.astype(np.float64)
+
+
+class OracleSampler:
+    """Times the fp64 oracle on the workload step, chunk by chunk and in the
+    step's order (calls, then passes, then chunks), one state carried across
+    chunks exactly as one call carries it.  Each sample runs chunks until its
+    budget of oracle time is spent; the next sample continues where it
+    stopped, and the walk starts over from the initial tables after the last
+    chunk of the step."""
+
+    def __init__(self, wl, inp):
+        self.wl, self.inp = wl, inp
+        self.seq = [(c, t0) for c in range(wl.calls) for _ in range(wl.passes)
+                    for t0 in range(0, wl.T, wl.chunk)]
+        self.pos = 0
+        self.state = None
+
+    def _fresh(self):
+        from oracle import oracle as orc
+        wl, inp = self.wl, self.inp
+        self.state = orc.State(inp.subkeys, inp.values, topk=wl.topk, chunk=wl.chunk,
+                               eps=wl.eps)
+
+    def sample(self, budget_s: float):
+        from oracle import oracle as orc
+        wl, inp = self.wl, self.inp
+        tokens, elapsed, chunks = 0, 0.0, 0
+        while elapsed < budget_s:
+            if self.pos == 0 or self.state is None:
+                self._fresh()
+            c, t0 = self.seq[self.pos]
+            lo, hi = c * wl.T + t0, c * wl.T + min(wl.T, t0 + wl.chunk)
+            Q = widen_inputs(inp.Q[:, lo:hi])
+            Vt = widen_inputs(inp.Vt[:, lo:hi])
+            g = inp.gate[:, lo:hi]
+            t = time.perf_counter()
+            self.state.step(Q, Vt, g, wl.eta, wl.lam)
+            elapsed += time.perf_counter() - t
+            tokens += wl.B * (hi - lo)
+            chunks += 1
+            self.pos = (self.pos + 1) % len(self.seq)
+        desc = (f"{chunks} chunk(s) of the workload step in order ({tokens} tokens; "
+                f"{len(self.seq)} chunks per step), fp64 oracle")
+        return tokens / elapsed, elapsed, desc, orc.num_threads()
 
 
 def run_reference(args, wl):
@@ -199,8 +218,9 @@ def run_reference(args, wl):
     inp = make_inputs(wl)
     vals = []
     info = None
+    sampler = OracleSampler(wl, inp)
     for i in range(args.warmup + args.steps):
-        v, el, sample, cores = oracle_sample(wl, inp, budget_s=args.ref_budget)
+        v, el, sample, cores = sampler.sample(args.ref_budget)
         if i >= args.warmup:
             vals.append((v, el))
         info = (sample, cores)
@@ -454,7 +474,7 @@ def run_gpu(args, wl):
         clocks = clk.summary()
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            v, el, sample, cores = oracle_sample(wl, inp, budget_s=args.ref_budget)
+            v, el, sample, cores = OracleSampler(wl, inp).sample(args.ref_budget)
             cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
         launches = sum(int(round(x["launches_per_step"])) for x in kernels.values()) * args.steps
         line = {
@@ -494,11 +514,11 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="library", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="longctx", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--ref-budget", type=float, default=8.0,
-                    help="seconds of oracle time per reference sample (one step, or "
-                         "a prefix of it when one step takes longer)")
+    ap.add_argument("--ref-budget", type=float, default=5.0,
+                    help="seconds of oracle time per reference sample (the chunks of "
+                         "the step in order, continued by the next sample)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=0,
                     help="tokens per sequence and call (default: the workload's T); a "

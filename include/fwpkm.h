@@ -201,17 +201,46 @@ fwpkm_status fwpkm_profile_read(fwpkm_state *s, const char **names, double *ms,
  * chunks of distinct value rows written, distinct sub-key rows written and
  * member records grouped (pairs plus sub-key entries; the write traffic of
  * the step is proportional to these).  device_errors receives the sticky
- * device error bits (1 = a bounded mbarrier wait -- the score's TMA ring or
- * the read's bulk copies -- gave up, 2 = a capacity the launch sizing rules
- * out was exceeded and the excess work skipped, 4 = a bucket-scan CTA gave
- * up waiting for an earlier one); when any is set the call returns
- * FWPKM_ECUDA.  reset != 0
- * zeroes the counters and the bits after reading.  Any output pointer may be
- * NULL.
+ * device error bits:
+ *    1  the read's bounded wait for its bulk row copies gave up,
+ *    2  the apply's partial pool overflowed (the launch sizing rules it out),
+ *    4  a bucket-scan CTA gave up waiting for an earlier CTA's total,
+ *    8  the score's bounded wait on its TMA ring or its MMAs gave up,
+ *   16  the sort met more large buckets than it lists (ruled out likewise).
+ * A kernel that gives up still lets its own copies in flight land and
+ * returns; no kernel traps.  Once a bit is set, the kernels after the bucket
+ * scan (read, sort, apply) skip the rest of the call and of later calls,
+ * writing nothing, until the bits are reset: the tables keep the values of
+ * the last complete chunk.  When any bit is set the call returns
+ * FWPKM_ECUDA.  reset != 0 zeroes the counters and the bits after reading.
+ * Any output pointer may be NULL.
  */
 fwpkm_status fwpkm_read_stats(fwpkm_state *s, int64_t *chunks, int64_t *value_rows,
                               int64_t *key_rows, int64_t *records, uint32_t *device_errors,
                               int reset, void *stream);
+
+/*
+ * fwpkm_set_wait_limits -- bounds of the device-side waits of this state's
+ * steps (and of fwpkm_select_noalloc on it), for failure detection and its
+ * tests.  mbar_polls bounds the first wait on an mbarrier (the score's TMA
+ * ring and MMA completion, the read's bulk row copies; default 2^26 polls);
+ * scan_polls bounds a bucket-scan CTA's wait for the totals of the CTAs
+ * before it (default 2^24).  A negative value restores the default; 0 makes
+ * the wait give up at once.  A wait that gives up sets its error bit
+ * (fwpkm_read_stats), and the kernel still waits, with a fixed bound of its
+ * own, for the copies it has in flight before it returns.
+ */
+fwpkm_status fwpkm_set_wait_limits(fwpkm_state *s, int64_t mbar_polls, int64_t scan_polls);
+
+/*
+ * fwpkm_inject_alloc_failures -- make the next `count` device allocations of
+ * the library (tables in fwpkm_state_init, scratch growth in fwpkm_step,
+ * staging in fwpkm_step_host) fail as an exhausted device would, returning
+ * FWPKM_ENOMEM with the state unchanged.  Process-wide; 0 disarms.  For
+ * failure-detection tests: it exercises the allocation error paths without
+ * exhausting a shared device.
+ */
+void fwpkm_inject_alloc_failures(int count);
 
 /*
  * fwpkm_select_noalloc -- the product-key selection of the read, for callers
@@ -236,15 +265,25 @@ fwpkm_status fwpkm_read_stats(fwpkm_state *s, int64_t *chunks, int64_t *value_ro
  * its norm, its n distances); on top comes a fixed part: the hi/lo split of
  * the sub-key tables, their norms, and rounding to whole 128-row score tiles.
  * A call whose single time step does not fit in 16 MiB is rejected with
- * FWPKM_ESHAPE before anything is enqueued.  The
- * first call on a device looks the array's address up (cudaGetSymbolAddress,
+ * FWPKM_ESHAPE before anything is enqueued; when the fixed part alone (the
+ * sub-key tables' split, e.g. heads >= 1 with n = 1024 and dq = 2048) is
+ * over 16 MiB, no batch size fits, and the message says so.  The
+ * first call on a device looks the arrays' addresses up (cudaGetSymbolAddress,
  * once per device, with that device current); make that first call before any
- * stream capture.  All calls share the array: calls that overlap on the GPU
+ * stream capture.  All calls share the arrays: calls that overlap on the GPU
  * (other streams or threads) race and must be ordered by the caller.
+ *   device_errors  optional (NULL = not reported): device or host memory
+ *            that receives, stream-ordered after the call's kernels, the
+ *            call's device error bits (8 = the score's bounded TMA/MMA wait
+ *            gave up, see fwpkm_set_wait_limits; 0 = none).  When it is
+ *            non-zero the slots and weights of the call are not meaningful
+ *            (slots stay in [0, N)).  The bits live in a second static block
+ *            of the library image that every call zeroes on its stream first.
  * Asynchronous on `stream`.
  */
 fwpkm_status fwpkm_select_noalloc(fwpkm_state *s, int B, int T, const void *Q, int q_dtype,
-                                  int32_t *slots, float *weights, void *stream);
+                                  int32_t *slots, float *weights, uint32_t *device_errors,
+                                  void *stream);
 
 /* Message of the last failure on this thread ("" if none). */
 const char *fwpkm_last_error(void);

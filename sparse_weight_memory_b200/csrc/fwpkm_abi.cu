@@ -7,6 +7,7 @@
 // kernels are ordered after chunk c's update by the stream itself
 // (gist.science section 2: updates are applied after a chunk; the next chunk
 // reads the updated weights).
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -36,6 +37,22 @@ fwpkm_status fail(fwpkm_status st, const char *fmt, ...) {
 
 fwpkm_status cuda_fail(cudaError_t e, const char *what) {
   return fail(FWPKM_ECUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// Device allocations the library is still told to fail (fwpkm_inject_alloc_failures).
+std::atomic<int> g_fail_allocs{0};
+
+// cudaMalloc, unless an injected failure is pending: then nothing is
+// allocated and the call reports what an exhausted device would.
+cudaError_t dev_malloc(void **p, size_t bytes) {
+  int n = g_fail_allocs.load();
+  while (n > 0) {
+    if (g_fail_allocs.compare_exchange_weak(n, n - 1)) {
+      *p = nullptr;
+      return cudaErrorMemoryAllocation;
+    }
+  }
+  return cudaMalloc(p, bytes);
 }
 
 enum Kind { K_PREP, K_SCORE, K_TOPK, K_SCAN, K_READ, K_BSORT, K_APPLY, K_PGRAD, K_COUNT };
@@ -82,6 +99,8 @@ struct fwpkm_state {
   float eps = 1e-3f;
   int device = 0;
   int sm_count = 148;
+  // bounds of the device-side waits (fwpkm_set_wait_limits)
+  long long mbar_polls = kDefaultMbarPolls, scan_polls = kDefaultScanPolls;
   float *K = nullptr;  // [H][2][n][dh]
   float *V = nullptr;  // [N][dv]
   // scratch arena
@@ -200,7 +219,7 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
     if (e != cudaSuccess) return cuda_fail(e, "scratch growth: synchronise");
   }
   void *arena = nullptr;
-  e = cudaMalloc(&arena, total);
+  e = dev_malloc(&arena, total);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return fail(FWPKM_ENOMEM, "scratch allocation of %zu bytes failed: %s", total,
@@ -303,6 +322,8 @@ Dims chunk_dims(const fwpkm_state *st, int B, int T, int c, float eta, float lam
   d.eps = st->eps;
   d.eta = eta;
   d.lam = lambda_entropy;
+  d.mbar_polls = st->mbar_polls;
+  d.scan_polls = st->scan_polls;
   return d;
 }
 
@@ -440,6 +461,7 @@ bool state_view(const fwpkm_state *st, StateView *v) {
   v->sm_count = st->sm_count;
   v->eps = st->eps;
   v->K = st->K;
+  v->mbar_polls = st->mbar_polls;
   return true;
 }
 void set_last_error(const char *msg) { g_last_error = msg; }
@@ -489,8 +511,8 @@ fwpkm_status fwpkm_state_init(int64_t N, int dq, int dv, int topk, int chunk, in
   if (st->sm_count < 1) st->sm_count = 1;
   const size_t kbytes = sizeof(float) * (size_t)heads * 2 * n * st->dh;
   const size_t vbytes = sizeof(float) * (size_t)N * dv;
-  cudaError_t e = cudaMalloc(&st->K, kbytes);
-  if (e == cudaSuccess) e = cudaMalloc(&st->V, vbytes);
+  cudaError_t e = dev_malloc((void **)&st->K, kbytes);
+  if (e == cudaSuccess) e = dev_malloc((void **)&st->V, vbytes);
   if (e == cudaSuccess) e = cudaMemset(st->K, 0, kbytes);
   if (e == cudaSuccess) e = cudaMemset(st->V, 0, vbytes);
   if (e != cudaSuccess) {
@@ -542,6 +564,16 @@ fwpkm_status fwpkm_state_set_eps(fwpkm_state *st, float eps) {
   clear_graphs(st);  // eps is a kernel parameter of the captured launches
   return FWPKM_OK;
 }
+
+fwpkm_status fwpkm_set_wait_limits(fwpkm_state *st, int64_t mbar_polls, int64_t scan_polls) {
+  if (!st) return fail(FWPKM_EINVAL, "set_wait_limits: state is NULL");
+  st->mbar_polls = mbar_polls < 0 ? kDefaultMbarPolls : (long long)mbar_polls;
+  st->scan_polls = scan_polls < 0 ? kDefaultScanPolls : (long long)scan_polls;
+  clear_graphs(st);  // the limits are kernel parameters of the captured launches
+  return FWPKM_OK;
+}
+
+void fwpkm_inject_alloc_failures(int count) { g_fail_allocs.store(count > 0 ? count : 0); }
 
 fwpkm_status fwpkm_set_graphs(fwpkm_state *st, int enable) {
   if (!st) return fail(FWPKM_EINVAL, "set_graphs: state is NULL");
@@ -664,7 +696,7 @@ fwpkm_status fwpkm_step_host(fwpkm_state *st, int B, int T, const void *Q_host, 
     cudaFree(st->stage);
     st->stage = nullptr;
     st->stage_bytes = 0;
-    cudaError_t e = cudaMalloc(&st->stage, total);
+    cudaError_t e = dev_malloc(&st->stage, total);
     if (e != cudaSuccess) {
       cudaGetLastError();
       return fail(FWPKM_ENOMEM, "step_host: staging allocation of %zu bytes failed", total);
@@ -854,8 +886,10 @@ fwpkm_status fwpkm_read_stats(fwpkm_state *st, int64_t *chunks, int64_t *value_r
   }
   if (m.err)
     return fail(FWPKM_ECUDA,
-                "device error bits 0x%x (1 = an mbarrier wait timed out, 2 = a capacity "
-                "was exceeded and work skipped, 4 = a bucket-scan wait timed out)",
+                "device error bits 0x%x (1 = the read's row-copy wait gave up, 2 = the "
+                "apply's partial pool overflowed, 4 = a bucket-scan wait gave up, 8 = the "
+                "score's TMA/MMA wait gave up, 16 = the sort's list of large buckets "
+                "overflowed; the write kernels of that chunk and later ones were skipped)",
                 m.err);
   return FWPKM_OK;
 }

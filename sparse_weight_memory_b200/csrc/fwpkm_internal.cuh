@@ -27,12 +27,23 @@ struct fwpkm_state;
 namespace fwpkm {
 
 constexpr unsigned FULL = 0xffffffffu;
-// Device-side error bits (meta->err).
+// Device-side error bits (meta->err), one per kernel that can set them, so
+// that a kernel checking the word at entry never sees a bit change under it:
+// every bit it looks at belongs to a kernel that completed before it started.
 enum : unsigned {
-  ERR_MBAR_TIMEOUT = 1u,   // a bounded mbarrier wait gave up
-  ERR_POOL_OVERFLOW = 2u,  // more long-group blocks than the partial pool holds
+  ERR_READ_TIMEOUT = 1u,   // the read's wait for its bulk row copies gave up
+  ERR_POOL_OVERFLOW = 2u,  // apply: more long-group blocks than the partial pool holds
   ERR_SCAN_TIMEOUT = 4u,   // a scan CTA gave up waiting for an earlier CTA's total
+  ERR_SCORE_TIMEOUT = 8u,  // the score's TMA ring or MMA completion wait gave up
+  ERR_SORT_OVERFLOW = 16u, // bsort: a CTA met more large buckets than it lists
+  ERR_ALL = 31u,
 };
+// Default bound of a wait (polls): a bounded wait that gives up sets its bit,
+// and the kernel then still waits, up to kDrainPolls, for its own copies in
+// flight before it returns.
+constexpr long long kDefaultMbarPolls = 1ll << 26;
+constexpr long long kDefaultScanPolls = 1ll << 24;
+constexpr long long kDrainPolls = 1ll << 26;
 
 // Written by the kernels, read by later kernels and by the host.
 struct Meta {
@@ -64,6 +75,8 @@ struct Dims {
   int sm_count;       // multiprocessors of the device (grid sizing)
   int pdl;            // launch with programmatic dependent launch (see launch_k)
   float eps, eta, lam;
+  long long mbar_polls;  // bound of the first wait on an mbarrier (score ring, read copies)
+  long long scan_polls;  // bound of a scan CTA's wait for an earlier CTA's total
 };
 
 // Device scratch owned by the state (sized for the largest chunk seen).
@@ -224,13 +237,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
   return ok != 0;
 }
 // Bounded wait: gives up after `limit` polls (each try_wait may itself block
-// for a hardware-defined interval), records ERR_MBAR_TIMEOUT and returns false.
+// for a hardware-defined interval), records `bit` in meta->err (when meta is
+// not null) and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity, Meta *meta,
-                                                  long long limit = (1ll << 26)) {
+                                                  long long limit, unsigned bit) {
   for (long long it = 0; it < limit; ++it)
     if (mbar_try_wait(bar, parity)) return true;
-  atomicOr(&meta->err, ERR_MBAR_TIMEOUT);
+  if (meta) atomicOr(&meta->err, bit);
   return false;
+}
+// Error bits set by kernels that ran before the caller (its `own` bits
+// excluded): a kernel after the bucket scan returns at entry, writing
+// nothing, when one is set, since the chunk's offsets or selection may then
+// be wrong.  The word is sticky, so the rest of the call is skipped too.
+__device__ __forceinline__ bool chunk_aborted(const Scratch &s, unsigned own) {
+  return (*reinterpret_cast<volatile const unsigned *>(&s.meta->err) & (ERR_ALL & ~own)) != 0u;
 }
 // One query half (warp w = (h*2 + half)*rows + row of chunk d) into its TF32
 // split and squared norm: Qs_hi / Qs_lo [h][half][row][:], qn (rows at
@@ -368,6 +389,7 @@ struct StateView {
   int n, dq, dh, dv, k, chunk, H, device, sm_count;
   float eps;
   const float *K;
+  long long mbar_polls;
 };
 bool state_view(const struct ::fwpkm_state *st, StateView *v);
 // Records `msg` as the calling thread's last error (fwpkm_last_error).

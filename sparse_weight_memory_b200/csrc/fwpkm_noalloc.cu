@@ -17,6 +17,10 @@
 // must order them.  Nothing in it needs to start at zero: each call writes
 // every scratch element it later reads.  The array stays resident on every
 // GPU that loads the library until the process exits.
+//
+// The score kernel's waits are bounded; one that gives up sets a bit in a
+// second static block, g_noalloc_meta, which every call zeroes on its stream
+// before its kernels and copies out to the caller's error word after them.
 #include <cstdio>
 #include <mutex>
 
@@ -28,23 +32,29 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = 16u << 20;  // 16 MiB per device
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+// Error bits and counters the kernels write (only `err` is used here).
+__device__ __align__(256) fwpkm::Meta g_noalloc_meta;
 
-// The array's device address, looked up once per device with that device
-// current (host code cannot use the symbol itself as a device pointer).
+// The arrays' device addresses, looked up once per device with that device
+// current (host code cannot use the symbols themselves as device pointers).
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void *g_scratch_ptr[kMaxDevices] = {};
+fwpkm::Meta *g_meta_ptr[kMaxDevices] = {};
 
-cudaError_t scratch_on(int dev, void **out) {
+cudaError_t scratch_on(int dev, void **out, fwpkm::Meta **meta) {
   std::lock_guard<std::mutex> lock(g_mu);
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   if (!g_scratch_ptr[dev]) {
-    void *p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    void *p = nullptr, *m = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e == cudaSuccess) e = cudaGetSymbolAddress(&m, g_noalloc_meta);
     if (e != cudaSuccess) return e;
+    g_meta_ptr[dev] = static_cast<fwpkm::Meta *>(m);
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];
+  *meta = g_meta_ptr[dev];
   return cudaSuccess;
 }
 
@@ -59,7 +69,7 @@ fwpkm_status fail(fwpkm_status st, const char *msg) {
 
 extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, const void *Q,
                                              int q_dtype, int32_t *slots, float *weights,
-                                             void *stream_) {
+                                             uint32_t *device_errors, void *stream_) {
   using namespace fwpkm;
   StateView v;
   if (!state_view(state, &v)) return fail(FWPKM_EINVAL, "select_noalloc: state is NULL");
@@ -81,6 +91,15 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
   const size_t fixed = 2 * up256((H2 * v.n + 128) * v.dh * 4) + up256(H2 * v.n * kKnChunks * 4) +
                        4 * 256 + 128 * (2 * H2 * v.dh + H2 + H2 * v.n) * 4;
   const size_t per_row = (2 * H2 * v.dh + H2 + H2 * v.n) * 4;
+  if (fixed + per_row > kNoAllocScratchBytes) {
+    char msg[256];
+    snprintf(msg, sizeof msg,
+             "select_noalloc: the state's sub-key tables (heads=%d, n=%d, dq=%d) need %zu "
+             "bytes of scratch with one token, more than the %zu-byte static scratch; no "
+             "batch size fits",
+             v.H, v.n, v.dq, fixed + per_row, kNoAllocScratchBytes);
+    return fail(FWPKM_ESHAPE, msg);
+  }
   if (fixed + per_row * (size_t)B > kNoAllocScratchBytes) {
     char msg[256];
     snprintf(msg, sizeof msg,
@@ -95,7 +114,8 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
   const int rows_max = (B * Tc + 127) / 128 * 128;  // whole 128-row score tiles
 
   void *base = nullptr;
-  const cudaError_t e = scratch_on(dev, &base);
+  Meta *meta = nullptr;
+  const cudaError_t e = scratch_on(dev, &base, &meta);
   if (e != cudaSuccess) {
     char msg[256];
     snprintf(msg, sizeof msg, "select_noalloc: cudaGetSymbolAddress failed: %s",
@@ -117,6 +137,7 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
   s.kn = reinterpret_cast<float *>(p);
   p += up256(H2 * v.n * kKnChunks * 4);
   s.D = reinterpret_cast<float *>(p);
+  s.meta = meta;
   TcMaps maps;  // host-side descriptors of the operands above (no allocation)
   const cudaError_t me = encode_score_maps(&maps, s, v.H, rows_max, v.n, v.dh);
   if (me != cudaSuccess) return fail(FWPKM_ECUDA, "select_noalloc: tensor map encoding failed");
@@ -125,6 +146,14 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
   x.rec_slots = slots;
   x.rec_w = weights;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  // this call's error bits start at zero (a memset allocates nothing)
+  cudaError_t ze = cudaMemsetAsync(&meta->err, 0, sizeof(meta->err), stream);
+  if (ze != cudaSuccess) {
+    char msg[256];
+    snprintf(msg, sizeof msg, "select_noalloc: clearing the error word failed: %s",
+             cudaGetErrorString(ze));
+    return fail(FWPKM_ECUDA, msg);
+  }
   for (int t0 = 0; t0 < T; t0 += Tc) {
     Dims d{};
     d.n = v.n;
@@ -144,12 +173,26 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
     d.sm_count = v.sm_count;
     d.pdl = 1;
     d.eps = v.eps;
-    cudaError_t ke = launch_prep(d, Q, q_dtype, v.K, s, stream);
+    d.mbar_polls = v.mbar_polls;
+    d.scan_polls = kDefaultScanPolls;
+    // the sub-key split once per call, the query halves once per pass
+    cudaError_t ke = t0 == 0 ? launch_prep(d, Q, q_dtype, v.K, s, stream)
+                             : launch_prep_q(d, Q, q_dtype, s, stream);
     if (ke == cudaSuccess) ke = launch_score(d, s, maps, stream);
     if (ke == cudaSuccess) ke = launch_topk_select(d, s, x, stream);
     if (ke != cudaSuccess) {
       char msg[256];
       snprintf(msg, sizeof msg, "select_noalloc: launch failed: %s", cudaGetErrorString(ke));
+      return fail(FWPKM_ECUDA, msg);
+    }
+  }
+  if (device_errors) {
+    const cudaError_t ce = cudaMemcpyAsync(device_errors, &meta->err, sizeof(uint32_t),
+                                           cudaMemcpyDefault, stream);
+    if (ce != cudaSuccess) {
+      char msg[256];
+      snprintf(msg, sizeof msg, "select_noalloc: copying the error word failed: %s",
+               cudaGetErrorString(ce));
       return fail(FWPKM_ECUDA, msg);
     }
   }

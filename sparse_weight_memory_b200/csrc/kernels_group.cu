@@ -61,7 +61,6 @@ __device__ __forceinline__ void store_member(Member *p, const Member &m) {
 constexpr int kScanThreads = 1024;
 constexpr int kScanPer = 16;                        // counts per thread
 constexpr int kScanTile = kScanThreads * kScanPer;  // counts per CTA
-constexpr long long kScanSpinLimit = 1ll << 24;
 
 __device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v) {
   asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
@@ -128,7 +127,7 @@ __global__ void __launch_bounds__(kScanThreads) k_bucket_scan(Dims d, Scratch s)
     if (lane < c) {
       bool ok = false;
       unsigned long long a = 0;
-      for (long long it = 0; it < kScanSpinLimit; ++it) {
+      for (long long it = 0; it < d.scan_polls; ++it) {
         a = ld_acquire_u64(&s.scan_sync[1 + lane]);
         if ((a >> 32) == (epoch & 0xffffffffull)) {
           ok = true;
@@ -475,6 +474,10 @@ __global__ void __launch_bounds__(kSortThreads)
     if (w < (int64_t)2 * dn.H * dn.rows) prep_query_half(dn, Q, s, w);
     return;
   }
+  // An earlier kernel of the chunk gave up: its offsets or selection may be
+  // wrong, so nothing is sorted (the next chunk's halves above are still
+  // prepared; they index nothing).
+  if (chunk_aborted(s, ERR_SORT_OVERFLOW)) return;
   if (threadIdx.x < 2) nseg[threadIdx.x] = 0;
   if (threadIdx.x == 0) big_n = 0;
   __syncthreads();
@@ -497,7 +500,7 @@ __global__ void __launch_bounds__(kSortThreads)
       if (lane == 0) {
         const int slot = atomicAdd(&big_n, 1);
         if (slot < kSortWarps * 8) big_b[slot] = b;
-        else atomicOr(&s.meta->err, ERR_POOL_OVERFLOW);  // cannot happen: see launch_bsort
+        else atomicOr(&s.meta->err, ERR_SORT_OVERFLOW);  // cannot happen: see launch_bsort
       }
       continue;
     }
@@ -718,6 +721,7 @@ __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__res
                                                             int part) {
   griddep_wait();
   griddep_launch();
+  if (chunk_aborted(s, ERR_POOL_OVERFLOW)) return;  // an earlier kernel gave up
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * kApplyWarps + (threadIdx.x >> 5);
   const int nw = gridDim.x * kApplyWarps;
@@ -892,6 +896,7 @@ cudaError_t launch_apply(const Dims &d, float *V, float *K, const void *Q, int q
 __global__ void __launch_bounds__(256) k_pgrad(Dims d, Scratch s) {
   griddep_wait();
   griddep_launch();
+  if (chunk_aborted(s, 0u)) return;  // an earlier kernel gave up
   const int lane = threadIdx.x & 31;
   const int m = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (m >= d.M) return;

@@ -118,6 +118,9 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
                                                        int per) {
   griddep_wait();
   griddep_launch();
+  // An earlier kernel gave up (the bits are stable here, so every CTA of a
+  // cluster takes the same branch): nothing of this chunk is read or written.
+  if (chunk_aborted(s, ERR_READ_TIMEOUT)) return;
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
   const int HK = d.H * d.k, dv = d.dv, dv4 = dv >> 2;
@@ -215,8 +218,8 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   }
   // On a timeout the error bit is set and the CTA still takes every cluster
   // barrier (its results are then meaningless, and the host reports it).
-  if (kStaged && j1 > j0 && !mbar_wait_bounded(bar, 0, s.meta))
-    mbar_wait_bounded(bar, 0, s.meta);  // let copies in flight land
+  if (kStaged && j1 > j0 && !mbar_wait_bounded(bar, 0, s.meta, d.mbar_polls, ERR_READ_TIMEOUT))
+    mbar_wait_bounded(bar, 0, nullptr, kDrainPolls, 0u);  // let copies in flight land
 
   // pass 1: partial weighted sum of this CTA's rows
   for (int c4 = tid; c4 < dv4; c4 += blockDim.x) {

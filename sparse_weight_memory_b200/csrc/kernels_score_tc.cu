@@ -21,8 +21,10 @@
 //   warp 1:           allocates the accumulator columns in tensor memory;
 //                     one lane issues the MMAs and commits each stage back;
 //   warps 0-3:        epilogue, one accumulator lane (= output row) per thread.
-// Every mbarrier wait is bounded; a wait that gives up sets an error bit,
-// the kernel still releases its tensor memory and returns.
+// Every mbarrier wait is bounded; a wait that gives up sets an error bit.
+// The kernel then still waits (up to a fixed drain bound) for the TMA loads
+// it issued and for the MMAs in flight, writes zero distances for its tile,
+// releases its tensor memory and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -165,13 +167,16 @@ __global__ void __launch_bounds__(128, 1)
   griddep_wait();
   griddep_launch();
 
+  int issued = 0;  // k-blocks whose loads the producer issued (thread 0)
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer ----------------
     const int ya = hh * d.qstride + m0;  // row of the query-half tensor
     const int yb = hh * d.n + n0;        // row of the sub-key tensor
-    for (int kb = 0; kb < nkb; ++kb) {
+    for (int kb = 0; kb < nkb; ++kb, issued = kb) {
       const int st = kb % kTcStages, round = kb / kTcStages;
-      if (!mbar_wait_bounded(&empty[st], (round & 1) ^ 1, s.meta)) break;
+      if (!mbar_wait_bounded(&empty[st], (round & 1) ^ 1, s.meta, d.mbar_polls,
+                             ERR_SCORE_TIMEOUT))
+        break;
       unsigned char *stage = smem + st * L::kStage;
       mbar_arrive_expect_tx(&full[st], L::kStage);
       const int x = kb * kTcKBlock;
@@ -186,7 +191,7 @@ __global__ void __launch_bounds__(128, 1)
     bool ok = true;
     for (int kb = 0; kb < nkb && ok; ++kb) {
       const int st = kb % kTcStages, round = kb / kTcStages;
-      ok = mbar_wait_bounded(&full[st], round & 1, s.meta);
+      ok = mbar_wait_bounded(&full[st], round & 1, s.meta, d.mbar_polls, ERR_SCORE_TIMEOUT);
       if (!ok) break;
       tc_fence_after();
       const unsigned char *stage = smem + st * L::kStage;
@@ -211,8 +216,21 @@ __global__ void __launch_bounds__(128, 1)
   // values go through a padded shared-memory tile (the stage buffers are free
   // now) so that every store writes 32 consecutive columns of one row.
   // warp-uniform: tcgen05.ld below is a warp-collective instruction
-  const bool ready = __all_sync(FULL, mbar_wait_bounded(done, 0, s.meta));
+  const bool ready =
+      __all_sync(FULL, mbar_wait_bounded(done, 0, s.meta, d.mbar_polls, ERR_SCORE_TIMEOUT));
+  // After a give-up the MMAs already issued must still finish before the
+  // tensor memory is released.
+  if (!ready) mbar_wait_bounded(done, 0, nullptr, kDrainPolls, 0u);
   tc_fence_after();
+  if (!ready) {
+    // zero distances: the selection that follows still sees valid values
+    float *Dh = s.D + (int64_t)hh * d.rows * d.n;
+    for (int r = 0; r < 32; ++r) {
+      const int row = m0 + warp * 32 + r;
+      for (int c = lane; c < BN; c += 32)
+        if (row < d.rows && n0 + c < d.n) Dh[(int64_t)row * d.n + n0 + c] = 0.f;
+    }
+  }
   if (ready) {
     float *tile = reinterpret_cast<float *>(smem) + warp * 32 * 33;
     const int row0 = m0 + warp * 32;
@@ -243,6 +261,11 @@ __global__ void __launch_bounds__(128, 1)
       __syncwarp();
     }
   }
+  // Loads the producer issued that no MMA consumed (after a give-up) land
+  // before the CTA exits; in a completed run every such wait returns at once.
+  if (warp == 0 && lane == 0)
+    for (int kb = issued > kTcStages ? issued - kTcStages : 0; kb < issued; ++kb)
+      mbar_wait_bounded(&full[kb % kTcStages], (kb / kTcStages) & 1, nullptr, kDrainPolls, 0u);
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -141,7 +141,9 @@ __device__ __forceinline__ void half_topk(const float *__restrict__ drow, int n,
 #pragma unroll
   for (int v = 0; v < NV; ++v) {
     const int i = lane + 32 * v;
-    key[v] = i < n ? __float_as_uint(drow[i]) : 0xffffffffu;  // d >= 0: bits order = value order
+    // d >= 0: the bit order is the value order; a used entry never takes the
+    // unused marker 0xffffffff, whatever the distance's bits
+    key[v] = i < n ? min(__float_as_uint(drow[i]), 0xfffffffeu) : 0xffffffffu;
     idx[v] = (uint32_t)i;
   }
   const uint32_t sel = warp_select_smallest<NV>(key, idx, k);

@@ -60,14 +60,23 @@ def load_library():
                                      ctypes.POINTER(ctypes.c_double), i64p, i32,
                                      ctypes.POINTER(i32), _vp]
     L.fwpkm_read_stats.argtypes = [_vp, i64p, i64p, i64p, i64p, u32p, i32, _vp]
-    L.fwpkm_select_noalloc.argtypes = [_vp, i32, i32, _vp, i32, _vp, _vp, _vp]
+    L.fwpkm_select_noalloc.argtypes = [_vp, i32, i32, _vp, i32, _vp, _vp, _vp, _vp]
+    L.fwpkm_set_wait_limits.argtypes = [_vp, i64, i64]
+    L.fwpkm_inject_alloc_failures.argtypes = [i32]
+    L.fwpkm_inject_alloc_failures.restype = None
     for name in ("fwpkm_state_init", "fwpkm_state_set_eps", "fwpkm_step", "fwpkm_step_host",
                  "fwpkm_state_get", "fwpkm_state_set", "fwpkm_record_selection",
                  "fwpkm_force_selection", "fwpkm_set_profiling", "fwpkm_profile_read",
-                 "fwpkm_read_stats", "fwpkm_select_noalloc", "fwpkm_set_graphs"):
+                 "fwpkm_read_stats", "fwpkm_select_noalloc", "fwpkm_set_graphs",
+                 "fwpkm_set_wait_limits"):
         getattr(L, name).restype = i32
     _lib = L
     return L
+
+
+def inject_alloc_failures(count: int):
+    """Make the library's next ``count`` device allocations fail (ENOMEM)."""
+    load_library().fwpkm_inject_alloc_failures(int(count))
 
 
 def _check(rc: int):
@@ -184,13 +193,19 @@ class FwPKMState:
     def force_selection(self, slots=None, mask=None):
         _check(load_library().fwpkm_force_selection(self._h, _ptr(slots), _ptr(mask)))
 
-    def select_noalloc(self, Q, slots, weights, stream=None):
-        """Selection only (slots, weights) into caller buffers; allocates nothing."""
+    def select_noalloc(self, Q, slots, weights, errors=None, stream=None):
+        """Selection only (slots, weights) into caller buffers; allocates nothing.
+        ``errors``: optional one-element uint32 buffer (device tensor or host
+        array) that receives the call's device error bits."""
         B, T = Q.shape[0], Q.shape[1]
         _check(load_library().fwpkm_select_noalloc(self._h, B, T, _ptr(Q), _dtype_code(Q),
-                                                   _ptr(slots), _ptr(weights),
+                                                   _ptr(slots), _ptr(weights), _ptr(errors),
                                                    _stream(stream)))
         return slots, weights
+
+    def set_wait_limits(self, mbar_polls: int = -1, scan_polls: int = -1):
+        """Bounds of the device-side waits (negative = the default)."""
+        _check(load_library().fwpkm_set_wait_limits(self._h, mbar_polls, scan_polls))
 
     def set_graphs(self, enable: bool):
         """Replay repeated calls as CUDA graphs (default on)."""

@@ -78,8 +78,10 @@ def test_null_arguments_are_rejected(lib):
     assert lib.fwpkm_set_graphs(None, 1) == fwpkm.FWPKM_EINVAL
     assert lib.fwpkm_set_profiling(None, 1) == fwpkm.FWPKM_EINVAL
     assert lib.fwpkm_profile_read(None, None, None, None, 0, None, None) == fwpkm.FWPKM_EINVAL
-    assert lib.fwpkm_select_noalloc(None, 1, 1, None, 0, None, None, None) == \
+    assert lib.fwpkm_select_noalloc(None, 1, 1, None, 0, None, None, None, None) == \
         fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_set_wait_limits(None, 0, 0) == fwpkm.FWPKM_EINVAL
+    lib.fwpkm_inject_alloc_failures(0)  # takes no state; 0 disarms
     lib.fwpkm_state_free(None)  # no-op
 
 
@@ -102,3 +104,17 @@ def test_product_path_has_no_oracle_or_fallback():
         for f in files:
             if f.endswith(".py"):
                 assert not pat.search(open(os.path.join(dirpath, f)).read()), f
+
+
+def test_injected_allocation_failure_is_enomem(lib):
+    """An injected device-allocation failure makes state_init return ENOMEM
+    with no state, before any table exists; the injection is consumed."""
+    h = ctypes.c_void_p()
+    lib.fwpkm_inject_alloc_failures(1)
+    try:
+        rc = lib.fwpkm_state_init(1024, 64, 64, 4, 32, 1, ctypes.byref(h))
+    finally:
+        lib.fwpkm_inject_alloc_failures(0)
+    assert rc == fwpkm.FWPKM_ENOMEM
+    assert h.value is None
+    assert "allocation" in lib.fwpkm_last_error().decode()

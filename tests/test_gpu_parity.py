@@ -205,7 +205,37 @@ EDGE = {
                         eta=0.3, lam=0.0, gate="one"),
     "many_heads_big_k": Workload("e7", B=1, T=40, chunk=20, heads=4, dq=32, n=64, dv=1024,
                                  topk=32, eta=0.2, lam=0.01, gate="uniform"),
+    # 16 heads x k = 32 rows of 4 KB per token: a cluster CTA's share (64 rows)
+    # does not fit in shared memory, so the read takes its unstaged variant
+    "heads16_unstaged_read": Workload("e8", B=1, T=24, chunk=12, heads=16, dq=32, n=32,
+                                      dv=1024, topk=32, eta=0.2, lam=0.0, gate="uniform"),
+    "heads16_unstaged_read_entropy": Workload("e9", B=1, T=20, chunk=10, heads=16, dq=32,
+                                              n=32, dv=2048, topk=32, eta=0.2, lam=0.05,
+                                              gate="uniform"),
+    # dq/2 = 1024: 32 k-blocks in the score ring and 8 chunk norms per sub-key row
+    "dq2048": Workload("e10", B=2, T=40, chunk=16, heads=1, dq=2048, n=16, dv=8, topk=4,
+                       eta=0.05, lam=0.1, gate="uniform"),
+    "heads16_small_dv": Workload("e11", B=2, T=30, chunk=16, heads=16, dq=32, n=8, dv=8,
+                                 topk=4, eta=0.3, lam=0.02, gate="beta25"),
 }
+
+
+def read_is_staged(wl) -> bool:
+    """The read kernel's sizing rule: a cluster of G <= 8 CTAs per token, G
+    doubled while a CTA's share of the H*k rows exceeds 32 KB; the share is
+    staged in shared memory when it fits in 200 KB with the per-token arrays."""
+    HK, row = wl.heads * wl.topk, wl.dv * 4
+    G = 1
+    while G < 8 and G < HK and -(-HK // G) * row > 32 * 1024:
+        G *= 2
+    per = -(-HK // G)
+    return 128 + per * row + 2 * row + HK * 20 + 2 * HK * 16 <= 200 * 1024
+
+
+def test_edge_table_reaches_both_read_variants():
+    assert not read_is_staged(EDGE["heads16_unstaged_read"])
+    assert not read_is_staged(EDGE["heads16_unstaged_read_entropy"])
+    assert read_is_staged(EDGE["many_heads_big_k"])
 
 
 @pytest.mark.parametrize("name", sorted(EDGE))
