@@ -49,6 +49,8 @@ def describe(wl) -> str:
         s += f" x{wl.calls} chained calls"
     if wl.passes > 1:
         s += f" x{wl.passes} passes"
+    if wl.lookahead:
+        s += " lookahead (q_t written towards v_t+1)"
     return s
 
 
@@ -198,10 +200,20 @@ class OracleSampler:
             c, t0 = self.seq[self.pos]
             lo, hi = c * wl.T + t0, c * wl.T + min(wl.T, t0 + wl.chunk)
             Q = widen_inputs(inp.Q[:, lo:hi])
-            Vt = widen_inputs(inp.Vt[:, lo:hi])
             g = inp.gate[:, lo:hi]
+            om = None
+            if wl.lookahead:
+                # the call's pairing q_t -> v_{t+1}; its last token has weight 0
+                end = (c + 1) * wl.T
+                Vt = widen_inputs(inp.Vt[:, lo + 1:min(hi + 1, end)])
+                om = g.astype(np.float64).copy()
+                if hi == end:
+                    Vt = np.concatenate([Vt, np.zeros_like(Vt[:, :1])], axis=1)
+                    om[:, -1] = 0.0
+            else:
+                Vt = widen_inputs(inp.Vt[:, lo:hi])
             t = time.perf_counter()
-            self.state.step(Q, Vt, g, wl.eta, wl.lam)
+            self.state.step(Q, Vt, g, wl.eta, wl.lam, omega=om)
             elapsed += time.perf_counter() - t
             tokens += wl.B * (hi - lo)
             chunks += 1
@@ -348,7 +360,7 @@ def run_gpu(args, wl):
 
     def one_step():
         for (q, v, g), o in zip(segs, outs):
-            st.step(q, v, g, wl.eta, wl.lam, out=o)
+            st.step(q, v, g, wl.eta, wl.lam, out=o, lookahead=wl.lookahead)
 
     for _ in range(args.warmup):
         reset()
@@ -430,7 +442,7 @@ def run_gpu(args, wl):
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for q, v, g in hsegs:
-            st.step_host(q, v, g, wl.eta, wl.lam, out=hout)
+            st.step_host(q, v, g, wl.eta, wl.lam, out=hout, lookahead=wl.lookahead)
         b.record(stream)
         torch.cuda.synchronize()
         if i >= args.warmup:
@@ -523,10 +535,20 @@ def main():
     ap.add_argument("--tokens", type=int, default=0,
                     help="tokens per sequence and call (default: the workload's T); a "
                          "shorter run of the same shape, for profiler captures")
+    ap.add_argument("--passes", type=int, default=0,
+                    help="reads of each segment with the memory carried over (default: the "
+                         "workload's)")
+    ap.add_argument("--lookahead", action="store_true",
+                    help="write query t towards the target of token t+1 (each call's last "
+                         "token has weight 0)")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
     if args.tokens:
         wl = wl.replace(T=args.tokens)
+    if args.passes:
+        wl = wl.replace(passes=args.passes)
+    if args.lookahead:
+        wl = wl.replace(lookahead=True)
     if args.impl == "reference":
         run_reference(args, wl)
     else:

@@ -122,6 +122,34 @@ fwpkm_status fwpkm_step(fwpkm_state *s, int B, int T, const void *Q, int q_dtype
                         const void *Vtarget, int v_dtype, const float *gate, float eta,
                         float lambda_entropy, float *out, void *stream);
 
+/* Flags of fwpkm_step_ex. */
+#define FWPKM_LOOKAHEAD 1 /* write query t towards the target of token t+1 */
+
+/*
+ * fwpkm_step_ex -- fwpkm_step with the write's token weights and target
+ * pairing chosen by the caller.  [GS-2 lookahead targets; SS-TOC weighting
+ * the MSE loss by token importance]
+ *   omega     device fp32 [B][T], or NULL: the weight w_t of token t in the
+ *             MSE loss, L = sum_t w_t ||yhat_t - target_t||^2 + lambda * ...,
+ *             used for dL/dV and dL/dK; NULL makes it the gate, as in
+ *             fwpkm_step.  The gate still scales the output, out_t = g_t yhat_t.
+ *             A token with weight 0 is read but pulls no row towards its
+ *             target (its pairs still count in the rows' C_i = sum of w/H).
+ *   flags     0 or FWPKM_LOOKAHEAD.  With FWPKM_LOOKAHEAD the query of token
+ *             t is written towards Vtarget[t+1] (of the same sequence), and
+ *             the last token of the call, which has no next target, gets
+ *             weight 0; the call's tokens are the unit, so chained calls each
+ *             lose their last token's write.  Vtarget is then read one row
+ *             ahead, the whole [B][T] buffer as in fwpkm_step.
+ * Other arguments, checks and asynchrony as fwpkm_step (which is
+ * fwpkm_step_ex with omega = NULL and flags = 0).  FWPKM_EINVAL for unknown
+ * flags.
+ */
+fwpkm_status fwpkm_step_ex(fwpkm_state *s, int B, int T, const void *Q, int q_dtype,
+                           const void *Vtarget, int v_dtype, const float *gate,
+                           const float *omega, int flags, float eta, float lambda_entropy,
+                           float *out, void *stream);
+
 /*
  * fwpkm_step_host -- fwpkm_step over HOST buffers (same layouts).  Copies Q,
  * Vtarget and gate to state-owned device staging buffers, runs the step, and
@@ -136,6 +164,18 @@ fwpkm_status fwpkm_step(fwpkm_state *s, int B, int T, const void *Q, int q_dtype
 fwpkm_status fwpkm_step_host(fwpkm_state *s, int B, int T, const void *Q_host, int q_dtype,
                              const void *Vtarget_host, int v_dtype, const float *gate_host,
                              float eta, float lambda_entropy, float *out_host, void *stream);
+
+/*
+ * fwpkm_step_host_ex -- fwpkm_step_ex over HOST buffers: omega_host (fp32
+ * [B][T] or NULL) and flags as in fwpkm_step_ex, everything else as in
+ * fwpkm_step_host (which is this call with omega_host = NULL, flags = 0).
+ * With FWPKM_LOOKAHEAD a chunk's read waits for the next chunk's input copy,
+ * whose first target row it takes.
+ */
+fwpkm_status fwpkm_step_host_ex(fwpkm_state *s, int B, int T, const void *Q_host, int q_dtype,
+                                const void *Vtarget_host, int v_dtype, const float *gate_host,
+                                const float *omega_host, int flags, float eta,
+                                float lambda_entropy, float *out_host, void *stream);
 
 /*
  * fwpkm_state_get / fwpkm_state_set -- copy the fast weights out / in, for

@@ -74,13 +74,15 @@ struct Timing {
 struct StepKey {
   int B, T, q_dtype, v_dtype;
   const void *Q, *Vt;
-  const float *gate;
+  const float *gate, *omega;
+  int lookahead;
   float *out;
   float eta, lam;
   Extras x;
   bool operator==(const StepKey &o) const {
     return B == o.B && T == o.T && q_dtype == o.q_dtype && v_dtype == o.v_dtype && Q == o.Q &&
-           Vt == o.Vt && gate == o.gate && out == o.out && eta == o.eta && lam == o.lam &&
+           Vt == o.Vt && gate == o.gate && omega == o.omega && lookahead == o.lookahead &&
+           out == o.out && eta == o.eta && lam == o.lam &&
            x.force_slots == o.x.force_slots && x.force_mask == o.x.force_mask &&
            x.rec_slots == o.x.rec_slots && x.rec_w == o.x.rec_w;
   }
@@ -359,7 +361,8 @@ struct ChunkHooks {
 // The chunk loop of one call: every kernel of every chunk, in order, on
 // `stream`.  No host synchronisation.
 fwpkm_status enqueue_chunks(fwpkm_state *st, int B, int T, const void *Q, int q_dtype,
-                            const void *Vtarget, int v_dtype, const float *gate, float eta,
+                            const void *Vtarget, int v_dtype, const float *gate,
+                            const float *omega, int lookahead, float eta,
                             float lambda_entropy, float *out, const Extras &x,
                             cudaStream_t stream, const ChunkHooks *hooks = nullptr) {
   fwpkm_status rc = FWPKM_OK;
@@ -372,7 +375,8 @@ fwpkm_status enqueue_chunks(fwpkm_state *st, int B, int T, const void *Q, int q_
   const Scratch &s = st->s;
   const int n_chunks = (T + st->chunk - 1) / st->chunk;
   for (int c = 0; c < n_chunks; ++c) {
-    const Dims d = chunk_dims(st, B, T, c, eta, lambda_entropy);
+    Dims d = chunk_dims(st, B, T, c, eta, lambda_entropy);
+    d.lookahead = lookahead;
     // the next chunk of this call, whose query halves the sort prepares
     Dims dn{};
     if (c + 1 < n_chunks) dn = chunk_dims(st, B, T, c + 1, eta, lambda_entropy);
@@ -386,12 +390,17 @@ fwpkm_status enqueue_chunks(fwpkm_state *st, int B, int T, const void *Q, int q_
       return rc;
     if ((rc = run(st, K_TOPK, stream, [&] { return launch_topk(d, s, x, stream); }))) return rc;
     if ((rc = run(st, K_SCAN, stream, [&] { return launch_scan(d, s, stream); }))) return rc;
+    // with the lookahead pairing the read also takes the first target row of
+    // the next chunk, so that chunk's inputs are needed before it
+    if (lookahead && dn.rows > 0 && (rc = hook(hooks ? hooks->need_inputs : nullptr, c + 1)))
+      return rc;
     if ((rc = run(st, K_READ, stream, [&] {
-           return launch_read(d, V, Vtarget, v_dtype, gate, out, s, stream);
+           return launch_read(d, V, Vtarget, v_dtype, gate, omega, out, s, stream);
          })))
       return rc;
     if ((rc = hook(hooks ? hooks->read_done : nullptr, c))) return rc;
-    if (dn.rows > 0 && (rc = hook(hooks ? hooks->need_inputs : nullptr, c + 1))) return rc;
+    if (!lookahead && dn.rows > 0 && (rc = hook(hooks ? hooks->need_inputs : nullptr, c + 1)))
+      return rc;
     if ((rc = run(st, K_BSORT, stream,
                   [&] { return launch_bsort(d, s, dn, Q, q_dtype, stream); })))
       return rc;
@@ -424,8 +433,9 @@ cudaGraphExec_t capture_chunks(fwpkm_state *st, const StepKey &key) {
     return nullptr;
   }
   const fwpkm_status rc =
-      enqueue_chunks(st, key.B, key.T, key.Q, key.q_dtype, key.Vt, key.v_dtype, key.gate, key.eta,
-                     key.lam, key.out, key.x, st->capture_stream);
+      enqueue_chunks(st, key.B, key.T, key.Q, key.q_dtype, key.Vt, key.v_dtype, key.gate,
+                     key.omega, key.lookahead, key.eta, key.lam, key.out, key.x,
+                     st->capture_stream);
   cudaGraph_t graph = nullptr;
   const cudaError_t e = cudaStreamEndCapture(st->capture_stream, &graph);
   cudaGraphExec_t exec = nullptr;
@@ -582,13 +592,16 @@ fwpkm_status fwpkm_set_graphs(fwpkm_state *st, int enable) {
   return FWPKM_OK;
 }
 
-fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtype,
-                        const void *Vtarget, int v_dtype, const float *gate, float eta,
-                        float lambda_entropy, float *out, void *stream_) {
+fwpkm_status fwpkm_step_ex(fwpkm_state *st, int B, int T, const void *Q, int q_dtype,
+                           const void *Vtarget, int v_dtype, const float *gate,
+                           const float *omega, int flags, float eta, float lambda_entropy,
+                           float *out, void *stream_) {
   if (!st) return fail(FWPKM_EINVAL, "step: state is NULL");
   if (!Q || !Vtarget || !gate || !out) return fail(FWPKM_EINVAL, "step: NULL tensor pointer");
   if (!is_dtype(q_dtype) || !is_dtype(v_dtype))
     return fail(FWPKM_EINVAL, "step: dtype must be FWPKM_F32 or FWPKM_BF16");
+  if (flags & ~FWPKM_LOOKAHEAD) return fail(FWPKM_EINVAL, "step: unknown flags 0x%x", flags);
+  const int lookahead = (flags & FWPKM_LOOKAHEAD) ? 1 : 0;
   if (B < 1 || T < 1) return fail(FWPKM_ESHAPE, "step: B=%d and T=%d must be >= 1", B, T);
   if (!(eta >= 0.f) || !std::isfinite(eta))
     return fail(FWPKM_EINVAL, "step: eta must be finite and >= 0");
@@ -615,12 +628,13 @@ fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtyp
   const Extras x = st->x;
   st->x = Extras{};  // armed extras apply to this step only
   if (!st->graphs || st->profiling)
-    return enqueue_chunks(st, B, T, Q, q_dtype, Vtarget, v_dtype, gate, eta, lambda_entropy, out,
-                          x, stream);
+    return enqueue_chunks(st, B, T, Q, q_dtype, Vtarget, v_dtype, gate, omega, lookahead, eta,
+                          lambda_entropy, out, x, stream);
   // A call that repeats an earlier call's arguments replays a CUDA graph of
   // its whole chunk sequence (captured the second time the arguments are
   // seen); anything else is launched kernel by kernel.
-  const StepKey key{B, T, q_dtype, v_dtype, Q, Vtarget, gate, out, eta, lambda_entropy, x};
+  const StepKey key{B,   T,         q_dtype, v_dtype, Q,  Vtarget, gate, omega, lookahead,
+                    out, eta, lambda_entropy, x};
   for (auto &g : st->graph_cache) {
     if (g.key == key) {
       g.last_use = ++st->graph_tick;
@@ -639,13 +653,13 @@ fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtyp
   if (!seen) {
     if (st->graph_seen.size() >= kGraphSeen) st->graph_seen.erase(st->graph_seen.begin());
     st->graph_seen.push_back(key);
-    return enqueue_chunks(st, B, T, Q, q_dtype, Vtarget, v_dtype, gate, eta, lambda_entropy, out,
-                          x, stream);
+    return enqueue_chunks(st, B, T, Q, q_dtype, Vtarget, v_dtype, gate, omega, lookahead, eta,
+                          lambda_entropy, out, x, stream);
   }
   cudaGraphExec_t exec = capture_chunks(st, key);
   if (!exec)  // not capturable here: launch directly (reports any real error)
-    return enqueue_chunks(st, B, T, Q, q_dtype, Vtarget, v_dtype, gate, eta, lambda_entropy, out,
-                          x, stream);
+    return enqueue_chunks(st, B, T, Q, q_dtype, Vtarget, v_dtype, gate, omega, lookahead, eta,
+                          lambda_entropy, out, x, stream);
   if (st->graph_cache.size() >= kGraphCache) {
     size_t lru = 0;
     for (size_t i = 1; i < st->graph_cache.size(); ++i)
@@ -658,14 +672,24 @@ fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtyp
   return e == cudaSuccess ? FWPKM_OK : cuda_fail(e, "step: graph launch");
 }
 
-fwpkm_status fwpkm_step_host(fwpkm_state *st, int B, int T, const void *Q_host, int q_dtype,
-                             const void *Vt_host, int v_dtype, const float *gate_host,
-                             float eta, float lambda_entropy, float *out_host, void *stream_) {
+fwpkm_status fwpkm_step(fwpkm_state *st, int B, int T, const void *Q, int q_dtype,
+                        const void *Vtarget, int v_dtype, const float *gate, float eta,
+                        float lambda_entropy, float *out, void *stream) {
+  return fwpkm_step_ex(st, B, T, Q, q_dtype, Vtarget, v_dtype, gate, nullptr, 0, eta,
+                       lambda_entropy, out, stream);
+}
+
+fwpkm_status fwpkm_step_host_ex(fwpkm_state *st, int B, int T, const void *Q_host, int q_dtype,
+                                const void *Vt_host, int v_dtype, const float *gate_host,
+                                const float *omega_host, int flags, float eta,
+                                float lambda_entropy, float *out_host, void *stream_) {
   if (!st) return fail(FWPKM_EINVAL, "step_host: state is NULL");
   if (!Q_host || !Vt_host || !gate_host || !out_host)
     return fail(FWPKM_EINVAL, "step_host: NULL tensor pointer");
   if (!is_dtype(q_dtype) || !is_dtype(v_dtype))
     return fail(FWPKM_EINVAL, "step_host: dtype must be FWPKM_F32 or FWPKM_BF16");
+  if (flags & ~FWPKM_LOOKAHEAD) return fail(FWPKM_EINVAL, "step_host: unknown flags 0x%x", flags);
+  const int lookahead = (flags & FWPKM_LOOKAHEAD) ? 1 : 0;
   if (B < 1 || T < 1) return fail(FWPKM_ESHAPE, "step_host: B=%d and T=%d must be >= 1", B, T);
   if (!(eta >= 0.f) || !std::isfinite(eta))
     return fail(FWPKM_EINVAL, "step_host: eta must be finite and >= 0");
@@ -690,7 +714,9 @@ fwpkm_status fwpkm_step_host(fwpkm_state *st, int B, int T, const void *Q_host, 
   const size_t grow = 4, orow = (size_t)st->dv * 4;
   const size_t tok = (size_t)B * T;
   const size_t oq = 0, ov = align_up(tok * qrow, 256), og = ov + align_up(tok * vrow, 256),
-               oo = og + align_up(tok * grow, 256), total = oo + align_up(tok * orow, 256);
+               ow = og + align_up(tok * grow, 256),
+               oo = ow + (omega_host ? align_up(tok * grow, 256) : 0),
+               total = oo + align_up(tok * orow, 256);
   if (total > st->stage_bytes) {
     cudaDeviceSynchronize();
     cudaFree(st->stage);
@@ -742,6 +768,9 @@ fwpkm_status fwpkm_step_host(fwpkm_state *st, int B, int T, const void *Q_host, 
     if (e == cudaSuccess)
       e = cudaMemcpy2DAsync(base + og + t0 * grow, T * grow, (const char *)gate_host + t0 * grow,
                             T * grow, tc * grow, B, cudaMemcpyHostToDevice, st->h2d_stream);
+    if (e == cudaSuccess && omega_host)
+      e = cudaMemcpy2DAsync(base + ow + t0 * grow, T * grow, (const char *)omega_host + t0 * grow,
+                            T * grow, tc * grow, B, cudaMemcpyHostToDevice, st->h2d_stream);
     if (e == cudaSuccess) e = cudaEventRecord(in_ev[c], st->h2d_stream);
   }
   if (e != cudaSuccess) rc = cuda_fail(e, "step_host: host-to-device copy");
@@ -761,8 +790,9 @@ fwpkm_status fwpkm_step_host(fwpkm_state *st, int B, int T, const void *Q_host, 
       return r;
     };
     rc = enqueue_chunks(st, B, T, base + oq, q_dtype, base + ov, v_dtype,
-                        (const float *)(base + og), eta, lambda_entropy, (float *)(base + oo), x,
-                        stream, &hooks);
+                        (const float *)(base + og),
+                        omega_host ? (const float *)(base + ow) : nullptr, lookahead, eta,
+                        lambda_entropy, (float *)(base + oo), x, stream, &hooks);
   }
   // everything this call enqueued is done before it returns (and before its
   // events go back to the pool)
@@ -777,6 +807,13 @@ fwpkm_status fwpkm_step_host(fwpkm_state *st, int B, int T, const void *Q_host, 
     return cuda_fail(s1 != cudaSuccess ? s1 : (s2 != cudaSuccess ? s2 : s3),
                      "step_host: synchronise");
   return FWPKM_OK;
+}
+
+fwpkm_status fwpkm_step_host(fwpkm_state *st, int B, int T, const void *Q_host, int q_dtype,
+                             const void *Vt_host, int v_dtype, const float *gate_host,
+                             float eta, float lambda_entropy, float *out_host, void *stream) {
+  return fwpkm_step_host_ex(st, B, T, Q_host, q_dtype, Vt_host, v_dtype, gate_host, nullptr, 0,
+                            eta, lambda_entropy, out_host, stream);
 }
 
 fwpkm_status fwpkm_state_get(const fwpkm_state *st, float *subkeys, float *values, void *stream) {

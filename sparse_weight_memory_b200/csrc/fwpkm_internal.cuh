@@ -77,6 +77,7 @@ struct Dims {
   float eps, eta, lam;
   long long mbar_polls;  // bound of the first wait on an mbarrier (score ring, read copies)
   long long scan_polls;  // bound of a scan CTA's wait for an earlier CTA's total
+  int lookahead;         // token t is written towards the target of token t+1
 };
 
 // Device scratch owned by the state (sized for the largest chunk seen).
@@ -370,8 +371,12 @@ cudaError_t launch_topk(const Dims &d, const Scratch &s, const Extras &x, cudaSt
 cudaError_t launch_topk_select(const Dims &d, const Scratch &s, const Extras &x,
                                cudaStream_t st);
 cudaError_t launch_scan(const Dims &d, const Scratch &s, cudaStream_t st);
+// omega: the tokens' MSE weights [B][T] (null: the gate).
 cudaError_t launch_read(const Dims &d, const float *V, const void *Vt, int v_dtype,
-                        const float *gate, float *out, const Scratch &s, cudaStream_t st);
+                        const float *gate, const float *omega, float *out, const Scratch &s,
+                        cudaStream_t st);
+// Whether the read stages its rows in shared memory at these shapes.
+bool read_is_staged(const Dims &d);
 // The bucket sort; with dn.rows > 0 extra CTAs also prepare the query halves
 // of the next chunk dn (nothing reads this chunk's halves after the score).
 cudaError_t launch_bsort(const Dims &d, const Scratch &s, const Dims &dn, const void *Q,

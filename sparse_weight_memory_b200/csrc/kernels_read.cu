@@ -5,9 +5,14 @@
 //   yhat_t = (1/H) sum_h sum_r w_{t,h,r} V[slot_{t,h,r}]
 //   out_t  = g_t * yhat_t
 // and, for the write that follows (MSE memorisation loss weighted by the
-// token's gate, sciencestack table of contents sections 8-12):
+// token's importance, sciencestack table of contents sections 8-12):
 //   e_t          = yhat_t - v_t
-//   dL/dw_{t,h,r} = (2 g_t / H) e_t . V[slot_{t,h,r}]   (pre-update rows)
+//   dL/dw_{t,h,r} = (2 w_t / H) e_t . V[slot_{t,h,r}]   (pre-update rows)
+// The token weight w_t is the caller's omega_t, or the gate g_t when no
+// omega is given.  With the lookahead pairing (gist.science section 2,
+// lookahead targets) token t is written towards v_{t+1}: the target row is
+// the next token's, and the last token of the call, which has no target, is
+// read with weight 0.
 // and, when the entropy term is off (so dL/dw is complete here), the softmax
 // Jacobian dL/ds_r = w_r (dL/dw_r - sum_r' w_r' dL/dw_r') and, per sub-key
 // entry, alpha = (sum of dL/ds over its pairs) / (eps + d).
@@ -114,6 +119,7 @@ template <typename TV, bool kStaged>
 __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__restrict__ V,
                                                        const TV *__restrict__ Vt,
                                                        const float *__restrict__ gate,
+                                                       const float *__restrict__ omega,
                                                        float *__restrict__ out, Scratch s, int G,
                                                        int per) {
   griddep_wait();
@@ -144,6 +150,9 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   const int b = row / d.Tc, tl = row % d.Tc;
   const int64_t tok = (int64_t)b * d.T + d.t0 + tl;
   const int64_t p0 = (int64_t)row * HK;
+  // target row of the token, and whether it has one (lookahead: the next token's)
+  const bool last = d.lookahead && d.t0 + tl == d.T - 1;
+  const int64_t ttok = d.lookahead && !last ? tok + 1 : tok;
 
   // Everything that does not depend on the rows is loaded at once: the
   // token's pairs, this CTA's entries (x = rank mod G), the gate and the
@@ -170,6 +179,7 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
       bulk_g2s(rows_s + (size_t)(j - j0) * dv, V + (int64_t)slot_s[j] * dv, row_bytes, bar);
   }
   const float g = gate[tok];
+  const float om = last ? 0.f : (omega ? omega[tok] : g);  // the token's MSE weight
   const float invH = 1.f / (float)d.H;
   // the token's target row, loaded now so that it is here when e is formed
   constexpr int kVt = 4;  // float4 per thread held (dv <= 4 * 4 * kReadThreads)
@@ -177,7 +187,7 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
 #pragma unroll
   for (int q = 0; q < kVt; ++q) {
     const int c4 = tid + q * kReadThreads;
-    vt[q] = c4 < dv4 ? load4(Vt, tok * dv + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    vt[q] = c4 < dv4 ? load4(Vt, ttok * dv + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 
   // Member records go to their buckets while the gather is in flight (none
@@ -193,7 +203,7 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
     m.id = (uint32_t)p;
     m.srow = row;
     m.gstart = 0;
-    m.coef = 2.f * g * w * invH;
+    m.coef = 2.f * om * w * invH;
     m.c0 = w * invH;
     m.c1 = w;
     m.glen = 0;
@@ -264,7 +274,7 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   __syncthreads();
 
   // dL/dw of this CTA's pairs: warp `wid` takes pairs j0 + wid, j0 + wid + 4, ...
-  const float coef = 2.f * g * invH;
+  const float coef = 2.f * om * invH;
   for (int j = j0 + wid; j < j1; j += kReadThreads / 32) {
     const float *vr = kStaged ? rows_s + (size_t)(j - j0) * dv : V + (int64_t)slot_s[j] * dv;
     float acc = 0.f;
@@ -332,21 +342,25 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
 
 template <typename TV>
 static cudaError_t launch_read_t(const Dims &d, const float *V, const TV *Vt, const float *gate,
-                                 float *out, const Scratch &s, cudaStream_t st) {
+                                 const float *omega, float *out, const Scratch &s,
+                                 cudaStream_t st) {
   const ReadPlan p = read_plan(d);
   auto kernel = p.staged ? k_read<TV, true> : k_read<TV, false>;
   cudaError_t e =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
   if (e != cudaSuccess) return e;
   return launch_kc(d.pdl, p.G, kernel, d.rows * p.G, kReadThreads, p.smem, st, d, V, Vt, gate,
-                   out, s, p.G, p.per);
+                   omega, out, s, p.G, p.per);
 }
 
 cudaError_t launch_read(const Dims &d, const float *V, const void *Vt, int v_dtype,
-                        const float *gate, float *out, const Scratch &s, cudaStream_t st) {
+                        const float *gate, const float *omega, float *out, const Scratch &s,
+                        cudaStream_t st) {
   if (v_dtype == 1)
-    return launch_read_t(d, V, (const __nv_bfloat16 *)Vt, gate, out, s, st);
-  return launch_read_t(d, V, (const float *)Vt, gate, out, s, st);
+    return launch_read_t(d, V, (const __nv_bfloat16 *)Vt, gate, omega, out, s, st);
+  return launch_read_t(d, V, (const float *)Vt, gate, omega, out, s, st);
 }
+
+bool read_is_staged(const Dims &d) { return read_plan(d).staged; }
 
 }  // namespace fwpkm

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libfwpkm.so")
 FWPKM_OK, FWPKM_EINVAL, FWPKM_ESHAPE, FWPKM_ENOMEM, FWPKM_ECUDA, FWPKM_EUNSUPPORTED = (
     0, -1, -2, -3, -4, -5)
 FWPKM_F32, FWPKM_BF16 = 0, 1
+FWPKM_LOOKAHEAD = 1
 STATUS_NAMES = {0: "OK", -1: "EINVAL", -2: "ESHAPE", -3: "ENOMEM", -4: "ECUDA",
                 -5: "EUNSUPPORTED"}
 
@@ -50,6 +51,9 @@ def load_library():
     L.fwpkm_state_set_eps.argtypes = [_vp, f32]
     L.fwpkm_step.argtypes = [_vp, i32, i32, _vp, i32, _vp, i32, _vp, f32, f32, _vp, _vp]
     L.fwpkm_step_host.argtypes = [_vp, i32, i32, _vp, i32, _vp, i32, _vp, f32, f32, _vp, _vp]
+    L.fwpkm_step_ex.argtypes = [_vp, i32, i32, _vp, i32, _vp, i32, _vp, _vp, i32, f32, f32, _vp,
+                                _vp]
+    L.fwpkm_step_host_ex.argtypes = L.fwpkm_step_ex.argtypes
     L.fwpkm_state_get.argtypes = [_vp, _vp, _vp, _vp]
     L.fwpkm_state_set.argtypes = [_vp, _vp, _vp, _vp]
     L.fwpkm_record_selection.argtypes = [_vp, _vp, _vp]
@@ -65,6 +69,7 @@ def load_library():
     L.fwpkm_inject_alloc_failures.argtypes = [i32]
     L.fwpkm_inject_alloc_failures.restype = None
     for name in ("fwpkm_state_init", "fwpkm_state_set_eps", "fwpkm_step", "fwpkm_step_host",
+                 "fwpkm_step_ex", "fwpkm_step_host_ex",
                  "fwpkm_state_get", "fwpkm_state_set", "fwpkm_record_selection",
                  "fwpkm_force_selection", "fwpkm_set_profiling", "fwpkm_profile_read",
                  "fwpkm_read_stats", "fwpkm_select_noalloc", "fwpkm_set_graphs",
@@ -164,26 +169,44 @@ class FwPKMState:
         return subkeys, values
 
     # -- the step ----------------------------------------------------------
-    def step(self, Q, Vt, gate, eta: float, lam: float = 0.0, out=None, stream=None):
-        """Device step: Q [B,T,H*dq], Vt [B,T,dv] (fp32 or bf16), gate [B,T] fp32."""
+    def step(self, Q, Vt, gate, eta: float, lam: float = 0.0, out=None, stream=None,
+             omega=None, lookahead: bool = False):
+        """Device step: Q [B,T,H*dq], Vt [B,T,dv] (fp32 or bf16), gate [B,T] fp32.
+        ``omega`` [B,T] fp32: the tokens' MSE weights (default: the gate);
+        ``lookahead``: query t is written towards the target of token t+1."""
         import torch
         B, T = gate.shape
         if out is None:
             out = torch.empty((B, T, self.dv), dtype=torch.float32, device=gate.device)
-        _check(load_library().fwpkm_step(self._h, B, T, _ptr(Q), _dtype_code(Q), _ptr(Vt),
-                                         _dtype_code(Vt), _ptr(gate), eta, lam, _ptr(out),
-                                         _stream(stream)))
+        L = load_library()
+        if omega is None and not lookahead:
+            _check(L.fwpkm_step(self._h, B, T, _ptr(Q), _dtype_code(Q), _ptr(Vt),
+                                _dtype_code(Vt), _ptr(gate), eta, lam, _ptr(out),
+                                _stream(stream)))
+        else:
+            _check(L.fwpkm_step_ex(self._h, B, T, _ptr(Q), _dtype_code(Q), _ptr(Vt),
+                                   _dtype_code(Vt), _ptr(gate), _ptr(omega),
+                                   FWPKM_LOOKAHEAD if lookahead else 0, eta, lam, _ptr(out),
+                                   _stream(stream)))
         return out
 
     def step_host(self, Q: np.ndarray, Vt: np.ndarray, gate: np.ndarray, eta: float,
-                  lam: float = 0.0, out: Optional[np.ndarray] = None, stream=None):
+                  lam: float = 0.0, out: Optional[np.ndarray] = None, stream=None,
+                  omega: Optional[np.ndarray] = None, lookahead: bool = False):
         """Host-buffer step (copies in and out inside the call; synchronous)."""
         B, T = gate.shape
         if out is None:
             out = np.empty((B, T, self.dv), dtype=np.float32)
-        _check(load_library().fwpkm_step_host(self._h, B, T, _ptr(Q), _dtype_code(Q), _ptr(Vt),
-                                              _dtype_code(Vt), _ptr(gate), eta, lam, _ptr(out),
-                                              _stream(stream)))
+        L = load_library()
+        if omega is None and not lookahead:
+            _check(L.fwpkm_step_host(self._h, B, T, _ptr(Q), _dtype_code(Q), _ptr(Vt),
+                                     _dtype_code(Vt), _ptr(gate), eta, lam, _ptr(out),
+                                     _stream(stream)))
+        else:
+            _check(L.fwpkm_step_host_ex(self._h, B, T, _ptr(Q), _dtype_code(Q), _ptr(Vt),
+                                        _dtype_code(Vt), _ptr(gate), _ptr(omega),
+                                        FWPKM_LOOKAHEAD if lookahead else 0, eta, lam,
+                                        _ptr(out), _stream(stream)))
         return out
 
     # -- selection record / replay ---------------------------------------

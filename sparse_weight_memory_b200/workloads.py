@@ -62,6 +62,7 @@ class Workload:
     plant_frac: float = 0.0
     seed: int = 0
     eps: float = 1e-3
+    lookahead: bool = False  # each call writes query t towards the target of token t+1
 
     @property
     def N(self) -> int:

@@ -41,12 +41,14 @@ def to_dev(a: np.ndarray):
     return torch.from_numpy(a).cuda()
 
 
-def schedule(wl: Workload, inp: Inputs):
-    """The calls of one workload step: chained segments, each read `passes` times."""
+def schedule(wl: Workload, inp: Inputs, omega=None):
+    """The calls of one workload step: chained segments, each read `passes`
+    times; (Q, Vt, gate, omega) per call (omega None unless given)."""
     calls = []
     for c in range(wl.calls):
         sl = slice(c * wl.T, (c + 1) * wl.T)
-        seg = (inp.Q[:, sl], inp.Vt[:, sl], inp.gate[:, sl])
+        seg = (inp.Q[:, sl], inp.Vt[:, sl], inp.gate[:, sl],
+               None if omega is None else omega[:, sl])
         for _ in range(wl.passes):
             calls.append(seg)
     return calls
@@ -64,14 +66,15 @@ class RunResult:
 
 
 def oracle_run(wl: Workload, inp: Inputs, oracle, max_chunks: int = 0,
-               state=None) -> RunResult:
-    """Oracle over the workload's calls; continues `state` in place if given."""
+               state=None, omega=None) -> RunResult:
+    """Oracle over the workload's calls; continues `state` in place if given.
+    ``omega`` [B][T_total]: the tokens' MSE weights (default: the gate)."""
     st = state if state is not None else oracle.State(inp.subkeys, inp.values, topk=wl.topk,
                                                       chunk=wl.chunk, eps=wl.eps)
     outs, sels, ws, gaps, touched = [], [], [], [], 0
-    for Q, Vt, g in schedule(wl, inp):
+    for Q, Vt, g, om in schedule(wl, inp, omega):
         r = st.step(widen(Q), widen(Vt), g, wl.eta, wl.lam, want_sel=True, want_gap=True,
-                    max_chunks=max_chunks)
+                    max_chunks=max_chunks, omega=om, lookahead=wl.lookahead)
         outs.append(r["out"])
         sels.append(r["sel_slot"])
         ws.append(r["sel_w"])
@@ -82,9 +85,10 @@ def oracle_run(wl: Workload, inp: Inputs, oracle, max_chunks: int = 0,
 
 
 def gpu_run(wl: Workload, inp: Inputs, ref: Optional[RunResult] = None, force: bool = True,
-            K0=None, V0=None, with_stats: bool = False) -> RunResult:
+            K0=None, V0=None, with_stats: bool = False, omega=None) -> RunResult:
     """Run the workload through the C ABI.  With `ref` and `force`, token-heads
-    where the oracle has a near tie read the oracle's slots."""
+    where the oracle has a near tie read the oracle's slots.  ``omega`` as in
+    oracle_run; the workload's lookahead flag is passed on."""
     import torch
 
     from sparse_weight_memory_b200 import FwPKMState
@@ -94,7 +98,7 @@ def gpu_run(wl: Workload, inp: Inputs, ref: Optional[RunResult] = None, force: b
     if with_stats:
         st.read_stats(reset=True)
     outs, sels, ws, keep = [], [], [], []
-    for i, (Q, Vt, g) in enumerate(schedule(wl, inp)):
+    for i, (Q, Vt, g, om) in enumerate(schedule(wl, inp, omega)):
         B, T = g.shape
         rs = torch.empty((B, T, wl.heads, wl.topk), dtype=torch.int32, device="cuda")
         rw = torch.empty((B, T, wl.heads, wl.topk), dtype=torch.float32, device="cuda")
@@ -104,8 +108,10 @@ def gpu_run(wl: Workload, inp: Inputs, ref: Optional[RunResult] = None, force: b
             slots = to_dev(ref.sels[i].astype(np.int32))
             st.force_selection(slots, mask)
             keep += [mask, slots]
-        out = st.step(to_dev(Q), to_dev(Vt), to_dev(g), wl.eta, wl.lam)
-        keep += [rs, rw, out]
+        om_d = None if om is None else to_dev(np.ascontiguousarray(om, dtype=np.float32))
+        out = st.step(to_dev(Q), to_dev(Vt), to_dev(g), wl.eta, wl.lam, omega=om_d,
+                      lookahead=wl.lookahead)
+        keep += [rs, rw, out, om_d]
         outs.append(out)
         sels.append(rs)
         ws.append(rw)

@@ -69,3 +69,28 @@ def test_hand_step_on_gpu(entropy):
     wl, inp = padded_case(hs, lam)
     res = gpu_run(wl, inp, None, force=False, with_stats=True)
     check_against_hand_values(hs, res, lam)
+
+
+def test_hand_step_lookahead_on_gpu():
+    """The hand-worked step with the lookahead pairing q_t -> v_{t+1}: the
+    reads are those of the plain step; the write follows the fixture's
+    lookahead section (the last token, weight 0, pulls no row)."""
+    hs = load_hand_step()
+    la = hs.raw["lookahead"]
+    wl, inp = padded_case(hs, 0.0)
+    res = gpu_run(wl.replace(lookahead=True), inp, None, force=False, with_stats=True)
+    exp = hs.expected
+    assert np.array_equal(np.sort(res.sels[0].astype(np.int64), axis=-1),
+                          np.sort(np.array(exp["sel_slot"]), axis=-1))
+    out = res.outs[0]
+    check_close(out[..., :hs.dv], arr(exp["out"]), OUT_ATOL, OUT_RTOL, "lookahead out")
+    V = hs.V.copy()
+    for r, row in la["values_after"].items():
+        V[int(r)] = arr(row)
+    check_table(res.V[:, :hs.dv], V, 1e-4, "lookahead values")
+    assert not res.V[:, hs.dv:].any()
+    K = hs.K.copy()
+    for key, row in la["subkeys_after"].items():
+        K[tuple(int(v) for v in key.split(","))] = arr(row)
+    check_table(res.K[..., :hs.dq // 2], K, 1e-4, "lookahead sub-keys")
+    assert not res.K[..., hs.dq // 2:].any()
