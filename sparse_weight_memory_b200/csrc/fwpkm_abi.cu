@@ -377,6 +377,7 @@ fwpkm_status enqueue_chunks(fwpkm_state *st, int B, int T, const void *Q, int q_
   for (int c = 0; c < n_chunks; ++c) {
     Dims d = chunk_dims(st, B, T, c, eta, lambda_entropy);
     d.lookahead = lookahead;
+    d.q_tf32_exact = q_dtype == FWPKM_BF16 ? 1 : 0;
     // the next chunk of this call, whose query halves the sort prepares
     Dims dn{};
     if (c + 1 < n_chunks) dn = chunk_dims(st, B, T, c + 1, eta, lambda_entropy);

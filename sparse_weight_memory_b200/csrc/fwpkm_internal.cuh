@@ -78,10 +78,11 @@ struct Dims {
   long long mbar_polls;  // bound of the first wait on an mbarrier (score ring, read copies)
   long long scan_polls;  // bound of a scan CTA's wait for an earlier CTA's total
   int lookahead;         // token t is written towards the target of token t+1
+  int q_tf32_exact;      // the queries are bf16, so exact in TF32 (their lo part is zero)
 };
 
 // Device scratch owned by the state (sized for the largest chunk seen).
-constexpr int kScanMaxCtas = 8;  // bucket-scan CTAs: 8 x 16384 buckets
+constexpr int kScanMaxCtas = 64;  // bucket-scan CTAs: 64 x 2048 buckets
 constexpr int kKnChunks = 8;     // 128-float chunks of a sub-key row (dq/2 <= 1024)
 constexpr int kMaxChunks = 16;   // 128-float column chunks of the widest row (2048 floats)
 constexpr int kPartHead = 2 * kMaxChunks;  // partial slot header: (C, W) per column chunk
@@ -273,7 +274,10 @@ __device__ __forceinline__ void prep_query_half(const Dims &d, const TQ *__restr
   float acc = 0.f;
   for (int c = lane * 4; c < dh; c += 128) {
     const float4 v = load4(Q, src + c);
-    split_store(s.Qs_hi + o, s.Qs_lo + o, c, v);
+    // a bf16 value is its own TF32 part: no remainder to write (the score
+    // skips the remainder's product for bf16 queries)
+    if (sizeof(TQ) == 2) *reinterpret_cast<float4 *>(s.Qs_hi + o + c) = v;
+    else split_store(s.Qs_hi + o, s.Qs_lo + o, c, v);
     acc = fmaf(v.x, v.x, acc);
     acc = fmaf(v.y, v.y, acc);
     acc = fmaf(v.z, v.z, acc);

@@ -175,6 +175,7 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
     d.eps = v.eps;
     d.mbar_polls = v.mbar_polls;
     d.scan_polls = kDefaultScanPolls;
+    d.q_tf32_exact = q_dtype == FWPKM_BF16 ? 1 : 0;
     // the sub-key split once per call, the query halves once per pass
     cudaError_t ke = t0 == 0 ? launch_prep(d, Q, q_dtype, v.K, s, stream)
                              : launch_prep_q(d, Q, q_dtype, s, stream);

@@ -54,20 +54,28 @@ __device__ __forceinline__ void store_member(Member *p, const Member &m) {
 // scan: bucket offsets, one pass over up to kScanMaxCtas CTAs.  Each CTA
 // holds kScanTile counts in registers (16-byte loads), scans them, publishes
 // its total tagged with the chunk's epoch, and adds the totals of the CTAs
-// before it (all CTAs of the grid are resident together: at most 8).  The
+// before it (all CTAs of the grid are resident together: at most 64 small
+// ones).  Many small CTAs rather than one large one: the kernel is bound by
+// the load and store instructions a multiprocessor issues, not by bytes.  The
 // waits for those totals are bounded; a timeout sets ERR_SCAN_TIMEOUT.
 // Counts are zeroed for the next chunk; CTA 0 resets the work-list counters.
 // ---------------------------------------------------------------------------
-constexpr int kScanThreads = 1024;
-constexpr int kScanPer = 16;                        // counts per thread
+constexpr int kScanThreads = 256;
+constexpr int kScanWarps = kScanThreads / 32;
+constexpr int kScanPer = 8;                         // counts per thread
 constexpr int kScanTile = kScanThreads * kScanPer;  // counts per CTA
+static_assert(kScanTile * kScanMaxCtas >= 65536 + 2 * 16 * 1024, "every bucket count fits");
 
-__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+// A CTA's total is read by the later CTAs for its own value only (nothing
+// else this CTA wrote is read through it), and the epoch in its upper half
+// tells a stale word from the current one: relaxed stores and loads at GPU
+// scope are enough, and the store does not wait for the CTA's earlier ones.
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
   unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
 
@@ -81,7 +89,7 @@ __global__ void __launch_bounds__(kScanThreads) k_bucket_scan(Dims d, Scratch s)
   const unsigned long long epoch = s.scan_sync[0];  // advanced by this chunk's selection
   const int b0 = c * kScanTile + tid * kScanPer;
   int v[kScanPer];
-  if (b0 + kScanPer <= NB) {  // bcnt is 256-byte aligned and b0 a multiple of 16
+  if (b0 + kScanPer <= NB) {  // bcnt is 256-byte aligned and b0 a multiple of 8
 #pragma unroll
     for (int q = 0; q < kScanPer / 4; ++q) {
       const int4 x = *reinterpret_cast<const int4 *>(s.bcnt + b0 + 4 * q);
@@ -110,7 +118,7 @@ __global__ void __launch_bounds__(kScanThreads) k_bucket_scan(Dims d, Scratch s)
   if (lane == 31) red[w] = incl;
   __syncthreads();
   if (w == 0) {
-    int x = red[lane];
+    int x = lane < kScanWarps ? red[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int t = __shfl_up_sync(FULL, x, o);
@@ -119,24 +127,27 @@ __global__ void __launch_bounds__(kScanThreads) k_bucket_scan(Dims d, Scratch s)
     red[lane] = x;
   }
   __syncthreads();
-  const int cta_total = red[31];
+  const int cta_total = red[kScanWarps - 1];
   if (tid == 0 && gridDim.x > 1)
-    st_release_u64(&s.scan_sync[1 + c], (epoch << 32) | (unsigned)cta_total);
+    st_relaxed_u64(&s.scan_sync[1 + c], (epoch << 32) | (unsigned)cta_total);
   if (w == 0) {
+    // totals of CTAs 0 .. c-1, one per lane and round
     int pre = 0;
-    if (lane < c) {
+    bool ok_all = true;
+    for (int j = lane; j < c; j += 32) {
       bool ok = false;
       unsigned long long a = 0;
       for (long long it = 0; it < d.scan_polls; ++it) {
-        a = ld_acquire_u64(&s.scan_sync[1 + lane]);
+        a = ld_relaxed_u64(&s.scan_sync[1 + j]);
         if ((a >> 32) == (epoch & 0xffffffffull)) {
           ok = true;
           break;
         }
       }
-      if (!ok) atomicOr(&s.meta->err, ERR_SCAN_TIMEOUT);
-      pre = ok ? (int)(unsigned)a : 0;
+      ok_all = ok_all && ok;
+      pre += ok ? (int)(unsigned)a : 0;
     }
+    if (!ok_all) atomicOr(&s.meta->err, ERR_SCAN_TIMEOUT);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) pre += __shfl_xor_sync(FULL, pre, o);
     if (lane == 0) prefix_s = pre;
@@ -278,7 +289,6 @@ constexpr int kRankGroups = 256;      // groups per bucket (slots per value buck
 struct RankSmem {
   uint32_t *bits;  // [kRankWords]
   uint32_t *pre;   // [kRankWords]
-  int *gcnt;       // [kRankGroups]
   int *red;        // [32]
   int *flag;
 };
@@ -292,7 +302,6 @@ __device__ bool rank_big_bucket(const Dims &d, const Scratch &s, int off, int le
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t kdiv = value ? (uint32_t)d.k : 2u * (uint32_t)d.k;  // id -> token-head
   for (int i = tid; i < W; i += blockDim.x) r.bits[i] = 0u;
-  for (int i = tid; i < G; i += blockDim.x) r.gcnt[i] = 0;
   if (tid == 0) *r.flag = 0;
   __syncthreads();
   for (int i = tid; i < len; i += blockDim.x) {
@@ -301,7 +310,6 @@ __device__ bool rank_big_bucket(const Dims &d, const Scratch &s, int off, int le
     const uint32_t m = (uint32_t)gi.y / kdiv;
     const uint32_t bit = 1u << (m & 31u);
     if (atomicOr(&r.bits[lg * Mw + (int)(m >> 5)], bit) & bit) *r.flag = 1;
-    atomicAdd(&r.gcnt[lg], 1);
   }
   __syncthreads();
   if (*r.flag) return false;
@@ -347,8 +355,10 @@ __device__ bool rank_big_bucket(const Dims &d, const Scratch &s, int off, int le
     const int wi = lg * Mw + (int)(m >> 5);
     const int pos = (int)r.pre[wi] + __popc(r.bits[wi] & ((1u << (m & 31u)) - 1u));
     const int first = (int)r.pre[lg * Mw];
+    // every member set one bit, so the group's size is its words' popcount
+    const int end = (lg + 1) * Mw < W ? (int)r.pre[(lg + 1) * Mw] : len;
     mr.gstart = off + first;
-    mr.glen = r.gcnt[lg];
+    mr.glen = end - first;
     store_member(s.rec + off + pos, mr);
     if (pos == first) {
       my_seg += 1;
@@ -463,7 +473,7 @@ __global__ void __launch_bounds__(kSortThreads)
   __shared__ int nseg[2];  // distinct value rows / sub-key rows seen by this CTA
   __shared__ int big_n;
   __shared__ int big_b[kSortWarps * 8];  // large buckets met in phase 1
-  __shared__ int rank_gcnt[kRankGroups], rank_red[32], rank_flag;
+  __shared__ int rank_red[32], rank_flag;
   griddep_wait();
   griddep_launch();
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
@@ -572,7 +582,7 @@ __global__ void __launch_bounds__(kSortThreads)
     const uint32_t gbase =
         value ? ((uint32_t)b << d.vshift) : (uint32_t)d.N + (uint32_t)(b - d.NBv);
     const RankSmem rs{reinterpret_cast<uint32_t *>(buf), reinterpret_cast<uint32_t *>(buf) + kRankWords,
-                      rank_gcnt, rank_red, &rank_flag};
+                      rank_red, &rank_flag};
     sort_big_bucket(d, s, off, len, value, gbase, buf, rs, &nseg[value ? 0 : 1]);
   }
   __syncthreads();
@@ -812,12 +822,20 @@ __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__res
       if (!__shfl_sync(FULL, last, 0)) continue;
       __threadfence();
       const float *pp = s.partial + (size_t)slot0 * s.pwidth;
-      float Ct = 0.f, Wt = 0.f;  // block order
-      for (int b = 0; b < nb; ++b) {
+      // the blocks' scalar sums: lane b takes blocks b, b + 32, ... (in that
+      // order), then a butterfly over the lanes; one round of loads, and an
+      // order fixed by the group's length alone
+      float Ct = 0.f, Wt = 0.f;
+      for (int b = lane; b < nb; b += 32) {
         const float2 cw = __ldcg(reinterpret_cast<const float2 *>(pp + (size_t)b * s.pwidth +
                                                                   2 * chunk));
         Ct += cw.x;
         Wt += cw.y;
+      }
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        Ct += __shfl_xor_sync(FULL, Ct, o);
+        Wt += __shfl_xor_sync(FULL, Wt, o);
       }
       float *row = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.N) * d.dh;
       if (!value || Ct > 0.f) {

@@ -13,11 +13,13 @@
 // them for the sub-key rows it changes).  The dropped
 // lo*lo term and the truncation of lo are ~2^-21 relative, so the distances
 // match an fp32 evaluation to a few ulps and the selection is decided at
-// fp32 accuracy.
+// fp32 accuracy.  A bf16 query is exact in TF32 (its lo part is zero), so
+// for bf16 queries the lo*hi product and the query's lo tile are skipped:
+// two MMAs per k-step instead of three.
 //
 // CTA = one 128-row x BN-column output tile of one (head, half); 4 warps.
 //   warp 0, one lane: TMA producer over k-blocks of 32 elements (128 bytes,
-//                     128-byte swizzle), 3- to 5-deep ring;
+//                     128-byte swizzle), 2- or 3-deep ring;
 //   warp 1:           allocates the accumulator columns in tensor memory;
 //                     one lane issues the MMAs and commits each stage back;
 //   warps 0-3:        epilogue, one accumulator lane (= output row) per thread.
@@ -34,10 +36,17 @@ namespace fwpkm {
 
 constexpr int kTcRows = 128;      // M of every MMA (cta_group::1)
 constexpr int kTcKBlock = 32;     // fp32 elements per 128-byte swizzle row
-// Ring depth: as many 32-element k-blocks in flight as fit in ~200 KB.
+// Ring depth.  Up to 64 columns: two stages, so that two CTAs share a
+// multiprocessor and one's epilogue and ring fill overlap the other's MMAs
+// (measured on the 1M-slot shape: 29 -> 20 us per chunk against four stages
+// and one CTA); 128 columns: three stages, one CTA.
 template <int BN>
 constexpr int tc_stages() {
-  return BN <= 32 ? 5 : (BN <= 64 ? 4 : 3);
+  return BN <= 64 ? 2 : 3;
+}
+template <int BN>
+constexpr int tc_ctas_per_sm() {
+  return BN <= 64 ? 2 : 1;
 }
 
 // --- tcgen05 helpers (inline PTX, sm_100a) --------------------------------
@@ -129,8 +138,8 @@ struct TcSmem {
   static_assert(kStage >= 4 * 32 * 33 * 4, "epilogue tile fits in stage 0");
 };
 
-template <int BN>
-__global__ void __launch_bounds__(128, 1)
+template <int BN, bool kALo>
+__global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
     k_score_tc(const __grid_constant__ CUtensorMap mapAhi, const __grid_constant__ CUtensorMap mapAlo,
                const __grid_constant__ CUtensorMap mapBhi, const __grid_constant__ CUtensorMap mapBlo,
                Dims d, Scratch s) {
@@ -178,10 +187,10 @@ __global__ void __launch_bounds__(128, 1)
                              ERR_SCORE_TIMEOUT))
         break;
       unsigned char *stage = smem + st * L::kStage;
-      mbar_arrive_expect_tx(&full[st], L::kStage);
+      mbar_arrive_expect_tx(&full[st], kALo ? L::kStage : L::kStage - L::kA);
       const int x = kb * kTcKBlock;
       tma_load_2d(stage, &mapAhi, x, ya, &full[st]);
-      tma_load_2d(stage + L::kA, &mapAlo, x, ya, &full[st]);
+      if (kALo) tma_load_2d(stage + L::kA, &mapAlo, x, ya, &full[st]);
       tma_load_2d(stage + 2 * L::kA, &mapBhi, x, yb, &full[st]);
       tma_load_2d(stage + 2 * L::kA + L::kB, &mapBlo, x, yb, &full[st]);
     }
@@ -203,7 +212,8 @@ __global__ void __launch_bounds__(128, 1)
         const uint32_t acc = (kb > 0 || k8 > 0) ? 1u : 0u;
         mma_tf32(tmem, kmajor_sw128_desc(ahi + off), kmajor_sw128_desc(bhi + off), idesc, acc);
         mma_tf32(tmem, kmajor_sw128_desc(ahi + off), kmajor_sw128_desc(blo + off), idesc, 1u);
-        mma_tf32(tmem, kmajor_sw128_desc(alo + off), kmajor_sw128_desc(bhi + off), idesc, 1u);
+        if (kALo)
+          mma_tf32(tmem, kmajor_sw128_desc(alo + off), kmajor_sw128_desc(bhi + off), idesc, 1u);
       }
       mma_commit(&empty[st]);  // stage free once these MMAs have read it
     }
@@ -278,12 +288,13 @@ __global__ void __launch_bounds__(128, 1)
 template <int BN>
 static cudaError_t launch_tc(const Dims &d, const Scratch &s, const TcMaps &maps, int v,
                              cudaStream_t st) {
+  auto kernel = d.q_tf32_exact ? k_score_tc<BN, false> : k_score_tc<BN, true>;
   // set on every launch: the attribute belongs to the current device's context
-  cudaError_t e = cudaFuncSetAttribute(k_score_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        TcSmem<BN>::kBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((d.n + BN - 1) / BN, (d.rows + kTcRows - 1) / kTcRows, 2 * d.H);
-  return launch_k(d.pdl, k_score_tc<BN>, grid, 128, TcSmem<BN>::kBytes, st,
+  return launch_k(d.pdl, kernel, grid, 128, TcSmem<BN>::kBytes, st,
                   *reinterpret_cast<const CUtensorMap *>(maps.a_hi),
                   *reinterpret_cast<const CUtensorMap *>(maps.a_lo),
                   *reinterpret_cast<const CUtensorMap *>(maps.b_hi[v]),

@@ -8,12 +8,16 @@
 // N = n^2 slots.  Weights are the softmax of the selected slot scores.
 // Order: score descending, index ascending on ties.
 //
-// One warp per token-head.  Each lane holds n/32 squared distances of a half
-// in registers; an MSB-first bisection over the fp32 bit patterns (distances
-// are >= 0, so the bit order is the value order) finds the k smallest, which
-// are compacted one per lane.  For the merge each lane holds one row of the
-// k*k candidate grid and the same bisection, over order-preserving keys of
-// the negated scores, picks the k best.
+// Two warps per token-head, one per half.  Each lane holds n/32 squared
+// distances of its half in registers; an MSB-first bisection over the fp32
+// bit patterns (distances are >= 0, so the bit order is the value order)
+// finds the k smallest, which are compacted one per lane and sorted by
+// (score desc, index asc).  The merge then searches only the candidates
+// (a, b) of half-1 rank a and half-2 rank b with (a+1)(b+1) <= k, with the
+// same bisection over order-preserving keys of the negated scores; an exact
+// score tie with a candidate outside that set sends the token-head through
+// the full k*k merge, so the result is exactly the top-k under (score desc,
+// slot asc).
 #include <math_constants.h>
 
 #include "fwpkm_internal.cuh"
@@ -133,6 +137,15 @@ __device__ __forceinline__ uint32_t float_order(float x) {
 
 // Top-k smallest distances of one half row drow[0..n) (n <= 32*NV), ties by
 // index.  Lane r < k returns one winner (distance, index); order unspecified.
+// wbuf holds 64 entries.
+//
+// With 4 or more entries per lane the search is narrowed first: every lane
+// offers its two smallest keys, and the k-th smallest t0 of those 64 is at
+// least the k-th smallest of the whole row (they are a subset of it).  So the
+// top-k are among the keys <= t0 -- about 1.5k of them for continuous data --
+// which are gathered two per lane and selected exactly.  Past 64 such keys
+// (heavy ties) the whole row is searched instead.  Either way the result is
+// the exact top-k under (key asc, index asc).
 template <int NV>
 __device__ __forceinline__ void half_topk(const float *__restrict__ drow, int n, int k,
                                           float &d_out, int &i_out, uint2 *wbuf) {
@@ -146,150 +159,314 @@ __device__ __forceinline__ void half_topk(const float *__restrict__ drow, int n,
     key[v] = i < n ? min(__float_as_uint(drow[i]), 0xfffffffeu) : 0xffffffffu;
     idx[v] = (uint32_t)i;
   }
-  const uint32_t sel = warp_select_smallest<NV>(key, idx, k);
   uint32_t kk, ii;
   int v_out, src;
+  if (NV >= 4) {
+    // the two smallest keys of this lane (n > 96: every lane has two)
+    uint32_t m1 = 0xffffffffu, m2 = 0xffffffffu;
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const uint32_t x = key[v];
+      m2 = min(m2, max(m1, x));
+      m1 = min(m1, x);
+    }
+    const uint32_t pk[2] = {m1, m2};
+    const uint32_t pt[2] = {(uint32_t)lane, (uint32_t)lane + 32u};
+    const uint32_t psel = warp_select_smallest<2>(pk, pt, k);
+    const uint32_t t0 = __reduce_max_sync(
+        FULL, max((psel & 1u) ? m1 : 0u, (psel & 2u) ? m2 : 0u));
+    // gather the keys <= t0, up to 64, in (lane, v) order
+    int cnt = 0;
+#pragma unroll
+    for (int v = 0; v < NV; ++v) cnt += key[v] <= t0 ? 1 : 0;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(FULL, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const int total = __shfl_sync(FULL, incl, 31);
+    if (total <= 64) {
+      int pos = incl - cnt;
+#pragma unroll
+      for (int v = 0; v < NV; ++v)
+        if (key[v] <= t0) wbuf[pos++] = make_uint2(key[v], idx[v]);
+      __syncwarp();
+      uint32_t ck[2], ci[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int c = lane + 32 * q;
+        const uint2 e = c < total ? wbuf[c] : make_uint2(0xffffffffu, 0xffffffffu);
+        ck[q] = e.x;
+        ci[q] = e.y;
+      }
+      __syncwarp();
+      const uint32_t sel = warp_select_smallest<2>(ck, ci, k);
+      compact_selected<2>(sel, ck, ci, wbuf, kk, ii, v_out, src);
+      d_out = __uint_as_float(kk);
+      i_out = (int)ii;
+      return;
+    }
+  }
+  const uint32_t sel = warp_select_smallest<NV>(key, idx, k);
   compact_selected<NV>(sel, key, idx, wbuf, kk, ii, v_out, src);
   d_out = __uint_as_float(kk);
   i_out = (int)ii;
 }
 
+// Bitonic sort of one 64-bit key per lane, ascending across the warp; `src`
+// follows each key to the lane it came from.
+__device__ __forceinline__ uint64_t shfl_xor64(uint64_t v, int o) {
+  const uint32_t lo = __shfl_xor_sync(FULL, (uint32_t)v, o);
+  const uint32_t hi = __shfl_xor_sync(FULL, (uint32_t)(v >> 32), o);
+  return ((uint64_t)hi << 32) | lo;
+}
+__device__ __forceinline__ uint64_t warp_sort_asc(uint64_t key, int &src) {
+  const int lane = threadIdx.x & 31;
+  src = lane;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int st = size >> 1; st > 0; st >>= 1) {
+      const uint64_t ok = shfl_xor64(key, st);
+      const int os = __shfl_xor_sync(FULL, src, st);
+      const bool up = (lane & size) == 0;
+      const bool lower = (lane & st) == 0;
+      const bool keep = (lower == up) ? (key <= ok) : (key >= ok);
+      if (!keep) {
+        key = ok;
+        src = os;
+      }
+    }
+  }
+  return key;
+}
+
+// Candidates of the merge: with both halves' winners sorted by (score desc,
+// index asc), rank a of half 1 and rank b of half 2, every candidate (a, b)
+// of the top-k has (a+1)(b+1) <= k -- the (a+1)(b+1) - 1 candidates it
+// dominates rank ahead of it -- so only that staircase (130 candidates for
+// k = 32, instead of k^2 = 1024) is searched.  Per token-head, at most
+// kMergeV candidates per lane.
+constexpr int kMergeV = 5;
+constexpr int kTopkHeads = 4;  // token-heads per CTA, two warps each
+
+// Per-CTA shared memory of the selection.
+struct TopkSmem {
+  float s[kTopkHeads][2][32];     // winners of each half, sorted: score,
+  float dist[kTopkHeads][2][32];  //   distance,
+  int idx[kTopkHeads][2][32];     //   sub-key row
+  int fin[kTopkHeads][2][32];     // final pairs: sub-key row of each half,
+  float find[kTopkHeads][2][32];  //   and its distance
+  uint2 wbuf[2 * kTopkHeads][64];
+  uint16_t cand[kMergeV * 32];    // staircase candidates, (a << 8) | b
+  int ncand;
+};
+
 // kSelectOnly: write only the selection record (x.rec_slots / x.rec_w); no
 // pair, entry or bucket outputs.
+//
+// CTA = kTopkHeads token-heads, two warps each: warp 2t + half selects the
+// top-k of its half and sorts them; warp 2t merges; then each warp writes
+// its half's sub-key entries.  A token-head whose selection is forced reads
+// the given slots instead.
 template <int NV, int KV, bool kSelectOnly>
-__global__ void __launch_bounds__(128) k_topk(Dims d, Scratch s, Extras x) {
-  __shared__ uint2 wbuf_all[4][32];
+__global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Extras x) {
+  __shared__ TopkSmem sm;
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
-  const int m = blockIdx.x * 4 + wib;  // token-head m = row*H + h
+  const int t = wib >> 1, half = wib & 1;
+  const int m = blockIdx.x * kTopkHeads + t;  // token-head m = row*H + h
+  const int k = d.k, n = d.n;
+  const float eps = d.eps;
+  // the staircase for this k (warp 0, before the halves are selected)
+  if (wib == 0) {
+    const int len = lane < k ? min(k, k / (lane + 1)) : 0;
+    int incl = len;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(FULL, incl, o);
+      if (lane >= o) incl += v;
+    }
+    for (int b = 0; b < len; ++b) sm.cand[incl - len + b] = (uint16_t)((lane << 8) | b);
+    if (lane == 31) sm.ncand = incl;
+  }
   griddep_wait();
   griddep_launch();
   // a new chunk epoch for the bucket scan that follows (the step, not the selection-only call)
   if (!kSelectOnly && blockIdx.x == 0 && threadIdx.x == 0) s.scan_sync[0] += 1ull;
-  if (m >= d.M) return;
-  const int row = m / d.H, h = m % d.H;
-  const int k = d.k, n = d.n;
-  const float eps = d.eps;
-  uint2 *wbuf = wbuf_all[wib];
+  const bool valid = m < d.M;
+  const int row = valid ? m / d.H : 0, h = valid ? m % d.H : 0;
   const float *D1 = s.D + ((int64_t)(h * 2 + 0) * d.rows + row) * n;
   const float *D2 = s.D + ((int64_t)(h * 2 + 1) * d.rows + row) * n;
 
   // Global token coordinates of this row (for the optional per-token arrays).
   const int b = row / d.Tc, tl = row % d.Tc;
   const int64_t th = ((int64_t)b * d.T + d.t0 + tl) * d.H + h;  // [B][T][H] index
+  const bool forced = valid && x.force_mask != nullptr && x.force_mask[th] != 0;
 
-  float s_r = -CUDART_INF_F, d1_r = 0.f, d2_r = 0.f;
-  int slot_r = 0, i_r = 0, j_r = 0;
-  const bool forced = x.force_mask != nullptr && x.force_mask[th] != 0;
-  if (forced) {
+  // ---- each half: top-k, sorted by (score desc, index asc) ----
+  if (valid && !forced) {
+    float dw;
+    int iw;
+    half_topk<NV>(half == 0 ? D1 : D2, n, k, dw, iw, sm.wbuf[wib]);
+    const float sw = -logf(eps + dw);
+    const uint64_t key =
+        lane < k ? ((uint64_t)float_order(-sw) << 32) | (uint32_t)iw : ~0ull;
+    int src;
+    const uint64_t sk = warp_sort_asc(key, src);
+    const float s_sorted = __shfl_sync(FULL, sw, src);
+    const float d_sorted = __shfl_sync(FULL, dw, src);
     if (lane < k) {
-      int64_t sl = x.force_slots[th * k + lane];
-      sl = sl < 0 ? 0 : (sl >= d.N ? d.N - 1 : sl);
-      slot_r = (int)sl;
-      i_r = slot_r / n;
-      j_r = slot_r % n;
-      d1_r = D1[i_r];
-      d2_r = D2[j_r];
-      s_r = -logf(eps + d1_r) - logf(eps + d2_r);
+      sm.s[t][half][lane] = s_sorted;
+      sm.dist[t][half][lane] = d_sorted;
+      sm.idx[t][half][lane] = (int)(uint32_t)sk;
     }
-  } else {
-    float da, db;
-    int ia, jb;
-    half_topk<NV>(D1, n, k, da, ia, wbuf);
-    half_topk<NV>(D2, n, k, db, jb, wbuf);
-    const float sa = -logf(eps + da);  // lane a < k: one winner of half 1
-    const float sb = -logf(eps + db);  // lane b < k: one winner of half 2
-    // Lane a holds row a of the k x k candidate grid: s = sa + sb[b], slot =
-    // ia * n + jb[b]; the k best candidates (score desc, slot asc) are the
-    // k smallest keys of the negated scores, ties by slot.
-    uint32_t key[KV], slot[KV];
+  }
+  __syncthreads();
+
+  // ---- merge (warp 2t) ----
+  float s_r = -CUDART_INF_F;
+  int slot_r = 0;
+  if (valid && half == 0) {
+    int i_r = 0, j_r = 0;
+    float d1_r = 0.f, d2_r = 0.f;
+    if (forced) {
+      if (lane < k) {
+        int64_t sl = x.force_slots[th * k + lane];
+        sl = sl < 0 ? 0 : (sl >= d.N ? d.N - 1 : sl);
+        slot_r = (int)sl;
+        i_r = slot_r / n;
+        j_r = slot_r % n;
+        d1_r = D1[i_r];
+        d2_r = D2[j_r];
+        s_r = -logf(eps + d1_r) - logf(eps + d2_r);
+      }
+    } else {
+      const float *S1 = sm.s[t][0], *S2 = sm.s[t][1];
+      const int *I1 = sm.idx[t][0], *I2 = sm.idx[t][1];
+      const int nc = sm.ncand;
+      uint32_t key[kMergeV], slot[kMergeV];
 #pragma unroll
-    for (int b = 0; b < KV; ++b) {
-      const float s2 = __shfl_sync(FULL, sb, b);
-      const int j2 = __shfl_sync(FULL, jb, b);
-      const bool ok = lane < k && b < k;
-      key[b] = ok ? float_order(-(sa + s2)) : 0xffffffffu;
-      slot[b] = ok ? (uint32_t)(ia * n + j2) : 0xffffffffu;
+      for (int v = 0; v < kMergeV; ++v) {
+        const int c = lane + 32 * v;
+        key[v] = slot[v] = 0xffffffffu;
+        if (c < nc) {
+          const int a = sm.cand[c] >> 8, bb = sm.cand[c] & 255;
+          key[v] = float_order(-(S1[a] + S2[bb]));
+          slot[v] = (uint32_t)(I1[a] * n + I2[bb]);
+        }
+      }
+      const uint32_t sel = warp_select_smallest<kMergeV>(key, slot, k);
+      uint32_t wkey, wslot;
+      int v_out, src;
+      compact_selected<kMergeV>(sel, key, slot, sm.wbuf[wib], wkey, wslot, v_out, src);
+      // An exact tie of an outside candidate with the k-th score could change
+      // which equal-score slot wins the last places: take the full k x k merge.
+      const uint32_t kth = __reduce_max_sync(FULL, lane < k ? wkey : 0u);
+      bool tie = false;
+      if (lane < k)
+        for (int bb = k / (lane + 1); bb < k; ++bb)
+          tie |= float_order(-(S1[lane] + S2[bb])) == kth;
+      if (__any_sync(FULL, tie)) {
+        uint32_t fkey[KV], fslot[KV];
+        const float sa = lane < k ? S1[lane] : 0.f;
+        const int ia = lane < k ? I1[lane] : 0;
+#pragma unroll
+        for (int bb = 0; bb < KV; ++bb) {
+          const bool ok = lane < k && bb < k;
+          fkey[bb] = ok ? float_order(-(sa + S2[bb])) : 0xffffffffu;
+          fslot[bb] = ok ? (uint32_t)(ia * n + I2[bb]) : 0xffffffffu;
+        }
+        const uint32_t fsel = warp_select_smallest<KV>(fkey, fslot, k);
+        int b_out, a_out;
+        compact_selected<KV>(fsel, fkey, fslot, sm.wbuf[wib], wkey, wslot, b_out, a_out);
+        if (lane < k) {
+          i_r = I1[a_out];
+          j_r = I2[b_out];
+          s_r = S1[a_out] + S2[b_out];
+          d1_r = sm.dist[t][0][a_out];
+          d2_r = sm.dist[t][1][b_out];
+          slot_r = (int)wslot;
+        }
+      } else if (lane < k) {
+        const int c = src + 32 * v_out;
+        const int a = sm.cand[c] >> 8, bb = sm.cand[c] & 255;
+        i_r = I1[a];
+        j_r = I2[bb];
+        s_r = S1[a] + S2[bb];
+        d1_r = sm.dist[t][0][a];
+        d2_r = sm.dist[t][1][bb];
+        slot_r = (int)wslot;
+      }
     }
-    const uint32_t sel = warp_select_smallest<KV>(key, slot, k);
-    uint32_t wkey, wslot;
-    int b_out, a_out;
-    compact_selected<KV>(sel, key, slot, wbuf, wkey, wslot, b_out, a_out);
-    // winner r (lane r): row a_out of half 1, column b_out of half 2
-    const float w_sa = __shfl_sync(FULL, sa, a_out);
-    const float w_sb = __shfl_sync(FULL, sb, b_out);
-    const float w_d1 = __shfl_sync(FULL, da, a_out);
-    const float w_d2 = __shfl_sync(FULL, db, b_out);
-    const int w_i = __shfl_sync(FULL, ia, a_out);
-    const int w_j = __shfl_sync(FULL, jb, b_out);
     if (lane < k) {
-      s_r = w_sa + w_sb;
-      slot_r = (int)wslot;
-      i_r = w_i;
-      j_r = w_j;
-      d1_r = w_d1;
-      d2_r = w_d2;
+      sm.fin[t][0][lane] = i_r;
+      sm.fin[t][1][lane] = j_r;
+      sm.find[t][0][lane] = d1_r;
+      sm.find[t][1][lane] = d2_r;
+    }
+    // Softmax over the k selected scores.
+    const float smax = warp_max(lane < k ? s_r : -CUDART_INF_F);
+    const float ex = lane < k ? expf(s_r - smax) : 0.f;
+    const float z = warp_sum(ex);
+    const float w = ex / z;
+    if (kSelectOnly) {
+      if (lane < k) {
+        x.rec_slots[th * k + lane] = slot_r;
+        x.rec_w[th * k + lane] = w;
+      }
+    } else {
+      const int64_t p = (int64_t)m * k + lane;
+      if (lane < k) {
+        s.pslot[p] = slot_r;
+        s.pw[p] = w;
+        s.pclaim[p] = atomicAdd(&s.bcnt[slot_r >> d.vshift], 1);  // value bucket
+        if (x.rec_slots) {
+          x.rec_slots[th * k + lane] = slot_r;
+          x.rec_w[th * k + lane] = w;
+        }
+      }
     }
   }
+  if (kSelectOnly) return;
+  __syncthreads();
 
-  // Softmax over the k selected scores.
-  const float smax = warp_max(lane < k ? s_r : -CUDART_INF_F);
-  const float ex = lane < k ? expf(s_r - smax) : 0.f;
-  const float z = warp_sum(ex);
-  const float w = ex / z;
-
-  if (kSelectOnly) {
-    if (lane < k) {
-      x.rec_slots[th * k + lane] = slot_r;
-      x.rec_w[th * k + lane] = w;
-    }
-    return;
-  }
-  const int64_t p = (int64_t)m * k + lane;
-  if (lane < k) {
-    s.pslot[p] = slot_r;
-    s.pw[p] = w;
-    s.pclaim[p] = atomicAdd(&s.bcnt[slot_r >> d.vshift], 1);  // value bucket
-    if (x.rec_slots) {
-      x.rec_slots[th * k + lane] = slot_r;
-      x.rec_w[th * k + lane] = w;
-    }
-  }
-  // Sub-key entries: one per distinct row of each half among the k pairs.
+  // ---- sub-key entries of this warp's half: one per distinct row among the
+  // k pairs ----
+  if (!valid) return;
+  const int sub = lane < k ? sm.fin[t][half][lane] : 0;
+  const float dist = lane < k ? sm.find[t][half][lane] : 0.f;
   const unsigned act = k == 32 ? FULL : ((1u << k) - 1u);
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int sub = half == 0 ? i_r : j_r;
-    const float dist = half == 0 ? d1_r : d2_r;
-    unsigned peers = 0;
-    if (lane < k) peers = __match_any_sync(act, sub);
-    const bool leader = lane < k && (__ffs(peers) - 1) == lane;
-    const unsigned lb = __ballot_sync(FULL, leader);
-    if (leader) {
-      const int idx = __popc(lb & lanemask_lt());
-      const int64_t e = ((int64_t)m * 2 + half) * k + idx;
-      s.esub[e] = sub;
-      s.emask[e] = peers;
-      s.einv[e] = 1.f / (eps + dist);
-      s.eclaim[e] = atomicAdd(&s.bcnt[d.NBv + (h * 2 + half) * n + sub], 1);
-    }
-    // unused entry slots of this half are marked -1
-    if (lane >= __popc(lb) && lane < k) s.esub[((int64_t)m * 2 + half) * k + lane] = -1;
-    if (lane == 0) s.ecount[(int64_t)m * 2 + half] = __popc(lb);
+  unsigned peers = 0;
+  if (lane < k) peers = __match_any_sync(act, sub);
+  const bool leader = lane < k && (__ffs(peers) - 1) == lane;
+  const unsigned lb = __ballot_sync(FULL, leader);
+  if (leader) {
+    const int idx = __popc(lb & lanemask_lt());
+    const int64_t e = ((int64_t)m * 2 + half) * k + idx;
+    s.esub[e] = sub;
+    s.emask[e] = peers;
+    s.einv[e] = 1.f / (eps + dist);
+    s.eclaim[e] = atomicAdd(&s.bcnt[d.NBv + (h * 2 + half) * n + sub], 1);
   }
+  // unused entry slots of this half are marked -1
+  if (lane >= __popc(lb) && lane < k) s.esub[((int64_t)m * 2 + half) * k + lane] = -1;
+  if (lane == 0) s.ecount[(int64_t)m * 2 + half] = __popc(lb);
 }
 
 template <int KV, bool kSelectOnly>
 static cudaError_t launch_topk_kv(const Dims &d, const Scratch &s, const Extras &x,
                                   cudaStream_t st) {
-  const int blocks = (d.M + 3) / 4;
+  const int blocks = (d.M + kTopkHeads - 1) / kTopkHeads;
   const int nv = (d.n + 31) / 32;
-  if (nv <= 1) return launch_k(d.pdl, k_topk<1, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
-  if (nv <= 2) return launch_k(d.pdl, k_topk<2, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
-  if (nv <= 4) return launch_k(d.pdl, k_topk<4, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
-  if (nv <= 8) return launch_k(d.pdl, k_topk<8, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
-  if (nv <= 16) return launch_k(d.pdl, k_topk<16, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
-  if (nv <= 32) return launch_k(d.pdl, k_topk<32, KV, kSelectOnly>, blocks, 128, 0, st, d, s, x);
+  const int th = 64 * kTopkHeads;
+  if (nv <= 1) return launch_k(d.pdl, k_topk<1, KV, kSelectOnly>, blocks, th, 0, st, d, s, x);
+  if (nv <= 2) return launch_k(d.pdl, k_topk<2, KV, kSelectOnly>, blocks, th, 0, st, d, s, x);
+  if (nv <= 4) return launch_k(d.pdl, k_topk<4, KV, kSelectOnly>, blocks, th, 0, st, d, s, x);
+  if (nv <= 8) return launch_k(d.pdl, k_topk<8, KV, kSelectOnly>, blocks, th, 0, st, d, s, x);
+  if (nv <= 16) return launch_k(d.pdl, k_topk<16, KV, kSelectOnly>, blocks, th, 0, st, d, s, x);
+  if (nv <= 32) return launch_k(d.pdl, k_topk<32, KV, kSelectOnly>, blocks, th, 0, st, d, s, x);
   return cudaErrorInvalidValue;  // n > 1024: rejected when the state is made
 }
 
