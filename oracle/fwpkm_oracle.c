@@ -191,10 +191,21 @@ void orc_softmax(const double *s, int k, double *w) {
 /* ------------------------------------------------------------------------ */
 /* Shapes shared by the chunk routines.                                      */
 /* ------------------------------------------------------------------------ */
+/* Readings of two points the pages leave open, as options (section 2 of the
+ * gist.science page: averaging of repeated-slot gradients; the pypi page's
+ * multi-head variant).  Default 0: heads averaged, a value row's gradient
+ * divided by its row contribution C_i = sum of w/H.                        */
+enum {
+  ORC_HEADS_SUM = 1, /* head readouts summed, not averaged                   */
+  ORC_AGG_COUNT = 2, /* value-row gradient divided by the row's access count */
+  ORC_AGG_SUM = 4,   /* value-row gradient not divided (plain sum)           */
+};
+
 typedef struct {
   int64_t N;
   int n, dq, dh, dv, k, chunk, H;
   double eps;
+  int variant; /* ORC_* bits */
 } dims_t;
 
 static int check_dims(int64_t N, int n, int dq, int dv, int topk, int chunk, int heads) {
@@ -250,15 +261,19 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
   int64_t *ulist = (int64_t *)malloc(sizeof(int64_t) * P);
   double *GV = (double *)calloc((size_t)P * dv, sizeof(double));
   double *Csum = (double *)calloc((size_t)P, sizeof(double));
+  double *Cnt = (double *)calloc((size_t)P, sizeof(double)); /* accesses per row */
   double *psum = (double *)calloc((size_t)P, sizeof(double));
   double *GK = (double *)calloc((size_t)H * 2 * n * dh, sizeof(double));
   unsigned char *ktouched = (unsigned char *)calloc((size_t)H * 2 * n, 1);
   if (!slot || !ia || !jb || !w || !d1 || !d2 || !yhat || !e || !ulist || !GV || !Csum ||
-      !psum || !GK || !ktouched) {
+      !Cnt || !psum || !GK || !ktouched) {
     free(slot); free(ia); free(jb); free(w); free(d1); free(d2); free(yhat); free(e);
-    free(ulist); free(GV); free(Csum); free(psum); free(GK); free(ktouched);
+    free(ulist); free(GV); free(Csum); free(Cnt); free(psum); free(GK); free(ktouched);
     return -3;
   }
+  /* head divisor of the readout and of its gradients: H (heads averaged) or
+   * 1 (heads summed) */
+  const double Hd = (dm->variant & ORC_HEADS_SUM) ? 1.0 : (double)H;
   int status = 0;
   int64_t U = 0; /* distinct value rows touched by the chunk */
 
@@ -318,7 +333,8 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
   if (status) goto done;
 
   /* 2. Readout [GS-2 "retrieved value"; heads averaged]: yhat_t = (1/H)     */
-  /*    sum_h sum_r w V[slot]; out_t = g_t * yhat_t  [GS-2 gate, AF gate]     */
+  /*    sum_h sum_r w V[slot] (Hd = 1: heads summed); out_t = g_t * yhat_t    */
+  /*    [GS-2 gate, AF gate]                                                  */
   for (int b = 0; b < B; ++b)
     for (int tl = 0; tl < Tc; ++tl) {
       double *y = yhat + ((int64_t)b * Tc + tl) * dv;
@@ -329,7 +345,7 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
           for (int c = 0; c < dv; ++c) y[c] += w[m * k + r] * vr[c];
         }
       }
-      for (int c = 0; c < dv; ++c) y[c] /= H;
+      for (int c = 0; c < dv; ++c) y[c] /= Hd;
       double g = row_of(gate, T, b, t0 + tl, 1)[0];
       const double *vt = row_of(Vt, T, b, t0 + tl, dv);
       double *ev = e + ((int64_t)b * Tc + tl) * dv;
@@ -356,8 +372,9 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
       }
       int64_t u = rowmap[s_];
       double wr = w[m * k + r];
-      for (int c = 0; c < dv; ++c) GV[u * dv + c] += (2.0 * om / H) * wr * ev[c];
-      Csum[u] += wr / H;
+      for (int c = 0; c < dv; ++c) GV[u * dv + c] += (2.0 * om / Hd) * wr * ev[c];
+      Csum[u] += wr / Hd;
+      Cnt[u] += 1.0;
       psum[u] += wr;
     }
   }
@@ -386,7 +403,7 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
         const double *vr = V + slot[m * k + r] * dv;
         double dot = 0.0;
         for (int c = 0; c < dv; ++c) dot += ev[c] * vr[c];
-        gam[r] = (2.0 * om / H) * dot;
+        gam[r] = (2.0 * om / Hd) * dot;
         if (lam != 0.0) gam[r] += (lam / (double)M) * (log(psum[rowmap[slot[m * k + r]]]) + 1.0);
         wg += w[m * k + r] * gam[r];
       }
@@ -436,9 +453,13 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
 
   /* 5. Update [AF theta' = theta - eta grad; GS-2 averaging; SS-TOC no     */
   /*    clipping]: V_i -= eta G_i / C_i on touched rows; K -= eta dL/dK.      */
+  /*    The divisor of a value row: C_i (row contribution, default), its      */
+  /*    access count (ORC_AGG_COUNT), or 1 (ORC_AGG_SUM).                     */
   if (apply) {
     for (int64_t u = 0; u < U; ++u) {
       double *vr = V + ulist[u] * dv;
+      if (dm->variant & ORC_AGG_COUNT) Csum[u] = Cnt[u];
+      if (dm->variant & ORC_AGG_SUM) Csum[u] = 1.0;
       for (int c = 0; c < dv; ++c) vr[c] -= eta * GV[u * dv + c] / Csum[u];
     }
     for (int64_t row = 0; row < (int64_t)H * 2 * n; ++row)
@@ -449,7 +470,7 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
 done:
   for (int64_t u = 0; u < U; ++u) rowmap[ulist[u]] = -1;
   free(slot); free(ia); free(jb); free(w); free(d1); free(d2); free(yhat); free(e);
-  free(ulist); free(GV); free(Csum); free(psum); free(GK); free(ktouched);
+  free(ulist); free(GV); free(Csum); free(Cnt); free(psum); free(GK); free(ktouched);
   return status;
 }
 
@@ -464,14 +485,15 @@ done:
  * number of distinct value rows written per chunk.  omega [B][T] (optional)
  * is the MSE weight of each token; NULL = the gate. */
 int orc_step(int64_t N, int n, int dq, int dv, int topk, int chunk, int heads, double eps,
-             double *K, double *V, int B, int T, const double *Q, const double *Vt,
-             const double *gate, const double *omega, double eta, double lam, double *out,
-             int64_t *sel_slot,
-             double *sel_w, double *gap, int64_t *touched, int max_chunks) {
+             int variant, double *K, double *V, int B, int T, const double *Q,
+             const double *Vt, const double *gate, const double *omega, double eta,
+             double lam, double *out, int64_t *sel_slot, double *sel_w, double *gap,
+             int64_t *touched, int max_chunks) {
   int rc = check_dims(N, n, dq, dv, topk, chunk, heads);
   if (rc) return rc;
   if (B < 1 || T < 1) return -2;
-  dims_t dm = {N, n, dq, dq / 2, dv, topk, chunk, heads, eps};
+  if ((variant & ORC_AGG_COUNT) && (variant & ORC_AGG_SUM)) return -1;
+  dims_t dm = {N, n, dq, dq / 2, dv, topk, chunk, heads, eps, variant};
   int64_t *rowmap = (int64_t *)malloc(sizeof(int64_t) * (size_t)N);
   if (!rowmap) return -3;
   for (int64_t i = 0; i < N; ++i) rowmap[i] = -1;
@@ -492,13 +514,13 @@ int orc_step(int64_t N, int n, int dq, int dv, int topk, int chunk, int heads, d
 /* One chunk (tokens t0 .. t0+Tc-1) without any update: raw gradients, the
  * loss and p_bar for finite-difference and invariant checks. */
 int orc_chunk_grads(int64_t N, int n, int dq, int dv, int topk, int chunk, int heads,
-                    double eps, const double *K, const double *V, int B, int T, int t0,
-                    int Tc, const double *Q, const double *Vt, const double *gate,
+                    double eps, int variant, const double *K, const double *V, int B, int T,
+                    int t0, int Tc, const double *Q, const double *Vt, const double *gate,
                     const double *omega, double lam, double *dLdV, double *dLdK, double *pbar,
                     double *loss, int64_t *sel_slot, double *sel_w) {
   int rc = check_dims(N, n, dq, dv, topk, chunk, heads);
   if (rc) return rc;
-  dims_t dm = {N, n, dq, dq / 2, dv, topk, chunk, heads, eps};
+  dims_t dm = {N, n, dq, dq / 2, dv, topk, chunk, heads, eps, variant};
   int64_t *rowmap = (int64_t *)malloc(sizeof(int64_t) * (size_t)N);
   if (!rowmap) return -3;
   for (int64_t i = 0; i < N; ++i) rowmap[i] = -1;
@@ -511,15 +533,17 @@ int orc_chunk_grads(int64_t N, int n, int dq, int dv, int topk, int chunk, int h
 /* The chunk loss written straight from its definition for a FROZEN selection
  * slots [B][Tc][H][k] (as returned by orc_chunk_grads for the same chunk):
  *   s_r = -log(eps + ||q1 - K1[i_r]||^2) - log(eps + ||q2 - K2[j_r]||^2)
- *   w   = softmax(s);  yhat_t = (1/H) sum_h sum_r w_r V[slot_r]
+ *   w   = softmax(s);  yhat_t = (1/H) sum_h sum_r w_r V[slot_r]  (summed heads:
+ *         no 1/H)
  *   L   = sum_t w_t ||yhat_t - v_t||^2 + lam * sum_i p_bar_i log p_bar_i
  *         (w_t = omega_t if omega is given, else the gate g_t)
  * Used only for finite differences of the analytic gradients. */
 double orc_chunk_loss(int64_t N, int n, int dq, int dv, int topk, int heads, double eps,
-                      const double *K, const double *V, int B, int T, int t0, int Tc,
-                      const double *Q, const double *Vt, const double *gate,
+                      int variant, const double *K, const double *V, int B, int T, int t0,
+                      int Tc, const double *Q, const double *Vt, const double *gate,
                       const double *omega, double lam, const int64_t *slots) {
   const int dh = dq / 2, k = topk, H = heads;
+  const double Hd = (variant & ORC_HEADS_SUM) ? 1.0 : (double)H;
   const int64_t M = (int64_t)B * Tc * H;
   double *pb = (double *)calloc((size_t)N, sizeof(double));
   double *y = (double *)malloc(sizeof(double) * dv);
@@ -553,7 +577,7 @@ double orc_chunk_loss(int64_t N, int n, int dq, int dv, int topk, int heads, dou
       const double *vt = row_of(Vt, T, b, t0 + tl, dv);
       double sq = 0.0;
       for (int c = 0; c < dv; ++c) {
-        double ec = y[c] / H - vt[c];
+        double ec = y[c] / Hd - vt[c];
         sq += ec * ec;
       }
       L += wt * sq;

@@ -49,13 +49,13 @@ def lib():
         L.orc_pk_select.argtypes = [_dp, _dp, i32, i32, _ip, _dp, _ip, _ip]
         L.orc_brute_select.argtypes = [_dp, _dp, i32, i32, _ip, _dp]
         L.orc_softmax.argtypes = [_dp, i32, _dp]
-        L.orc_step.argtypes = [i64, i32, i32, i32, i32, i32, i32, f64, _dp, _dp, i32, i32,
-                               _dp, _dp, _dp, _dp, f64, f64, _dp, _ip, _dp, _dp, _ip, i32]
-        L.orc_chunk_grads.argtypes = [i64, i32, i32, i32, i32, i32, i32, f64, _dp, _dp, i32,
-                                      i32, i32, i32, _dp, _dp, _dp, _dp, f64, _dp, _dp, _dp,
-                                      _dp, _ip, _dp]
-        L.orc_chunk_loss.argtypes = [i64, i32, i32, i32, i32, i32, f64, _dp, _dp, i32, i32,
-                                     i32, i32, _dp, _dp, _dp, _dp, f64, _ip]
+        L.orc_step.argtypes = [i64, i32, i32, i32, i32, i32, i32, f64, i32, _dp, _dp, i32,
+                               i32, _dp, _dp, _dp, _dp, f64, f64, _dp, _ip, _dp, _dp, _ip, i32]
+        L.orc_chunk_grads.argtypes = [i64, i32, i32, i32, i32, i32, i32, f64, i32, _dp, _dp,
+                                      i32, i32, i32, i32, _dp, _dp, _dp, _dp, f64, _dp, _dp,
+                                      _dp, _dp, _ip, _dp]
+        L.orc_chunk_loss.argtypes = [i64, i32, i32, i32, i32, i32, f64, i32, _dp, _dp, i32,
+                                     i32, i32, i32, _dp, _dp, _dp, _dp, f64, _ip]
         L.orc_chunk_loss.restype = f64
         _lib = L
     return _lib
@@ -146,10 +146,22 @@ def lookahead_targets(Vt, weight):
 # --------------------------------------------------------------------------
 # Memory state and the step
 # --------------------------------------------------------------------------
-class State:
-    """fp64 copy of the fast weights: K [H][2][n][dq/2], V [N][dv]."""
+# Options of two readings (fwpkm_oracle.c): how head readouts combine and what
+# a value row's gradient is divided by.
+HEADS = {"mean": 0, "sum": 1}
+AGG = {"weight": 0, "count": 2, "sum": 4}
 
-    def __init__(self, subkeys, values, *, topk: int, chunk: int, eps: float = 1e-3):
+
+class State:
+    """fp64 copy of the fast weights: K [H][2][n][dq/2], V [N][dv].
+
+    ``heads``: "mean" (head readouts averaged, the default reading) or "sum".
+    ``agg``: a value row's gradient divided by its row contribution C_i =
+    sum of w/H ("weight", the default), by its access count ("count"), or not
+    divided ("sum")."""
+
+    def __init__(self, subkeys, values, *, topk: int, chunk: int, eps: float = 1e-3,
+                 heads: str = "mean", agg: str = "weight"):
         self.K = _f64(subkeys).copy()
         self.V = _f64(values).copy()
         self.H, two, self.n, self.dh = self.K.shape
@@ -157,6 +169,7 @@ class State:
         self.N, self.dv = self.V.shape
         self.dq = 2 * self.dh
         self.topk, self.chunk, self.eps = topk, chunk, eps
+        self.variant = HEADS[heads] | AGG[agg]
 
     def copy(self) -> "State":
         s = State.__new__(State)
@@ -166,7 +179,8 @@ class State:
         return s
 
     def _dims(self):
-        return (self.N, self.n, self.dq, self.dv, self.topk, self.chunk, self.H, self.eps)
+        return (self.N, self.n, self.dq, self.dv, self.topk, self.chunk, self.H, self.eps,
+                self.variant)
 
     def step(self, Q, Vt, gate, eta: float, lam: float, *, want_sel: bool = False,
              want_gap: bool = False, max_chunks: int = 0, omega=None,
@@ -230,6 +244,7 @@ class State:
         B, T = gate.shape
         slots = np.ascontiguousarray(slots, dtype=np.int64)
         return float(lib().orc_chunk_loss(self.N, self.n, self.dq, self.dv, self.topk, self.H,
-                                          self.eps, _p(self.K), _p(self.V), B, T, t0, Tc,
+                                          self.eps, self.variant, _p(self.K), _p(self.V), B,
+                                          T, t0, Tc,
                                           _p(Q), _p(Vt), _p(gate), _p(omega), lam,
                                           _p(slots)))

@@ -100,3 +100,46 @@ def test_hand_step_lookahead(hs):
     for key, row in la["dLdK"].items():
         dK[row_key(key)] = arr(row)
     np.testing.assert_allclose(gr["dLdK"], dK, rtol=RTOL, atol=1e-15)
+
+
+@pytest.mark.parametrize("agg", ["count", "sum"])
+def test_hand_step_other_row_divisors(hs, agg):
+    """A value row's gradient divided by its access count, or not divided:
+    reads and sub-keys as in the main step, value rows as worked by hand."""
+    part = hs.raw.get("aggregation")
+    if part is None:
+        pytest.skip("this example has no aggregation part")
+    st = oracle.State(hs.K, hs.V, topk=hs.topk, chunk=hs.chunk, eps=hs.eps, agg=agg)
+    res = st.step(hs.Q, hs.Vt, hs.gate, hs.eta, 0.0)
+    np.testing.assert_allclose(res["out"], arr(hs.expected["out"]), rtol=RTOL)
+    V = hs.V.copy()
+    for r, row in part[agg]["values_after"].items():
+        V[int(r)] = arr(row)
+    np.testing.assert_allclose(st.V, V, rtol=RTOL, atol=0)
+    np.testing.assert_allclose(st.K, hs.subkeys_after(), rtol=RTOL, atol=1e-15)
+
+
+def test_hand_step_summed_heads(hs):
+    """The head readouts summed, not averaged (the 1/H of the readout, of its
+    gradients and of C_i goes): read, loss, dL/dK and both updated tables."""
+    part = hs.raw.get("heads_sum")
+    if part is None:
+        pytest.skip("this example has no summed-heads part")
+    st = oracle.State(hs.K, hs.V, topk=hs.topk, chunk=hs.chunk, eps=hs.eps, heads="sum")
+    gr = st.chunk_grads(hs.Q, hs.Vt, hs.gate, 0.0, 0, hs.chunk)
+    assert gr["loss"] == pytest.approx(sum(frac(x) for x in part["loss"]), rel=RTOL)
+    dK = np.zeros_like(hs.K)
+    for key, row in part["dLdK"].items():
+        dK[row_key(key)] = arr(row)
+    np.testing.assert_allclose(gr["dLdK"], dK, rtol=RTOL, atol=1e-15)
+    res = st.step(hs.Q, hs.Vt, hs.gate, hs.eta, 0.0, want_sel=True)
+    assert np.array_equal(res["sel_slot"], np.array(hs.expected["sel_slot"]))
+    np.testing.assert_allclose(res["out"], arr(part["out"]), rtol=RTOL)
+    V = hs.V.copy()
+    for r, row in part["values_after"].items():
+        V[int(r)] = arr(row)
+    np.testing.assert_allclose(st.V, V, rtol=RTOL, atol=0)
+    K = hs.K.copy()
+    for key, row in part["subkeys_after"].items():
+        K[row_key(key)] = arr(row)
+    np.testing.assert_allclose(st.K, K, rtol=RTOL, atol=1e-15)

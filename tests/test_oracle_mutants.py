@@ -19,11 +19,11 @@ MUTANTS = {
     "second_half_uses_first_query_half": ("G2[c] += c2 * (q[dh + c] - K2[c]);",
                                           "G2[c] += c2 * (q[c] - K2[c]);"),
     "entropy_term_dropped": ("if (lam != 0.0) gam[r] +=", "if (0) gam[r] +="),
-    "heads_summed_not_averaged": ("for (int c = 0; c < dv; ++c) y[c] /= H;", ""),
+    "heads_summed_not_averaged": ("for (int c = 0; c < dv; ++c) y[c] /= Hd;", ""),
     "no_row_contribution_average": ("vr[c] -= eta * GV[u * dv + c] / Csum[u];",
                                     "vr[c] -= eta * GV[u * dv + c];"),
-    "gate_not_weighting_mse": ("GV[u * dv + c] += (2.0 * om / H) * wr * ev[c];",
-                               "GV[u * dv + c] += (2.0 / H) * wr * ev[c];"),
+    "gate_not_weighting_mse": ("GV[u * dv + c] += (2.0 * om / Hd) * wr * ev[c];",
+                               "GV[u * dv + c] += (2.0 / Hd) * wr * ev[c];"),
     "softmax_not_normalised": ("for (int r = 0; r < k; ++r) w[r] /= z;", ""),
     "slot_index_transposed": ("cand[a * k + b].idx = top1[a] * (int64_t)n + top2[b];",
                               "cand[a * k + b].idx = top2[b] * (int64_t)n + top1[a];"),
@@ -33,8 +33,11 @@ MUTANTS = {
     "marginal_not_normalised": ("for (int64_t u = 0; u < U; ++u) psum[u] /= (double)M;",
                                 "for (int64_t u = 0; u < U; ++u) psum[u] /= (double)(M + 1);"),
     "distance_of_wrong_half_index": ("d1[m * k + r] = dd1[a_[r]];", "d1[m * k + r] = dd1[b_[r]];"),
-    "mse_grad_factor_two_dropped": ("gam[r] = (2.0 * om / H) * dot;",
-                                    "gam[r] = (1.0 * om / H) * dot;"),
+    "mse_grad_factor_two_dropped": ("gam[r] = (2.0 * om / Hd) * dot;",
+                                    "gam[r] = (1.0 * om / Hd) * dot;"),
+    "count_divisor_is_the_weight": ("if (dm->variant & ORC_AGG_COUNT) Csum[u] = Cnt[u];", ""),
+    "summed_heads_still_averaged": ("(dm->variant & ORC_HEADS_SUM) ? 1.0 : (double)H;",
+                                    "(double)H;"),
     "keys_not_updated": ("if (ktouched[row])", "if (0)"),
 }
 

@@ -25,8 +25,8 @@ def tiny_case(rng, B=2, T=8, H=2, dq=8, n=6, dv=5, k=3, gate="rand"):
     return K, V, Q, Vt, g
 
 
-def make_state(oracle, K, V, k, chunk):
-    return oracle.State(K, V, topk=k, chunk=chunk, eps=EPS)
+def make_state(oracle, K, V, k, chunk, **opts):
+    return oracle.State(K, V, topk=k, chunk=chunk, eps=EPS, **opts)
 
 
 # ---------------------------------------------------------------------------
@@ -131,16 +131,18 @@ def test_gap_is_kth_minus_next(oracle):
 # ---------------------------------------------------------------------------
 # Gradients: central finite differences of the loss definition
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("lam,H,gate,own_weight", [(0.0, 1, "one", False), (0.0, 2, "rand", False),
-                                                   (0.3, 2, "rand", False), (1.5, 1, "rand", False),
-                                                   (0.3, 2, "rand", True)])
-def test_gradients_match_finite_differences(oracle, lam, H, gate, own_weight):
+@pytest.mark.parametrize("lam,H,gate,own_weight,heads", [
+    (0.0, 1, "one", False, "mean"), (0.0, 2, "rand", False, "mean"),
+    (0.3, 2, "rand", False, "mean"), (1.5, 1, "rand", False, "mean"),
+    (0.3, 2, "rand", True, "mean"), (0.0, 3, "rand", False, "sum"),
+    (0.4, 2, "rand", True, "sum")])
+def test_gradients_match_finite_differences(oracle, lam, H, gate, own_weight, heads):
     rng = np.random.default_rng(int(lam * 10) + H + (7 if own_weight else 0))
     B, T, dq, n, dv, k = 2, 6, 8, 6, 5, 3
     K, V, Q, Vt, g = tiny_case(rng, B=B, T=T, H=H, dq=dq, n=n, dv=dv, k=k, gate=gate)
     # a per-token MSE weight of its own (some tokens 0), else the gate
     om = rng.uniform(0.0, 1.5, (B, T)) * (rng.random((B, T)) > 0.3) if own_weight else None
-    st = make_state(oracle, K, V, k, T)
+    st = make_state(oracle, K, V, k, T, heads=heads)
     gr = st.chunk_grads(Q, Vt, g, lam, 0, T, omega=om)
     slots = gr["sel_slot"]
     L0 = st.chunk_loss(Q, Vt, g, lam, 0, T, slots, omega=om)
@@ -385,3 +387,64 @@ def test_duplicated_heads_reduce_to_one_head(oracle, lam):
     assert np.allclose(a.V, b.V, rtol=1e-12, atol=1e-15)
     for h in range(2):
         assert np.allclose(b.K[h] - K1[0], 0.5 * (a.K[0] - K1[0]), rtol=1e-9, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# Options of two readings: the divisor of a value row's gradient, and summed
+# heads (each against a closed form or a reduction, like the defaults above)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("agg", ["count", "sum"])
+def test_single_access_update_without_row_contribution(oracle, agg):
+    """A row written once: divided by its access count (1) or not divided, it
+    moves by the raw gradient -eta (2 g / H) w (yhat - v) -- the weight w no
+    longer cancels as it does under the default divisor."""
+    rng = np.random.default_rng(31)
+    for H in (1, 2):
+        K, V, Q, Vt, g = tiny_case(rng, B=1, T=1, H=H, dq=8, n=12, dv=4, k=3)
+        st = make_state(oracle, K, V, 3, 1, agg=agg)
+        st0 = st.copy()
+        eta = 0.37
+        res = st.step(Q, Vt, g, eta, 0.0, want_sel=True)
+        yhat = res["out"][0, 0] / g[0, 0]
+        sl = res["sel_slot"][0, 0].ravel()
+        w = res["sel_w"][0, 0].ravel()
+        uniq, cnt = np.unique(sl, return_counts=True)
+        checked = 0
+        for s_, c_ in zip(uniq, cnt):
+            if c_ == 1:
+                wi = w[sl == s_][0]
+                expect = st0.V[s_] - eta * (2 * g[0, 0] / H) * wi * (yhat - Vt[0, 0])
+                assert np.allclose(st.V[s_], expect, rtol=1e-12, atol=1e-14)
+                checked += 1
+        assert checked > 0
+
+
+@pytest.mark.parametrize("agg,factor", [("count", 1.0), ("sum", 2.0)])
+def test_two_writers_without_row_contribution(oracle, agg, factor):
+    """Two identical queries (same slots, same weights w) with targets v_a,
+    v_b: G = 2 w (2 yhat - v_a - v_b); divided by the count 2 the row moves by
+    -2 eta w (yhat - mean v), undivided by twice that."""
+    rng = np.random.default_rng(4)
+    K, V, Q, Vt, g = tiny_case(rng, B=1, T=2, H=1, dq=8, n=6, dv=3, k=3, gate="one")
+    Q[0, 1] = Q[0, 0]
+    st = make_state(oracle, K, V, 3, 2, agg=agg)
+    st0 = st.copy()
+    eta = 0.25
+    res = st.step(Q, Vt, g, eta, 0.0, want_sel=True)
+    yhat = res["out"][0, 0]
+    for s_, w_ in zip(res["sel_slot"][0, 0, 0], res["sel_w"][0, 0, 0]):
+        expect = st0.V[s_] - factor * 2 * eta * w_ * (yhat - 0.5 * (Vt[0, 0] + Vt[0, 1]))
+        assert np.allclose(st.V[s_], expect, rtol=1e-12, atol=1e-14)
+
+
+def test_summed_duplicated_heads_read_twice_one_head(oracle):
+    """H = 2 with identical queries and sub-keys per head, readouts summed:
+    every read is twice the single head's (eta = 0, so every chunk reads the
+    same tables)."""
+    rng = np.random.default_rng(19)
+    K1, V, Q1, Vt, g = tiny_case(rng, B=2, T=6, H=1, dq=8, n=6, dv=4, k=3)
+    a = make_state(oracle, K1, V, 3, 3)
+    ra = a.step(Q1, Vt, g, 0.0, 0.0)
+    b = make_state(oracle, np.concatenate([K1, K1], axis=0), V, 3, 3, heads="sum")
+    rb = b.step(np.concatenate([Q1, Q1], axis=2), Vt, g, 0.0, 0.0)
+    assert np.allclose(rb["out"], 2.0 * ra["out"], rtol=1e-13, atol=1e-15)
