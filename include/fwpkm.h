@@ -85,6 +85,26 @@ void fwpkm_state_free(fwpkm_state *s);
 /* IDW constant: score = -log(eps + ||q_half - K_row||^2).  [GS-2]  eps > 0. */
 fwpkm_status fwpkm_state_set_eps(fwpkm_state *s, float eps);
 
+/* Options of fwpkm_state_set_options. */
+#define FWPKM_HEADS_SUM 1u /* head readouts summed, not averaged                   */
+#define FWPKM_AGG_COUNT 2u /* value-row gradient divided by the row's access count */
+#define FWPKM_AGG_SUM 4u   /* value-row gradient not divided                       */
+
+/*
+ * fwpkm_state_set_options -- other readings of two points the pages leave
+ * open, for the steps that follow (0 restores the defaults).
+ *   [PYPI multi-head variant]  By default the heads' readouts are averaged,
+ *     yhat = (1/H) sum_h sum_r w V[slot]; FWPKM_HEADS_SUM sums them, and the
+ *     1/H of the gradients and of C_i goes with it.
+ *   [GS-2 averaging of repeated-slot gradients; SS-TOC gradient weighted by
+ *     row contribution]  By default a written value row moves by
+ *     eta G_i / C_i, C_i = sum of its pairs' w/H; FWPKM_AGG_COUNT divides by
+ *     the number of pairs on the row instead, FWPKM_AGG_SUM not at all.
+ *     The two exclude each other (FWPKM_EINVAL).
+ * The sub-keys always take the raw summed gradient.
+ */
+fwpkm_status fwpkm_state_set_options(fwpkm_state *s, unsigned options);
+
 /*
  * fwpkm_step -- run the chunk loop over one call.  [GS-2, AF]
  * For every chunk c = 0 .. ceil(T/chunk)-1 in order (the last may be
@@ -242,7 +262,8 @@ fwpkm_status fwpkm_profile_read(fwpkm_state *s, const char **names, double *ms,
  * member records grouped (pairs plus sub-key entries; the write traffic of
  * the step is proportional to these).  device_errors receives the sticky
  * device error bits:
- *    1  the read's bounded wait for its bulk row copies gave up,
+ *    1  reserved (no longer set: the read reads its rows directly and waits
+ *       for nothing),
  *    2  the apply's partial pool overflowed (the launch sizing rules it out),
  *    4  a bucket-scan CTA gave up waiting for an earlier CTA's total,
  *    8  the score's bounded wait on its TMA ring or its MMAs gave up,
@@ -263,7 +284,7 @@ fwpkm_status fwpkm_read_stats(fwpkm_state *s, int64_t *chunks, int64_t *value_ro
  * fwpkm_set_wait_limits -- bounds of the device-side waits of this state's
  * steps (and of fwpkm_select_noalloc on it), for failure detection and its
  * tests.  mbar_polls bounds the first wait on an mbarrier (the score's TMA
- * ring and MMA completion, the read's bulk row copies; default 2^26 polls);
+ * ring and MMA completion; default 2^26 polls);
  * scan_polls bounds a bucket-scan CTA's wait for the totals of the CTAs
  * before it (default 2^24).  A negative value restores the default; 0 makes
  * the wait give up at once.  A wait that gives up sets its error bit

@@ -103,6 +103,8 @@ struct fwpkm_state {
   int sm_count = 148;
   // bounds of the device-side waits (fwpkm_set_wait_limits)
   long long mbar_polls = kDefaultMbarPolls, scan_polls = kDefaultScanPolls;
+  // readings (fwpkm_state_set_options)
+  int heads_sum = 0, agg = AGG_WEIGHT;
   float *K = nullptr;  // [H][2][n][dh]
   float *V = nullptr;  // [N][dv]
   // scratch arena
@@ -326,6 +328,8 @@ Dims chunk_dims(const fwpkm_state *st, int B, int T, int c, float eta, float lam
   d.lam = lambda_entropy;
   d.mbar_polls = st->mbar_polls;
   d.scan_polls = st->scan_polls;
+  d.heads_sum = st->heads_sum;
+  d.agg = st->agg;
   return d;
 }
 
@@ -374,10 +378,32 @@ fwpkm_status enqueue_chunks(fwpkm_state *st, int B, int T, const void *Q, int q_
 
   const Scratch &s = st->s;
   const int n_chunks = (T + st->chunk - 1) / st->chunk;
+  // eta = 0 changes no table, so the write kernels are skipped altogether (a
+  // read-only memory, as a static product-key memory is): each chunk is its
+  // query halves, the score, the selection and the read.
+  const bool readonly = eta == 0.f;
   for (int c = 0; c < n_chunks; ++c) {
     Dims d = chunk_dims(st, B, T, c, eta, lambda_entropy);
     d.lookahead = lookahead;
     d.q_tf32_exact = q_dtype == FWPKM_BF16 ? 1 : 0;
+    d.readonly = readonly ? 1 : 0;
+    if (readonly) {
+      if ((rc = hook(hooks ? hooks->need_inputs : nullptr, c))) return rc;
+      if (lookahead && c + 1 < n_chunks &&
+          (rc = hook(hooks ? hooks->need_inputs : nullptr, c + 1)))
+        return rc;
+      if ((rc = run(st, K_PREP, stream, [&] { return launch_prep_q(d, Q, q_dtype, s, stream); })))
+        return rc;
+      if ((rc = run(st, K_SCORE, stream, [&] { return launch_score(d, s, st->maps, stream); })))
+        return rc;
+      if ((rc = run(st, K_TOPK, stream, [&] { return launch_topk(d, s, x, stream); }))) return rc;
+      if ((rc = run(st, K_READ, stream, [&] {
+             return launch_read(d, st->V, Vtarget, v_dtype, gate, omega, out, s, stream);
+           })))
+        return rc;
+      if ((rc = hook(hooks ? hooks->read_done : nullptr, c))) return rc;
+      continue;
+    }
     // the next chunk of this call, whose query halves the sort prepares
     Dims dn{};
     if (c + 1 < n_chunks) dn = chunk_dims(st, B, T, c + 1, eta, lambda_entropy);
@@ -585,6 +611,18 @@ fwpkm_status fwpkm_set_wait_limits(fwpkm_state *st, int64_t mbar_polls, int64_t 
 }
 
 void fwpkm_inject_alloc_failures(int count) { g_fail_allocs.store(count > 0 ? count : 0); }
+
+fwpkm_status fwpkm_state_set_options(fwpkm_state *st, unsigned options) {
+  if (!st) return fail(FWPKM_EINVAL, "set_options: state is NULL");
+  const unsigned known = FWPKM_HEADS_SUM | FWPKM_AGG_COUNT | FWPKM_AGG_SUM;
+  if (options & ~known) return fail(FWPKM_EINVAL, "set_options: unknown bits 0x%x", options);
+  if ((options & FWPKM_AGG_COUNT) && (options & FWPKM_AGG_SUM))
+    return fail(FWPKM_EINVAL, "set_options: FWPKM_AGG_COUNT and FWPKM_AGG_SUM exclude each other");
+  st->heads_sum = (options & FWPKM_HEADS_SUM) ? 1 : 0;
+  st->agg = (options & FWPKM_AGG_COUNT) ? AGG_COUNT : ((options & FWPKM_AGG_SUM) ? AGG_SUM : AGG_WEIGHT);
+  clear_graphs(st);  // the options are kernel parameters of the captured launches
+  return FWPKM_OK;
+}
 
 fwpkm_status fwpkm_set_graphs(fwpkm_state *st, int enable) {
   if (!st) return fail(FWPKM_EINVAL, "set_graphs: state is NULL");

@@ -31,7 +31,7 @@ constexpr unsigned FULL = 0xffffffffu;
 // that a kernel checking the word at entry never sees a bit change under it:
 // every bit it looks at belongs to a kernel that completed before it started.
 enum : unsigned {
-  ERR_READ_TIMEOUT = 1u,   // the read's wait for its bulk row copies gave up
+  ERR_READ_TIMEOUT = 1u,   // reserved: the read's wait for staged rows (it now waits for nothing)
   ERR_POOL_OVERFLOW = 2u,  // apply: more long-group blocks than the partial pool holds
   ERR_SCAN_TIMEOUT = 4u,   // a scan CTA gave up waiting for an earlier CTA's total
   ERR_SCORE_TIMEOUT = 8u,  // the score's TMA ring or MMA completion wait gave up
@@ -75,11 +75,18 @@ struct Dims {
   int sm_count;       // multiprocessors of the device (grid sizing)
   int pdl;            // launch with programmatic dependent launch (see launch_k)
   float eps, eta, lam;
-  long long mbar_polls;  // bound of the first wait on an mbarrier (score ring, read copies)
+  long long mbar_polls;  // bound of the first wait on an mbarrier (the score's ring and MMAs)
   long long scan_polls;  // bound of a scan CTA's wait for an earlier CTA's total
   int lookahead;         // token t is written towards the target of token t+1
   int q_tf32_exact;      // the queries are bf16, so exact in TF32 (their lo part is zero)
+  int heads_sum;         // head readouts summed instead of averaged
+  int readonly;          // eta = 0: the read alone (no claims, entries, records, gradients)
+  int agg;               // divisor of a value row's gradient (AGG_*)
 };
+// Divisor of a value row's gradient: its row contribution C_i = sum of w/H
+// (the sum of its members' c0), its access count (every member's c0 is 1), or
+// none.
+enum { AGG_WEIGHT = 0, AGG_COUNT = 1, AGG_SUM = 2 };
 
 // Device scratch owned by the state (sized for the largest chunk seen).
 constexpr int kScanMaxCtas = 64;  // bucket-scan CTAs: 64 x 2048 buckets
@@ -287,17 +294,6 @@ __device__ __forceinline__ void prep_query_half(const Dims &d, const TQ *__restr
   if (lane == 0) s.qn[(int64_t)hh * d.qstride + row] = acc;
 }
 
-// 1-D bulk copy global -> shared, completion counted on `bar` (bytes % 16 == 0,
-// both addresses 16-byte aligned).
-__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, unsigned bytes,
-                                         uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_u32(dst_smem)),
-      "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // Programmatic dependent launch.  A kernel started by launch_k with d.pdl set
 // may become resident while its predecessor on the stream is still running;
 // griddep_wait() blocks until that predecessor has completed and its writes
@@ -379,8 +375,8 @@ cudaError_t launch_scan(const Dims &d, const Scratch &s, cudaStream_t st);
 cudaError_t launch_read(const Dims &d, const float *V, const void *Vt, int v_dtype,
                         const float *gate, const float *omega, float *out, const Scratch &s,
                         cudaStream_t st);
-// Whether the read stages its rows in shared memory at these shapes.
-bool read_is_staged(const Dims &d);
+// CTAs per token of the read at these shapes (1 unless a token's rows exceed 1 MB).
+int read_cluster_size(const Dims &d);
 // The bucket sort; with dn.rows > 0 extra CTAs also prepare the query halves
 // of the next chunk dn (nothing reads this chunk's halves after the score).
 cudaError_t launch_bsort(const Dims &d, const Scratch &s, const Dims &dn, const void *Q,

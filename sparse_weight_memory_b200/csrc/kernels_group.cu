@@ -669,7 +669,7 @@ __device__ __forceinline__ void add4(float4 &a, const float4 &x) {
 __device__ __forceinline__ float4 updated(const Dims &d, bool value, const float4 &t,
                                           const float4 &g, float c0) {
   if (value) {
-    const float sc = d.eta / c0;
+    const float sc = d.agg == AGG_SUM ? d.eta : d.eta / c0;
     return make_float4(t.x - sc * g.x, t.y - sc * g.y, t.z - sc * g.z, t.w - sc * g.w);
   }
   const float te = 2.f * d.eta;

@@ -17,43 +17,39 @@
 // Jacobian dL/ds_r = w_r (dL/dw_r - sum_r' w_r' dL/dw_r') and, per sub-key
 // entry, alpha = (sum of dL/ds over its pairs) / (eps + d).
 //
-// One thread-block cluster of G CTAs per token row.  The token's H*k value
-// rows are split into G consecutive ranges; each CTA fetches its range by
-// 1-D bulk async copies (TMA) straight into its shared memory, completing on
-// one mbarrier, and writes its share of the token's member records while the
-// rows land.  Each CTA then forms the partial weighted sum of its rows; the
-// cluster exchanges the partials through distributed shared memory and every
-// CTA adds them in rank order (the same yhat everywhere), so each can take
-// the dot products of its own rows with e_t.  G grows with the token's gather
-// (about 32 KB of rows per CTA) so that several tokens are in flight per
-// multiprocessor whatever H*k*dv is.  Rows that do not fit in shared memory
-// are read from global memory in both passes.
+// One CTA per token, one float4 column of the value rows per thread (32, 64
+// or 128 threads, as the row is wide).  Each thread sums its column over the
+// token's H*k rows straight from global memory, every row load independent
+// of the others, so the rows of many tokens are in flight per
+// multiprocessor; the dot products then read the rows again, from L1 or L2.
+// The token's member records are written while the rows are in flight.
+// Only a token whose rows exceed 1 MB is split over a thread-block cluster
+// of G CTAs, which exchange their partial sums through distributed shared
+// memory and add them in rank order (the same yhat everywhere).  (Staging
+// the rows in shared memory by bulk copies, with clusters of about 32 KB of
+// rows per CTA, was measured slower: it limits the CTAs resident per
+// multiprocessor and adds barriers to each token's chain.)
 #include "fwpkm_internal.cuh"
 
 namespace fwpkm {
 
-constexpr int kReadThreads = 128;
-constexpr size_t kReadSmemBudget = 200 * 1024;
-constexpr size_t kReadCtaRows = 32 * 1024;  // staged bytes per CTA the cluster size aims at
-constexpr int kReadMaxCluster = 8;          // portable cluster size
+constexpr size_t kReadCtaRows = 1024 * 1024;  // value-row bytes per CTA before a cluster splits
+constexpr int kReadMaxCluster = 8;            // portable cluster size
 
 struct ReadPlan {
   int G;        // CTAs per token (cluster size, a power of two <= 8)
   int per;      // pairs per CTA, ceil(H*k / G)
-  bool staged;  // rows staged in shared memory
+  int threads;  // 32, 64 or 128: about one float4 column per thread
   size_t smem;  // dynamic shared memory per CTA
 };
 
-// Dynamic shared memory layout (bytes):
-//   [0, 16)                      mbarrier
-//   [128, 128 + R)               staged rows of this CTA, R = per*dv*4 (staged only)
-//   then ypart, e                dv floats each (ypart is read by the whole cluster)
-//   then w, slot, a, dl, claim   H*k each (a is read by the whole cluster)
-//   then esub, eclaim, emask, einv   2*H*k each (this CTA's entries only)
-static size_t read_smem_bytes(const Dims &d, int per, bool staged) {
+// Dynamic shared memory layout (floats / ints):
+//   ypart, e                dv each (ypart is read by the whole cluster)
+//   w, slot, a, dl, claim   H*k each (a is read by the whole cluster)
+//   esub, eclaim, emask, einv   2*H*k each (this CTA's entries only)
+static size_t read_smem_bytes(const Dims &d) {
   const size_t HK = (size_t)d.H * d.k;
-  return 128 + (staged ? (size_t)per * d.dv * 4 : 0) + 2 * (size_t)d.dv * 4 + HK * 20 +
-         2 * HK * 16;
+  return 2 * (size_t)d.dv * 4 + HK * 20 + 2 * HK * 16;
 }
 
 static ReadPlan read_plan(const Dims &d) {
@@ -65,8 +61,9 @@ static ReadPlan read_plan(const Dims &d) {
          (size_t)((HK + p.G - 1) / p.G) * row_bytes > kReadCtaRows)
     p.G <<= 1;
   p.per = (HK + p.G - 1) / p.G;
-  p.staged = read_smem_bytes(d, p.per, true) <= kReadSmemBudget;
-  p.smem = read_smem_bytes(d, p.per, p.staged);
+  const int dv4 = d.dv / 4;
+  p.threads = dv4 <= 32 ? 32 : (dv4 <= 64 ? 64 : 128);
+  p.smem = read_smem_bytes(d);
   return p;
 }
 
@@ -115,8 +112,8 @@ __device__ __forceinline__ float ld_peer(uint32_t addr) {
   return v;
 }
 
-template <typename TV, bool kStaged>
-__global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__restrict__ V,
+template <typename TV, int kThreads>
+__global__ void __launch_bounds__(kThreads) k_read(Dims d, const float *__restrict__ V,
                                                        const TV *__restrict__ Vt,
                                                        const float *__restrict__ gate,
                                                        const float *__restrict__ omega,
@@ -128,10 +125,8 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   // cluster takes the same branch): nothing of this chunk is read or written.
   if (chunk_aborted(s, ERR_READ_TIMEOUT)) return;
   extern __shared__ __align__(128) unsigned char smem[];
-  uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
   const int HK = d.H * d.k, dv = d.dv, dv4 = dv >> 2;
-  float *rows_s = reinterpret_cast<float *>(smem + 128);
-  float *ypart = rows_s + (kStaged ? (size_t)per * dv : 0);
+  float *ypart = reinterpret_cast<float *>(smem);
   float *e_s = ypart + dv;
   float *w_s = e_s + dv;
   int *slot_s = reinterpret_cast<int *>(w_s + HK);
@@ -163,31 +158,26 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
     claim_s[j] = s.pclaim[p0 + j];
   }
   const int64_t e0 = (int64_t)row * 2 * HK;  // entries of this row: e0 + (h*2 + half)*k + idx
-  for (int x = rank + G * tid; x < 2 * HK; x += G * blockDim.x) {
+  // d.readonly (eta = 0): the read alone -- no records, residual, dL/dw or
+  // alphas (the selection wrote no claims or entries either)
+  for (int x = rank + G * tid; x < (d.readonly ? 0 : 2 * HK); x += G * blockDim.x) {
     esub_s[x] = s.esub[e0 + x];
     eclaim_s[x] = s.eclaim[e0 + x];
     emask_s[x] = s.emask[e0 + x];
     einv_s[x] = s.einv[e0 + x];
   }
-  if (kStaged && tid == 0) mbar_init(bar, 1);
   __syncthreads();
-  const unsigned row_bytes = (unsigned)dv * 4u;
-  if (kStaged && wid == 0 && j1 > j0) {
-    if (lane == 0) mbar_arrive_expect_tx(bar, row_bytes * (unsigned)(j1 - j0));
-    __syncwarp();
-    for (int j = j0 + lane; j < j1; j += 32)
-      bulk_g2s(rows_s + (size_t)(j - j0) * dv, V + (int64_t)slot_s[j] * dv, row_bytes, bar);
-  }
   const float g = gate[tok];
   const float om = last ? 0.f : (omega ? omega[tok] : g);  // the token's MSE weight
-  const float invH = 1.f / (float)d.H;
+  const float invH = d.heads_sum ? 1.f : 1.f / (float)d.H;  // head readouts averaged or summed
   // the token's target row, loaded now so that it is here when e is formed
-  constexpr int kVt = 4;  // float4 per thread held (dv <= 4 * 4 * kReadThreads)
+  constexpr int kVt = 4;  // float4 per thread held (dv <= 4 * 4 * kThreads)
   float4 vt[kVt];
 #pragma unroll
   for (int q = 0; q < kVt; ++q) {
-    const int c4 = tid + q * kReadThreads;
-    vt[q] = c4 < dv4 ? load4(Vt, ttok * dv + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int c4 = tid + q * kThreads;
+    vt[q] = c4 < dv4 && !d.readonly ? load4(Vt, ttok * dv + 4 * c4)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 
   // Member records go to their buckets while the gather is in flight (none
@@ -195,7 +185,7 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   // slot >> vshift; entries x = rank (mod G) -> sub-key row bucket
   // NBv + (h*2+half)*n + row.  An entry's alpha is filled in later from
   // ealpha (by the sort, or by the apply when the entropy term is on).
-  for (int j = j0 + tid; j < j1; j += blockDim.x) {
+  for (int j = j0 + tid; j < (d.readonly ? j0 : j1); j += blockDim.x) {
     const int64_t p = p0 + j;
     const float w = w_s[j];
     Member m;
@@ -204,12 +194,12 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
     m.srow = row;
     m.gstart = 0;
     m.coef = 2.f * om * w * invH;
-    m.c0 = w * invH;
+    m.c0 = d.agg == AGG_COUNT ? 1.f : w * invH;  // the group's sum is the row's divisor
     m.c1 = w;
     m.glen = 0;
     s.rec_in[s.boff[slot_s[j] >> d.vshift] + claim_s[j]] = m;
   }
-  for (int x = rank + G * tid; x < 2 * HK; x += G * blockDim.x) {
+  for (int x = rank + G * tid; x < (d.readonly ? 0 : 2 * HK); x += G * blockDim.x) {
     const int mh = x / d.k;  // entry (h*2 + half)*k + idx of this row
     const int sub = esub_s[x];
     if (sub >= 0) {
@@ -226,19 +216,12 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
       s.rec_in[s.boff[d.NBv + mh * d.n + sub] + eclaim_s[x]] = m;
     }
   }
-  // On a timeout the error bit is set and the CTA still takes every cluster
-  // barrier (its results are then meaningless, and the host reports it).
-  if (kStaged && j1 > j0 && !mbar_wait_bounded(bar, 0, s.meta, d.mbar_polls, ERR_READ_TIMEOUT))
-    mbar_wait_bounded(bar, 0, nullptr, kDrainPolls, 0u);  // let copies in flight land
-
-  // pass 1: partial weighted sum of this CTA's rows
+  // pass 1: partial weighted sum of this CTA's rows, one column per thread
   for (int c4 = tid; c4 < dv4; c4 += blockDim.x) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = j0; j < j1; ++j) {
       const float w = w_s[j];
-      const float4 v =
-          kStaged ? *reinterpret_cast<const float4 *>(rows_s + (size_t)(j - j0) * dv + 4 * c4)
-                  : *reinterpret_cast<const float4 *>(V + (int64_t)slot_s[j] * dv + 4 * c4);
+      const float4 v = *reinterpret_cast<const float4 *>(V + (int64_t)slot_s[j] * dv + 4 * c4);
       acc.x = fmaf(w, v.x, acc.x);
       acc.y = fmaf(w, v.y, acc.y);
       acc.z = fmaf(w, v.z, acc.z);
@@ -254,7 +237,7 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   float4 y[kVt], e[kVt];
 #pragma unroll
   for (int q = 0; q < kVt; ++q) {
-    const int c4 = tid + q * kReadThreads;
+    const int c4 = tid + q * kThreads;
     y[q] = e[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (c4 >= dv4) continue;
     float4 yy = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -273,10 +256,10 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   }
   __syncthreads();
 
-  // dL/dw of this CTA's pairs: warp `wid` takes pairs j0 + wid, j0 + wid + 4, ...
+  // dL/dw of this CTA's pairs: warp `wid` takes pairs j0 + wid, j0 + wid + warps, ...
   const float coef = 2.f * om * invH;
-  for (int j = j0 + wid; j < j1; j += kReadThreads / 32) {
-    const float *vr = kStaged ? rows_s + (size_t)(j - j0) * dv : V + (int64_t)slot_s[j] * dv;
+  for (int j = j0 + wid; j < (d.readonly ? j0 : j1); j += kThreads / 32) {
+    const float *vr = V + (int64_t)slot_s[j] * dv;
     float acc = 0.f;
     for (int c4 = lane; c4 < dv4; c4 += 32) {
       const float4 v = *reinterpret_cast<const float4 *>(vr + 4 * c4);
@@ -300,18 +283,18 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   if (rank == 0) {
 #pragma unroll
     for (int q = 0; q < kVt; ++q) {
-      const int c4 = tid + q * kReadThreads;
+      const int c4 = tid + q * kThreads;
       if (c4 >= dv4) continue;
       *reinterpret_cast<float4 *>(out + tok * dv + 4 * c4) =
           make_float4(g * y[q].x, g * y[q].y, g * y[q].z, g * y[q].w);
-      *reinterpret_cast<float4 *>(s.E + (int64_t)row * dv + 4 * c4) = e[q];
+      if (!d.readonly) *reinterpret_cast<float4 *>(s.E + (int64_t)row * dv + 4 * c4) = e[q];
     }
   }
-  for (int j = j0 + tid; j < j1; j += blockDim.x) s.pa[p0 + j] = a_s[j];
+  for (int j = j0 + tid; j < (d.readonly ? j0 : j1); j += blockDim.x) s.pa[p0 + j] = a_s[j];
 
   // dL/ds and alpha per entry when the entropy term is off (dL/dw complete)
-  if (d.lam == 0.f) {
-    for (int h = wid; h < d.H; h += kReadThreads / 32) {
+  if (d.lam == 0.f && !d.readonly) {
+    for (int h = wid; h < d.H; h += kThreads / 32) {
       const int j = h * d.k + lane;
       float w = 0.f, a = 0.f;
       if (lane < d.k) {
@@ -340,17 +323,26 @@ __global__ void __launch_bounds__(kReadThreads) k_read(Dims d, const float *__re
   }
 }
 
+template <typename TV, int kThreads>
+static cudaError_t launch_read_tn(const Dims &d, const float *V, const TV *Vt, const float *gate,
+                                  const float *omega, float *out, const Scratch &s,
+                                  const ReadPlan &p, cudaStream_t st) {
+  auto kernel = k_read<TV, kThreads>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+  if (e != cudaSuccess) return e;
+  return launch_kc(d.pdl, p.G, kernel, d.rows * p.G, kThreads, p.smem, st, d, V, Vt, gate,
+                   omega, out, s, p.G, p.per);
+}
+
 template <typename TV>
 static cudaError_t launch_read_t(const Dims &d, const float *V, const TV *Vt, const float *gate,
                                  const float *omega, float *out, const Scratch &s,
                                  cudaStream_t st) {
   const ReadPlan p = read_plan(d);
-  auto kernel = p.staged ? k_read<TV, true> : k_read<TV, false>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
-  if (e != cudaSuccess) return e;
-  return launch_kc(d.pdl, p.G, kernel, d.rows * p.G, kReadThreads, p.smem, st, d, V, Vt, gate,
-                   omega, out, s, p.G, p.per);
+  if (p.threads == 32) return launch_read_tn<TV, 32>(d, V, Vt, gate, omega, out, s, p, st);
+  if (p.threads == 64) return launch_read_tn<TV, 64>(d, V, Vt, gate, omega, out, s, p, st);
+  return launch_read_tn<TV, 128>(d, V, Vt, gate, omega, out, s, p, st);
 }
 
 cudaError_t launch_read(const Dims &d, const float *V, const void *Vt, int v_dtype,
@@ -361,6 +353,6 @@ cudaError_t launch_read(const Dims &d, const float *V, const void *Vt, int v_dty
   return launch_read_t(d, V, (const float *)Vt, gate, omega, out, s, st);
 }
 
-bool read_is_staged(const Dims &d) { return read_plan(d).staged; }
+int read_cluster_size(const Dims &d) { return read_plan(d).G; }
 
 }  // namespace fwpkm

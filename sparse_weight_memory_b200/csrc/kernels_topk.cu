@@ -421,7 +421,7 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
       if (lane < k) {
         s.pslot[p] = slot_r;
         s.pw[p] = w;
-        s.pclaim[p] = atomicAdd(&s.bcnt[slot_r >> d.vshift], 1);  // value bucket
+        if (!d.readonly) s.pclaim[p] = atomicAdd(&s.bcnt[slot_r >> d.vshift], 1);  // value bucket
         if (x.rec_slots) {
           x.rec_slots[th * k + lane] = slot_r;
           x.rec_w[th * k + lane] = w;
@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
       }
     }
   }
-  if (kSelectOnly) return;
+  if (kSelectOnly || d.readonly) return;  // no write follows: no entries
   __syncthreads();
 
   // ---- sub-key entries of this warp's half: one per distinct row among the

@@ -20,6 +20,7 @@ FWPKM_OK, FWPKM_EINVAL, FWPKM_ESHAPE, FWPKM_ENOMEM, FWPKM_ECUDA, FWPKM_EUNSUPPOR
     0, -1, -2, -3, -4, -5)
 FWPKM_F32, FWPKM_BF16 = 0, 1
 FWPKM_LOOKAHEAD = 1
+FWPKM_HEADS_SUM, FWPKM_AGG_COUNT, FWPKM_AGG_SUM = 1, 2, 4
 STATUS_NAMES = {0: "OK", -1: "EINVAL", -2: "ESHAPE", -3: "ENOMEM", -4: "ECUDA",
                 -5: "EUNSUPPORTED"}
 
@@ -66,6 +67,7 @@ def load_library():
     L.fwpkm_read_stats.argtypes = [_vp, i64p, i64p, i64p, i64p, u32p, i32, _vp]
     L.fwpkm_select_noalloc.argtypes = [_vp, i32, i32, _vp, i32, _vp, _vp, _vp, _vp]
     L.fwpkm_set_wait_limits.argtypes = [_vp, i64, i64]
+    L.fwpkm_state_set_options.argtypes = [_vp, ctypes.c_uint]
     L.fwpkm_inject_alloc_failures.argtypes = [i32]
     L.fwpkm_inject_alloc_failures.restype = None
     for name in ("fwpkm_state_init", "fwpkm_state_set_eps", "fwpkm_step", "fwpkm_step_host",
@@ -73,7 +75,7 @@ def load_library():
                  "fwpkm_state_get", "fwpkm_state_set", "fwpkm_record_selection",
                  "fwpkm_force_selection", "fwpkm_set_profiling", "fwpkm_profile_read",
                  "fwpkm_read_stats", "fwpkm_select_noalloc", "fwpkm_set_graphs",
-                 "fwpkm_set_wait_limits"):
+                 "fwpkm_set_wait_limits", "fwpkm_state_set_options"):
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -225,6 +227,13 @@ class FwPKMState:
                                                    _ptr(slots), _ptr(weights), _ptr(errors),
                                                    _stream(stream)))
         return slots, weights
+
+    def set_options(self, heads: str = "mean", agg: str = "weight"):
+        """Readings of the step: ``heads`` "mean" or "sum"; ``agg`` (divisor
+        of a value row's gradient) "weight", "count" or "sum"."""
+        opts = {"mean": 0, "sum": FWPKM_HEADS_SUM}[heads] | \
+            {"weight": 0, "count": FWPKM_AGG_COUNT, "sum": FWPKM_AGG_SUM}[agg]
+        _check(load_library().fwpkm_state_set_options(self._h, opts))
 
     def set_wait_limits(self, mbar_polls: int = -1, scan_polls: int = -1):
         """Bounds of the device-side waits (negative = the default)."""

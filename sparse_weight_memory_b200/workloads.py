@@ -63,6 +63,8 @@ class Workload:
     seed: int = 0
     eps: float = 1e-3
     lookahead: bool = False  # each call writes query t towards the target of token t+1
+    heads_mode: str = "mean"  # head readouts "mean" or "sum"
+    agg: str = "weight"       # divisor of a value row's gradient: "weight", "count", "sum"
 
     @property
     def N(self) -> int:

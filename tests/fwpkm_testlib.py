@@ -70,7 +70,8 @@ def oracle_run(wl: Workload, inp: Inputs, oracle, max_chunks: int = 0,
     """Oracle over the workload's calls; continues `state` in place if given.
     ``omega`` [B][T_total]: the tokens' MSE weights (default: the gate)."""
     st = state if state is not None else oracle.State(inp.subkeys, inp.values, topk=wl.topk,
-                                                      chunk=wl.chunk, eps=wl.eps)
+                                                      chunk=wl.chunk, eps=wl.eps,
+                                                      heads=wl.heads_mode, agg=wl.agg)
     outs, sels, ws, gaps, touched = [], [], [], [], 0
     for Q, Vt, g, om in schedule(wl, inp, omega):
         r = st.step(widen(Q), widen(Vt), g, wl.eta, wl.lam, want_sel=True, want_gap=True,
@@ -93,6 +94,7 @@ def gpu_run(wl: Workload, inp: Inputs, ref: Optional[RunResult] = None, force: b
 
     from sparse_weight_memory_b200 import FwPKMState
     st = FwPKMState(wl.N, wl.dq, wl.dv, wl.topk, wl.chunk, wl.heads, eps=wl.eps)
+    st.set_options(heads=wl.heads_mode, agg=wl.agg)
     st.set_tables(to_dev(inp.subkeys if K0 is None else K0),
                   to_dev(inp.values if V0 is None else V0))
     if with_stats:

@@ -81,6 +81,7 @@ def test_null_arguments_are_rejected(lib):
     assert lib.fwpkm_select_noalloc(None, 1, 1, None, 0, None, None, None, None) == \
         fwpkm.FWPKM_EINVAL
     assert lib.fwpkm_set_wait_limits(None, 0, 0) == fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_state_set_options(None, 0) == fwpkm.FWPKM_EINVAL
     assert lib.fwpkm_step_ex(None, 1, 1, None, 0, None, 0, None, None, 0, 1.0, 0.0, None,
                              None) == fwpkm.FWPKM_EINVAL
     assert lib.fwpkm_step_host_ex(None, 1, 1, None, 0, None, 0, None, None, 0, 1.0, 0.0, None,

@@ -74,10 +74,10 @@ def check_recovers(st, wl, inp):
         assert np.array_equal(a, b)
 
 
-# The smallest shape whose bucket scan spans two CTAs (16,384 buckets each):
-# 128 x 128 slots, 2048 rows per chunk with 32 pairs each, so 16,384 value
-# buckets plus 256 sub-key rows.  The first CTA never waits; the second gives
-# up at once with a bound of 0, which the error bit then proves.
+# A shape whose bucket scan spans several CTAs (2048 buckets each): 128 x 128
+# slots, 2048 rows per chunk with 32 pairs each, so 16,384 value buckets plus
+# 256 sub-key rows.  The first CTA never waits; the later ones give up at once
+# with a bound of 0, which the error bit then proves.
 SCAN2 = Workload("scan2", B=1, T=4096, chunk=2048, heads=1, dq=16, n=128, dv=4, topk=32,
                  eta=0.5, lam=0.0, gate="uniform")
 

@@ -94,3 +94,35 @@ def test_hand_step_lookahead_on_gpu():
         K[tuple(int(v) for v in key.split(","))] = arr(row)
     check_table(res.K[..., :hs.dq // 2], K, 1e-4, "lookahead sub-keys")
     assert not res.K[..., hs.dq // 2:].any()
+
+
+@pytest.mark.parametrize("agg", ["count", "sum"])
+def test_hand_step_other_row_divisors_on_gpu(agg):
+    """The fixture's value rows divided by their access count, or not at all."""
+    hs = load_hand_step()
+    wl, inp = padded_case(hs, 0.0)
+    res = gpu_run(wl.replace(agg=agg), inp, None, force=False)
+    V = hs.V.copy()
+    for r, row in hs.raw["aggregation"][agg]["values_after"].items():
+        V[int(r)] = arr(row)
+    check_table(res.V[:, :hs.dv], V, 1e-4, f"{agg} values")
+    assert not res.V[:, hs.dv:].any()
+    check_table(res.K[..., :hs.dq // 2], hs.subkeys_after(), 1e-4, f"{agg} sub-keys")
+
+
+def test_hand_step_two_heads_summed_on_gpu():
+    """The two-head fixture with the head readouts summed."""
+    hs = load_hand_step("hand_step_two_heads.yaml")
+    part = hs.raw["heads_sum"]
+    wl, inp = padded_case(hs, 0.0)
+    res = gpu_run(wl.replace(heads_mode="sum"), inp, None, force=False)
+    check_close(res.outs[0][..., :hs.dv], arr(part["out"]), OUT_ATOL, OUT_RTOL, "summed out")
+    V = hs.V.copy()
+    for r, row in part["values_after"].items():
+        V[int(r)] = arr(row)
+    check_table(res.V[:, :hs.dv], V, 1e-4, "summed values")
+    K = hs.K.copy()
+    for key, row in part["subkeys_after"].items():
+        K[tuple(int(v) for v in key.split(","))] = arr(row)
+    check_table(res.K[..., :hs.dq // 2], K, 1e-4, "summed sub-keys")
+    assert not res.K[..., hs.dq // 2:].any()

@@ -159,7 +159,7 @@ def test_second_pass_equals_step_from_pass1_state():
     assert np.array_equal(two.V, again.V) and np.array_equal(two.K, again.K)
 
 
-@pytest.mark.parametrize("case", ["library", "multihead", "ragged"])
+@pytest.mark.parametrize("case", ["library", "multihead", "ragged", "read_only"])
 def test_host_buffer_step_equals_device_step(case):
     """Host buffers (copied in and out chunk by chunk, overlapping the step)
     give the device call's results bit for bit: several sequences, bf16
@@ -170,6 +170,8 @@ def test_host_buffer_step_equals_device_step(case):
     if case == "ragged":
         base = REDUCED["library"]
         wl = base.replace(calls=1, B=3, T=3 * base.chunk + 7)
+    elif case == "read_only":
+        wl = REDUCED["iterative"].replace(calls=1, passes=1, eta=0.0)
     else:
         wl = REDUCED[case].replace(calls=1, passes=1)
     inp = make_inputs(wl)
@@ -205,11 +207,11 @@ EDGE = {
                         eta=0.3, lam=0.0, gate="one"),
     "many_heads_big_k": Workload("e7", B=1, T=40, chunk=20, heads=4, dq=32, n=64, dv=1024,
                                  topk=32, eta=0.2, lam=0.01, gate="uniform"),
-    # 16 heads x k = 32 rows of 4 KB per token: a cluster CTA's share (64 rows)
-    # does not fit in shared memory, so the read takes its unstaged variant
-    "heads16_unstaged_read": Workload("e8", B=1, T=24, chunk=12, heads=16, dq=32, n=32,
+    # 16 heads x k = 32 rows of 4 KB (8 KB) per token: 2 MB (4 MB) of rows, so
+    # the read splits each token over a cluster of 2 (4) CTAs
+    "heads16_cluster2_read": Workload("e8", B=1, T=24, chunk=12, heads=16, dq=32, n=32,
                                       dv=1024, topk=32, eta=0.2, lam=0.0, gate="uniform"),
-    "heads16_unstaged_read_entropy": Workload("e9", B=1, T=20, chunk=10, heads=16, dq=32,
+    "heads16_cluster4_read_entropy": Workload("e9", B=1, T=20, chunk=10, heads=16, dq=32,
                                               n=32, dv=2048, topk=32, eta=0.2, lam=0.05,
                                               gate="uniform"),
     # dq/2 = 1024: 32 k-blocks in the score ring and 8 chunk norms per sub-key row
@@ -220,22 +222,20 @@ EDGE = {
 }
 
 
-def read_is_staged(wl) -> bool:
-    """The read kernel's sizing rule: a cluster of G <= 8 CTAs per token, G
-    doubled while a CTA's share of the H*k rows exceeds 32 KB; the share is
-    staged in shared memory when it fits in 200 KB with the per-token arrays."""
+def read_cluster_size(wl) -> int:
+    """The read kernel's sizing rule: one CTA per token, doubled into a
+    cluster of G <= 8 CTAs while a CTA's share of the H*k rows exceeds 1 MB."""
     HK, row = wl.heads * wl.topk, wl.dv * 4
     G = 1
-    while G < 8 and G < HK and -(-HK // G) * row > 32 * 1024:
+    while G < 8 and G < HK and -(-HK // G) * row > 1024 * 1024:
         G *= 2
-    per = -(-HK // G)
-    return 128 + per * row + 2 * row + HK * 20 + 2 * HK * 16 <= 200 * 1024
+    return G
 
 
-def test_edge_table_reaches_both_read_variants():
-    assert not read_is_staged(EDGE["heads16_unstaged_read"])
-    assert not read_is_staged(EDGE["heads16_unstaged_read_entropy"])
-    assert read_is_staged(EDGE["many_heads_big_k"])
+def test_edge_table_reaches_the_cluster_read():
+    assert read_cluster_size(EDGE["heads16_cluster2_read"]) == 2
+    assert read_cluster_size(EDGE["heads16_cluster4_read_entropy"]) == 4
+    assert read_cluster_size(EDGE["many_heads_big_k"]) == 1
 
 
 @pytest.mark.parametrize("name", sorted(EDGE))
@@ -290,3 +290,33 @@ def test_invalid_arguments_launch_nothing():
         FwPKMState(1000, 64, 64, 4, 32)
     assert e.value.status == FWPKM_ESHAPE
     st.close()
+
+
+def test_eta_zero_runs_the_read_alone():
+    """eta = 0 changes no table, so the step is the read alone: the write
+    kernels do not launch, the first chunk's outputs equal those of a step
+    with a tiny eta bit for bit (the read is the same), and the tables stay."""
+    import torch
+
+    from sparse_weight_memory_b200 import FwPKMState
+    wl = REDUCED["multihead"].replace(calls=1)
+    inp = make_inputs(wl)
+    Q, Vt, g = to_dev(inp.Q), to_dev(inp.Vt), to_dev(inp.gate)
+    outs = []
+    for eta in (0.0, 1e-30):
+        st = FwPKMState(wl.N, wl.dq, wl.dv, wl.topk, wl.chunk, wl.heads, eps=wl.eps)
+        st.set_tables(to_dev(inp.subkeys), to_dev(inp.values))
+        st.set_profiling(True)
+        out = st.step(Q, Vt, g, eta, wl.lam)
+        prof = st.profile_read()
+        outs.append(out[:, :wl.chunk].cpu().numpy())
+        if eta == 0.0:
+            for kind in ("fwpkm_scan", "fwpkm_bsort", "fwpkm_apply", "fwpkm_pgrad"):
+                assert prof[kind][1] == 0, (kind, prof[kind])
+            assert prof["fwpkm_read"][1] == wl.n_chunks()
+            K, V = st.get_tables()
+            torch.cuda.synchronize()
+            assert np.array_equal(K.cpu().numpy(), inp.subkeys)
+            assert np.array_equal(V.cpu().numpy(), inp.values)
+        st.close()
+    assert np.array_equal(outs[0], outs[1])
