@@ -51,6 +51,8 @@ def describe(wl) -> str:
         s += f" x{wl.passes} passes"
     if wl.lookahead:
         s += " lookahead (q_t written towards v_t+1)"
+    if wl.per_sequence:
+        s += f" one memory per sequence ({wl.B} memories)"
     return s
 
 
@@ -187,8 +189,11 @@ class OracleSampler:
     def _fresh(self):
         from oracle import oracle as orc
         wl, inp = self.wl, self.inp
-        self.state = orc.State(inp.subkeys, inp.values, topk=wl.topk, chunk=wl.chunk,
-                               eps=wl.eps)
+        # one state shared by the sequences, or one per sequence (all starting
+        # from the workload's tables)
+        self.state = [orc.State(inp.subkeys, inp.values, topk=wl.topk, chunk=wl.chunk,
+                                eps=wl.eps)
+                      for _ in range(wl.B if wl.per_sequence else 1)]
 
     def sample(self, budget_s: float):
         from oracle import oracle as orc
@@ -213,7 +218,12 @@ class OracleSampler:
             else:
                 Vt = widen_inputs(inp.Vt[:, lo:hi])
             t = time.perf_counter()
-            self.state.step(Q, Vt, g, wl.eta, wl.lam, omega=om)
+            if len(self.state) == 1:
+                self.state[0].step(Q, Vt, g, wl.eta, wl.lam, omega=om)
+            else:
+                for b, st in enumerate(self.state):
+                    st.step(Q[b:b + 1], Vt[b:b + 1], g[b:b + 1], wl.eta, wl.lam,
+                            omega=None if om is None else om[b:b + 1])
             elapsed += time.perf_counter() - t
             tokens += wl.B * (hi - lo)
             chunks += 1
@@ -342,7 +352,12 @@ def run_gpu(args, wl):
             return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
         return torch.from_numpy(a).to(dev)
 
-    K0, V0 = to_dev(inp.subkeys), to_dev(inp.values)
+    mem = wl.B if wl.per_sequence else 1
+    if mem > 1:  # every memory starts from the workload's tables
+        K0 = to_dev(np.stack([inp.subkeys] * mem))
+        V0 = to_dev(np.stack([inp.values] * mem))
+    else:
+        K0, V0 = to_dev(inp.subkeys), to_dev(inp.values)
     segs = []
     for c in range(wl.calls):
         sl = slice(c * wl.T, (c + 1) * wl.T)
@@ -350,7 +365,7 @@ def run_gpu(args, wl):
         for _ in range(wl.passes):
             segs.append((dq_, dv_, dg_))
     outs = [torch.empty((wl.B, wl.T, wl.dv), dtype=torch.float32, device=dev) for _ in segs]
-    st = FwPKMState(wl.N, wl.dq, wl.dv, wl.topk, wl.chunk, wl.heads, eps=wl.eps)
+    st = FwPKMState(wl.N, wl.dq, wl.dv, wl.topk, wl.chunk, wl.heads, eps=wl.eps, memories=mem)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -538,6 +553,9 @@ def main():
     ap.add_argument("--passes", type=int, default=0,
                     help="reads of each segment with the memory carried over (default: the "
                          "workload's)")
+    ap.add_argument("--per-sequence", action="store_true",
+                    help="one memory per sequence: the B sequences of a call each read and "
+                         "write their own memory, in the same launches")
     ap.add_argument("--lookahead", action="store_true",
                     help="write query t towards the target of token t+1 (each call's last "
                          "token has weight 0)")
@@ -549,6 +567,8 @@ def main():
         wl = wl.replace(passes=args.passes)
     if args.lookahead:
         wl = wl.replace(lookahead=True)
+    if args.per_sequence:
+        wl = wl.replace(per_sequence=True)
     if args.impl == "reference":
         run_reference(args, wl)
     else:

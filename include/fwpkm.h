@@ -78,6 +78,25 @@ enum { FWPKM_F32 = 0, FWPKM_BF16 = 1 };
 fwpkm_status fwpkm_state_init(int64_t N, int dq, int dv, int topk, int chunk, int heads,
                               fwpkm_state **out);
 
+/*
+ * fwpkm_state_init_batched -- `memories` independent memories in one state,
+ * one per sequence: a step over B = memories sequences reads and writes
+ * memory b with sequence b only, all of them in the same launches.  (The
+ * other reading of a memory per sequence; the package page chains one
+ * memory per call, pypi.org fast-weight-product-key-memory, Usage.)  Each
+ * memory is a state of fwpkm_state_init's shape; the arguments and limits
+ * are those, plus memories >= 1 with memories * (N + 2*heads*n) < 2^31.
+ * The tables stack the memories: sub-keys [memories][heads][2][n][dq/2],
+ * values [memories][N][dv] (fwpkm_state_get / set copy all of them).  A
+ * step's B must equal `memories` (FWPKM_ESHAPE otherwise).  The marginal of
+ * the entropy term is each memory's own (its M = chunk * heads
+ * token-heads).  Selections read and forced (fwpkm_record_selection /
+ * fwpkm_force_selection) are slots of the token's own memory, 0 .. N-1.
+ * fwpkm_select_noalloc does not take such a state (FWPKM_EUNSUPPORTED).
+ */
+fwpkm_status fwpkm_state_init_batched(int64_t N, int dq, int dv, int topk, int chunk, int heads,
+                                      int memories, fwpkm_state **out);
+
 /* Release the state and all memory it owns (NULL is a no-op).  Synchronises
  * the device first so no enqueued work still uses the memory. */
 void fwpkm_state_free(fwpkm_state *s);

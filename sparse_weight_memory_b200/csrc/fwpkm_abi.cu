@@ -98,6 +98,7 @@ constexpr size_t kGraphSeen = 16;
 struct fwpkm_state {
   int64_t N = 0;
   int n = 0, dq = 0, dh = 0, dv = 0, k = 0, chunk = 0, H = 0;
+  int nmem = 1;  // memories: 1 shared, or one per sequence (fwpkm_state_init_batched)
   float eps = 1e-3f;
   int device = 0;
   int sm_count = 148;
@@ -105,8 +106,8 @@ struct fwpkm_state {
   long long mbar_polls = kDefaultMbarPolls, scan_polls = kDefaultScanPolls;
   // readings (fwpkm_state_set_options)
   int heads_sum = 0, agg = AGG_WEIGHT;
-  float *K = nullptr;  // [H][2][n][dh]
-  float *V = nullptr;  // [N][dv]
+  float *K = nullptr;  // [nmem][H][2][n][dh]
+  float *V = nullptr;  // [nmem][N][dv]
   // scratch arena
   void *arena = nullptr;
   size_t arena_bytes = 0;
@@ -164,7 +165,8 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
   if (rows <= st->cap_rows) return FWPKM_OK;
   rows = (rows + 127) / 128 * 128;  // query-half stride: whole 128-row score tiles
   const int64_t H = st->H, n = st->n, dh = st->dh, dv = st->dv, k = st->k;
-  const int64_t M = rows * H, P = M * k, NB = value_buckets(st->N, P) + 2 * H * n;
+  const int64_t nm = st->nmem, Nt = st->N * nm;  // all memories' value rows
+  const int64_t M = rows * H, P = M * k, NB = value_buckets(Nt, P) + 2 * H * nm * n;
   const int64_t Lcap = 3 * P;  // pairs + at most 2 entries per pair
   // Blocks of groups of more than 4 members, 32 members a block: at most
   // L/32 + L/5 of them, under L/4.
@@ -179,9 +181,9 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
       {(void **)&s.Qs_hi, sizeof(float) * (size_t)(H * 2 * rows * dh)},
       {(void **)&s.Qs_lo, sizeof(float) * (size_t)(H * 2 * rows * dh)},
       {(void **)&s.qn, sizeof(float) * (size_t)(H * 2 * rows)},
-      {(void **)&s.K_hi, sizeof(float) * (size_t)((H * 2 * n + 128) * dh)},
-      {(void **)&s.K_lo, sizeof(float) * (size_t)((H * 2 * n + 128) * dh)},
-      {(void **)&s.kn, sizeof(float) * (size_t)(H * 2 * n * kKnChunks)},
+      {(void **)&s.K_hi, sizeof(float) * (size_t)((H * nm * 2 * n + 128) * dh)},
+      {(void **)&s.K_lo, sizeof(float) * (size_t)((H * nm * 2 * n + 128) * dh)},
+      {(void **)&s.kn, sizeof(float) * (size_t)(H * nm * 2 * n * kKnChunks)},
       {(void **)&s.D, sizeof(float) * (size_t)(H * 2 * rows * n)},
       {(void **)&s.pslot, sizeof(int32_t) * (size_t)P},
       {(void **)&s.pw, sizeof(float) * (size_t)P},
@@ -253,7 +255,7 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
     return cuda_fail(e, "scratch initialisation");
   }
   TcMaps maps;
-  e = encode_score_maps(&maps, s, (int)H, (int)rows, (int)n, (int)dh);
+  e = encode_score_maps(&maps, s, (int)H, (int)nm, (int)rows, (int)n, (int)dh);
   if (e != cudaSuccess) {
     cudaFree(arena);
     return cuda_fail(e, "scratch initialisation: tensor maps");
@@ -317,10 +319,15 @@ Dims chunk_dims(const fwpkm_state *st, int B, int T, int c, float eta, float lam
   d.rows = B * d.Tc;
   d.qstride = (int)st->cap_rows;
   d.M = d.rows * st->H;
+  d.nmem = st->nmem;
+  d.Nt = st->N * st->nmem;
+  d.rstride = st->nmem > 1 ? (d.Tc + 127) / 128 * 128 : d.Tc;
+  d.drows = B * d.rstride;
+  d.Mmem = d.M / st->nmem;
   const int64_t cap_pairs = st->cap_rows * st->H * st->k;  // bcnt was sized for this
-  d.vshift = value_shift(st->N, cap_pairs);
-  d.NBv = (int)value_buckets(st->N, cap_pairs);
-  d.NB = d.NBv + 2 * st->H * st->n;
+  d.vshift = value_shift(d.Nt, cap_pairs);
+  d.NBv = (int)value_buckets(d.Nt, cap_pairs);
+  d.NB = d.NBv + 2 * st->H * st->nmem * st->n;
   d.sm_count = st->sm_count;
   d.pdl = st->profiling ? 0 : 1;  // per-kernel events need plain stream order
   d.eps = st->eps;
@@ -496,6 +503,7 @@ bool state_view(const fwpkm_state *st, StateView *v) {
   v->H = st->H;
   v->device = st->device;
   v->sm_count = st->sm_count;
+  v->nmem = st->nmem;
   v->eps = st->eps;
   v->K = st->K;
   v->mbar_polls = st->mbar_polls;
@@ -513,6 +521,11 @@ const char *fwpkm_last_error(void) { return g_last_error.c_str(); }
 
 fwpkm_status fwpkm_state_init(int64_t N, int dq, int dv, int topk, int chunk, int heads,
                               fwpkm_state **out) {
+  return fwpkm_state_init_batched(N, dq, dv, topk, chunk, heads, 1, out);
+}
+
+fwpkm_status fwpkm_state_init_batched(int64_t N, int dq, int dv, int topk, int chunk, int heads,
+                                      int memories, fwpkm_state **out) {
   if (!out) return fail(FWPKM_EINVAL, "state_init: out is NULL");
   *out = nullptr;
   int64_t n = (int64_t)std::llround(std::sqrt((double)N));
@@ -532,6 +545,10 @@ fwpkm_status fwpkm_state_init(int64_t N, int dq, int dv, int topk, int chunk, in
     return fail(FWPKM_ESHAPE, "state_init: chunk=%d must be in [1, 2^20]", chunk);
   if (heads < 1 || heads > 16)
     return fail(FWPKM_ESHAPE, "state_init: heads=%d must be in [1, 16]", heads);
+  // member groups are 32-bit: every value row and sub-key row of all memories
+  if (memories < 1 || (int64_t)memories * (N + 2 * heads * n) >= ((int64_t)1 << 31))
+    return fail(FWPKM_ESHAPE, "state_init: memories=%d must be >= 1 with memories * (N + "
+                "2*heads*n) < 2^31", memories);
 
   fwpkm_state *st = new (std::nothrow) fwpkm_state();
   if (!st) return fail(FWPKM_ENOMEM, "state_init: host allocation failed");
@@ -543,11 +560,12 @@ fwpkm_status fwpkm_state_init(int64_t N, int dq, int dv, int topk, int chunk, in
   st->k = topk;
   st->chunk = chunk;
   st->H = heads;
+  st->nmem = memories;
   cudaGetDevice(&st->device);
   cudaDeviceGetAttribute(&st->sm_count, cudaDevAttrMultiProcessorCount, st->device);
   if (st->sm_count < 1) st->sm_count = 1;
-  const size_t kbytes = sizeof(float) * (size_t)heads * 2 * n * st->dh;
-  const size_t vbytes = sizeof(float) * (size_t)N * dv;
+  const size_t kbytes = sizeof(float) * (size_t)memories * heads * 2 * n * st->dh;
+  const size_t vbytes = sizeof(float) * (size_t)memories * N * dv;
   cudaError_t e = dev_malloc((void **)&st->K, kbytes);
   if (e == cudaSuccess) e = dev_malloc((void **)&st->V, vbytes);
   if (e == cudaSuccess) e = cudaMemset(st->K, 0, kbytes);
@@ -564,7 +582,8 @@ fwpkm_status fwpkm_state_init(int64_t N, int dq, int dv, int topk, int chunk, in
   // ensure_scratch ends with a device synchronisation, so the zeroed tables
   // are in place before a caller's stream (non-blocking ones included) copies
   // into them.
-  fwpkm_status rc = ensure_scratch(st, chunk);
+  fwpkm_status rc =
+      ensure_scratch(st, memories > 1 ? (int64_t)memories * ((chunk + 127) / 128 * 128) : chunk);
   if (rc != FWPKM_OK) {
     cudaFree(st->K);
     cudaFree(st->V);
@@ -646,7 +665,12 @@ fwpkm_status fwpkm_step_ex(fwpkm_state *st, int B, int T, const void *Q, int q_d
     return fail(FWPKM_EINVAL, "step: eta must be finite and >= 0");
   if (!(lambda_entropy >= 0.f) || !std::isfinite(lambda_entropy))
     return fail(FWPKM_EINVAL, "step: lambda_entropy must be finite and >= 0");
-  const int64_t rows_max = (int64_t)B * (T < st->chunk ? T : st->chunk);
+  if (st->nmem > 1 && B != st->nmem)
+    return fail(FWPKM_ESHAPE, "step: B=%d must equal the state's %d memories (one per sequence)",
+                B, st->nmem);
+  const int64_t tc_max = T < st->chunk ? T : st->chunk;
+  // rows of the query-half layout: one memory per sequence starts each on a whole score tile
+  const int64_t rows_max = (int64_t)B * (st->nmem > 1 ? (tc_max + 127) / 128 * 128 : tc_max);
   if (rows_max * st->H * st->k * 3 >= (int64_t)1 << 31 || (int64_t)B * T * st->dv >= (int64_t)1 << 40)
     return fail(FWPKM_ESHAPE, "step: B*chunk*heads*topk too large for 32-bit pair ids");
   if ((int64_t)B * T * 2 * st->H >= (int64_t)1 << 31)
@@ -734,7 +758,12 @@ fwpkm_status fwpkm_step_host_ex(fwpkm_state *st, int B, int T, const void *Q_hos
     return fail(FWPKM_EINVAL, "step_host: eta must be finite and >= 0");
   if (!(lambda_entropy >= 0.f) || !std::isfinite(lambda_entropy))
     return fail(FWPKM_EINVAL, "step_host: lambda_entropy must be finite and >= 0");
-  const int64_t rows_max = (int64_t)B * (T < st->chunk ? T : st->chunk);
+  if (st->nmem > 1 && B != st->nmem)
+    return fail(FWPKM_ESHAPE,
+                "step_host: B=%d must equal the state's %d memories (one per sequence)", B,
+                st->nmem);
+  const int64_t tc_max = T < st->chunk ? T : st->chunk;
+  const int64_t rows_max = (int64_t)B * (st->nmem > 1 ? (tc_max + 127) / 128 * 128 : tc_max);
   if (rows_max * st->H * st->k * 3 >= (int64_t)1 << 31 || (int64_t)B * T * st->dv >= (int64_t)1 << 40)
     return fail(FWPKM_ESHAPE, "step_host: B*chunk*heads*topk too large for 32-bit pair ids");
   if ((int64_t)B * T * 2 * st->H >= (int64_t)1 << 31)
@@ -860,10 +889,11 @@ fwpkm_status fwpkm_state_get(const fwpkm_state *st, float *subkeys, float *value
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaSuccess;
   if (subkeys)
-    e = cudaMemcpyAsync(subkeys, st->K, sizeof(float) * (size_t)st->H * 2 * st->n * st->dh,
+    e = cudaMemcpyAsync(subkeys, st->K,
+                        sizeof(float) * (size_t)st->nmem * st->H * 2 * st->n * st->dh,
                         cudaMemcpyDefault, s);
   if (e == cudaSuccess && values)
-    e = cudaMemcpyAsync(values, st->V, sizeof(float) * (size_t)st->N * st->dv,
+    e = cudaMemcpyAsync(values, st->V, sizeof(float) * (size_t)st->nmem * st->N * st->dv,
                         cudaMemcpyDefault, s);
   if (e != cudaSuccess) return cuda_fail(e, "state_get");
   return FWPKM_OK;
@@ -875,10 +905,11 @@ fwpkm_status fwpkm_state_set(fwpkm_state *st, const float *subkeys, const float 
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaSuccess;
   if (subkeys)
-    e = cudaMemcpyAsync(st->K, subkeys, sizeof(float) * (size_t)st->H * 2 * st->n * st->dh,
+    e = cudaMemcpyAsync(st->K, subkeys,
+                        sizeof(float) * (size_t)st->nmem * st->H * 2 * st->n * st->dh,
                         cudaMemcpyDefault, s);
   if (e == cudaSuccess && values)
-    e = cudaMemcpyAsync(st->V, values, sizeof(float) * (size_t)st->N * st->dv,
+    e = cudaMemcpyAsync(st->V, values, sizeof(float) * (size_t)st->nmem * st->N * st->dv,
                         cudaMemcpyDefault, s);
   if (e != cudaSuccess) return cuda_fail(e, "state_set");
   if (subkeys && st->arena) {  // new sub-keys: their split, stream-ordered after the copy

@@ -79,6 +79,14 @@ struct Dims {
   long long scan_polls;  // bound of a scan CTA's wait for an earlier CTA's total
   int lookahead;         // token t is written towards the target of token t+1
   int q_tf32_exact;      // the queries are bf16, so exact in TF32 (their lo part is zero)
+  // Memories: 1 (all sequences share the one memory), or one per sequence
+  // (sequence b reads and writes memory b: sub-key tables b*H .. b*H+H-1,
+  // value rows b*N .. b*N+N-1).
+  int nmem;
+  int64_t Nt;            // value rows of all memories, nmem * N
+  int rstride;           // rows per sequence in the query-half and distance layouts
+  int drows;             // B * rstride: rows of those layouts
+  int Mmem;              // token-heads per memory, M / nmem
   int heads_sum;         // head readouts summed instead of averaged
   int readonly;          // eta = 0: the read alone (no claims, entries, records, gradients)
   int agg;               // divisor of a value row's gradient (AGG_*)
@@ -262,8 +270,19 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity
 __device__ __forceinline__ bool chunk_aborted(const Scratch &s, unsigned own) {
   return (*reinterpret_cast<volatile const unsigned *>(&s.meta->err) & (ERR_ALL & ~own)) != 0u;
 }
+// Memory of token row `row` (b * Tc + tl) of chunk d, and the row's place in
+// the query-half and distance layouts (b * rstride + tl: with one memory per
+// sequence every sequence starts a new 128-row score tile, so that a tile
+// scores against one memory's sub-keys).
+__device__ __forceinline__ int mem_of(const Dims &d, int row) {
+  return d.nmem > 1 ? row / d.Tc : 0;
+}
+__device__ __forceinline__ int lrow_of(const Dims &d, int row) {
+  return (row / d.Tc) * d.rstride + row % d.Tc;
+}
+
 // One query half (warp w = (h*2 + half)*rows + row of chunk d) into its TF32
-// split and squared norm: Qs_hi / Qs_lo [h][half][row][:], qn (rows at
+// split and squared norm: Qs_hi / Qs_lo [h][half][lrow][:], qn (rows at
 // stride qstride).  Warp-level; used by the prep and by the bucket sort's
 // extra CTAs (the next chunk's halves).
 template <typename TQ>
@@ -277,7 +296,7 @@ __device__ __forceinline__ void prep_query_half(const Dims &d, const TQ *__restr
   const int b = row / d.Tc, tl = row % d.Tc;
   const int64_t src = ((int64_t)b * d.T + d.t0 + tl) * ((int64_t)d.H * d.dq) +
                       (int64_t)h * d.dq + (int64_t)half * dh;
-  const int64_t o = ((int64_t)hh * d.qstride + row) * dh;
+  const int64_t o = ((int64_t)hh * d.qstride + lrow_of(d, row)) * dh;
   float acc = 0.f;
   for (int c = lane * 4; c < dh; c += 128) {
     const float4 v = load4(Q, src + c);
@@ -291,7 +310,7 @@ __device__ __forceinline__ void prep_query_half(const Dims &d, const TQ *__restr
     acc = fmaf(v.w, v.w, acc);
   }
   acc = warp_sum(acc);
-  if (lane == 0) s.qn[(int64_t)hh * d.qstride + row] = acc;
+  if (lane == 0) s.qn[(int64_t)hh * d.qstride + lrow_of(d, row)] = acc;
 }
 
 // Programmatic dependent launch.  A kernel started by launch_k with d.pdl set
@@ -361,10 +380,10 @@ struct TcMaps {
   alignas(64) unsigned char b_lo[4][128];
 };
 // Encodes the four maps over Qs_hi / Qs_lo ([2H*qstride][dh], qstride a
-// multiple of 128) and K_hi / K_lo ([2H*n + 128][dh]).  Host only; returns a
-// CUDA error code.
-cudaError_t encode_score_maps(TcMaps *maps, const Scratch &s, int H, int qstride, int n,
-                              int dh);
+// multiple of 128) and K_hi / K_lo ([2H*nmem*n + 128][dh]).  Host only;
+// returns a CUDA error code.
+cudaError_t encode_score_maps(TcMaps *maps, const Scratch &s, int H, int nmem, int qstride,
+                              int n, int dh);
 cudaError_t launch_score(const Dims &d, const Scratch &s, const TcMaps &maps, cudaStream_t st);
 cudaError_t launch_topk(const Dims &d, const Scratch &s, const Extras &x, cudaStream_t st);
 // Selection only: fills x.rec_slots / x.rec_w from the distances in s.D.
@@ -391,7 +410,7 @@ cudaError_t launch_pgrad(const Dims &d, const Scratch &s, cudaStream_t st);
 // Read-only view of a state's shape and sub-key tables (fwpkm_abi.cu).
 struct StateView {
   int64_t N;
-  int n, dq, dh, dv, k, chunk, H, device, sm_count;
+  int n, dq, dh, dv, k, chunk, H, device, sm_count, nmem;
   float eps;
   const float *K;
   long long mbar_polls;

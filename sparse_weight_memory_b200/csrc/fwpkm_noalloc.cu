@@ -82,6 +82,9 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
   cudaGetDevice(&dev);
   if (dev != v.device)
     return fail(FWPKM_EINVAL, "select_noalloc: current device is not the state's device");
+  if (v.nmem > 1)
+    return fail(FWPKM_EUNSUPPORTED, "select_noalloc: states with one memory per sequence are "
+                "not supported");
 
   // Scratch of one pass of `rows` token rows (fp32, each piece 256-byte
   // aligned; rows rounded up to 128): Qs_hi, Qs_lo [2H][rows][dh], qn
@@ -139,7 +142,7 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
   s.D = reinterpret_cast<float *>(p);
   s.meta = meta;
   TcMaps maps;  // host-side descriptors of the operands above (no allocation)
-  const cudaError_t me = encode_score_maps(&maps, s, v.H, rows_max, v.n, v.dh);
+  const cudaError_t me = encode_score_maps(&maps, s, v.H, 1, rows_max, v.n, v.dh);
   if (me != cudaSuccess) return fail(FWPKM_ECUDA, "select_noalloc: tensor map encoding failed");
 
   Extras x{};
@@ -170,6 +173,11 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
     d.rows = B * d.Tc;
     d.qstride = rows_max;
     d.M = d.rows * v.H;
+    d.nmem = 1;
+    d.Nt = v.N;
+    d.rstride = d.Tc;
+    d.drows = d.rows;
+    d.Mmem = d.M;
     d.sm_count = v.sm_count;
     d.pdl = 1;
     d.eps = v.eps;

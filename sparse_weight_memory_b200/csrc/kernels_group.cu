@@ -251,7 +251,7 @@ __device__ __forceinline__ int lower_rank(const uint64_t *r, int len, uint64_t k
 // only after pgrad and the apply reads it itself.
 __device__ __forceinline__ Member fetch_member(const Dims &d, const Scratch &s, const Member *p) {
   Member m = load_member(p);
-  if (d.lam == 0.f && m.g >= (uint32_t)d.N) m.coef = m.c0 = s.ealpha[m.id];
+  if (d.lam == 0.f && m.g >= (uint32_t)d.Nt) m.coef = m.c0 = s.ealpha[m.id];
   return m;
 }
 
@@ -580,7 +580,7 @@ __global__ void __launch_bounds__(kSortThreads)
     const int off = s.boff[b], len = s.boff[b + 1] - off;
     const bool value = b < d.NBv;
     const uint32_t gbase =
-        value ? ((uint32_t)b << d.vshift) : (uint32_t)d.N + (uint32_t)(b - d.NBv);
+        value ? ((uint32_t)b << d.vshift) : (uint32_t)d.Nt + (uint32_t)(b - d.NBv);
     const RankSmem rs{reinterpret_cast<uint32_t *>(buf), reinterpret_cast<uint32_t *>(buf) + kRankWords,
                       rank_red, &rank_flag};
     sort_big_bucket(d, s, off, len, value, gbase, buf, rs, &nseg[value ? 0 : 1]);
@@ -678,9 +678,10 @@ __device__ __forceinline__ float4 updated(const Dims &d, bool value, const float
 }
 
 // Entropy term of a value row: dL_addr/dw = (lam/M)(log pbar + 1) for every
-// pair of the group, pbar = (sum of the group's weights) / M.
+// pair of the group, pbar = (sum of the group's weights) / M, M the
+// token-heads of the row's memory.
 __device__ __forceinline__ float entropy_term(const Dims &d, float wsum) {
-  return (d.lam / (float)d.M) * (logf(wsum / (float)d.M) + 1.f);
+  return (d.lam / (float)d.Mmem) * (logf(wsum / (float)d.Mmem) + 1.f);
 }
 
 // Sum of a warp's members (lane j < cnt holds member j's srow and coef) over
@@ -837,7 +838,7 @@ __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__res
         Ct += __shfl_xor_sync(FULL, Ct, o);
         Wt += __shfl_xor_sync(FULL, Wt, o);
       }
-      float *row = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.N) * d.dh;
+      float *row = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.Nt) * d.dh;
       if (!value || Ct > 0.f) {
         const int c4 = cb + lane;
         const float4 t = load_chunk(row, c4, n4);
@@ -856,7 +857,7 @@ __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__res
         }
         const float4 nv = updated(d, value, t, tot, Ct);
         if (c4 < n4) *reinterpret_cast<float4 *>(row + 4 * c4) = nv;
-        if (!value) resplit_key_chunk(d, s, (int64_t)(g - (uint32_t)d.N), chunk, c4, n4, nv);
+        if (!value) resplit_key_chunk(d, s, (int64_t)(g - (uint32_t)d.Nt), chunk, c4, n4, nv);
       }
       if (chunk == 0 && value && d.lam != 0.f) {
         const float bt = entropy_term(d, Wt);
@@ -865,7 +866,7 @@ __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__res
       continue;
     }
     // a short group: the whole row, two column chunks at a time
-    float *dst = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.N) * d.dh;
+    float *dst = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.Nt) * d.dh;
     if (!value || C > 0.f) {
       for (int cb = 0; cb < n4; cb += 2 * kChunk4) {
         const float4 t0 = load_chunk(dst, cb + lane, n4);
@@ -878,7 +879,7 @@ __global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__res
         if (cb + lane < n4) *reinterpret_cast<float4 *>(dst + 4 * (cb + lane)) = nv0;
         if (cb + lane + 32 < n4) *reinterpret_cast<float4 *>(dst + 4 * (cb + lane + 32)) = nv1;
         if (!value) {
-          const int64_t r = (int64_t)(g - (uint32_t)d.N);
+          const int64_t r = (int64_t)(g - (uint32_t)d.Nt);
           resplit_key_chunk(d, s, r, cb / kChunk4, cb + lane, n4, nv0);
           if (cb + kChunk4 < n4) resplit_key_chunk(d, s, r, cb / kChunk4 + 1, cb + lane + 32, n4, nv1);
         }

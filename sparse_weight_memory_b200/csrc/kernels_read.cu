@@ -180,8 +180,40 @@ __global__ void __launch_bounds__(kThreads) k_read(Dims d, const float *__restri
                                      : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 
-  // Member records go to their buckets while the gather is in flight (none
-  // of their fields depends on the rows): this CTA's pairs -> value bucket
+  // pass 1: partial weighted sum of this CTA's rows, one column per thread.
+  // Eight rows are loaded before any is added, so that their loads are in
+  // flight together; the sum still runs in row order.
+  for (int c4 = tid; c4 < dv4; c4 += blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float *col = V + 4 * c4;
+    int j = j0;
+    for (; j + 8 <= j1; j += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        v[u] = *reinterpret_cast<const float4 *>(col + (int64_t)slot_s[j + u] * dv);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float w = w_s[j + u];
+        acc.x = fmaf(w, v[u].x, acc.x);
+        acc.y = fmaf(w, v[u].y, acc.y);
+        acc.z = fmaf(w, v[u].z, acc.z);
+        acc.w = fmaf(w, v[u].w, acc.w);
+      }
+    }
+    for (; j < j1; ++j) {
+      const float w = w_s[j];
+      const float4 v = *reinterpret_cast<const float4 *>(col + (int64_t)slot_s[j] * dv);
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+    *reinterpret_cast<float4 *>(ypart + 4 * c4) = acc;
+  }
+  // Member records go to their buckets after the rows (none of their fields
+  // depends on them, and their bucket offsets are one more dependent load
+  // that would otherwise delay the rows): this CTA's pairs -> value bucket
   // slot >> vshift; entries x = rank (mod G) -> sub-key row bucket
   // NBv + (h*2+half)*n + row.  An entry's alpha is filled in later from
   // ealpha (by the sort, or by the apply when the entropy term is on).
@@ -199,13 +231,14 @@ __global__ void __launch_bounds__(kThreads) k_read(Dims d, const float *__restri
     m.glen = 0;
     s.rec_in[s.boff[slot_s[j] >> d.vshift] + claim_s[j]] = m;
   }
+  const int tab0 = mem_of(d, row) * 2 * d.H;  // the token's memory's first sub-key table
   for (int x = rank + G * tid; x < (d.readonly ? 0 : 2 * HK); x += G * blockDim.x) {
     const int mh = x / d.k;  // entry (h*2 + half)*k + idx of this row
     const int sub = esub_s[x];
     if (sub >= 0) {
       const int64_t e = e0 + x;
       Member m;
-      m.g = (uint32_t)d.N + (uint32_t)(mh * d.n + sub);
+      m.g = (uint32_t)d.Nt + (uint32_t)((tab0 + mh) * d.n + sub);
       m.id = (uint32_t)e;
       m.srow = (int)(tok * 2 * d.H + mh);  // this query half in the caller's Q
       m.gstart = 0;
@@ -213,21 +246,8 @@ __global__ void __launch_bounds__(kThreads) k_read(Dims d, const float *__restri
       m.c0 = 0.f;
       m.c1 = 0.f;
       m.glen = 0;
-      s.rec_in[s.boff[d.NBv + mh * d.n + sub] + eclaim_s[x]] = m;
+      s.rec_in[s.boff[d.NBv + (tab0 + mh) * d.n + sub] + eclaim_s[x]] = m;
     }
-  }
-  // pass 1: partial weighted sum of this CTA's rows, one column per thread
-  for (int c4 = tid; c4 < dv4; c4 += blockDim.x) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = j0; j < j1; ++j) {
-      const float w = w_s[j];
-      const float4 v = *reinterpret_cast<const float4 *>(V + (int64_t)slot_s[j] * dv + 4 * c4);
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
-    }
-    *reinterpret_cast<float4 *>(ypart + 4 * c4) = acc;
   }
   if (G > 1) cluster_barrier();
   else __syncthreads();
@@ -256,21 +276,36 @@ __global__ void __launch_bounds__(kThreads) k_read(Dims d, const float *__restri
   }
   __syncthreads();
 
-  // dL/dw of this CTA's pairs: warp `wid` takes pairs j0 + wid, j0 + wid + warps, ...
+  // dL/dw of this CTA's pairs: warp `wid` takes pairs j0 + wid, j0 + wid + warps, ...,
+  // two at a time so that both rows' loads are in flight together
   const float coef = 2.f * om * invH;
-  for (int j = j0 + wid; j < (d.readonly ? j0 : j1); j += kThreads / 32) {
+  constexpr int kWarps = kThreads / 32;
+  const int jend = d.readonly ? j0 : j1;
+  for (int j = j0 + wid; j < jend; j += 2 * kWarps) {
+    const int j2 = j + kWarps;
+    const bool two = j2 < jend;
     const float *vr = V + (int64_t)slot_s[j] * dv;
-    float acc = 0.f;
+    const float *vr2 = two ? V + (int64_t)slot_s[j2] * dv : vr;
+    float acc = 0.f, acc2 = 0.f;
     for (int c4 = lane; c4 < dv4; c4 += 32) {
       const float4 v = *reinterpret_cast<const float4 *>(vr + 4 * c4);
+      const float4 v2 = *reinterpret_cast<const float4 *>(vr2 + 4 * c4);
       const float4 e = *reinterpret_cast<const float4 *>(e_s + 4 * c4);
       acc = fmaf(e.x, v.x, acc);
       acc = fmaf(e.y, v.y, acc);
       acc = fmaf(e.z, v.z, acc);
       acc = fmaf(e.w, v.w, acc);
+      acc2 = fmaf(e.x, v2.x, acc2);
+      acc2 = fmaf(e.y, v2.y, acc2);
+      acc2 = fmaf(e.z, v2.z, acc2);
+      acc2 = fmaf(e.w, v2.w, acc2);
     }
     acc = warp_sum(acc);
-    if (lane == 0) a_s[j] = coef * acc;
+    acc2 = warp_sum(acc2);
+    if (lane == 0) {
+      a_s[j] = coef * acc;
+      if (two) a_s[j2] = coef * acc2;
+    }
   }
   // Every CTA is done reading the partials; with the entropy term off the
   // a values are published to the cluster for the alphas.

@@ -44,14 +44,15 @@ __global__ void __launch_bounds__(256) k_prep(Dims d, const TQ *__restrict__ Q,
   griddep_launch();
   const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nq = do_q ? (int64_t)2 * d.H * d.rows : 0;
-  const int64_t nk = do_k ? (int64_t)2 * d.H * d.n : 0;
+  const int64_t nk = do_k ? (int64_t)2 * d.H * d.nmem * d.n : 0;
   if (warp < nq) prep_query_half(d, Q, s, warp);
   else if (warp < nq + nk) prep_subkey_row(d, K, s, warp - nq);
 }
 
 static cudaError_t launch_prep_parts(const Dims &d, const void *Q, int q_dtype, const float *K,
                                      const Scratch &s, cudaStream_t st, int do_q, int do_k) {
-  const int64_t warps = (do_q ? (int64_t)2 * d.H * d.rows : 0) + (do_k ? (int64_t)2 * d.H * d.n : 0);
+  const int64_t warps =
+      (do_q ? (int64_t)2 * d.H * d.rows : 0) + (do_k ? (int64_t)2 * d.H * d.nmem * d.n : 0);
   const int blocks = (int)((warps + 7) / 8);
   if (blocks == 0) return cudaSuccess;
   if (q_dtype == 1)

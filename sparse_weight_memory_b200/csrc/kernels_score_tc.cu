@@ -156,7 +156,9 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hh = blockIdx.z;
-  const int m0 = blockIdx.y * kTcRows, n0 = blockIdx.x * BN;
+  const int m0 = blockIdx.y * kTcRows, n0 = blockIdx.x * BN;  // m0: a row of the layout
+  // the sub-key table of this tile: (memory, head, half)
+  const int tab = (d.nmem > 1 ? m0 / d.rstride : 0) * 2 * d.H + hh;
   const int nkb = (d.dh + kTcKBlock - 1) / kTcKBlock;
 
   if (threadIdx.x == 0) {
@@ -180,7 +182,7 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer ----------------
     const int ya = hh * d.qstride + m0;  // row of the query-half tensor
-    const int yb = hh * d.n + n0;        // row of the sub-key tensor
+    const int yb = tab * d.n + n0;       // row of the sub-key tensor
     for (int kb = 0; kb < nkb; ++kb, issued = kb) {
       const int st = kb % kTcStages, round = kb / kTcStages;
       if (!mbar_wait_bounded(&empty[st], (round & 1) ^ 1, s.meta, d.mbar_polls,
@@ -234,21 +236,21 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
   tc_fence_after();
   if (!ready) {
     // zero distances: the selection that follows still sees valid values
-    float *Dh = s.D + (int64_t)hh * d.rows * d.n;
+    float *Dh = s.D + (int64_t)hh * d.drows * d.n;
     for (int r = 0; r < 32; ++r) {
       const int row = m0 + warp * 32 + r;
       for (int c = lane; c < BN; c += 32)
-        if (row < d.rows && n0 + c < d.n) Dh[(int64_t)row * d.n + n0 + c] = 0.f;
+        if (row < d.drows && n0 + c < d.n) Dh[(int64_t)row * d.n + n0 + c] = 0.f;
     }
   }
   if (ready) {
     float *tile = reinterpret_cast<float *>(smem) + warp * 32 * 33;
     const int row0 = m0 + warp * 32;
     const int my_row = row0 + lane;
-    const float my_qn = my_row < d.rows ? s.qn[(int64_t)hh * d.qstride + my_row] : 0.f;
-    const float *kn = s.kn + (int64_t)hh * d.n * kKnChunks;
+    const float my_qn = my_row < d.drows ? s.qn[(int64_t)hh * d.qstride + my_row] : 0.f;
+    const float *kn = s.kn + (int64_t)tab * d.n * kKnChunks;
     const int nkc = (d.dh / 4 + 31) / 32;  // 128-float chunks of a sub-key row
-    float *Dh = s.D + (int64_t)hh * d.rows * d.n;
+    float *Dh = s.D + (int64_t)hh * d.drows * d.n;
 #pragma unroll 1
     for (int c0 = 0; c0 < BN; c0 += 32) {
       float v[32];
@@ -265,7 +267,7 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
       for (int r = 0; r < 32; ++r) {
         const float qn_r = __shfl_sync(FULL, my_qn, r);
         const float dist = qn_r + kn_l - 2.f * tile[r * 33 + lane];
-        if (col_ok && row0 + r < d.rows)
+        if (col_ok && row0 + r < d.drows)
           Dh[(int64_t)(row0 + r) * d.n + col] = dist > 0.f ? dist : 0.f;
       }
       __syncwarp();
@@ -293,7 +295,7 @@ static cudaError_t launch_tc(const Dims &d, const Scratch &s, const TcMaps &maps
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        TcSmem<BN>::kBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((d.n + BN - 1) / BN, (d.rows + kTcRows - 1) / kTcRows, 2 * d.H);
+  dim3 grid((d.n + BN - 1) / BN, (d.drows + kTcRows - 1) / kTcRows, 2 * d.H);
   return launch_k(d.pdl, kernel, grid, 128, TcSmem<BN>::kBytes, st,
                   *reinterpret_cast<const CUtensorMap *>(maps.a_hi),
                   *reinterpret_cast<const CUtensorMap *>(maps.a_lo),
@@ -304,7 +306,7 @@ static cudaError_t launch_tc(const Dims &d, const Scratch &s, const TcMaps &maps
 // Column-tile width: the widest of 128 / 64 / 32 / 16 that still gives at
 // least one CTA per multiprocessor (narrower tiles when the chunk is small).
 cudaError_t launch_score(const Dims &d, const Scratch &s, const TcMaps &maps, cudaStream_t st) {
-  const int64_t base = (int64_t)((d.rows + kTcRows - 1) / kTcRows) * 2 * d.H;
+  const int64_t base = (int64_t)((d.drows + kTcRows - 1) / kTcRows) * 2 * d.H;
   int bn = 128;
   while (bn > 16 && (bn >= 2 * d.n || base * ((d.n + bn - 1) / bn) < d.sm_count)) bn >>= 1;
   if (bn == 16) return launch_tc<16>(d, s, maps, 0, st);
@@ -339,10 +341,10 @@ static cudaError_t encode_2d(void *out, const float *base, uint64_t inner, uint6
 
 // qstride must be a multiple of 128 and K_hi / K_lo must hold 128 rows past
 // the 2*H*n sub-key rows, so that every box lies inside its tensor.
-cudaError_t encode_score_maps(TcMaps *maps, const Scratch &s, int H, int qstride, int n,
-                              int dh) {
+cudaError_t encode_score_maps(TcMaps *maps, const Scratch &s, int H, int nmem, int qstride,
+                              int n, int dh) {
   if (qstride % kTcRows) return cudaErrorInvalidValue;
-  const uint64_t qrows = 2ull * H * qstride, krows = 2ull * H * n + kTcRows;
+  const uint64_t qrows = 2ull * H * qstride, krows = 2ull * H * nmem * n + kTcRows;
   cudaError_t e = encode_2d(maps->a_hi, s.Qs_hi, dh, qrows, kTcRows);
   if (e == cudaSuccess) e = encode_2d(maps->a_lo, s.Qs_lo, dh, qrows, kTcRows);
   for (int v = 0; v < 4 && e == cudaSuccess; ++v) {  // column tiles of 16, 32, 64, 128

@@ -297,8 +297,10 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
   if (!kSelectOnly && blockIdx.x == 0 && threadIdx.x == 0) s.scan_sync[0] += 1ull;
   const bool valid = m < d.M;
   const int row = valid ? m / d.H : 0, h = valid ? m % d.H : 0;
-  const float *D1 = s.D + ((int64_t)(h * 2 + 0) * d.rows + row) * n;
-  const float *D2 = s.D + ((int64_t)(h * 2 + 1) * d.rows + row) * n;
+  const int lrow = lrow_of(d, row), mb = mem_of(d, row);  // layout row, memory
+  const int64_t slot0 = (int64_t)mb * d.N;                // the memory's first value row
+  const float *D1 = s.D + ((int64_t)(h * 2 + 0) * d.drows + lrow) * n;
+  const float *D2 = s.D + ((int64_t)(h * 2 + 1) * d.drows + lrow) * n;
 
   // Global token coordinates of this row (for the optional per-token arrays).
   const int b = row / d.Tc, tl = row % d.Tc;
@@ -333,11 +335,11 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
     float d1_r = 0.f, d2_r = 0.f;
     if (forced) {
       if (lane < k) {
-        int64_t sl = x.force_slots[th * k + lane];
+        int64_t sl = x.force_slots[th * k + lane];  // a slot of the token's memory
         sl = sl < 0 ? 0 : (sl >= d.N ? d.N - 1 : sl);
-        slot_r = (int)sl;
-        i_r = slot_r / n;
-        j_r = slot_r % n;
+        i_r = (int)sl / n;
+        j_r = (int)sl % n;
+        slot_r = (int)(slot0 + sl);
         d1_r = D1[i_r];
         d2_r = D2[j_r];
         s_r = -logf(eps + d1_r) - logf(eps + d2_r);
@@ -399,6 +401,7 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
         d2_r = sm.dist[t][1][bb];
         slot_r = (int)wslot;
       }
+      slot_r += (int)slot0;  // the selection is within the memory; pairs carry the global row
     }
     if (lane < k) {
       sm.fin[t][0][lane] = i_r;
@@ -413,7 +416,7 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
     const float w = ex / z;
     if (kSelectOnly) {
       if (lane < k) {
-        x.rec_slots[th * k + lane] = slot_r;
+        x.rec_slots[th * k + lane] = slot_r - (int)slot0;
         x.rec_w[th * k + lane] = w;
       }
     } else {
@@ -423,7 +426,7 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
         s.pw[p] = w;
         if (!d.readonly) s.pclaim[p] = atomicAdd(&s.bcnt[slot_r >> d.vshift], 1);  // value bucket
         if (x.rec_slots) {
-          x.rec_slots[th * k + lane] = slot_r;
+          x.rec_slots[th * k + lane] = slot_r - (int)slot0;
           x.rec_w[th * k + lane] = w;
         }
       }
@@ -448,7 +451,7 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
     s.esub[e] = sub;
     s.emask[e] = peers;
     s.einv[e] = 1.f / (eps + dist);
-    s.eclaim[e] = atomicAdd(&s.bcnt[d.NBv + (h * 2 + half) * n + sub], 1);
+    s.eclaim[e] = atomicAdd(&s.bcnt[d.NBv + ((mb * d.H + h) * 2 + half) * n + sub], 1);
   }
   // unused entry slots of this half are marked -1
   if (lane >= __popc(lb) && lane < k) s.esub[((int64_t)m * 2 + half) * k + lane] = -1;

@@ -47,6 +47,8 @@ def load_library():
     i64p = ctypes.POINTER(ctypes.c_int64)
     L.fwpkm_last_error.restype = ctypes.c_char_p
     L.fwpkm_state_init.argtypes = [i64, i32, i32, i32, i32, i32, ctypes.POINTER(_vp)]
+    L.fwpkm_state_init_batched.argtypes = [i64, i32, i32, i32, i32, i32, i32,
+                                           ctypes.POINTER(_vp)]
     L.fwpkm_state_free.argtypes = [_vp]
     L.fwpkm_state_free.restype = None
     L.fwpkm_state_set_eps.argtypes = [_vp, f32]
@@ -70,7 +72,8 @@ def load_library():
     L.fwpkm_state_set_options.argtypes = [_vp, ctypes.c_uint]
     L.fwpkm_inject_alloc_failures.argtypes = [i32]
     L.fwpkm_inject_alloc_failures.restype = None
-    for name in ("fwpkm_state_init", "fwpkm_state_set_eps", "fwpkm_step", "fwpkm_step_host",
+    for name in ("fwpkm_state_init", "fwpkm_state_init_batched", "fwpkm_state_set_eps",
+                 "fwpkm_step", "fwpkm_step_host",
                  "fwpkm_step_ex", "fwpkm_step_host_ex",
                  "fwpkm_state_get", "fwpkm_state_set", "fwpkm_record_selection",
                  "fwpkm_force_selection", "fwpkm_set_profiling", "fwpkm_profile_read",
@@ -127,16 +130,23 @@ def _dtype_code(t) -> int:
 class FwPKMState:
     """One fast-weight product-key memory (sub-key tables + value table).
 
-    Mirrors fwpkm_state_init / step / get / set of include/fwpkm.h.
+    Mirrors fwpkm_state_init / step / get / set of include/fwpkm.h.  With
+    ``memories`` > 1 the state holds one memory per sequence
+    (fwpkm_state_init_batched): a step's B must equal ``memories``.
     """
 
     def __init__(self, N: int, dq: int, dv: int, topk: int, chunk: int, heads: int = 1,
-                 eps: float = 1e-3):
+                 eps: float = 1e-3, memories: int = 1):
         L = load_library()
         h = _vp()
-        _check(L.fwpkm_state_init(N, dq, dv, topk, chunk, heads, ctypes.byref(h)))
+        if memories == 1:
+            _check(L.fwpkm_state_init(N, dq, dv, topk, chunk, heads, ctypes.byref(h)))
+        else:
+            _check(L.fwpkm_state_init_batched(N, dq, dv, topk, chunk, heads, memories,
+                                              ctypes.byref(h)))
         self._h = h
         self.N, self.dq, self.dv, self.topk, self.chunk, self.heads = N, dq, dv, topk, chunk, heads
+        self.memories = memories
         self.n = int(round(N ** 0.5))
         if eps != 1e-3:
             _check(L.fwpkm_state_set_eps(h, eps))
@@ -161,11 +171,12 @@ class FwPKMState:
     def get_tables(self, subkeys=None, values=None, stream=None):
         """Copy the tables into the given buffers (allocates CUDA tensors if None)."""
         import torch
+        lead = (self.memories,) if self.memories > 1 else ()
         if subkeys is None:
-            subkeys = torch.empty((self.heads, 2, self.n, self.dq // 2), dtype=torch.float32,
-                                  device="cuda")
+            subkeys = torch.empty(lead + (self.heads, 2, self.n, self.dq // 2),
+                                  dtype=torch.float32, device="cuda")
         if values is None:
-            values = torch.empty((self.N, self.dv), dtype=torch.float32, device="cuda")
+            values = torch.empty(lead + (self.N, self.dv), dtype=torch.float32, device="cuda")
         _check(load_library().fwpkm_state_get(self._h, _ptr(subkeys), _ptr(values),
                                               _stream(stream)))
         return subkeys, values

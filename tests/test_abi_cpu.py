@@ -65,6 +65,7 @@ def test_state_init_rejects_bad_shapes(lib, N, dq, dv, topk, chunk, heads):
 
 def test_null_arguments_are_rejected(lib):
     assert lib.fwpkm_state_init(1024, 64, 64, 4, 32, 1, None) == fwpkm.FWPKM_EINVAL
+    assert lib.fwpkm_state_init_batched(1024, 64, 64, 4, 32, 1, 2, None) == fwpkm.FWPKM_EINVAL
     assert lib.fwpkm_step(None, 1, 1, None, 0, None, 0, None, 1.0, 0.0, None, None) == \
         fwpkm.FWPKM_EINVAL
     assert lib.fwpkm_state_get(None, None, None, None) == fwpkm.FWPKM_EINVAL
@@ -123,3 +124,13 @@ def test_injected_allocation_failure_is_enomem(lib):
     assert rc == fwpkm.FWPKM_ENOMEM
     assert h.value is None
     assert "allocation" in lib.fwpkm_last_error().decode()
+
+
+@pytest.mark.parametrize("memories", [0, -1, 2048])
+def test_batched_init_rejects_bad_memory_counts(lib, memories):
+    """memories >= 1, and every value and sub-key row of all memories must
+    have a 32-bit group id (2048 memories of 1M slots do not)."""
+    h = ctypes.c_void_p()
+    rc = lib.fwpkm_state_init_batched(1024 * 1024, 64, 64, 4, 32, 1, memories, ctypes.byref(h))
+    assert rc == fwpkm.FWPKM_ESHAPE
+    assert h.value is None
