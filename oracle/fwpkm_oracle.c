@@ -69,6 +69,8 @@ int orc_num_threads(void) {
 /* Scoring: IDW score of one query half against one sub-key table.  [GS-2]   */
 /* s[i] = -log(eps + sum_d (q_d - K[i][d])^2), direct-difference form.       */
 /* dist[i] (optional) receives the squared distance itself.                  */
+/* (orc_half_scores_dot, below, is the dot-product score the IDW one is      */
+/* chosen over.)                                                            */
 /* ------------------------------------------------------------------------ */
 void orc_half_scores(const double *q, const double *K, int n, int dh, double eps,
                      double *s, double *dist) {
@@ -80,6 +82,16 @@ void orc_half_scores(const double *q, const double *K, int n, int dh, double eps
     }
     s[i] = -log(eps + d);
     if (dist) dist[i] = d;
+  }
+}
+
+/* The other scoring the pages set the IDW score against [GS-2 Key Technical */
+/* Choices]: the plain dot product s[i] = sum_d q_d K[i][d].                 */
+void orc_half_scores_dot(const double *q, const double *K, int n, int dh, double *s) {
+  for (int i = 0; i < n; ++i) {
+    double d = 0.0;
+    for (int c = 0; c < dh; ++c) d += q[c] * K[(int64_t)i * dh + c];
+    s[i] = d;
   }
 }
 
@@ -199,6 +211,7 @@ enum {
   ORC_HEADS_SUM = 1, /* head readouts summed, not averaged                   */
   ORC_AGG_COUNT = 2, /* value-row gradient divided by the row's access count */
   ORC_AGG_SUM = 4,   /* value-row gradient not divided (plain sum)           */
+  ORC_SCORE_DOT = 8, /* sub-key score q . K instead of -log(eps + |q - K|^2)  */
 };
 
 typedef struct {
@@ -302,6 +315,10 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
         const double *K2 = K + ((int64_t)h * 2 + 1) * n * dh;
         orc_half_scores(q, K1, n, dh, dm->eps, s1, dd1);      /* first half of q  */
         orc_half_scores(q + dh, K2, n, dh, dm->eps, s2, dd2); /* second half of q */
+        if (dm->variant & ORC_SCORE_DOT) { /* the dot-product score instead      */
+          orc_half_scores_dot(q, K1, n, dh, s1);
+          orc_half_scores_dot(q + dh, K2, n, dh, s2);
+        }
         orc_pk_select(s1, s2, n, k, sl, sc, a_, b_);
         orc_softmax(sc, k, w + m * k);
         for (int r = 0; r < k; ++r) {
@@ -414,11 +431,19 @@ static int orc_chunk(const dims_t *dm, double *K, double *V, int B, int T, int t
         double *G2 = GK + (((int64_t)h * 2 + 1) * n + j) * dh;
         const double *K1 = K + (((int64_t)h * 2 + 0) * n + i) * dh;
         const double *K2 = K + (((int64_t)h * 2 + 1) * n + j) * dh;
-        double c1 = dLds * 2.0 / (dm->eps + d1[m * k + r]);
-        double c2 = dLds * 2.0 / (dm->eps + d2[m * k + r]);
-        for (int c = 0; c < dh; ++c) {
-          G1[c] += c1 * (q[c] - K1[c]);
-          G2[c] += c2 * (q[dh + c] - K2[c]);
+        if (dm->variant & ORC_SCORE_DOT) {
+          /* ds/dK_h,i = q_h for the dot-product score */
+          for (int c = 0; c < dh; ++c) {
+            G1[c] += dLds * q[c];
+            G2[c] += dLds * q[dh + c];
+          }
+        } else {
+          double c1 = dLds * 2.0 / (dm->eps + d1[m * k + r]);
+          double c2 = dLds * 2.0 / (dm->eps + d2[m * k + r]);
+          for (int c = 0; c < dh; ++c) {
+            G1[c] += c1 * (q[c] - K1[c]);
+            G2[c] += c2 * (q[dh + c] - K2[c]);
+          }
         }
         ktouched[((int64_t)h * 2 + 0) * n + i] = 1;
         ktouched[((int64_t)h * 2 + 1) * n + j] = 1;
@@ -566,6 +591,14 @@ double orc_chunk_loss(int64_t N, int n, int dq, int dv, int topk, int heads, dou
             db += (q[dh + c] - K2[c]) * (q[dh + c] - K2[c]);
           }
           s[r] = -log(eps + da) - log(eps + db);
+          if (variant & ORC_SCORE_DOT) {
+            double pa = 0.0, pb = 0.0;
+            for (int c = 0; c < dh; ++c) {
+              pa += q[c] * K1[c];
+              pb += q[dh + c] * K2[c];
+            }
+            s[r] = pa + pb;
+          }
         }
         orc_softmax(s, k, w);
         for (int r = 0; r < k; ++r) {

@@ -45,6 +45,7 @@ def lib():
         i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
         L.orc_num_threads.restype = i32
         L.orc_half_scores.argtypes = [_dp, _dp, i32, i32, f64, _dp, _dp]
+        L.orc_half_scores_dot.argtypes = [_dp, _dp, i32, i32, _dp]
         L.orc_topk.argtypes = [_dp, i32, i32, _ip, _dp]
         L.orc_pk_select.argtypes = [_dp, _dp, i32, i32, _ip, _dp, _ip, _ip]
         L.orc_brute_select.argtypes = [_dp, _dp, i32, i32, _ip, _dp]
@@ -94,6 +95,15 @@ def half_scores(q, K, eps):
     d = np.empty(n)
     lib().orc_half_scores(_p(q), _p(K), n, dh, eps, _p(s), _p(d))
     return s, d
+
+
+def half_scores_dot(q, K):
+    """The dot-product score q . K of one query half against a sub-key table."""
+    q, K = _f64(q), _f64(K)
+    n, dh = K.shape
+    s = np.empty(n)
+    lib().orc_half_scores_dot(_p(q), _p(K), n, dh, _p(s))
+    return s
 
 
 def topk(s, k):
@@ -150,6 +160,7 @@ def lookahead_targets(Vt, weight):
 # a value row's gradient is divided by.
 HEADS = {"mean": 0, "sum": 1}
 AGG = {"weight": 0, "count": 2, "sum": 4}
+SCORE = {"idw": 0, "dot": 8}
 
 
 class State:
@@ -158,10 +169,11 @@ class State:
     ``heads``: "mean" (head readouts averaged, the default reading) or "sum".
     ``agg``: a value row's gradient divided by its row contribution C_i =
     sum of w/H ("weight", the default), by its access count ("count"), or not
-    divided ("sum")."""
+    divided ("sum").  ``score``: the sub-key score, "idw" (-log(eps + |q -
+    K|^2), the default) or "dot" (q . K)."""
 
     def __init__(self, subkeys, values, *, topk: int, chunk: int, eps: float = 1e-3,
-                 heads: str = "mean", agg: str = "weight"):
+                 heads: str = "mean", agg: str = "weight", score: str = "idw"):
         self.K = _f64(subkeys).copy()
         self.V = _f64(values).copy()
         self.H, two, self.n, self.dh = self.K.shape
@@ -169,7 +181,7 @@ class State:
         self.N, self.dv = self.V.shape
         self.dq = 2 * self.dh
         self.topk, self.chunk, self.eps = topk, chunk, eps
-        self.variant = HEADS[heads] | AGG[agg]
+        self.variant = HEADS[heads] | AGG[agg] | SCORE[score]
 
     def copy(self) -> "State":
         s = State.__new__(State)

@@ -143,3 +143,32 @@ def test_hand_step_summed_heads(hs):
     for key, row in part["subkeys_after"].items():
         K[row_key(key)] = arr(row)
     np.testing.assert_allclose(st.K, K, rtol=RTOL, atol=1e-15)
+
+
+def test_hand_step_dot_product_score(hs):
+    """The dot-product sub-key score: selection (ties by slot), gap, read,
+    loss, dL/dK (ds/dK = q) and both updated tables, as worked by hand."""
+    part = hs.raw.get("dot_score")
+    if part is None:
+        pytest.skip("this example has no dot-product part")
+    Q = arr(part["Q"])
+    st = oracle.State(hs.K, hs.V, topk=hs.topk, chunk=hs.chunk, eps=hs.eps, score="dot")
+    gr = st.chunk_grads(Q, hs.Vt, hs.gate, 0.0, 0, hs.chunk)
+    assert gr["loss"] == pytest.approx(sum(frac(x) for x in part["loss"]), rel=RTOL)
+    dK = np.zeros_like(hs.K)
+    for key, row in part["dLdK"].items():
+        dK[row_key(key)] = arr(row)
+    np.testing.assert_allclose(gr["dLdK"], dK, rtol=RTOL, atol=1e-15)
+    res = st.step(Q, hs.Vt, hs.gate, hs.eta, 0.0, want_sel=True, want_gap=True)
+    assert np.array_equal(res["sel_slot"], np.array(part["sel_slot"]))
+    np.testing.assert_allclose(res["sel_w"], 0.5, rtol=RTOL)
+    np.testing.assert_allclose(res["gap"], arr(part["gap"]), rtol=RTOL, atol=1e-15)
+    np.testing.assert_allclose(res["out"], arr(part["out"]), rtol=RTOL)
+    V = hs.V.copy()
+    for r, row in part["values_after"].items():
+        V[int(r)] = arr(row)
+    np.testing.assert_allclose(st.V, V, rtol=RTOL, atol=0)
+    K = hs.K.copy()
+    for key, row in part["subkeys_after"].items():
+        K[row_key(key)] = arr(row)
+    np.testing.assert_allclose(st.K, K, rtol=RTOL, atol=1e-15)

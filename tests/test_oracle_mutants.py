@@ -39,6 +39,8 @@ MUTANTS = {
     "summed_heads_still_averaged": ("(dm->variant & ORC_HEADS_SUM) ? 1.0 : (double)H;",
                                     "(double)H;"),
     "keys_not_updated": ("if (ktouched[row])", "if (0)"),
+    "dot_key_grad_of_the_first_half": ("G2[c] += dLds * q[dh + c];", "G2[c] += dLds * q[c];"),
+    "dot_score_ignored_in_selection": ("orc_half_scores_dot(q + dh, K2, n, dh, s2);", ""),
 }
 
 

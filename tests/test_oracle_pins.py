@@ -135,14 +135,17 @@ def test_gap_is_kth_minus_next(oracle):
     (0.0, 1, "one", False, "mean"), (0.0, 2, "rand", False, "mean"),
     (0.3, 2, "rand", False, "mean"), (1.5, 1, "rand", False, "mean"),
     (0.3, 2, "rand", True, "mean"), (0.0, 3, "rand", False, "sum"),
-    (0.4, 2, "rand", True, "sum")])
+    (0.4, 2, "rand", True, "sum"), (0.0, 2, "rand", False, "dot"),
+    (0.5, 1, "rand", True, "dot")])
 def test_gradients_match_finite_differences(oracle, lam, H, gate, own_weight, heads):
     rng = np.random.default_rng(int(lam * 10) + H + (7 if own_weight else 0))
     B, T, dq, n, dv, k = 2, 6, 8, 6, 5, 3
     K, V, Q, Vt, g = tiny_case(rng, B=B, T=T, H=H, dq=dq, n=n, dv=dv, k=k, gate=gate)
     # a per-token MSE weight of its own (some tokens 0), else the gate
     om = rng.uniform(0.0, 1.5, (B, T)) * (rng.random((B, T)) > 0.3) if own_weight else None
-    st = make_state(oracle, K, V, k, T, heads=heads)
+    # "dot": heads averaged, the dot-product sub-key score
+    opts = {"score": "dot"} if heads == "dot" else {"heads": heads}
+    st = make_state(oracle, K, V, k, T, **opts)
     gr = st.chunk_grads(Q, Vt, g, lam, 0, T, omega=om)
     slots = gr["sel_slot"]
     L0 = st.chunk_loss(Q, Vt, g, lam, 0, T, slots, omega=om)
@@ -448,3 +451,25 @@ def test_summed_duplicated_heads_read_twice_one_head(oracle):
     b = make_state(oracle, np.concatenate([K1, K1], axis=0), V, 3, 3, heads="sum")
     rb = b.step(np.concatenate([Q1, Q1], axis=2), Vt, g, 0.0, 0.0)
     assert np.allclose(rb["out"], 2.0 * ra["out"], rtol=1e-13, atol=1e-15)
+
+
+def test_dot_product_selection_is_the_brute_force_top_k(oracle):
+    """With the dot-product score, the product-key selection equals the top-k
+    over all N slots of q1.K1[i] + q2.K2[j], computed here with numpy (ties
+    by slot), and the weights are their softmax."""
+    rng = np.random.default_rng(23)
+    for n, k in ((6, 3), (9, 5), (12, 12)):
+        K, V, Q, Vt, g = tiny_case(rng, B=1, T=5, H=1, dq=8, n=n, dv=3, k=k)
+        st = make_state(oracle, K, V, k, 5, score="dot")
+        res = st.step(Q, Vt, g, 0.0, 0.0, want_sel=True)
+        for t in range(5):
+            s1 = K[0, 0] @ Q[0, t, :4]
+            s2 = K[0, 1] @ Q[0, t, 4:]
+            full = (s1[:, None] + s2[None, :]).ravel()
+            order = np.lexsort((np.arange(n * n), -full))[:k]
+            assert np.array_equal(np.sort(res["sel_slot"][0, t, 0]), np.sort(order))
+            w = np.exp(full[order] - full[order].max())
+            got = dict(zip(res["sel_slot"][0, t, 0], res["sel_w"][0, t, 0]))
+            for sl, wi in zip(order, w / w.sum()):
+                assert np.isclose(got[sl], wi, rtol=1e-12)
+        assert np.allclose(oracle.half_scores_dot(Q[0, 0, :4], K[0, 0]), K[0, 0] @ Q[0, 0, :4])
