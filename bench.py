@@ -53,6 +53,8 @@ def describe(wl) -> str:
         s += " lookahead (q_t written towards v_t+1)"
     if wl.per_sequence:
         s += f" one memory per sequence ({wl.B} memories)"
+    if wl.score != "idw":
+        s += f" score={wl.score}"
     return s
 
 
@@ -192,7 +194,7 @@ class OracleSampler:
         # one state shared by the sequences, or one per sequence (all starting
         # from the workload's tables)
         self.state = [orc.State(inp.subkeys, inp.values, topk=wl.topk, chunk=wl.chunk,
-                                eps=wl.eps)
+                                eps=wl.eps, heads=wl.heads_mode, agg=wl.agg, score=wl.score)
                       for _ in range(wl.B if wl.per_sequence else 1)]
 
     def sample(self, budget_s: float):
@@ -371,6 +373,7 @@ def run_gpu(args, wl):
             segs.append((dq_, dv_, dg_))
     outs = [torch.empty((wl.B, wl.T, wl.dv), dtype=torch.float32, device=dev) for _ in segs]
     st = FwPKMState(wl.N, wl.dq, wl.dv, wl.topk, wl.chunk, wl.heads, eps=wl.eps, memories=mem)
+    st.set_options(heads=wl.heads_mode, agg=wl.agg, score=wl.score)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -561,6 +564,10 @@ def main():
     ap.add_argument("--per-sequence", action="store_true",
                     help="one memory per sequence: the B sequences of a call each read and "
                          "write their own memory, in the same launches")
+    ap.add_argument("--eta", type=float, default=None,
+                    help="learning rate of the update (default: the workload's)")
+    ap.add_argument("--score", choices=["idw", "dot"], default="idw",
+                    help="sub-key score: -log(eps + |q - K|^2) (default) or the dot product")
     ap.add_argument("--lookahead", action="store_true",
                     help="write query t towards the target of token t+1 (each call's last "
                          "token has weight 0)")
@@ -574,6 +581,10 @@ def main():
         wl = wl.replace(lookahead=True)
     if args.per_sequence:
         wl = wl.replace(per_sequence=True)
+    if args.score != "idw":
+        wl = wl.replace(score=args.score)
+    if args.eta is not None:
+        wl = wl.replace(eta=args.eta)
     if args.impl == "reference":
         run_reference(args, wl)
     else:

@@ -108,10 +108,12 @@ fwpkm_status fwpkm_state_set_eps(fwpkm_state *s, float eps);
 #define FWPKM_HEADS_SUM 1u /* head readouts summed, not averaged                   */
 #define FWPKM_AGG_COUNT 2u /* value-row gradient divided by the row's access count */
 #define FWPKM_AGG_SUM 4u   /* value-row gradient not divided                       */
+#define FWPKM_SCORE_DOT 8u /* sub-key score q_half . K_row instead of the IDW one  */
 
 /*
- * fwpkm_state_set_options -- other readings of two points the pages leave
- * open, for the steps that follow (0 restores the defaults).
+ * fwpkm_state_set_options -- other readings of points the pages leave open,
+ * and the score they name as the alternative, for the steps and selections
+ * that follow (0 restores the defaults).
  *   [PYPI multi-head variant]  By default the heads' readouts are averaged,
  *     yhat = (1/H) sum_h sum_r w V[slot]; FWPKM_HEADS_SUM sums them, and the
  *     1/H of the gradients and of C_i goes with it.
@@ -120,6 +122,11 @@ fwpkm_status fwpkm_state_set_eps(fwpkm_state *s, float eps);
  *     eta G_i / C_i, C_i = sum of its pairs' w/H; FWPKM_AGG_COUNT divides by
  *     the number of pairs on the row instead, FWPKM_AGG_SUM not at all.
  *     The two exclude each other (FWPKM_EINVAL).
+ *   [GS-2 Key Technical Choices]  By default a sub-key row scores
+ *     -log(eps + ||q_half - K_row||^2) (IDW); FWPKM_SCORE_DOT scores the
+ *     dot product q_half . K_row instead, the alternative the page names.
+ *     The selection then takes the largest dot products, and a sub-key row
+ *     moves by eta sum(dL/ds q_half) (ds/dK = q_half); eps is unused.
  * The sub-keys always take the raw summed gradient.
  */
 fwpkm_status fwpkm_state_set_options(fwpkm_state *s, unsigned options);

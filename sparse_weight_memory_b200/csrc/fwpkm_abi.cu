@@ -105,7 +105,7 @@ struct fwpkm_state {
   // bounds of the device-side waits (fwpkm_set_wait_limits)
   long long mbar_polls = kDefaultMbarPolls, scan_polls = kDefaultScanPolls;
   // readings (fwpkm_state_set_options)
-  int heads_sum = 0, agg = AGG_WEIGHT;
+  int heads_sum = 0, agg = AGG_WEIGHT, score_dot = 0;
   float *K = nullptr;  // [nmem][H][2][n][dh]
   float *V = nullptr;  // [nmem][N][dv]
   // scratch arena
@@ -337,6 +337,7 @@ Dims chunk_dims(const fwpkm_state *st, int B, int T, int c, float eta, float lam
   d.scan_polls = st->scan_polls;
   d.heads_sum = st->heads_sum;
   d.agg = st->agg;
+  d.score_dot = st->score_dot;
   return d;
 }
 
@@ -507,6 +508,7 @@ bool state_view(const fwpkm_state *st, StateView *v) {
   v->eps = st->eps;
   v->K = st->K;
   v->mbar_polls = st->mbar_polls;
+  v->score_dot = st->score_dot;
   return true;
 }
 void set_last_error(const char *msg) { g_last_error = msg; }
@@ -633,11 +635,12 @@ void fwpkm_inject_alloc_failures(int count) { g_fail_allocs.store(count > 0 ? co
 
 fwpkm_status fwpkm_state_set_options(fwpkm_state *st, unsigned options) {
   if (!st) return fail(FWPKM_EINVAL, "set_options: state is NULL");
-  const unsigned known = FWPKM_HEADS_SUM | FWPKM_AGG_COUNT | FWPKM_AGG_SUM;
+  const unsigned known = FWPKM_HEADS_SUM | FWPKM_AGG_COUNT | FWPKM_AGG_SUM | FWPKM_SCORE_DOT;
   if (options & ~known) return fail(FWPKM_EINVAL, "set_options: unknown bits 0x%x", options);
   if ((options & FWPKM_AGG_COUNT) && (options & FWPKM_AGG_SUM))
     return fail(FWPKM_EINVAL, "set_options: FWPKM_AGG_COUNT and FWPKM_AGG_SUM exclude each other");
   st->heads_sum = (options & FWPKM_HEADS_SUM) ? 1 : 0;
+  st->score_dot = (options & FWPKM_SCORE_DOT) ? 1 : 0;
   st->agg = (options & FWPKM_AGG_COUNT) ? AGG_COUNT : ((options & FWPKM_AGG_SUM) ? AGG_SUM : AGG_WEIGHT);
   clear_graphs(st);  // the options are kernel parameters of the captured launches
   return FWPKM_OK;

@@ -90,6 +90,7 @@ struct Dims {
   int heads_sum;         // head readouts summed instead of averaged
   int readonly;          // eta = 0: the read alone (no claims, entries, records, gradients)
   int agg;               // divisor of a value row's gradient (AGG_*)
+  int score_dot;         // sub-key score q . K (D holds -q.K) instead of the IDW one
 };
 // Divisor of a value row's gradient: its row contribution C_i = sum of w/H
 // (the sum of its members' c0), its access count (every member's c0 is 1), or
@@ -414,6 +415,7 @@ struct StateView {
   float eps;
   const float *K;
   long long mbar_polls;
+  int score_dot;
 };
 bool state_view(const struct ::fwpkm_state *st, StateView *v);
 // Records `msg` as the calling thread's last error (fwpkm_last_error).

@@ -181,6 +181,7 @@ extern "C" fwpkm_status fwpkm_select_noalloc(fwpkm_state *state, int B, int T, c
     d.sm_count = v.sm_count;
     d.pdl = 1;
     d.eps = v.eps;
+    d.score_dot = v.score_dot;
     d.mbar_polls = v.mbar_polls;
     d.scan_polls = kDefaultScanPolls;
     d.q_tf32_exact = q_dtype == FWPKM_BF16 ? 1 : 0;

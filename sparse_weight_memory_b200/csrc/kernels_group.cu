@@ -665,13 +665,17 @@ __device__ __forceinline__ void add4(float4 &a, const float4 &x) {
 
 // New value of one float4 of a target row from the group's complete sums.
 //   value row : v - (eta / C) * G          (C = sum of w/H)
-//   sub-key   : k - 2 eta (G - A k)        (A = sum of alpha)
+//   sub-key   : k - 2 eta (G - A k)        (A = sum of alpha; IDW score)
+//               k - eta G                  (dot-product score: ds/dK = q)
 __device__ __forceinline__ float4 updated(const Dims &d, bool value, const float4 &t,
                                           const float4 &g, float c0) {
   if (value) {
     const float sc = d.agg == AGG_SUM ? d.eta : d.eta / c0;
     return make_float4(t.x - sc * g.x, t.y - sc * g.y, t.z - sc * g.z, t.w - sc * g.w);
   }
+  if (d.score_dot)
+    return make_float4(t.x - d.eta * g.x, t.y - d.eta * g.y, t.z - d.eta * g.z,
+                       t.w - d.eta * g.w);
   const float te = 2.f * d.eta;
   return make_float4(t.x - te * (g.x - c0 * t.x), t.y - te * (g.y - c0 * t.y),
                      t.z - te * (g.z - c0 * t.z), t.w - te * (g.w - c0 * t.w));

@@ -7,6 +7,8 @@
 // (kind::tf32, fp32 accumulate in tensor memory) on operand tiles brought in
 // by TMA, and writes
 //     D[h][half][row][i] = |q|^2 + |K_i|^2 - 2 q.K_i      (clamped at 0)
+// or, with the dot-product score, D = -q.K_i (the selection takes the
+// smallest D either way).
 //
 // Precision: three TF32 products, hi*hi + hi*lo + lo*hi, where x = hi + lo and
 // hi is x rounded to TF32 (the prep writes both parts, and the update rewrites
@@ -247,7 +249,9 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
     float *tile = reinterpret_cast<float *>(smem) + warp * 32 * 33;
     const int row0 = m0 + warp * 32;
     const int my_row = row0 + lane;
-    const float my_qn = my_row < d.drows ? s.qn[(int64_t)hh * d.qstride + my_row] : 0.f;
+    const bool dot = d.score_dot != 0;
+    const float my_qn =
+        !dot && my_row < d.drows ? s.qn[(int64_t)hh * d.qstride + my_row] : 0.f;
     const float *kn = s.kn + (int64_t)tab * d.n * kKnChunks;
     const int nkc = (d.dh / 4 + 31) / 32;  // 128-float chunks of a sub-key row
     float *Dh = s.D + (int64_t)hh * d.drows * d.n;
@@ -261,14 +265,15 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
       const int col = n0 + c0 + lane;
       const bool col_ok = col < d.n && c0 + lane < BN;
       float kn_l = 0.f;  // |K_col|^2: the chunk norms in chunk order
-      if (col_ok)
+      if (col_ok && !dot)
         for (int ch = 0; ch < nkc; ++ch) kn_l += kn[(int64_t)col * kKnChunks + ch];
 #pragma unroll 4
       for (int r = 0; r < 32; ++r) {
         const float qn_r = __shfl_sync(FULL, my_qn, r);
         const float dist = qn_r + kn_l - 2.f * tile[r * 33 + lane];
         if (col_ok && row0 + r < d.drows)
-          Dh[(int64_t)(row0 + r) * d.n + col] = dist > 0.f ? dist : 0.f;
+          Dh[(int64_t)(row0 + r) * d.n + col] =
+              dot ? -tile[r * 33 + lane] : (dist > 0.f ? dist : 0.f);
       }
       __syncwarp();
     }

@@ -129,15 +129,20 @@ __device__ __forceinline__ void compact_selected(uint32_t sel, const uint32_t (&
   }
 }
 
-// Order-preserving map of a float to an unsigned key (larger float, larger key).
+// Order-preserving map of a float to an unsigned key (larger float, larger
+// key), and its inverse on the bits.
 __device__ __forceinline__ uint32_t float_order(float x) {
   const uint32_t u = __float_as_uint(x);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+__device__ __forceinline__ uint32_t float_unorder(uint32_t u) {
+  return (u & 0x80000000u) ? (u & 0x7fffffffu) : ~u;
+}
 
 // Top-k smallest distances of one half row drow[0..n) (n <= 32*NV), ties by
 // index.  Lane r < k returns one winner (distance, index); order unspecified.
-// wbuf holds 64 entries.
+// wbuf holds 64 entries.  `sgn`: the values may be negative (the negated dot
+// products of the dot-product score), so they are keyed by float_order.
 //
 // With 4 or more entries per lane the search is narrowed first: every lane
 // offers its two smallest keys, and the k-th smallest t0 of those 64 is at
@@ -147,7 +152,7 @@ __device__ __forceinline__ uint32_t float_order(float x) {
 // (heavy ties) the whole row is searched instead.  Either way the result is
 // the exact top-k under (key asc, index asc).
 template <int NV>
-__device__ __forceinline__ void half_topk(const float *__restrict__ drow, int n, int k,
+__device__ __forceinline__ void half_topk(const float *__restrict__ drow, int n, int k, bool sgn,
                                           float &d_out, int &i_out, uint2 *wbuf) {
   const int lane = threadIdx.x & 31;
   uint32_t key[NV], idx[NV];
@@ -156,7 +161,9 @@ __device__ __forceinline__ void half_topk(const float *__restrict__ drow, int n,
     const int i = lane + 32 * v;
     // d >= 0: the bit order is the value order; a used entry never takes the
     // unused marker 0xffffffff, whatever the distance's bits
-    key[v] = i < n ? min(__float_as_uint(drow[i]), 0xfffffffeu) : 0xffffffffu;
+    const float dv = i < n ? drow[i] : 0.f;
+    key[v] = i < n ? min(sgn ? float_order(dv) : __float_as_uint(dv), 0xfffffffeu)
+                   : 0xffffffffu;
     idx[v] = (uint32_t)i;
   }
   uint32_t kk, ii;
@@ -203,14 +210,14 @@ __device__ __forceinline__ void half_topk(const float *__restrict__ drow, int n,
       __syncwarp();
       const uint32_t sel = warp_select_smallest<2>(ck, ci, k);
       compact_selected<2>(sel, ck, ci, wbuf, kk, ii, v_out, src);
-      d_out = __uint_as_float(kk);
+      d_out = __uint_as_float(sgn ? float_unorder(kk) : kk);
       i_out = (int)ii;
       return;
     }
   }
   const uint32_t sel = warp_select_smallest<NV>(key, idx, k);
   compact_selected<NV>(sel, key, idx, wbuf, kk, ii, v_out, src);
-  d_out = __uint_as_float(kk);
+  d_out = __uint_as_float(sgn ? float_unorder(kk) : kk);
   i_out = (int)ii;
 }
 
@@ -279,6 +286,7 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
   const int m = blockIdx.x * kTopkHeads + t;  // token-head m = row*H + h
   const int k = d.k, n = d.n;
   const float eps = d.eps;
+  const bool dot = d.score_dot != 0;  // D = -q.K: the score is -D, ds/dK = q
   // the staircase for this k (warp 0, before the halves are selected)
   if (wib == 0) {
     const int len = lane < k ? min(k, k / (lane + 1)) : 0;
@@ -311,8 +319,8 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
   if (valid && !forced) {
     float dw;
     int iw;
-    half_topk<NV>(half == 0 ? D1 : D2, n, k, dw, iw, sm.wbuf[wib]);
-    const float sw = -logf(eps + dw);
+    half_topk<NV>(half == 0 ? D1 : D2, n, k, dot, dw, iw, sm.wbuf[wib]);
+    const float sw = dot ? -dw : -logf(eps + dw);
     const uint64_t key =
         lane < k ? ((uint64_t)float_order(-sw) << 32) | (uint32_t)iw : ~0ull;
     int src;
@@ -342,7 +350,7 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
         slot_r = (int)(slot0 + sl);
         d1_r = D1[i_r];
         d2_r = D2[j_r];
-        s_r = -logf(eps + d1_r) - logf(eps + d2_r);
+        s_r = dot ? -d1_r - d2_r : -logf(eps + d1_r) - logf(eps + d2_r);
       }
     } else {
       const float *S1 = sm.s[t][0], *S2 = sm.s[t][1];
@@ -450,7 +458,7 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
     const int64_t e = ((int64_t)m * 2 + half) * k + idx;
     s.esub[e] = sub;
     s.emask[e] = peers;
-    s.einv[e] = 1.f / (eps + dist);
+    s.einv[e] = dot ? 1.f : 1.f / (eps + dist);
     s.eclaim[e] = atomicAdd(&s.bcnt[d.NBv + ((mb * d.H + h) * 2 + half) * n + sub], 1);
   }
   // unused entry slots of this half are marked -1

@@ -20,7 +20,7 @@ FWPKM_OK, FWPKM_EINVAL, FWPKM_ESHAPE, FWPKM_ENOMEM, FWPKM_ECUDA, FWPKM_EUNSUPPOR
     0, -1, -2, -3, -4, -5)
 FWPKM_F32, FWPKM_BF16 = 0, 1
 FWPKM_LOOKAHEAD = 1
-FWPKM_HEADS_SUM, FWPKM_AGG_COUNT, FWPKM_AGG_SUM = 1, 2, 4
+FWPKM_HEADS_SUM, FWPKM_AGG_COUNT, FWPKM_AGG_SUM, FWPKM_SCORE_DOT = 1, 2, 4, 8
 STATUS_NAMES = {0: "OK", -1: "EINVAL", -2: "ESHAPE", -3: "ENOMEM", -4: "ECUDA",
                 -5: "EUNSUPPORTED"}
 
@@ -239,11 +239,13 @@ class FwPKMState:
                                                    _stream(stream)))
         return slots, weights
 
-    def set_options(self, heads: str = "mean", agg: str = "weight"):
+    def set_options(self, heads: str = "mean", agg: str = "weight", score: str = "idw"):
         """Readings of the step: ``heads`` "mean" or "sum"; ``agg`` (divisor
-        of a value row's gradient) "weight", "count" or "sum"."""
+        of a value row's gradient) "weight", "count" or "sum"; ``score``
+        (sub-key score) "idw" or "dot"."""
         opts = {"mean": 0, "sum": FWPKM_HEADS_SUM}[heads] | \
-            {"weight": 0, "count": FWPKM_AGG_COUNT, "sum": FWPKM_AGG_SUM}[agg]
+            {"weight": 0, "count": FWPKM_AGG_COUNT, "sum": FWPKM_AGG_SUM}[agg] | \
+            {"idw": 0, "dot": FWPKM_SCORE_DOT}[score]
         _check(load_library().fwpkm_state_set_options(self._h, opts))
 
     def set_wait_limits(self, mbar_polls: int = -1, scan_polls: int = -1):

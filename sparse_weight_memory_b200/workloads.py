@@ -65,6 +65,7 @@ class Workload:
     lookahead: bool = False  # each call writes query t towards the target of token t+1
     heads_mode: str = "mean"  # head readouts "mean" or "sum"
     agg: str = "weight"       # divisor of a value row's gradient: "weight", "count", "sum"
+    score: str = "idw"        # sub-key score: "idw" (-log(eps + |q - K|^2)) or "dot" (q . K)
     per_sequence: bool = False  # one memory per sequence (B memories in one state)
 
     @property
