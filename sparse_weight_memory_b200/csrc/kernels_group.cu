@@ -640,7 +640,7 @@ cudaError_t launch_bsort(const Dims &d, const Scratch &s, const Dims &dn, const 
 constexpr int kApplyThreads = 256;
 constexpr int kApplyWarps = kApplyThreads / 32;
 constexpr int kChunk4 = 32;  // float4 per column chunk (one per lane)
-constexpr int kU = 8;        // source rows in flight per warp
+constexpr int kU = 4;        // source rows in flight per warp
 
 __device__ __forceinline__ float4 load_chunk(const float *row, int c4, int n4) {
   return c4 < n4 ? *reinterpret_cast<const float4 *>(row + 4 * c4)
@@ -730,7 +730,7 @@ __device__ __forceinline__ void resplit_key_chunk(const Dims &d, const Scratch &
 }
 
 template <typename TQ>
-__global__ void __launch_bounds__(kApplyThreads, 3) k_apply(Dims d, float *__restrict__ V,
+__global__ void __launch_bounds__(kApplyThreads, 4) k_apply(Dims d, float *__restrict__ V,
                                                             float *__restrict__ K,
                                                             const TQ *__restrict__ Qin, Scratch s,
                                                             int part) {

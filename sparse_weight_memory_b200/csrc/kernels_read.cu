@@ -112,8 +112,12 @@ __device__ __forceinline__ float ld_peer(uint32_t addr) {
   return v;
 }
 
-template <typename TV, int kThreads>
-__global__ void __launch_bounds__(kThreads) k_read(Dims d, const float *__restrict__ V,
+// kVt: float4 columns per thread, ceil(dv / 4 / kThreads) (1, 2 or 4), so
+// that the registers holding the target, yhat and e rows are only those the
+// row width needs: at dv = 512 the CTAs of a 1024-token chunk then fit the
+// multiprocessors in one wave.
+template <typename TV, int kThreads, int kVt>
+__global__ void __launch_bounds__(kThreads, kThreads == 128 ? 7 : 1) k_read(Dims d, const float *__restrict__ V,
                                                        const TV *__restrict__ Vt,
                                                        const float *__restrict__ gate,
                                                        const float *__restrict__ omega,
@@ -171,7 +175,6 @@ __global__ void __launch_bounds__(kThreads) k_read(Dims d, const float *__restri
   const float om = last ? 0.f : (omega ? omega[tok] : g);  // the token's MSE weight
   const float invH = d.heads_sum ? 1.f : 1.f / (float)d.H;  // head readouts averaged or summed
   // the token's target row, loaded now so that it is here when e is formed
-  constexpr int kVt = 4;  // float4 per thread held (dv <= 4 * 4 * kThreads)
   float4 vt[kVt];
 #pragma unroll
   for (int q = 0; q < kVt; ++q) {
@@ -358,11 +361,11 @@ __global__ void __launch_bounds__(kThreads) k_read(Dims d, const float *__restri
   }
 }
 
-template <typename TV, int kThreads>
+template <typename TV, int kThreads, int kVt>
 static cudaError_t launch_read_tn(const Dims &d, const float *V, const TV *Vt, const float *gate,
                                   const float *omega, float *out, const Scratch &s,
                                   const ReadPlan &p, cudaStream_t st) {
-  auto kernel = k_read<TV, kThreads>;
+  auto kernel = k_read<TV, kThreads, kVt>;
   cudaError_t e =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
   if (e != cudaSuccess) return e;
@@ -375,9 +378,12 @@ static cudaError_t launch_read_t(const Dims &d, const float *V, const TV *Vt, co
                                  const float *omega, float *out, const Scratch &s,
                                  cudaStream_t st) {
   const ReadPlan p = read_plan(d);
-  if (p.threads == 32) return launch_read_tn<TV, 32>(d, V, Vt, gate, omega, out, s, p, st);
-  if (p.threads == 64) return launch_read_tn<TV, 64>(d, V, Vt, gate, omega, out, s, p, st);
-  return launch_read_tn<TV, 128>(d, V, Vt, gate, omega, out, s, p, st);
+  if (p.threads == 32) return launch_read_tn<TV, 32, 1>(d, V, Vt, gate, omega, out, s, p, st);
+  if (p.threads == 64) return launch_read_tn<TV, 64, 1>(d, V, Vt, gate, omega, out, s, p, st);
+  const int dv4 = d.dv / 4;  // at most 4 * 128 (dv <= 2048)
+  if (dv4 <= 128) return launch_read_tn<TV, 128, 1>(d, V, Vt, gate, omega, out, s, p, st);
+  if (dv4 <= 256) return launch_read_tn<TV, 128, 2>(d, V, Vt, gate, omega, out, s, p, st);
+  return launch_read_tn<TV, 128, 4>(d, V, Vt, gate, omega, out, s, p, st);
 }
 
 cudaError_t launch_read(const Dims &d, const float *V, const void *Vt, int v_dtype,

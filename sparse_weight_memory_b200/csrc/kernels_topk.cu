@@ -141,7 +141,7 @@ __device__ __forceinline__ uint32_t float_unorder(uint32_t u) {
 
 // Top-k smallest distances of one half row drow[0..n) (n <= 32*NV), ties by
 // index.  Lane r < k returns one winner (distance, index); order unspecified.
-// wbuf holds 64 entries.  `sgn`: the values may be negative (the negated dot
+// wbuf holds 64 entries.  kSgn: the values may be negative (the negated dot
 // products of the dot-product score), so they are keyed by float_order.
 //
 // With 4 or more entries per lane the search is narrowed first: every lane
@@ -151,8 +151,8 @@ __device__ __forceinline__ uint32_t float_unorder(uint32_t u) {
 // which are gathered two per lane and selected exactly.  Past 64 such keys
 // (heavy ties) the whole row is searched instead.  Either way the result is
 // the exact top-k under (key asc, index asc).
-template <int NV>
-__device__ __forceinline__ void half_topk(const float *__restrict__ drow, int n, int k, bool sgn,
+template <int NV, bool kSgn>
+__device__ __forceinline__ void half_topk(const float *__restrict__ drow, int n, int k,
                                           float &d_out, int &i_out, uint2 *wbuf) {
   const int lane = threadIdx.x & 31;
   uint32_t key[NV], idx[NV];
@@ -162,7 +162,7 @@ __device__ __forceinline__ void half_topk(const float *__restrict__ drow, int n,
     // d >= 0: the bit order is the value order; a used entry never takes the
     // unused marker 0xffffffff, whatever the distance's bits
     const float dv = i < n ? drow[i] : 0.f;
-    key[v] = i < n ? min(sgn ? float_order(dv) : __float_as_uint(dv), 0xfffffffeu)
+    key[v] = i < n ? min(kSgn ? float_order(dv) : __float_as_uint(dv), 0xfffffffeu)
                    : 0xffffffffu;
     idx[v] = (uint32_t)i;
   }
@@ -210,14 +210,14 @@ __device__ __forceinline__ void half_topk(const float *__restrict__ drow, int n,
       __syncwarp();
       const uint32_t sel = warp_select_smallest<2>(ck, ci, k);
       compact_selected<2>(sel, ck, ci, wbuf, kk, ii, v_out, src);
-      d_out = __uint_as_float(sgn ? float_unorder(kk) : kk);
+      d_out = __uint_as_float(kSgn ? float_unorder(kk) : kk);
       i_out = (int)ii;
       return;
     }
   }
   const uint32_t sel = warp_select_smallest<NV>(key, idx, k);
   compact_selected<NV>(sel, key, idx, wbuf, kk, ii, v_out, src);
-  d_out = __uint_as_float(sgn ? float_unorder(kk) : kk);
+  d_out = __uint_as_float(kSgn ? float_unorder(kk) : kk);
   i_out = (int)ii;
 }
 
@@ -277,7 +277,7 @@ struct TopkSmem {
 // top-k of its half and sorts them; warp 2t merges; then each warp writes
 // its half's sub-key entries.  A token-head whose selection is forced reads
 // the given slots instead.
-template <int NV, int KV, bool kSelectOnly>
+template <int NV, int KV, bool kSelectOnly, bool kDot>
 __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Extras x) {
   __shared__ TopkSmem sm;
   const int lane = threadIdx.x & 31;
@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
   const int m = blockIdx.x * kTopkHeads + t;  // token-head m = row*H + h
   const int k = d.k, n = d.n;
   const float eps = d.eps;
-  const bool dot = d.score_dot != 0;  // D = -q.K: the score is -D, ds/dK = q
+  constexpr bool dot = kDot;  // D = -q.K: the score is -D, ds/dK = q
   // the staircase for this k (warp 0, before the halves are selected)
   if (wib == 0) {
     const int len = lane < k ? min(k, k / (lane + 1)) : 0;
@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
   if (valid && !forced) {
     float dw;
     int iw;
-    half_topk<NV>(half == 0 ? D1 : D2, n, k, dot, dw, iw, sm.wbuf[wib]);
+    half_topk<NV, kDot>(half == 0 ? D1 : D2, n, k, dw, iw, sm.wbuf[wib]);
     const float sw = dot ? -dw : -logf(eps + dw);
     const uint64_t key =
         lane < k ? ((uint64_t)float_order(-sw) << 32) | (uint32_t)iw : ~0ull;
@@ -374,10 +374,11 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
       // An exact tie of an outside candidate with the k-th score could change
       // which equal-score slot wins the last places: take the full k x k merge.
       const uint32_t kth = __reduce_max_sync(FULL, lane < k ? wkey : 0u);
-      bool tie = false;
-      if (lane < k)
-        for (int bb = k / (lane + 1); bb < k; ++bb)
-          tie |= float_order(-(S1[lane] + S2[bb])) == kth;
+      // Only the first outside candidate of each rank a can tie: the ones after
+      // it score no higher (S2 descends, and a rounded sum is monotone in each
+      // term), and none scores above the k-th, which dominates it.
+      const int b0 = lane < k ? k / (lane + 1) : k;
+      const bool tie = b0 < k && float_order(-(S1[lane] + S2[b0])) == kth;
       if (__any_sync(FULL, tie)) {
         uint32_t fkey[KV], fslot[KV];
         const float sa = lane < k ? S1[lane] : 0.f;
@@ -466,27 +467,38 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
   if (lane == 0) s.ecount[(int64_t)m * 2 + half] = __popc(lb);
 }
 
-template <int KV, bool kSelectOnly>
+template <int KV, bool kSelectOnly, bool kDot>
 static cudaError_t launch_topk_kv(const Dims &d, const Scratch &s, const Extras &x,
                                   cudaStream_t st) {
   const int blocks = (d.M + kTopkHeads - 1) / kTopkHeads;
   const int nv = (d.n + 31) / 32;
   const int th = 64 * kTopkHeads;
-  if (nv <= 1) return launch_k(d.pdl, k_topk<1, KV, kSelectOnly>, blocks, th, 0, st, d, s, x);
-  if (nv <= 2) return launch_k(d.pdl, k_topk<2, KV, kSelectOnly>, blocks, th, 0, st, d, s, x);
-  if (nv <= 4) return launch_k(d.pdl, k_topk<4, KV, kSelectOnly>, blocks, th, 0, st, d, s, x);
-  if (nv <= 8) return launch_k(d.pdl, k_topk<8, KV, kSelectOnly>, blocks, th, 0, st, d, s, x);
-  if (nv <= 16) return launch_k(d.pdl, k_topk<16, KV, kSelectOnly>, blocks, th, 0, st, d, s, x);
-  if (nv <= 32) return launch_k(d.pdl, k_topk<32, KV, kSelectOnly>, blocks, th, 0, st, d, s, x);
+  if (nv <= 1)
+    return launch_k(d.pdl, k_topk<1, KV, kSelectOnly, kDot>, blocks, th, 0, st, d, s, x);
+  if (nv <= 2)
+    return launch_k(d.pdl, k_topk<2, KV, kSelectOnly, kDot>, blocks, th, 0, st, d, s, x);
+  if (nv <= 4)
+    return launch_k(d.pdl, k_topk<4, KV, kSelectOnly, kDot>, blocks, th, 0, st, d, s, x);
+  if (nv <= 8)
+    return launch_k(d.pdl, k_topk<8, KV, kSelectOnly, kDot>, blocks, th, 0, st, d, s, x);
+  if (nv <= 16)
+    return launch_k(d.pdl, k_topk<16, KV, kSelectOnly, kDot>, blocks, th, 0, st, d, s, x);
+  if (nv <= 32)
+    return launch_k(d.pdl, k_topk<32, KV, kSelectOnly, kDot>, blocks, th, 0, st, d, s, x);
   return cudaErrorInvalidValue;  // n > 1024: rejected when the state is made
 }
 
 template <bool kSelectOnly>
 static cudaError_t launch_topk_t(const Dims &d, const Scratch &s, const Extras &x,
                                  cudaStream_t st) {
-  if (d.k <= 8) return launch_topk_kv<8, kSelectOnly>(d, s, x, st);
-  if (d.k <= 16) return launch_topk_kv<16, kSelectOnly>(d, s, x, st);
-  return launch_topk_kv<32, kSelectOnly>(d, s, x, st);
+  if (d.score_dot) {
+    if (d.k <= 8) return launch_topk_kv<8, kSelectOnly, true>(d, s, x, st);
+    if (d.k <= 16) return launch_topk_kv<16, kSelectOnly, true>(d, s, x, st);
+    return launch_topk_kv<32, kSelectOnly, true>(d, s, x, st);
+  }
+  if (d.k <= 8) return launch_topk_kv<8, kSelectOnly, false>(d, s, x, st);
+  if (d.k <= 16) return launch_topk_kv<16, kSelectOnly, false>(d, s, x, st);
+  return launch_topk_kv<32, kSelectOnly, false>(d, s, x, st);
 }
 
 cudaError_t launch_topk(const Dims &d, const Scratch &s, const Extras &x, cudaStream_t st) {
