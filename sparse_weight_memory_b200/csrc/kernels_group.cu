@@ -466,6 +466,18 @@ __device__ void sort_big_bucket(const Dims &d, const Scratch &s, int off, int le
   __syncthreads();
 }
 
+// Work-list entries a sort CTA stages in shared memory per list (short and
+// long groups of each kind) before it appends them to the global lists with
+// one reservation each; past that many, an entry is appended at once.
+constexpr int kListStage = 512;
+
+__device__ __forceinline__ void stage_list(const Scratch &s, int (*lst)[kListStage], int kind,
+                                           bool lng, int i, int x) {
+  if (i < kListStage) lst[(lng ? 2 : 0) + kind][i] = x;
+  else if (lng) s.longlist[kind][atomicAdd(&s.meta->nlong[kind], 1)] = x;
+  else s.shortlist[kind][atomicAdd(&s.meta->nshort[kind], 1)] = x;
+}
+
 template <typename TQ>
 __global__ void __launch_bounds__(kSortThreads)
     k_bucket_sort(Dims d, Scratch s, Dims dn, const TQ *__restrict__ Q, int sort_blocks) {
@@ -474,6 +486,8 @@ __global__ void __launch_bounds__(kSortThreads)
   __shared__ int big_n;
   __shared__ int big_b[kSortWarps * 8];  // large buckets met in phase 1
   __shared__ int rank_red[32], rank_flag;
+  __shared__ int lst[4][kListStage];  // staged entries: short[kind], then long[kind]
+  __shared__ int lst_n[4], lst_base[4];
   griddep_wait();
   griddep_launch();
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
@@ -489,6 +503,7 @@ __global__ void __launch_bounds__(kSortThreads)
   // prepared; they index nothing).
   if (chunk_aborted(s, ERR_SORT_OVERFLOW)) return;
   if (threadIdx.x < 2) nseg[threadIdx.x] = 0;
+  if (threadIdx.x < 4) lst_n[threadIdx.x] = 0;
   if (threadIdx.x == 0) big_n = 0;
   __syncthreads();
   const int stride = sort_blocks * kSortWarps;
@@ -563,13 +578,13 @@ __global__ void __launch_bounds__(kSortThreads)
     const unsigned sb = __ballot_sync(FULL, sh), lb = __ballot_sync(FULL, lg);
     int sbase = 0, lbase = 0;
     if (lane == 0) {
-      if (sb) sbase = atomicAdd(&s.meta->nshort[kind], __popc(sb));
-      if (lb) lbase = atomicAdd(&s.meta->nlong[kind], __popc(lb));
+      if (sb) sbase = atomicAdd(&lst_n[kind], __popc(sb));
+      if (lb) lbase = atomicAdd(&lst_n[2 + kind], __popc(lb));
     }
     sbase = __shfl_sync(FULL, sbase, 0);
     lbase = __shfl_sync(FULL, lbase, 0);
-    if (sh) s.shortlist[kind][sbase + __popc(sb & lanemask_lt())] = off + lane;
-    if (lg) s.longlist[kind][lbase + __popc(lb & lanemask_lt())] = off + lane;
+    if (sh) stage_list(s, lst, kind, false, sbase + __popc(sb & lanemask_lt()), off + lane);
+    if (lg) stage_list(s, lst, kind, true, lbase + __popc(lb & lanemask_lt()), off + lane);
     if (lane == 0) atomicAdd(&nseg[b < d.NBv ? 0 : 1], __popc(heads));
   }
   __syncthreads();
@@ -589,6 +604,19 @@ __global__ void __launch_bounds__(kSortThreads)
   if (threadIdx.x == 0) {
     if (nseg[0]) atomicAdd(&s.meta->stat_value_rows, (unsigned long long)nseg[0]);
     if (nseg[1]) atomicAdd(&s.meta->stat_key_rows, (unsigned long long)nseg[1]);
+  }
+  // the staged entries go to the global lists, one reservation per list
+  if (threadIdx.x < 4) {
+    const int q = threadIdx.x, c = min(lst_n[q], kListStage);
+    int *ctr = q < 2 ? &s.meta->nshort[q] : &s.meta->nlong[q - 2];
+    lst_base[q] = c ? atomicAdd(ctr, c) : 0;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c = min(lst_n[q], kListStage);
+    int *dst = q < 2 ? s.shortlist[q] : s.longlist[q - 2];
+    for (int i = threadIdx.x; i < c; i += blockDim.x) dst[lst_base[q] + i] = lst[q][i];
   }
 }
 

@@ -136,7 +136,8 @@ struct TcSmem {
   static constexpr int kB = BN * kTcKBlock * 4;
   static constexpr int kStage = 2 * kA + 2 * kB;      // hi and lo of A and B
   static constexpr int kStages = tc_stages<BN>();
-  static constexpr int kBytes = kStages * kStage + 1024 /* align */ + 256 /* barriers */;
+  static constexpr int kBytes =
+      kStages * kStage + 1024 /* align */ + 256 /* barriers */ + 4 * BN /* column norms */;
   static_assert(kStage >= 4 * 32 * 33 * 4, "epilogue tile fits in stage 0");
 };
 
@@ -155,6 +156,7 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
   uint64_t *empty = full + kTcStages;
   uint64_t *done = empty + kTcStages;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+  float *kn_s = reinterpret_cast<float *>(smem + kTcStages * L::kStage + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hh = blockIdx.z;
@@ -179,6 +181,24 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
   const uint32_t tmem = *tmem_slot;
   griddep_wait();
   griddep_launch();
+
+  // The norms the epilogue adds do not depend on the products, so they are
+  // loaded before the main loop: each thread's row norm into a register, the
+  // tile's column norms (chunk norms added in chunk order) into shared memory
+  // by warps 2 and 3, which have nothing else to do until the epilogue.
+  const bool dot = d.score_dot != 0;
+  const int my_row = m0 + warp * 32 + lane;
+  const float my_qn = !dot && my_row < d.drows ? s.qn[(int64_t)hh * d.qstride + my_row] : 0.f;
+  if (warp >= 2 && !dot) {
+    const float *kn = s.kn + (int64_t)tab * d.n * kKnChunks;
+    const int nkc = (d.dh / 4 + 31) / 32;  // 128-float chunks of a sub-key row
+    for (int c = threadIdx.x - 64; c < BN; c += 64) {
+      float v = 0.f;
+      if (n0 + c < d.n)
+        for (int ch = 0; ch < nkc; ++ch) v += kn[(int64_t)(n0 + c) * kKnChunks + ch];
+      kn_s[c] = v;
+    }
+  }
 
   int issued = 0;  // k-blocks whose loads the producer issued (thread 0)
   if (warp == 0 && lane == 0) {
@@ -224,6 +244,7 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
     mma_commit(done);  // accumulator complete (or abandoned after an error)
   }
   __syncwarp();
+  __syncthreads();  // the column norms are in shared memory
 
   // ---------------- epilogue: TMEM -> distances ----------------
   // Each warp owns 32 accumulator lanes (rows).  Per block of 32 columns the
@@ -248,12 +269,6 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
   if (ready) {
     float *tile = reinterpret_cast<float *>(smem) + warp * 32 * 33;
     const int row0 = m0 + warp * 32;
-    const int my_row = row0 + lane;
-    const bool dot = d.score_dot != 0;
-    const float my_qn =
-        !dot && my_row < d.drows ? s.qn[(int64_t)hh * d.qstride + my_row] : 0.f;
-    const float *kn = s.kn + (int64_t)tab * d.n * kKnChunks;
-    const int nkc = (d.dh / 4 + 31) / 32;  // 128-float chunks of a sub-key row
     float *Dh = s.D + (int64_t)hh * d.drows * d.n;
 #pragma unroll 1
     for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -264,9 +279,7 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
       __syncwarp();
       const int col = n0 + c0 + lane;
       const bool col_ok = col < d.n && c0 + lane < BN;
-      float kn_l = 0.f;  // |K_col|^2: the chunk norms in chunk order
-      if (col_ok && !dot)
-        for (int ch = 0; ch < nkc; ++ch) kn_l += kn[(int64_t)col * kKnChunks + ch];
+      const float kn_l = col_ok && !dot ? kn_s[c0 + lane] : 0.f;  // |K_col|^2
 #pragma unroll 4
       for (int r = 0; r < 32; ++r) {
         const float qn_r = __shfl_sync(FULL, my_qn, r);
