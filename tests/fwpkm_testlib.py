@@ -70,9 +70,10 @@ class RunResult:
 
 
 def oracle_run(wl: Workload, inp: Inputs, oracle, max_chunks: int = 0,
-               state=None, omega=None) -> RunResult:
+               state=None, omega=None, tables: bool = True) -> RunResult:
     """Oracle over the workload's calls; continues `state` in place if given.
-    ``omega`` [B][T_total]: the tokens' MSE weights (default: the gate)."""
+    ``omega`` [B][T_total]: the tokens' MSE weights (default: the gate).
+    ``tables=False``: K and V of the result are None (read them from `state`)."""
     st = state if state is not None else oracle.State(inp.subkeys, inp.values, topk=wl.topk,
                                                       chunk=wl.chunk, eps=wl.eps,
                                                       heads=wl.heads_mode, agg=wl.agg,
@@ -86,22 +87,29 @@ def oracle_run(wl: Workload, inp: Inputs, oracle, max_chunks: int = 0,
         ws.append(r["sel_w"])
         gaps.append(r["gap"])
         touched += int(r["touched"].sum())
-    K, V = (st.K.copy(), st.V.copy()) if state is not None else (st.K, st.V)
+    K = V = None
+    if tables:
+        K, V = (st.K.copy(), st.V.copy()) if state is not None else (st.K, st.V)
     return RunResult(outs, sels, ws, gaps, K, V, touched)
 
 
 def gpu_run(wl: Workload, inp: Inputs, ref: Optional[RunResult] = None, force: bool = True,
-            K0=None, V0=None, with_stats: bool = False, omega=None) -> RunResult:
+            K0=None, V0=None, with_stats: bool = False, omega=None, state=None,
+            tables: bool = True) -> RunResult:
     """Run the workload through the C ABI.  With `ref` and `force`, token-heads
     where the oracle has a near tie read the oracle's slots.  ``omega`` as in
-    oracle_run; the workload's lookahead flag is passed on."""
+    oracle_run; the workload's lookahead flag is passed on.  ``state``: an
+    existing FwPKMState with its tables already set (the caller keeps it);
+    ``tables=False`` leaves the tables on the device (K and V are None)."""
     import torch
 
     from sparse_weight_memory_b200 import FwPKMState
-    st = FwPKMState(wl.N, wl.dq, wl.dv, wl.topk, wl.chunk, wl.heads, eps=wl.eps)
-    st.set_options(heads=wl.heads_mode, agg=wl.agg, score=wl.score)
-    st.set_tables(to_dev(inp.subkeys if K0 is None else K0),
-                  to_dev(inp.values if V0 is None else V0))
+    st = state
+    if st is None:
+        st = FwPKMState(wl.N, wl.dq, wl.dv, wl.topk, wl.chunk, wl.heads, eps=wl.eps)
+        st.set_options(heads=wl.heads_mode, agg=wl.agg, score=wl.score)
+        st.set_tables(to_dev(inp.subkeys if K0 is None else K0),
+                      to_dev(inp.values if V0 is None else V0))
     if with_stats:
         st.read_stats(reset=True)
     outs, sels, ws, keep = [], [], [], []
@@ -123,17 +131,20 @@ def gpu_run(wl: Workload, inp: Inputs, ref: Optional[RunResult] = None, force: b
         sels.append(rs)
         ws.append(rw)
     torch.cuda.synchronize()
-    K, V = st.get_tables()
-    torch.cuda.synchronize()
+    K = V = None
+    if tables:
+        K, V = st.get_tables()
+        torch.cuda.synchronize()
+        K, V = K.cpu().numpy(), V.cpu().numpy()
     touched = None
     if with_stats:
         stats = st.read_stats()
         assert stats["device_errors"] == 0
         touched = stats["value_rows"]
     res = RunResult([o.cpu().numpy() for o in outs], [s.cpu().numpy() for s in sels],
-                    [w.cpu().numpy() for w in ws], [None] * len(outs), K.cpu().numpy(),
-                    V.cpu().numpy(), touched)
-    st.close()
+                    [w.cpu().numpy() for w in ws], [None] * len(outs), K, V, touched)
+    if state is None:
+        st.close()
     return res
 
 

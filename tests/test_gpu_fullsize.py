@@ -4,7 +4,7 @@ bench.py times (same shapes, same chained calls and passes, same seeds).
 The oracle runs every chunk (OpenMP over token-heads), so these tests take
 minutes; near ties are forced to the oracle's choice (see fwpkm_testlib).
 The long-context workload runs its first 64 chunks free from the initial
-tables, then the rest in segments re-synchronised to the oracle's tables.
+tables, then every later chunk from the oracle's tables.
 """
 import numpy as np
 import pytest
@@ -47,15 +47,19 @@ def test_fullsize_longctx_64_and_128_chunks(oracle):
     workload is expanding (max |K| grows from ~1 to ~300 by chunk 90) and the
     tables turn chaotic: the oracle against itself, perturbed by one fp32 ulp
     at chunk 80, differs in selections beyond the tie band by chunk 95
-    (test_oracle_sensitivity).  So the second 64 chunks run as sixteen 4-chunk
-    segments, each started with both sides on the oracle's tables rounded to
-    fp32 (oracle -> GPU only), compared at every segment's end.
+    (test_oracle_sensitivity).  Past chunk 100 the value rows are of order 1
+    and many outputs nearly cancel, so the fp32 rounding of one chunk's table
+    update (a few 1e-6 on rows summed over ~1000 members) grows within three
+    chunks to the output bound's absolute term.  So each of the second 64
+    chunks starts with both sides on the oracle's tables rounded to fp32
+    (oracle -> GPU only) and is compared on its own: selection, outputs and
+    both tables, with the bounds of a single chunk (tables at 1e-4).
     """
     import copy
     import gc
     full = WORKLOADS["longctx"]
     inp = make_inputs(full)
-    seg_chunks = 4
+    seg_chunks = 1
 
     def segment(t0, T):
         part = copy.copy(inp)
@@ -77,23 +81,59 @@ def test_fullsize_longctx_64_and_128_chunks(oracle):
     del g
     gc.collect()
 
-    seg = full.replace(T=seg_chunks * full.chunk)
-    for t0 in range(64 * full.chunk, full.T, seg.T):
-        K0 = state.K.astype(np.float32)
-        V0 = state.V.astype(np.float32)
-        state.K[...] = K0  # both sides start the segment from the same fp32 tables
-        state.V[...] = V0
-        part = segment(t0, seg.T)
-        part.wl = seg
-        o = oracle_run(seg, part, oracle, state=state)
-        g = gpu_run(seg, part, o, force=True, K0=K0, V0=V0)
+    # One GPU state for the second half.  A chunk writes only the value rows
+    # it selects (and sub-key rows, a small table), so after each chunk only
+    # those rows are rounded to fp32 again and re-sent; the GPU's result is
+    # compared on them, and it must have written no other value row.
+    import torch
+
+    from sparse_weight_memory_b200 import FwPKMState
+    from fwpkm_testlib import to_dev
+    one = full.replace(T=seg_chunks * full.chunk)
+    st = FwPKMState(full.N, full.dq, full.dv, full.topk, full.chunk, full.heads, eps=full.eps)
+    K0 = state.K.astype(np.float32)
+    V0 = state.V.astype(np.float32)
+    state.K[...] = K0  # both sides start every chunk from the same fp32 tables
+    state.V[...] = V0
+    V0d = to_dev(V0)
+    ss0 = float(np.einsum("ij,ij->", V0, V0, dtype=np.float64))  # sum of squares of V0
+    for t0 in range(64 * full.chunk, full.T, one.T):
         c = t0 // full.chunk
-        check_selection(g.sels[0], o.sels[0], o.gaps[0], f"longctx chunks {c}-{c + seg_chunks - 1}")
-        check_close(g.outs[0], o.outs[0], OUT_ATOL, OUT_RTOL, f"longctx chunks from {c} out")
-        check_table(g.V, o.V, 1e-3, f"longctx values after chunk {c + seg_chunks - 1}")
-        check_table(g.K, o.K, 1e-3, f"longctx sub-keys after chunk {c + seg_chunks - 1}")
-        print(f"longctx chunks {c}-{c + seg_chunks - 1}: update rel err V "
-              f"{update_rel_error(g.V, o.V, V0):.2e} K {update_rel_error(g.K, o.K, K0):.2e}, "
-              f"max |K| {np.abs(o.K).max():.1f}")
-        del g, K0, V0
-        gc.collect()
+        st.set_tables(to_dev(K0), V0d)
+        part = segment(t0, one.T)
+        part.wl = one
+        o = oracle_run(one, part, oracle, state=state, tables=False)
+        g = gpu_run(one, part, o, force=True, state=st, tables=False)
+        check_selection(g.sels[0], o.sels[0], o.gaps[0], f"longctx chunk {c}")
+        ratio = float((np.abs(g.outs[0].astype(np.float64) - o.outs[0]) /
+                       (OUT_ATOL + OUT_RTOL * np.abs(o.outs[0]))).max())
+        check_close(g.outs[0], o.outs[0], OUT_ATOL, OUT_RTOL, f"longctx chunk {c} out")
+        Kg, Vg = st.get_tables()
+        rows = np.unique(o.sels[0])
+        rows_d = torch.from_numpy(rows).cuda()
+        changed = torch.nonzero((Vg != V0d).any(dim=1)).flatten().cpu().numpy()
+        assert np.isin(changed, rows).all(), f"chunk {c}: value rows written outside the selection"
+        vg, vo, v0 = Vg[rows_d].cpu().numpy(), state.V[rows], V0[rows]
+        # the bound of check_table: tol |ref| + tol rms(ref), rms over the whole table
+        ss = ss0 - float(np.einsum("ij,ij->", v0, v0, dtype=np.float64)) + float((vo ** 2).sum())
+        rms = np.sqrt(ss / V0.size)
+        err = np.abs(vg.astype(np.float64) - vo)
+        assert (err <= 1e-4 * np.abs(vo) + 1e-4 * rms).all(), (
+            f"longctx values after chunk {c}: worst abs err {err.max():.3g} (rms {rms:.3g})")
+        kg = Kg.cpu().numpy()
+        check_table(kg, state.K, 1e-4, f"longctx sub-keys after chunk {c}")
+        dv_rel = np.linalg.norm(vg - vo) / max(np.linalg.norm(vo - v0), 1e-300)
+        print(f"longctx chunk {c}: worst out err / bound {ratio:.3f}, update rel err V "
+              f"{dv_rel:.2e} K {update_rel_error(kg, state.K, K0):.2e}, "
+              f"max |K| {np.abs(state.K).max():.1f}")
+        # round the rows the chunk changed, for the next chunk on both sides
+        vr = state.V[rows].astype(np.float32)
+        state.V[rows] = vr
+        V0[rows] = vr
+        V0d[rows_d] = torch.from_numpy(vr).cuda()
+        ss0 = ss - float((vo ** 2).sum()) + float(np.einsum("ij,ij->", vr, vr, dtype=np.float64))
+        K0 = state.K.astype(np.float32)
+        state.K[...] = K0
+        del g, Kg, Vg
+    st.close()
+    gc.collect()
