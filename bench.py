@@ -265,12 +265,21 @@ def run_reference(args, wl):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
-def algorithmic_work(wl, tokens, value_rows, key_rows, records):
+def algorithmic_work(wl, tokens, segments, value_rows, key_rows, records, memories=1):
     """Algorithmic bytes (HBM-bound kernels) or flops (score) over `tokens`
-    tokens whose chunks wrote `value_rows` / `key_rows` distinct rows and
-    grouped `records` member records."""
+    tokens in `segments` step calls, whose chunks wrote `value_rows` /
+    `key_rows` distinct rows and grouped `records` member records."""
     in_b = 2 if wl.in_dtype == BF16 else 4
     gather = tokens * wl.heads * wl.topk * wl.dv * 4
+    dh = wl.dq // 2
+    # query halves of `t` tokens: read, written as TF32 hi + lo, and a norm per half
+    def halves(t):
+        return t * wl.heads * (wl.dq * (in_b + 8) + 2 * 4)
+    # the prep makes the first chunk's halves of each call and splits every
+    # sub-key row once per call (hi + lo + its 128-float chunk norms); the
+    # sort's extra CTAs make the halves of every later chunk
+    first = segments * wl.B * min(wl.chunk, wl.T)
+    split = segments * memories * 2 * wl.heads * wl.n * (dh * (4 + 8) + -(-dh // 128) * 4)
     return {
         # gathered value rows + Vtarget read + out written
         "fwpkm_read": ("hbm", gather + tokens * wl.dv * in_b + tokens * wl.dv * 4),
@@ -278,12 +287,12 @@ def algorithmic_work(wl, tokens, value_rows, key_rows, records):
         "fwpkm_apply": ("hbm", 2 * value_rows * wl.dv * 4 + 2 * key_rows * (wl.dq // 2) * 4),
         # q_half . K_row for every sub-key of both halves (fp32 products)
         "fwpkm_score": ("tensor", 2.0 * tokens * wl.heads * wl.n * wl.dq),
-        # member records read in claim order and written grouped (32 bytes each)
-        "fwpkm_bsort": ("hbm", 2 * 32 * records),
+        # member records read in claim order and written grouped (32 bytes each),
+        # and the next chunks' query halves
+        "fwpkm_bsort": ("hbm", 2 * 32 * records + halves(tokens - first)),
         # distance matrix read once, slots + weights written
         "fwpkm_topk": ("hbm", tokens * wl.heads * (2 * wl.n * 4 + wl.topk * 8)),
-        # queries read once, split into hi/lo halves + norms written
-        "fwpkm_prep": ("hbm", tokens * wl.heads * wl.dq * (in_b + 8) + tokens * wl.heads * 8),
+        "fwpkm_prep": ("hbm", halves(first) + split),
     }
 
 
@@ -476,8 +485,9 @@ def run_gpu(args, wl):
     if rank == 0:
         hbm_gbs, bf16_tf, peak_kind = peaks()
         rows_sum = wl.B * wl.T * wl.calls * wl.passes * prof_steps
-        work = algorithmic_work(wl, rows_sum, pstats["value_rows"], pstats["key_rows"],
-                                pstats["records"])
+        segs_sum = wl.calls * wl.passes * prof_steps
+        work = algorithmic_work(wl, rows_sum, segs_sum, pstats["value_rows"], pstats["key_rows"],
+                                pstats["records"], wl.B if wl.per_sequence else 1)
         traffic = NCU_TRAFFIC.get(wl.name, {})
         fracs = {k: kernel_roofline(k, work[k], ms, n, hbm_gbs, bf16_tf, peak_kind,
                                     traffic.get(k))

@@ -12,8 +12,9 @@ from sparse_weight_memory_b200.workloads import BF16, WORKLOADS
 
 def test_algorithmic_work_matches_the_per_unit_definitions():
     wl = WORKLOADS["library"]  # fp32 inputs, H=1, k=8, dv=dq=512, n=256
-    tokens, U_v, U_k, records = 512, 3000, 400, 10000
-    w = bench.algorithmic_work(wl, tokens, U_v, U_k, records)
+    segments = 3
+    tokens, U_v, U_k, records = segments * wl.B * wl.T, 3000, 400, 10000
+    w = bench.algorithmic_work(wl, tokens, segments, U_v, U_k, records)
     # read, per token: H*k*dv*4 gathered + dv*4 target (fp32) + dv*4 out
     assert w["fwpkm_read"] == ("hbm", tokens * (1 * 8 * 512 * 4 + 512 * 4 + 512 * 4))
     # apply: read-modify-write of the written value rows and sub-key rows
@@ -22,14 +23,21 @@ def test_algorithmic_work_matches_the_per_unit_definitions():
     assert w["fwpkm_score"] == ("tensor", 2.0 * tokens * 1 * 256 * 512)
     # topk, per token-head: both halves' n distances read, k (slot, weight) written
     assert w["fwpkm_topk"] == ("hbm", tokens * (2 * 256 * 4 + 8 * 8))
-    assert w["fwpkm_bsort"] == ("hbm", 2 * 32 * records)
+    # query halves per token-head: q read (4 B), hi + lo written (8 B), a norm per half
+    halves = lambda t: t * (512 * (4 + 8) + 2 * 4)
+    first = segments * wl.B * min(wl.chunk, wl.T)  # the first chunk of each call
+    # prep: the first chunk's halves and, once per call, every sub-key row of
+    # both halves split (fp32 read, hi + lo written, two 128-float chunk norms)
+    assert w["fwpkm_prep"] == ("hbm", halves(first) + segments * 2 * 256 * (256 * 12 + 2 * 4))
+    # sort: records read and written (32 B each), and the later chunks' halves
+    assert w["fwpkm_bsort"] == ("hbm", 2 * 32 * records + halves(tokens - first))
 
 
 def test_bf16_inputs_halve_the_streamed_target_bytes():
     wl = WORKLOADS["multihead"]
     assert wl.in_dtype == BF16
     tokens = 1000
-    w = bench.algorithmic_work(wl, tokens, 0, 0, 0)
+    w = bench.algorithmic_work(wl, tokens, 1, 0, 0, 0)
     gather = tokens * wl.heads * wl.topk * wl.dv * 4
     assert w["fwpkm_read"][1] == gather + tokens * wl.dv * 2 + tokens * wl.dv * 4
 
