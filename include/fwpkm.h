@@ -293,7 +293,7 @@ fwpkm_status fwpkm_profile_read(fwpkm_state *s, const char **names, double *ms,
  *    2  the apply's partial pool overflowed (the launch sizing rules it out),
  *    4  a bucket-scan CTA gave up waiting for an earlier CTA's total,
  *    8  the score's bounded wait on its TMA ring or its MMAs gave up,
- *   16  the sort met more large buckets than it lists (ruled out likewise).
+ *   16  reserved (no longer set: the list of large buckets holds them all).
  * A kernel that gives up still lets its own copies in flight land and
  * returns; no kernel traps.  Once a bit is set, the kernels after the bucket
  * scan (read, sort, apply) skip the rest of the call and of later calls,

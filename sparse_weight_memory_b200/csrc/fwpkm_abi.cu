@@ -203,6 +203,7 @@ fwpkm_status ensure_scratch(fwpkm_state *st, int64_t rows) {
       {(void **)&s.posmap, sizeof(int32_t) * (size_t)Lcap},
       {(void **)&s.shortlist[0], sizeof(int32_t) * (size_t)Lcap},
       {(void **)&s.shortlist[1], sizeof(int32_t) * (size_t)Lcap},
+      {(void **)&s.biglist, sizeof(int32_t) * (size_t)NB},
       {(void **)&s.longlist[0], sizeof(int32_t) * (size_t)Lcap},
       {(void **)&s.longlist[1], sizeof(int32_t) * (size_t)Lcap},
       {(void **)&s.arrive, sizeof(int32_t) * (size_t)pool_cap * kMaxChunks},
@@ -998,8 +999,8 @@ fwpkm_status fwpkm_read_stats(fwpkm_state *st, int64_t *chunks, int64_t *value_r
     return fail(FWPKM_ECUDA,
                 "device error bits 0x%x (1 = the read's row-copy wait gave up, 2 = the "
                 "apply's partial pool overflowed, 4 = a bucket-scan wait gave up, 8 = the "
-                "score's TMA/MMA wait gave up, 16 = the sort's list of large buckets "
-                "overflowed; the write kernels of that chunk and later ones were skipped)",
+                "score's TMA/MMA wait gave up, 16 = reserved; the write kernels of that "
+                "chunk and later ones were skipped)",
                 m.err);
   return FWPKM_OK;
 }

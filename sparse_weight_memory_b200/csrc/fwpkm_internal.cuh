@@ -35,7 +35,7 @@ enum : unsigned {
   ERR_POOL_OVERFLOW = 2u,  // apply: more long-group blocks than the partial pool holds
   ERR_SCAN_TIMEOUT = 4u,   // a scan CTA gave up waiting for an earlier CTA's total
   ERR_SCORE_TIMEOUT = 8u,  // the score's TMA ring or MMA completion wait gave up
-  ERR_SORT_OVERFLOW = 16u, // bsort: a CTA met more large buckets than it lists
+  ERR_SORT_OVERFLOW = 16u, // reserved: the large buckets' list holds every bucket
   ERR_ALL = 31u,
 };
 // Default bound of a wait (polls): a bounded wait that gives up sets its bit,
@@ -48,7 +48,7 @@ constexpr long long kDrainPolls = 1ll << 26;
 // Written by the kernels, read by later kernels and by the host.
 struct Meta {
   int32_t L;              // members of the chunk (pairs + sub-key entries)
-  int32_t pad1;
+  int32_t nbig;           // buckets of more than 32 members, listed by the scan in biglist
   unsigned err;           // ERR_* bits, sticky until the host clears them
   // Work lists of the chunk, per kind (0: value rows, 1: sub-key rows),
   // reset per chunk by the scan:
@@ -130,6 +130,7 @@ struct Scratch {
   uint64_t *sort_tmp;  // [2*Lcap] merge buffers for oversized buckets
   int32_t *posmap;  // [Lcap]  position inside its bucket, by member id (oversized buckets)
   int32_t *shortlist[2];  // [Lcap] per kind: first position of every group of <= 4 members
+  int32_t *biglist;       // [NB] buckets of more than 32 members (the scan lists them)
   int32_t *longlist[2];   // [Lcap] per kind: first position of every 32-member block of a
                           //        longer group (a group's blocks are consecutive)
   int32_t *arrive;        // [pool_cap][kMaxChunks] blocks of a longer group done with a

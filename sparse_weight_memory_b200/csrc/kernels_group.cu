@@ -30,6 +30,10 @@
 
 namespace fwpkm {
 
+// A bucket of more than this many members is sorted by a whole CTA (the scan
+// lists it); smaller ones by one warp.
+constexpr int kWarpBucket = 32;
+
 __device__ __forceinline__ Member load_member(const Member *p) {
   const int4 a = *reinterpret_cast<const int4 *>(p);
   const int4 b = *(reinterpret_cast<const int4 *>(p) + 1);
@@ -106,9 +110,23 @@ __global__ void __launch_bounds__(kScanThreads) k_bucket_scan(Dims d, Scratch s)
       if (b0 + i < NB) s.bcnt[b0 + i] = 0;
     }
   }
-  int total = 0;
+  int total = 0, nbig = 0;
 #pragma unroll
-  for (int i = 0; i < kScanPer; ++i) total += v[i];
+  for (int i = 0; i < kScanPer; ++i) {
+    total += v[i];
+    nbig += v[i] > kWarpBucket ? 1 : 0;
+  }
+  // The large buckets are listed for the sort, one reservation per warp that
+  // has any; the reservation is taken now and its result used only at the
+  // end, so that its round trip overlaps the scan.
+  int ib = nbig;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(FULL, ib, o);
+    if (lane >= o) ib += t;
+  }
+  int big_base = 0;
+  if (lane == 31 && ib) big_base = atomicAdd(&s.meta->nbig, ib);
   int incl = total;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -174,6 +192,12 @@ __global__ void __launch_bounds__(kScanThreads) k_bucket_scan(Dims d, Scratch s)
       if (b0 + i < NB) s.boff[b0 + i] = run;
       run += v[i];
     }
+  }
+  if (__any_sync(FULL, nbig > 0)) {
+    int pos = __shfl_sync(FULL, big_base, 31) + ib - nbig;
+#pragma unroll
+    for (int i = 0; i < kScanPer; ++i)
+      if (v[i] > kWarpBucket) s.biglist[pos++] = b0 + i;
   }
   if (tid == 0 && c == gridDim.x - 1) {
     const int L = prefix_s + cta_total;
@@ -483,8 +507,6 @@ __global__ void __launch_bounds__(kSortThreads)
     k_bucket_sort(Dims d, Scratch s, Dims dn, const TQ *__restrict__ Q, int sort_blocks) {
   __shared__ uint64_t buf[kSortCap];
   __shared__ int nseg[2];  // distinct value rows / sub-key rows seen by this CTA
-  __shared__ int big_n;
-  __shared__ int big_b[kSortWarps * 8];  // large buckets met in phase 1
   __shared__ int rank_red[32], rank_flag;
   __shared__ int lst[4][kListStage];  // staged entries: short[kind], then long[kind]
   __shared__ int lst_n[4], lst_base[4];
@@ -504,10 +526,9 @@ __global__ void __launch_bounds__(kSortThreads)
   if (chunk_aborted(s, ERR_SORT_OVERFLOW)) return;
   if (threadIdx.x < 2) nseg[threadIdx.x] = 0;
   if (threadIdx.x < 4) lst_n[threadIdx.x] = 0;
-  if (threadIdx.x == 0) big_n = 0;
   __syncthreads();
   const int stride = sort_blocks * kSortWarps;
-  // phase 1: small buckets, one warp each; large ones are listed.  Bucket b
+  // phase 1: small buckets, one warp each; large ones are left to phase 2.  Bucket b
   // goes to CTA b % sort_blocks: neighbouring buckets (slots of one popular
   // sub-key row) land in different CTAs.
   // The offsets of a warp's next 32 buckets are loaded together, one per lane.
@@ -521,14 +542,7 @@ __global__ void __launch_bounds__(kSortThreads)
     const int off = __shfl_sync(FULL, nxt_off, i & 31);
     const int len = __shfl_sync(FULL, nxt_end, i & 31) - off;
     if (len == 0) continue;
-    if (len > 32) {
-      if (lane == 0) {
-        const int slot = atomicAdd(&big_n, 1);
-        if (slot < kSortWarps * 8) big_b[slot] = b;
-        else atomicOr(&s.meta->err, ERR_SORT_OVERFLOW);  // cannot happen: see launch_bsort
-      }
-      continue;
-    }
+    if (len > kWarpBucket) continue;  // listed by the scan; sorted in phase 2
     Member m{};
     uint64_t key = ~0ull;
     if (lane < len) {
@@ -588,10 +602,11 @@ __global__ void __launch_bounds__(kSortThreads)
     if (lane == 0) atomicAdd(&nseg[b < d.NBv ? 0 : 1], __popc(heads));
   }
   __syncthreads();
-  // phase 2: the large buckets, each by the whole CTA
-  const int nbig = min(big_n, kSortWarps * 8);
-  for (int i = 0; i < nbig; ++i) {
-    const int b = big_b[i];
+  // phase 2: the large buckets, each by a whole CTA, dealt out in the order
+  // of the scan's list (one each while there are CTAs enough)
+  const int nbig = s.meta->nbig;
+  for (int i = blockIdx.x; i < nbig; i += sort_blocks) {
+    const int b = s.biglist[i];
     const int off = s.boff[b], len = s.boff[b + 1] - off;
     const bool value = b < d.NBv;
     const uint32_t gbase =
@@ -620,8 +635,7 @@ __global__ void __launch_bounds__(kSortThreads)
   }
 }
 
-// Every CTA meets at most 8 buckets per warp (so big_b cannot overflow):
-// the sorting grid holds at least NB / (8 * kSortWarps) CTAs.  The extra
+// The sorting grid: a warp per bucket up to the resident CTAs.  The extra
 // CTAs after it prepare the next chunk's query halves (dn.rows > 0).
 template <typename TQ>
 static cudaError_t launch_bsort_t(const Dims &d, const Scratch &s, const Dims &dn, const TQ *Q,
@@ -632,9 +646,7 @@ static cudaError_t launch_bsort_t(const Dims &d, const Scratch &s, const Dims &d
     if (per_sm < 1) per_sm = 1;
   }
   int blocks = (d.NB + kSortWarps - 1) / kSortWarps;
-  const int min_blocks = (d.NB + 8 * kSortWarps - 1) / (8 * kSortWarps);
-  int cap = d.sm_count * per_sm;
-  if (cap < min_blocks) cap = min_blocks;
+  const int cap = d.sm_count * per_sm;
   if (blocks > cap) blocks = cap;
   const int64_t qwarps = dn.rows > 0 ? (int64_t)2 * dn.H * dn.rows : 0;
   const int extra = (int)((qwarps + kSortWarps - 1) / kSortWarps);

@@ -302,7 +302,11 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
   griddep_wait();
   griddep_launch();
   // a new chunk epoch for the bucket scan that follows (the step, not the selection-only call)
-  if (!kSelectOnly && blockIdx.x == 0 && threadIdx.x == 0) s.scan_sync[0] += 1ull;
+  // (and an empty list of large buckets, which the scan fills)
+  if (!kSelectOnly && blockIdx.x == 0 && threadIdx.x == 0) {
+    s.scan_sync[0] += 1ull;
+    s.meta->nbig = 0;
+  }
   const bool valid = m < d.M;
   const int row = valid ? m / d.H : 0, h = valid ? m % d.H : 0;
   const int lrow = lrow_of(d, row), mb = mem_of(d, row);  // layout row, memory
