@@ -396,6 +396,9 @@ fwpkm_status enqueue_chunks(fwpkm_state *st, int B, int T, const void *Q, int q_
     d.lookahead = lookahead;
     d.q_tf32_exact = q_dtype == FWPKM_BF16 ? 1 : 0;
     d.readonly = readonly ? 1 : 0;
+    // the halves of a later chunk of the write path come from the previous
+    // chunk's sort, two grids or more before this chunk's score
+    d.q_early = !readonly && c > 0 ? 1 : 0;
     if (readonly) {
       if ((rc = hook(hooks ? hooks->need_inputs : nullptr, c))) return rc;
       if (lookahead && c + 1 < n_chunks &&

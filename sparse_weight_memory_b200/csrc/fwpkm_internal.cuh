@@ -91,6 +91,8 @@ struct Dims {
   int readonly;          // eta = 0: the read alone (no claims, entries, records, gradients)
   int agg;               // divisor of a value row's gradient (AGG_*)
   int score_dot;         // sub-key score q . K (D holds -q.K) instead of the IDW one
+  int q_early;           // the query halves come from a grid two or more before the score
+                         // (the previous chunk's sort): loading them needs no wait
 };
 // Divisor of a value row's gradient: its row contribution C_i = sum of w/H
 // (the sum of its members' c0), its access count (every member's c0 is 1), or

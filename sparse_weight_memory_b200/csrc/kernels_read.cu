@@ -22,7 +22,9 @@
 // token's H*k rows straight from global memory, every row load independent
 // of the others, so the rows of many tokens are in flight per
 // multiprocessor; the dot products then read the rows again, from L1 or L2.
-// The token's member records are written while the rows are in flight.
+// The token's member records, which go to the bucket scan's offsets, are
+// written last: only they wait for the scan, so the rest of the read runs
+// while the scan does.
 // Only a token whose rows exceed 1 MB is split over a thread-block cluster
 // of G CTAs, which exchange their partial sums through distributed shared
 // memory and add them in rank order (the same yhat everywhere).  (Staging
@@ -123,9 +125,15 @@ __global__ void __launch_bounds__(kThreads, kThreads == 128 ? 7 : 1) k_read(Dims
                                                        const float *__restrict__ omega,
                                                        float *__restrict__ out, Scratch s, int G,
                                                        int per) {
-  griddep_wait();
+  // After the bucket scan (the grid this one follows in the write path) the
+  // read waits only before its member records, which go to the scan's bucket
+  // offsets.  Everything else it reads was written by the selection and
+  // earlier kernels: the selection's grid completed before any scan CTA got
+  // past its own wait, and this grid is launched only after every scan CTA
+  // has.  At eta = 0 the selection itself comes just before: wait at once.
+  if (d.readonly) griddep_wait();
   griddep_launch();
-  // An earlier kernel gave up (the bits are stable here, so every CTA of a
+  // An earlier kernel gave up (its bits are stable here, so every CTA of a
   // cluster takes the same branch): nothing of this chunk is read or written.
   if (chunk_aborted(s, ERR_READ_TIMEOUT)) return;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -213,44 +221,6 @@ __global__ void __launch_bounds__(kThreads, kThreads == 128 ? 7 : 1) k_read(Dims
       acc.w = fmaf(w, v.w, acc.w);
     }
     *reinterpret_cast<float4 *>(ypart + 4 * c4) = acc;
-  }
-  // Member records go to their buckets after the rows (none of their fields
-  // depends on them, and their bucket offsets are one more dependent load
-  // that would otherwise delay the rows): this CTA's pairs -> value bucket
-  // slot >> vshift; entries x = rank (mod G) -> sub-key row bucket
-  // NBv + (h*2+half)*n + row.  An entry's alpha is filled in later from
-  // ealpha (by the sort, or by the apply when the entropy term is on).
-  for (int j = j0 + tid; j < (d.readonly ? j0 : j1); j += blockDim.x) {
-    const int64_t p = p0 + j;
-    const float w = w_s[j];
-    Member m;
-    m.g = (uint32_t)slot_s[j];
-    m.id = (uint32_t)p;
-    m.srow = row;
-    m.gstart = 0;
-    m.coef = 2.f * om * w * invH;
-    m.c0 = d.agg == AGG_COUNT ? 1.f : w * invH;  // the group's sum is the row's divisor
-    m.c1 = w;
-    m.glen = 0;
-    s.rec_in[s.boff[slot_s[j] >> d.vshift] + claim_s[j]] = m;
-  }
-  const int tab0 = mem_of(d, row) * 2 * d.H;  // the token's memory's first sub-key table
-  for (int x = rank + G * tid; x < (d.readonly ? 0 : 2 * HK); x += G * blockDim.x) {
-    const int mh = x / d.k;  // entry (h*2 + half)*k + idx of this row
-    const int sub = esub_s[x];
-    if (sub >= 0) {
-      const int64_t e = e0 + x;
-      Member m;
-      m.g = (uint32_t)d.Nt + (uint32_t)((tab0 + mh) * d.n + sub);
-      m.id = (uint32_t)e;
-      m.srow = (int)(tok * 2 * d.H + mh);  // this query half in the caller's Q
-      m.gstart = 0;
-      m.coef = 0.f;
-      m.c0 = 0.f;
-      m.c1 = 0.f;
-      m.glen = 0;
-      s.rec_in[s.boff[d.NBv + (tab0 + mh) * d.n + sub] + eclaim_s[x]] = m;
-    }
   }
   if (G > 1) cluster_barrier();
   else __syncthreads();
@@ -358,6 +328,48 @@ __global__ void __launch_bounds__(kThreads, kThreads == 128 ? 7 : 1) k_read(Dims
     }
     // no CTA leaves while another may still read its a values
     if (G > 1) cluster_barrier_relaxed();
+  }
+  if (d.readonly) return;  // no write follows: no records
+  griddep_wait();
+  // the scan gave up: its offsets may be wrong, so no record is written (the
+  // bits are stable after the wait: every CTA of a cluster takes this branch)
+  if (chunk_aborted(s, ERR_READ_TIMEOUT)) return;
+  // Member records go to their buckets last, at the scan's offsets: this
+  // CTA's pairs -> value bucket slot >> vshift; entries x = rank (mod G) ->
+  // sub-key row bucket NBv + (h*2+half)*n + row.  An entry's alpha is filled
+  // in later from ealpha (by the sort, or by the apply when the entropy term
+  // is on).
+  for (int j = j0 + tid; j < j1; j += blockDim.x) {
+    const int64_t p = p0 + j;
+    const float w = w_s[j];
+    Member m;
+    m.g = (uint32_t)slot_s[j];
+    m.id = (uint32_t)p;
+    m.srow = row;
+    m.gstart = 0;
+    m.coef = 2.f * om * w * invH;
+    m.c0 = d.agg == AGG_COUNT ? 1.f : w * invH;  // the group's sum is the row's divisor
+    m.c1 = w;
+    m.glen = 0;
+    s.rec_in[s.boff[slot_s[j] >> d.vshift] + claim_s[j]] = m;
+  }
+  const int tab0 = mem_of(d, row) * 2 * d.H;  // the token's memory's first sub-key table
+  for (int x = rank + G * tid; x < 2 * HK; x += G * blockDim.x) {
+    const int mh = x / d.k;  // entry (h*2 + half)*k + idx of this row
+    const int sub = esub_s[x];
+    if (sub >= 0) {
+      const int64_t e = e0 + x;
+      Member m;
+      m.g = (uint32_t)d.Nt + (uint32_t)((tab0 + mh) * d.n + sub);
+      m.id = (uint32_t)e;
+      m.srow = (int)(tok * 2 * d.H + mh);  // this query half in the caller's Q
+      m.gstart = 0;
+      m.coef = 0.f;
+      m.c0 = 0.f;
+      m.c1 = 0.f;
+      m.glen = 0;
+      s.rec_in[s.boff[d.NBv + (tab0 + mh) * d.n + sub] + eclaim_s[x]] = m;
+    }
   }
 }
 

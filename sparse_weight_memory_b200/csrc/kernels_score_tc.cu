@@ -179,6 +179,21 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The query tiles of the first stages are loaded before the grid dependency
+  // wait when they come from an earlier grid than the one just before (which
+  // updates the sub-keys): each stage's full byte count is expected now, its
+  // sub-key tiles are loaded after the wait.
+  int pre = 0;  // k-blocks whose query tiles are in flight before the wait (thread 0)
+  if (d.q_early && warp == 0 && lane == 0) {
+    pre = nkb < kTcStages ? nkb : kTcStages;
+    const int ya = hh * d.qstride + m0;
+    for (int kb = 0; kb < pre; ++kb) {
+      unsigned char *stage = smem + kb * L::kStage;
+      mbar_arrive_expect_tx(&full[kb], kALo ? L::kStage : L::kStage - L::kA);
+      tma_load_2d(stage, &mapAhi, kb * kTcKBlock, ya, &full[kb]);
+      if (kALo) tma_load_2d(stage + L::kA, &mapAlo, kb * kTcKBlock, ya, &full[kb]);
+    }
+  }
   griddep_wait();
   griddep_launch();
 
@@ -207,14 +222,16 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
     const int yb = tab * d.n + n0;       // row of the sub-key tensor
     for (int kb = 0; kb < nkb; ++kb, issued = kb) {
       const int st = kb % kTcStages, round = kb / kTcStages;
-      if (!mbar_wait_bounded(&empty[st], (round & 1) ^ 1, s.meta, d.mbar_polls,
-                             ERR_SCORE_TIMEOUT))
-        break;
       unsigned char *stage = smem + st * L::kStage;
-      mbar_arrive_expect_tx(&full[st], kALo ? L::kStage : L::kStage - L::kA);
       const int x = kb * kTcKBlock;
-      tma_load_2d(stage, &mapAhi, x, ya, &full[st]);
-      if (kALo) tma_load_2d(stage + L::kA, &mapAlo, x, ya, &full[st]);
+      if (kb >= pre) {  // (a stage of the first round is free without waiting)
+        if (!mbar_wait_bounded(&empty[st], (round & 1) ^ 1, s.meta, d.mbar_polls,
+                               ERR_SCORE_TIMEOUT))
+          break;
+        mbar_arrive_expect_tx(&full[st], kALo ? L::kStage : L::kStage - L::kA);
+        tma_load_2d(stage, &mapAhi, x, ya, &full[st]);
+        if (kALo) tma_load_2d(stage + L::kA, &mapAlo, x, ya, &full[st]);
+      }
       tma_load_2d(stage + 2 * L::kA, &mapBhi, x, yb, &full[st]);
       tma_load_2d(stage + 2 * L::kA + L::kB, &mapBlo, x, yb, &full[st]);
     }
