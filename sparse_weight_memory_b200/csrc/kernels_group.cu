@@ -911,7 +911,29 @@ __global__ void __launch_bounds__(kApplyThreads, 4) k_apply(Dims d, float *__res
     }
     // a short group: the whole row, two column chunks at a time
     float *dst = value ? V + (int64_t)g * d.dv : K + (int64_t)(g - (uint32_t)d.Nt) * d.dh;
-    if (!value || C > 0.f) {
+    if ((!value || C > 0.f) && cnt == 1 && n4 <= 4 * kChunk4) {
+      // One member (most groups while slot use is spread): its source row and
+      // the target row in one round of loads; the same arithmetic as below.
+      const int sr = __shfl_sync(FULL, mj.srow, 0);
+      const float cj = __shfl_sync(FULL, coef, 0);
+      float4 t[4], x[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        t[q] = load_chunk(dst, lane + q * kChunk4, n4);
+        x[q] = value ? load_chunk(s.E + (int64_t)sr * d.dv, lane + q * kChunk4, n4)
+                     : load_chunk(Qin + (int64_t)sr * d.dh, lane + q * kChunk4, n4);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int c4 = lane + q * kChunk4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        fma4(acc, cj, x[q]);
+        const float4 nv = updated(d, value, t[q], acc, C);
+        if (c4 < n4) *reinterpret_cast<float4 *>(dst + 4 * c4) = nv;
+        if (!value && q * kChunk4 < n4)
+          resplit_key_chunk(d, s, (int64_t)(g - (uint32_t)d.Nt), q, c4, n4, nv);
+      }
+    } else if (!value || C > 0.f) {
       for (int cb = 0; cb < n4; cb += 2 * kChunk4) {
         const float4 t0 = load_chunk(dst, cb + lane, n4);
         const float4 t1 = load_chunk(dst, cb + lane + 32, n4);
