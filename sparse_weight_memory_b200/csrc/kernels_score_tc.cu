@@ -138,7 +138,6 @@ struct TcSmem {
   static constexpr int kStages = tc_stages<BN>();
   static constexpr int kBytes =
       kStages * kStage + 1024 /* align */ + 256 /* barriers */ + 4 * BN /* column norms */;
-  static_assert(kStage >= 4 * 32 * 33 * 4, "epilogue tile fits in stage 0");
 };
 
 template <int BN, bool kALo>
@@ -264,9 +263,8 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
   __syncthreads();  // the column norms are in shared memory
 
   // ---------------- epilogue: TMEM -> distances ----------------
-  // Each warp owns 32 accumulator lanes (rows).  Per block of 32 columns the
-  // values go through a padded shared-memory tile (the stage buffers are free
-  // now) so that every store writes 32 consecutive columns of one row.
+  // Each warp owns 32 accumulator lanes (rows), one per thread, read 32
+  // columns at a time.
   // warp-uniform: tcgen05.ld below is a warp-collective instruction
   const bool ready =
       __all_sync(FULL, mbar_wait_bounded(done, 0, s.meta, d.mbar_polls, ERR_SCORE_TIMEOUT));
@@ -284,28 +282,35 @@ __global__ void __launch_bounds__(128, tc_ctas_per_sm<BN>())
     }
   }
   if (ready) {
-    float *tile = reinterpret_cast<float *>(smem) + warp * 32 * 33;
-    const int row0 = m0 + warp * 32;
-    float *Dh = s.D + (int64_t)hh * d.drows * d.n;
+    // Each thread holds its own row's 32 consecutive columns: it forms their
+    // distances with its row norm and stores them as 16-byte pieces (rows of
+    // a length that is a multiple of 4 are 16-byte aligned), else one by one.
+    float *Drow = s.D + ((int64_t)hh * d.drows + my_row) * d.n;
+    const bool vec = (d.n & 3) == 0;
 #pragma unroll 1
     for (int c0 = 0; c0 < BN; c0 += 32) {
       float v[32];
       tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+      const int cbase = n0 + c0;
+      const int ncols = min(min(32, BN - c0), d.n - cbase);  // columns of the tile and table
 #pragma unroll
-      for (int j = 0; j < 32; ++j) tile[lane * 33 + j] = v[j];
-      __syncwarp();
-      const int col = n0 + c0 + lane;
-      const bool col_ok = col < d.n && c0 + lane < BN;
-      const float kn_l = col_ok && !dot ? kn_s[c0 + lane] : 0.f;  // |K_col|^2
-#pragma unroll 4
-      for (int r = 0; r < 32; ++r) {
-        const float qn_r = __shfl_sync(FULL, my_qn, r);
-        const float dist = qn_r + kn_l - 2.f * tile[r * 33 + lane];
-        if (col_ok && row0 + r < d.drows)
-          Dh[(int64_t)(row0 + r) * d.n + col] =
-              dot ? -tile[r * 33 + lane] : (dist > 0.f ? dist : 0.f);
+      for (int j = 0; j < 32; ++j) {
+        const float kn_j = !dot && c0 + j < BN ? kn_s[c0 + j] : 0.f;  // |K_col|^2
+        const float dist = my_qn + kn_j - 2.f * v[j];
+        v[j] = dot ? -v[j] : (dist > 0.f ? dist : 0.f);
       }
-      __syncwarp();
+      if (my_row < d.drows) {
+        if (vec && ncols == 32) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4 *>(Drow + cbase + 4 * q) =
+                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < ncols) Drow[cbase + j] = v[j];
+        }
+      }
     }
   }
   // Loads the producer issued that no MMA consumed (after a give-up) land
