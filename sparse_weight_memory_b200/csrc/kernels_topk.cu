@@ -156,15 +156,35 @@ __device__ __forceinline__ void half_topk(const float *__restrict__ drow, int n,
                                           float &d_out, int &i_out, uint2 *wbuf) {
   const int lane = threadIdx.x & 31;
   uint32_t key[NV], idx[NV];
+  // d >= 0: the bit order is the value order; a used entry never takes the
+  // unused marker 0xffffffff, whatever the distance's bits.  Rows of a length
+  // that is a multiple of 4 are read 16 bytes a lane (entry v of the lane is
+  // i = 128 (v / 4) + 4 lane + v % 4); the selection depends only on the set
+  // of (key, index) pairs, not on which lane holds which.
+  if (NV % 4 == 0 && (n & 3) == 0) {
 #pragma unroll
-  for (int v = 0; v < NV; ++v) {
-    const int i = lane + 32 * v;
-    // d >= 0: the bit order is the value order; a used entry never takes the
-    // unused marker 0xffffffff, whatever the distance's bits
-    const float dv = i < n ? drow[i] : 0.f;
-    key[v] = i < n ? min(kSgn ? float_order(dv) : __float_as_uint(dv), 0xfffffffeu)
-                   : 0xffffffffu;
-    idx[v] = (uint32_t)i;
+    for (int q = 0; q < NV / 4; ++q) {
+      const int i0 = 128 * q + 4 * lane;
+      const float4 f = i0 < n ? *reinterpret_cast<const float4 *>(drow + i0)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        key[4 * q + c] = i0 < n ? min(kSgn ? float_order(fv[c]) : __float_as_uint(fv[c]),
+                                      0xfffffffeu)
+                                : 0xffffffffu;
+        idx[4 * q + c] = (uint32_t)(i0 + c);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const int i = lane + 32 * v;
+      const float dv = i < n ? drow[i] : 0.f;
+      key[v] = i < n ? min(kSgn ? float_order(dv) : __float_as_uint(dv), 0xfffffffeu)
+                     : 0xffffffffu;
+      idx[v] = (uint32_t)i;
+    }
   }
   uint32_t kk, ii;
   int v_out, src;
@@ -341,6 +361,7 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
 
   // ---- merge (warp 2t) ----
   float s_r = -CUDART_INF_F;
+  int vclaim = -1;  // this lane's value-bucket claim (merge warps, lane < k)
   int slot_r = 0;
   if (valid && half == 0) {
     int i_r = 0, j_r = 0;
@@ -437,7 +458,9 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
       if (lane < k) {
         s.pslot[p] = slot_r;
         s.pw[p] = w;
-        if (!d.readonly) s.pclaim[p] = atomicAdd(&s.bcnt[slot_r >> d.vshift], 1);  // value bucket
+        // the value bucket's claim; stored at the end, so that its round trip
+        // overlaps the entries' claims
+        if (!d.readonly) vclaim = atomicAdd(&s.bcnt[slot_r >> d.vshift], 1);
         if (x.rec_slots) {
           x.rec_slots[th * k + lane] = slot_r - (int)slot0;
           x.rec_w[th * k + lane] = w;
@@ -469,6 +492,7 @@ __global__ void __launch_bounds__(64 * kTopkHeads) k_topk(Dims d, Scratch s, Ext
   // unused entry slots of this half are marked -1
   if (lane >= __popc(lb) && lane < k) s.esub[((int64_t)m * 2 + half) * k + lane] = -1;
   if (lane == 0) s.ecount[(int64_t)m * 2 + half] = __popc(lb);
+  if (vclaim >= 0) s.pclaim[(int64_t)m * k + lane] = vclaim;
 }
 
 template <int KV, bool kSelectOnly, bool kDot>
