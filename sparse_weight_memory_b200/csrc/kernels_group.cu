@@ -510,16 +510,20 @@ __global__ void __launch_bounds__(kSortThreads)
   __shared__ int rank_red[32], rank_flag;
   __shared__ int lst[4][kListStage];  // staged entries: short[kind], then long[kind]
   __shared__ int lst_n[4], lst_base[4];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  // The next chunk's query halves, one warp per half row, made before the
+  // grid dependency wait, while the read finishes: they need only the
+  // caller's Q (which the caller's stream orders before this grid), and the
+  // halves they overwrite were last read by this chunk's score, which
+  // completed before the read was launched.
+  {
+    const int64_t nq = dn.rows > 0 ? (int64_t)2 * dn.H * dn.rows : 0;
+    for (int64_t w = (int64_t)blockIdx.x * kSortWarps + wib; w < nq;
+         w += (int64_t)gridDim.x * kSortWarps)
+      prep_query_half(dn, Q, s, w);
+  }
   griddep_wait();
   griddep_launch();
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  if ((int)blockIdx.x >= sort_blocks) {
-    // Extra CTAs: the next chunk's query halves, one warp each (this chunk's
-    // halves are not read after its score).
-    const int64_t w = (int64_t)(blockIdx.x - sort_blocks) * kSortWarps + wib;
-    if (w < (int64_t)2 * dn.H * dn.rows) prep_query_half(dn, Q, s, w);
-    return;
-  }
   // An earlier kernel of the chunk gave up: its offsets or selection may be
   // wrong, so nothing is sorted (the next chunk's halves above are still
   // prepared; they index nothing).
@@ -635,8 +639,8 @@ __global__ void __launch_bounds__(kSortThreads)
   }
 }
 
-// The sorting grid: a warp per bucket up to the resident CTAs.  The extra
-// CTAs after it prepare the next chunk's query halves (dn.rows > 0).
+// The sorting grid: a warp per bucket up to the resident CTAs.  Its warps
+// first prepare the next chunk's query halves (dn.rows > 0).
 template <typename TQ>
 static cudaError_t launch_bsort_t(const Dims &d, const Scratch &s, const Dims &dn, const TQ *Q,
                                   cudaStream_t st) {
@@ -648,10 +652,7 @@ static cudaError_t launch_bsort_t(const Dims &d, const Scratch &s, const Dims &d
   int blocks = (d.NB + kSortWarps - 1) / kSortWarps;
   const int cap = d.sm_count * per_sm;
   if (blocks > cap) blocks = cap;
-  const int64_t qwarps = dn.rows > 0 ? (int64_t)2 * dn.H * dn.rows : 0;
-  const int extra = (int)((qwarps + kSortWarps - 1) / kSortWarps);
-  return launch_k(d.pdl, k_bucket_sort<TQ>, blocks + extra, kSortThreads, 0, st, d, s, dn, Q,
-                  blocks);
+  return launch_k(d.pdl, k_bucket_sort<TQ>, blocks, kSortThreads, 0, st, d, s, dn, Q, blocks);
 }
 
 cudaError_t launch_bsort(const Dims &d, const Scratch &s, const Dims &dn, const void *Q,
