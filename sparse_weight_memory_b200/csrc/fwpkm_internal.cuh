@@ -123,7 +123,8 @@ struct Scratch {
   uint32_t *emask;  // [2*M*k] pairs r of token-head m that use that row
   float *einv;      // [2*M*k] 1 / (eps + d_half(row))
   int32_t *eclaim;  // [2*M*k] position inside the entry's bucket
-  float *ealpha;    // [2*M*k] sum of dL/ds over the entry's pairs / (eps + d)
+  float *ealpha;    // [2*M*k] sum of dL/ds over the entry's pairs / (eps + d) (pgrad,
+                    // with the entropy term on; else the read puts it in the record)
   int32_t *ecount;  // [M*2]   entries per (m, half)
   int32_t *bcnt;    // [NB]    members per bucket (zero between chunks)
   int32_t *boff;    // [NB+1]  bucket offsets into rec_in / rec

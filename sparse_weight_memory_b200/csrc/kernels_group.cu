@@ -269,14 +269,11 @@ __device__ __forceinline__ int lower_rank(const uint64_t *r, int len, uint64_t k
   return lo;
 }
 
-// A record on its way from rec_in to rec.  When the entropy term is off the
-// read kernel has already computed every entry's alpha (ealpha): it becomes
-// the sub-key record's coefficient here.  With the term on, alpha is known
-// only after pgrad and the apply reads it itself.
-__device__ __forceinline__ Member fetch_member(const Dims &d, const Scratch &s, const Member *p) {
-  Member m = load_member(p);
-  if (d.lam == 0.f && m.g >= (uint32_t)d.Nt) m.coef = m.c0 = s.ealpha[m.id];
-  return m;
+// A record on its way from rec_in to rec.  A sub-key record already carries
+// its alpha when the entropy term is off (the read wrote it); with the term
+// on, alpha is known only after pgrad and the apply reads it itself.
+__device__ __forceinline__ Member fetch_member(const Dims &, const Scratch &, const Member *p) {
+  return load_member(p);
 }
 
 constexpr int kShortMax = 4;  // groups up to this size are applied by one warp, whole rows

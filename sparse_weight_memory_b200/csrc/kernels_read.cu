@@ -323,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, kThreads == 128 ? 7 : 1) k_read(Dims
           sum += dl[__ffs(mask) - 1];
           mask &= mask - 1;
         }
-        s.ealpha[e0 + x] = einv_s[x] * sum;
+        einv_s[x] *= sum;  // alpha, which goes into the entry's record below
       }
     }
     // no CTA leaves while another may still read its a values
@@ -336,9 +336,9 @@ __global__ void __launch_bounds__(kThreads, kThreads == 128 ? 7 : 1) k_read(Dims
   if (chunk_aborted(s, ERR_READ_TIMEOUT)) return;
   // Member records go to their buckets last, at the scan's offsets: this
   // CTA's pairs -> value bucket slot >> vshift; entries x = rank (mod G) ->
-  // sub-key row bucket NBv + (h*2+half)*n + row.  An entry's alpha is filled
-  // in later from ealpha (by the sort, or by the apply when the entropy term
-  // is on).
+  // sub-key row bucket NBv + (h*2+half)*n + row.  An entry carries its alpha
+  // when the entropy term is off; with it on, the apply reads the alpha
+  // pgrad computes.
   for (int j = j0 + tid; j < j1; j += blockDim.x) {
     const int64_t p = p0 + j;
     const float w = w_s[j];
@@ -364,8 +364,7 @@ __global__ void __launch_bounds__(kThreads, kThreads == 128 ? 7 : 1) k_read(Dims
       m.id = (uint32_t)e;
       m.srow = (int)(tok * 2 * d.H + mh);  // this query half in the caller's Q
       m.gstart = 0;
-      m.coef = 0.f;
-      m.c0 = 0.f;
+      m.coef = m.c0 = d.lam == 0.f ? einv_s[x] : 0.f;
       m.c1 = 0.f;
       m.glen = 0;
       s.rec_in[s.boff[d.NBv + (tab0 + mh) * d.n + sub] + eclaim_s[x]] = m;
