@@ -303,11 +303,11 @@ def algorithmic_work(wl, tokens, segments, value_rows, key_rows, records, memori
 NCU_TRAFFIC = {
     # library: captures of commit 1b28857 (fwpkm_topk: d6e5ae0, kernel unchanged since)
     "library": {"fwpkm_apply": 10.44e6, "fwpkm_bsort": 1.425e6, "fwpkm_topk": 1.134e6},
-    # longctx: captures of commit cde205f, one chunk of 1024 tokens (the unit of a launch at
+    # longctx: captures of commit a3bdd73, one chunk of 1024 tokens (the unit of a launch at
     # any call length) taken in a 32-chunk call, chunk 29 of the last warm-up step; ncu
     # flushes the caches before each pass, so these are cold-cache bytes
-    "longctx": {"fwpkm_read": 17.806e6, "fwpkm_apply": 21.634e6, "fwpkm_bsort": 4.216e6,
-                "fwpkm_topk": 8.497e6, "fwpkm_score": 8.482e6, "fwpkm_scan": 0.050e6},
+    "longctx": {"fwpkm_read": 17.811e6, "fwpkm_apply": 21.718e6, "fwpkm_bsort": 3.958e6,
+                "fwpkm_topk": 8.496e6, "fwpkm_score": 8.485e6, "fwpkm_scan": 0.052e6},
 }
 
 
