@@ -301,8 +301,6 @@ def algorithmic_work(wl, tokens, segments, value_rows, key_rows, records, memori
 # kernel; the captures and their commands are summarised in profiles/.
 # Missing = no capture of the current kernel.
 NCU_TRAFFIC = {
-    # library: captures of commit 1b28857 (fwpkm_topk: d6e5ae0, kernel unchanged since)
-    "library": {"fwpkm_apply": 10.44e6, "fwpkm_bsort": 1.425e6, "fwpkm_topk": 1.134e6},
     # longctx: captures of commit a3bdd73, one chunk of 1024 tokens (the unit of a launch at
     # any call length) taken in a 32-chunk call, chunk 29 of the last warm-up step; ncu
     # flushes the caches before each pass, so these are cold-cache bytes
