@@ -702,14 +702,22 @@ __device__ __forceinline__ void add4(float4 &a, const float4 &x) {
 }
 
 // New value of one float4 of a target row from the group's complete sums.
-//   value row : v - (eta / C) * G          (C = sum of w/H)
+//   value row : v - (eta / C) * G          (C = sum of w/H; G / C first
+//                                           when eta / C overflows)
 //   sub-key   : k - 2 eta (G - A k)        (A = sum of alpha; IDW score)
 //               k - eta G                  (dot-product score: ds/dK = q)
 __device__ __forceinline__ float4 updated(const Dims &d, bool value, const float4 &t,
                                           const float4 &g, float c0) {
   if (value) {
-    const float sc = d.agg == AGG_SUM ? d.eta : d.eta / c0;
-    return make_float4(t.x - sc * g.x, t.y - sc * g.y, t.z - sc * g.z, t.w - sc * g.w);
+    if (d.agg == AGG_SUM || c0 * 0x1p+120f > d.eta) {  // eta / C is finite
+      const float sc = d.agg == AGG_SUM ? d.eta : d.eta / c0;
+      return make_float4(t.x - sc * g.x, t.y - sc * g.y, t.z - sc * g.z, t.w - sc * g.w);
+    }
+    // A row whose members' softmax weights are all denormal (scores that far
+    // apart, as the dot-product score can give) has a denormal C, and eta / C
+    // overflows: G / C first, both tiny, their ratio of the order of e.
+    return make_float4(t.x - d.eta * (g.x / c0), t.y - d.eta * (g.y / c0),
+                       t.z - d.eta * (g.z / c0), t.w - d.eta * (g.w / c0));
   }
   if (d.score_dot)
     return make_float4(t.x - d.eta * g.x, t.y - d.eta * g.y, t.z - d.eta * g.z,

@@ -112,3 +112,28 @@ def test_dot_selection_without_allocation_is_the_steps():
                                        want_gap=True)
     check_selection(slots.cpu().numpy(), o["sel_slot"], o["gap"], "dot selection",
                     tie_gap(wl, inp))
+
+
+def test_dot_score_long_run_stays_finite():
+    """With the dot-product score the top-k scores can lie hundreds apart, so
+    some fp32 softmax weights are denormal, and a value row written only by
+    such pairs has a denormal divisor C.  Scaling by eta / C overflowed there
+    (NaN in the outputs within a 128-chunk long-context call).  The update
+    divides G by C first: every output and table entry stays finite over the
+    whole call, as the oracle's do (max |K| about 50 by its last chunk)."""
+    import torch
+
+    from sparse_weight_memory_b200 import FwPKMState
+
+    from fwpkm_testlib import to_dev
+    wl = WORKLOADS["longctx"].replace(score="dot", eta=0.05)
+    inp = make_inputs(wl)
+    st = FwPKMState(wl.N, wl.dq, wl.dv, wl.topk, wl.chunk, wl.heads, eps=wl.eps)
+    st.set_options(score="dot")
+    st.set_tables(to_dev(inp.subkeys), to_dev(inp.values))
+    out = st.step(to_dev(inp.Q), to_dev(inp.Vt), to_dev(inp.gate), wl.eta, wl.lam)
+    K, V = st.get_tables()
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(out).all()), "non-finite outputs"
+    assert bool(torch.isfinite(K).all()) and bool(torch.isfinite(V).all()), "non-finite tables"
+    st.close()
