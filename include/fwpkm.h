@@ -337,7 +337,8 @@ void fwpkm_inject_alloc_failures(int count);
  * synchronise the device).  The paper has no counterpart of this entry point;
  * it is a deployment variant of the selection done inside fwpkm_step.
  *   For every token t of the B sequences and every head h, scores both query
- *   halves against the state's current sub-key tables, takes the product-key
+ *   halves against the state's current sub-key tables (with the state's
+ *   score: IDW, or the dot product under FWPKM_SCORE_DOT), takes the product-key
  *   top-k and writes the slots and their softmax weights -- the same values
  *   fwpkm_step reads for that token with the same tables.  No readout and no
  *   update: the tables are not modified.
