@@ -702,22 +702,15 @@ __device__ __forceinline__ void add4(float4 &a, const float4 &x) {
 }
 
 // New value of one float4 of a target row from the group's complete sums.
-//   value row : v - (eta / C) * G          (C = sum of w/H; G / C first
-//                                           when eta / C overflows)
+//   value row : v - (eta / C) * G          (C = sum of w/H; see k_apply for a
+//                                           C so small that eta / C overflows)
 //   sub-key   : k - 2 eta (G - A k)        (A = sum of alpha; IDW score)
 //               k - eta G                  (dot-product score: ds/dK = q)
 __device__ __forceinline__ float4 updated(const Dims &d, bool value, const float4 &t,
                                           const float4 &g, float c0) {
   if (value) {
-    if (d.agg == AGG_SUM || c0 * 0x1p+120f > d.eta) {  // eta / C is finite
-      const float sc = d.agg == AGG_SUM ? d.eta : d.eta / c0;
-      return make_float4(t.x - sc * g.x, t.y - sc * g.y, t.z - sc * g.z, t.w - sc * g.w);
-    }
-    // A row whose members' softmax weights are all denormal (scores that far
-    // apart, as the dot-product score can give) has a denormal C, and eta / C
-    // overflows: G / C first, both tiny, their ratio of the order of e.
-    return make_float4(t.x - d.eta * (g.x / c0), t.y - d.eta * (g.y / c0),
-                       t.z - d.eta * (g.z / c0), t.w - d.eta * (g.w / c0));
+    const float sc = d.agg == AGG_SUM ? d.eta : d.eta / c0;
+    return make_float4(t.x - sc * g.x, t.y - sc * g.y, t.z - sc * g.z, t.w - sc * g.w);
   }
   if (d.score_dot)
     return make_float4(t.x - d.eta * g.x, t.y - d.eta * g.y, t.z - d.eta * g.z,
@@ -839,6 +832,15 @@ __global__ void __launch_bounds__(kApplyThreads, 4) k_apply(Dims d, float *__res
       C += __shfl_xor_sync(FULL, C, o);
       W += __shfl_xor_sync(FULL, W, o);
     }
+    // A value row whose members' softmax weights are all denormal (scores that
+    // far apart, as the dot-product score can give) has a C so small that
+    // eta / C overflows: its coefficients and C are scaled by 2^64 first, which
+    // is exact and leaves G / C as it is.  (A longer group's block partials are
+    // scaled at the group's combine.)
+    if (!block && value && d.agg != AGG_SUM && !(C * 0x1p+120f > d.eta)) {
+      C *= 0x1p+64f;
+      coef *= 0x1p+64f;
+    }
     const int n4 = (value ? d.dv : d.dh) >> 2;
     if (block) {
       // one column chunk of a longer group's block, into its partial slot
@@ -904,6 +906,11 @@ __global__ void __launch_bounds__(kApplyThreads, 4) k_apply(Dims d, float *__res
 #pragma unroll
           for (int u = 0; u < kU; ++u)
             if (b0 + u < nb) add4(tot, r[u]);
+        }
+        if (value && d.agg != AGG_SUM && !(Ct * 0x1p+120f > d.eta)) {  // as above
+          Ct *= 0x1p+64f;
+          tot = make_float4(tot.x * 0x1p+64f, tot.y * 0x1p+64f, tot.z * 0x1p+64f,
+                            tot.w * 0x1p+64f);
         }
         const float4 nv = updated(d, value, t, tot, Ct);
         if (c4 < n4) *reinterpret_cast<float4 *>(row + 4 * c4) = nv;
