@@ -301,10 +301,10 @@ def algorithmic_work(wl, tokens, segments, value_rows, key_rows, records, memori
 # kernel; the captures and their commands are summarised in profiles/.
 # Missing = no capture of the current kernel.
 NCU_TRAFFIC = {
-    # longctx: captures of commit a3bdd73, one chunk of 1024 tokens (the unit of a launch at
-    # any call length) taken in a 32-chunk call, chunk 29 of the last warm-up step; ncu
-    # flushes the caches before each pass, so these are cold-cache bytes
-    "longctx": {"fwpkm_read": 17.811e6, "fwpkm_apply": 21.718e6, "fwpkm_bsort": 3.958e6,
+    # longctx: captures of commit a3bdd73 (fwpkm_apply: 3b2b6da), one chunk of 1024 tokens
+    # (the unit of a launch at any call length) taken in a 32-chunk call, chunk 29 of the last
+    # warm-up step; ncu flushes the caches before each pass, so these are cold-cache bytes
+    "longctx": {"fwpkm_read": 17.811e6, "fwpkm_apply": 21.680e6, "fwpkm_bsort": 3.958e6,
                 "fwpkm_topk": 8.496e6, "fwpkm_score": 8.485e6, "fwpkm_scan": 0.052e6},
 }
 
