@@ -289,7 +289,7 @@ __device__ __forceinline__ int lrow_of(const Dims &d, int row) {
 // One query half (warp w = (h*2 + half)*rows + row of chunk d) into its TF32
 // split and squared norm: Qs_hi / Qs_lo [h][half][lrow][:], qn (rows at
 // stride qstride).  Warp-level; used by the prep and by the bucket sort's
-// extra CTAs (the next chunk's halves).
+// CTAs before their grid dependency wait (the next chunk's halves).
 template <typename TQ>
 __device__ __forceinline__ void prep_query_half(const Dims &d, const TQ *__restrict__ Q,
                                                 const Scratch &s, int64_t w) {
@@ -321,9 +321,19 @@ __device__ __forceinline__ void prep_query_half(const Dims &d, const TQ *__restr
 // Programmatic dependent launch.  A kernel started by launch_k with d.pdl set
 // may become resident while its predecessor on the stream is still running;
 // griddep_wait() blocks until that predecessor has completed and its writes
-// are visible, so every kernel calls it before its first global-memory access
-// (and griddep_launch() right after, letting its own successor get scheduled
-// early).  Both are no-ops for a kernel launched without the attribute.
+// are visible, so a kernel calls it before it reads anything its predecessor
+// writes, and griddep_launch() early, letting its own successor get
+// scheduled.  A grid is launched only after every CTA of the one before has
+// called griddep_launch().  Every kernel here calls it right after its own
+// wait, except the read of the write path, which calls it first (it waits
+// only before its member records).  So when a kernel starts, every grid
+// before its predecessor has completed, except that the sort, which follows
+// the read, may start while the scan still runs.  Three kernels read before
+// their wait and rely on exactly that: the read on the selection's output (two
+// back), the score on the query halves the previous chunk's sort made (two
+// back), and the sort only on the caller's Q and on query-half storage last
+// read by the score (four back).  Both are no-ops for a kernel launched
+// without the attribute.
 __device__ __forceinline__ void griddep_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
@@ -401,7 +411,7 @@ cudaError_t launch_read(const Dims &d, const float *V, const void *Vt, int v_dty
                         cudaStream_t st);
 // CTAs per token of the read at these shapes (1 unless a token's rows exceed 1 MB).
 int read_cluster_size(const Dims &d);
-// The bucket sort; with dn.rows > 0 extra CTAs also prepare the query halves
+// The bucket sort; with dn.rows > 0 its CTAs first prepare the query halves
 // of the next chunk dn (nothing reads this chunk's halves after the score).
 cudaError_t launch_bsort(const Dims &d, const Scratch &s, const Dims &dn, const void *Q,
                          int q_dtype, cudaStream_t st);
