@@ -134,3 +134,21 @@ def test_batched_init_rejects_bad_memory_counts(lib, memories):
     rc = lib.fwpkm_state_init_batched(1024 * 1024, 64, 64, 4, 32, 1, memories, ctypes.byref(h))
     assert rc == fwpkm.FWPKM_ESHAPE
     assert h.value is None
+
+
+def test_binding_constants_equal_the_header():
+    """Every status code, dtype code, option bit and flag the binding passes
+    through equals the header's value (a mismatch would select another reading
+    of the method without any error)."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    values = {name: int(val) for name, val in
+              re.findall(r"#define\s+(FWPKM_[A-Z_]+)\s+(-?\d+)u?\b", src)}
+    values.update({name: int(val) for name, val in
+                   re.findall(r"\b(FWPKM_[A-Z0-9_]+)\s*=\s*(-?\d+)", src)})
+    binding = [name for name in dir(fwpkm) if name.startswith("FWPKM_")]
+    for name in binding:  # every constant of the binding is the header's
+        assert name in values, f"{name} is not in the header"
+        assert getattr(fwpkm, name) == values[name], name
+    for name in ("FWPKM_OK", "FWPKM_ECUDA", "FWPKM_BF16", "FWPKM_LOOKAHEAD", "FWPKM_HEADS_SUM",
+                 "FWPKM_AGG_COUNT", "FWPKM_AGG_SUM", "FWPKM_SCORE_DOT"):
+        assert name in binding, name
