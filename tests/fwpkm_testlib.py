@@ -216,6 +216,13 @@ def compare_runs(wl: Workload, inp: Inputs, g: RunResult, o: RunResult, what: st
     tol = table_tol(wl, T)
     check_table(g.V, o.V, tol, f"{what} values")
     check_table(g.K, o.K, tol, f"{what} sub-keys")
-    return {"dV_rel": update_rel_error(g.V, o.V, inp.values),
+    info = {"dV_rel": update_rel_error(g.V, o.V, inp.values),
             "dK_rel": update_rel_error(g.K, o.K, inp.subkeys),
             "near_ties": int(sum((x <= tg).sum() for x in o.gaps))}
+    # the achieved errors, so that a drift shows long before it reaches a bound
+    out_ratio = max(float((np.abs(g.outs[i].astype(np.float64) - o.outs[i]) /
+                           (OUT_ATOL + OUT_RTOL * np.abs(o.outs[i]))).max())
+                    for i in range(len(o.outs)))
+    print(f"{what}: worst out err / bound {out_ratio:.3f}, update rel err V {info['dV_rel']:.2e} "
+          f"K {info['dK_rel']:.2e}, near ties {info['near_ties']}")
+    return info
